@@ -1,0 +1,212 @@
+/*
+ * lsa.h — C ABI of liblsa.so, the B200 (sm_100a) implementation of the
+ * LongCat Sparse Attention (LSA) decode/prefill hot path.
+ *
+ * What the method is (the pages give mechanisms, not formulas):
+ *  - "LongCat-2.0: Meituan이 Nvidia GPU 없이 ... (molayo1419.me)", section
+ *    "1M 토큰에서의 Sparse Attention 문제": LSA extends DeepSeek Sparse
+ *    Attention (an indexer scores every cached token and a top-k is kept)
+ *    with Streaming-aware Indexing (SI), Cross-Layer Indexing (CLI) and
+ *    Hierarchical Indexing (HI).
+ *  - "LongCat-Flash-Lite-Sparse (aitrends.kr)", section "기술적 특징": SI
+ *    gives part of the budget to fixed sinks and a local sliding window so KV
+ *    reads become contiguous; CLI reuses one index result over adjacent
+ *    layers; HI keeps coarse candidate blocks first and selects fine tokens
+ *    only inside them.
+ *  The arithmetic this library fixes:
+ *    fine score   score_t = sum_h w_h * max(0, q_h . k_t), int8 q and k,
+ *                 exact integer accumulation;
+ *    coarse score c_b     = the same formula on S_b, the exact sum of the
+ *                 indexer keys of block b;
+ *    selection    the topk highest scores of the "middle" tokens, ties to
+ *                 the lower position (blocks: the lower block index);
+ *    index set    [0, s) U selected U [ws, L), ascending, padded with -1,
+ *                 where s = min(sink, L) and ws = max(s, L - window);
+ *    attention    o = softmax(q . k_j / sqrt(d)) v_j over the set, GQA with
+ *                 query head h reading kv head floor(h * H_kv / H_q), bf16
+ *                 inputs, fp32 accumulation and fp32 output.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" are CUDA device pointers (e.g. a torch tensor's
+ *    data_ptr()); pointers marked "host" are ordinary host memory read during
+ *    the call. The caller owns every buffer; the library allocates nothing,
+ *    keeps no state between calls, and never frees caller memory.
+ *  - `stream` is a cudaStream_t passed as void*. Every call is asynchronous
+ *    on that stream and returns without synchronising.
+ *  - Argument and shape errors are returned synchronously, before any launch,
+ *    as an lsa_status_t. LSA_ERR_CUDA reports a failed launch (call
+ *    lsa_last_cuda_error() for the CUDA error code).
+ *  - Errors only the device can see (bad lengths or indices in device arrays)
+ *    are OR-ed as LSA_DEV_* bits into *dev_status (device int32, may be
+ *    NULL); the caller reads it after synchronising. The offending query's
+ *    output is then unspecified but every access stays in bounds.
+ *  - No kernel in this library waits on another CTA, kernel or device, so no
+ *    call can hang; no kernel traps.
+ *  - Calls are thread-safe when they use distinct workspaces.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad shape */
+    LSA_ERR_UNSUPPORTED = 2, /* valid but outside the compiled range */
+    LSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    LSA_ERR_WORKSPACE = 4    /* workspace pointer null or smaller than required */
+} lsa_status_t;
+
+/* Bits OR-ed into *dev_status by device-side checks. */
+#define LSA_DEV_BAD_LENGTH 0x1 /* q_len/seq_lens outside [1, max_len] or past the cache */
+#define LSA_DEV_BAD_SEQ 0x2    /* q_seq outside [0, n_seq) */
+#define LSA_DEV_BAD_INDEX 0x4  /* an index-set entry < -1 or >= q_len (entry skipped) */
+#define LSA_DEV_BAD_WEIGHT 0x8 /* an indexer head weight outside [0, w_max] (treated as 0) */
+
+/* Selection budget. sink + window + topk is the index-set length ("budget").
+ * hi_block == 0 switches HI off; otherwise blocks of hi_block tokens aligned
+ * at position 0 are scored coarsely and the hi_topblocks best are kept. */
+typedef struct {
+    int32_t sink;
+    int32_t window;
+    int32_t topk;
+    int32_t hi_block;
+    int32_t hi_topblocks;
+} lsa_budget_t;
+
+/* A batch of query rows over packed sequences.
+ *  Decode: one row per sequence, q_len[r] = seq_lens[q_seq[r]] (the current
+ *  token's K/V and indexer key are already in the cache).
+ *  Prefill: the rows of a chunk of n new tokens appended to a cache of C
+ *  tokens see q_len = C + i + 1 for i = 0..n-1. */
+typedef struct {
+    int32_t n_seq;            /* number of sequences, >= 1 */
+    int32_t n_q;              /* number of query rows, >= 0 */
+    int32_t max_len;          /* host-side upper bound on every q_len and seq_lens */
+    int32_t reserved;         /* must be 0 */
+    int64_t total_tokens;     /* rows in the packed caches (bounds every access) */
+    const int64_t *kv_offset; /* device [n_seq]: first cache row of each sequence */
+    const int32_t *seq_lens;  /* device [n_seq]: tokens present in each sequence */
+    const int64_t *blk_offset;/* device [n_seq]: first block-sum row of each sequence
+                                 (HI only; NULL when HI is off) */
+    const int32_t *q_seq;     /* device [n_q]: sequence of each query row */
+    const int32_t *q_len;     /* device [n_q]: visible length of each query row */
+} lsa_batch_t;
+
+/* Largest sizes the kernels are compiled for. */
+#define LSA_MAX_HEADS_I 64    /* H_I */
+#define LSA_MAX_BUDGET 16384  /* sink + window + topk */
+#define LSA_MAX_HI_BLOCK 256  /* hi_block (block sums stay exact in 16 bits) */
+#define LSA_MAX_TOPBLOCKS 4096
+#define LSA_MAX_LAYERS 8      /* layers sharing one index set (CLI group) */
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t lsa_version(void);
+
+/* CUDA error code (cudaError_t) of the last LSA_ERR_CUDA on this thread. */
+int32_t lsa_last_cuda_error(void);
+
+/* Human-readable name of a status code (static string). */
+const char *lsa_status_string(int32_t status);
+
+/* ----------------------------------------------------------------------- */
+/* HI block-sum pre-pass                                                     */
+/* ----------------------------------------------------------------------- */
+/* Computes the per-block key sums S_b[d] = sum of k_t[d] over the present
+ * tokens t of block b (blocks of hi_block tokens aligned at position 0; the
+ * last may be partial). HI's "fast approximate block-level pass" scores
+ * these instead of every token (Flash-Lite-Sparse page, "기술적 특징",
+ * Hierarchical Indexing bullet).
+ *
+ * k_idx_cache  device int8 [total_tokens][d_I], sequences packed by kv_offset.
+ * block_sums   device int8 [rows][2*d_I]. Sequence b's blocks are the rows
+ *              blk_offset[b] .. blk_offset[b] + ceil(seq_lens[b]/hi_block) - 1.
+ *              Each row stores S_b exactly in two byte planes: bytes
+ *              [0, d_I) hold S >> 8 as int8 and bytes [d_I, 2*d_I) hold
+ *              S & 0xFF as uint8, so S = 256*hi + lo (|S| <= 128*hi_block).
+ * n_new        <= 0: rebuild every block of every sequence. > 0: rebuild only
+ *              the blocks that hold the last n_new tokens of each sequence
+ *              (the decode append update; n_new = 1 for one new token).
+ * Supported: d_I in {32, 64, 128}; 1 <= hi_block <= LSA_MAX_HI_BLOCK.
+ */
+lsa_status_t lsa_hi_block_sums(const int8_t *k_idx_cache, int32_t d_I,
+                               int32_t hi_block, const lsa_batch_t *batch,
+                               int32_t n_new, int8_t *block_sums,
+                               int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------------------------------- */
+/* Indexer: scores, HI, top-k, SI assembly                                   */
+/* ----------------------------------------------------------------------- */
+/* Workspace bytes lsa_index needs for this batch shape (reads only the host
+ * fields of *batch). 0 means no workspace is needed. */
+size_t lsa_index_workspace_size(const lsa_batch_t *batch, int32_t H_I,
+                                int32_t d_I, lsa_budget_t budget);
+
+/* One index set per query row (CLI: call once per group of layers and pass
+ * the result to lsa_attend with layers_per_index = G).
+ *
+ * q_idx        device int8 [n_q][H_I][d_I] indexer queries.
+ * k_idx_cache  device int8 [total_tokens][d_I] indexer keys (one per token,
+ *              shared by all indexer heads).
+ * w            device int32 [n_q][H_I] head weights in [0, w_max].
+ * w_max        host bound on w; H_I * w_max * d_I * 16384 must be < 2^31 so
+ *              that fine scores are exact in int32 (else LSA_ERR_UNSUPPORTED).
+ * block_sums   device, as written by lsa_hi_block_sums (HI on), or NULL when
+ *              hi_block == 0.
+ * index_sets   device int32 [n_q][sink+window+topk] output: positions relative
+ *              to the sequence start, ascending, -1 padded.
+ * workspace    device scratch of lsa_index_workspace_size() bytes (may be NULL
+ *              when that size is 0). Not needed after the call returns on the
+ *              stream.
+ * Supported: d_I in {32, 64, 128}; 1 <= H_I <= LSA_MAX_HEADS_I;
+ * budget <= LSA_MAX_BUDGET; hi_topblocks <= LSA_MAX_TOPBLOCKS.
+ */
+lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
+                       const int32_t *w, int32_t w_max, int32_t H_I, int32_t d_I,
+                       const lsa_batch_t *batch, lsa_budget_t budget,
+                       const int8_t *block_sums, int32_t *index_sets,
+                       void *workspace, size_t workspace_bytes,
+                       int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------------------------------- */
+/* Sparse attention over the index sets (all G layers of a CLI group)        */
+/* ----------------------------------------------------------------------- */
+/* Workspace bytes lsa_attend needs. The first 4*G*n_q bytes are arrival
+ * counters that must be zero before the first call; every call leaves them
+ * zero again. */
+size_t lsa_attend_workspace_size(const lsa_batch_t *batch, int32_t H_q,
+                                 int32_t H_kv, int32_t d, int32_t budget,
+                                 int32_t layers_per_index);
+
+/* o[g][r][h] = softmax_j(q . k_j / sqrt(d)) v_j over the entries j of
+ * index_sets[r] that are not -1, for every layer g < layers_per_index
+ * (Cross-Layer Indexing: all G layers share one set).
+ *
+ * q            host [G] array of device bf16 [n_q][H_q][d] (bit patterns).
+ * k_cache      host [G] array of device bf16 [total_tokens][H_kv][d].
+ * v_cache      host [G] array of device bf16 [total_tokens][H_kv][d].
+ * index_sets   device int32 [n_q][budget] (e.g. from lsa_index). Entries
+ *              < -1 or >= q_len set LSA_DEV_BAD_INDEX and are skipped.
+ * out          host [G] array of device fp32 [n_q][H_q][d]. A row whose set
+ *              is empty is written as zeros.
+ * Supported: d == 128; H_q % H_kv == 0 and H_q / H_kv in {1, 2, 4, 8, 16};
+ * H_kv in {1, 2, 4} or a multiple of 4; 1 <= G <= LSA_MAX_LAYERS;
+ * budget <= LSA_MAX_BUDGET.
+ */
+lsa_status_t lsa_attend(const uint16_t *const *q, const uint16_t *const *k_cache,
+                        const uint16_t *const *v_cache, int32_t H_q, int32_t H_kv,
+                        int32_t d, const int32_t *index_sets, int32_t budget,
+                        const lsa_batch_t *batch, int32_t layers_per_index,
+                        float *const *out, void *workspace, size_t workspace_bytes,
+                        int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */
