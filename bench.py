@@ -1,0 +1,393 @@
+"""Benchmark of the LSA decode hot path (one JSON line on rank 0).
+
+A step is one decode step of the batched 128K workload (16 sequences x
+131072 tokens, HI 64x256, sink/window/topk 64/1024/2048, 32 q heads over 4
+kv heads): the HI block-sum append update, the fused indexer (coarse pass,
+block selection, fine scores, top-k, SI assembly) and the split-K sparse
+attention with its merge. Inputs are seeded synthetic tensors resident in
+HBM. L2 is flushed (a 2 x L2-size write) before every timed step, outside the
+timed interval; every kernel is timed with CUDA events on the launching
+stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
+
+With torchrun (N > 1) every rank runs its own independent batch (weak
+scaling, no collective on the data path); the step time is the max over
+ranks. ``--impl reference`` times the CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_lsa_b200 import workloads as wls  # noqa: E402
+
+METRIC = "LSA decode queries/s at 128K & 1M ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "queries/s"
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must move; nothing avoided by HI counted)
+# ---------------------------------------------------------------------------
+def step_bytes(wl) -> dict:
+    n_q, G = wl.n_q, wl.G
+    ent = [min(L, wl.budget) for L in wl.lens] if not wl.prefill_new else None
+    kv_row = wl.H_kv * wl.d * 2  # bytes of one token's K (or V) in one layer
+    attend = 0
+    for e in ent:
+        attend += G * (2 * e * kv_row + wl.H_q * wl.d * 2 + wl.H_q * wl.d * 4 + wl.budget * 4)
+    index = 0
+    bsum = 0
+    for L in wl.lens:
+        s = min(wl.sink, L)
+        ws = max(s, L - wl.window)
+        if wl.hi_block > 0:
+            B = wl.hi_block
+            nb = (ws + B - 1) // B - s // B if ws > s else 0
+            kept = min(nb, wl.hi_topblocks)
+            index += nb * 2 * wl.d_I + kept * B * wl.d_I  # block sums read + kept keys
+            bsum += B * wl.d_I + 2 * wl.d_I  # append update: re-read one block, write one row
+        else:
+            index += (ws - s) * wl.d_I
+        index += wl.H_I * wl.d_I + wl.H_I * 4 + wl.budget * 4  # q, w, index-set write
+    return {"attend": attend, "index": index, "block_sums": bsum, "total": attend + index + bsum}
+
+
+# ---------------------------------------------------------------------------
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), "measured"
+    return 6650.0, "fallback"
+
+
+def _kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attend.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "long_context_sparse_lsa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kernel_hash: str, workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, if it was taken on this exact kernel source and workload."""
+    p = os.path.join(PROFILES, f"attend_{workload}.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_hash:
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def cpu_baseline(wl, t, max_seconds=20.0, max_queries=None):
+    """The oracle (one thread) on a bounded sample of the workload's queries:
+    index + G-layer attention per query; only the oracle calls are timed, and
+    the result is scaled to queries/s. ``t`` may live on any device: each
+    query's keys and the K/V rows its oracle set names are copied to the host
+    before its timed calls."""
+    import numpy as np
+
+    import oracle
+
+    orc = oracle.get()
+    u16 = lambda x: x.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    kv_off = t.kv_offset.cpu().numpy()
+    q_seq = t.q_seq.cpu().numpy()
+    q_len = t.q_len.cpu().numpy()
+    n = len(q_seq) if max_queries is None else min(max_queries, len(q_seq))
+    done, busy = 0, 0.0
+    for r in range(n):
+        base = int(kv_off[q_seq[r]])
+        L = int(q_len[r])
+        kseq = t.k_idx[base:base + L].cpu().numpy()
+        qi = t.q_idx[r].cpu().numpy()
+        wr = t.w[r].cpu().numpy()
+        c0 = time.perf_counter()
+        s = orc.index_query(qi, wr, kseq, L, wl.sink, wl.window, wl.topk, wl.hi_block, wl.hi_topblocks)
+        busy += time.perf_counter() - c0
+        valid = s[s >= 0]
+        local = np.full(s.shape[0], -1, np.int32)
+        local[: valid.shape[0]] = np.arange(valid.shape[0], dtype=np.int32)
+        rows = torch.as_tensor(valid.astype(np.int64) + base, device=t.k[0].device)
+        for g in range(len(t.q)):
+            kr, vr, qg = u16(t.k[g].index_select(0, rows)), u16(t.v[g].index_select(0, rows)), u16(t.q[g][r])
+            c0 = time.perf_counter()
+            orc.attend_query(qg, kr, vr, local)
+            busy += time.perf_counter() - c0
+        done += 1
+        if busy > max_seconds:
+            break
+    return {"value": done / busy, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} of {wl.n_q} queries of {wl.name} (index + {len(t.q)}-layer attention each), "
+                      f"single-threaded C oracle, {busy:.1f} s of oracle time"}
+
+
+def run_reference(args, wl):
+    """--impl reference: the CPU oracle as it stands, on a bounded sample
+    (the first sequence of the workload, drawn on the host)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sample = wls.small(wl, lens=wl.lens[:1], prefill_new=min(wl.prefill_new, 4) if wl.prefill_new else 0)
+    t = wls.make(sample, "cpu")
+    per_step = []
+    for _ in range(args.warmup):
+        cpu_baseline(sample, t, max_seconds=args.ref_seconds)
+    for _ in range(args.steps):
+        per_step.append(cpu_baseline(sample, t, max_seconds=args.ref_seconds))
+    value = statistics.median(p["value"] for p in per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.n_q / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
+            "data": "synthetic (seeded SplitMix64 draws)",
+            "config": {"workload": wl.name, "n_queries": wl.n_q, "context": max(wl.lens), "layers_per_index": wl.G},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": per_step[-1]["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
+    ap.add_argument("--workload", default=wls.BATCH128K.name)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    wl = wls.by_name(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    from long_context_sparse_lsa_b200 import binding as lsa
+    from long_context_sparse_lsa_b200.pipeline import LsaStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    # each rank draws its own independent batch (weak scaling)
+    wl_r = wls.small(wl, seed=wl.seed + 1000 * rank) if rank else wl
+    t = wls.make(wl_r, dev)
+    st = LsaStep(wl_r, t, dev)
+    st.build_block_sums()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    n_kernels = 3 if wl.hi_block > 0 else 2
+
+    def one_step(evs):
+        flush.fill_(1)
+        evs[0].record(stream)
+        if wl.hi_block > 0:
+            st.update_block_sums(1)
+        evs[1].record(stream)
+        st.index()
+        evs[2].record(stream)
+        st.attend()
+        evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        one_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize()
+    if st.status_bits() != 0:
+        raise RuntimeError(f"device status {st.status_bits():#x} after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        one_step(evs[i])
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clk = clocks.stop()
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    bs_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    ix_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    at_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    ms = sum(step_ms) / len(step_ms)
+    if pg:
+        tt = torch.tensor([ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # ---- end to end through the public API with host buffers ----
+    pin = lambda x: x.cpu().pin_memory()
+    h_q_idx, h_w = pin(t.q_idx), pin(t.w)
+    h_q = [pin(x) for x in t.q]
+    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.out]
+    h2d = h_q_idx.numel() + h_w.numel() * 4 + sum(x.numel() * 2 for x in h_q)
+    d2h = sum(o.numel() * 4 for o in st.out)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        t.q_idx.copy_(h_q_idx, non_blocking=True)
+        t.w.copy_(h_w, non_blocking=True)
+        for g in range(len(h_q)):
+            t.q[g].copy_(h_q[g], non_blocking=True)
+        st.step()
+        for g in range(len(h_out)):
+            h_out[g].copy_(st.out[g], non_blocking=True)
+        e1.record(stream)
+        if i >= args.warmup:
+            e2e_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e = sum(a.elapsed_time(b) for a, b in e2e_ms) / len(e2e_ms)
+    if pg:
+        tt = torch.tensor([e2e], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        e2e = float(tt.item())
+    if st.status_bits() != 0:
+        raise RuntimeError(f"device status {st.status_bits():#x} after timing")
+
+    nq_all = wl.n_q * world
+    value = nq_all / (ms / 1000.0)
+    e2e_value = nq_all / (e2e / 1000.0)
+    byts = step_bytes(wl)
+    peak, peak_kind = _peaks()
+    at = sum(at_ms) / len(at_ms)
+    ix = sum(ix_ms) / len(ix_ms)
+    bsu = sum(bs_ms) / len(bs_ms)
+    khash = _kernel_hash()
+    roof = {"bound": "hbm", "kernel": "attend_kernel (split-K sparse attention + merge)",
+            "achieved": byts["attend"] / (at / 1000.0) / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": byts["attend"] / (at / 1000.0) / 1e9 / peak, "peak_kind": peak_kind,
+            "traffic": _ncu_traffic(khash, wl.name),
+            "bytes_per_launch": byts["attend"]}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8->int32 (indexer), bf16->f32 (attention)",
+            "data": "synthetic (seeded SplitMix64 draws; no weights or datasets)",
+            "config": {"workload": wl.name, "n_queries_per_gpu": wl.n_q, "context": max(wl.lens),
+                       "layers_per_index": wl.G, "budget": {"sink": wl.sink, "window": wl.window,
+                                                            "topk": wl.topk, "hi_block": wl.hi_block,
+                                                            "hi_topblocks": wl.hi_topblocks},
+                       "heads": {"H_I": wl.H_I, "d_I": wl.d_I, "H_q": wl.H_q, "H_kv": wl.H_kv, "d": wl.d},
+                       "l2": "flushed before every timed step (2 x L2 write, outside the timed interval)",
+                       "parallelism": f"replicas x{world} (independent batches, no collective)"},
+            "step_breakdown_ms": {"block_sums_update": bsu, "index": ix, "attend": at},
+            "step_gbs": byts["total"] / (ms / 1000.0) / 1e9,
+            "step_frac_of_measured_hbm": byts["total"] / (ms / 1000.0) / 1e9 / peak,
+            "step_frac_of_8tbs": byts["total"] / (ms / 1000.0) / 1e9 / 8000.0,
+            "algorithmic_bytes_per_step": byts,
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e},
+            "gpu_launches": n_kernels * args.steps,
+            "clocks": clk}
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, t, max_seconds=args.cpu_seconds)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -129,6 +129,8 @@ const char *lsa_status_string(int32_t status);
  *              Each row stores S_b exactly in two byte planes: bytes
  *              [0, d_I) hold S >> 8 as int8 and bytes [d_I, 2*d_I) hold
  *              S & 0xFF as uint8, so S = 256*hi + lo (|S| <= 128*hi_block).
+ * block_rows   rows of block_sums (a sequence whose rows would fall outside
+ *              sets LSA_DEV_BAD_LENGTH and is skipped).
  * n_new        <= 0: rebuild every block of every sequence. > 0: rebuild only
  *              the blocks that hold the last n_new tokens of each sequence
  *              (the decode append update; n_new = 1 for one new token).
@@ -137,7 +139,8 @@ const char *lsa_status_string(int32_t status);
 lsa_status_t lsa_hi_block_sums(const int8_t *k_idx_cache, int32_t d_I,
                                int32_t hi_block, const lsa_batch_t *batch,
                                int32_t n_new, int8_t *block_sums,
-                               int32_t *dev_status, void *stream);
+                               int64_t block_rows, int32_t *dev_status,
+                               void *stream);
 
 /* ----------------------------------------------------------------------- */
 /* Indexer: scores, HI, top-k, SI assembly                                   */
@@ -157,7 +160,7 @@ size_t lsa_index_workspace_size(const lsa_batch_t *batch, int32_t H_I,
  * w_max        host bound on w; H_I * w_max * d_I * 16384 must be < 2^31 so
  *              that fine scores are exact in int32 (else LSA_ERR_UNSUPPORTED).
  * block_sums   device, as written by lsa_hi_block_sums (HI on), or NULL when
- *              hi_block == 0.
+ *              hi_block == 0; block_rows is its row count.
  * index_sets   device int32 [n_q][sink+window+topk] output: positions relative
  *              to the sequence start, ascending, -1 padded.
  * workspace    device scratch of lsa_index_workspace_size() bytes (may be NULL
@@ -169,7 +172,8 @@ size_t lsa_index_workspace_size(const lsa_batch_t *batch, int32_t H_I,
 lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
                        const int32_t *w, int32_t w_max, int32_t H_I, int32_t d_I,
                        const lsa_batch_t *batch, lsa_budget_t budget,
-                       const int8_t *block_sums, int32_t *index_sets,
+                       const int8_t *block_sums, int64_t block_rows,
+                       int32_t *index_sets,
                        void *workspace, size_t workspace_bytes,
                        int32_t *dev_status, void *stream);
 

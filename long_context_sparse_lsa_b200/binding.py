@@ -1,0 +1,198 @@
+"""Python binding of liblsa.so (include/lsa.h): argument marshalling only.
+
+Every function takes torch tensors, passes their device pointers and sizes to
+the C ABI on the current CUDA stream, and raises LsaError on a non-zero
+status. Every step of the hot path runs in the library's CUDA kernels; there
+is no fallback. If the library is missing, loading it raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblsa.so")
+
+LSA_DEV_BAD_LENGTH = 0x1
+LSA_DEV_BAD_SEQ = 0x2
+LSA_DEV_BAD_INDEX = 0x4
+LSA_DEV_BAD_WEIGHT = 0x8
+
+STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "LSA_ERR_CUDA",
+          4: "LSA_ERR_WORKSPACE"}
+
+EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums",
+           "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend"]
+
+
+class LsaError(RuntimeError):
+    def __init__(self, func: str, status: int, cuda_error: int = 0):
+        self.status = status
+        self.cuda_error = cuda_error
+        msg = f"{func} failed: {STATUS.get(status, status)}"
+        if status == 3:
+            msg += f" (cudaError {cuda_error})"
+        super().__init__(msg)
+
+
+class _Budget(ctypes.Structure):
+    _fields_ = [("sink", ctypes.c_int32), ("window", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("hi_block", ctypes.c_int32), ("hi_topblocks", ctypes.c_int32)]
+
+
+class _Batch(ctypes.Structure):
+    _fields_ = [("n_seq", ctypes.c_int32), ("n_q", ctypes.c_int32), ("max_len", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("total_tokens", ctypes.c_int64),
+                ("kv_offset", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p), ("blk_offset", ctypes.c_void_p),
+                ("q_seq", ctypes.c_void_p), ("q_len", ctypes.c_void_p)]
+
+
+@dataclass
+class Budget:
+    sink: int
+    window: int
+    topk: int
+    hi_block: int = 0
+    hi_topblocks: int = 0
+
+    @property
+    def length(self) -> int:
+        return self.sink + self.window + self.topk
+
+    def c(self) -> _Budget:
+        return _Budget(self.sink, self.window, self.topk, self.hi_block, self.hi_topblocks)
+
+
+@dataclass
+class Batch:
+    """Packed-sequence batch; tensors live on the device that runs the call."""
+    kv_offset: torch.Tensor   # int64 [n_seq]
+    seq_lens: torch.Tensor    # int32 [n_seq]
+    q_seq: torch.Tensor       # int32 [n_q]
+    q_len: torch.Tensor       # int32 [n_q]
+    max_len: int
+    total_tokens: int
+    blk_offset: torch.Tensor | None = None  # int64 [n_seq]
+
+    def c(self) -> _Batch:
+        for name, t, dt in (("kv_offset", self.kv_offset, torch.int64), ("seq_lens", self.seq_lens, torch.int32),
+                            ("q_seq", self.q_seq, torch.int32), ("q_len", self.q_len, torch.int32)):
+            if t.dtype != dt or not t.is_contiguous():
+                raise TypeError(f"{name} must be a contiguous {dt} tensor")
+        if self.blk_offset is not None and (self.blk_offset.dtype != torch.int64 or not self.blk_offset.is_contiguous()):
+            raise TypeError("blk_offset must be a contiguous int64 tensor")
+        return _Batch(int(self.seq_lens.numel()), int(self.q_seq.numel()), int(self.max_len), 0,
+                      int(self.total_tokens), self.kv_offset.data_ptr(), self.seq_lens.data_ptr(),
+                      self.blk_offset.data_ptr() if self.blk_offset is not None else None,
+                      self.q_seq.data_ptr(), self.q_len.data_ptr())
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load liblsa.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m long_context_sparse_lsa_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.lsa_version.restype = i32
+    lib.lsa_version.argtypes = []
+    lib.lsa_last_cuda_error.restype = i32
+    lib.lsa_last_cuda_error.argtypes = []
+    lib.lsa_status_string.restype = ctypes.c_char_p
+    lib.lsa_status_string.argtypes = [i32]
+    lib.lsa_hi_block_sums.restype = i32
+    lib.lsa_hi_block_sums.argtypes = [vp, i32, i32, ctypes.POINTER(_Batch), i32, vp, i64, vp, vp]
+    lib.lsa_index_workspace_size.restype = sz
+    lib.lsa_index_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
+    lib.lsa_index.restype = i32
+    lib.lsa_index.argtypes = [vp, vp, vp, i32, i32, i32, ctypes.POINTER(_Batch), _Budget, vp, i64, vp, vp, sz, vp, vp]
+    lib.lsa_attend_workspace_size.restype = sz
+    lib.lsa_attend_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, i32, i32, i32]
+    lib.lsa_attend.restype = i32
+    lib.lsa_attend.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp, i32,
+                               ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, sz, vp, vp]
+    _lib = lib
+    return lib
+
+
+def _check(func: str, status: int):
+    if status != 0:
+        raise LsaError(func, status, load_library().lsa_last_cuda_error() if status == 3 else 0)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def lsa_version() -> int:
+    return load_library().lsa_version()
+
+
+def lsa_hi_block_sums(k_idx: torch.Tensor, hi_block: int, batch: Batch, block_sums: torch.Tensor,
+                      n_new: int = 0, dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """HI block sums into ``block_sums`` (int8 [rows, 2*d_I]); n_new > 0 only
+    refreshes the blocks holding each sequence's last n_new tokens."""
+    lib = load_library()
+    d_I = k_idx.shape[-1]
+    cb = batch.c()
+    st = lib.lsa_hi_block_sums(_ptr(k_idx), d_I, hi_block, ctypes.byref(cb), n_new, _ptr(block_sums),
+                               block_sums.shape[0], _ptr(dev_status), _stream(stream))
+    _check("lsa_hi_block_sums", st)
+
+
+def lsa_index_workspace_size(batch: Batch, H_I: int, d_I: int, budget: Budget) -> int:
+    cb = batch.c()
+    return int(load_library().lsa_index_workspace_size(ctypes.byref(cb), H_I, d_I, budget.c()))
+
+
+def lsa_index(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, w_max: int, batch: Batch,
+              budget: Budget, index_sets: torch.Tensor, block_sums: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """Index sets [n_q, sink+window+topk] (int32) into ``index_sets``."""
+    lib = load_library()
+    n_q, H_I, d_I = q_idx.shape
+    cb = batch.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.lsa_index(_ptr(q_idx), _ptr(k_idx), _ptr(w), w_max, H_I, d_I, ctypes.byref(cb), budget.c(),
+                       _ptr(block_sums), 0 if block_sums is None else block_sums.shape[0], _ptr(index_sets),
+                       _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    _check("lsa_index", st)
+
+
+def lsa_attend_workspace_size(batch: Batch, H_q: int, H_kv: int, d: int, budget: int, layers: int) -> int:
+    cb = batch.c()
+    return int(load_library().lsa_attend_workspace_size(ctypes.byref(cb), H_q, H_kv, d, budget, layers))
+
+
+def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list,
+               workspace: torch.Tensor, dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """Sparse attention of G layers (lists of G tensors) over one index set per row."""
+    lib = load_library()
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k[0].shape[1]
+    arr = ctypes.c_void_p * G
+    qa, ka, va, oa = (arr(*[t.data_ptr() for t in x]) for x in (q, k, v, out))
+    cb = batch.c()
+    st = lib.lsa_attend(qa, ka, va, H_q, H_kv, d, _ptr(index_sets), index_sets.shape[1], ctypes.byref(cb), G, oa,
+                        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                        _stream(stream))
+    _check("lsa_attend", st)

@@ -1,0 +1,312 @@
+// abi.cu — the extern "C" entry points of liblsa.so (declared in
+// include/lsa.h): argument validation, launch planning, and the launches.
+// Every check that can be made on the host is made here, before any launch;
+// nothing in this file allocates device memory or synchronises.
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "internal.h"
+
+namespace {
+
+thread_local int32_t g_last_cuda = 0;
+
+lsa_status_t cuda_fail(cudaError_t e) {
+    g_last_cuda = (int32_t)e;
+    return LSA_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool batch_ok(const lsa_batch_t* b, bool need_queries) {
+    if (b == nullptr) return false;
+    if (b->n_seq < 1 || b->n_q < 0 || b->max_len < 1 || b->reserved != 0 || b->total_tokens < 0) return false;
+    if (b->kv_offset == nullptr || b->seq_lens == nullptr) return false;
+    if (need_queries && b->n_q > 0 && (b->q_seq == nullptr || b->q_len == nullptr)) return false;
+    return true;
+}
+
+bool budget_ok(const lsa_budget_t& b) {
+    return b.sink >= 0 && b.window >= 0 && b.topk >= 0 && b.hi_block >= 0 && b.hi_topblocks >= 0;
+}
+
+int64_t budget_len(const lsa_budget_t& b) { return (int64_t)b.sink + b.window + b.topk; }
+
+std::mutex g_mu;
+std::map<int, int> g_sms;
+std::map<std::tuple<int, int, int, int, int64_t, int, int, int, int, int>, lsa::IndexPlan> g_index_plans;
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return dev;
+}
+
+}  // namespace
+
+namespace lsa {
+int device_sm_count() {
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_sms.find(dev);
+    if (it != g_sms.end()) return it->second;
+    int n = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 148;  // B200
+    }
+    g_sms[dev] = n;
+    return n;
+}
+}  // namespace lsa
+
+extern "C" {
+
+int32_t lsa_version(void) { return 100; }
+
+int32_t lsa_last_cuda_error(void) { return g_last_cuda; }
+
+const char* lsa_status_string(int32_t status) {
+    switch (status) {
+        case LSA_OK: return "LSA_OK";
+        case LSA_ERR_INVALID_ARG: return "LSA_ERR_INVALID_ARG";
+        case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED";
+        case LSA_ERR_CUDA: return "LSA_ERR_CUDA";
+        case LSA_ERR_WORKSPACE: return "LSA_ERR_WORKSPACE";
+        default: return "LSA_ERR_UNKNOWN";
+    }
+}
+
+// ---------------------------------------------------------------------------
+lsa_status_t lsa_hi_block_sums(const int8_t* k_idx_cache, int32_t d_I, int32_t hi_block, const lsa_batch_t* batch,
+                               int32_t n_new, int8_t* block_sums, int64_t block_rows, int32_t* dev_status,
+                               void* stream) {
+    if (!batch_ok(batch, false)) return LSA_ERR_INVALID_ARG;
+    if (k_idx_cache == nullptr || block_sums == nullptr || batch->blk_offset == nullptr || block_rows < 0)
+        return LSA_ERR_INVALID_ARG;
+    if (hi_block < 1 || d_I < 1) return LSA_ERR_INVALID_ARG;
+    if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+    if (hi_block > LSA_MAX_HI_BLOCK) return LSA_ERR_UNSUPPORTED;
+    if (!aligned(k_idx_cache, 16) || !aligned(block_sums, 16)) return LSA_ERR_INVALID_ARG;
+    lsa::BlockSumArgs a;
+    a.k_idx = k_idx_cache;
+    a.block_sums = block_sums;
+    a.kv_offset = batch->kv_offset;
+    a.seq_lens = batch->seq_lens;
+    a.blk_offset = batch->blk_offset;
+    a.dev_status = dev_status;
+    a.total_tokens = batch->total_tokens;
+    a.block_rows = block_rows;
+    a.n_seq = batch->n_seq;
+    a.max_len = batch->max_len;
+    a.hi_block = hi_block;
+    a.n_new = n_new;
+    const int64_t full = ((int64_t)batch->max_len + hi_block - 1) / hi_block;
+    int64_t cover = n_new > 0 ? ((int64_t)n_new + hi_block - 1) / hi_block + 1 : full;
+    if (cover > full) cover = full;
+    a.blocks_per_seq = (int32_t)cover;
+    if (batch->n_seq > 65535) return LSA_ERR_UNSUPPORTED;
+    cudaError_t e = lsa::launch_block_sums(a, d_I, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+// ---------------------------------------------------------------------------
+size_t lsa_index_workspace_size(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, lsa_budget_t budget) {
+    (void)H_I;
+    (void)d_I;
+    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1 || !budget_ok(budget)) return 0;
+    size_t best = 0;
+    for (int C : {1, 2, 4, 8, 16}) {
+        lsa::IndexPlan p = lsa::plan_index(C, batch->n_q, batch->max_len, budget);
+        size_t need = (p.ws_coarse + 255) / 256 * 256 + (p.ws_fine + 255) / 256 * 256;
+        if (need > best) best = need;
+    }
+    return best;
+}
+
+static lsa_status_t index_validate(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max,
+                                   int32_t H_I, int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget,
+                                   const int8_t* block_sums, int64_t block_rows, const int32_t* index_sets) {
+    if (!batch_ok(batch, true) || !budget_ok(budget)) return LSA_ERR_INVALID_ARG;
+    if (H_I < 1 || d_I < 1 || w_max < 0) return LSA_ERR_INVALID_ARG;
+    if (batch->n_q > 0 && (q_idx == nullptr || k_idx_cache == nullptr || w == nullptr || index_sets == nullptr))
+        return LSA_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(k_idx_cache, 16) || !aligned(w, 4) || !aligned(index_sets, 4))
+        return LSA_ERR_INVALID_ARG;
+    if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+    if (H_I > LSA_MAX_HEADS_I) return LSA_ERR_UNSUPPORTED;
+    if (budget_len(budget) > LSA_MAX_BUDGET) return LSA_ERR_UNSUPPORTED;
+    // fine scores are exact in int32 when H_I * w_max * d_I * 128 * 128 < 2^31
+    if ((double)H_I * (double)w_max * (double)d_I * 16384.0 >= 2147483648.0) return LSA_ERR_UNSUPPORTED;
+    if (budget.hi_block > 0) {
+        if (budget.hi_block > LSA_MAX_HI_BLOCK || budget.hi_topblocks > LSA_MAX_TOPBLOCKS) return LSA_ERR_UNSUPPORTED;
+        if (block_sums == nullptr || batch->blk_offset == nullptr || block_rows < 0) return LSA_ERR_INVALID_ARG;
+        if (!aligned(block_sums, 16)) return LSA_ERR_INVALID_ARG;
+    }
+    return LSA_OK;
+}
+
+lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max, int32_t H_I,
+                       int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget, const int8_t* block_sums,
+                       int64_t block_rows, int32_t* index_sets, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, void* stream) {
+    lsa_status_t st = index_validate(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums, block_rows,
+                                     index_sets);
+    if (st != LSA_OK) return st;
+    if (batch->n_q == 0) return LSA_OK;
+    if (budget.hi_block == 0) budget.hi_topblocks = 0;
+
+    const int dev = current_device();
+    lsa::IndexPlan plan;
+    {
+        const auto key = std::make_tuple(dev, d_I, (H_I + 7) / 8, batch->n_q, (int64_t)batch->max_len, budget.sink,
+                                         budget.window, budget.topk, budget.hi_block, budget.hi_topblocks);
+        std::unique_lock<std::mutex> lk(g_mu);
+        auto it = g_index_plans.find(key);
+        if (it != g_index_plans.end()) {
+            plan = it->second;
+        } else {
+            lk.unlock();
+            cudaError_t e = lsa::choose_index_cluster(d_I, H_I, batch->n_q, batch->max_len, budget, &plan);
+            if (e != cudaSuccess) return cuda_fail(e);
+            lk.lock();
+            g_index_plans[key] = plan;
+        }
+    }
+    const size_t need_c = (plan.ws_coarse + 255) / 256 * 256;
+    const size_t need = need_c + (plan.ws_fine + 255) / 256 * 256;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
+        return LSA_ERR_WORKSPACE;
+    if ((int64_t)batch->n_q * plan.cluster > 0x7fffffffLL) return LSA_ERR_UNSUPPORTED;
+
+    lsa::IndexArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.q_idx = q_idx;
+    a.k_idx = k_idx_cache;
+    a.w = w;
+    a.block_sums = block_sums;
+    a.index_sets = index_sets;
+    a.dev_status = dev_status;
+    a.kv_offset = batch->kv_offset;
+    a.seq_lens = batch->seq_lens;
+    a.blk_offset = batch->blk_offset;
+    a.q_seq = batch->q_seq;
+    a.q_len = batch->q_len;
+    a.total_tokens = batch->total_tokens;
+    a.block_rows = block_rows;
+    a.n_seq = batch->n_seq;
+    a.n_q = batch->n_q;
+    a.max_len = batch->max_len;
+    a.H_I = H_I;
+    a.w_max = w_max;
+    a.sink = budget.sink;
+    a.window = budget.window;
+    a.topk = budget.topk;
+    a.hi_block = budget.hi_block;
+    a.hi_topblocks = budget.hi_topblocks;
+    a.budget = (int32_t)budget_len(budget);
+    a.coarse_cap = plan.coarse_cap;
+    a.fine_cap = plan.fine_cap;
+    a.kept_cap = plan.kept_cap;
+    a.smem_coarse = plan.smem_coarse;
+    a.smem_fine = plan.smem_fine;
+    a.smem_kept = plan.smem_kept;
+    a.smem_kept_local = plan.smem_kept_local;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.g_coarse = plan.ws_coarse ? reinterpret_cast<uint64_t*>(ws) : nullptr;
+    a.g_fine = plan.ws_fine ? reinterpret_cast<uint32_t*>(ws + need_c) : nullptr;
+    cudaError_t e = lsa::launch_index(a, plan, d_I, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+// ---------------------------------------------------------------------------
+static bool attend_shape_ok(int32_t H_q, int32_t H_kv, int32_t d, int32_t budget, int32_t G) {
+    if (d != 128) return false;
+    if (H_kv < 1 || H_q < 1 || H_q % H_kv != 0) return false;
+    const int ratio = H_q / H_kv;
+    if (ratio != 1 && ratio != 2 && ratio != 4 && ratio != 8 && ratio != 16) return false;
+    if (!(H_kv == 1 || H_kv == 2 || H_kv == 4 || H_kv % 4 == 0)) return false;
+    if (G < 1 || G > LSA_MAX_LAYERS) return false;
+    if (budget < 0 || budget > LSA_MAX_BUDGET) return false;
+    return true;
+}
+
+size_t lsa_attend_workspace_size(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, int32_t budget,
+                                 int32_t layers_per_index) {
+    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1) return 0;
+    if (!attend_shape_ok(H_q, H_kv, d, budget, layers_per_index)) return 0;
+    lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, budget, layers_per_index,
+                                         lsa::device_sm_count());
+    return p.ws_bytes;
+}
+
+lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache, const uint16_t* const* v_cache,
+                        int32_t H_q, int32_t H_kv, int32_t d, const int32_t* index_sets, int32_t budget,
+                        const lsa_batch_t* batch, int32_t layers_per_index, float* const* out, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    if (!batch_ok(batch, true)) return LSA_ERR_INVALID_ARG;
+    if (H_q < 1 || H_kv < 1 || d < 1 || budget < 0 || layers_per_index < 1) return LSA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return LSA_ERR_INVALID_ARG;
+    if (!attend_shape_ok(H_q, H_kv, d, budget, layers_per_index)) return LSA_ERR_UNSUPPORTED;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr) return LSA_ERR_INVALID_ARG;
+    if (batch->n_q == 0) return LSA_OK;
+    if (budget > 0 && (index_sets == nullptr || !aligned(index_sets, 4))) return LSA_ERR_INVALID_ARG;
+    for (int g = 0; g < layers_per_index; ++g) {
+        if (q[g] == nullptr || k_cache[g] == nullptr || v_cache[g] == nullptr || out[g] == nullptr)
+            return LSA_ERR_INVALID_ARG;
+        if (!aligned(q[g], 16) || !aligned(k_cache[g], 16) || !aligned(v_cache[g], 16) || !aligned(out[g], 16))
+            return LSA_ERR_INVALID_ARG;
+    }
+    if ((int64_t)batch->n_q > 65535) return LSA_ERR_UNSUPPORTED;
+    lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, budget, layers_per_index,
+                                         lsa::device_sm_count());
+    if (workspace == nullptr || workspace_bytes < p.ws_bytes || !aligned(workspace, 256)) return LSA_ERR_WORKSPACE;
+    lsa::AttendArgs a;
+    std::memset(&a, 0, sizeof a);
+    for (int g = 0; g < layers_per_index; ++g) {
+        a.q[g] = q[g];
+        a.k[g] = k_cache[g];
+        a.v[g] = v_cache[g];
+        a.out[g] = out[g];
+    }
+    a.sets = index_sets;
+    a.kv_offset = batch->kv_offset;
+    a.seq_lens = batch->seq_lens;
+    a.q_seq = batch->q_seq;
+    a.q_len = batch->q_len;
+    a.dev_status = dev_status;
+    const size_t rows_q = (size_t)layers_per_index * batch->n_q;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.counters = reinterpret_cast<uint32_t*>(ws);
+    size_t off = (rows_q * 4 + 255) / 256 * 256;
+    const size_t n_parts = (size_t)p.n_splits * p.wph;
+    if (n_parts > 1) {
+        a.part_o = reinterpret_cast<float*>(ws + off);
+        off += rows_q * n_parts * H_q * 128 * 4;
+        off = (off + 255) / 256 * 256;
+        a.part_ml = reinterpret_cast<float*>(ws + off);
+    }
+    a.total_tokens = batch->total_tokens;
+    a.n_seq = batch->n_seq;
+    a.n_q = batch->n_q;
+    a.max_len = batch->max_len;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.budget = budget;
+    a.G = layers_per_index;
+    a.n_splits = p.n_splits;
+    a.entries_per_split = p.entries_per_split;
+    a.wph = p.wph;
+    a.head_groups = p.head_groups;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    cudaError_t e = lsa::launch_attend(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

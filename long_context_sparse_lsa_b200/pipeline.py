@@ -1,0 +1,61 @@
+"""A decode step of the LSA hot path over one workload, through the C ABI.
+
+Allocation and call sequencing only (device buffers via torch, calls via
+``binding``): the HI block-sum append update, one ``lsa_index`` per group of
+G layers (Cross-Layer Indexing) and one ``lsa_attend`` for the G layers.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as lsa
+from .workloads import Tensors, Workload
+
+
+class LsaStep:
+    def __init__(self, wl: Workload, t: Tensors, device="cuda"):
+        self.wl = wl
+        self.t = t
+        self.device = device
+        self.G = len(t.q)
+        self.batch = lsa.Batch(t.kv_offset, t.seq_lens, t.q_seq, t.q_len, max(wl.lens), wl.total_tokens,
+                               t.blk_offset if wl.hi_block > 0 else None)
+        self.budget = lsa.Budget(wl.sink, wl.window, wl.topk, wl.hi_block, wl.hi_topblocks)
+        n_q = wl.n_q
+        self.sets = torch.empty((n_q, self.budget.length), dtype=torch.int32, device=device)
+        self.out = [torch.empty((n_q, wl.H_q, wl.d), dtype=torch.float32, device=device) for _ in range(self.G)]
+        self.block_sums = None
+        if wl.hi_block > 0:
+            self.block_sums = torch.zeros((max(1, t.n_blk_rows), 2 * wl.d_I), dtype=torch.int8, device=device)
+        ws_i = lsa.lsa_index_workspace_size(self.batch, wl.H_I, wl.d_I, self.budget)
+        self.ws_index = torch.empty(max(1, ws_i), dtype=torch.uint8, device=device) if ws_i else None
+        ws_a = lsa.lsa_attend_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
+        self.ws_attend = torch.zeros(max(256, ws_a), dtype=torch.uint8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    # -- the three calls --------------------------------------------------------
+    def build_block_sums(self, stream=None):
+        if self.block_sums is not None:
+            lsa.lsa_hi_block_sums(self.t.k_idx, self.wl.hi_block, self.batch, self.block_sums, 0, self.status, stream)
+
+    def update_block_sums(self, n_new: int = 1, stream=None):
+        if self.block_sums is not None:
+            lsa.lsa_hi_block_sums(self.t.k_idx, self.wl.hi_block, self.batch, self.block_sums, n_new, self.status,
+                                  stream)
+
+    def index(self, stream=None):
+        lsa.lsa_index(self.t.q_idx, self.t.k_idx, self.t.w, self.wl.w_max, self.batch, self.budget, self.sets,
+                      self.block_sums, self.ws_index, self.status, stream)
+
+    def attend(self, stream=None):
+        lsa.lsa_attend(self.t.q, self.t.k, self.t.v, self.sets, self.batch, self.out, self.ws_attend, self.status,
+                       stream)
+
+    def step(self, stream=None):
+        """One decode step: append update of the block sums, index, attend."""
+        self.update_block_sums(1, stream)
+        self.index(stream)
+        self.attend(stream)
+
+    def status_bits(self) -> int:
+        return int(self.status.item())

@@ -1,0 +1,113 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every entry
+point include/lsa.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_sparse_lsa_b200 import binding as lsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("lsa_index", "lsa_attend", "lsa_hi_block_sums", "lsa_index_workspace_size",
+              "lsa_attend_workspace_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = lsa.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {lsa.library_path()}").read()
+    exported = set(re.findall(r" T (lsa_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_version_and_status_strings():
+    lib = lsa.load_library()
+    assert lib.lsa_version() >= 100
+    assert lib.lsa_status_string(0) == b"LSA_OK"
+    assert lib.lsa_status_string(4) == b"LSA_ERR_WORKSPACE"
+
+
+def _batch(n_seq=1, n_q=1, max_len=100, total=100, ptr=0x1000):
+    b = lsa._Batch()
+    b.n_seq, b.n_q, b.max_len, b.reserved, b.total_tokens = n_seq, n_q, max_len, 0, total
+    b.kv_offset = b.seq_lens = b.blk_offset = b.q_seq = b.q_len = ptr
+    return b
+
+
+def _budget(sink=4, window=8, topk=16, hb=0, ht=0):
+    return lsa._Budget(sink, window, topk, hb, ht)
+
+
+P = 0x10000  # a fake, 256-byte aligned device address: never dereferenced (validation fails first)
+
+
+def _index(lib, **kw):
+    args = dict(q=P, k=P, w=P, w_max=8, H_I=16, d_I=128, batch=_batch(), budget=_budget(), bs=None, rows=0,
+                sets=P, ws=None, ws_bytes=0)
+    args.update(kw)
+    return lib.lsa_index(args["q"], args["k"], args["w"], args["w_max"], args["H_I"], args["d_I"],
+                         ctypes.byref(args["batch"]), args["budget"], args["bs"], args["rows"], args["sets"],
+                         args["ws"], args["ws_bytes"], None, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(w=None), 1), (dict(sets=None), 1),
+    (dict(d_I=96), 2), (dict(d_I=0), 1), (dict(H_I=0), 1), (dict(H_I=65), 2), (dict(w_max=-1), 1),
+    (dict(w_max=1 << 20), 2),                       # fine scores would overflow int32
+    (dict(budget=_budget(sink=-1)), 1), (dict(budget=_budget(topk=20000)), 2),
+    (dict(budget=_budget(hb=64, ht=8)), 1),         # HI on without block sums
+    (dict(budget=_budget(hb=512, ht=8), bs=P, rows=10), 2),
+    (dict(budget=_budget(hb=64, ht=5000), bs=P, rows=10), 2),
+    (dict(batch=_batch(n_seq=0)), 1), (dict(batch=_batch(max_len=0)), 1), (dict(q=P + 4), 1),
+])
+def test_index_rejects_before_launch(kw, want):
+    lib = lsa.load_library()
+    assert _index(lib, **kw) == want
+
+
+def test_index_empty_batch_is_ok_without_launch():
+    lib = lsa.load_library()
+    assert _index(lib, batch=_batch(n_q=0)) == 0
+
+
+def test_block_sums_rejects():
+    lib = lsa.load_library()
+    b = _batch()
+    f = lib.lsa_hi_block_sums
+    assert f(None, 128, 64, ctypes.byref(b), 0, P, 10, None, None) == 1
+    assert f(P, 100, 64, ctypes.byref(b), 0, P, 10, None, None) == 2
+    assert f(P, 128, 0, ctypes.byref(b), 0, P, 10, None, None) == 1
+    assert f(P, 128, 300, ctypes.byref(b), 0, P, 10, None, None) == 2
+    b.blk_offset = None
+    assert f(P, 128, 64, ctypes.byref(b), 0, P, 10, None, None) == 1
+
+
+def test_attend_rejects_and_sizes():
+    lib = lsa.load_library()
+    b = _batch(n_q=16, max_len=131072, total=16 * 131072)
+    arr = (ctypes.c_void_p * 1)(P)
+    f = lib.lsa_attend
+    assert f(arr, arr, arr, 32, 4, 64, P, 3136, ctypes.byref(b), 1, arr, P, 1 << 30, None, None) == 2  # d != 128
+    assert f(arr, arr, arr, 30, 4, 128, P, 3136, ctypes.byref(b), 1, arr, P, 1 << 30, None, None) == 1
+    assert f(arr, arr, arr, 96, 4, 128, P, 3136, ctypes.byref(b), 1, arr, P, 1 << 30, None, None) == 2  # ratio 24
+    assert f(arr, arr, arr, 32, 4, 128, P, 3136, ctypes.byref(b), 9, arr, P, 1 << 30, None, None) == 2  # G > 8
+    assert f(arr, arr, arr, 32, 4, 128, None, 3136, ctypes.byref(b), 1, arr, P, 1 << 30, None, None) == 1
+    assert f(arr, arr, arr, 32, 4, 128, P, 3136, ctypes.byref(b), 1, arr, P, 16, None, None) == 4  # workspace
+    need = lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 1)
+    assert need >= 16 * 4
+    need4 = lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 4)
+    assert need4 >= 4 * 16 * 4  # counters for every (layer, row)

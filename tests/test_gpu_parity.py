@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs. Index sets must match bit for bit; attention must satisfy
+max|err| <= 5e-3 and rel-L2 <= 1e-3 (tests/parity.py). Sizes span several
+tiles, clusters and ragged tails; the edge cases of the method (empty middle,
+budget covering the context, SI-only budgets, HI keeping every block, ties)
+each have a case."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from long_context_sparse_lsa_b200 import binding as lsa
+from long_context_sparse_lsa_b200 import workloads as wls
+from long_context_sparse_lsa_b200.pipeline import LsaStep
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def run_case(wl, check_attn=True, layers=None):
+    t = wls.make(wl, DEV, layers=layers)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    st.index()
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    want = parity.oracle_sets(wl, t)
+    parity.check_sets(parity.host(st.sets), want, wl.name)
+    if check_attn:
+        ref = parity.oracle_attend_full(t, want)
+        for g in range(len(t.q)):
+            parity.check_attention(parity.host(st.out[g]), ref[g], f"{wl.name} layer {g}")
+    return st, t
+
+
+def test_tiny_decode_workload():
+    run_case(wls.TINY)
+
+
+BASE = wls.small(wls.BATCH128K, name="small", lens=(3000,), G=1)
+
+CASES = {
+    # HI off, several clusters' worth of tiles and ragged lengths
+    "flat_ragged": dict(lens=(37, 1, 4096, 513, 2049), hi_block=0, hi_topblocks=0, sink=16, window=64, topk=300),
+    "flat_long": dict(lens=(40000,), hi_block=0, hi_topblocks=0),
+    # HI on with partial last blocks and blocks that straddle sink/window
+    "hi_ragged": dict(lens=(5000, 777, 64, 12001), hi_block=64, hi_topblocks=8, sink=70, window=100, topk=200),
+    "hi_b16": dict(lens=(6000, 3333), hi_block=16, hi_topblocks=40, topk=300, window=50, sink=3),
+    "hi_b128_many": dict(lens=(70000,), hi_block=128, hi_topblocks=300, topk=2048, window=2048, sink=64),
+    "hi_b256": dict(lens=(20000, 9000), hi_block=256, hi_topblocks=20, topk=1000, window=300, sink=10),
+    "hi_all_blocks_kept": dict(lens=(4000,), hi_block=64, hi_topblocks=4096, topk=500, window=100, sink=10),
+    "hi_b1_like_flat": dict(lens=(3000,), hi_block=1, hi_topblocks=600, topk=500, window=100, sink=10),
+    # budgets: covering the context, SI only, no sink / no window
+    "dense_equivalent": dict(lens=(900, 50, 1), hi_block=0, hi_topblocks=0, sink=64, window=512, topk=400),
+    "si_only": dict(lens=(5000,), hi_block=0, hi_topblocks=0, sink=32, window=256, topk=0),
+    "no_sink_no_window": dict(lens=(3000, 2000), hi_block=0, hi_topblocks=0, sink=0, window=0, topk=777),
+    "hi_empty_middle": dict(lens=(1000,), hi_block=64, hi_topblocks=4, sink=600, window=600, topk=100),
+    # ties: a tiny value range makes many equal scores
+    "ties": dict(lens=(9000,), hi_block=0, hi_topblocks=0, qk_lo=-1, qk_hi=1, w_hi=1, topk=1000),
+    "ties_hi": dict(lens=(9000,), hi_block=32, hi_topblocks=50, qk_lo=-1, qk_hi=1, w_hi=1, topk=1000),
+    # indexer head counts and key widths
+    "heads1_d32": dict(lens=(5000,), H_I=1, d_I=32, qk_lo=-128, qk_hi=127, w_hi=16, hi_block=0, hi_topblocks=0),
+    "heads20_d64": dict(lens=(7000, 100), H_I=20, d_I=64, hi_block=32, hi_topblocks=30),
+    "heads64": dict(lens=(4000,), H_I=64, d_I=128, qk_lo=-16, qk_hi=15, w_hi=4, hi_block=0, hi_topblocks=0),
+    "full_int8_range": dict(lens=(6000,), H_I=8, d_I=128, qk_lo=-128, qk_hi=127, w_hi=2, hi_block=64,
+                            hi_topblocks=16),
+    # attention shapes: GQA ratios and kv-head counts
+    "gqa_1to1": dict(lens=(2000,), H_q=4, H_kv=4, hi_block=0, hi_topblocks=0),
+    "gqa_16": dict(lens=(2000, 300), H_q=32, H_kv=2, hi_block=0, hi_topblocks=0),
+    "gqa_kv8": dict(lens=(2500,), H_q=16, H_kv=8, hi_block=0, hi_topblocks=0),
+    "gqa_kv1": dict(lens=(2500,), H_q=4, H_kv=1, hi_block=0, hi_topblocks=0),
+    # cross-layer indexing: one set, three layers
+    "cli_g3": dict(lens=(3000, 1500), G=3, hi_block=64, hi_topblocks=10),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_small_cases(name):
+    kw = dict(CASES[name])
+    kw.setdefault("seed", 100 + sorted(CASES).index(name))
+    wl = wls.small(BASE, name=name, **kw)
+    run_case(wl)
+
+
+def test_prefill_rows_through_decode_kernel():
+    """Many rows of one sequence with causal visible lengths (a prefill chunk)."""
+    wl = wls.small(wls.PREFILL, name="prefill_small", lens=(3000 + 200,), prefill_new=200, seed=7)
+    run_case(wl)
+
+
+def test_dense_equivalence_matches_textbook_attention():
+    wl = wls.small(BASE, name="dense", lens=(600,), hi_block=0, hi_topblocks=0, sink=8, window=100, topk=600,
+                   seed=11)
+    st, t = run_case(wl, check_attn=False)
+    sets = parity.host(st.sets)
+    assert [x for x in sets[0] if x >= 0] == list(range(600))
+    q = parity.u16(t.q[0])[0]
+    k = parity.u16(t.k[0])
+    v = parity.u16(t.v[0])
+    f = lambda b: (np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64)
+    qf, kf, vf = f(q), f(k), f(v)
+    H_q, H_kv = qf.shape[0], kf.shape[1]
+    want = np.zeros_like(qf)
+    for h in range(H_q):
+        kvh = h * H_kv // H_q
+        z = kf[:, kvh] @ qf[h] / np.sqrt(128.0)
+        p = np.exp(z - z.max())
+        want[h] = p @ vf[:, kvh] / p.sum()
+    parity.check_attention(parity.host(st.out[0])[0], want, "dense textbook")
+
+
+def test_block_sums_exact_and_append_update():
+    wl = wls.small(BASE, name="bsums", lens=(1000, 64, 1, 5000), hi_block=64, hi_topblocks=8, seed=21)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    torch.cuda.synchronize()
+    orc = oracle.get()
+    got = parity.decode_block_sums(st.block_sums, wl.d_I)
+    k = parity.host(t.k_idx)
+    offs = parity.host(t.kv_offset)
+    boffs = parity.host(t.blk_offset)
+    for b, L in enumerate(wl.lens):
+        want = orc.block_sums(k[offs[b]:offs[b] + L], wl.hi_block)
+        np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
+    # overwrite the last 3 tokens of every sequence, refresh with n_new = 3
+    for b, L in enumerate(wl.lens):
+        lo = max(0, L - 3)
+        t.k_idx[offs[b] + lo:offs[b] + L] = 7
+    st.update_block_sums(3)
+    torch.cuda.synchronize()
+    got = parity.decode_block_sums(st.block_sums, wl.d_I)
+    k = parity.host(t.k_idx)
+    for b, L in enumerate(wl.lens):
+        want = orc.block_sums(k[offs[b]:offs[b] + L], wl.hi_block)
+        np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
+
+
+def test_extreme_block_sums_hi_block_256():
+    """|S| reaches 128 * 256 = 32768: the byte planes stay exact."""
+    wl = wls.small(BASE, name="bs_extreme", lens=(512,), hi_block=256, hi_topblocks=1, seed=3)
+    t = wls.make(wl, DEV)
+    t.k_idx[:256] = -128
+    t.k_idx[256:] = 127
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    torch.cuda.synchronize()
+    got = parity.decode_block_sums(st.block_sums, wl.d_I)
+    assert np.all(got[0] == -32768) and np.all(got[1] == 127 * 256)
+
+
+def test_device_status_flags():
+    wl = wls.small(BASE, name="status", lens=(2000, 3000), hi_block=0, hi_topblocks=0, seed=5)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    # a query whose visible length exceeds its sequence
+    st.t.q_len[1] = 5000
+    st.index()
+    torch.cuda.synchronize()
+    assert st.status_bits() & lsa.LSA_DEV_BAD_LENGTH
+    assert np.all(parity.host(st.sets)[1] == -1)
+    # corrupted index-set entries are skipped and flagged
+    st.t.q_len[1] = 3000
+    st.status.zero_()
+    st.index()
+    sets = st.sets.clone()
+    sets[0, 5] = 999999
+    sets[0, 6] = -7
+    lsa.lsa_attend(t.q, t.k, t.v, sets, st.batch, st.out, st.ws_attend, st.status)
+    torch.cuda.synchronize()
+    assert st.status_bits() & lsa.LSA_DEV_BAD_INDEX
+    assert np.all(np.isfinite(parity.host(st.out[0])))
+    # head weight above w_max
+    st.status.zero_()
+    t.w[0, 0] = wl.w_max + 1
+    st.index()
+    torch.cuda.synchronize()
+    assert st.status_bits() & lsa.LSA_DEV_BAD_WEIGHT
+
+
+def test_repeated_calls_are_deterministic():
+    wl = wls.small(BASE, name="det", lens=(20000, 17000), hi_block=64, hi_topblocks=32, seed=9)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    outs, sets = [], []
+    for _ in range(3):
+        st.index()
+        st.attend()
+        torch.cuda.synchronize()
+        sets.append(parity.host(st.sets).copy())
+        outs.append(parity.host(st.out[0]).copy())
+    assert all(np.array_equal(sets[0], s) for s in sets)
+    assert all(np.array_equal(outs[0], o) for o in outs)
