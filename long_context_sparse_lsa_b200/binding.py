@@ -196,3 +196,4 @@ def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch
                         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
                         _stream(stream))
     _check("lsa_attend", st)
+

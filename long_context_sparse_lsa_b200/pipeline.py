@@ -59,3 +59,37 @@ class LsaStep:
 
     def status_bits(self) -> int:
         return int(self.status.item())
+
+    # -- CUDA graphs ------------------------------------------------------------
+    def capture(self):
+        """Capture the three calls as CUDA graphs (block-sum append update,
+        index, attend) so a step replays without host launch overhead. The
+        graphs keep this object's buffers; changing their contents between
+        replays is how new inputs enter."""
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):  # one eager pass fills the launch-plan caches
+            self.step()
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        torch.cuda.synchronize(self.device)
+        self.graphs = {}
+        for name, fn in (("block_sums", lambda: self.update_block_sums(1)), ("index", self.index),
+                         ("attend", self.attend)):
+            if name == "block_sums" and self.block_sums is None:
+                continue
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                fn()
+            self.graphs[name] = g
+        torch.cuda.synchronize(self.device)
+        return self.graphs
+
+    def replay(self, name: str | None = None):
+        """Replay one captured call, or the whole step when name is None."""
+        if name is not None:
+            if name in self.graphs:
+                self.graphs[name].replay()
+            return
+        for n in ("block_sums", "index", "attend"):
+            if n in self.graphs:
+                self.graphs[n].replay()

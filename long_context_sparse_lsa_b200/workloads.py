@@ -73,13 +73,20 @@ PREFILL = Workload("prefill_8192_on_262144", 3, (262144 + 8192,), 16, 128, -16, 
                    note="causal prefill chunk of 8192 tokens on a 262144-token cache, HI off")
 
 
+# The batched-decode shape on a 32768-token context: the same per-query
+# attention and fine-index work as the 128K case on a 4x smaller cache, for
+# profiler captures that must stay a few GB on the device.
+PROFILE32K = Workload("decode_b16_32k_hi64x256", 1, (32768,) * 16, 16, 128, -16, 15, 8, 64, 1024, 2048,
+                      64, 256, 32, 4, 128, 1, note="batched decode, 16 seqs x 32768, HI 64x256 (profiling size)")
+
+
 def ragged() -> Workload:
     return Workload("ragged_decode_64seq_lognormal", 4, _ragged_lens(4), 16, 128, -16, 15, 8, 64, 1024, 2048,
                     64, 256, 32, 4, 128, 2, note="64 ragged seqs, lognormal median 32768, G=2, HI 64x256")
 
 
 def all_workloads() -> list[Workload]:
-    return [TINY, BATCH128K, CTX1M, PREFILL, ragged()]
+    return [TINY, BATCH128K, CTX1M, PREFILL, ragged(), PROFILE32K]
 
 
 def by_name(name: str) -> Workload:

@@ -195,3 +195,26 @@ def test_repeated_calls_are_deterministic():
         outs.append(parity.host(st.out[0]).copy())
     assert all(np.array_equal(sets[0], s) for s in sets)
     assert all(np.array_equal(outs[0], o) for o in outs)
+
+
+def test_graph_replay_matches_eager():
+    wl = wls.small(BASE, name="graph", lens=(30000, 4000, 9000), hi_block=64, hi_topblocks=64, G=2, seed=13)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    st.step()
+    torch.cuda.synchronize()
+    sets0 = parity.host(st.sets).copy()
+    outs0 = [parity.host(o).copy() for o in st.out]
+    st.capture()
+    st.sets.fill_(-5)
+    for o in st.out:
+        o.fill_(float("nan"))
+    for _ in range(2):
+        st.replay()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    np.testing.assert_array_equal(parity.host(st.sets), sets0)
+    for g in range(len(outs0)):
+        np.testing.assert_array_equal(parity.host(st.out[g]), outs0[g])
+    parity.check_sets(sets0, parity.oracle_sets(wl, t), "graph")
