@@ -209,6 +209,38 @@ lsa_status_t lsa_attend(const uint16_t *const *q, const uint16_t *const *k_cache
                         float *const *out, void *workspace, size_t workspace_bytes,
                         int32_t *dev_status, void *stream);
 
+/* ----------------------------------------------------------------------- */
+/* Allocation-free attention (no counterpart in the pages)                   */
+/* ----------------------------------------------------------------------- */
+/* Largest scratch lsa_attend_noalloc can use. Every GPU on which the library
+ * is loaded holds one array of this size until the process exits. */
+#define LSA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* lsa_attend without a workspace argument, for callers that cannot call
+ * cudaMalloc on this path: an engine whose device memory belongs entirely to
+ * its own pool allocator, or a decode loop that must not run an allocation
+ * (cudaMalloc and cudaFree can synchronise the device). The scratch that
+ * lsa_attend takes as `workspace` lives instead in a static device array of
+ * LSA_NOALLOC_SCRATCH_BYTES bytes inside the library; nothing is allocated.
+ *
+ * Arguments, output and device-side errors are those of lsa_attend. The
+ * caller still owns and passes every input and output buffer.
+ *  - A shape whose lsa_attend_workspace_size() exceeds
+ *    LSA_NOALLOC_SCRATCH_BYTES returns LSA_ERR_UNSUPPORTED before any launch.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls on a device share the one array, which keeps the previous
+ *    call's contents. Each call clears the part that must start at zero (on
+ *    `stream`) before its kernel runs. Calls that overlap on the GPU (other
+ *    streams, other host threads on the same device) race on the array:
+ *    order them on one stream.
+ */
+lsa_status_t lsa_attend_noalloc(const uint16_t *const *q, const uint16_t *const *k_cache,
+                                const uint16_t *const *v_cache, int32_t H_q, int32_t H_kv,
+                                int32_t d, const int32_t *index_sets, int32_t budget,
+                                const lsa_batch_t *batch, int32_t layers_per_index,
+                                float *const *out, int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

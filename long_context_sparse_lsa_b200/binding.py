@@ -25,7 +25,8 @@ STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "L
           4: "LSA_ERR_WORKSPACE"}
 
 EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums",
-           "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend"]
+           "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend",
+           "lsa_attend_noalloc"]
 
 
 class LsaError(RuntimeError):
@@ -123,6 +124,9 @@ def load_library():
     lib.lsa_attend.restype = i32
     lib.lsa_attend.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp, i32,
                                ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, sz, vp, vp]
+    lib.lsa_attend_noalloc.restype = i32
+    lib.lsa_attend_noalloc.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
+                                       i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, vp]
     _lib = lib
     return lib
 
@@ -197,3 +201,19 @@ def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch
                         _stream(stream))
     _check("lsa_attend", st)
 
+
+def lsa_attend_noalloc(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list,
+                       dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """lsa_attend without a workspace: for callers that cannot allocate device
+    memory on this path; the library's fixed static scratch is used instead
+    (see include/lsa.h for the size limit and the sharing rules)."""
+    lib = load_library()
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k[0].shape[1]
+    arr = ctypes.c_void_p * G
+    qa, ka, va, oa = (arr(*[t.data_ptr() for t in x]) for x in (q, k, v, out))
+    cb = batch.c()
+    st = lib.lsa_attend_noalloc(qa, ka, va, H_q, H_kv, d, _ptr(index_sets), index_sets.shape[1], ctypes.byref(cb),
+                                G, oa, _ptr(dev_status), _stream(stream))
+    _check("lsa_attend_noalloc", st)
