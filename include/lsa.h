@@ -40,8 +40,10 @@
  *    are OR-ed as LSA_DEV_* bits into *dev_status (device int32, may be
  *    NULL); the caller reads it after synchronising. The offending query's
  *    output is then unspecified but every access stays in bounds.
- *  - No kernel in this library waits on another CTA, kernel or device, so no
- *    call can hang; no kernel traps.
+ *  - No kernel waits on another CTA, kernel or device. Waits inside a CTA
+ *    (on its own asynchronous copies) are bounded by a time limit after which
+ *    the kernel sets LSA_DEV_TIMEOUT and returns, so no call can hang; no
+ *    kernel traps.
  *  - Calls are thread-safe when they use distinct workspaces.
  */
 #ifndef LSA_H_
@@ -67,6 +69,7 @@ typedef enum {
 #define LSA_DEV_BAD_SEQ 0x2    /* q_seq outside [0, n_seq) */
 #define LSA_DEV_BAD_INDEX 0x4  /* an index-set entry < -1 or >= q_len (entry skipped) */
 #define LSA_DEV_BAD_WEIGHT 0x8 /* an indexer head weight outside [0, w_max] (treated as 0) */
+#define LSA_DEV_TIMEOUT 0x10   /* a bounded wait inside a kernel gave up (output unspecified) */
 
 /* Selection budget. sink + window + topk is the index-set length ("budget").
  * hi_block == 0 switches HI off; otherwise blocks of hi_block tokens aligned
@@ -180,9 +183,8 @@ lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
 /* ----------------------------------------------------------------------- */
 /* Sparse attention over the index sets (all G layers of a CLI group)        */
 /* ----------------------------------------------------------------------- */
-/* Workspace bytes lsa_attend needs. The first 4*G*n_q bytes are arrival
- * counters that must be zero before the first call; every call leaves them
- * zero again. */
+/* Workspace bytes lsa_attend needs (split partials; contents need no
+ * initialisation: every call writes what it later reads). */
 size_t lsa_attend_workspace_size(const lsa_batch_t *batch, int32_t H_q,
                                  int32_t H_kv, int32_t d, int32_t budget,
                                  int32_t layers_per_index);
@@ -230,10 +232,10 @@ lsa_status_t lsa_attend(const uint16_t *const *q, const uint16_t *const *k_cache
  *  - The first call on each device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
  *  - All calls on a device share the one array, which keeps the previous
- *    call's contents. Each call clears the part that must start at zero (on
- *    `stream`) before its kernel runs. Calls that overlap on the GPU (other
- *    streams, other host threads on the same device) race on the array:
- *    order them on one stream.
+ *    call's contents; nothing in it needs to start at zero, because every
+ *    call writes the scratch it later reads. Calls that overlap on the GPU
+ *    (other streams, other host threads on the same device) race on the
+ *    array: order them on one stream.
  */
 lsa_status_t lsa_attend_noalloc(const uint16_t *const *q, const uint16_t *const *k_cache,
                                 const uint16_t *const *v_cache, int32_t H_q, int32_t H_kv,

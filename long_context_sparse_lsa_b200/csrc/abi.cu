@@ -37,7 +37,6 @@ int64_t budget_len(const lsa_budget_t& b) { return (int64_t)b.sink + b.window + 
 
 std::mutex g_mu;
 std::map<int, int> g_sms;
-std::map<std::tuple<int, int, int, int, int64_t, int, int, int, int, int>, lsa::IndexPlan> g_index_plans;
 
 int current_device() {
     int dev = -1;
@@ -121,13 +120,8 @@ size_t lsa_index_workspace_size(const lsa_batch_t* batch, int32_t H_I, int32_t d
     (void)H_I;
     (void)d_I;
     if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1 || !budget_ok(budget)) return 0;
-    size_t best = 0;
-    for (int C : {1, 2, 4, 8, 16}) {
-        lsa::IndexPlan p = lsa::plan_index(C, batch->n_q, batch->max_len, budget);
-        size_t need = (p.ws_coarse + 255) / 256 * 256 + (p.ws_fine + 255) / 256 * 256;
-        if (need > best) best = need;
-    }
-    return best;
+    if (budget.hi_block == 0) budget.hi_topblocks = 0;
+    return lsa::plan_index(batch->n_q, batch->max_len, budget).ws_bytes;
 }
 
 static lsa_status_t index_validate(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max,
@@ -162,28 +156,10 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     if (batch->n_q == 0) return LSA_OK;
     if (budget.hi_block == 0) budget.hi_topblocks = 0;
 
-    const int dev = current_device();
-    lsa::IndexPlan plan;
-    {
-        const auto key = std::make_tuple(dev, d_I, (H_I + 7) / 8, batch->n_q, (int64_t)batch->max_len, budget.sink,
-                                         budget.window, budget.topk, budget.hi_block, budget.hi_topblocks);
-        std::unique_lock<std::mutex> lk(g_mu);
-        auto it = g_index_plans.find(key);
-        if (it != g_index_plans.end()) {
-            plan = it->second;
-        } else {
-            lk.unlock();
-            cudaError_t e = lsa::choose_index_cluster(d_I, H_I, batch->n_q, batch->max_len, budget, &plan);
-            if (e != cudaSuccess) return cuda_fail(e);
-            lk.lock();
-            g_index_plans[key] = plan;
-        }
-    }
-    const size_t need_c = (plan.ws_coarse + 255) / 256 * 256;
-    const size_t need = need_c + (plan.ws_fine + 255) / 256 * 256;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
+    const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget);
+    if (plan.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < plan.ws_bytes || !aligned(workspace, 256)))
         return LSA_ERR_WORKSPACE;
-    if ((int64_t)batch->n_q * plan.cluster > 0x7fffffffLL) return LSA_ERR_UNSUPPORTED;
+    if (batch->n_q > 65535) return LSA_ERR_UNSUPPORTED;
 
     lsa::IndexArgs a;
     std::memset(&a, 0, sizeof a);
@@ -211,17 +187,23 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     a.hi_block = budget.hi_block;
     a.hi_topblocks = budget.hi_topblocks;
     a.budget = (int32_t)budget_len(budget);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.coarse_keys = reinterpret_cast<uint64_t*>(ws + plan.off_coarse);
+    a.kept = reinterpret_cast<int32_t*>(ws + plan.off_kept);
+    a.n_kept = reinterpret_cast<int32_t*>(ws + plan.off_nkept);
+    a.fine_keys = reinterpret_cast<uint32_t*>(ws + plan.off_fine);
     a.coarse_cap = plan.coarse_cap;
     a.fine_cap = plan.fine_cap;
-    a.kept_cap = plan.kept_cap;
-    a.smem_coarse = plan.smem_coarse;
-    a.smem_fine = plan.smem_fine;
-    a.smem_kept = plan.smem_kept;
-    a.smem_kept_local = plan.smem_kept_local;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    a.g_coarse = plan.ws_coarse ? reinterpret_cast<uint64_t*>(ws) : nullptr;
-    a.g_fine = plan.ws_fine ? reinterpret_cast<uint32_t*>(ws + need_c) : nullptr;
-    cudaError_t e = lsa::launch_index(a, plan, d_I, reinterpret_cast<cudaStream_t>(stream));
+    a.coarse_in_smem = plan.coarse_in_smem ? 1 : 0;
+    a.fine_in_smem = plan.fine_in_smem ? 1 : 0;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (budget.hi_block > 0) {
+        e = lsa::launch_index_scores(a, d_I, true, cs);
+        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, plan.smem_blocks, cs);
+    }
+    if (e == cudaSuccess) e = lsa::launch_index_scores(a, d_I, false, cs);
+    if (e == cudaSuccess) e = lsa::launch_index_select(a, false, plan.smem_tokens, cs);
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 
@@ -283,13 +265,9 @@ lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache
     a.dev_status = dev_status;
     const size_t rows_q = (size_t)layers_per_index * batch->n_q;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    a.counters = reinterpret_cast<uint32_t*>(ws);
-    size_t off = (rows_q * 4 + 255) / 256 * 256;
-    const size_t n_parts = (size_t)p.n_splits * p.wph;
-    if (n_parts > 1) {
-        a.part_o = reinterpret_cast<float*>(ws + off);
-        off += rows_q * n_parts * H_q * 128 * 4;
-        off = (off + 255) / 256 * 256;
+    if (p.n_splits > 1) {
+        a.part_o = reinterpret_cast<float*>(ws);
+        const size_t off = (rows_q * p.n_splits * H_q * 128 * 4 + 255) / 256 * 256;
         a.part_ml = reinterpret_cast<float*>(ws + off);
     }
     a.total_tokens = batch->total_tokens;
@@ -302,10 +280,14 @@ lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache
     a.G = layers_per_index;
     a.n_splits = p.n_splits;
     a.entries_per_split = p.entries_per_split;
-    a.wph = p.wph;
     a.head_groups = p.head_groups;
+    a.hpc = p.hpc;
+    a.n_stages = p.n_stages;
+    a.row_stride = p.row_stride;
+    a.bar_off = p.bar_off;
+    a.stage_off = p.stage_off;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
-    cudaError_t e = lsa::launch_attend(a, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = lsa::launch_attend(a, p.smem_bytes, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 

@@ -7,60 +7,95 @@
 // consecutive layers reuse one index set (same section, CLI bullet).
 //
 // Design (B200):
-//  * grid = (splits x head groups, query rows, layers). A CTA has 4 warps;
-//    each warp owns one (kv head, sub-range of entries) and gathers its
-//    selected 256-byte K and V rows with 16-byte cp.async into a 4-stage
-//    shared-memory ring (XOR-swizzled so ldmatrix is conflict-free). Masked
-//    entries are zero-filled without touching memory.
-//  * S^T = K Q^T on bf16 tensor cores (mma.m16n8k16): the 16 gathered tokens
-//    are the M dimension and the GQA group's query heads (8 per tile) the N
-//    dimension, so no MMA row is wasted on padding.
-//  * Online softmax in fp32 with exp2f and a log2(e)/sqrt(d) scale.
-//  * O^T = V^T P^T: P^T is moved from the accumulator layout into the B
-//    operand with movmatrix.trans; P is split into a bf16 high part and a
-//    bf16 remainder (two MMAs) so it keeps ~16 significant bits, and V^T comes
-//    from ldmatrix.trans.
-//  * Each warp writes an unnormalised partial (m, l, o). The last CTA to
-//    finish a (layer, query) — found with an atomic ticket, never a wait —
-//    merges the partials with the log-sum-exp rule and resets the ticket.
+//  * grid = (splits x kv-head groups, query rows, layers); one CTA per SM.
+//    A CTA covers up to 4 kv heads, whose rows of one token are contiguous
+//    (4 x 256 B), over one contiguous range of index-set entries whose
+//    indices are staged in shared memory first.
+//  * The gather uses two independent load paths so that neither caps the
+//    bandwidth: K rows come through the TMA engine (one cp.async.bulk of
+//    hpc*256 bytes per selected token into a ring of 16-token stages, padded
+//    by 16 bytes per row so ldmatrix reads of 8 tokens hit 8 bank groups,
+//    completing on an mbarrier); V rows are loaded by the consumer warps
+//    themselves with 16-byte vector loads straight into registers, two tiles
+//    ahead of their use.
+//  * Eight consumer warps: each owns one kv head and every (8/hpc)-th stage.
+//    S^T = K Q^T on bf16 tensor cores (mma.m16n8k16): the 16 tokens are M and
+//    the GQA group's query heads (8 per tile) are N. Online softmax in fp32
+//    (exp2f, log2(e)/sqrt(d) scale). O^T = V^T P^T: P^T is moved into the B
+//    operand with movmatrix.trans and split into a bf16 high part plus a bf16
+//    remainder (two MMAs, ~16 significant bits). For V^T the output dims are
+//    permuted so that lane (g, t) needs 16-byte chunks g and 8+g of tokens
+//    2t, 2t+1, 2t+8, 2t+9; byte permutes assemble the A fragments.
+//  * The consumers of one kv head merge in registers (log-sum-exp rule; the
+//    partner warps park their fragments in shared memory); each CTA writes
+//    its output directly when there is one split, else one partial per query
+//    head, which a small merge kernel (one warp per query head, every partial
+//    loaded at once) combines.
+//  * Every mbarrier wait is bounded by a time limit; on expiry the kernel
+//    flags LSA_DEV_TIMEOUT, waits (bounded) for the copies it issued and
+//    returns.
 #include "common.cuh"
 #include "internal.h"
 
 namespace lsa {
 namespace {
 
-constexpr int kAtThreads = 128;
-constexpr int kAtWarps = 4;
-constexpr int kTile = 16;       // tokens per pipeline stage
-constexpr int kStages = 4;
-constexpr int kRowBytes = 256;  // one (token, kv head) row at d = 128
+constexpr int kConsumers = 8;
+constexpr int kAtThreads = (kConsumers + 1) * kWarp;  // + one producer warp
+constexpr int kTile = 16;                              // tokens per stage
 constexpr int kD = 128;
-constexpr int kStageBytes = 2 * kTile * kRowBytes;  // K and V
-constexpr int kWarpSmem = kStages * kStageBytes;
-constexpr int kAtSmem = kAtWarps * kWarpSmem;
+constexpr int kHeadBytes = kD * 2;                     // one (token, kv head) row
+constexpr int kMaxEntriesPerSplit = 4096;
+constexpr int kMaxStages = 8;
+constexpr size_t kAtSmemBudget = 200 * 1024;
 
-// Byte offset of 16-byte chunk c of row r inside a [16 rows][256 B] tile.
-__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * kRowBytes + ((c ^ (r & 7)) << 4)); }
+// V rows of one 16-token tile for one kv head, in the registers of lane
+// (g, t): tokens 2t, 2t+1, 2t+8, 2t+9 (index j = 0..3), 16-byte chunks g and
+// 8+g (index c = 0..1).
+struct VTile {
+    uint4 r[4][2];
+};
+
+__device__ __forceinline__ void load_vtile(VTile& v, const uint16_t* vbase, int64_t tok_stride, const int32_t* ent,
+                                           int g, int t4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int row = 2 * t4 + (j & 1) + 8 * (j >> 1);
+        const int e = ent[row];
+        if (e >= 0) {
+            const uint16_t* p = vbase + (int64_t)e * tok_stride;
+            v.r[j][0] = ldg16(p + 8 * g);
+            v.r[j][1] = ldg16(p + 64 + 8 * g);
+        } else {
+            v.r[j][0] = make_uint4(0, 0, 0, 0);
+            v.r[j][1] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& x, int j) {
+    return j == 0 ? x.x : (j == 1 ? x.y : (j == 2 ? x.z : x.w));
+}
 
 template <int NT>
-__global__ void __launch_bounds__(kAtThreads) attend_kernel(const __grid_constant__ AttendArgs a) {
+__global__ void __launch_bounds__(kAtThreads, 1) attend_kernel(const __grid_constant__ AttendArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint32_t s_last;
+    __shared__ uint32_t s_fail;
 
-    const int lane = lane_id(), wid = warp_id();
+    const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
     const int g = lane >> 2, t4 = lane & 3;
     const int split = blockIdx.x / a.head_groups;
     const int hgrp = blockIdx.x % a.head_groups;
     const int r = blockIdx.y;
     const int layer = blockIdx.z;
     const int ratio = a.H_q / a.H_kv;
-    const int heads_per_cta = kAtWarps / a.wph;
-    const int kvh = hgrp * heads_per_cta + wid / a.wph;
-    const int sub = wid % a.wph;
-    const int n_parts = a.n_splits * a.wph;
-    const int part = split * a.wph + sub;
+    const int hpc = a.hpc;
+    const int NS = a.n_stages;
+    const int row_stride = a.row_stride;
+    const int stage_bytes = kTile * row_stride;
+    const int q_heads_cta = hpc * ratio;
 
-    // ---- query row validation ----
+    // ---- query row validation (uniform over the CTA) ----
     const int seq = a.q_seq[r];
     const int L = a.q_len[r];
     bool bad = seq < 0 || seq >= a.n_seq;
@@ -70,291 +105,349 @@ __global__ void __launch_bounds__(kAtThreads) attend_kernel(const __grid_constan
         const int slen = a.seq_lens[seq];
         bad = L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens;
     }
-    if (bad && threadIdx.x == 0 && blockIdx.x == 0 && layer == 0)
-        flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
-    const bool warp_live = !bad && kvh < a.H_kv;
-
-    // entries of this warp
-    const int n_entries = bad ? 0 : min(L, a.budget);
-    const int per_sub = a.entries_per_split / a.wph;
-    const int e_begin = split * a.entries_per_split + sub * per_sub;
-    const int e_end = warp_live ? min(n_entries, e_begin + per_sub) : e_begin;
-    const int32_t* set = a.sets + (int64_t)r * a.budget;
-
-    const uint16_t* kbase = a.k[layer] + (off * a.H_kv + kvh) * kD;
-    const uint16_t* vbase = a.v[layer] + (off * a.H_kv + kvh) * kD;
-    const int64_t tok_stride = (int64_t)a.H_kv * kD;  // elements between consecutive tokens
-
-    uint8_t* wsm = smem + wid * kWarpSmem;
-    const uint32_t wsm_u32 = smem_u32(wsm);
-
-    // ---- query fragments (B operand of S^T = K Q^T) ----
-    uint32_t qb[NT][kD / 16][2];
-    {
-        const uint16_t* qrow = a.q[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int hh = 8 * n + g;
-            const bool ok = warp_live && hh < ratio;
-#pragma unroll
-            for (int ks = 0; ks < kD / 16; ++ks) {
-                uint32_t b0 = 0, b1 = 0;
-                if (ok) {
-                    b0 = __ldg(reinterpret_cast<const uint32_t*>(qrow + hh * kD + 16 * ks + 2 * t4));
-                    b1 = __ldg(reinterpret_cast<const uint32_t*>(qrow + hh * kD + 16 * ks + 8 + 2 * t4));
-                }
-                qb[n][ks][0] = b0;
-                qb[n][ks][1] = b1;
-            }
-        }
-    }
-
-    // ---- gather pipeline ----
-    // Entry of tile i, row j (j = lane for lanes < 16): token position or -1.
-    auto fetch_entry = [&](int e) -> int {
-        if (e >= e_end) return -1;
-        const int idx = set[e];
-        if (idx < -1 || idx >= L) {
-            flag(a.dev_status, LSA_DEV_BAD_INDEX);
-            return -1;
-        }
-        return idx;
-    };
-    const int n_tiles = e_end > e_begin ? (e_end - e_begin + kTile - 1) / kTile : 0;
-    auto issue = [&](int tile, int stage) {
-        // lane < 16 holds the token of row `lane`
-        const int my_tok = lane < kTile ? fetch_entry(e_begin + tile * kTile + lane) : -1;
-        const uint32_t kst = wsm_u32 + stage * kStageBytes;
-        const uint32_t vst = kst + kTile * kRowBytes;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int c = lane + 32 * j;  // chunk id in [0, 256): row = c / 16, chunk-in-row = c % 16
-            const int row = c >> 4, cir = c & 15;
-            const int tok = __shfl_sync(0xffffffffu, my_tok, row);
-            const bool ok = tok >= 0;
-            const int64_t eo = ok ? (int64_t)tok * tok_stride + cir * 8 : 0;
-            cp_async16(kst + swz(row, cir), kbase + eo, ok ? 16u : 0u);
-            cp_async16(vst + swz(row, cir), vbase + eo, ok ? 16u : 0u);
-        }
-        return (uint64_t)__ballot_sync(0xffffffffu, lane < kTile && my_tok >= 0);  // valid rows
-    };
-
-    float o[NT][kD / 16][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int mt = 0; mt < kD / 16; ++mt) o[n][mt][0] = o[n][mt][1] = o[n][mt][2] = o[n][mt][3] = 0.f;
-    float m_run[NT][2], l_run[NT][2];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        m_run[n][0] = m_run[n][1] = -INFINITY;
-        l_run[n][0] = l_run[n][1] = 0.f;
-    }
-
-    // bits [16 s, 16 s + 16) of vmask: valid rows of pipeline stage s
-    uint64_t vmask = 0;
-#pragma unroll
-    for (int st = 0; st < kStages - 1; ++st) {
-        if (st < n_tiles) vmask |= issue(st, st) << (16 * st);
-        cp_async_commit();
-    }
-
-    for (int tile = 0; tile < n_tiles; ++tile) {
-        const int stage = tile % kStages;
-        {
-            const int nt = tile + kStages - 1;
-            if (nt < n_tiles) {
-                const int ns = nt % kStages;
-                const uint64_t m = issue(nt, ns);
-                vmask = (vmask & ~(0xFFFFull << (16 * ns))) | (m << (16 * ns));
-            }
-            cp_async_commit();
-        }
-        cp_async_wait<kStages - 1>();
-        __syncwarp();
-        const uint32_t kst = wsm_u32 + stage * kStageBytes;
-        const uint32_t vst = kst + kTile * kRowBytes;
-        const uint32_t rows_ok = (uint32_t)(vmask >> (16 * stage)) & 0xFFFFu;
-        const bool ok_g = (rows_ok >> g) & 1u;
-        const bool ok_g8 = (rows_ok >> (g + 8)) & 1u;
-
-        // S^T tile: 16 tokens x (8 * NT) heads
-        float sacc[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            const int mi = lane >> 3, rr = lane & 7;
-            const int row = rr + 8 * (mi & 1);
-            const int chunk = 2 * ks + (mi >> 1);
-            uint32_t afr[4];
-            ldmatrix_x4(afr, kst + swz(row, chunk));
-#pragma unroll
-            for (int n = 0; n < NT; ++n) mma_bf16(sacc[n], afr, qb[n][ks][0], qb[n][ks][1]);
-        }
-        // online softmax (log2 domain)
-        uint32_t phi[NT][2], plo[NT][2];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            float z0 = ok_g ? sacc[n][0] * a.scale_log2 : -INFINITY;   // (tok g,   head 2t)
-            float z1 = ok_g ? sacc[n][1] * a.scale_log2 : -INFINITY;   // (tok g,   head 2t+1)
-            float z2 = ok_g8 ? sacc[n][2] * a.scale_log2 : -INFINITY;  // (tok g+8, head 2t)
-            float z3 = ok_g8 ? sacc[n][3] * a.scale_log2 : -INFINITY;  // (tok g+8, head 2t+1)
-            float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
-#pragma unroll
-            for (int msk = 4; msk < 32; msk <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
-            }
-            const float mn0 = fmaxf(m_run[n][0], mx0), mn1 = fmaxf(m_run[n][1], mx1);
-            const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-            const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float al0 = exp2f(m_run[n][0] - base0), al1 = exp2f(m_run[n][1] - base1);
-            const float p0 = exp2f(z0 - base0), p1 = exp2f(z1 - base1);
-            const float p2 = exp2f(z2 - base0), p3 = exp2f(z3 - base1);
-            m_run[n][0] = mn0;
-            m_run[n][1] = mn1;
-            l_run[n][0] = l_run[n][0] * al0 + p0 + p2;
-            l_run[n][1] = l_run[n][1] * al1 + p1 + p3;
-#pragma unroll
-            for (int mt = 0; mt < kD / 16; ++mt) {
-                o[n][mt][0] *= al0;
-                o[n][mt][1] *= al1;
-                o[n][mt][2] *= al0;
-                o[n][mt][3] *= al1;
-            }
-            // P split into bf16 high part + bf16 remainder; transpose into B fragments.
-            const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
-            const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
-            const float2 fh01 = __bfloat1622float2(h01), fh23 = __bfloat1622float2(h23);
-            const uint32_t l01 = pack_bf16(p0 - fh01.x, p1 - fh01.y);
-            const uint32_t l23 = pack_bf16(p2 - fh23.x, p3 - fh23.y);
-            phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
-            phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-            plo[n][0] = movmatrix_trans(l01);
-            plo[n][1] = movmatrix_trans(l23);
-        }
-        // O^T += V^T P^T
-#pragma unroll
-        for (int mt = 0; mt < kD / 16; ++mt) {
-            const int mi = lane >> 3, rr = lane & 7;
-            const int row = rr + 8 * (mi >> 1);
-            const int chunk = 2 * mt + (mi & 1);
-            uint32_t vfr[4];
-            ldmatrix_x4_trans(vfr, vst + swz(row, chunk));
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                mma_bf16(o[n][mt], vfr, phi[n][0], phi[n][1]);
-                mma_bf16(o[n][mt], vfr, plo[n][0], plo[n][1]);
-            }
-        }
-        __syncwarp();  // the stage is refilled on the next iteration
-    }
-    cp_async_wait<0>();
-
-    // ---- finish this warp's partial ----
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int msk = 4; msk < 32; msk <<= 1) l_run[n][j] += __shfl_xor_sync(0xffffffffu, l_run[n][j], msk);
-
-    const int64_t row_q = (int64_t)layer * a.n_q + r;
-    if (warp_live) {
-        if (n_parts == 1) {
-            float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int h0 = 8 * n + 2 * t4, h1 = h0 + 1;
-                const float i0 = l_run[n][0] > 0.f ? 1.f / l_run[n][0] : 0.f;
-                const float i1 = l_run[n][1] > 0.f ? 1.f / l_run[n][1] : 0.f;
-#pragma unroll
-                for (int mt = 0; mt < kD / 16; ++mt) {
-                    const int d0 = 16 * mt + g, d1 = d0 + 8;
-                    if (h0 < ratio) {
-                        orow[h0 * kD + d0] = o[n][mt][0] * i0;
-                        orow[h0 * kD + d1] = o[n][mt][2] * i0;
-                    }
-                    if (h1 < ratio) {
-                        orow[h1 * kD + d0] = o[n][mt][1] * i1;
-                        orow[h1 * kD + d1] = o[n][mt][3] * i1;
-                    }
-                }
-            }
-        } else {
-            const int64_t pbase = (row_q * n_parts + part) * a.H_q + (int64_t)kvh * ratio;
-            float* po = a.part_o + pbase * kD;
-            float* pml = a.part_ml + pbase * 2;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int h0 = 8 * n + 2 * t4, h1 = h0 + 1;
-#pragma unroll
-                for (int mt = 0; mt < kD / 16; ++mt) {
-                    const int d0 = 16 * mt + g, d1 = d0 + 8;
-                    if (h0 < ratio) {
-                        po[h0 * kD + d0] = o[n][mt][0];
-                        po[h0 * kD + d1] = o[n][mt][2];
-                    }
-                    if (h1 < ratio) {
-                        po[h1 * kD + d0] = o[n][mt][1];
-                        po[h1 * kD + d1] = o[n][mt][3];
-                    }
-                }
-                if (g == 0) {
-                    if (h0 < ratio) {
-                        pml[h0 * 2] = m_run[n][0];
-                        pml[h0 * 2 + 1] = l_run[n][0];
-                    }
-                    if (h1 < ratio) {
-                        pml[h1 * 2] = m_run[n][1];
-                        pml[h1 * 2 + 1] = l_run[n][1];
-                    }
-                }
-            }
-        }
-    }
-    if (n_parts == 1 || bad) {
-        if (bad) {
-            // zero this CTA's heads so the output is defined
-            for (int i = threadIdx.x; i < heads_per_cta * ratio * kD; i += kAtThreads) {
-                const int hh = hgrp * heads_per_cta * ratio + i / kD;
-                if (hh < a.H_q && split == 0) a.out[layer][((int64_t)r * a.H_q + hh) * kD + i % kD] = 0.f;
-            }
+    if (bad) {
+        if (tid == 0 && blockIdx.x == 0 && layer == 0)
+            flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
+        if (split == 0) {
+            float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)hgrp * q_heads_cta) * kD;
+            for (int i = tid; i < q_heads_cta * kD; i += kAtThreads) orow[i] = 0.f;
         }
         return;
     }
 
-    // ---- last-arriving CTA of this (layer, row) merges ----
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t total = (uint32_t)(a.n_splits * a.head_groups);
-        const uint32_t prev = atomicAdd(&a.counters[row_q], 1u);
-        s_last = (prev == total - 1) ? 1u : 0u;
+    const int n_entries = min(L, a.budget);
+    const int e0 = split * a.entries_per_split;
+    const int n_local = max(0, min(n_entries - e0, a.entries_per_split));
+    const int n_tiles = (n_local + kTile - 1) / kTile;
+    const int32_t* set = a.sets + (int64_t)r * a.budget + e0;
+
+    int32_t* s_ent = reinterpret_cast<int32_t*>(smem);
+    const uint32_t bar_base = smem_u32(smem + a.bar_off);
+    const uint32_t st_base = smem_u32(smem + a.stage_off);
+    auto full_bar = [&](int s) { return bar_base + 8u * (uint32_t)s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (uint32_t)(NS + s); };
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), (uint32_t)hpc);
+        }
+        mbar_fence_init();
+        s_fail = 0;
     }
     __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    float* orow = a.out[layer] + (int64_t)r * a.H_q * kD;
-    const float* po = a.part_o + row_q * n_parts * a.H_q * kD;
-    const float* pml = a.part_ml + row_q * n_parts * a.H_q * 2;
-    for (int hd = threadIdx.x; hd < a.H_q * kD; hd += kAtThreads) {
-        const int h = hd / kD;
-        float M = -INFINITY;
-        for (int p = 0; p < n_parts; ++p) M = fmaxf(M, __ldcg(pml + ((int64_t)p * a.H_q + h) * 2));
-        float acc = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-            for (int p = 0; p < n_parts; ++p) {
-                const float mp = __ldcg(pml + ((int64_t)p * a.H_q + h) * 2);
-                const float wgt = exp2f(mp - M);
-                den += wgt * __ldcg(pml + ((int64_t)p * a.H_q + h) * 2 + 1);
-                acc += wgt * __ldcg(po + ((int64_t)p * a.H_q) * kD + hd);
+    // Entry i of this split, validated (invalid entries read as -1).
+    auto entry = [&](int i) -> int {
+        if (i >= n_local) return -1;
+        const int v = set[i];
+        if (v < -1 || v >= L) {
+            flag(a.dev_status, LSA_DEV_BAD_INDEX);
+            return -1;
+        }
+        return v;
+    };
+    if (warp < kConsumers) {
+        // the consumers stage the split's entries; the producer reads its own
+        // straight from global memory so its first copies start at once
+        for (int i = tid; i < n_tiles * kTile; i += kConsumers * kWarp) s_ent[i] = entry(i);
+        asm volatile("bar.sync 1, %0;" ::"r"(kConsumers * kWarp) : "memory");
+    }
+
+    // per-consumer state
+    float o[NT][kD / 16][4];
+    float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+        for (int mt = 0; mt < kD / 16; ++mt) o[n][mt][0] = o[n][mt][1] = o[n][mt][2] = o[n][mt][3] = 0.f;
+        m_run[n][0] = m_run[n][1] = -INFINITY;
+        l_run[n][0] = l_run[n][1] = 0.f;
+    }
+    int issued = 0;  // producer: tiles whose copies were issued
+    const int64_t tok_stride = (int64_t)a.H_kv * kD;  // elements between tokens
+
+    if (warp == kConsumers) {
+        // ------------------------------ producer (K) --------------------------
+        const uint16_t* kb = a.k[layer] + (off * a.H_kv + (int64_t)hgrp * hpc) * kD;
+        const uint32_t bytes = (uint32_t)(hpc * kHeadBytes);
+        for (int i = 0; i < n_tiles; ++i) {
+            const int s = i % NS;
+            const int u = i / NS;
+            if (u > 0 && !mbar_wait_bounded(empty_bar(s), (uint32_t)((u - 1) & 1), kWaitLimitNs)) {
+                if (lane == 0) s_fail = 1;
+                break;
+            }
+            const int ent = lane < kTile ? entry(i * kTile + lane) : -1;
+            const bool valid = ent >= 0;
+            const uint32_t nv = __popc(__ballot_sync(0xffffffffu, valid));
+            if (lane == 0) mbar_arrive_expect_tx(full_bar(s), nv * bytes);
+            __syncwarp();
+            if (valid)
+                bulk_g2s(st_base + (uint32_t)(s * stage_bytes + lane * row_stride), kb + (int64_t)ent * tok_stride,
+                         bytes, full_bar(s));
+            issued = i + 1;
+        }
+    } else {
+        // ------------------------------ consumers -----------------------------
+        const int h_local = warp % hpc;
+        const int wsel = warp / hpc;
+        const int n_sel = kConsumers / hpc;
+        const int kvh = hgrp * hpc + h_local;
+        const uint16_t* vbase = a.v[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
+        uint32_t qb[NT][kD / 16][2];
+        {
+            const uint16_t* qrow = a.q[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int hh = 8 * n + g;
+                const bool ok = hh < ratio;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    qb[n][ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + hh * kD + 16 * ks + 2 * t4)) : 0u;
+                    qb[n][ks][1] =
+                        ok ? __ldg(reinterpret_cast<const uint32_t*>(qrow + hh * kD + 16 * ks + 8 + 2 * t4)) : 0u;
+                }
             }
         }
-        orow[hd] = den > 0.f ? acc / den : 0.f;
+        const uint32_t head_off = (uint32_t)(h_local * kHeadBytes);
+        // V of this warp's next two tiles stays in flight (double buffer;
+        // the loop is unrolled by two so each buffer is a fixed register set)
+        VTile va, vbuf;
+        if (wsel < n_tiles) load_vtile(va, vbase, tok_stride, s_ent + wsel * kTile, g, t4);
+        if (wsel + n_sel < n_tiles) load_vtile(vbuf, vbase, tok_stride, s_ent + (wsel + n_sel) * kTile, g, t4);
+        auto tile = [&](int i, VTile& v) -> bool {
+            const int s = i % NS;
+            const int u = i / NS;
+            if (!mbar_wait_bounded(full_bar(s), (uint32_t)(u & 1), kWaitLimitNs)) {
+                if (lane == 0) s_fail = 1;
+                return false;
+            }
+            const uint32_t kst = st_base + (uint32_t)(s * stage_bytes) + head_off;
+            const int ent_lane = lane < kTile ? s_ent[i * kTile + lane] : 0;
+            const uint32_t masked = __ballot_sync(0xffffffffu, lane < kTile && ent_lane < 0);
+            const bool ok_g = !((masked >> g) & 1u);
+            const bool ok_g8 = !((masked >> (g + 8)) & 1u);
+            // S^T tile: 16 tokens x (8 * NT) heads
+            float sacc[NT][4];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+            {
+                const int mi = lane >> 3, rr = lane & 7;
+                const uint32_t kaddr = kst + (uint32_t)((rr + 8 * (mi & 1)) * row_stride + (mi >> 1) * 16);
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    uint32_t afr[4];
+                    ldmatrix_x4(afr, kaddr + ks * 32);
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) mma_bf16(sacc[n], afr, qb[n][ks][0], qb[n][ks][1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(s));  // K of this stage is no longer read
+            uint32_t phi[NT][2], plo[NT][2];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const float z0 = ok_g ? sacc[n][0] * a.scale_log2 : -INFINITY;   // (tok g,   head 2t)
+                const float z1 = ok_g ? sacc[n][1] * a.scale_log2 : -INFINITY;   // (tok g,   head 2t+1)
+                const float z2 = ok_g8 ? sacc[n][2] * a.scale_log2 : -INFINITY;  // (tok g+8, head 2t)
+                const float z3 = ok_g8 ? sacc[n][3] * a.scale_log2 : -INFINITY;  // (tok g+8, head 2t+1)
+                float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+#pragma unroll
+                for (int msk = 4; msk < 32; msk <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+                }
+                const float mn0 = fmaxf(m_run[n][0], mx0), mn1 = fmaxf(m_run[n][1], mx1);
+                const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+                const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+                const float al0 = exp2f(m_run[n][0] - base0), al1 = exp2f(m_run[n][1] - base1);
+                const float p0 = exp2f(z0 - base0), p1 = exp2f(z1 - base1);
+                const float p2 = exp2f(z2 - base0), p3 = exp2f(z3 - base1);
+                // the running max rarely moves after the first tiles: rescale o
+                // only when it did for some head of this warp
+                const bool moved = __any_sync(0xffffffffu, mn0 != m_run[n][0] || mn1 != m_run[n][1]);
+                m_run[n][0] = mn0;
+                m_run[n][1] = mn1;
+                l_run[n][0] = l_run[n][0] * al0 + p0 + p2;
+                l_run[n][1] = l_run[n][1] * al1 + p1 + p3;
+                if (moved) {
+#pragma unroll
+                    for (int mt = 0; mt < kD / 16; ++mt) {
+                        o[n][mt][0] *= al0;
+                        o[n][mt][1] *= al1;
+                        o[n][mt][2] *= al0;
+                        o[n][mt][3] *= al1;
+                    }
+                }
+                const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
+                const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
+                const float2 fh01 = __bfloat1622float2(h01), fh23 = __bfloat1622float2(h23);
+                phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+                phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+                plo[n][0] = movmatrix_trans(pack_bf16(p0 - fh01.x, p1 - fh01.y));
+                plo[n][1] = movmatrix_trans(pack_bf16(p2 - fh23.x, p3 - fh23.y));
+            }
+            // O^T += V^T P^T from the registers of this tile's V
+#pragma unroll
+            for (int mt = 0; mt < kD / 16; ++mt) {
+                const int c = mt >> 2, j = mt & 3;
+                const uint32_t w0 = word(v.r[0][c], j), w1 = word(v.r[1][c], j);
+                const uint32_t w8 = word(v.r[2][c], j), w9 = word(v.r[3][c], j);
+                const uint32_t vfr[4] = {__byte_perm(w0, w1, 0x5410), __byte_perm(w0, w1, 0x7632),
+                                         __byte_perm(w8, w9, 0x5410), __byte_perm(w8, w9, 0x7632)};
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    mma_bf16(o[n][mt], vfr, phi[n][0], phi[n][1]);
+                    mma_bf16(o[n][mt], vfr, plo[n][0], plo[n][1]);
+                }
+            }
+            // V two tiles ahead, in flight during the next tile's K wait and math
+            if (i + 2 * n_sel < n_tiles) load_vtile(v, vbase, tok_stride, s_ent + (i + 2 * n_sel) * kTile, g, t4);
+                    return true;
+        };
+        for (int i = wsel; i < n_tiles; i += 2 * n_sel) {
+            if (!tile(i, va)) break;
+            if (i + n_sel < n_tiles && !tile(i + n_sel, vbuf)) break;
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int msk = 4; msk < 32; msk <<= 1)
+                    l_run[n][j] += __shfl_xor_sync(0xffffffffu, l_run[n][j], msk);
     }
-    if (threadIdx.x == 0) a.counters[row_q] = 0u;
+    __syncthreads();
+
+    if (s_fail) {
+        // wait (bounded) for every copy this CTA issued, then give up
+        if (warp == kConsumers) {
+            for (int i = max(0, issued - NS); i < issued; ++i)
+                mbar_wait_bounded(full_bar(i % NS), (uint32_t)((i / NS) & 1), kWaitLimitNs);
+        }
+        if (tid == 0) flag(a.dev_status, LSA_DEV_TIMEOUT);
+        return;
+    }
+
+    // ---- merge the consumers of each kv head, in registers ----
+    // All warps hold O^T in the same fragment layout, so warps with wsel > 0
+    // park theirs in shared memory (lane-major: conflict free) and the wsel ==
+    // 0 warp of the head folds them in with the log-sum-exp rule.
+    constexpr int kRegs = NT * (kD / 16) * 4;
+    float* xo = reinterpret_cast<float*>(smem + a.stage_off);  // [kConsumers][kRegs][32]
+    float* xml = xo + kConsumers * kRegs * kWarp;              // [kConsumers][NT*4][32]
+    const int wsel_me = warp / hpc;
+    if (warp < kConsumers && wsel_me > 0) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int mt = 0; mt < kD / 16; ++mt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) xo[(warp * kRegs + (n * (kD / 16) + mt) * 4 + c) * kWarp + lane] = o[n][mt][c];
+            xml[(warp * NT * 4 + n * 4 + 0) * kWarp + lane] = m_run[n][0];
+            xml[(warp * NT * 4 + n * 4 + 1) * kWarp + lane] = m_run[n][1];
+            xml[(warp * NT * 4 + n * 4 + 2) * kWarp + lane] = l_run[n][0];
+            xml[(warp * NT * 4 + n * 4 + 3) * kWarp + lane] = l_run[n][1];
+        }
+    }
+    __syncthreads();
+    const bool direct = a.n_splits == 1;
+    const int64_t row_q = (int64_t)layer * a.n_q + r;
+    if (warp < kConsumers && wsel_me == 0) {
+        const int h_local = warp % hpc;
+        const int n_sel = kConsumers / hpc;
+        for (int j = 1; j < n_sel; ++j) {
+            const int w = h_local + hpc * j;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const float mb = xml[(w * NT * 4 + n * 4 + c) * kWarp + lane];
+                    const float lb = xml[(w * NT * 4 + n * 4 + 2 + c) * kWarp + lane];
+                    const float M = fmaxf(m_run[n][c], mb);
+                    const float sa = M == -INFINITY ? 0.f : exp2f(m_run[n][c] - M);
+                    const float sb = M == -INFINITY ? 0.f : exp2f(mb - M);
+                    m_run[n][c] = M;
+                    l_run[n][c] = l_run[n][c] * sa + lb * sb;
+#pragma unroll
+                    for (int mt = 0; mt < kD / 16; ++mt) {
+                        o[n][mt][c] = o[n][mt][c] * sa + xo[(w * kRegs + (n * (kD / 16) + mt) * 4 + c) * kWarp + lane] * sb;
+                        o[n][mt][c + 2] =
+                            o[n][mt][c + 2] * sa + xo[(w * kRegs + (n * (kD / 16) + mt) * 4 + c + 2) * kWarp + lane] * sb;
+                    }
+                }
+            }
+        }
+        // write this kv head's query heads: the final output, or one split partial
+        const int kvh = hgrp * hpc + h_local;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int hh = 8 * n + 2 * t4 + c;
+                if (hh >= ratio) continue;
+                const int64_t qh = (int64_t)kvh * ratio + hh;
+                const float inv = l_run[n][c] > 0.f ? 1.f / l_run[n][c] : 0.f;
+                float* dst = direct ? a.out[layer] + ((int64_t)r * a.H_q + qh) * kD
+                                    : a.part_o + ((row_q * a.n_splits + split) * a.H_q + qh) * kD;
+                const float sc = direct ? inv : 1.f;
+#pragma unroll
+                for (int mt = 0; mt < kD / 16; ++mt) {
+                    const int d0 = 8 * ((mt >> 2) ? 8 + g : g) + 2 * (mt & 3);
+                    *reinterpret_cast<float2*>(dst + d0) = make_float2(o[n][mt][c] * sc, o[n][mt][c + 2] * sc);
+                }
+                if (!direct && g == 0)
+                    *reinterpret_cast<float2*>(a.part_ml + ((row_q * a.n_splits + split) * a.H_q + qh) * 2) =
+                        make_float2(m_run[n][c], l_run[n][c]);
+            }
+        }
+    }
+}
+
+// Split merge: one warp per (query head, row, layer); lane l owns dims
+// 4l..4l+3. All partials are combined with the log-sum-exp rule.
+__global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_constant__ AttendArgs a) {
+    const int h = blockIdx.x, r = blockIdx.y, layer = blockIdx.z, lane = threadIdx.x;
+    const int seq = a.q_seq[r];
+    const int L = a.q_len[r];
+    if (seq < 0 || seq >= a.n_seq) return;
+    const int64_t off = a.kv_offset[seq];
+    const int slen = a.seq_lens[seq];
+    if (L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens) return;  // zeroed already
+    const int64_t row_q = (int64_t)layer * a.n_q + r;
+    const float* P = a.part_o + (row_q * a.n_splits * a.H_q + h) * kD;
+    const float* PML = a.part_ml + (row_q * a.n_splits * a.H_q + h) * 2;
+    const int64_t pstride = (int64_t)a.H_q;  // between consecutive splits, in rows
+    constexpr int kU = 8;
+    float M = -INFINITY, den = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < a.n_splits; p0 += kU) {
+        float2 ml[kU];
+        float4 v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int p = p0 + u;
+            const bool ok = p < a.n_splits;
+            ml[u] = ok ? __ldcg(reinterpret_cast<const float2*>(PML + p * pstride * 2)) : make_float2(-INFINITY, 0.f);
+            v[u] = ok ? __ldcg(reinterpret_cast<const float4*>(P + p * pstride * kD) + lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (ml[u].x == -INFINITY) continue;
+            const float nm = fmaxf(M, ml[u].x);
+            const float so = exp2f(M - nm), sn = exp2f(ml[u].x - nm);
+            den = den * so + ml[u].y * sn;
+            acc.x = acc.x * so + v[u].x * sn;
+            acc.y = acc.y * so + v[u].y * sn;
+            acc.z = acc.z * so + v[u].z * sn;
+            acc.w = acc.w * so + v[u].w * sn;
+            M = nm;
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    reinterpret_cast<float4*>(a.out[layer] + ((int64_t)r * a.H_q + h) * kD)[lane] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }
 
 }  // namespace
@@ -362,46 +455,66 @@ __global__ void __launch_bounds__(kAtThreads) attend_kernel(const __grid_constan
 AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms) {
     AttendPlan p;
     (void)d;
-    p.wph = H_kv >= kAtWarps ? 1 : kAtWarps / H_kv;
-    p.head_groups = H_kv >= kAtWarps ? H_kv / kAtWarps : 1;
+    p.hpc = H_kv < 4 ? H_kv : 4;
+    p.head_groups = H_kv / p.hpc;
+    p.row_stride = p.hpc * kHeadBytes + 16;
     const int entries = budget < max_len ? budget : max_len;
     const long rows = (long)n_q * G * p.head_groups;
     int splits = rows > 0 ? (int)((num_sms + rows / 2) / rows) : 1;
     if (splits < 1) splits = 1;
-    const int gran = kTile * p.wph;
-    const int max_splits = (entries + 4 * gran - 1) / (4 * gran);  // >= 64 entries per warp
-    if (splits > max_splits) splits = max_splits < 1 ? 1 : max_splits;
+    const int min_splits = (entries + kMaxEntriesPerSplit - 1) / kMaxEntriesPerSplit;
+    const int max_splits = (entries + 63) / 64;  // at least 4 tiles per split
+    if (splits > max_splits) splits = max_splits;
+    if (splits < min_splits) splits = min_splits;
+    if (splits < 1) splits = 1;
     int eps = (entries + splits - 1) / splits;
-    eps = (eps + gran - 1) / gran * gran;
-    if (eps < gran) eps = gran;
+    eps = (eps + kTile - 1) / kTile * kTile;
+    if (eps < kTile) eps = kTile;
     splits = (entries + eps - 1) / eps;
     if (splits < 1) splits = 1;
     p.n_splits = splits;
     p.entries_per_split = eps;
-    const size_t n_parts = (size_t)splits * p.wph;
+    // shared memory: entries | barriers | K stages (the stages are reused for the merge)
+    const size_t ent = ((size_t)eps * 4 + 127) / 128 * 128;
+    const size_t stage = (size_t)kTile * p.row_stride;
+    int ns = (int)((kAtSmemBudget - ent - 2 * kMaxStages * 8 - 128) / stage);
+    if (ns > kMaxStages) ns = kMaxStages;
+    p.n_stages = ns;
+    p.bar_off = (int)ent;
+    p.stage_off = (int)(ent + ((2 * kMaxStages * 8 + 127) / 128) * 128);
+    const int NT = (H_q / H_kv + 7) / 8;
+    size_t merge = (size_t)kConsumers * (NT * (kD / 16) * 4 + NT * 4) * kWarp * 4;
+    size_t stages_bytes = (size_t)ns * stage;
+    p.smem_bytes = p.stage_off + (stages_bytes > merge ? stages_bytes : merge);
     const size_t rows_q = (size_t)G * n_q;
-    size_t ws = (rows_q * 4 + 255) / 256 * 256;  // counters first
-    if (n_parts > 1) {
-        ws += rows_q * n_parts * H_q * 128 * 4;
+    size_t ws = 256;
+    if (splits > 1) {
+        ws = rows_q * splits * H_q * kD * 4;
         ws = (ws + 255) / 256 * 256;
-        ws += rows_q * n_parts * H_q * 2 * 4;
+        ws += rows_q * splits * H_q * 2 * 4;
+        ws = (ws + 255) / 256 * 256;
     }
     p.ws_bytes = ws;
     return p;
 }
 
-cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
+cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream) {
     const int ratio = a.H_q / a.H_kv;
     dim3 grid((unsigned)(a.n_splits * a.head_groups), (unsigned)a.n_q, (unsigned)a.G);
     if (ratio <= 8) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAtSmem);
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_bytes);
         if (e != cudaSuccess) return e;
-        attend_kernel<1><<<grid, kAtThreads, kAtSmem, stream>>>(a);
+        attend_kernel<1><<<grid, kAtThreads, smem_bytes, stream>>>(a);
     } else {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAtSmem);
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_bytes);
         if (e != cudaSuccess) return e;
-        attend_kernel<2><<<grid, kAtThreads, kAtSmem, stream>>>(a);
+        attend_kernel<2><<<grid, kAtThreads, smem_bytes, stream>>>(a);
     }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || a.n_splits == 1) return e;
+    attend_merge_kernel<<<dim3((unsigned)a.H_q, (unsigned)a.n_q, (unsigned)a.G), kWarp, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -30,7 +30,7 @@ struct BlockSumArgs {
 };
 cudaError_t launch_block_sums(const BlockSumArgs& a, int d_I, cudaStream_t stream);
 
-// ---- fused decode indexer -------------------------------------------------
+// ---- indexer: scoring kernels + selection kernels -------------------------
 struct IndexArgs {
     const int8_t* q_idx;
     const int8_t* k_idx;
@@ -48,32 +48,25 @@ struct IndexArgs {
     int32_t n_seq, n_q, max_len;
     int32_t H_I, w_max;
     int32_t sink, window, topk, hi_block, hi_topblocks, budget;
-    // storage plan (see plan_index)
-    int32_t coarse_cap;   // coarse key slots per CTA
-    int32_t fine_cap;     // fine key slots per CTA
-    int32_t kept_cap;     // kept-block list entries (leader CTA)
-    int32_t smem_coarse;  // byte offset in dynamic smem, or -1 (global)
-    int32_t smem_fine;    // byte offset in dynamic smem, or -1 (global)
-    int32_t smem_kept;    // byte offset in dynamic smem
-    int32_t smem_kept_local;
-    uint64_t* g_coarse;   // [n_q * C * coarse_cap] when smem_coarse < 0
-    uint32_t* g_fine;     // [n_q * C * fine_cap] when smem_fine < 0
+    // workspace (see plan_index)
+    uint64_t* coarse_keys;  // [n_q][coarse_cap] HI block keys (score + 1)
+    int32_t* kept;          // [n_q][hi_topblocks] kept block ids, ascending
+    int32_t* n_kept;        // [n_q]
+    uint32_t* fine_keys;    // [n_q][fine_cap] token keys (score + 1, 0 = none)
+    int32_t coarse_cap, fine_cap;
+    int32_t coarse_in_smem, fine_in_smem;
 };
 
 struct IndexPlan {
-    int cluster = 1;
-    int coarse_cap = 0, fine_cap = 0, kept_cap = 0;
-    int smem_coarse = -1, smem_fine = -1, smem_kept = 0, smem_kept_local = 0;
-    size_t dyn_smem = 0;
-    size_t ws_coarse = 0, ws_fine = 0;  // global bytes
+    int coarse_cap = 0, fine_cap = 0;
+    bool coarse_in_smem = false, fine_in_smem = false;
+    size_t smem_blocks = 0, smem_tokens = 0;  // dynamic smem of the selection kernels
+    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0;
+    size_t ws_bytes = 0;
 };
-
-// Storage plan for a given cluster size (pure host arithmetic).
-IndexPlan plan_index(int cluster, int n_q, int max_len, const lsa_budget_t& b);
-// Chooses the cluster size for this device and batch.
-cudaError_t choose_index_cluster(int d_I, int H_I, int n_q, int max_len, const lsa_budget_t& b,
-                                 IndexPlan* out);
-cudaError_t launch_index(const IndexArgs& a, const IndexPlan& plan, int d_I, cudaStream_t stream);
+IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b);
+cudaError_t launch_index_scores(const IndexArgs& a, int d_I, bool coarse, cudaStream_t stream);
+cudaError_t launch_index_select(const IndexArgs& a, bool blocks, size_t smem, cudaStream_t stream);
 
 // ---- sparse attention -----------------------------------------------------
 struct AttendArgs {
@@ -87,22 +80,25 @@ struct AttendArgs {
     const int32_t* q_seq;
     const int32_t* q_len;
     int32_t* dev_status;
-    float* part_o;        // [G][n_q][n_parts][H_q][d]
-    float* part_ml;       // [G][n_q][n_parts][H_q][2]
-    uint32_t* counters;   // [G][n_q]
+    float* part_o;        // [G][n_q][n_splits][H_q][d]
+    float* part_ml;       // [G][n_q][n_splits][H_q][2]
     int64_t total_tokens;
     int32_t n_seq, n_q, max_len;
     int32_t H_q, H_kv, budget, G;
-    int32_t n_splits, entries_per_split, wph, head_groups;
+    int32_t n_splits, entries_per_split, head_groups;
+    int32_t hpc;          // kv heads per CTA
+    int32_t n_stages, row_stride, bar_off, stage_off;  // shared-memory plan
     float scale_log2;     // log2(e) / sqrt(d)
 };
 
 struct AttendPlan {
-    int n_splits = 1, entries_per_split = 16, wph = 1, head_groups = 1;
+    int n_splits = 1, entries_per_split = 16, head_groups = 1, hpc = 1;
+    int n_stages = 2, row_stride = 272, bar_off = 0, stage_off = 0;
+    size_t smem_bytes = 0;
     size_t ws_bytes = 0;
 };
 AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms);
-cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream);
+cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
 
 int device_sm_count();
 

@@ -1,8 +1,8 @@
 // noalloc.cu — lsa_attend_noalloc: sparse attention for callers that cannot
 // allocate device memory.
 //
-// lsa_attend needs a caller-provided workspace for its split partials and
-// arrival counters. Some callers cannot call cudaMalloc on this path: an
+// lsa_attend needs a caller-provided workspace for its split partials. Some
+// callers cannot call cudaMalloc on this path: an
 // engine whose device memory is owned entirely by its own pool allocator
 // (a raw cudaMalloc would fail or fragment that pool), or a decode loop that
 // must never run an allocation (cudaMalloc/cudaFree may synchronise the
@@ -61,15 +61,8 @@ extern "C" lsa_status_t lsa_attend_noalloc(const uint16_t* const* q, const uint1
     void* scratch = nullptr;
     const lsa_status_t st = scratch_on_current_device(&scratch);
     if (st != LSA_OK) return st;
-    if (need > 0 && batch->n_q > 0) {
-        // The arrival counters (the first 4 * G * n_q bytes) must start at zero;
-        // the array keeps whatever the previous call left in it.
-        const size_t counters = (size_t)4 * (size_t)layers_per_index * (size_t)batch->n_q;
-        if (cudaMemsetAsync(scratch, 0, counters, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
-            cudaGetLastError();
-            return LSA_ERR_CUDA;
-        }
-    }
+    // The array keeps the previous call's contents; lsa_attend writes every
+    // partial before reading it, so nothing needs clearing.
     return lsa_attend(q, k_cache, v_cache, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, scratch,
                       (size_t)LSA_NOALLOC_SCRATCH_BYTES, dev_status, stream);
 }

@@ -53,18 +53,19 @@ def test_noalloc_matches_workspace_version_twice(wl):
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    # 2048 rows x 8 layers x 4 sub-splits of partials (one kv head) do not fit
-    n_q = 2048
+    # 8 rows x 8 layers with 16384-entry sets are split four ways; the split
+    # partials of 64 query heads need more than the static scratch holds
+    n_q, G, H_q, H_kv, budget = 8, 8, 64, 4, 16384
     dev = "cuda"
     batch = lsa.Batch(torch.zeros(1, dtype=torch.int64, device=dev), torch.full((1,), 100000, dtype=torch.int32,
                       device=dev), torch.zeros(n_q, dtype=torch.int32, device=dev),
                       torch.full((n_q,), 100000, dtype=torch.int32, device=dev), 100000, 100000)
-    need = lsa.lsa_attend_workspace_size(batch, 8, 1, 128, 4096, 8)
+    need = lsa.lsa_attend_workspace_size(batch, H_q, H_kv, 128, budget, G)
     assert need > (8 << 20)
-    q = [torch.zeros((n_q, 8, 128), dtype=torch.bfloat16, device=dev) for _ in range(8)]
-    kv = [torch.zeros((16, 1, 128), dtype=torch.bfloat16, device=dev) for _ in range(8)]
-    out = [torch.zeros((n_q, 8, 128), dtype=torch.float32, device=dev) for _ in range(8)]
-    sets = torch.full((n_q, 4096), -1, dtype=torch.int32, device=dev)
+    q = [torch.zeros((n_q, H_q, 128), dtype=torch.bfloat16, device=dev) for _ in range(G)]
+    kv = [torch.zeros((16, H_kv, 128), dtype=torch.bfloat16, device=dev) for _ in range(G)]
+    out = [torch.zeros((n_q, H_q, 128), dtype=torch.float32, device=dev) for _ in range(G)]
+    sets = torch.full((n_q, budget), -1, dtype=torch.int32, device=dev)  # nothing would be read
     with pytest.raises(lsa.LsaError) as e:
         lsa.lsa_attend_noalloc(q, kv, kv, sets, batch, out)
     assert e.value.status == 2  # LSA_ERR_UNSUPPORTED
