@@ -192,6 +192,7 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     a.kept = reinterpret_cast<int32_t*>(ws + plan.off_kept);
     a.n_kept = reinterpret_cast<int32_t*>(ws + plan.off_nkept);
     a.fine_keys = reinterpret_cast<uint32_t*>(ws + plan.off_fine);
+    a.hist = reinterpret_cast<uint32_t*>(ws + plan.off_hist);
     a.coarse_cap = plan.coarse_cap;
     a.fine_cap = plan.fine_cap;
     a.coarse_in_smem = plan.coarse_in_smem ? 1 : 0;
@@ -201,6 +202,9 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     if (budget.hi_block > 0) {
         e = lsa::launch_index_scores(a, d_I, true, cs);
         if (e == cudaSuccess) e = lsa::launch_index_select(a, true, plan.smem_blocks, cs);
+    } else {
+        // with HI the coarse scoring kernel clears the fine-key histograms
+        e = cudaMemsetAsync(a.hist, 0, (size_t)batch->n_q * lsa::kHistBins * sizeof(uint32_t), cs);
     }
     if (e == cudaSuccess) e = lsa::launch_index_scores(a, d_I, false, cs);
     if (e == cudaSuccess) e = lsa::launch_index_select(a, false, plan.smem_tokens, cs);

@@ -10,16 +10,18 @@
 // Attention 문제").
 //
 // Design (B200): one 1024-thread CTA per query row, so every synchronisation
-// is a CTA barrier. The row's keys (score + 1, 0 = not a candidate) are
-// staged in shared memory when they fit (the maximum and the candidate count
-// are taken during staging). An MSD radix select finds the exact k-th largest
-// key T and the number of keys equal to T to keep: its first 8-bit digit is
-// the top 8 bits below the row maximum's leading bit; the keys of the
-// threshold bin are then gathered into a short list on which one warp
-// resolves the remaining digits. Compaction is bitmap based: warp ballots
-// build "key > T" and "key == T" words, each thread counts its words, one CTA
-// prefix ranks them, and every thread emits its kept positions in order — a
-// fixed number of barriers whatever the row length.
+// is a CTA barrier. Selection starts from a histogram of the row's keys
+// (score + 1, 0 = not a candidate) on the logarithmic scale of key_bin: the
+// fine scoring kernel accumulates it in global memory while it writes the
+// keys; for HI blocks it is built here while the keys are staged. One suffix
+// scan of the histogram gives the bin holding the k-th largest key, one pass
+// over the keys (staging them in shared memory when they fit) gathers that
+// bin's keys into a short list, and 12-bit radix levels over the list give
+// the exact k-th largest key T and how many keys equal to T are kept (a bin
+// too full for the list is refined over all keys instead). Compaction is
+// bitmap based: warp ballots build "key > T" and "key == T" words, each
+// thread counts its word, one CTA prefix ranks them, and every thread emits
+// its kept positions in order.
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,27 +30,25 @@ namespace {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / kWarp;
-constexpr int kBins = 256;
-constexpr int kCandCap = 2048;        // keys of the threshold bin resolved by one warp
-constexpr int kWordsPerThread = 1;    // compaction: bitmap words per thread per chunk
-constexpr int kChunkWords = kSelThreads * kWordsPerThread;  // 1024 words = 32768 keys
-constexpr int kUnroll = 4;            // independent key loads in flight per thread
+static_assert(kHistBins == 4 * kSelThreads, "the scan gives each thread four bins");
+constexpr int kDigitBits = 12;            // refinement digit: 4096 bins
+constexpr int kCandCap = 2048;            // keys of the threshold bin held in a list
+constexpr int kChunkWords = kSelThreads;  // compaction: one bitmap word per thread per chunk
+constexpr int kUnroll = 4;                // independent loads in flight per thread
 
 struct SelShared {
-    uint32_t hist[kBins];
+    uint32_t hist[kHistBins];
     uint32_t wsum[kSelWarps];
     uint32_t wsum2[kSelWarps];
-    unsigned long long wmax[kSelWarps];
     uint32_t gt_words[kChunkWords];
     uint32_t eq_words[kChunkWords];
-    uint32_t digit, above, in_bin, count;
-    uint32_t carry_gt, carry_eq;
+    uint32_t bin, above, in_bin, count;
 };
 
-template <typename K>
-__device__ __forceinline__ int key_bits(K v) {
-    if constexpr (sizeof(K) == 8) return 64 - __clzll((long long)v);
-    else return 32 - __clz((int)v);
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
 // Keys of one row, either staged in shared memory or read from global memory.
@@ -70,248 +70,168 @@ struct Keys {
         }
         return __ldcg(g + i);
     }
+    // 16-byte vector i (keys 16/sizeof(K) * i onwards)
+    __device__ __forceinline__ uint4 vec(int i) const {
+        if (s != 0u) {
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(s + 16u * (uint32_t)i));
+            return v;
+        }
+        return __ldcg(reinterpret_cast<const uint4*>(g) + i);
+    }
 };
 
-// Block sum of two counters and maximum of a 64-bit value.
-__device__ void block_reduce(SelShared& sh, uint32_t& a, uint32_t& b, unsigned long long& m) {
-    const int lane = lane_id(), wid = warp_id();
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        a += __shfl_xor_sync(0xffffffffu, a, o);
-        b += __shfl_xor_sync(0xffffffffu, b, o);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    }
-    if (lane == 0) {
-        sh.wsum[wid] = a;
-        sh.wsum2[wid] = b;
-        sh.wmax[wid] = m;
-    }
-    __syncthreads();
-    a = 0;
-    b = 0;
-    m = 0;
-    for (int w = 0; w < kSelWarps; ++w) {
-        a += sh.wsum[w];
-        b += sh.wsum2[w];
-        m = max(m, sh.wmax[w]);
-    }
-    __syncthreads();
-}
-
-// Stages the row's keys in shared memory (when planned) and returns the
-// maximum key and the number of nonzero keys.
-template <typename K>
-__device__ Keys<K> stage_keys(SelShared& sh, const K* g, int n, uint8_t* dyn, bool in_smem, unsigned long long& kmax,
-                              uint32_t& nvalid) {
-    Keys<K> k{g, 0u};
-    unsigned long long m = 0;
-    uint32_t c = 0, unused = 0;
-    auto see = [&](K v) {
-        m = max(m, (unsigned long long)v);
-        c += v != 0 ? 1u : 0u;
-    };
-    constexpr int kPer16 = 16 / (int)sizeof(K);
-    const int n16 = n / kPer16;
-    K* st = reinterpret_cast<K*>(dyn);
-    for (int i = threadIdx.x; i < n16; i += kSelThreads) {
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(g) + i);
-        if (in_smem) reinterpret_cast<uint4*>(st)[i] = v;
-        const K* e = reinterpret_cast<const K*>(&v);
-#pragma unroll
-        for (int j = 0; j < kPer16; ++j) see(e[j]);
-    }
-    for (int i = n16 * kPer16 + threadIdx.x; i < n; i += kSelThreads) {
-        const K v = __ldcg(g + i);
-        if (in_smem) st[i] = v;
-        see(v);
-    }
-    block_reduce(sh, c, unused, m);
-    kmax = m;
-    nvalid = c;
-    if (in_smem) k.s = smem_u32(st);
-    return k;
-}
-
-// Block-level histogram pass: counts the `width`-bit digit at `shift` of the
-// keys whose bits above shift+width equal `prefix`, then finds the digit d*
-// where the running count from the top reaches krem.
-template <typename K>
-__device__ void hist_pass(SelShared& sh, const Keys<K>& keys, int n, int shift, int width, K prefix, uint32_t krem,
-                          uint32_t& digit, uint32_t& above, uint32_t& in_bin) {
-    constexpr int kKeyBits = 8 * sizeof(K);
+// Suffix scan of sh.hist. Returns the number of counted keys; when
+// 1 <= krem <= total also gives the bin d holding the krem-th largest key,
+// the count above it (bins > d) and the count in it.
+__device__ uint32_t find_bin(SelShared& sh, uint32_t krem, uint32_t& bin, uint32_t& above, uint32_t& in_bin) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
-    if (tid < kBins) sh.hist[tid] = 0;
-    __syncthreads();
-    for (int i0 = tid; i0 < n; i0 += kSelThreads * kUnroll) {
-        K kv[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = i0 + u * kSelThreads;
-            kv[u] = i < n ? keys[i] : K(0);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = i0 + u * kSelThreads;
-            const K key = kv[u];
-            const K hi = (shift + width >= kKeyBits) ? K(0) : (K)(key >> (shift + width));
-            if (i < n && hi == prefix) atomicAdd(&sh.hist[(uint32_t)(key >> shift) & ((1u << width) - 1u)], 1u);
-        }
-    }
-    __syncthreads();
-    uint32_t tot = 0, x = 0;
-    if (tid < kBins) {
-        tot = sh.hist[tid];
-        x = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_down_sync(0xffffffffu, x, o);
-            if (lane + o < 32) x += v;
-        }
-        if (lane == 0) sh.wsum[wid] = x;
-    }
-    __syncthreads();
-    if (tid < kBins) {
-        uint32_t later = 0;
-        for (int w2 = wid + 1; w2 < kBins / kWarp; ++w2) later += sh.wsum[w2];
-        const uint32_t S = x + later;  // count with digit >= tid
-        if (S >= krem && S - tot < krem) {
-            sh.digit = tid;
-            sh.above = S - tot;
-            sh.in_bin = tot;
-        }
-    }
-    __syncthreads();
-    digit = sh.digit;
-    above = sh.above;
-    in_bin = sh.in_bin;
-    __syncthreads();
-}
-
-// Warp-level histogram pass over a short list (warp 0 only; no CTA barrier).
-template <typename K>
-__device__ void warp_hist_pass(SelShared& sh, const K* cand, int m, int shift, int width, uint32_t krem,
-                               uint32_t& digit, uint32_t& above) {
-    const int lane = lane_id();
-#pragma unroll
-    for (int j = 0; j < kBins / kWarp; ++j) sh.hist[lane * (kBins / kWarp) + j] = 0;
-    __syncwarp();
-    for (int i = lane; i < m; i += kWarp) atomicAdd(&sh.hist[(uint32_t)(cand[i] >> shift) & ((1u << width) - 1u)], 1u);
-    __syncwarp();
-    // lane l owns bins [8l, 8l+8); suffix sums across lanes, then within the lane
-    uint32_t own = 0;
-#pragma unroll
-    for (int j = 0; j < kBins / kWarp; ++j) own += sh.hist[lane * (kBins / kWarp) + j];
-    uint32_t x = own;
+    const uint4 h = reinterpret_cast<const uint4*>(sh.hist)[tid];  // bins 4*tid .. 4*tid+3
+    const uint32_t own = h.x + h.y + h.z + h.w;
+    uint32_t x = own;  // bins >= 4*tid within this warp
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_down_sync(0xffffffffu, x, o);
         if (lane + o < 32) x += v;
     }
-    uint32_t S = x;  // count with digit >= 8*lane
-    uint32_t d_found = 0xffffffffu, a_found = 0;
-    if (S >= krem && S - own < krem) {
-        // the crossing is inside this lane's bins: walk them from the top
-        uint32_t run = S - own;
-        for (int j = kBins / kWarp - 1; j >= 0; --j) {
-            const uint32_t c = sh.hist[lane * (kBins / kWarp) + j];
-            if (run + c >= krem) {
-                d_found = (uint32_t)(lane * (kBins / kWarp) + j);
-                a_found = run;
-                break;
-            }
+    if (lane == 0) sh.wsum[wid] = x;
+    __syncthreads();
+    const uint32_t wt = sh.wsum[lane];
+    const uint32_t later = warp_sum(lane > wid ? wt : 0u);
+    const uint32_t total = warp_sum(wt);
+    const uint32_t S = x + later;  // keys in bins >= 4*tid
+    if (krem >= 1u && S >= krem && S - own < krem) {
+        uint32_t run = S - own, b = 4 * tid + 3, c = h.w;
+        if (run + c < krem) {
             run += c;
+            b = 4 * tid + 2;
+            c = h.z;
+            if (run + c < krem) {
+                run += c;
+                b = 4 * tid + 1;
+                c = h.y;
+                if (run + c < krem) {
+                    run += c;
+                    b = 4 * tid;
+                    c = h.x;
+                }
+            }
         }
+        sh.bin = b;
+        sh.above = run;
+        sh.in_bin = c;
     }
-    const uint32_t who = __ballot_sync(0xffffffffu, d_found != 0xffffffffu);
-    const int src = __ffs(who) - 1;
-    digit = __shfl_sync(0xffffffffu, d_found, src);
-    above = __shfl_sync(0xffffffffu, a_found, src);
-    __syncwarp();
+    __syncthreads();
+    bin = sh.bin;
+    above = sh.above;
+    in_bin = sh.in_bin;
+    return total;
 }
 
-// Exact k-th largest key: keys > thresh plus the first `quota` keys equal to
-// thresh (in position order) are the k_target largest.
-template <typename K>
-__device__ void block_select(SelShared& sh, const Keys<K>& keys, int n, uint32_t k_target, unsigned long long kmax,
-                             uint32_t nvalid, K* cand, K& thresh, uint32_t& quota) {
-    if (k_target == 0) {
-        thresh = ~K(0);
-        quota = 0;
-        return;
+// One radix level over m keys: histogram of the `width`-bit digit at `shift`
+// of the keys whose bits above shift+width equal `prefix`, then the digit
+// holding the krem-th largest of them; prefix grows by that digit and krem
+// drops by the count above it.
+template <typename K, typename Get>
+__device__ void radix_level(SelShared& sh, Get get, int m, int shift, int width, K& prefix, uint32_t& krem) {
+    const int tid = threadIdx.x;
+    reinterpret_cast<uint4*>(sh.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    const uint32_t mask = (1u << width) - 1u;
+    for (int i0 = tid; i0 < m; i0 += kSelThreads * kUnroll) {
+        K kv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kSelThreads;
+            kv[u] = i < m ? get(i) : K(0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (i0 + u * kSelThreads < m && (K)(kv[u] >> (shift + width)) == prefix)
+                atomicAdd(&sh.hist[(uint32_t)(kv[u] >> shift) & mask], 1u);
     }
-    if (k_target >= nvalid) {  // every candidate is kept
-        thresh = K(1);
-        quota = 0xffffffffu;
-        return;
-    }
-    int nbits = key_bits<K>((K)kmax);
-    if (nbits < 1) nbits = 1;
-    int width = nbits < 8 ? nbits : 8;
-    int shift = nbits - width;
+    __syncthreads();
     uint32_t d, above, in_bin;
-    hist_pass<K>(sh, keys, n, shift, width, K(0), k_target, d, above, in_bin);
-    K prefix = (K)d;
-    uint32_t krem = k_target - above;
-    if (shift > 0 && (int)in_bin <= kCandCap) {
-        // gather the threshold bin's keys; one warp resolves the rest
-        if (threadIdx.x == 0) sh.count = 0;
-        __syncthreads();
-        for (int i0 = threadIdx.x; i0 < n; i0 += kSelThreads * kUnroll) {
-            K kv[kUnroll];
+    find_bin(sh, krem, d, above, in_bin);
+    prefix = (K)((prefix << width) | (K)d);
+    krem -= above;
+}
+
+// One pass over the row's n keys in 16-byte vectors: copies them to `stage`
+// (shared memory) when given, adds the nonzero ones to sh.hist when
+// `add_hist`, and when `gather` appends the keys k with (k >> shift) == prefix
+// to cand (at most kCandCap; sh.count ends as the number found).
+template <typename K>
+__device__ void key_pass(SelShared& sh, const Keys<K>& src, int n, K* stage, bool add_hist, bool gather, int shift,
+                         K prefix, K* cand) {
+    constexpr int kPer = 16 / (int)sizeof(K);
+    const int nv = (n + kPer - 1) / kPer;
+    const int lane = lane_id();
+    for (int b0 = warp_id() * kWarp; b0 < nv; b0 += kSelThreads * kUnroll) {  // warp-uniform
+        uint4 v[kUnroll];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int i = i0 + u * kSelThreads;
-                kv[u] = i < n ? keys[i] : K(0);
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u)
-                if (i0 + u * kSelThreads < n && (K)(kv[u] >> shift) == prefix) cand[atomicAdd(&sh.count, 1u)] = kv[u];
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = b0 + u * kSelThreads + lane;
+            v[u] = i < nv ? src.vec(i) : make_uint4(0u, 0u, 0u, 0u);
         }
-        __syncthreads();
-        if (warp_id() == 0) {
-            while (shift > 0) {
-                width = shift < 8 ? shift : 8;
-                shift -= width;
-                // only keys matching the prefix are in the list at the first
-                // refinement; later refinements filter by the grown prefix
-                uint32_t dd, aa;
-                // compact the list to the keys matching the current prefix
-                const int m0 = (int)in_bin;
-                int m = 0;
-                for (int base = 0; base < m0; base += kWarp) {
-                    const int i = base + lane_id();
-                    const K key = i < m0 ? cand[i] : K(0);
-                    const bool keep = i < m0 && (K)(key >> (shift + width)) == prefix;
-                    const uint32_t mk = __ballot_sync(0xffffffffu, keep);
-                    const int pos = m + __popc(mk & lanemask_lt());
-                    __syncwarp();
-                    if (keep) cand[pos] = key;
-                    m += __popc(mk);
-                    __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = b0 + u * kSelThreads + lane;
+            if (stage != nullptr && i < nv) reinterpret_cast<uint4*>(stage)[i] = v[u];
+            const K* e = reinterpret_cast<const K*>(&v[u]);
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const K key = (kPer * i + j < n) ? e[j] : K(0);
+                if (add_hist && key != K(0)) atomicAdd(&sh.hist[key_bin((unsigned long long)key)], 1u);
+                if (gather) {
+                    const bool hit = key != K(0) && (K)(key >> shift) == prefix;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+                    if (bal != 0u) {
+                        const int leader = __ffs(bal) - 1;
+                        uint32_t base = 0;
+                        if (lane == leader) base = atomicAdd(&sh.count, (uint32_t)__popc(bal));
+                        base = __shfl_sync(0xffffffffu, base, leader);
+                        const uint32_t p = base + (uint32_t)__popc(bal & lanemask_lt());
+                        if (hit && p < (uint32_t)kCandCap) cand[p] = key;
+                    }
                 }
-                in_bin = (uint32_t)m;
-                warp_hist_pass<K>(sh, cand, m, shift, width, krem, dd, aa);
-                prefix = (K)((prefix << width) | (K)dd);
-                krem -= aa;
-            }
-            if (lane_id() == 0) {
-                sh.digit = (uint32_t)0;
-                sh.above = krem;
-                *reinterpret_cast<K*>(&sh.hist[0]) = prefix;
             }
         }
+    }
+}
+
+// Exact k-th largest key, 1 <= k < total, from the row's log-bin histogram
+// (in sh.hist; bin tb holds the k-th largest key, `above` keys lie in higher
+// bins, in_bin in tb). Keys > thresh plus the first `quota` keys == thresh in
+// position order are the k largest. `stage`, when given, receives the keys
+// and `keys` is switched to it.
+template <typename K>
+__device__ void resolve_threshold(SelShared& sh, Keys<K>& keys, int n, K* stage, bool keys_staged, uint32_t k,
+                                  uint32_t tb, uint32_t above, uint32_t in_bin, K* cand, K& thresh,
+                                  uint32_t& quota) {
+    if (tb < 64u) {  // small bins hold a single key value
+        thresh = (K)tb;
+        quota = k - above;
+        return;
+    }
+    const int nb = (int)(tb >> 6) + 6;  // bit length of the bin's keys
+    int shift = nb - 7;
+    K prefix = (K)(64u | (tb & 63u));
+    const bool list = in_bin <= (uint32_t)kCandCap;
+    if (list || (stage != nullptr && !keys_staged)) {
+        key_pass<K>(sh, keys, n, keys_staged ? nullptr : stage, false, list, shift, prefix, cand);
         __syncthreads();
-        prefix = *reinterpret_cast<const K*>(&sh.hist[0]);
-        krem = sh.above;
-        __syncthreads();
-    } else {
-        while (shift > 0) {
-            width = shift < 8 ? shift : 8;
-            shift -= width;
-            hist_pass<K>(sh, keys, n, shift, width, prefix, krem, d, above, in_bin);
-            prefix = (K)((prefix << width) | (K)d);
-            krem -= above;
-        }
+        if (stage != nullptr) keys.s = smem_u32(stage);
+    }
+    uint32_t krem = k - above;
+    const int m = list ? (int)min(sh.count, (uint32_t)kCandCap) : n;
+    while (shift > 0) {
+        const int width = shift < kDigitBits ? shift : kDigitBits;
+        shift -= width;
+        if (list) radix_level<K>(sh, [&](int i) { return cand[i]; }, m, shift, width, prefix, krem);
+        else radix_level<K>(sh, [&](int i) { return keys[i]; }, m, shift, width, prefix, krem);
     }
     thresh = prefix;
     quota = krem;
@@ -322,10 +242,7 @@ __device__ void block_select(SelShared& sh, const Keys<K>& keys, int n, uint32_t
 template <typename K, typename Emit>
 __device__ void block_compact(SelShared& sh, const Keys<K>& keys, int n, K thresh, uint32_t quota, Emit emit) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
-    if (tid == 0) {
-        sh.carry_gt = 0;
-        sh.carry_eq = 0;
-    }
+    uint32_t carry_g = 0, carry_e = 0;  // kept keys before this chunk
     for (int c0 = 0; c0 < n; c0 += kChunkWords * 32) {
         const int nw = min(kChunkWords, (n - c0 + 31) / 32);
         // bitmap words of this chunk: word w covers keys c0 + 32w .. c0 + 32w + 31
@@ -349,17 +266,10 @@ __device__ void block_compact(SelShared& sh, const Keys<K>& keys, int n, K thres
             }
         }
         __syncthreads();
-        const int w0 = tid * kWordsPerThread;
-        uint32_t cg = 0, ce = 0;
-#pragma unroll
-        for (int j = 0; j < kWordsPerThread; ++j) {
-            if (w0 + j < nw) {
-                cg += __popc(sh.gt_words[w0 + j]);
-                ce += __popc(sh.eq_words[w0 + j]);
-            }
-        }
-        // exclusive prefix of (cg, ce) over threads, in thread order
-        uint32_t xg = cg, xe = ce;
+        const uint32_t g = tid < nw ? sh.gt_words[tid] : 0u;
+        const uint32_t e = tid < nw ? sh.eq_words[tid] : 0u;
+        const uint32_t cg = (uint32_t)__popc(g), ce = (uint32_t)__popc(e);
+        uint32_t xg = cg, xe = ce;  // inclusive prefix over the warp
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t vg = __shfl_up_sync(0xffffffffu, xg, o);
@@ -374,35 +284,22 @@ __device__ void block_compact(SelShared& sh, const Keys<K>& keys, int n, K thres
             sh.wsum2[wid] = xe;
         }
         __syncthreads();
-        uint32_t gb = sh.carry_gt, eb = sh.carry_eq;
-        for (int w2 = 0; w2 < wid; ++w2) {
-            gb += sh.wsum[w2];
-            eb += sh.wsum2[w2];
+        const uint32_t tg = sh.wsum[lane], te = sh.wsum2[lane];
+        uint32_t gb = carry_g + warp_sum(lane < wid ? tg : 0u) + xg - cg;
+        uint32_t eb = carry_e + warp_sum(lane < wid ? te : 0u) + xe - ce;
+        carry_g += warp_sum(tg);
+        carry_e += warp_sum(te);
+        uint32_t both = g | e;
+        while (both) {
+            const int b = __ffs(both) - 1;
+            both &= both - 1;
+            const uint32_t below = (1u << b) - 1u;
+            const uint32_t pg = gb + (uint32_t)__popc(g & below), pe = eb + (uint32_t)__popc(e & below);
+            const int slot = c0 + 32 * tid + b;
+            if ((g >> b) & 1u) emit(slot, pg + min(pe, quota));
+            else if (pe < quota) emit(slot, pg + pe);
         }
-        gb += xg - cg;
-        eb += xe - ce;
-        for (int j = 0; j < kWordsPerThread; ++j) {
-            if (w0 + j >= nw) break;
-            const uint32_t g = sh.gt_words[w0 + j], e = sh.eq_words[w0 + j];
-            uint32_t both = g | e;
-            while (both) {
-                const int b = __ffs(both) - 1;
-                both &= both - 1;
-                const uint32_t below = (1u << b) - 1u;
-                const uint32_t pg = gb + __popc(g & below), pe = eb + __popc(e & below);
-                const int slot = c0 + 32 * (w0 + j) + b;
-                if ((g >> b) & 1u) emit(slot, pg + min(pe, quota));
-                else if (pe < quota) emit(slot, pg + pe);
-            }
-            gb += __popc(g);
-            eb += __popc(e);
-        }
-        __syncthreads();
-        if (tid == kSelThreads - 1) {
-            sh.carry_gt = gb;
-            sh.carry_eq = eb;
-        }
-        __syncthreads();
+        __syncthreads();  // the words and warp sums are rewritten by the next chunk
     }
 }
 
@@ -425,6 +322,10 @@ __device__ __forceinline__ bool row_ok_sel(const IndexArgs& a, int r, int64_t& o
     return true;
 }
 
+__host__ __device__ __forceinline__ size_t kept_smem_bytes(int hi_topblocks) {
+    return ((size_t)hi_topblocks * 4 + 15) / 16 * 16;
+}
+
 // HI: keep the hi_topblocks best candidate blocks (ascending block index).
 __global__ void __launch_bounds__(kSelThreads, 1) select_blocks_kernel(const __grid_constant__ IndexArgs a) {
     extern __shared__ __align__(16) uint8_t dyn[];
@@ -444,15 +345,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_blocks_kernel(const __g
     const int B = a.hi_block;
     const int b_lo = s / B;
     const int nb = ws > s ? (ws + B - 1) / B - b_lo : 0;
-    unsigned long long kmax;
-    uint32_t nvalid;
-    const Keys<uint64_t> keys =
-        stage_keys<uint64_t>(sh, a.coarse_keys + (int64_t)r * a.coarse_cap, nb, dyn, a.coarse_in_smem, kmax, nvalid);
-    const uint32_t k = min((uint32_t)a.hi_topblocks, nvalid);
-    uint64_t thr;
-    uint32_t quota;
-    block_select<uint64_t>(sh, keys, nb, k, kmax, nvalid, s_cand, thr, quota);
-    block_compact<uint64_t>(sh, keys, nb, thr, quota, [&](int slot, uint32_t rank) { kept[rank] = b_lo + slot; });
+    reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
+    if (threadIdx.x == 0) sh.count = 0;
+    __syncthreads();
+    uint64_t* stage = a.coarse_in_smem ? reinterpret_cast<uint64_t*>(dyn) : nullptr;
+    Keys<uint64_t> keys{a.coarse_keys + (int64_t)r * a.coarse_cap, 0u};
+    key_pass<uint64_t>(sh, keys, nb, stage, true, false, 0, 0ull, s_cand);
+    __syncthreads();
+    if (stage != nullptr) keys.s = smem_u32(stage);
+    uint32_t tb, above, in_bin;
+    const uint32_t total = find_bin(sh, (uint32_t)a.hi_topblocks, tb, above, in_bin);
+    const uint32_t k = min((uint32_t)a.hi_topblocks, total);
+    if (k > 0u) {
+        uint64_t thr = 1ull;
+        uint32_t quota = 0xffffffffu;  // k == total: every candidate is kept
+        if (k < total) resolve_threshold<uint64_t>(sh, keys, nb, stage, true, k, tb, above, in_bin, s_cand, thr, quota);
+        block_compact<uint64_t>(sh, keys, nb, thr, quota, [&](int slot, uint32_t rank) {
+            if (rank < k) kept[rank] = b_lo + slot;
+        });
+    }
     if (threadIdx.x == 0) a.n_kept[r] = (int32_t)k;
 }
 
@@ -460,7 +371,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_blocks_kernel(const __g
 __global__ void __launch_bounds__(kSelThreads, 1) select_tokens_kernel(const __grid_constant__ IndexArgs a) {
     extern __shared__ __align__(16) uint8_t dyn[];
     __shared__ SelShared sh;
-    __shared__ int32_t s_kept[LSA_MAX_TOPBLOCKS];
     __shared__ uint32_t s_cand[kCandCap];
     const int r = blockIdx.x;
     int64_t off;
@@ -476,6 +386,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tokens_kernel(const __g
     const int ws = max(s, L - a.window);
     const bool hi = a.hi_block > 0;
     const int B = a.hi_block;
+    int32_t* s_kept = reinterpret_cast<int32_t*>(dyn);
+    uint32_t* stage = a.fine_in_smem ? reinterpret_cast<uint32_t*>(dyn + (hi ? kept_smem_bytes(a.hi_topblocks) : 0))
+                                     : nullptr;
     int n_kept = 0;
     if (hi) {
         n_kept = a.n_kept[r];
@@ -483,24 +396,30 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tokens_kernel(const __g
         for (int i = threadIdx.x; i < n_kept; i += kSelThreads) s_kept[i] = kept[i];
     }
     const int n = hi ? n_kept * B : ws - s;
-    unsigned long long kmax;
-    uint32_t nvalid;
-    const Keys<uint32_t> keys =
-        stage_keys<uint32_t>(sh, a.fine_keys + (int64_t)r * a.fine_cap, n, dyn, a.fine_in_smem, kmax, nvalid);
-    const uint32_t k = min((uint32_t)a.topk, nvalid);
-    uint32_t thr, quota;
-    block_select<uint32_t>(sh, keys, n, k, kmax, nvalid, s_cand, thr, quota);
-    const int lgB = (hi && (B & (B - 1)) == 0) ? __ffs(B) - 1 : -1;  // power-of-two block: shift, not divide
-    block_compact<uint32_t>(sh, keys, n, thr, quota, [&](int slot, uint32_t rank) {
-        int tok;
-        if (hi) {
-            const int kb = lgB >= 0 ? slot >> lgB : slot / B;
-            tok = s_kept[kb] * B + (slot - kb * B);
-        } else {
-            tok = s + slot;
-        }
-        out[s + rank] = tok;
-    });
+    // the scoring kernel's histogram of this row's keys
+    reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] =
+        __ldcg(reinterpret_cast<const uint4*>(a.hist + (int64_t)r * kHistBins) + threadIdx.x);
+    if (threadIdx.x == 0) sh.count = 0;
+    __syncthreads();
+    uint32_t tb, above, in_bin;
+    const uint32_t total = find_bin(sh, (uint32_t)a.topk, tb, above, in_bin);
+    const uint32_t k = min((uint32_t)a.topk, total);
+    if (k > 0u) {
+        Keys<uint32_t> keys{a.fine_keys + (int64_t)r * a.fine_cap, 0u};
+        uint32_t thr = 1u, quota = 0xffffffffu;  // k == total: every candidate is kept
+        if (k < total) resolve_threshold<uint32_t>(sh, keys, n, stage, false, k, tb, above, in_bin, s_cand, thr, quota);
+        const int lgB = (hi && (B & (B - 1)) == 0) ? __ffs(B) - 1 : -1;  // power-of-two block: shift, not divide
+        block_compact<uint32_t>(sh, keys, n, thr, quota, [&](int slot, uint32_t rank) {
+            int tok;
+            if (hi) {
+                const int kb = lgB >= 0 ? slot >> lgB : slot / B;
+                tok = s_kept[kb] * B + (slot - kb * B);
+            } else {
+                tok = s + slot;
+            }
+            if (rank < k) out[s + rank] = tok;
+        });
+    }
     const int win0 = s + (int)k;
     const int n_win = L - ws;
     for (int e = threadIdx.x; e < a.budget; e += kSelThreads) {
@@ -516,7 +435,7 @@ static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Selection kernels keep the row's keys in shared memory up to these sizes.
 constexpr size_t kBlockKeySmem = 160 * 1024;
-constexpr size_t kTokenKeySmem = 180 * 1024;
+constexpr size_t kTokenKeySmem = 160 * 1024;
 
 IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     IndexPlan p;
@@ -533,7 +452,7 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     p.coarse_in_smem = hi && (size_t)p.coarse_cap * 8 <= kBlockKeySmem;
     p.fine_in_smem = (size_t)p.fine_cap * 4 <= kTokenKeySmem;
     p.smem_blocks = p.coarse_in_smem ? (size_t)p.coarse_cap * 8 : 0;
-    p.smem_tokens = p.fine_in_smem ? (size_t)p.fine_cap * 4 : 0;
+    p.smem_tokens = (hi ? kept_smem_bytes(b.hi_topblocks) : 0) + (p.fine_in_smem ? (size_t)p.fine_cap * 4 : 0);
     size_t off = 0;
     p.off_coarse = off;
     off = align256(off + (size_t)n_q * p.coarse_cap * 8);
@@ -543,6 +462,8 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     off = align256(off + (size_t)n_q * 4);
     p.off_fine = off;
     off = align256(off + (size_t)n_q * p.fine_cap * 4);
+    p.off_hist = off;
+    off = align256(off + (size_t)n_q * kHistBins * 4);
     p.ws_bytes = off;
     return p;
 }

@@ -31,6 +31,19 @@ struct BlockSumArgs {
 cudaError_t launch_block_sums(const BlockSumArgs& a, int d_I, cudaStream_t stream);
 
 // ---- indexer: scoring kernels + selection kernels -------------------------
+// Keys (score + 1) are histogrammed on a monotone logarithmic scale: the bit
+// length of the key and the 6 bits after its leading one (keys below 64 map
+// to themselves). 3776 bins cover every 64-bit key.
+constexpr int kHistBins = 4096;
+__host__ __device__ __forceinline__ uint32_t key_bin(unsigned long long key) {
+#ifdef __CUDA_ARCH__
+    const int nb = 64 - __clzll((long long)key);
+#else
+    const int nb = key ? 64 - __builtin_clzll(key) : 0;
+#endif
+    if (nb <= 6) return (uint32_t)key;
+    return ((uint32_t)(nb - 6) << 6) | (uint32_t)((key >> (nb - 7)) & 63ull);
+}
 struct IndexArgs {
     const int8_t* q_idx;
     const int8_t* k_idx;
@@ -53,6 +66,7 @@ struct IndexArgs {
     int32_t* kept;          // [n_q][hi_topblocks] kept block ids, ascending
     int32_t* n_kept;        // [n_q]
     uint32_t* fine_keys;    // [n_q][fine_cap] token keys (score + 1, 0 = none)
+    uint32_t* hist;         // [n_q][2][kHistBins] key histograms (coarse, fine); zero between calls
     int32_t coarse_cap, fine_cap;
     int32_t coarse_in_smem, fine_in_smem;
 };
@@ -61,7 +75,7 @@ struct IndexPlan {
     int coarse_cap = 0, fine_cap = 0;
     bool coarse_in_smem = false, fine_in_smem = false;
     size_t smem_blocks = 0, smem_tokens = 0;  // dynamic smem of the selection kernels
-    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0;
+    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0, off_hist = 0;
     size_t ws_bytes = 0;
 };
 IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b);

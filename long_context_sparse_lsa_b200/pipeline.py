@@ -57,13 +57,25 @@ class LsaStep:
         self.index(stream)
         self.attend(stream)
 
+    def overlap_ok(self, n_new: int = 1) -> bool:
+        """True when the block-sum append update may run beside the index call.
+
+        The update rewrites only the blocks holding the n_new newest tokens;
+        the coarse HI scores read only blocks that end before the window
+        start. With window >= hi_block + n_new - 1 those blocks lie inside the
+        window and the two calls touch disjoint rows."""
+        wl = self.wl
+        return self.block_sums is not None and wl.window >= wl.hi_block + n_new - 1
+
     def status_bits(self) -> int:
         return int(self.status.item())
 
     # -- CUDA graphs ------------------------------------------------------------
     def capture(self):
         """Capture the three calls as CUDA graphs (block-sum append update,
-        index, attend) so a step replays without host launch overhead. The
+        index, attend), and the whole step as one more graph ("step") in which
+        the block-sum update runs on a forked stream beside the index call when
+        overlap_ok(). A step then replays without host launch overhead. The
         graphs keep this object's buffers; changing their contents between
         replays is how new inputs enter."""
         side = torch.cuda.Stream(self.device)
@@ -81,15 +93,35 @@ class LsaStep:
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 fn()
             self.graphs[name] = g
+        g = torch.cuda.CUDAGraph()
+        fork = torch.cuda.Stream(self.device)
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            cur = torch.cuda.current_stream(self.device)
+            if self.overlap_ok(1):
+                fork.wait_stream(cur)
+                with torch.cuda.stream(fork):
+                    self.update_block_sums(1)
+                self.index()
+                cur.wait_stream(fork)
+                self.attend()
+            else:
+                self.step()
+        self.graphs["step"] = g
         torch.cuda.synchronize(self.device)
         return self.graphs
 
     def replay(self, name: str | None = None):
-        """Replay one captured call, or the whole step when name is None."""
-        if name is not None:
-            if name in self.graphs:
-                self.graphs[name].replay()
-            return
-        for n in ("block_sums", "index", "attend"):
-            if n in self.graphs:
-                self.graphs[n].replay()
+        """Replay one captured graph, or the whole step when name is None."""
+        name = name if name is not None else "step"
+        if name in self.graphs:
+            self.graphs[name].replay()
+
+    def kernels_per_step(self) -> int:
+        """Kernel launches of one step: the block-sum update (HI), the index
+        call's scoring and selection kernels (coarse ones only with HI) and the
+        attention kernel, plus its merge kernel when the call splits the
+        budget (it then asks for a partials workspace)."""
+        hi = self.block_sums is not None
+        ws_a = lsa.lsa_attend_workspace_size(self.batch, self.wl.H_q, self.wl.H_kv, self.wl.d, self.budget.length,
+                                             self.G)
+        return (1 if hi else 0) + (4 if hi else 2) + 1 + (1 if ws_a > 256 else 0)

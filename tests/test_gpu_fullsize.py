@@ -1,0 +1,92 @@
+"""Parity at the full workload sizes, in the launch configuration the bench
+times: the step graph captured through the C ABI (block-sum append update,
+index, attend) replayed once on seeded inputs.
+
+  * batched decode, 16 sequences x 131072 tokens, HI 64 x 256: every row;
+  * 1M-token decode with one index set for G = 4 layers, HI 128 x 512: the row
+    and all four layers;
+  * 64 ragged sequences (lognormal lengths, G = 2): a seeded sample of rows
+    plus the longest and the shortest;
+  * a causal prefill chunk of 8192 rows on a 262144-token cache (HI off): a
+    sample spanning the chunk.
+
+Index sets are compared bit-exact with the oracle; attention within
+max|err| 5e-3 and rel-L2 1e-3 of its fp64 evaluation on the K/V rows the
+oracle's own sets name.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import parity
+from long_context_sparse_lsa_b200 import workloads as wls
+from long_context_sparse_lsa_b200.pipeline import LsaStep
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run_graph(wl):
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    torch.cuda.synchronize()
+    st.capture()
+    st.sets.fill_(-7)
+    st.replay()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    return st, t
+
+
+def _check(wl, st, t, rows):
+    rows = np.asarray(rows)
+    want = parity.oracle_sets(wl, t, rows=rows)
+    parity.check_sets(parity.host(st.sets)[rows], want, wl.name)
+    ref = parity.oracle_attend_rows(t, want, rows)
+    for g in range(len(t.q)):
+        parity.check_attention(parity.host(st.out[g])[rows], ref[g], f"{wl.name} layer {g}")
+
+
+def _release(*objs):
+    for o in objs:
+        del o
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def test_batched_decode_128k_every_row():
+    wl = wls.BATCH128K
+    st, t = _run_graph(wl)
+    _check(wl, st, t, np.arange(wl.n_q))
+    _release(st, t)
+
+
+def test_1m_cross_layer_decode_every_layer():
+    wl = wls.CTX1M
+    st, t = _run_graph(wl)
+    assert len(t.q) == 4
+    _check(wl, st, t, np.arange(wl.n_q))
+    _release(st, t)
+
+
+def test_ragged_batch_sample():
+    wl = wls.ragged()
+    lens = np.asarray(wl.lens)
+    rng = np.random.default_rng(4)
+    rows = set(rng.choice(wl.n_q, size=10, replace=False).tolist())
+    rows |= {int(lens.argmax()), int(lens.argmin())}
+    st, t = _run_graph(wl)
+    _check(wl, st, t, sorted(rows))
+    _release(st, t)
+
+
+def test_prefill_chunk_sample():
+    wl = wls.PREFILL
+    st, t = _run_graph(wl)
+    n = wl.n_q
+    rows = [0, 1, 2047, 4096, 6000, n - 2, n - 1]
+    _check(wl, st, t, rows)
+    _release(st, t)

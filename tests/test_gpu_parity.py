@@ -61,6 +61,14 @@ CASES = {
     # ties: a tiny value range makes many equal scores
     "ties": dict(lens=(9000,), hi_block=0, hi_topblocks=0, qk_lo=-1, qk_hi=1, w_hi=1, topk=1000),
     "ties_hi": dict(lens=(9000,), hi_block=32, hi_topblocks=50, qk_lo=-1, qk_hi=1, w_hi=1, topk=1000),
+    # selection paths: every key equal and large (the threshold bin overflows
+    # the candidate list), keys small enough to be their own histogram bins,
+    # and rows too long to stage in shared memory (several compaction chunks)
+    "all_equal_big": dict(lens=(9000,), qk_lo=3, qk_hi=3, hi_block=0, hi_topblocks=0, topk=1500),
+    "all_equal_big_hi": dict(lens=(9000,), qk_lo=3, qk_hi=3, hi_block=32, hi_topblocks=60, topk=1500),
+    "small_keys": dict(lens=(6000,), H_I=1, d_I=32, qk_lo=0, qk_hi=1, w_hi=1, hi_block=0, hi_topblocks=0,
+                       topk=700),
+    "flat_60k": dict(lens=(60000, 45000), hi_block=0, hi_topblocks=0, topk=3000),
     # indexer head counts and key widths
     "heads1_d32": dict(lens=(5000,), H_I=1, d_I=32, qk_lo=-128, qk_hi=127, w_hi=16, hi_block=0, hi_topblocks=0),
     "heads20_d64": dict(lens=(7000, 100), H_I=20, d_I=64, hi_block=32, hi_topblocks=30),
