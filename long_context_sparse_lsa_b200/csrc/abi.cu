@@ -192,22 +192,19 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     a.kept = reinterpret_cast<int32_t*>(ws + plan.off_kept);
     a.n_kept = reinterpret_cast<int32_t*>(ws + plan.off_nkept);
     a.fine_keys = reinterpret_cast<uint32_t*>(ws + plan.off_fine);
-    a.hist = reinterpret_cast<uint32_t*>(ws + plan.off_hist);
     a.coarse_cap = plan.coarse_cap;
     a.fine_cap = plan.fine_cap;
-    a.coarse_in_smem = plan.coarse_in_smem ? 1 : 0;
-    a.fine_in_smem = plan.fine_in_smem ? 1 : 0;
+    a.coarse_stage = plan.coarse_stage;
+    a.fine_stage = plan.fine_stage;
+    a.kept_slots = plan.kept_slots;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (budget.hi_block > 0) {
         e = lsa::launch_index_scores(a, d_I, true, cs);
-        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, plan.smem_blocks, cs);
-    } else {
-        // with HI the coarse scoring kernel clears the fine-key histograms
-        e = cudaMemsetAsync(a.hist, 0, (size_t)batch->n_q * lsa::kHistBins * sizeof(uint32_t), cs);
+        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, plan.cluster, plan.smem_blocks, cs);
     }
     if (e == cudaSuccess) e = lsa::launch_index_scores(a, d_I, false, cs);
-    if (e == cudaSuccess) e = lsa::launch_index_select(a, false, plan.smem_tokens, cs);
+    if (e == cudaSuccess) e = lsa::launch_index_select(a, false, plan.cluster, plan.smem_tokens, cs);
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 

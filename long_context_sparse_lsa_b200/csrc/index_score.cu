@@ -12,10 +12,7 @@
 // 16-byte vector loads straight into MMA fragments; small CTAs and modest
 // register use keep several CTAs — and thus many loads in flight — on every
 // SM. Scores are written as keys (score + 1; 0 = not a candidate) to an
-// L2-resident workspace for the selection kernels; the fine kernel also adds
-// each key to its row's log-bin histogram (key_bin) there, which the coarse
-// kernel clears first, so that the token selection starts from a finished
-// histogram instead of a pass over the keys.
+// L2-resident workspace for the selection kernels.
 #include "index_common.cuh"
 
 namespace lsa {
@@ -46,10 +43,6 @@ __device__ __forceinline__ bool row_ok(const IndexArgs& a, int r, int64_t& off, 
 template <int D_I, int NT>
 __global__ void __launch_bounds__(kScThreads) coarse_score_kernel(const __grid_constant__ IndexArgs a) {
     const int r = blockIdx.y;
-    if (blockIdx.x == 0) {  // clear the row's fine-key histogram before the fine kernel runs
-        uint4* h = reinterpret_cast<uint4*>(a.hist + (int64_t)r * kHistBins);
-        for (int i = threadIdx.x; i < kHistBins / 4; i += kScThreads) h[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
     int64_t off;
     int L;
     if (!row_ok(a, r, off, L)) return;
@@ -124,7 +117,6 @@ __global__ void __launch_bounds__(kScThreads) fine_score_kernel(const __grid_con
     QueryFrag<D_I, NT> qf;
     load_query<D_I, NT>(qf, a, r);
     uint32_t* keys = a.fine_keys + (int64_t)r * a.fine_cap;
-    uint32_t* hist = a.hist + (int64_t)r * kHistBins;
 #pragma unroll
     for (int u = 0; u < kFineTilesPerWarp; ++u) {
         const int2 sc = fine_tile<D_I, NT>(qf, ra[u], rb[u]);
@@ -135,7 +127,6 @@ __global__ void __launch_bounds__(kScThreads) fine_score_kernel(const __grid_con
             const bool valid = t4 == 0 ? va[u] : vb[u];
             const uint32_t key = valid ? (uint32_t)(t4 == 0 ? sc.x : sc.y) + 1u : 0u;
             keys[slot] = key;
-            if (key != 0u) atomicAdd(hist + key_bin(key), 1u);
         }
     }
 }

@@ -9,41 +9,117 @@
 // HI bullets; "LongCat-2.0 (molayo1419.me)", section "1M 토큰에서의 Sparse
 // Attention 문제").
 //
-// Design (B200): one 1024-thread CTA per query row, so every synchronisation
-// is a CTA barrier. Selection starts from a histogram of the row's keys
-// (score + 1, 0 = not a candidate) on the logarithmic scale of key_bin: the
-// fine scoring kernel accumulates it in global memory while it writes the
-// keys; for HI blocks it is built here while the keys are staged. One suffix
-// scan of the histogram gives the bin holding the k-th largest key, one pass
-// over the keys (staging them in shared memory when they fit) gathers that
-// bin's keys into a short list, and 12-bit radix levels over the list give
-// the exact k-th largest key T and how many keys equal to T are kept (a bin
-// too full for the list is refined over all keys instead). Compaction is
-// bitmap based: warp ballots build "key > T" and "key == T" words, each
-// thread counts its word, one CTA prefix ranks them, and every thread emits
-// its kept positions in order.
+// Design (B200): a query row is selected by one thread-block cluster of C
+// CTAs, each owning a contiguous slice of the row's keys (score + 1, 0 = not
+// a candidate), so a pass over a row costs 1/C of a pass on one SM. The few
+// cross-CTA steps go through distributed shared memory and cluster barriers:
+//   1. every CTA stages its slice in shared memory and builds the slice's
+//      histogram on the logarithmic scale of key_bin, then adds its nonzero
+//      bins into every CTA's copy of the row histogram (remote red.add);
+//   2. each CTA scans the row histogram for the bin holding the k-th largest
+//      key (all CTAs reach the same answer), gathers its keys of that bin and
+//      appends them to every CTA's candidate list; 12-bit radix levels over
+//      that short list give the exact k-th largest key T and how many keys
+//      equal to T are kept (a bin too full for the list is refined by more
+//      cluster histograms over the slices instead);
+//   3. each CTA counts its kept keys and publishes the count; the counts of
+//      lower-ranked CTAs give its first output position, and bitmap ballots
+//      with one CTA prefix give every kept key its rank in position order.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace lsa {
 namespace {
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / kWarp;
-static_assert(kHistBins == 4 * kSelThreads, "the scan gives each thread four bins");
+constexpr int kBinsPerThread = kHistBins / kSelThreads;  // 8
+static_assert(kBinsPerThread == 8, "the scan gives each thread two 4-bin vectors");
+constexpr int kMaxCluster = 16;
 constexpr int kDigitBits = 12;            // refinement digit: 4096 bins
 constexpr int kCandCap = 2048;            // keys of the threshold bin held in a list
 constexpr int kChunkWords = kSelThreads;  // compaction: one bitmap word per thread per chunk
 constexpr int kUnroll = 4;                // independent loads in flight per thread
 
 struct SelShared {
-    uint32_t hist[kHistBins];
-    uint32_t wsum[kSelWarps];
-    uint32_t wsum2[kSelWarps];
+    uint32_t local_hist[kHistBins];  // this CTA's slice
+    uint32_t hist[kHistBins];        // the row: every CTA adds its slice into every CTA's copy
     uint32_t gt_words[kChunkWords];
     uint32_t eq_words[kChunkWords];
-    uint32_t bin, above, in_bin, count;
+    uint32_t wsum[kSelWarps];
+    uint32_t wsum2[kSelWarps];
+    uint32_t cta_gt[kMaxCluster];  // kept keys per CTA slice (each CTA writes its own into all)
+    uint32_t cta_eq[kMaxCluster];
+    uint32_t push_base[kMaxCluster];
+    uint32_t bin, above, in_bin;
+    uint32_t count;        // length of the row's candidate list (remote adds)
+    uint32_t local_count;  // candidates of this slice
 };
+
+// Dynamic shared memory: SelShared | candidate list | this slice's candidates
+// | staged slice keys | kept-block ids of the slice (tokens only).
+struct SelLayout {
+    uint32_t off_cand, off_mine, off_stage, off_kept, bytes;
+};
+
+__host__ __device__ __forceinline__ uint32_t align16u(uint32_t x) { return (x + 15u) / 16u * 16u; }
+
+__host__ __device__ __forceinline__ SelLayout sel_layout(int key_bytes, int stage_keys, int kept_slots) {
+    SelLayout L;
+    uint32_t o = align16u((uint32_t)sizeof(SelShared));
+    L.off_cand = o;
+    o += (uint32_t)(kCandCap * key_bytes);
+    L.off_mine = o;
+    o += (uint32_t)(kCandCap * key_bytes);
+    L.off_stage = o;
+    o += align16u((uint32_t)stage_keys * (uint32_t)key_bytes);
+    L.off_kept = o;
+    o += align16u((uint32_t)kept_slots * 4u);
+    L.bytes = o;
+    return L;
+}
+
+// ---- cluster primitives ----------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_cta(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t addr, uint32_t v) {
+    uint32_t r;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(r) : "r"(addr), "r"(v) : "memory");
+    return r;
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+template <typename K>
+__device__ __forceinline__ void st_cluster_key(uint32_t addr, K v) {
+    if constexpr (sizeof(K) == 4) {
+        st_cluster(addr, (uint32_t)v);
+    } else {
+        asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"((unsigned long long)v) : "memory");
+    }
+}
 
 __device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
 #pragma unroll
@@ -51,11 +127,12 @@ __device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
     return v;
 }
 
-// Keys of one row, either staged in shared memory or read from global memory.
+// Keys of this CTA's slice, either staged in shared memory or read from
+// global memory; index i is relative to the slice start.
 template <typename K>
 struct Keys {
-    const K* g;     // global copy
-    uint32_t s;     // shared-memory address of the staged copy (0 when not staged)
+    const K* g;  // global copy
+    uint32_t s;  // shared-memory address of the staged copy (0 when not staged)
     __device__ __forceinline__ K operator[](int i) const {
         if (s != 0u) {
             if constexpr (sizeof(K) == 4) {
@@ -83,14 +160,18 @@ struct Keys {
     }
 };
 
-// Suffix scan of sh.hist. Returns the number of counted keys; when
-// 1 <= krem <= total also gives the bin d holding the krem-th largest key,
-// the count above it (bins > d) and the count in it.
+// Suffix scan of the row histogram sh.hist. Returns the number of counted
+// keys; when 1 <= krem <= total also gives the bin holding the krem-th
+// largest key, the count above it (higher bins) and the count in it.
 __device__ uint32_t find_bin(SelShared& sh, uint32_t krem, uint32_t& bin, uint32_t& above, uint32_t& in_bin) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
-    const uint4 h = reinterpret_cast<const uint4*>(sh.hist)[tid];  // bins 4*tid .. 4*tid+3
-    const uint32_t own = h.x + h.y + h.z + h.w;
-    uint32_t x = own;  // bins >= 4*tid within this warp
+    const uint4 h0 = reinterpret_cast<const uint4*>(sh.hist)[2 * tid];  // bins 8*tid .. 8*tid+7
+    const uint4 h1 = reinterpret_cast<const uint4*>(sh.hist)[2 * tid + 1];
+    const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+    uint32_t own = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) own += c[j];
+    uint32_t x = own;  // keys in bins >= 8*tid within this warp
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_down_sync(0xffffffffu, x, o);
@@ -98,30 +179,22 @@ __device__ uint32_t find_bin(SelShared& sh, uint32_t krem, uint32_t& bin, uint32
     }
     if (lane == 0) sh.wsum[wid] = x;
     __syncthreads();
-    const uint32_t wt = sh.wsum[lane];
+    const uint32_t wt = lane < kSelWarps ? sh.wsum[lane] : 0u;
     const uint32_t later = warp_sum(lane > wid ? wt : 0u);
     const uint32_t total = warp_sum(wt);
-    const uint32_t S = x + later;  // keys in bins >= 4*tid
+    const uint32_t S = x + later;  // keys in bins >= 8*tid
     if (krem >= 1u && S >= krem && S - own < krem) {
-        uint32_t run = S - own, b = 4 * tid + 3, c = h.w;
-        if (run + c < krem) {
-            run += c;
-            b = 4 * tid + 2;
-            c = h.z;
-            if (run + c < krem) {
-                run += c;
-                b = 4 * tid + 1;
-                c = h.y;
-                if (run + c < krem) {
-                    run += c;
-                    b = 4 * tid;
-                    c = h.x;
-                }
+        uint32_t run = S - own;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+            if (run + c[j] >= krem) {
+                sh.bin = (uint32_t)(8 * tid + j);
+                sh.above = run;
+                sh.in_bin = c[j];
+                break;
             }
+            run += c[j];
         }
-        sh.bin = b;
-        sh.above = run;
-        sh.in_bin = c;
     }
     __syncthreads();
     bin = sh.bin;
@@ -130,17 +203,63 @@ __device__ uint32_t find_bin(SelShared& sh, uint32_t krem, uint32_t& bin, uint32
     return total;
 }
 
-// One radix level over m keys: histogram of the `width`-bit digit at `shift`
-// of the keys whose bits above shift+width equal `prefix`, then the digit
-// holding the krem-th largest of them; prefix grows by that digit and krem
-// drops by the count above it.
+// Adds this CTA's slice histogram (sh.local_hist) into every CTA's row
+// histogram; the caller brackets it with cluster barriers.
+__device__ void push_hist(SelShared& sh, uint32_t C) {
+    const uint32_t base = smem_u32(sh.hist);
+#pragma unroll
+    for (int j = 0; j < kBinsPerThread; ++j) {
+        const int b = threadIdx.x + j * kSelThreads;
+        const uint32_t v = sh.local_hist[b];
+        if (v != 0u)
+            for (uint32_t t = 0; t < C; ++t) red_add_cluster(map_cta(base + 4u * (uint32_t)b, t), v);
+    }
+}
+
+__device__ __forceinline__ void zero_hists(SelShared& sh) {
+    uint4* l = reinterpret_cast<uint4*>(sh.local_hist);
+    uint4* h = reinterpret_cast<uint4*>(sh.hist);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    l[threadIdx.x] = z;
+    l[threadIdx.x + kSelThreads] = z;
+    h[threadIdx.x] = z;
+    h[threadIdx.x + kSelThreads] = z;
+}
+
+// One pass over the slice's m keys in 16-byte vectors: copies them to `stage`
+// when given and adds the nonzero ones to sh.local_hist.
+template <typename K>
+__device__ void stage_pass(SelShared& sh, const Keys<K>& src, int m, K* stage) {
+    constexpr int kPer = 16 / (int)sizeof(K);
+    const int nv = (m + kPer - 1) / kPer;
+    for (int i0 = threadIdx.x; i0 < nv; i0 += kSelThreads * kUnroll) {
+        uint4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kSelThreads;
+            v[u] = i < nv ? src.vec(i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kSelThreads;
+            if (i >= nv) break;
+            if (stage != nullptr) reinterpret_cast<uint4*>(stage)[i] = v[u];
+            const K* e = reinterpret_cast<const K*>(&v[u]);
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const K key = (kPer * i + j < m) ? e[j] : K(0);
+                if (key != K(0)) atomicAdd(&sh.local_hist[key_bin((unsigned long long)key)], 1u);
+            }
+        }
+    }
+}
+
+// Local histogram of the `width`-bit digit at `shift` over the keys whose
+// bits above shift+width equal `prefix`.
 template <typename K, typename Get>
-__device__ void radix_level(SelShared& sh, Get get, int m, int shift, int width, K& prefix, uint32_t& krem) {
-    const int tid = threadIdx.x;
-    reinterpret_cast<uint4*>(sh.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();
+__device__ void digit_hist(uint32_t* hist, Get get, int m, int shift, int width, K prefix) {
     const uint32_t mask = (1u << width) - 1u;
-    for (int i0 = tid; i0 < m; i0 += kSelThreads * kUnroll) {
+    for (int i0 = threadIdx.x; i0 < m; i0 += kSelThreads * kUnroll) {
         K kv[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -150,66 +269,16 @@ __device__ void radix_level(SelShared& sh, Get get, int m, int shift, int width,
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
             if (i0 + u * kSelThreads < m && (K)(kv[u] >> (shift + width)) == prefix)
-                atomicAdd(&sh.hist[(uint32_t)(kv[u] >> shift) & mask], 1u);
-    }
-    __syncthreads();
-    uint32_t d, above, in_bin;
-    find_bin(sh, krem, d, above, in_bin);
-    prefix = (K)((prefix << width) | (K)d);
-    krem -= above;
-}
-
-// One pass over the row's n keys in 16-byte vectors: copies them to `stage`
-// (shared memory) when given, adds the nonzero ones to sh.hist when
-// `add_hist`, and when `gather` appends the keys k with (k >> shift) == prefix
-// to cand (at most kCandCap; sh.count ends as the number found).
-template <typename K>
-__device__ void key_pass(SelShared& sh, const Keys<K>& src, int n, K* stage, bool add_hist, bool gather, int shift,
-                         K prefix, K* cand) {
-    constexpr int kPer = 16 / (int)sizeof(K);
-    const int nv = (n + kPer - 1) / kPer;
-    const int lane = lane_id();
-    for (int b0 = warp_id() * kWarp; b0 < nv; b0 += kSelThreads * kUnroll) {  // warp-uniform
-        uint4 v[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = b0 + u * kSelThreads + lane;
-            v[u] = i < nv ? src.vec(i) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = b0 + u * kSelThreads + lane;
-            if (stage != nullptr && i < nv) reinterpret_cast<uint4*>(stage)[i] = v[u];
-            const K* e = reinterpret_cast<const K*>(&v[u]);
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const K key = (kPer * i + j < n) ? e[j] : K(0);
-                if (add_hist && key != K(0)) atomicAdd(&sh.hist[key_bin((unsigned long long)key)], 1u);
-                if (gather) {
-                    const bool hit = key != K(0) && (K)(key >> shift) == prefix;
-                    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-                    if (bal != 0u) {
-                        const int leader = __ffs(bal) - 1;
-                        uint32_t base = 0;
-                        if (lane == leader) base = atomicAdd(&sh.count, (uint32_t)__popc(bal));
-                        base = __shfl_sync(0xffffffffu, base, leader);
-                        const uint32_t p = base + (uint32_t)__popc(bal & lanemask_lt());
-                        if (hit && p < (uint32_t)kCandCap) cand[p] = key;
-                    }
-                }
-            }
-        }
+                atomicAdd(&hist[(uint32_t)(kv[u] >> shift) & mask], 1u);
     }
 }
 
-// Exact k-th largest key, 1 <= k < total, from the row's log-bin histogram
-// (in sh.hist; bin tb holds the k-th largest key, `above` keys lie in higher
-// bins, in_bin in tb). Keys > thresh plus the first `quota` keys == thresh in
-// position order are the k largest. `stage`, when given, receives the keys
-// and `keys` is switched to it.
+// Exact k-th largest key of the row, 1 <= k < total, given the bin tb that
+// holds it (`above` keys in higher bins, in_bin in tb). Keys > thresh plus
+// the first `quota` keys == thresh in position order are the k largest.
 template <typename K>
-__device__ void resolve_threshold(SelShared& sh, Keys<K>& keys, int n, K* stage, bool keys_staged, uint32_t k,
-                                  uint32_t tb, uint32_t above, uint32_t in_bin, K* cand, K& thresh,
+__device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, K* cand, K* mine, uint32_t C,
+                                  uint32_t k, uint32_t tb, uint32_t above, uint32_t in_bin, K& thresh,
                                   uint32_t& quota) {
     if (tb < 64u) {  // small bins hold a single key value
         thresh = (K)tb;
@@ -219,46 +288,134 @@ __device__ void resolve_threshold(SelShared& sh, Keys<K>& keys, int n, K* stage,
     const int nb = (int)(tb >> 6) + 6;  // bit length of the bin's keys
     int shift = nb - 7;
     K prefix = (K)(64u | (tb & 63u));
-    const bool list = in_bin <= (uint32_t)kCandCap;
-    if (list || (stage != nullptr && !keys_staged)) {
-        key_pass<K>(sh, keys, n, keys_staged ? nullptr : stage, false, list, shift, prefix, cand);
-        __syncthreads();
-        if (stage != nullptr) keys.s = smem_u32(stage);
-    }
     uint32_t krem = k - above;
-    const int m = list ? (int)min(sh.count, (uint32_t)kCandCap) : n;
-    while (shift > 0) {
-        const int width = shift < kDigitBits ? shift : kDigitBits;
-        shift -= width;
-        if (list) radix_level<K>(sh, [&](int i) { return cand[i]; }, m, shift, width, prefix, krem);
-        else radix_level<K>(sh, [&](int i) { return keys[i]; }, m, shift, width, prefix, krem);
+    if (in_bin <= (uint32_t)kCandCap) {
+        // gather this slice's keys of the bin, then append them to every
+        // CTA's candidate list
+        for (int i0 = threadIdx.x; i0 < m; i0 += kSelThreads * kUnroll) {
+            K kv[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = i0 + u * kSelThreads;
+                kv[u] = i < m ? keys[i] : K(0);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (i0 + u * kSelThreads < m && kv[u] != K(0) && (K)(kv[u] >> shift) == prefix) {
+                    const uint32_t p = atomicAdd(&sh.local_count, 1u);
+                    if (p < (uint32_t)kCandCap) mine[p] = kv[u];
+                }
+            }
+        }
+        __syncthreads();
+        const uint32_t mc = min(sh.local_count, (uint32_t)kCandCap);
+        if (threadIdx.x < C) sh.push_base[threadIdx.x] = atom_add_cluster(map_cta(smem_u32(&sh.count), threadIdx.x), mc);
+        __syncthreads();
+        const uint32_t cbase = smem_u32(cand);
+        for (uint32_t i = threadIdx.x; i < mc; i += kSelThreads) {
+            const K key = mine[i];
+            for (uint32_t t = 0; t < C; ++t) {
+                const uint32_t p = sh.push_base[t] + i;
+                if (p < (uint32_t)kCandCap) st_cluster_key<K>(map_cta(cbase + (uint32_t)sizeof(K) * p, t), key);
+            }
+        }
+        cluster_sync();
+        const int mm = (int)min(sh.count, (uint32_t)kCandCap);
+        while (shift > 0) {  // identical in every CTA
+            const int width = shift < kDigitBits ? shift : kDigitBits;
+            shift -= width;
+            reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4*>(sh.hist)[threadIdx.x + kSelThreads] = make_uint4(0u, 0u, 0u, 0u);
+            __syncthreads();
+            digit_hist<K>(sh.hist, [&](int i) { return cand[i]; }, mm, shift, width, prefix);
+            __syncthreads();
+            uint32_t d, ab, ib;
+            find_bin(sh, krem, d, ab, ib);
+            prefix = (K)((prefix << width) | (K)d);
+            krem -= ab;
+        }
+    } else {
+        // refine over the slices: one cluster histogram per digit
+        while (shift > 0) {
+            const int width = shift < kDigitBits ? shift : kDigitBits;
+            shift -= width;
+            zero_hists(sh);
+            __syncthreads();
+            digit_hist<K>(sh.local_hist, [&](int i) { return keys[i]; }, m, shift, width, prefix);
+            __syncthreads();
+            cluster_sync();  // every CTA's row histogram is clear and its slice counted
+            push_hist(sh, C);
+            cluster_sync();
+            uint32_t d, ab, ib;
+            find_bin(sh, krem, d, ab, ib);
+            prefix = (K)((prefix << width) | (K)d);
+            krem -= ab;
+        }
     }
     thresh = prefix;
     quota = krem;
 }
 
-// emit(slot, rank) for every kept key (key > thresh, plus the first `quota`
-// keys == thresh in position order), rank = its position among kept keys.
+// Kept keys (key > thresh, plus the first `quota` keys == thresh of the row
+// in position order) of this CTA's slice; emit(slot, rank) with slot relative
+// to the slice and rank the key's position among the row's kept keys.
 template <typename K, typename Emit>
-__device__ void block_compact(SelShared& sh, const Keys<K>& keys, int n, K thresh, uint32_t quota, Emit emit) {
+__device__ void cluster_compact(SelShared& sh, const Keys<K>& keys, int m, uint32_t C, uint32_t c, K thresh,
+                                uint32_t quota, Emit emit) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
-    uint32_t carry_g = 0, carry_e = 0;  // kept keys before this chunk
-    for (int c0 = 0; c0 < n; c0 += kChunkWords * 32) {
-        const int nw = min(kChunkWords, (n - c0 + 31) / 32);
-        // bitmap words of this chunk: word w covers keys c0 + 32w .. c0 + 32w + 31
+    // 1. this slice's counts, published to every CTA
+    const int nw_all = (m + 31) / 32;
+    uint32_t ng = 0, ne = 0;
+    for (int w0 = wid; w0 < nw_all; w0 += kSelWarps * kUnroll) {
+        K kv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = 32 * (w0 + u * kSelWarps) + lane;
+            kv[u] = i < m ? keys[i] : K(0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = 32 * (w0 + u * kSelWarps) + lane;
+            ng += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] > thresh));
+            ne += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] == thresh));
+        }
+    }
+    if (lane == 0) {
+        sh.wsum[wid] = ng;
+        sh.wsum2[wid] = ne;
+    }
+    __syncthreads();
+    if (tid < (int)C) {
+        uint32_t tg = 0, te = 0;
+        for (int w = 0; w < kSelWarps; ++w) {
+            tg += sh.wsum[w];
+            te += sh.wsum2[w];
+        }
+        st_cluster(map_cta(smem_u32(&sh.cta_gt[c]), (uint32_t)tid), tg);
+        st_cluster(map_cta(smem_u32(&sh.cta_eq[c]), (uint32_t)tid), te);
+    }
+    cluster_sync();  // after this no CTA touches another CTA's shared memory
+    uint32_t carry_g = 0, carry_e = 0;
+    for (uint32_t t = 0; t < c; ++t) {
+        carry_g += sh.cta_gt[t];
+        carry_e += sh.cta_eq[t];
+    }
+    // 2. ranks within the slice, one bitmap chunk at a time
+    for (int c0 = 0; c0 < m; c0 += kChunkWords * 32) {
+        const int nw = min(kChunkWords, (m - c0 + 31) / 32);
         for (int w0 = wid; w0 < nw; w0 += kSelWarps * kUnroll) {
             K kv[kUnroll];
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int i = c0 + 32 * (w0 + u * kSelWarps) + lane;
-                kv[u] = i < n ? keys[i] : K(0);
+                kv[u] = i < m ? keys[i] : K(0);
             }
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int w = w0 + u * kSelWarps;
                 const int i = c0 + 32 * w + lane;
-                const uint32_t g = __ballot_sync(0xffffffffu, i < n && kv[u] > thresh);
-                const uint32_t e = __ballot_sync(0xffffffffu, i < n && kv[u] == thresh);
+                const uint32_t g = __ballot_sync(0xffffffffu, i < m && kv[u] > thresh);
+                const uint32_t e = __ballot_sync(0xffffffffu, i < m && kv[u] == thresh);
                 if (lane == 0 && w < nw) {
                     sh.gt_words[w] = g;
                     sh.eq_words[w] = e;
@@ -284,7 +441,8 @@ __device__ void block_compact(SelShared& sh, const Keys<K>& keys, int n, K thres
             sh.wsum2[wid] = xe;
         }
         __syncthreads();
-        const uint32_t tg = sh.wsum[lane], te = sh.wsum2[lane];
+        const uint32_t tg = lane < kSelWarps ? sh.wsum[lane] : 0u;
+        const uint32_t te = lane < kSelWarps ? sh.wsum2[lane] : 0u;
         uint32_t gb = carry_g + warp_sum(lane < wid ? tg : 0u) + xg - cg;
         uint32_t eb = carry_e + warp_sum(lane < wid ? te : 0u) + xe - ce;
         carry_g += warp_sum(tg);
@@ -322,110 +480,115 @@ __device__ __forceinline__ bool row_ok_sel(const IndexArgs& a, int r, int64_t& o
     return true;
 }
 
-__host__ __device__ __forceinline__ size_t kept_smem_bytes(int hi_topblocks) {
-    return ((size_t)hi_topblocks * 4 + 15) / 16 * 16;
+// Slice of CTA c of C over n keys, in whole 32-key words: [k_lo, k_lo + m).
+__device__ __forceinline__ void slice_of(int n, uint32_t C, uint32_t c, int& k_lo, int& m) {
+    const int W = (n + 31) / 32;
+    const int w_lo = (int)((int64_t)W * c / C), w_hi = (int)((int64_t)W * (c + 1) / C);
+    k_lo = 32 * w_lo;
+    m = max(0, min(n, 32 * w_hi) - k_lo);
 }
 
-// HI: keep the hi_topblocks best candidate blocks (ascending block index).
-__global__ void __launch_bounds__(kSelThreads, 1) select_blocks_kernel(const __grid_constant__ IndexArgs a) {
+// Selection of one row by one cluster. kTokens: fine top-k and the SI
+// assembly of the index set; otherwise the HI block top-k.
+template <typename K, bool kTokens>
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_constant__ IndexArgs a) {
     extern __shared__ __align__(16) uint8_t dyn[];
-    __shared__ SelShared sh;
-    __shared__ uint64_t s_cand[kCandCap];
-    const int r = blockIdx.x;
-    int64_t off;
-    int L;
-    int32_t bits;
-    int32_t* kept = a.kept + (int64_t)r * a.hi_topblocks;
-    if (!row_ok_sel(a, r, off, L, bits)) {
-        if (threadIdx.x == 0) a.n_kept[r] = 0;
-        return;  // the token selection reports the row
-    }
-    const int s = min(a.sink, L);
-    const int ws = max(s, L - a.window);
-    const int B = a.hi_block;
-    const int b_lo = s / B;
-    const int nb = ws > s ? (ws + B - 1) / B - b_lo : 0;
-    reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
-    if (threadIdx.x == 0) sh.count = 0;
-    __syncthreads();
-    uint64_t* stage = a.coarse_in_smem ? reinterpret_cast<uint64_t*>(dyn) : nullptr;
-    Keys<uint64_t> keys{a.coarse_keys + (int64_t)r * a.coarse_cap, 0u};
-    key_pass<uint64_t>(sh, keys, nb, stage, true, false, 0, 0ull, s_cand);
-    __syncthreads();
-    if (stage != nullptr) keys.s = smem_u32(stage);
-    uint32_t tb, above, in_bin;
-    const uint32_t total = find_bin(sh, (uint32_t)a.hi_topblocks, tb, above, in_bin);
-    const uint32_t k = min((uint32_t)a.hi_topblocks, total);
-    if (k > 0u) {
-        uint64_t thr = 1ull;
-        uint32_t quota = 0xffffffffu;  // k == total: every candidate is kept
-        if (k < total) resolve_threshold<uint64_t>(sh, keys, nb, stage, true, k, tb, above, in_bin, s_cand, thr, quota);
-        block_compact<uint64_t>(sh, keys, nb, thr, quota, [&](int slot, uint32_t rank) {
-            if (rank < k) kept[rank] = b_lo + slot;
-        });
-    }
-    if (threadIdx.x == 0) a.n_kept[r] = (int32_t)k;
-}
-
-// Fine top-k plus the SI assembly of the index set.
-__global__ void __launch_bounds__(kSelThreads, 1) select_tokens_kernel(const __grid_constant__ IndexArgs a) {
-    extern __shared__ __align__(16) uint8_t dyn[];
-    __shared__ SelShared sh;
-    __shared__ uint32_t s_cand[kCandCap];
-    const int r = blockIdx.x;
-    int64_t off;
-    int L;
-    int32_t bits;
+    SelShared& sh = *reinterpret_cast<SelShared*>(dyn);
+    const int r = blockIdx.y;
+    const uint32_t C = cluster_size(), c = cluster_rank();
+    const int stage_cap = kTokens ? a.fine_stage : a.coarse_stage;
+    const SelLayout lay = sel_layout((int)sizeof(K), stage_cap, kTokens ? a.kept_slots : 0);
+    K* cand = reinterpret_cast<K*>(dyn + lay.off_cand);
+    K* mine = reinterpret_cast<K*>(dyn + lay.off_mine);
+    K* stage = stage_cap > 0 ? reinterpret_cast<K*>(dyn + lay.off_stage) : nullptr;
+    int32_t* s_kept = reinterpret_cast<int32_t*>(dyn + lay.off_kept);
     int32_t* out = a.index_sets + (int64_t)r * a.budget;
-    if (!row_ok_sel(a, r, off, L, bits)) {
-        if (threadIdx.x == 0) flag(a.dev_status, bits);
-        for (int e = threadIdx.x; e < a.budget; e += kSelThreads) out[e] = -1;
+    const int n_kept_row = (kTokens && a.hi_block > 0) ? a.n_kept[r] : 0;
+    int64_t off;
+    int L;
+    int32_t bits;
+    if (!row_ok_sel(a, r, off, L, bits)) {  // uniform over the cluster: no cluster barrier is reached
+        if (kTokens) {
+            if (c == 0 && threadIdx.x == 0) flag(a.dev_status, bits);
+            for (int e = (int)(c * kSelThreads) + threadIdx.x; e < a.budget; e += (int)(C * kSelThreads)) out[e] = -1;
+        } else if (c == 0 && threadIdx.x == 0) {
+            a.n_kept[r] = 0;  // the token selection reports the row
+        }
         return;
     }
     const int s = min(a.sink, L);
     const int ws = max(s, L - a.window);
-    const bool hi = a.hi_block > 0;
     const int B = a.hi_block;
-    int32_t* s_kept = reinterpret_cast<int32_t*>(dyn);
-    uint32_t* stage = a.fine_in_smem ? reinterpret_cast<uint32_t*>(dyn + (hi ? kept_smem_bytes(a.hi_topblocks) : 0))
-                                     : nullptr;
-    int n_kept = 0;
-    if (hi) {
-        n_kept = a.n_kept[r];
+    int n, first;  // keys of the row; first slot's block (blocks) or token (flat tokens)
+    if (kTokens) {
+        n = B > 0 ? n_kept_row * B : ws - s;
+        first = s;
+    } else {
+        first = s / B;
+        n = ws > s ? (ws + B - 1) / B - first : 0;
+    }
+    int k_lo, m;
+    slice_of(n, C, c, k_lo, m);
+    const K* row_keys = kTokens ? reinterpret_cast<const K*>(a.fine_keys + (int64_t)r * a.fine_cap)
+                                : reinterpret_cast<const K*>(a.coarse_keys + (int64_t)r * a.coarse_cap);
+    Keys<K> keys{row_keys + k_lo, 0u};
+    int kb_lo = 0;
+    if (kTokens && B > 0 && m > 0) {  // kept blocks that this slice's slots fall in
+        kb_lo = k_lo / B;
+        const int kb_hi = (k_lo + m - 1) / B;
         const int32_t* kept = a.kept + (int64_t)r * a.hi_topblocks;
-        for (int i = threadIdx.x; i < n_kept; i += kSelThreads) s_kept[i] = kept[i];
+        for (int i = threadIdx.x; i <= kb_hi - kb_lo && i < a.kept_slots; i += kSelThreads) s_kept[i] = kept[kb_lo + i];
     }
-    const int n = hi ? n_kept * B : ws - s;
-    // the scoring kernel's histogram of this row's keys
-    reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] =
-        __ldcg(reinterpret_cast<const uint4*>(a.hist + (int64_t)r * kHistBins) + threadIdx.x);
-    if (threadIdx.x == 0) sh.count = 0;
+    zero_hists(sh);
+    if (threadIdx.x == 0) {
+        sh.count = 0;
+        sh.local_count = 0;
+    }
     __syncthreads();
+    stage_pass<K>(sh, keys, m, stage);
+    __syncthreads();
+    if (stage != nullptr) keys.s = smem_u32(stage);
+    cluster_sync();  // every CTA's row histogram is clear and its slice counted
+    push_hist(sh, C);
+    cluster_sync();
+    const uint32_t want = (uint32_t)(kTokens ? a.topk : a.hi_topblocks);
     uint32_t tb, above, in_bin;
-    const uint32_t total = find_bin(sh, (uint32_t)a.topk, tb, above, in_bin);
-    const uint32_t k = min((uint32_t)a.topk, total);
+    const uint32_t total = find_bin(sh, want, tb, above, in_bin);
+    const uint32_t k = min(want, total);
     if (k > 0u) {
-        Keys<uint32_t> keys{a.fine_keys + (int64_t)r * a.fine_cap, 0u};
-        uint32_t thr = 1u, quota = 0xffffffffu;  // k == total: every candidate is kept
-        if (k < total) resolve_threshold<uint32_t>(sh, keys, n, stage, false, k, tb, above, in_bin, s_cand, thr, quota);
-        const int lgB = (hi && (B & (B - 1)) == 0) ? __ffs(B) - 1 : -1;  // power-of-two block: shift, not divide
-        block_compact<uint32_t>(sh, keys, n, thr, quota, [&](int slot, uint32_t rank) {
-            int tok;
-            if (hi) {
-                const int kb = lgB >= 0 ? slot >> lgB : slot / B;
-                tok = s_kept[kb] * B + (slot - kb * B);
-            } else {
-                tok = s + slot;
-            }
-            if (rank < k) out[s + rank] = tok;
-        });
+        K thr = K(1);
+        uint32_t quota = 0xffffffffu;  // k == total: every candidate is kept
+        if (k < total) resolve_threshold<K>(sh, keys, m, cand, mine, C, k, tb, above, in_bin, thr, quota);
+        if (kTokens) {
+            const int lgB = (B > 0 && (B & (B - 1)) == 0) ? __ffs(B) - 1 : -1;  // power-of-two block: shift
+            cluster_compact<K>(sh, keys, m, C, c, thr, quota, [&](int slot, uint32_t rank) {
+                const int gs = k_lo + slot;
+                int tok;
+                if (B > 0) {
+                    const int kb = lgB >= 0 ? gs >> lgB : gs / B;
+                    tok = s_kept[kb - kb_lo] * B + (gs - kb * B);
+                } else {
+                    tok = first + gs;
+                }
+                if (rank < k) out[s + rank] = tok;
+            });
+        } else {
+            int32_t* kept = a.kept + (int64_t)r * a.hi_topblocks;
+            cluster_compact<K>(sh, keys, m, C, c, thr, quota, [&](int slot, uint32_t rank) {
+                if (rank < k) kept[rank] = first + k_lo + slot;
+            });
+        }
     }
-    const int win0 = s + (int)k;
-    const int n_win = L - ws;
-    for (int e = threadIdx.x; e < a.budget; e += kSelThreads) {
-        if (e < s) out[e] = e;
-        else if (e >= win0 && e < win0 + n_win) out[e] = ws + (e - win0);
-        else if (e >= win0 + n_win) out[e] = -1;
+    if (kTokens) {
+        const int win0 = s + (int)k;
+        const int n_win = L - ws;
+        for (int e = (int)(c * kSelThreads) + threadIdx.x; e < a.budget; e += (int)(C * kSelThreads)) {
+            if (e < s) out[e] = e;
+            else if (e >= win0 && e < win0 + n_win) out[e] = ws + (e - win0);
+            else if (e >= win0 + n_win) out[e] = -1;
+        }
+    } else if (c == 0 && threadIdx.x == 0) {
+        a.n_kept[r] = (int32_t)k;
     }
 }
 
@@ -433,9 +596,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tokens_kernel(const __g
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Selection kernels keep the row's keys in shared memory up to these sizes.
-constexpr size_t kBlockKeySmem = 160 * 1024;
-constexpr size_t kTokenKeySmem = 160 * 1024;
+// Staged slice keys plus kept-block ids stay within this much shared memory.
+constexpr size_t kStageSmem = 144 * 1024;
 
 IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     IndexPlan p;
@@ -449,10 +611,20 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     }
     p.fine_cap = (p.fine_cap + 3) / 4 * 4;
     if (p.fine_cap < 4) p.fine_cap = 4;
-    p.coarse_in_smem = hi && (size_t)p.coarse_cap * 8 <= kBlockKeySmem;
-    p.fine_in_smem = (size_t)p.fine_cap * 4 <= kTokenKeySmem;
-    p.smem_blocks = p.coarse_in_smem ? (size_t)p.coarse_cap * 8 : 0;
-    p.smem_tokens = (hi ? kept_smem_bytes(b.hi_topblocks) : 0) + (p.fine_in_smem ? (size_t)p.fine_cap * 4 : 0);
+    p.cluster = 8;
+    // largest slice: whole 32-key words split over the cluster
+    auto slice_max = [&](int cap) { return 32 * (((cap + 31) / 32 + p.cluster - 1) / p.cluster); };
+    if (hi) {
+        const int sm = slice_max(p.coarse_cap);
+        p.coarse_stage = (size_t)sm * 8 <= kStageSmem ? sm : 0;
+        p.smem_blocks = sel_layout(8, p.coarse_stage, 0).bytes;
+    }
+    {
+        const int sm = slice_max(p.fine_cap);
+        p.kept_slots = hi ? std::min(b.hi_topblocks, sm / b.hi_block + 2) : 0;
+        p.fine_stage = (size_t)sm * 4 + (size_t)p.kept_slots * 4 <= kStageSmem ? sm : 0;
+        p.smem_tokens = sel_layout(4, p.fine_stage, p.kept_slots).bytes;
+    }
     size_t off = 0;
     p.off_coarse = off;
     off = align256(off + (size_t)n_q * p.coarse_cap * 8);
@@ -462,25 +634,37 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     off = align256(off + (size_t)n_q * 4);
     p.off_fine = off;
     off = align256(off + (size_t)n_q * p.fine_cap * 4);
-    p.off_hist = off;
-    off = align256(off + (size_t)n_q * kHistBins * 4);
     p.ws_bytes = off;
     return p;
 }
 
-cudaError_t launch_index_select(const IndexArgs& a, bool blocks, size_t smem, cudaStream_t stream) {
-    if (blocks) {
-        cudaError_t e = cudaFuncSetAttribute(select_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+template <typename Kern>
+static cudaError_t launch_cluster(Kern kern, const IndexArgs& a, int cluster, size_t smem, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (cluster > 8) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
-        select_blocks_kernel<<<a.n_q, kSelThreads, smem, stream>>>(a);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(select_tokens_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        select_tokens_kernel<<<a.n_q, kSelThreads, smem, stream>>>(a);
     }
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cluster, (unsigned)a.n_q, 1);
+    cfg.blockDim = dim3(kSelThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream) {
+    if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
+    return blocks ? launch_cluster(select_kernel<uint64_t, false>, a, cluster, smem, stream)
+                  : launch_cluster(select_kernel<uint32_t, true>, a, cluster, smem, stream);
 }
 
 }  // namespace lsa

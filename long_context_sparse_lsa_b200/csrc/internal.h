@@ -66,21 +66,23 @@ struct IndexArgs {
     int32_t* kept;          // [n_q][hi_topblocks] kept block ids, ascending
     int32_t* n_kept;        // [n_q]
     uint32_t* fine_keys;    // [n_q][fine_cap] token keys (score + 1, 0 = none)
-    uint32_t* hist;         // [n_q][2][kHistBins] key histograms (coarse, fine); zero between calls
     int32_t coarse_cap, fine_cap;
-    int32_t coarse_in_smem, fine_in_smem;
+    // selection: keys of one CTA's slice staged in shared memory (0 = read
+    // from global memory) and kept-block slots per slice
+    int32_t coarse_stage, fine_stage, kept_slots;
 };
 
 struct IndexPlan {
     int coarse_cap = 0, fine_cap = 0;
-    bool coarse_in_smem = false, fine_in_smem = false;
+    int cluster = 8;                          // CTAs per query row in the selection kernels
+    int coarse_stage = 0, fine_stage = 0, kept_slots = 0;
     size_t smem_blocks = 0, smem_tokens = 0;  // dynamic smem of the selection kernels
-    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0, off_hist = 0;
+    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0;
     size_t ws_bytes = 0;
 };
 IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b);
 cudaError_t launch_index_scores(const IndexArgs& a, int d_I, bool coarse, cudaStream_t stream);
-cudaError_t launch_index_select(const IndexArgs& a, bool blocks, size_t smem, cudaStream_t stream);
+cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream);
 
 // ---- sparse attention -----------------------------------------------------
 struct AttendArgs {
