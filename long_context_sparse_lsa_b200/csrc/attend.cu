@@ -1,5 +1,5 @@
 // attend.cu — sparse GQA softmax attention over LSA index sets, split over
-// the set entries, with the split partials merged in the same launch.
+// the set entries, and the merge of the split partials.
 //
 // The method: attention runs only over the tokens the indexer selected; SI
 // makes the sink and window parts contiguous KV runs ("LongCat-Flash-Lite-
