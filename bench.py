@@ -2,12 +2,13 @@
 
 A step is one decode step of the batched 128K workload (16 sequences x
 131072 tokens, HI 64x256, sink/window/topk 64/1024/2048, 32 q heads over 4
-kv heads): the HI block-sum append update, the fused indexer (coarse pass,
-block selection, fine scores, top-k, SI assembly) and the split-K sparse
+kv heads): the HI block-sum append update, the indexer (coarse scores, HI
+block selection, fine scores, top-k and SI assembly) and the split-K sparse
 attention with its merge. Inputs are seeded synthetic tensors resident in
 HBM. L2 is flushed (a 2 x L2-size write) before every timed step, outside the
-timed interval; every kernel is timed with CUDA events on the launching
-stream.
+timed interval; every step is timed with CUDA events on the launching
+stream. On one GPU the line also carries the 1M-token decode (one index set
+for G = 4 layers) and the 8192-token causal prefill chunk under "secondary".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
 
@@ -45,14 +46,15 @@ PROFILES = os.path.join(ROOT, "profiles")
 # ---------------------------------------------------------------------------
 def step_bytes(wl) -> dict:
     n_q, G = wl.n_q, wl.G
-    ent = [min(L, wl.budget) for L in wl.lens] if not wl.prefill_new else None
     kv_row = wl.H_kv * wl.d * 2  # bytes of one token's K (or V) in one layer
+    rows = _rows(wl)
     attend = 0
-    for e in ent:
+    for L in rows:
+        e = min(L, wl.budget)
         attend += G * (2 * e * kv_row + wl.H_q * wl.d * 2 + wl.H_q * wl.d * 4 + wl.budget * 4)
     index = 0
     bsum = 0
-    for L in wl.lens:
+    for L in rows:
         s = min(wl.sink, L)
         ws = max(s, L - wl.window)
         if wl.hi_block > 0:
@@ -64,7 +66,27 @@ def step_bytes(wl) -> dict:
         else:
             index += (ws - s) * wl.d_I
         index += wl.H_I * wl.d_I + wl.H_I * 4 + wl.budget * 4  # q, w, index-set write
+    if wl.prefill_new:  # one cache shared by every row of the chunk: read it once
+        index = wl.lens[0] * wl.d_I + n_q * (wl.H_I * wl.d_I + wl.H_I * 4 + wl.budget * 4)
     return {"attend": attend, "index": index, "block_sums": bsum, "total": attend + index + bsum}
+
+
+def _rows(wl):
+    """Visible length of every query row."""
+    if wl.prefill_new:
+        C = wl.lens[0] - wl.prefill_new
+        return [C + i + 1 for i in range(wl.prefill_new)]
+    return list(wl.lens)
+
+
+def index_int8_ops(wl) -> int:
+    """Multiply-adds x 2 of the fine scores (every middle token of every row)."""
+    tot = 0
+    for L in _rows(wl):
+        s = min(wl.sink, L)
+        ws = max(s, L - wl.window)
+        tot += ws - s
+    return 2 * tot * wl.H_I * wl.d_I
 
 
 # ---------------------------------------------------------------------------
@@ -75,6 +97,18 @@ def _peaks():
             d = json.load(f)
         return float(d.get("hbm_gbs", 6650.0)), "measured"
     return 6650.0, "fallback"
+
+
+def _int8_peak():
+    """Dense int8 tensor peak in TOP/s: the measured bf16 GEMM rate x 2 (the
+    nominal int8/bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return 2.0 * float(d["bf16_tflops"]), "measured bf16 x 2 (nominal int8/bf16 ratio)"
+    return 2.0 * 1590.0, "fallback bf16 x 2 (nominal int8/bf16 ratio)"
 
 
 def _kernel_hash() -> str:
@@ -157,12 +191,14 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def cpu_baseline(wl, t, max_seconds=20.0, max_queries=None):
+def cpu_baseline(wl, t, max_seconds=20.0, max_queries=None, min_seconds=0.0):
     """The oracle (one thread) on a bounded sample of the workload's queries:
     index + G-layer attention per query; only the oracle calls are timed, and
-    the result is scaled to queries/s. ``t`` may live on any device: each
-    query's keys and the K/V rows its oracle set names are copied to the host
-    before its timed calls."""
+    the result is scaled to queries/s. The queries are taken in order (and
+    again from the first, until at least `min_seconds` of oracle time) and
+    the sample stops once `max_seconds` are spent. ``t`` may live on any
+    device: each query's keys and the K/V rows its oracle set names are copied
+    to the host before its timed calls."""
     import numpy as np
 
     import oracle
@@ -173,31 +209,36 @@ def cpu_baseline(wl, t, max_seconds=20.0, max_queries=None):
     q_seq = t.q_seq.cpu().numpy()
     q_len = t.q_len.cpu().numpy()
     n = len(q_seq) if max_queries is None else min(max_queries, len(q_seq))
-    done, busy = 0, 0.0
-    for r in range(n):
-        base = int(kv_off[q_seq[r]])
-        L = int(q_len[r])
-        kseq = t.k_idx[base:base + L].cpu().numpy()
-        qi = t.q_idx[r].cpu().numpy()
-        wr = t.w[r].cpu().numpy()
-        c0 = time.perf_counter()
-        s = orc.index_query(qi, wr, kseq, L, wl.sink, wl.window, wl.topk, wl.hi_block, wl.hi_topblocks)
-        busy += time.perf_counter() - c0
-        valid = s[s >= 0]
-        local = np.full(s.shape[0], -1, np.int32)
-        local[: valid.shape[0]] = np.arange(valid.shape[0], dtype=np.int32)
-        rows = torch.as_tensor(valid.astype(np.int64) + base, device=t.k[0].device)
-        for g in range(len(t.q)):
-            kr, vr, qg = u16(t.k[g].index_select(0, rows)), u16(t.v[g].index_select(0, rows)), u16(t.q[g][r])
+    done, busy, passes = 0, 0.0, 0
+    while True:
+        for r in range(n):
+            base = int(kv_off[q_seq[r]])
+            L = int(q_len[r])
+            kseq = t.k_idx[base:base + L].cpu().numpy()
+            qi = t.q_idx[r].cpu().numpy()
+            wr = t.w[r].cpu().numpy()
             c0 = time.perf_counter()
-            orc.attend_query(qg, kr, vr, local)
+            s = orc.index_query(qi, wr, kseq, L, wl.sink, wl.window, wl.topk, wl.hi_block, wl.hi_topblocks)
             busy += time.perf_counter() - c0
-        done += 1
-        if busy > max_seconds:
+            valid = s[s >= 0]
+            local = np.full(s.shape[0], -1, np.int32)
+            local[: valid.shape[0]] = np.arange(valid.shape[0], dtype=np.int32)
+            rows = torch.as_tensor(valid.astype(np.int64) + base, device=t.k[0].device)
+            for g in range(len(t.q)):
+                kr, vr, qg = u16(t.k[g].index_select(0, rows)), u16(t.v[g].index_select(0, rows)), u16(t.q[g][r])
+                c0 = time.perf_counter()
+                orc.attend_query(qg, kr, vr, local)
+                busy += time.perf_counter() - c0
+            done += 1
+            if busy > max_seconds:
+                break
+        passes += 1
+        if busy > max_seconds or busy >= min_seconds or done == 0:
             break
     return {"value": done / busy, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{done} of {wl.n_q} queries of {wl.name} (index + {len(t.q)}-layer attention each), "
-                      f"single-threaded C oracle, {busy:.1f} s of oracle time"}
+            "sample": f"{done} query evaluations ({passes} pass(es) over {n} of the {wl.n_q} queries) of {wl.name} "
+                      f"(index + {len(t.q)}-layer attention each), single-threaded C oracle, {busy:.1f} s of "
+                      f"oracle time"}
 
 
 def run_reference(args, wl):
@@ -227,52 +268,17 @@ def run_reference(args, wl):
 
 
 # ---------------------------------------------------------------------------
-def main(argv=None):
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
-    ap.add_argument("--workload", default=wls.BATCH128K.name)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-seconds", type=float, default=8.0)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    args = ap.parse_args(argv)
-    args.warmup = max(3, args.warmup)
-    wl = wls.by_name(args.workload)
-    if args.impl == "reference":
-        return run_reference(args, wl)
-
-    from long_context_sparse_lsa_b200 import binding as lsa
+def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
+    """Draws the workload, captures its step graphs and times `steps` steps
+    (after `warmup`), each after an L2 flush: the whole step graph for the
+    headline, then the three calls one by one for the breakdown."""
     from long_context_sparse_lsa_b200.pipeline import LsaStep
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
-        pg = dist
-
-    # each rank draws its own independent batch (weak scaling)
-    wl_r = wls.small(wl, seed=wl.seed + 1000 * rank) if rank else wl
-    t = wls.make(wl_r, dev)
-    st = LsaStep(wl_r, t, dev)
+    t = wls.make(wl, dev)
+    st = LsaStep(wl, t, dev)
     st.build_block_sums()
     torch.cuda.synchronize()
-    stream = torch.cuda.current_stream(dev)
-
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-
     st.capture()
-    n_kernels = st.kernels_per_step()
 
     def one_step(evs):
         """The timed step: the captured step graph (block-sum update beside
@@ -293,40 +299,132 @@ def main(argv=None):
         st.replay("attend")
         evs[3].record(stream)
 
-    for _ in range(args.warmup):
-        one_step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
-        split_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    ev = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for _ in range(warmup):
+        one_step(ev(2))
+        split_step(ev(4))
     torch.cuda.synchronize()
     if st.status_bits() != 0:
-        raise RuntimeError(f"device status {st.status_bits():#x} after warm-up")
-
-    clocks = ClockSampler(local)
-    clocks.start()
+        raise RuntimeError(f"device status {st.status_bits():#x} after warm-up ({wl.name})")
+    if clocks is not None:
+        clocks.start()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for i in range(args.steps):
+    evs = [ev(2) for _ in range(steps)]
+    for i in range(steps):
         one_step(evs[i])
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    ms = sum(step_ms) / len(step_ms)
+    clk = clocks.stop() if clocks is not None else None
+    ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    # per-call breakdown (outside the timed region)
+    sevs = [ev(4) for _ in range(steps)]
+    for i in range(steps):
+        split_step(sevs[i])
+    torch.cuda.synchronize()
+    if st.status_bits() != 0:
+        raise RuntimeError(f"device status {st.status_bits():#x} after timing ({wl.name})")
+    return {"st": st, "t": t, "ms": ms, "clocks": clk, "n_kernels": st.kernels_per_step(),
+            "bs": [e[0].elapsed_time(e[1]) for e in sevs], "ix": [e[1].elapsed_time(e[2]) for e in sevs],
+            "at": [e[2].elapsed_time(e[3]) for e in sevs]}
+
+
+def secondary(dev, flush, stream, steps, warmup, peak):
+    """The 1M-token decode (G = 4) and the 8192-token prefill chunk, each
+    measured like the headline (step graph, L2 flush, CUDA events)."""
+    from long_context_sparse_lsa_b200 import binding as lsa
+
+    out = {}
+    mean = lambda xs: sum(xs) / len(xs)
+    for wl in (wls.CTX1M, wls.PREFILL):
+        run = time_workload(wl, dev, flush, stream, steps, warmup)
+        st = run["st"]
+        ms = run["ms"]
+        byts = step_bytes(wl)
+        ix, at = mean(run["ix"]), mean(run["at"])
+        rec = {"ms_per_step": ms, "steps": steps, "warmup": warmup,
+               "step_breakdown_ms": {"block_sums_update": mean(run["bs"]), "index": ix, "attend": at},
+               "algorithmic_bytes_per_step": byts,
+               "step_gbs": byts["total"] / (ms / 1000.0) / 1e9,
+               "step_frac_of_measured_hbm": byts["total"] / (ms / 1000.0) / 1e9 / peak,
+               "attend_gbs": byts["attend"] / (at / 1000.0) / 1e9,
+               "attend_frac_of_measured_hbm": byts["attend"] / (at / 1000.0) / 1e9 / peak,
+               "gpu_launches_per_step": run["n_kernels"]}
+        if wl.prefill_new:
+            ops = index_int8_ops(wl)
+            p8, kind8 = _int8_peak()
+            rec.update({"metric": "prefill tokens/s (index + attention of a causal chunk)", "unit": "tokens/s",
+                        "value": wl.n_q / (ms / 1000.0),
+                        "index_tensor_path": bool(lsa.lsa_index_uses_tensor_cores(st.batch, wl.H_I, wl.d_I,
+                                                                                  st.budget)),
+                        "index_int8_ops": ops,
+                        "index_tops": ops / (ix / 1000.0) / 1e12,
+                        "index_tops_frac_of_int8_peak": ops / (ix / 1000.0) / 1e12 / p8,
+                        "int8_peak_tops": p8, "int8_peak_kind": kind8,
+                        "note": "index_tops: int8 ops of the fine-score contraction over the whole index call "
+                                "(scoring + selection), so a lower bound on the tensor kernel's rate"})
+        else:
+            rec.update({"metric": "LSA decode queries/s at 1M ctx", "unit": "queries/s",
+                        "value": wl.n_q / (ms / 1000.0), "layers_per_index": wl.G})
+        out[wl.name] = rec
+        del run, st
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lsa", choices=["lsa", "reference"])
+    ap.add_argument("--workload", default=wls.BATCH128K.name)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the 1M decode and prefill chunk measurements")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    wl = wls.by_name(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # each rank draws its own independent batch (weak scaling)
+    wl_r = wls.small(wl, seed=wl.seed + 1000 * rank) if rank else wl
+    clocks = ClockSampler(local)
+    run = time_workload(wl_r, dev, flush, stream, args.steps, args.warmup, pg, clocks)
+    st, t = run["st"], run["t"]
+    ms = run["ms"]
     if pg:
         tt = torch.tensor([ms], device=dev)
         pg.all_reduce(tt, op=pg.ReduceOp.MAX)
         ms = float(tt.item())
-
-    # per-call breakdown (outside the timed region)
-    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        split_step(sevs[i])
-    torch.cuda.synchronize()
-    bs_ms = [e[0].elapsed_time(e[1]) for e in sevs]
-    ix_ms = [e[1].elapsed_time(e[2]) for e in sevs]
-    at_ms = [e[2].elapsed_time(e[3]) for e in sevs]
+    clk = run["clocks"]
+    bs_ms, ix_ms, at_ms = run["bs"], run["ix"], run["at"]
+    n_kernels = run["n_kernels"]
 
     # ---- end to end through the public API with host buffers ----
     pin = lambda x: x.cpu().pin_memory()
@@ -396,7 +494,13 @@ def main(argv=None):
             "gpu_launches": n_kernels * args.steps,
             "clocks": clk}
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, t, max_seconds=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(wl, t, max_seconds=args.cpu_seconds,
+                                            min_seconds=min(10.0, args.cpu_seconds))
+    if world == 1 and not args.no_secondary:
+        del st, t, run
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        line["secondary"] = secondary(dev, flush, stream, min(args.steps, 10), args.warmup, peak)
     if pg:
         pg.barrier()
         pg.destroy_process_group()

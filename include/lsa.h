@@ -153,6 +153,16 @@ lsa_status_t lsa_hi_block_sums(const int8_t *k_idx_cache, int32_t d_I,
 size_t lsa_index_workspace_size(const lsa_batch_t *batch, int32_t H_I,
                                 int32_t d_I, lsa_budget_t budget);
 
+/* 1 when lsa_index would score this batch's fine candidates as one dense
+ * int8 contraction on the tcgen05 tensor cores, else 0 (reads only host
+ * fields). That path serves a prefill chunk: HI off, every row in one
+ * sequence (n_seq == 1), at least 64 rows, H_I == 16, d_I == 128; other
+ * batches are scored per row. Both paths give bit-identical index sets. The
+ * pages define the score, not how to evaluate it; this call only reports the
+ * evaluation strategy. */
+int32_t lsa_index_uses_tensor_cores(const lsa_batch_t *batch, int32_t H_I,
+                                    int32_t d_I, lsa_budget_t budget);
+
 /* One index set per query row (CLI: call once per group of layers and pass
  * the result to lsa_attend with layers_per_index = G).
  *

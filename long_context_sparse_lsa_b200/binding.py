@@ -118,6 +118,8 @@ def load_library():
     lib.lsa_hi_block_sums.argtypes = [vp, i32, i32, ctypes.POINTER(_Batch), i32, vp, i64, vp, vp]
     lib.lsa_index_workspace_size.restype = sz
     lib.lsa_index_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
+    lib.lsa_index_uses_tensor_cores.restype = i32
+    lib.lsa_index_uses_tensor_cores.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
     lib.lsa_index.restype = i32
     lib.lsa_index.argtypes = [vp, vp, vp, i32, i32, i32, ctypes.POINTER(_Batch), _Budget, vp, i64, vp, vp, sz, vp, vp]
     lib.lsa_attend_workspace_size.restype = sz
@@ -166,6 +168,12 @@ def lsa_hi_block_sums(k_idx: torch.Tensor, hi_block: int, batch: Batch, block_su
 def lsa_index_workspace_size(batch: Batch, H_I: int, d_I: int, budget: Budget) -> int:
     cb = batch.c()
     return int(load_library().lsa_index_workspace_size(ctypes.byref(cb), H_I, d_I, budget.c()))
+
+
+def lsa_index_uses_tensor_cores(batch: Batch, H_I: int, d_I: int, budget: Budget) -> bool:
+    """True when lsa_index scores this batch as one dense tcgen05 contraction."""
+    cb = batch.c()
+    return bool(load_library().lsa_index_uses_tensor_cores(ctypes.byref(cb), H_I, d_I, budget.c()))
 
 
 def lsa_index(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, w_max: int, batch: Batch,

@@ -124,6 +124,20 @@ size_t lsa_index_workspace_size(const lsa_batch_t* batch, int32_t H_I, int32_t d
     return lsa::plan_index(batch->n_q, batch->max_len, budget).ws_bytes;
 }
 
+// Rows from which a chunk of one sequence is scored as a dense contraction.
+constexpr int32_t kDenseMinRows = 64;
+
+static bool index_dense(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, const lsa_budget_t& budget) {
+    return budget.hi_block == 0 && batch->n_q >= kDenseMinRows &&
+           lsa::prefill_tc_supported(H_I, d_I, batch->n_seq, batch->total_tokens);
+}
+
+int32_t lsa_index_uses_tensor_cores(const lsa_batch_t* batch, int32_t H_I, int32_t d_I,
+                                               lsa_budget_t budget) {
+    if (batch == nullptr || !budget_ok(budget)) return 0;
+    return index_dense(batch, H_I, d_I, budget) ? 1 : 0;
+}
+
 static lsa_status_t index_validate(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max,
                                    int32_t H_I, int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget,
                                    const int8_t* block_sums, int64_t block_rows, const int32_t* index_sets) {
@@ -203,7 +217,12 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
         e = lsa::launch_index_scores(a, d_I, true, cs);
         if (e == cudaSuccess) e = lsa::launch_index_select(a, true, plan.cluster, plan.smem_blocks, cs);
     }
-    if (e == cudaSuccess) e = lsa::launch_index_scores(a, d_I, false, cs);
+    if (e == cudaSuccess) {
+        // a prefill chunk (many rows of one sequence, HI off) is one dense
+        // contraction: tensor-core path; otherwise per-row streaming scores
+        e = index_dense(batch, H_I, d_I, budget) ? lsa::launch_fine_scores_tc(a, cs)
+                                                  : lsa::launch_index_scores(a, d_I, false, cs);
+    }
     if (e == cudaSuccess) e = lsa::launch_index_select(a, false, plan.cluster, plan.smem_tokens, cs);
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }

@@ -26,6 +26,7 @@ __device__ __forceinline__ int sbyte(uint32_t w, int i) { return static_cast<int
 // of coalesced 16-byte loads (one round for hi_block <= 32 at d_I = 128).
 template <int D_I>
 __global__ void __launch_bounds__(kBsThreads) block_sums_kernel(const BlockSumArgs a) {
+    pdl_enter();
     constexpr int kCPR = D_I / 16;           // 16-byte chunks per row
     constexpr int kRPP = kBsThreads / kCPR;  // rows per pass
     __shared__ int s_part[kBsWarps][D_I];
@@ -92,12 +93,11 @@ __global__ void __launch_bounds__(kBsThreads) block_sums_kernel(const BlockSumAr
 cudaError_t launch_block_sums(const BlockSumArgs& a, int d_I, cudaStream_t stream) {
     dim3 grid((unsigned)a.blocks_per_seq, (unsigned)a.n_seq);
     switch (d_I) {
-        case 32: block_sums_kernel<32><<<grid, kBsThreads, 0, stream>>>(a); break;
-        case 64: block_sums_kernel<64><<<grid, kBsThreads, 0, stream>>>(a); break;
-        case 128: block_sums_kernel<128><<<grid, kBsThreads, 0, stream>>>(a); break;
+        case 32: return launch_pdl(block_sums_kernel<32>, grid, dim3(kBsThreads), 0, stream, 0, a);
+        case 64: return launch_pdl(block_sums_kernel<64>, grid, dim3(kBsThreads), 0, stream, 0, a);
+        case 128: return launch_pdl(block_sums_kernel<128>, grid, dim3(kBsThreads), 0, stream, 0, a);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace lsa

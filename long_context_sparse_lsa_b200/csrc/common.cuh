@@ -16,6 +16,15 @@ namespace lsa {
 constexpr int kWarp = 32;
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// Programmatic dependent launch: every kernel of the path is launched with
+// programmatic stream serialisation and waits for the grids it depends on
+// (and their memory) before its first global access; the next kernel may be
+// launched as this grid's CTAs exit. (Triggering the next launch at kernel
+// entry measured slower: the early dependents took SM space from the running
+// grid.)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() { pdl_wait(); }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
 __device__ __forceinline__ void flag(int32_t* status, int32_t bits) {

@@ -42,6 +42,7 @@ __device__ __forceinline__ bool row_ok(const IndexArgs& a, int r, int64_t& off, 
 
 template <int D_I, int NT>
 __global__ void __launch_bounds__(kScThreads) coarse_score_kernel(const __grid_constant__ IndexArgs a) {
+    pdl_enter();
     const int r = blockIdx.y;
     int64_t off;
     int L;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(kScThreads) coarse_score_kernel(const __grid_c
 
 template <int D_I, int NT>
 __global__ void __launch_bounds__(kScThreads) fine_score_kernel(const __grid_constant__ IndexArgs a) {
+    pdl_enter();
     const int r = blockIdx.y;
     int64_t off;
     int L;
@@ -135,12 +137,11 @@ template <int D_I, int NT>
 cudaError_t launch_scores_t(const IndexArgs& a, bool coarse, cudaStream_t st) {
     if (coarse) {
         dim3 grid((unsigned)((a.coarse_cap + kCoarseChunk - 1) / kCoarseChunk), (unsigned)a.n_q);
-        coarse_score_kernel<D_I, NT><<<grid, kScThreads, 0, st>>>(a);
+        return launch_pdl(coarse_score_kernel<D_I, NT>, grid, dim3(kScThreads), 0, st, 0, a);
     } else {
         dim3 grid((unsigned)((a.fine_cap + kFineChunk - 1) / kFineChunk), (unsigned)a.n_q);
-        fine_score_kernel<D_I, NT><<<grid, kScThreads, 0, st>>>(a);
+        return launch_pdl(fine_score_kernel<D_I, NT>, grid, dim3(kScThreads), 0, st, 0, a);
     }
-    return cudaGetLastError();
 }
 
 template <int D_I>

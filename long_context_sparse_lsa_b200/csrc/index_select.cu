@@ -359,12 +359,54 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, K* 
 // Kept keys (key > thresh, plus the first `quota` keys == thresh of the row
 // in position order) of this CTA's slice; emit(slot, rank) with slot relative
 // to the slice and rank the key's position among the row's kept keys.
+// This slice's counts of keys > thresh and == thresh without reading its keys:
+// the slice histogram's bins above `bin` hold only keys > thresh; bin `bin`
+// holds only keys == thresh (exact bins), or its keys are the slice's own
+// candidates `mine` (from_mine). Returns the counts in every thread.
+template <typename K>
+__device__ void slice_counts(SelShared& sh, uint32_t bin, bool from_mine, const K* mine, K thresh, uint32_t& ng,
+                             uint32_t& ne) {
+    const int lane = lane_id(), wid = warp_id();
+    uint32_t g = 0, e = 0;
+#pragma unroll
+    for (int j = 0; j < kBinsPerThread; ++j) {
+        const uint32_t b = threadIdx.x + (uint32_t)(j * kSelThreads);
+        const uint32_t v = sh.local_hist[b];
+        if (b > bin) g += v;
+        else if (b == bin && !from_mine) e += v;
+    }
+    if (from_mine) {
+        const uint32_t mc = min(sh.local_count, (uint32_t)kCandCap);
+        for (uint32_t i = threadIdx.x; i < mc; i += kSelThreads) {
+            const K key = mine[i];
+            g += key > thresh ? 1u : 0u;
+            e += key == thresh ? 1u : 0u;
+        }
+    }
+    g = warp_sum(g);
+    e = warp_sum(e);
+    if (lane == 0) {
+        sh.wsum[wid] = g;
+        sh.wsum2[wid] = e;
+    }
+    __syncthreads();
+    ng = 0;
+    ne = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+        ng += sh.wsum[w];
+        ne += sh.wsum2[w];
+    }
+    __syncthreads();  // the warp sums are rewritten by the compaction
+}
+
+// With `counted`, (ng, ne) are this slice's counts of keys > thresh and ==
+// thresh (slice_counts); otherwise a pass over the slice counts them.
 template <typename K, typename Emit>
 __device__ void cluster_compact(SelShared& sh, const Keys<K>& keys, int m, uint32_t C, uint32_t c, K thresh,
-                                uint32_t quota, Emit emit) {
+                                uint32_t quota, bool counted, uint32_t ng_in, uint32_t ne_in, Emit emit) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
     // 1. this slice's counts, published to every CTA
-    const int nw_all = (m + 31) / 32;
+    const int nw_all = counted ? 0 : (m + 31) / 32;
     uint32_t ng = 0, ne = 0;
     for (int w0 = wid; w0 < nw_all; w0 += kSelWarps * kUnroll) {
         K kv[kUnroll];
@@ -380,16 +422,22 @@ __device__ void cluster_compact(SelShared& sh, const Keys<K>& keys, int m, uint3
             ne += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] == thresh));
         }
     }
-    if (lane == 0) {
-        sh.wsum[wid] = ng;
-        sh.wsum2[wid] = ne;
+    if (!counted) {
+        if (lane == 0) {
+            sh.wsum[wid] = ng;
+            sh.wsum2[wid] = ne;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     if (tid < (int)C) {
-        uint32_t tg = 0, te = 0;
-        for (int w = 0; w < kSelWarps; ++w) {
-            tg += sh.wsum[w];
-            te += sh.wsum2[w];
+        uint32_t tg = ng_in, te = ne_in;
+        if (!counted) {
+            tg = 0;
+            te = 0;
+            for (int w = 0; w < kSelWarps; ++w) {
+                tg += sh.wsum[w];
+                te += sh.wsum2[w];
+            }
         }
         st_cluster(map_cta(smem_u32(&sh.cta_gt[c]), (uint32_t)tid), tg);
         st_cluster(map_cta(smem_u32(&sh.cta_eq[c]), (uint32_t)tid), te);
@@ -492,6 +540,7 @@ __device__ __forceinline__ void slice_of(int n, uint32_t C, uint32_t c, int& k_l
 // assembly of the index set; otherwise the HI block top-k.
 template <typename K, bool kTokens>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_constant__ IndexArgs a) {
+    pdl_enter();
     extern __shared__ __align__(16) uint8_t dyn[];
     SelShared& sh = *reinterpret_cast<SelShared*>(dyn);
     const int r = blockIdx.y;
@@ -559,9 +608,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
         K thr = K(1);
         uint32_t quota = 0xffffffffu;  // k == total: every candidate is kept
         if (k < total) resolve_threshold<K>(sh, keys, m, cand, mine, C, k, tb, above, in_bin, thr, quota);
+        // this slice's kept counts from its histogram (and candidates), unless
+        // the threshold bin was refined over the slices
+        const bool list = k < total && tb >= 64u && in_bin <= (uint32_t)kCandCap;
+        const bool counted = k == total || tb < 64u || list;
+        uint32_t ng = 0, ne = 0;
+        if (counted) slice_counts<K>(sh, k == total ? 1u : tb, list, mine, thr, ng, ne);
         if (kTokens) {
             const int lgB = (B > 0 && (B & (B - 1)) == 0) ? __ffs(B) - 1 : -1;  // power-of-two block: shift
-            cluster_compact<K>(sh, keys, m, C, c, thr, quota, [&](int slot, uint32_t rank) {
+            cluster_compact<K>(sh, keys, m, C, c, thr, quota, counted, ng, ne, [&](int slot, uint32_t rank) {
                 const int gs = k_lo + slot;
                 int tok;
                 if (B > 0) {
@@ -574,7 +629,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
             });
         } else {
             int32_t* kept = a.kept + (int64_t)r * a.hi_topblocks;
-            cluster_compact<K>(sh, keys, m, C, c, thr, quota, [&](int slot, uint32_t rank) {
+            cluster_compact<K>(sh, keys, m, C, c, thr, quota, counted, ng, ne, [&](int slot, uint32_t rank) {
                 if (rank < k) kept[rank] = first + k_lo + slot;
             });
         }
@@ -646,19 +701,7 @@ static cudaError_t launch_cluster(Kern kern, const IndexArgs& a, int cluster, si
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)cluster, (unsigned)a.n_q, 1);
-    cfg.blockDim = dim3(kSelThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    return launch_pdl(kern, dim3((unsigned)cluster, (unsigned)a.n_q, 1), dim3(kSelThreads), smem, stream, cluster, a);
 }
 
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream) {

@@ -82,6 +82,10 @@ struct IndexPlan {
 };
 IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b);
 cudaError_t launch_index_scores(const IndexArgs& a, int d_I, bool coarse, cudaStream_t stream);
+// Fine scores of a causal chunk of rows of one sequence (HI off) on the
+// tcgen05 tensor cores; same keys as launch_index_scores(coarse = false).
+bool prefill_tc_supported(int H_I, int d_I, int n_seq, int64_t total_tokens);
+cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream);
 
 // ---- sparse attention -----------------------------------------------------
@@ -117,5 +121,32 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
 cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
 
 int device_sm_count();
+
+// Launches `kernel` with programmatic stream serialisation (the kernel calls
+// pdl_enter() first) and, when cluster > 0, that cluster size along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       int cluster, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
 
 }  // namespace lsa

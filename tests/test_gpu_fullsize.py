@@ -21,6 +21,7 @@ import pytest
 import torch
 
 import parity
+from long_context_sparse_lsa_b200 import binding as lsa
 from long_context_sparse_lsa_b200 import workloads as wls
 from long_context_sparse_lsa_b200.pipeline import LsaStep
 
@@ -86,6 +87,7 @@ def test_ragged_batch_sample():
 def test_prefill_chunk_sample():
     wl = wls.PREFILL
     st, t = _run_graph(wl)
+    assert lsa.lsa_index_uses_tensor_cores(st.batch, wl.H_I, wl.d_I, st.budget)
     n = wl.n_q
     rows = [0, 1, 2047, 4096, 6000, n - 2, n - 1]
     _check(wl, st, t, rows)

@@ -94,9 +94,34 @@ def test_small_cases(name):
 
 
 def test_prefill_rows_through_decode_kernel():
-    """Many rows of one sequence with causal visible lengths (a prefill chunk)."""
-    wl = wls.small(wls.PREFILL, name="prefill_small", lens=(3000 + 200,), prefill_new=200, seed=7)
-    run_case(wl)
+    """Rows of one sequence with causal visible lengths, too few for the dense
+    path: scored row by row."""
+    wl = wls.small(wls.PREFILL, name="prefill_small", lens=(3000 + 40,), prefill_new=40, seed=7)
+    st, _ = run_case(wl)
+    assert not lsa.lsa_index_uses_tensor_cores(st.batch, wl.H_I, wl.d_I, st.budget)
+
+
+# Prefill chunks of one sequence (HI off, 64 rows or more): the fine scores
+# come from the tensor-core contraction. Row counts that leave a partial
+# 16-row tile, caches that are not a whole number of 128-token tiles, rows
+# whose middle is empty or shorter than the sink, and a second sequence
+# (which sends the chunk back to the per-row kernel).
+PREFILL_CASES = {
+    "tc_ragged_rows": dict(lens=(5000 + 77,), prefill_new=77),
+    "tc_short_cache": dict(lens=(40 + 300,), prefill_new=300, sink=16, window=64, topk=100),
+    "tc_wide_window": dict(lens=(1500 + 130,), prefill_new=130, sink=64, window=1400, topk=50),
+    "tc_full_range": dict(lens=(3000 + 96,), prefill_new=96, qk_lo=-128, qk_hi=127, w_hi=4, topk=500),
+    "tc_ties": dict(lens=(4000 + 64,), prefill_new=64, qk_lo=-1, qk_hi=1, w_hi=1, topk=700),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PREFILL_CASES))
+def test_prefill_chunks_tensor_core_scores(name):
+    kw = dict(PREFILL_CASES[name])
+    kw.setdefault("seed", 300 + sorted(PREFILL_CASES).index(name))
+    wl = wls.small(wls.PREFILL, name=name, **kw)
+    st, _ = run_case(wl)
+    assert lsa.lsa_index_uses_tensor_cores(st.batch, wl.H_I, wl.d_I, st.budget)
 
 
 def test_dense_equivalence_matches_textbook_attention():
