@@ -78,6 +78,158 @@ __device__ __forceinline__ uint32_t word(const uint4& x, int j) {
     return j == 0 ? x.x : (j == 1 ? x.y : (j == 2 ? x.z : x.w));
 }
 
+// Online softmax of one 16-token tile's scores (sacc: S^T fragments, tokens g
+// and g+8 of this lane, masked where ok_g / ok_g8 is false) and O^T += V^T P^T
+// from the tile's V registers.
+template <int NT>
+__device__ __forceinline__ void softmax_pv(const float (&sacc)[NT][4], bool ok_g, bool ok_g8, float scale_log2,
+                                           float (&m_run)[NT][2], float (&l_run)[NT][2], float (&o)[NT][kD / 16][4],
+                                           const VTile& v) {
+    uint32_t phi[NT][2], plo[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float z0 = ok_g ? sacc[n][0] * scale_log2 : -INFINITY;   // (tok g,   head 2t)
+        const float z1 = ok_g ? sacc[n][1] * scale_log2 : -INFINITY;   // (tok g,   head 2t+1)
+        const float z2 = ok_g8 ? sacc[n][2] * scale_log2 : -INFINITY;  // (tok g+8, head 2t)
+        const float z3 = ok_g8 ? sacc[n][3] * scale_log2 : -INFINITY;  // (tok g+8, head 2t+1)
+        float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+#pragma unroll
+        for (int msk = 4; msk < 32; msk <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
+        }
+        const float mn0 = fmaxf(m_run[n][0], mx0), mn1 = fmaxf(m_run[n][1], mx1);
+        const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = exp2f(m_run[n][0] - base0), al1 = exp2f(m_run[n][1] - base1);
+        const float p0 = exp2f(z0 - base0), p1 = exp2f(z1 - base1);
+        const float p2 = exp2f(z2 - base0), p3 = exp2f(z3 - base1);
+        // the running max rarely moves after the first tiles: rescale o
+        // only when it did for some head of this warp
+        const bool moved = __any_sync(0xffffffffu, mn0 != m_run[n][0] || mn1 != m_run[n][1]);
+        m_run[n][0] = mn0;
+        m_run[n][1] = mn1;
+        l_run[n][0] = l_run[n][0] * al0 + p0 + p2;
+        l_run[n][1] = l_run[n][1] * al1 + p1 + p3;
+        if (moved) {
+#pragma unroll
+            for (int mt = 0; mt < kD / 16; ++mt) {
+                o[n][mt][0] *= al0;
+                o[n][mt][1] *= al1;
+                o[n][mt][2] *= al0;
+                o[n][mt][3] *= al1;
+            }
+        }
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
+        const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
+        const float2 fh01 = __bfloat1622float2(h01), fh23 = __bfloat1622float2(h23);
+        phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+        phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+        plo[n][0] = movmatrix_trans(pack_bf16(p0 - fh01.x, p1 - fh01.y));
+        plo[n][1] = movmatrix_trans(pack_bf16(p2 - fh23.x, p3 - fh23.y));
+    }
+    // O^T += V^T P^T from the registers of this tile's V
+#pragma unroll
+    for (int mt = 0; mt < kD / 16; ++mt) {
+        const int c = mt >> 2, j = mt & 3;
+        const uint32_t w0 = word(v.r[0][c], j), w1 = word(v.r[1][c], j);
+        const uint32_t w8 = word(v.r[2][c], j), w9 = word(v.r[3][c], j);
+        const uint32_t vfr[4] = {__byte_perm(w0, w1, 0x5410), __byte_perm(w0, w1, 0x7632),
+                                 __byte_perm(w8, w9, 0x5410), __byte_perm(w8, w9, 0x7632)};
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            mma_bf16(o[n][mt], vfr, phi[n][0], phi[n][1]);
+            mma_bf16(o[n][mt], vfr, plo[n][0], plo[n][1]);
+        }
+    }
+}
+
+// Merges the consumer warps of each kv head (in registers: warps with
+// wsel > 0 park their fragments in `merge_area`, lane-major, and the wsel == 0
+// warp folds them in with the log-sum-exp rule), then writes the head's query
+// heads: the final output when there is one split, else one partial. Every
+// thread of the CTA calls it (it holds a CTA barrier); warps >= kConsumers
+// only take part in the barrier.
+template <int NT>
+__device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* merge_area, float (&o)[NT][kD / 16][4],
+                                                float (&m_run)[NT][2], float (&l_run)[NT][2], int warp, int lane,
+                                                int hpc, int hgrp, int r, int layer, int split, int ratio) {
+    const int g = lane >> 2, t4 = lane & 3;
+    // ---- merge the consumers of each kv head, in registers ----
+    // All warps hold O^T in the same fragment layout, so warps with wsel > 0
+    // park theirs in shared memory (lane-major: conflict free) and the wsel ==
+    // 0 warp of the head folds them in with the log-sum-exp rule.
+    constexpr int kRegs = NT * (kD / 16) * 4;
+    float* xo = reinterpret_cast<float*>(merge_area);  // [kConsumers][kRegs][32]
+    float* xml = xo + kConsumers * kRegs * kWarp;              // [kConsumers][NT*4][32]
+    const int wsel_me = warp / hpc;
+    if (warp < kConsumers && wsel_me > 0) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int mt = 0; mt < kD / 16; ++mt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) xo[(warp * kRegs + (n * (kD / 16) + mt) * 4 + c) * kWarp + lane] = o[n][mt][c];
+            xml[(warp * NT * 4 + n * 4 + 0) * kWarp + lane] = m_run[n][0];
+            xml[(warp * NT * 4 + n * 4 + 1) * kWarp + lane] = m_run[n][1];
+            xml[(warp * NT * 4 + n * 4 + 2) * kWarp + lane] = l_run[n][0];
+            xml[(warp * NT * 4 + n * 4 + 3) * kWarp + lane] = l_run[n][1];
+        }
+    }
+    __syncthreads();
+    const bool direct = a.n_splits == 1;
+    const int64_t row_q = (int64_t)layer * a.n_q + r;
+    if (warp < kConsumers && wsel_me == 0) {
+        const int h_local = warp % hpc;
+        const int n_sel = kConsumers / hpc;
+        for (int j = 1; j < n_sel; ++j) {
+            const int w = h_local + hpc * j;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const float mb = xml[(w * NT * 4 + n * 4 + c) * kWarp + lane];
+                    const float lb = xml[(w * NT * 4 + n * 4 + 2 + c) * kWarp + lane];
+                    const float M = fmaxf(m_run[n][c], mb);
+                    const float sa = M == -INFINITY ? 0.f : exp2f(m_run[n][c] - M);
+                    const float sb = M == -INFINITY ? 0.f : exp2f(mb - M);
+                    m_run[n][c] = M;
+                    l_run[n][c] = l_run[n][c] * sa + lb * sb;
+#pragma unroll
+                    for (int mt = 0; mt < kD / 16; ++mt) {
+                        o[n][mt][c] = o[n][mt][c] * sa + xo[(w * kRegs + (n * (kD / 16) + mt) * 4 + c) * kWarp + lane] * sb;
+                        o[n][mt][c + 2] =
+                            o[n][mt][c + 2] * sa + xo[(w * kRegs + (n * (kD / 16) + mt) * 4 + c + 2) * kWarp + lane] * sb;
+                    }
+                }
+            }
+        }
+        // write this kv head's query heads: the final output, or one split partial
+        const int kvh = hgrp * hpc + h_local;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int hh = 8 * n + 2 * t4 + c;
+                if (hh >= ratio) continue;
+                const int64_t qh = (int64_t)kvh * ratio + hh;
+                const float inv = l_run[n][c] > 0.f ? 1.f / l_run[n][c] : 0.f;
+                float* dst = direct ? a.out[layer] + ((int64_t)r * a.H_q + qh) * kD
+                                    : a.part_o + ((row_q * a.n_splits + split) * a.H_q + qh) * kD;
+                const float sc = direct ? inv : 1.f;
+#pragma unroll
+                for (int mt = 0; mt < kD / 16; ++mt) {
+                    const int d0 = 8 * ((mt >> 2) ? 8 + g : g) + 2 * (mt & 3);
+                    *reinterpret_cast<float2*>(dst + d0) = make_float2(o[n][mt][c] * sc, o[n][mt][c + 2] * sc);
+                }
+                if (!direct && g == 0)
+                    *reinterpret_cast<float2*>(a.part_ml + ((row_q * a.n_splits + split) * a.H_q + qh) * 2) =
+                        make_float2(m_run[n][c], l_run[n][c]);
+            }
+        }
+    }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kAtThreads, 1) attend_kernel(const __grid_constant__ AttendArgs a) {
     pdl_enter();
@@ -246,63 +398,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_kernel(const __grid_cons
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty_bar(s));  // K of this stage is no longer read
-            uint32_t phi[NT][2], plo[NT][2];
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const float z0 = ok_g ? sacc[n][0] * a.scale_log2 : -INFINITY;   // (tok g,   head 2t)
-                const float z1 = ok_g ? sacc[n][1] * a.scale_log2 : -INFINITY;   // (tok g,   head 2t+1)
-                const float z2 = ok_g8 ? sacc[n][2] * a.scale_log2 : -INFINITY;  // (tok g+8, head 2t)
-                const float z3 = ok_g8 ? sacc[n][3] * a.scale_log2 : -INFINITY;  // (tok g+8, head 2t+1)
-                float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
-#pragma unroll
-                for (int msk = 4; msk < 32; msk <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, msk));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, msk));
-                }
-                const float mn0 = fmaxf(m_run[n][0], mx0), mn1 = fmaxf(m_run[n][1], mx1);
-                const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-                const float base1 = mn1 == -INFINITY ? 0.f : mn1;
-                const float al0 = exp2f(m_run[n][0] - base0), al1 = exp2f(m_run[n][1] - base1);
-                const float p0 = exp2f(z0 - base0), p1 = exp2f(z1 - base1);
-                const float p2 = exp2f(z2 - base0), p3 = exp2f(z3 - base1);
-                // the running max rarely moves after the first tiles: rescale o
-                // only when it did for some head of this warp
-                const bool moved = __any_sync(0xffffffffu, mn0 != m_run[n][0] || mn1 != m_run[n][1]);
-                m_run[n][0] = mn0;
-                m_run[n][1] = mn1;
-                l_run[n][0] = l_run[n][0] * al0 + p0 + p2;
-                l_run[n][1] = l_run[n][1] * al1 + p1 + p3;
-                if (moved) {
-#pragma unroll
-                    for (int mt = 0; mt < kD / 16; ++mt) {
-                        o[n][mt][0] *= al0;
-                        o[n][mt][1] *= al1;
-                        o[n][mt][2] *= al0;
-                        o[n][mt][3] *= al1;
-                    }
-                }
-                const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
-                const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
-                const float2 fh01 = __bfloat1622float2(h01), fh23 = __bfloat1622float2(h23);
-                phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
-                phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-                plo[n][0] = movmatrix_trans(pack_bf16(p0 - fh01.x, p1 - fh01.y));
-                plo[n][1] = movmatrix_trans(pack_bf16(p2 - fh23.x, p3 - fh23.y));
-            }
-            // O^T += V^T P^T from the registers of this tile's V
-#pragma unroll
-            for (int mt = 0; mt < kD / 16; ++mt) {
-                const int c = mt >> 2, j = mt & 3;
-                const uint32_t w0 = word(v.r[0][c], j), w1 = word(v.r[1][c], j);
-                const uint32_t w8 = word(v.r[2][c], j), w9 = word(v.r[3][c], j);
-                const uint32_t vfr[4] = {__byte_perm(w0, w1, 0x5410), __byte_perm(w0, w1, 0x7632),
-                                         __byte_perm(w8, w9, 0x5410), __byte_perm(w8, w9, 0x7632)};
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    mma_bf16(o[n][mt], vfr, phi[n][0], phi[n][1]);
-                    mma_bf16(o[n][mt], vfr, plo[n][0], plo[n][1]);
-                }
-            }
+            softmax_pv<NT>(sacc, ok_g, ok_g8, a.scale_log2, m_run, l_run, o, v);
             // V two tiles ahead, in flight during the next tile's K wait and math
             if (i + 2 * n_sel < n_tiles) load_vtile(v, vbase, tok_stride, s_ent + (i + 2 * n_sel) * kTile, g, t4);
                     return true;
@@ -331,79 +427,157 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_kernel(const __grid_cons
         return;
     }
 
-    // ---- merge the consumers of each kv head, in registers ----
-    // All warps hold O^T in the same fragment layout, so warps with wsel > 0
-    // park theirs in shared memory (lane-major: conflict free) and the wsel ==
-    // 0 warp of the head folds them in with the log-sum-exp rule.
-    constexpr int kRegs = NT * (kD / 16) * 4;
-    float* xo = reinterpret_cast<float*>(smem + a.stage_off);  // [kConsumers][kRegs][32]
-    float* xml = xo + kConsumers * kRegs * kWarp;              // [kConsumers][NT*4][32]
-    const int wsel_me = warp / hpc;
-    if (warp < kConsumers && wsel_me > 0) {
+    merge_and_store<NT>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, hpc, hgrp, r, layer, split, ratio);
+}
+
+// K rows of one 16-token tile for one kv head, in the registers of lane
+// (g, t): tokens g and g+8 (index rr), 16-byte chunks t, t+4, t+8, t+12 of
+// the 256-byte row (index j). The QK^T contraction runs over the head dims in
+// the matching permuted order: MMA k-step ks takes chunk ks/2, words
+// 2*(ks&1) (k = 2t, 2t+1) and 2*(ks&1)+1 (k = 2t+8, 2t+9); the query
+// fragments are read in the same order, so the dot products are unchanged.
+struct KTile {
+    uint4 r[2][4];
+};
+
+__device__ __forceinline__ void load_ktile(KTile& k, const uint16_t* kbase, int64_t tok_stride, const int32_t* ent,
+                                           int g, int t4) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
+    for (int rr = 0; rr < 2; ++rr) {
+        const int e = ent[g + 8 * rr];
+        if (e >= 0) {
+            const uint16_t* p = kbase + (int64_t)e * tok_stride + 8 * t4;
 #pragma unroll
-            for (int mt = 0; mt < kD / 16; ++mt)
+            for (int j = 0; j < 4; ++j) k.r[rr][j] = ldg16(p + 32 * j);
+        } else {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) xo[(warp * kRegs + (n * (kD / 16) + mt) * 4 + c) * kWarp + lane] = o[n][mt][c];
-            xml[(warp * NT * 4 + n * 4 + 0) * kWarp + lane] = m_run[n][0];
-            xml[(warp * NT * 4 + n * 4 + 1) * kWarp + lane] = m_run[n][1];
-            xml[(warp * NT * 4 + n * 4 + 2) * kWarp + lane] = l_run[n][0];
-            xml[(warp * NT * 4 + n * 4 + 3) * kWarp + lane] = l_run[n][1];
+            for (int j = 0; j < 4; ++j) k.r[rr][j] = make_uint4(0, 0, 0, 0);
         }
+    }
+}
+
+// The register-streaming variant (GQA groups of at most 8 query heads): every
+// warp gathers its own K and V rows with 16-byte loads straight into MMA
+// fragments, two tiles ahead of use, so no copy engine, shared-memory ring or
+// producer warp sits between HBM and the tensor cores. Eight warps per CTA;
+// warp w owns kv head w % hpc of the CTA and every (8/hpc)-th tile.
+__global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const __grid_constant__ AttendArgs a) {
+    constexpr int NT = 1;
+    pdl_enter();
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+    const int g = lane >> 2, t4 = lane & 3;
+    const int split = blockIdx.x / a.head_groups;
+    const int hgrp = blockIdx.x % a.head_groups;
+    const int r = blockIdx.y;
+    const int layer = blockIdx.z;
+    const int ratio = a.H_q / a.H_kv;
+    const int hpc = a.hpc;
+    const int q_heads_cta = hpc * ratio;
+
+    const int seq = a.q_seq[r];
+    const int L = a.q_len[r];
+    bool bad = seq < 0 || seq >= a.n_seq;
+    int64_t off = 0;
+    if (!bad) {
+        off = a.kv_offset[seq];
+        const int slen = a.seq_lens[seq];
+        bad = L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens;
+    }
+    if (bad) {
+        if (tid == 0 && blockIdx.x == 0 && layer == 0)
+            flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
+        if (split == 0) {
+            float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)hgrp * q_heads_cta) * kD;
+            for (int i = tid; i < q_heads_cta * kD; i += kConsumers * kWarp) orow[i] = 0.f;
+        }
+        return;
+    }
+    const int n_entries = min(L, a.budget);
+    const int e0 = split * a.entries_per_split;
+    const int n_local = max(0, min(n_entries - e0, a.entries_per_split));
+    const int n_tiles = (n_local + kTile - 1) / kTile;
+    const int32_t* set = a.sets + (int64_t)r * a.budget + e0;
+    int32_t* s_ent = reinterpret_cast<int32_t*>(smem);
+    for (int i = tid; i < n_tiles * kTile; i += kConsumers * kWarp) {
+        int v = -1;
+        if (i < n_local) {
+            v = set[i];
+            if (v < -1 || v >= L) {
+                flag(a.dev_status, LSA_DEV_BAD_INDEX);
+                v = -1;
+            }
+        }
+        s_ent[i] = v;
     }
     __syncthreads();
-    const bool direct = a.n_splits == 1;
-    const int64_t row_q = (int64_t)layer * a.n_q + r;
-    if (warp < kConsumers && wsel_me == 0) {
-        const int h_local = warp % hpc;
-        const int n_sel = kConsumers / hpc;
-        for (int j = 1; j < n_sel; ++j) {
-            const int w = h_local + hpc * j;
+
+    float o[NT][kD / 16][4];
+    float m_run[NT][2], l_run[NT][2];
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
+    for (int mt = 0; mt < kD / 16; ++mt) o[0][mt][0] = o[0][mt][1] = o[0][mt][2] = o[0][mt][3] = 0.f;
+    m_run[0][0] = m_run[0][1] = -INFINITY;
+    l_run[0][0] = l_run[0][1] = 0.f;
+
+    const int h_local = warp % hpc;
+    const int wsel = warp / hpc;
+    const int n_sel = kConsumers / hpc;
+    const int kvh = hgrp * hpc + h_local;
+    const int64_t tok_stride = (int64_t)a.H_kv * kD;
+    const uint16_t* kbase = a.k[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
+    const uint16_t* vbase = a.v[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
+    // query fragments in the permuted dim order of KTile
+    uint32_t qb[kD / 16][2];
+    {
+        const uint16_t* qrow = a.q[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
+        const bool ok = g < ratio;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const float mb = xml[(w * NT * 4 + n * 4 + c) * kWarp + lane];
-                    const float lb = xml[(w * NT * 4 + n * 4 + 2 + c) * kWarp + lane];
-                    const float M = fmaxf(m_run[n][c], mb);
-                    const float sa = M == -INFINITY ? 0.f : exp2f(m_run[n][c] - M);
-                    const float sb = M == -INFINITY ? 0.f : exp2f(mb - M);
-                    m_run[n][c] = M;
-                    l_run[n][c] = l_run[n][c] * sa + lb * sb;
-#pragma unroll
-                    for (int mt = 0; mt < kD / 16; ++mt) {
-                        o[n][mt][c] = o[n][mt][c] * sa + xo[(w * kRegs + (n * (kD / 16) + mt) * 4 + c) * kWarp + lane] * sb;
-                        o[n][mt][c + 2] =
-                            o[n][mt][c + 2] * sa + xo[(w * kRegs + (n * (kD / 16) + mt) * 4 + c + 2) * kWarp + lane] * sb;
-                    }
-                }
-            }
-        }
-        // write this kv head's query heads: the final output, or one split partial
-        const int kvh = hgrp * hpc + h_local;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int hh = 8 * n + 2 * t4 + c;
-                if (hh >= ratio) continue;
-                const int64_t qh = (int64_t)kvh * ratio + hh;
-                const float inv = l_run[n][c] > 0.f ? 1.f / l_run[n][c] : 0.f;
-                float* dst = direct ? a.out[layer] + ((int64_t)r * a.H_q + qh) * kD
-                                    : a.part_o + ((row_q * a.n_splits + split) * a.H_q + qh) * kD;
-                const float sc = direct ? inv : 1.f;
-#pragma unroll
-                for (int mt = 0; mt < kD / 16; ++mt) {
-                    const int d0 = 8 * ((mt >> 2) ? 8 + g : g) + 2 * (mt & 3);
-                    *reinterpret_cast<float2*>(dst + d0) = make_float2(o[n][mt][c] * sc, o[n][mt][c + 2] * sc);
-                }
-                if (!direct && g == 0)
-                    *reinterpret_cast<float2*>(a.part_ml + ((row_q * a.n_splits + split) * a.H_q + qh) * 2) =
-                        make_float2(m_run[n][c], l_run[n][c]);
-            }
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint16_t* p = qrow + g * kD + 8 * (t4 + 4 * (ks >> 1)) + 4 * (ks & 1);
+            qb[ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p)) : 0u;
+            qb[ks][1] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p + 2)) : 0u;
         }
     }
+    KTile ka, kb2;
+    VTile va, vb2;
+    if (wsel < n_tiles) {
+        load_ktile(ka, kbase, tok_stride, s_ent + wsel * kTile, g, t4);
+        load_vtile(va, vbase, tok_stride, s_ent + wsel * kTile, g, t4);
+    }
+    if (wsel + n_sel < n_tiles) {
+        load_ktile(kb2, kbase, tok_stride, s_ent + (wsel + n_sel) * kTile, g, t4);
+        load_vtile(vb2, vbase, tok_stride, s_ent + (wsel + n_sel) * kTile, g, t4);
+    }
+    auto tile = [&](int i, KTile& k, VTile& v) {
+        const int ent_lane = lane < kTile ? s_ent[i * kTile + lane] : 0;
+        const uint32_t masked = __ballot_sync(0xffffffffu, lane < kTile && ent_lane < 0);
+        const bool ok_g = !((masked >> g) & 1u);
+        const bool ok_g8 = !((masked >> (g + 8)) & 1u);
+        float sacc[NT][4] = {{0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const int j = ks >> 1, w = 2 * (ks & 1);
+            const uint32_t afr[4] = {word(k.r[0][j], w), word(k.r[1][j], w), word(k.r[0][j], w + 1),
+                                     word(k.r[1][j], w + 1)};
+            mma_bf16(sacc[0], afr, qb[ks][0], qb[ks][1]);
+        }
+        softmax_pv<NT>(sacc, ok_g, ok_g8, a.scale_log2, m_run, l_run, o, v);
+        // K and V two tiles ahead, in flight during the next tile's math
+        if (i + 2 * n_sel < n_tiles) {
+            load_ktile(k, kbase, tok_stride, s_ent + (i + 2 * n_sel) * kTile, g, t4);
+            load_vtile(v, vbase, tok_stride, s_ent + (i + 2 * n_sel) * kTile, g, t4);
+        }
+    };
+    for (int i = wsel; i < n_tiles; i += 2 * n_sel) {
+        tile(i, ka, va);
+        if (i + n_sel < n_tiles) tile(i + n_sel, kb2, vb2);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int msk = 4; msk < 32; msk <<= 1) l_run[0][j] += __shfl_xor_sync(0xffffffffu, l_run[0][j], msk);
+    __syncthreads();  // the merge area reuses the entry list
+    merge_and_store<NT>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, hpc, hgrp, r, layer, split, ratio);
 }
 
 // Split merge: one warp per (query head, row, layer); lane l owns dims
@@ -488,6 +662,8 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
     const int NT = (H_q / H_kv + 7) / 8;
     size_t merge = (size_t)kConsumers * (NT * (kD / 16) * 4 + NT * 4) * kWarp * 4;
     size_t stages_bytes = (size_t)ns * stage;
+    // groups of at most 8 query heads run the register-streaming kernel: no K stages
+    if (H_q / H_kv <= 8) stages_bytes = 0;
     p.smem_bytes = p.stage_off + (stages_bytes > merge ? stages_bytes : merge);
     const size_t rows_q = (size_t)G * n_q;
     size_t ws = 256;
@@ -505,10 +681,10 @@ cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t s
     const int ratio = a.H_q / a.H_kv;
     dim3 grid((unsigned)(a.n_splits * a.head_groups), (unsigned)a.n_q, (unsigned)a.G);
     if (ratio <= 8) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(attend_rk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem_bytes);
         if (e != cudaSuccess) return e;
-        e = launch_pdl(attend_kernel<1>, grid, dim3(kAtThreads), smem_bytes, stream, 0, a);
+        e = launch_pdl(attend_rk_kernel, grid, dim3(kConsumers * kWarp), smem_bytes, stream, 0, a);
         if (e != cudaSuccess) return e;
     } else {
         cudaError_t e = cudaFuncSetAttribute(attend_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
