@@ -310,9 +310,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             for (int rr = 0; rr < 32 / H_I; ++rr) {
                 const int col = 32 * c + rr * H_I;  // first of this query row's columns
                 const int i = col / H_I;
-                int32_t acc = 0;
+                // four independent partial sums: a 16-long chain of dependent
+                // multiply-adds would stall on its own latency
+                int32_t acc4[4] = {0, 0, 0, 0};
 #pragma unroll
-                for (int h = 0; h < H_I; ++h) acc += max((int32_t)v[rr * H_I + h], 0) * w[rr * H_I + h];
+                for (int h = 0; h < H_I; ++h) acc4[h & 3] += max((int32_t)v[rr * H_I + h], 0) * w[rr * H_I + h];
+                const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 if (t >= rs[i] && t < rws[i]) keys0[(int64_t)i * a.fine_cap + (t - rs[i])] = (uint32_t)acc + 1u;
             }
         };

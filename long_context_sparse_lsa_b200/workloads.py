@@ -80,13 +80,20 @@ PROFILE32K = Workload("decode_b16_32k_hi64x256", 1, (32768,) * 16, 16, 128, -16,
                       64, 256, 32, 4, 128, 1, note="batched decode, 16 seqs x 32768, HI 64x256 (profiling size)")
 
 
+# A smaller prefill chunk (2048 rows on a 65536-token cache, same heads and
+# budget) for profiler captures of the tensor-core indexer.
+PREFILL_PROFILE = Workload("prefill_2048_on_65536", 3, (65536 + 2048,), 16, 128, -16, 15, 8, 64, 1024, 2048,
+                           0, 0, 32, 4, 128, 1, prefill_new=2048,
+                           note="causal prefill chunk of 2048 tokens on a 65536-token cache, HI off (profiling size)")
+
+
 def ragged() -> Workload:
     return Workload("ragged_decode_64seq_lognormal", 4, _ragged_lens(4), 16, 128, -16, 15, 8, 64, 1024, 2048,
                     64, 256, 32, 4, 128, 2, note="64 ragged seqs, lognormal median 32768, G=2, HI 64x256")
 
 
 def all_workloads() -> list[Workload]:
-    return [TINY, BATCH128K, CTX1M, PREFILL, ragged(), PROFILE32K]
+    return [TINY, BATCH128K, CTX1M, PREFILL, ragged(), PROFILE32K, PREFILL_PROFILE]
 
 
 def by_name(name: str) -> Workload:
