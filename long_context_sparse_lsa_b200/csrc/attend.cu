@@ -475,15 +475,21 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
     const int hpc = a.hpc;
     const int q_heads_cta = hpc * ratio;
 
+    // The set entries and the row's sequence metadata are fetched together
+    // (the entries are checked against q_len once it is known); nothing is
+    // written before the row check.
     const int seq = a.q_seq[r];
     const int L = a.q_len[r];
-    bool bad = seq < 0 || seq >= a.n_seq;
-    int64_t off = 0;
-    if (!bad) {
-        off = a.kv_offset[seq];
-        const int slen = a.seq_lens[seq];
-        bad = L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens;
-    }
+    const int seq_c = min(max(seq, 0), a.n_seq - 1);
+    const int64_t off = a.kv_offset[seq_c];
+    const int slen = a.seq_lens[seq_c];
+    const int e0 = split * a.entries_per_split;
+    const int32_t* set = a.sets + (int64_t)r * a.budget + e0;
+    const int n_cap = max(0, min(a.budget - e0, a.entries_per_split));  // entries this split may own
+    int32_t* s_ent = reinterpret_cast<int32_t*>(smem);
+    for (int i = tid; i < n_cap; i += kConsumers * kWarp) s_ent[i] = set[i];
+    const bool bad = seq < 0 || seq >= a.n_seq || L < 1 || L > a.max_len || L > slen || off < 0 ||
+                     off + slen > a.total_tokens;
     if (bad) {
         if (tid == 0 && blockIdx.x == 0 && layer == 0)
             flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
@@ -494,15 +500,12 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
         return;
     }
     const int n_entries = min(L, a.budget);
-    const int e0 = split * a.entries_per_split;
     const int n_local = max(0, min(n_entries - e0, a.entries_per_split));
     const int n_tiles = (n_local + kTile - 1) / kTile;
-    const int32_t* set = a.sets + (int64_t)r * a.budget + e0;
-    int32_t* s_ent = reinterpret_cast<int32_t*>(smem);
     for (int i = tid; i < n_tiles * kTile; i += kConsumers * kWarp) {
         int v = -1;
         if (i < n_local) {
-            v = set[i];
+            v = s_ent[i];  // written by this thread above (same index and stride)
             if (v < -1 || v >= L) {
                 flag(a.dev_status, LSA_DEV_BAD_INDEX);
                 v = -1;
@@ -585,12 +588,13 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
 __global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_constant__ AttendArgs a) {
     pdl_enter();
     const int h = blockIdx.x, r = blockIdx.y, layer = blockIdx.z, lane = threadIdx.x;
+    // the row check's loads overlap the partials' loads; the output is only
+    // written for a valid row (an invalid row's output was zeroed already)
     const int seq = a.q_seq[r];
     const int L = a.q_len[r];
-    if (seq < 0 || seq >= a.n_seq) return;
-    const int64_t off = a.kv_offset[seq];
-    const int slen = a.seq_lens[seq];
-    if (L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens) return;  // zeroed already
+    const int seq_c = min(max(seq, 0), a.n_seq - 1);
+    const int64_t off = a.kv_offset[seq_c];
+    const int slen = a.seq_lens[seq_c];
     const int64_t row_q = (int64_t)layer * a.n_q + r;
     const float* P = a.part_o + (row_q * a.n_splits * a.H_q + h) * kD;
     const float* PML = a.part_ml + (row_q * a.n_splits * a.H_q + h) * 2;
@@ -622,6 +626,8 @@ __global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_consta
             M = nm;
         }
     }
+    if (seq < 0 || seq >= a.n_seq || L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens)
+        return;
     const float inv = den > 0.f ? 1.f / den : 0.f;
     reinterpret_cast<float4*>(a.out[layer] + ((int64_t)r * a.H_q + h) * kD)[lane] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);

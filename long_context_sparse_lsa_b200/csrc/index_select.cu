@@ -489,25 +489,6 @@ __device__ void cluster_compact(SelShared& sh, const Keys<K>& keys, int m, uint3
     }
 }
 
-__device__ __forceinline__ bool row_ok_sel(const IndexArgs& a, int r, int64_t& off, int& L, int32_t& bits) {
-    const int seq = a.q_seq[r];
-    L = a.q_len[r];
-    if (seq < 0 || seq >= a.n_seq) {
-        bits = LSA_DEV_BAD_SEQ;
-        return false;
-    }
-    off = a.kv_offset[seq];
-    const int slen = a.seq_lens[seq];
-    bits = LSA_DEV_BAD_LENGTH;
-    if (L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens) return false;
-    if (a.hi_block > 0) {
-        const int64_t bo = a.blk_offset[seq];
-        if (bo < 0 || bo + (L + a.hi_block - 1) / a.hi_block > a.block_rows) return false;
-    }
-    bits = 0;
-    return true;
-}
-
 // Slice of CTA c of C over n keys, in whole 32-key words: [k_lo, k_lo + m).
 __device__ __forceinline__ void slice_of(int n, uint32_t C, uint32_t c, int& k_lo, int& m) {
     const int W = (n + 31) / 32;
@@ -532,19 +513,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     K* stage = stage_cap > 0 ? reinterpret_cast<K*>(dyn + lay.off_stage) : nullptr;
     int32_t* s_kept = reinterpret_cast<int32_t*>(dyn + lay.off_kept);
     int32_t* out = a.index_sets + (int64_t)r * a.budget;
-    const int n_kept_row = (kTokens && a.hi_block > 0) ? a.n_kept[r] : 0;
-    int64_t off;
-    int L;
-    int32_t bits;
-    if (!row_ok_sel(a, r, off, L, bits)) {  // uniform over the cluster: no cluster barrier is reached
-        if (kTokens) {
-            if (c == 0 && threadIdx.x == 0) flag(a.dev_status, bits);
-            for (int e = (int)(c * kSelThreads) + threadIdx.x; e < a.budget; e += (int)(C * kSelThreads)) out[e] = -1;
-        } else if (c == 0 && threadIdx.x == 0) {
-            a.n_kept[r] = 0;  // the token selection reports the row
-        }
-        return;
-    }
+    // Row geometry from q_len alone (clamped so every read below stays in
+    // bounds), so that the slice's keys stream in while the row's sequence
+    // metadata is fetched and checked; nothing is written before the check.
+    const int n_kept_row = (kTokens && a.hi_block > 0) ? min(max(a.n_kept[r], 0), a.hi_topblocks) : 0;
+    const int Lq = a.q_len[r];
+    const int seq_q = a.q_seq[r];
+    const int seq_c = min(max(seq_q, 0), a.n_seq - 1);
+    const int64_t off_q = a.kv_offset[seq_c];
+    const int slen_q = a.seq_lens[seq_c];
+    const int64_t boff_q = a.hi_block > 0 ? a.blk_offset[seq_c] : 0;
+    const int L = min(max(Lq, 0), a.max_len);
     const int s = min(a.sink, L);
     const int ws = max(s, L - a.window);
     const int B = a.hi_block;
@@ -577,6 +556,22 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     stage_pass<K>(sh, keys, m, stage);
     __syncthreads();
     if (stage != nullptr) keys.s = smem_u32(stage);
+    // the row check (as in the scoring kernels): uniform over the cluster, and
+    // before the first cluster barrier
+    int32_t bits = 0;
+    if (seq_q < 0 || seq_q >= a.n_seq) bits = LSA_DEV_BAD_SEQ;
+    else if (Lq < 1 || Lq > a.max_len || Lq > slen_q || off_q < 0 || off_q + slen_q > a.total_tokens ||
+             (a.hi_block > 0 && (boff_q < 0 || boff_q + (Lq + a.hi_block - 1) / a.hi_block > a.block_rows)))
+        bits = LSA_DEV_BAD_LENGTH;
+    if (bits != 0) {
+        if (kTokens) {
+            if (c == 0 && threadIdx.x == 0) flag(a.dev_status, bits);
+            for (int e = (int)(c * kSelThreads) + threadIdx.x; e < a.budget; e += (int)(C * kSelThreads)) out[e] = -1;
+        } else if (c == 0 && threadIdx.x == 0) {
+            a.n_kept[r] = 0;  // the token selection reports the row
+        }
+        return;
+    }
     cluster_sync();  // every CTA's row histogram is clear and its slice counted
     push_hist(sh, C);
     cluster_sync();
