@@ -112,13 +112,6 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-            "r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
 
 // 32 consecutive accumulator columns of this warp's 32 TMEM lanes. The load
 // is asynchronous: its registers are valid only after tmem_wait(v), which
@@ -359,50 +352,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
     }
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 2-D uint8 tensor map over [rows, 128] with a box of [box_rows, 128] and the
-// 128-byte swizzle; rows past the end read as zero.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)kTcK, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)kTcK};
-    const cuuint32_t box[2] = {(cuuint32_t)kTcK, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool prefill_tc_supported(int H_I, int d_I, int n_seq, int64_t total_tokens) {
     return d_I == kTcK && H_I == 16 && n_seq == 1 && total_tokens + kTcTokens < (int64_t)0x7fffffff &&
-           encode_fn() != nullptr;
+           tensor_maps_available();
 }
 
 cudaError_t launch_fine_scores_tc(const IndexArgs& ia, cudaStream_t stream) {
     TcArgs a;
     std::memset(&a, 0, sizeof a);
-    if (!make_map(&a.tmap_k, ia.k_idx, (uint64_t)ia.total_tokens, kTcTokens)) return cudaErrorInvalidValue;
-    if (!make_map(&a.tmap_q, ia.q_idx, (uint64_t)ia.n_q * ia.H_I, kTcCols)) return cudaErrorInvalidValue;
+    if (!tensor_map_rows128(&a.tmap_k, ia.k_idx, (uint64_t)ia.total_tokens, kTcTokens)) return cudaErrorInvalidValue;
+    if (!tensor_map_rows128(&a.tmap_q, ia.q_idx, (uint64_t)ia.n_q * ia.H_I, kTcCols)) return cudaErrorInvalidValue;
     a.w = ia.w;
     a.q_seq = ia.q_seq;
     a.q_len = ia.q_len;

@@ -13,6 +13,8 @@
 // register use keep several CTAs — and thus many loads in flight — on every
 // SM. Scores are written as keys (score + 1; 0 = not a candidate) to an
 // L2-resident workspace for the selection kernels.
+#include <cstring>
+
 #include "index_common.cuh"
 
 namespace lsa {
@@ -168,6 +170,190 @@ __global__ void __launch_bounds__(kScThreads, kFineCtasPerSm) fine_score_kernel(
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fine scores with HI on, d_I = 128, hi_block a multiple of 16: the kept
+// blocks are contiguous runs of key rows, so each one (or each 64-row part)
+// arrives as one TMA tensor copy (128-byte swizzle) instead of per-lane
+// gathers. A persistent CTA per SM takes a contiguous range of (row, kept
+// block, part) items. The producer warp looks up 32 items' kept-block ids
+// at once, then one lane issues their copies into a ring of 24 stages; item
+// k goes to stage k mod 24 and consumer warp k mod 8, which scores its
+// 16-row tiles from shared memory (the swizzle spreads the 8 rows a load
+// reads over all banks) and releases the stage.
+constexpr int kFtConsumers = 8;
+constexpr int kFtThreads = (kFtConsumers + 1) * kWarp;
+constexpr int kFtStages = 24;
+constexpr int kFtRows = 64;                   // key rows per item (box rows)
+constexpr int kFtStageBytes = kFtRows * 128;  // 8 KB
+
+struct FineTmaArgs {
+    CUtensorMap tmap;  // key cache [total_tokens, 128], box kFtRows x 128
+    IndexArgs a;
+    int32_t sb;        // rows per item: min(hi_block, kFtRows)
+};
+
+struct FtItem {
+    int32_t row;      // query row, -1: no more items for this warp
+    int32_t slot0;    // first slot of the item in the row's key list
+    int32_t tok0;     // first token of the item (in its sequence)
+    int32_t s, ws;    // the row's middle
+    int32_t pad;
+    int64_t key_row;  // first key row of the copy in the whole cache
+};
+
+struct FtShared {
+    uint64_t full[kFtStages];
+    uint64_t empty[kFtStages];
+    FtItem item[kFtStages];
+    FtItem batch[32];  // the producer warp's next 32 items
+    int32_t fail;
+};
+
+constexpr size_t kFtSmem = 1024 + (size_t)kFtStages * kFtStageBytes + sizeof(FtShared);
+
+template <int NT>
+__global__ void __launch_bounds__(kFtThreads, 1) fine_score_tma_kernel(const __grid_constant__ FineTmaArgs p) {
+    pdl_enter();
+    const IndexArgs& a = p.a;
+    extern __shared__ __align__(16) uint8_t ft_raw[];
+    const uint32_t raw = smem_u32(ft_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle atoms are 1024-byte aligned
+    FtShared& sh = *reinterpret_cast<FtShared*>(ft_raw + (base - raw) + kFtStages * kFtStageBytes);
+    const int warp = warp_id(), lane = lane_id(), g = lane >> 2, t4 = lane & 3;
+    const int SB = p.sb;
+    const int B = a.hi_block;
+    const int parts = B / SB;
+    const int64_t per_row = (int64_t)a.hi_topblocks * parts;
+    const int64_t total = (int64_t)a.n_q * per_row;
+    const int64_t i_lo = total * blockIdx.x / gridDim.x, i_hi = total * (blockIdx.x + 1) / gridDim.x;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kFtStages; ++st) {
+            mbar_init(smem_u32(&sh.full[st]), 1);
+            mbar_init(smem_u32(&sh.empty[st]), 1);
+        }
+        sh.fail = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    if (warp == kFtConsumers) {
+        // ------------------------------ producer ------------------------------
+        int k = 0;  // items issued
+        auto next_stage = [&](int kk) -> bool {  // lane 0: wait until stage kk % S is free
+            const int st = kk % kFtStages;
+            if (kk >= kFtStages &&
+                !mbar_wait_bounded(smem_u32(&sh.empty[st]), (uint32_t)(((kk / kFtStages) + 1) & 1), kWaitLimitNs)) {
+                sh.fail = 1;
+                return false;
+            }
+            return true;
+        };
+        bool ok = true;
+        for (int64_t c0 = i_lo; ok && c0 < i_hi; c0 += kWarp) {
+            // every lane looks up one item of the next 32 (three L2 round trips for all of them)
+            const int64_t i = c0 + lane;
+            FtItem it;
+            it.row = -1;
+            if (i < i_hi) {
+                const int r = (int)(i / per_row);
+                const int rem = (int)(i - (int64_t)r * per_row);
+                const int q = rem / parts, part = rem - q * parts;
+                // the kept count and id are fetched together with the row check
+                const int nk = a.n_kept[r];
+                const int kid = a.kept[(int64_t)r * a.hi_topblocks + q];
+                int64_t off;
+                int L;
+                if (row_ok(a, r, off, L) && q < min(max(nk, 0), a.hi_topblocks)) {
+                    it.row = r;
+                    it.slot0 = q * B + part * SB;
+                    it.tok0 = kid * B + part * SB;
+                    it.s = min(a.sink, L);
+                    it.ws = max(it.s, L - a.window);
+                    it.pad = 0;
+                    it.key_row = off + it.tok0;
+                }
+            }
+            sh.batch[lane] = it;
+            __syncwarp();
+            if (lane == 0) {
+                const int n = (int)min((int64_t)kWarp, i_hi - c0);
+                for (int j = 0; j < n; ++j) {
+                    const FtItem b = sh.batch[j];
+                    if (b.row < 0) continue;
+                    if (!next_stage(k)) {
+                        ok = false;
+                        break;
+                    }
+                    const int st = k % kFtStages;
+                    sh.item[st] = b;
+                    mbar_arrive_expect_tx(smem_u32(&sh.full[st]), (uint32_t)(SB * 128));
+                    tma_load_2d(base + (uint32_t)(st * kFtStageBytes), &p.tmap, 0, (int)b.key_row,
+                                smem_u32(&sh.full[st]));
+                    ++k;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            __syncwarp();
+        }
+        // one end marker per consumer warp
+        if (lane == 0) {
+            for (int w = 0; w < kFtConsumers; ++w) {
+                if (!next_stage(k)) break;
+                const int st = k % kFtStages;
+                sh.item[st].row = -1;
+                mbar_arrive(smem_u32(&sh.full[st]));
+                ++k;
+            }
+            // every issued copy lands before the CTA may exit
+            for (int kk = max(0, k - kFtStages); kk < k; ++kk)
+                mbar_wait_bounded(smem_u32(&sh.full[kk % kFtStages]), (uint32_t)((kk / kFtStages) & 1), kWaitLimitNs);
+        }
+    } else {
+        // ------------------------------ consumers -----------------------------
+        // the first item's row is known before any copy lands: fetch its query now
+        int qrow = i_lo < i_hi ? (int)(i_lo / per_row) : -1;
+        QueryFrag<128, NT> qf;
+        if (qrow >= 0) load_query<128, NT>(qf, a, qrow);
+        uint32_t* keys = qrow >= 0 ? a.fine_keys + (int64_t)qrow * a.fine_cap : nullptr;
+        for (int k = warp;; k += kFtConsumers) {
+            const int st = k % kFtStages;
+            if (!mbar_wait_bounded(smem_u32(&sh.full[st]), (uint32_t)((k / kFtStages) & 1), kWaitLimitNs)) {
+                if (lane == 0) sh.fail = 1;
+                break;
+            }
+            const FtItem it = sh.item[st];
+            if (it.row < 0) break;
+            if (it.row != qrow) {
+                load_query<128, NT>(qf, a, it.row);
+                qrow = it.row;
+                keys = a.fine_keys + (int64_t)it.row * a.fine_cap;
+            }
+            const uint32_t sbase = base + (uint32_t)(st * kFtStageBytes);
+            for (int t = 0; t < SB / 16; ++t) {
+                RowFrag<128> fa, fb;
+                const int ra = 16 * t + g, rb = ra + 8;
+                // logical 16-byte chunk c of row rr sits at chunk c ^ (rr & 7)
+                const uint4 a0 = ld_shared_v4(sbase + (uint32_t)(ra * 128 + 16 * (t4 ^ (ra & 7))));
+                const uint4 a1 = ld_shared_v4(sbase + (uint32_t)(ra * 128 + 16 * ((4 + t4) ^ (ra & 7))));
+                const uint4 b0 = ld_shared_v4(sbase + (uint32_t)(rb * 128 + 16 * (t4 ^ (rb & 7))));
+                const uint4 b1 = ld_shared_v4(sbase + (uint32_t)(rb * 128 + 16 * ((4 + t4) ^ (rb & 7))));
+                fa.w[0] = a0.x; fa.w[1] = a0.y; fa.w[2] = a0.z; fa.w[3] = a0.w;
+                fa.w[4] = a1.x; fa.w[5] = a1.y; fa.w[6] = a1.z; fa.w[7] = a1.w;
+                fb.w[0] = b0.x; fb.w[1] = b0.y; fb.w[2] = b0.z; fb.w[3] = b0.w;
+                fb.w[4] = b1.x; fb.w[5] = b1.y; fb.w[6] = b1.z; fb.w[7] = b1.w;
+                const int2 sc = fine_tile<128, NT>(qf, fa, fb);
+                const int ta = it.tok0 + ra, tb = it.tok0 + rb;
+                if (t4 == 0) keys[it.slot0 + ra] = (ta >= it.s && ta < it.ws) ? (uint32_t)sc.x + 1u : 0u;
+                if (t4 == 1) keys[it.slot0 + rb] = (tb >= it.s && tb < it.ws) ? (uint32_t)sc.y + 1u : 0u;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh.empty[st]));
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && sh.fail) flag(a.dev_status, LSA_DEV_TIMEOUT);
+}
+
 template <int D_I, int NT>
 cudaError_t launch_scores_t(const IndexArgs& a, bool coarse, cudaStream_t st) {
     if (coarse) {
@@ -179,9 +365,39 @@ cudaError_t launch_scores_t(const IndexArgs& a, bool coarse, cudaStream_t st) {
     }
 }
 
+template <int NT>
+cudaError_t launch_fine_tma(const IndexArgs& a, cudaStream_t st) {
+    FineTmaArgs p;
+    std::memset(&p, 0, sizeof p);
+    p.a = a;
+    p.sb = a.hi_block < kFtRows ? a.hi_block : kFtRows;
+    if (!tensor_map_rows128(&p.tmap, a.k_idx, (uint64_t)a.total_tokens, (uint32_t)p.sb)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(fine_score_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kFtSmem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(fine_score_tma_kernel<NT>, dim3((unsigned)device_sm_count()), dim3(kFtThreads), kFtSmem, st, 0,
+                      p);
+}
+
+// Kept blocks as whole TMA boxes: HI on, 128-byte keys, blocks of a multiple
+// of 16 rows that split into equal boxes of at most kFtRows rows.
+bool fine_tma_ok(const IndexArgs& a, int d_I) {
+    const int B = a.hi_block;
+    return B > 0 && d_I == 128 && B % 16 == 0 && (B <= kFtRows || B % kFtRows == 0) &&
+           a.total_tokens + kFtRows < (int64_t)0x7fffffff && tensor_maps_available();
+}
+
 template <int D_I>
 cudaError_t launch_scores_d(const IndexArgs& a, bool coarse, cudaStream_t st) {
     const int nt = (a.H_I + 7) / 8;
+    if constexpr (D_I == 128) {
+        if (!coarse && fine_tma_ok(a, D_I)) {
+            if (nt <= 1) return launch_fine_tma<1>(a, st);
+            if (nt <= 2) return launch_fine_tma<2>(a, st);
+            if (nt <= 4) return launch_fine_tma<4>(a, st);
+            return launch_fine_tma<8>(a, st);
+        }
+    }
     if (nt <= 1) return launch_scores_t<D_I, 1>(a, coarse, st);
     if (nt <= 2) return launch_scores_t<D_I, 2>(a, coarse, st);
     if (nt <= 4) return launch_scores_t<D_I, 4>(a, coarse, st);

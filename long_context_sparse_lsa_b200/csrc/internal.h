@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/lsa.h"
@@ -85,6 +86,10 @@ cudaError_t launch_index_scores(const IndexArgs& a, int d_I, bool coarse, cudaSt
 // Fine scores of a causal chunk of rows of one sequence (HI off) on the
 // tcgen05 tensor cores; same keys as launch_index_scores(coarse = false).
 bool prefill_tc_supported(int H_I, int d_I, int n_seq, int64_t total_tokens);
+// TMA tensor maps over [rows, 128] byte matrices (128-byte swizzle, box of
+// box_rows x 128 bytes, rows past the end read as zero).
+bool tensor_maps_available();
+bool tensor_map_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows);
 cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream);
 
