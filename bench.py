@@ -268,6 +268,30 @@ def run_reference(args, wl):
 
 
 # ---------------------------------------------------------------------------
+# multi-GPU plumbing (replicas: no collective on the data path)
+# ---------------------------------------------------------------------------
+def rank_workload(wl, rank: int):
+    """Each rank draws its own independent batch of the same shape (weak
+    scaling): rank 0 the workload's seed, rank i > 0 seed + 1000 i."""
+    return wls.small(wl, seed=wl.seed + 1000 * rank) if rank else wl
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The step time the job reports: the maximum of the ranks' times (one
+    all-reduce of a scalar; the only collective the bench issues)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed / the max-over-ranks time."""
+    return units_per_rank * world / (ms / 1000.0)
+
+
+# ---------------------------------------------------------------------------
 def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
     """Draws the workload, captures its step graphs and times `steps` steps
     (after `warmup`), each after an L2 flush: the whole step graph for the
@@ -413,15 +437,11 @@ def main(argv=None):
     stream = torch.cuda.current_stream(dev)
 
     # each rank draws its own independent batch (weak scaling)
-    wl_r = wls.small(wl, seed=wl.seed + 1000 * rank) if rank else wl
+    wl_r = rank_workload(wl, rank)
     clocks = ClockSampler(local)
     run = time_workload(wl_r, dev, flush, stream, args.steps, args.warmup, pg, clocks)
     st, t = run["st"], run["t"]
-    ms = run["ms"]
-    if pg:
-        tt = torch.tensor([ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(run["ms"], pg, dev)
     clk = run["clocks"]
     bs_ms, ix_ms, at_ms = run["bs"], run["ix"], run["at"]
     n_kernels = run["n_kernels"]
@@ -449,17 +469,12 @@ def main(argv=None):
         if i >= args.warmup:
             e2e_ms.append((e0, e1))
     torch.cuda.synchronize()
-    e2e = sum(a.elapsed_time(b) for a, b in e2e_ms) / len(e2e_ms)
-    if pg:
-        tt = torch.tensor([e2e], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        e2e = float(tt.item())
+    e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ms) / len(e2e_ms), pg, dev)
     if st.status_bits() != 0:
         raise RuntimeError(f"device status {st.status_bits():#x} after timing")
 
-    nq_all = wl.n_q * world
-    value = nq_all / (ms / 1000.0)
-    e2e_value = nq_all / (e2e / 1000.0)
+    value = job_rate(wl.n_q, world, ms)
+    e2e_value = job_rate(wl.n_q, world, e2e)
     byts = step_bytes(wl)
     peak, peak_kind = _peaks()
     at = sum(at_ms) / len(at_ms)
