@@ -53,10 +53,18 @@ struct SelShared {
     uint32_t cta_gt[kMaxCluster];  // kept keys per CTA slice (each CTA writes its own into all)
     uint32_t cta_eq[kMaxCluster];
     uint32_t push_base[kMaxCluster];
+    uint32_t cta_above[kMaxCluster];  // keys above the threshold bin per CTA slice (candidate path)
+    uint32_t og_gt[kMaxCluster];      // candidates > T and == T per originating CTA
+    uint32_t og_eq[kMaxCluster];
     uint32_t bin, above, in_bin;
     uint32_t count;        // length of the row's candidate list (remote adds)
     uint32_t local_count;  // candidates of this slice
 };
+
+// Candidate list entries: the key in the low 60 bits (scores stay below 2^40
+// under the ABI's bounds), the originating CTA's rank in the top 4.
+constexpr int kOriginShift = 60;
+constexpr uint64_t kKeyMask = (1ull << kOriginShift) - 1ull;
 
 // Dynamic shared memory: SelShared | candidate list | this slice's candidates
 // | staged slice keys | kept-block ids of the slice (tokens only).
@@ -70,7 +78,7 @@ __host__ __device__ __forceinline__ SelLayout sel_layout(int key_bytes, int stag
     SelLayout L;
     uint32_t o = align16u((uint32_t)sizeof(SelShared));
     L.off_cand = o;
-    o += (uint32_t)(kCandCap * key_bytes);
+    o += (uint32_t)(kCandCap * 8);
     L.off_mine = o;
     o += (uint32_t)(kCandCap * key_bytes);
     L.off_stage = o;
@@ -256,10 +264,15 @@ __device__ void digit_hist(uint32_t* hist, Get get, int m, int shift, int width,
 // Exact k-th largest key of the row, 1 <= k < total, given the bin tb that
 // holds it (`above` keys in higher bins, in_bin in tb). Keys > thresh plus
 // the first `quota` keys == thresh in position order are the k largest.
+// On the candidate-list path (`carried` set) it also gives this CTA's first
+// output ranks: every candidate carries its CTA of origin and every CTA
+// publishes its count above the bin with its candidates, so the kept counts
+// of the lower-ranked slices follow without another exchange.
 template <typename K>
-__device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, K* cand, K* mine, uint32_t C,
-                                  uint32_t k, uint32_t tb, uint32_t above, uint32_t in_bin, K& thresh,
-                                  uint32_t& quota) {
+__device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uint64_t* cand, K* mine, uint32_t C,
+                                  uint32_t c, uint32_t k, uint32_t tb, uint32_t above, uint32_t in_bin, K& thresh,
+                                  uint32_t& quota, bool& carried, uint32_t& carry_g, uint32_t& carry_e) {
+    carried = false;
     if (tb < 64u) {  // small bins hold a single key value
         thresh = (K)tb;
         quota = k - above;
@@ -287,19 +300,34 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, K* 
                 }
             }
         }
+        // this slice's keys above the bin
+        uint32_t ab = 0;
+#pragma unroll
+        for (int j = 0; j < kBinsPerThread; ++j) {
+            const uint32_t b = threadIdx.x + (uint32_t)(j * kSelThreads);
+            if (b > tb) ab += sh.local_hist[b];
+        }
+        ab = warp_sum(ab);
+        if (lane_id() == 0) sh.wsum[warp_id()] = ab;
         __syncthreads();
         const uint32_t mc = min(sh.local_count, (uint32_t)kCandCap);
-        if (threadIdx.x < C) sh.push_base[threadIdx.x] = atom_add_cluster(map_cta(smem_u32(&sh.count), threadIdx.x), mc);
+        if (threadIdx.x < C) {
+            uint32_t above_local = 0;
+            for (int w = 0; w < kSelWarps; ++w) above_local += sh.wsum[w];
+            sh.push_base[threadIdx.x] = atom_add_cluster(map_cta(smem_u32(&sh.count), threadIdx.x), mc);
+            st_cluster(map_cta(smem_u32(&sh.cta_above[c]), threadIdx.x), above_local);
+        }
         __syncthreads();
         const uint32_t cbase = smem_u32(cand);
+        const uint64_t tag = (uint64_t)c << kOriginShift;
         for (uint32_t i = threadIdx.x; i < mc; i += kSelThreads) {
-            const K key = mine[i];
+            const uint64_t e = (uint64_t)mine[i] | tag;
             for (uint32_t t = 0; t < C; ++t) {
                 const uint32_t p = sh.push_base[t] + i;
-                if (p < (uint32_t)kCandCap) st_cluster_key<K>(map_cta(cbase + (uint32_t)sizeof(K) * p, t), key);
+                if (p < (uint32_t)kCandCap) st_cluster_key<uint64_t>(map_cta(cbase + 8u * p, t), e);
             }
         }
-        cluster_sync();
+        cluster_sync();  // after this no CTA touches another CTA's shared memory
         const int mm = (int)min(sh.count, (uint32_t)kCandCap);
         while (shift > 0) {  // identical in every CTA
             const int width = shift < kDigitBits ? shift : kDigitBits;
@@ -307,13 +335,36 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, K* 
             reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
             reinterpret_cast<uint4*>(sh.hist)[threadIdx.x + kSelThreads] = make_uint4(0u, 0u, 0u, 0u);
             __syncthreads();
-            digit_hist<K>(sh.hist, [&](int i) { return cand[i]; }, mm, shift, width, prefix);
+            digit_hist<K>(sh.hist, [&](int i) { return (K)(cand[i] & kKeyMask); }, mm, shift, width, prefix);
             __syncthreads();
             uint32_t d, ab, ib;
             find_bin(sh, krem, d, ab, ib);
             prefix = (K)((prefix << width) | (K)d);
             krem -= ab;
         }
+        // kept counts per originating slice: keys above the bin plus its
+        // candidates > T, and its candidates == T
+        if (threadIdx.x < kMaxCluster) {
+            sh.og_gt[threadIdx.x] = 0;
+            sh.og_eq[threadIdx.x] = 0;
+        }
+        __syncthreads();
+        const K T = prefix;
+        for (int i = threadIdx.x; i < mm; i += kSelThreads) {
+            const uint64_t e = cand[i];
+            const K key = (K)(e & kKeyMask);
+            const uint32_t o = (uint32_t)(e >> kOriginShift);
+            if (key > T) atomicAdd(&sh.og_gt[o], 1u);
+            else if (key == T) atomicAdd(&sh.og_eq[o], 1u);
+        }
+        __syncthreads();
+        carry_g = 0;
+        carry_e = 0;
+        for (uint32_t o = 0; o < c; ++o) {
+            carry_g += sh.cta_above[o] + sh.og_gt[o];
+            carry_e += sh.og_eq[o];
+        }
+        carried = true;
     } else {
         // refine over the slices: one cluster histogram per digit
         while (shift > 0) {
@@ -381,52 +432,59 @@ __device__ void slice_counts(SelShared& sh, uint32_t bin, bool from_mine, const 
 
 // With `counted`, (ng, ne) are this slice's counts of keys > thresh and ==
 // thresh (slice_counts); otherwise a pass over the slice counts them.
+// With `carried`, (carry_g, carry_e) already give this slice's first ranks
+// (the candidate path) and no exchange is needed.
 template <typename K, typename Emit>
 __device__ void cluster_compact(SelShared& sh, const Keys<K>& keys, int m, uint32_t C, uint32_t c, K thresh,
-                                uint32_t quota, bool counted, uint32_t ng_in, uint32_t ne_in, Emit emit) {
+                                uint32_t quota, bool counted, uint32_t ng_in, uint32_t ne_in, bool carried,
+                                uint32_t carry_g_in, uint32_t carry_e_in, Emit emit) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
-    // 1. this slice's counts, published to every CTA
-    const int nw_all = counted ? 0 : (m + 31) / 32;
-    uint32_t ng = 0, ne = 0;
-    for (int w0 = wid; w0 < nw_all; w0 += kSelWarps * kUnroll) {
-        K kv[kUnroll];
+    uint32_t carry_g = carry_g_in, carry_e = carry_e_in;
+    if (!carried) {
+        // 1. this slice's counts, published to every CTA
+        const int nw_all = counted ? 0 : (m + 31) / 32;
+        uint32_t ng = 0, ne = 0;
+        for (int w0 = wid; w0 < nw_all; w0 += kSelWarps * kUnroll) {
+            K kv[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = 32 * (w0 + u * kSelWarps) + lane;
-            kv[u] = i < m ? keys[i] : K(0);
-        }
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = 32 * (w0 + u * kSelWarps) + lane;
+                kv[u] = i < m ? keys[i] : K(0);
+            }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int i = 32 * (w0 + u * kSelWarps) + lane;
-            ng += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] > thresh));
-            ne += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] == thresh));
-        }
-    }
-    if (!counted) {
-        if (lane == 0) {
-            sh.wsum[wid] = ng;
-            sh.wsum2[wid] = ne;
-        }
-        __syncthreads();
-    }
-    if (tid < (int)C) {
-        uint32_t tg = ng_in, te = ne_in;
-        if (!counted) {
-            tg = 0;
-            te = 0;
-            for (int w = 0; w < kSelWarps; ++w) {
-                tg += sh.wsum[w];
-                te += sh.wsum2[w];
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = 32 * (w0 + u * kSelWarps) + lane;
+                ng += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] > thresh));
+                ne += (uint32_t)__popc(__ballot_sync(0xffffffffu, i < m && kv[u] == thresh));
             }
         }
-        st_cluster(map_cta(smem_u32(&sh.cta_gt[c]), (uint32_t)tid), tg);
-        st_cluster(map_cta(smem_u32(&sh.cta_eq[c]), (uint32_t)tid), te);
-    }
-    cluster_sync();  // after this no CTA touches another CTA's shared memory
-    uint32_t carry_g = 0, carry_e = 0;
-    for (uint32_t t = 0; t < c; ++t) {
-        carry_g += sh.cta_gt[t];
-        carry_e += sh.cta_eq[t];
+        if (!counted) {
+            if (lane == 0) {
+                sh.wsum[wid] = ng;
+                sh.wsum2[wid] = ne;
+            }
+            __syncthreads();
+        }
+        if (tid < (int)C) {
+            uint32_t tg = ng_in, te = ne_in;
+            if (!counted) {
+                tg = 0;
+                te = 0;
+                for (int w = 0; w < kSelWarps; ++w) {
+                    tg += sh.wsum[w];
+                    te += sh.wsum2[w];
+                }
+            }
+            st_cluster(map_cta(smem_u32(&sh.cta_gt[c]), (uint32_t)tid), tg);
+            st_cluster(map_cta(smem_u32(&sh.cta_eq[c]), (uint32_t)tid), te);
+        }
+        cluster_sync();  // after this no CTA touches another CTA's shared memory
+        carry_g = 0;
+        carry_e = 0;
+        for (uint32_t t = 0; t < c; ++t) {
+            carry_g += sh.cta_gt[t];
+            carry_e += sh.cta_eq[t];
+        }
     }
     // 2. ranks within the slice, one bitmap chunk at a time
     for (int c0 = 0; c0 < m; c0 += kChunkWords * 32) {
@@ -508,7 +566,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     const uint32_t C = cluster_size(), c = cluster_rank();
     const int stage_cap = kTokens ? a.fine_stage : a.coarse_stage;
     const SelLayout lay = sel_layout((int)sizeof(K), stage_cap, kTokens ? a.kept_slots : 0);
-    K* cand = reinterpret_cast<K*>(dyn + lay.off_cand);
+    uint64_t* cand = reinterpret_cast<uint64_t*>(dyn + lay.off_cand);
     K* mine = reinterpret_cast<K*>(dyn + lay.off_mine);
     K* stage = stage_cap > 0 ? reinterpret_cast<K*>(dyn + lay.off_stage) : nullptr;
     int32_t* s_kept = reinterpret_cast<int32_t*>(dyn + lay.off_kept);
@@ -553,6 +611,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
         sh.local_count = 0;
     }
     __syncthreads();
+    // every CTA's row histogram and counters are clear once all CTAs have
+    // arrived here; the wait comes after this CTA's own staging pass
+    cluster_arrive();
     stage_pass<K>(sh, keys, m, stage);
     __syncthreads();
     if (stage != nullptr) keys.s = smem_u32(stage);
@@ -563,6 +624,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     else if (Lq < 1 || Lq > a.max_len || Lq > slen_q || off_q < 0 || off_q + slen_q > a.total_tokens ||
              (a.hi_block > 0 && (boff_q < 0 || boff_q + (Lq + a.hi_block - 1) / a.hi_block > a.block_rows)))
         bits = LSA_DEV_BAD_LENGTH;
+    cluster_wait();  // complete the barrier every CTA arrived at (an exiting CTA must too)
     if (bits != 0) {
         if (kTokens) {
             if (c == 0 && threadIdx.x == 0) flag(a.dev_status, bits);
@@ -572,7 +634,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
         }
         return;
     }
-    cluster_sync();  // every CTA's row histogram is clear and its slice counted
     push_hist(sh, C);
     cluster_sync();
     const uint32_t want = (uint32_t)(kTokens ? a.topk : a.hi_topblocks);
@@ -582,16 +643,20 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     if (k > 0u) {
         K thr = K(1);
         uint32_t quota = 0xffffffffu;  // k == total: every candidate is kept
-        if (k < total) resolve_threshold<K>(sh, keys, m, cand, mine, C, k, tb, above, in_bin, thr, quota);
-        // this slice's kept counts from its histogram (and candidates), unless
-        // the threshold bin was refined over the slices
-        const bool list = k < total && tb >= 64u && in_bin <= (uint32_t)kCandCap;
-        const bool counted = k == total || tb < 64u || list;
+        bool carried = false;
+        uint32_t carry_g = 0, carry_e = 0;
+        if (k < total)
+            resolve_threshold<K>(sh, keys, m, cand, mine, C, c, k, tb, above, in_bin, thr, quota, carried, carry_g,
+                                 carry_e);
+        // otherwise this slice's kept counts come from its histogram (exact
+        // bins) or a pass over its keys (bin refined over the slices)
+        const bool counted = !carried && (k == total || tb < 64u);
         uint32_t ng = 0, ne = 0;
-        if (counted) slice_counts<K>(sh, k == total ? 1u : tb, list, mine, thr, ng, ne);
+        if (counted) slice_counts<K>(sh, k == total ? 1u : tb, false, mine, thr, ng, ne);
         if (kTokens) {
             const int lgB = (B > 0 && (B & (B - 1)) == 0) ? __ffs(B) - 1 : -1;  // power-of-two block: shift
-            cluster_compact<K>(sh, keys, m, C, c, thr, quota, counted, ng, ne, [&](int slot, uint32_t rank) {
+            cluster_compact<K>(sh, keys, m, C, c, thr, quota, counted, ng, ne, carried, carry_g, carry_e,
+                               [&](int slot, uint32_t rank) {
                 const int gs = k_lo + slot;
                 int tok;
                 if (B > 0) {
@@ -604,7 +669,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
             });
         } else {
             int32_t* kept = a.kept + (int64_t)r * a.hi_topblocks;
-            cluster_compact<K>(sh, keys, m, C, c, thr, quota, counted, ng, ne, [&](int slot, uint32_t rank) {
+            cluster_compact<K>(sh, keys, m, C, c, thr, quota, counted, ng, ne, carried, carry_g, carry_e,
+                               [&](int slot, uint32_t rank) {
                 if (rank < k) kept[rank] = first + k_lo + slot;
             });
         }
