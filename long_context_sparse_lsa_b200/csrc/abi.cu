@@ -214,8 +214,8 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (budget.hi_block > 0) {
-        e = lsa::launch_index_scores(a, d_I, true, cs);
-        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, plan.cluster, plan.smem_blocks, cs);
+        if (!lsa::coarse_in_select(a)) e = lsa::launch_index_scores(a, d_I, true, cs);
+        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, d_I, plan.cluster, plan.smem_blocks, cs);
     }
     if (e == cudaSuccess) {
         // a prefill chunk (many rows of one sequence, HI off) is one dense
@@ -223,7 +223,7 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
         e = index_dense(batch, H_I, d_I, budget) ? lsa::launch_fine_scores_tc(a, cs)
                                                   : lsa::launch_index_scores(a, d_I, false, cs);
     }
-    if (e == cudaSuccess) e = lsa::launch_index_select(a, false, plan.cluster, plan.smem_tokens, cs);
+    if (e == cudaSuccess) e = lsa::launch_index_select(a, false, d_I, plan.cluster, plan.smem_tokens, cs);
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 

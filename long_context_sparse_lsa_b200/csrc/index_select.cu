@@ -28,6 +28,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "index_common.cuh"
 #include "internal.h"
 
 namespace lsa {
@@ -555,9 +556,47 @@ __device__ __forceinline__ void slice_of(int n, uint32_t C, uint32_t c, int& k_l
     m = max(0, min(n, 32 * w_hi) - k_lo);
 }
 
+// HI with the coarse scores computed in place: the slice's blocks
+// [blk0, blk0 + m) of the row are scored straight into `stage` (keys =
+// score + 1) and counted into the slice histogram; one 16-block MMA tile per
+// warp and pass (the fragment scheme of the coarse scoring kernel). Block-sum
+// rows are read at clamped indices, so an invalid row (checked afterwards,
+// before anything is written) reads in bounds.
+template <int D_I, int NT>
+__device__ void coarse_pass(SelShared& sh, const IndexArgs& a, int r, int64_t boff, int blk0, int m, uint64_t* stage) {
+    const int lane = lane_id(), g = lane >> 2, t4 = lane & 3;
+    QueryFrag<D_I, NT> qf;
+    load_query<D_I, NT>(qf, a, r);
+    for (int j = warp_id() * 16; j < m; j += kSelWarps * 16) {  // warp-uniform
+        const int j0 = j + g, j1 = j0 + 8;
+        const int64_t b0 = boff + blk0 + j0, b1 = boff + blk0 + j1;
+        const bool v0 = j0 < m && b0 >= 0 && b0 < a.block_rows;
+        const bool v1 = j1 < m && b1 >= 0 && b1 < a.block_rows;
+        RowFrag<D_I> hg, lg, hg8, lg8;
+        hg.load(a.block_sums + (v0 ? b0 : 0) * (2 * D_I), t4, v0);
+        lg.load(a.block_sums + (v0 ? b0 : 0) * (2 * D_I) + D_I, t4, v0);
+        hg8.load(a.block_sums + (v1 ? b1 : 0) * (2 * D_I), t4, v1);
+        lg8.load(a.block_sums + (v1 ? b1 : 0) * (2 * D_I) + D_I, t4, v1);
+        long long x, y;
+        coarse_tile<D_I, NT>(qf, hg, lg, hg8, lg8, x, y);
+        if (t4 == 0 && j0 < m) {
+            const uint64_t key = (unsigned long long)x + 1ull;
+            stage[j0] = key;
+            atomicAdd(&sh.local_hist[key_bin(key)], 1u);
+        }
+        if (t4 == 1 && j1 < m) {
+            const uint64_t key = (unsigned long long)y + 1ull;
+            stage[j1] = key;
+            atomicAdd(&sh.local_hist[key_bin(key)], 1u);
+        }
+    }
+}
+
 // Selection of one row by one cluster. kTokens: fine top-k and the SI
 // assembly of the index set; otherwise the HI block top-k.
-template <typename K, bool kTokens>
+// D_I > 0 (HI blocks only): the coarse scores are computed in place
+// (coarse_pass) instead of read from the coarse scoring kernel's workspace.
+template <typename K, bool kTokens, int D_I = 0, int NT = 0>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_constant__ IndexArgs a) {
     pdl_enter();
     extern __shared__ __align__(16) uint8_t dyn[];
@@ -614,7 +653,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     // every CTA's row histogram and counters are clear once all CTAs have
     // arrived here; the wait comes after this CTA's own staging pass
     cluster_arrive();
-    stage_pass<K>(sh, keys, m, stage);
+    if constexpr (!kTokens && D_I > 0) {
+        coarse_pass<D_I, NT>(sh, a, r, boff_q, first + k_lo, m, reinterpret_cast<uint64_t*>(stage));
+    } else {
+        stage_pass<K>(sh, keys, m, stage);
+    }
     __syncthreads();
     if (stage != nullptr) keys.s = smem_u32(stage);
     // the row check (as in the scoring kernels): uniform over the cluster, and
@@ -745,10 +788,23 @@ static cudaError_t launch_cluster(Kern kern, const IndexArgs& a, int cluster, si
     return launch_pdl(kern, dim3((unsigned)cluster, (unsigned)a.n_q, 1), dim3(kSelThreads), smem, stream, cluster, a);
 }
 
-cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream) {
+template <int D_I>
+static cudaError_t launch_blocks_fused(const IndexArgs& a, int cluster, size_t smem, cudaStream_t stream) {
+    if (a.H_I <= 8) return launch_cluster(select_kernel<uint64_t, false, D_I, 1>, a, cluster, smem, stream);
+    return launch_cluster(select_kernel<uint64_t, false, D_I, 2>, a, cluster, smem, stream);  // H_I <= 16
+}
+
+cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
+                                cudaStream_t stream) {
     if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
-    return blocks ? launch_cluster(select_kernel<uint64_t, false>, a, cluster, smem, stream)
-                  : launch_cluster(select_kernel<uint32_t, true>, a, cluster, smem, stream);
+    if (!blocks) return launch_cluster(select_kernel<uint32_t, true>, a, cluster, smem, stream);
+    if (!coarse_in_select(a)) return launch_cluster(select_kernel<uint64_t, false>, a, cluster, smem, stream);
+    switch (d_I) {
+        case 32: return launch_blocks_fused<32>(a, cluster, smem, stream);
+        case 64: return launch_blocks_fused<64>(a, cluster, smem, stream);
+        case 128: return launch_blocks_fused<128>(a, cluster, smem, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace lsa

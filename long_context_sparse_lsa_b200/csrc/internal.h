@@ -91,7 +91,17 @@ bool prefill_tc_supported(int H_I, int d_I, int n_seq, int64_t total_tokens);
 bool tensor_maps_available();
 bool tensor_map_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows);
 cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
-cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int cluster, size_t smem, cudaStream_t stream);
+// HI block selection computes the coarse scores itself when each cluster
+// CTA's slice of blocks fits in shared memory, the query has at most 16
+// indexer heads (more would not fit the selection kernel's 64 registers) and
+// there are enough rows for the clusters to cover the GPU (with a few rows
+// the coarse scoring kernel spreads the block sums over more SMs); otherwise
+// the coarse scoring kernel writes the scores to the workspace first.
+inline bool coarse_in_select(const IndexArgs& a) {
+    return a.hi_block > 0 && a.coarse_stage > 0 && a.H_I <= 16 && a.n_q >= 8;
+}
+cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
+                                cudaStream_t stream);
 
 // ---- sparse attention -----------------------------------------------------
 struct AttendArgs {
