@@ -163,6 +163,11 @@ size_t lsa_index_workspace_size(const lsa_batch_t *batch, int32_t H_I,
 int32_t lsa_index_uses_tensor_cores(const lsa_batch_t *batch, int32_t H_I,
                                     int32_t d_I, lsa_budget_t budget);
 
+/* Number of kernel launches lsa_index issues for this shape (host fields
+ * only), e.g. for accounting in benchmarks. 0 for an invalid shape. */
+int32_t lsa_index_launches(const lsa_batch_t *batch, int32_t H_I, int32_t d_I,
+                           lsa_budget_t budget);
+
 /* One index set per query row (CLI: call once per group of layers and pass
  * the result to lsa_attend with layers_per_index = G).
  *
@@ -198,6 +203,13 @@ lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
 size_t lsa_attend_workspace_size(const lsa_batch_t *batch, int32_t H_q,
                                  int32_t H_kv, int32_t d, int32_t budget,
                                  int32_t layers_per_index);
+
+/* Number of kernel launches lsa_attend issues for this shape (host fields
+ * only): the attention kernel, plus a merge kernel when the budget is split
+ * over several CTAs per row. 0 for an invalid shape. */
+int32_t lsa_attend_launches(const lsa_batch_t *batch, int32_t H_q,
+                            int32_t H_kv, int32_t d, int32_t budget,
+                            int32_t layers_per_index);
 
 /* o[g][r][h] = softmax_j(q . k_j / sqrt(d)) v_j over the entries j of
  * index_sets[r] that are not -1, for every layer g < layers_per_index

@@ -118,6 +118,10 @@ def load_library():
     lib.lsa_hi_block_sums.argtypes = [vp, i32, i32, ctypes.POINTER(_Batch), i32, vp, i64, vp, vp]
     lib.lsa_index_workspace_size.restype = sz
     lib.lsa_index_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
+    lib.lsa_index_launches.restype = i32
+    lib.lsa_index_launches.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
+    lib.lsa_attend_launches.restype = i32
+    lib.lsa_attend_launches.argtypes = [ctypes.POINTER(_Batch), i32, i32, i32, i32, i32]
     lib.lsa_index_uses_tensor_cores.restype = i32
     lib.lsa_index_uses_tensor_cores.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
     lib.lsa_index.restype = i32
@@ -168,6 +172,18 @@ def lsa_hi_block_sums(k_idx: torch.Tensor, hi_block: int, batch: Batch, block_su
 def lsa_index_workspace_size(batch: Batch, H_I: int, d_I: int, budget: Budget) -> int:
     cb = batch.c()
     return int(load_library().lsa_index_workspace_size(ctypes.byref(cb), H_I, d_I, budget.c()))
+
+
+def lsa_index_launches(batch: Batch, H_I: int, d_I: int, budget: Budget) -> int:
+    """Kernel launches lsa_index issues for this shape."""
+    cb = batch.c()
+    return int(load_library().lsa_index_launches(ctypes.byref(cb), H_I, d_I, budget.c()))
+
+
+def lsa_attend_launches(batch: Batch, H_q: int, H_kv: int, d: int, budget: int, layers: int) -> int:
+    """Kernel launches lsa_attend issues for this shape."""
+    cb = batch.c()
+    return int(load_library().lsa_attend_launches(ctypes.byref(cb), H_q, H_kv, d, budget, layers))
 
 
 def lsa_index_uses_tensor_cores(batch: Batch, H_I: int, d_I: int, budget: Budget) -> bool:

@@ -138,6 +138,15 @@ int32_t lsa_index_uses_tensor_cores(const lsa_batch_t* batch, int32_t H_I, int32
     return index_dense(batch, H_I, d_I, budget) ? 1 : 0;
 }
 
+int32_t lsa_index_launches(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, lsa_budget_t budget) {
+    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1 || !budget_ok(budget)) return 0;
+    (void)d_I;
+    if (budget.hi_block == 0) return 2;  // fine scores, token selection
+    const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget);
+    const bool fused = lsa::coarse_in_select(budget.hi_block, plan.coarse_stage, H_I, batch->n_q);
+    return (fused ? 1 : 2) + 2;  // [coarse scores,] block selection, fine scores, token selection
+}
+
 static lsa_status_t index_validate(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max,
                                    int32_t H_I, int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget,
                                    const int8_t* block_sums, int64_t block_rows, const int32_t* index_sets) {
@@ -246,6 +255,14 @@ size_t lsa_attend_workspace_size(const lsa_batch_t* batch, int32_t H_q, int32_t 
     lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, budget, layers_per_index,
                                          lsa::device_sm_count());
     return p.ws_bytes;
+}
+
+int32_t lsa_attend_launches(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, int32_t budget,
+                            int32_t layers_per_index) {
+    if (batch == nullptr || batch->n_q <= 0 || !attend_shape_ok(H_q, H_kv, d, budget, layers_per_index)) return 0;
+    const lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, budget, layers_per_index,
+                                               lsa::device_sm_count());
+    return p.n_splits > 1 ? 2 : 1;  // attention[, split merge]
 }
 
 lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache, const uint16_t* const* v_cache,

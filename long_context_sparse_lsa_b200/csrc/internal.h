@@ -97,9 +97,10 @@ cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
 // there are enough rows for the clusters to cover the GPU (with a few rows
 // the coarse scoring kernel spreads the block sums over more SMs); otherwise
 // the coarse scoring kernel writes the scores to the workspace first.
-inline bool coarse_in_select(const IndexArgs& a) {
-    return a.hi_block > 0 && a.coarse_stage > 0 && a.H_I <= 16 && a.n_q >= 8;
+inline bool coarse_in_select(int hi_block, int coarse_stage, int H_I, int n_q) {
+    return hi_block > 0 && coarse_stage > 0 && H_I <= 16 && n_q >= 8;
 }
+inline bool coarse_in_select(const IndexArgs& a) { return coarse_in_select(a.hi_block, a.coarse_stage, a.H_I, a.n_q); }
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
                                 cudaStream_t stream);
 

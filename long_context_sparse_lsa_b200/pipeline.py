@@ -117,11 +117,9 @@ class LsaStep:
             self.graphs[name].replay()
 
     def kernels_per_step(self) -> int:
-        """Kernel launches of one step: the block-sum update (HI), the index
-        call's scoring and selection kernels (coarse ones only with HI) and the
-        attention kernel, plus its merge kernel when the call splits the
-        budget (it then asks for a partials workspace)."""
-        hi = self.block_sums is not None
-        ws_a = lsa.lsa_attend_workspace_size(self.batch, self.wl.H_q, self.wl.H_kv, self.wl.d, self.budget.length,
-                                             self.G)
-        return (1 if hi else 0) + (4 if hi else 2) + 1 + (1 if ws_a > 256 else 0)
+        """Kernel launches of one step: the block-sum update (HI) and the
+        launches the index and attention calls report for this shape."""
+        wl = self.wl
+        n_idx = lsa.lsa_index_launches(self.batch, wl.H_I, wl.d_I, self.budget)
+        n_att = lsa.lsa_attend_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
+        return (1 if self.block_sums is not None else 0) + n_idx + n_att

@@ -111,3 +111,31 @@ def test_attend_rejects_and_sizes():
     assert need >= 16 * 4
     need4 = lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 4)
     assert need4 >= 4 * 16 * 4  # counters for every (layer, row)
+
+
+def test_launch_counts_follow_the_shape():
+    """The calls report how many kernels they launch (host fields only)."""
+    import torch
+
+    from long_context_sparse_lsa_b200 import workloads as wls
+
+    def batch(n_seq, L, n_q=None):
+        n_q = n_q or n_seq
+        return lsa.Batch(torch.arange(n_seq, dtype=torch.int64) * L, torch.full((n_seq,), L, dtype=torch.int32),
+                         torch.arange(n_q, dtype=torch.int32) % n_seq, torch.full((n_q,), L, dtype=torch.int32), L,
+                         n_seq * L, torch.arange(n_seq, dtype=torch.int64) * ((L + 63) // 64))
+
+    hi = lsa.Budget(64, 1024, 2048, 64, 256)
+    flat = lsa.Budget(64, 1024, 2048, 0, 0)
+    # 16 rows, 16 heads: coarse scores inside the block selection (3 launches)
+    assert lsa.lsa_index_launches(batch(16, 131072), 16, 128, hi) == 3
+    # one row: the coarse scoring kernel runs on its own (4 launches)
+    assert lsa.lsa_index_launches(batch(1, 131072), 16, 128, hi) == 4
+    # more than 16 indexer heads: separate coarse kernel
+    assert lsa.lsa_index_launches(batch(16, 131072), 20, 128, hi) == 4
+    # HI off: fine scores + token selection
+    assert lsa.lsa_index_launches(batch(16, 131072), 16, 128, flat) == 2
+    # attention: split over CTAs (+ merge) for few rows, one CTA per row for many
+    assert lsa.lsa_attend_launches(batch(16, 131072), 32, 4, 128, 3136, 1) == 2
+    assert lsa.lsa_attend_launches(batch(1, 300000, n_q=8192), 32, 4, 128, 3136, 1) == 1
+    assert lsa.lsa_attend_launches(batch(16, 131072), 32, 4, 96, 3136, 1) == 0  # d != 128: unsupported
