@@ -140,7 +140,9 @@ def _ncu_traffic(kernel_hash: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms (the bench
+    samples over a 0.6 s burst of replayed steps just before the timed steps
+    and through them)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -331,7 +333,15 @@ def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
     if st.status_bits() != 0:
         raise RuntimeError(f"device status {st.status_bits():#x} after warm-up ({wl.name})")
     if clocks is not None:
+        # the timed steps last milliseconds, nvidia-smi samples every 200 ms:
+        # sample over ~0.6 s of the same step replayed back to back right
+        # before the timed steps, and through them
         clocks.start()
+        t_end = time.perf_counter() + 0.6
+        while time.perf_counter() < t_end:
+            for _ in range(64):
+                st.replay()
+            torch.cuda.synchronize()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()

@@ -750,7 +750,9 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     }
     p.fine_cap = (p.fine_cap + 3) / 4 * 4;
     if (p.fine_cap < 4) p.fine_cap = 4;
-    p.cluster = 8;
+    // a few rows (the 1M decode has one): 16 CTAs per row (non-portable
+    // cluster size) halve each CTA's slice; otherwise 8
+    p.cluster = n_q <= 4 ? 16 : 8;
     // largest slice: whole 32-key words split over the cluster
     auto slice_max = [&](int cap) { return 32 * (((cap + 31) / 32 + p.cluster - 1) / p.cluster); };
     if (hi) {
