@@ -575,6 +575,7 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
         tile(i, ka, va);
         if (i + n_sel < n_tiles) tile(i + n_sel, kb2, vb2);
     }
+    pdl_trigger();  // only the head merge and the stores are left
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -662,6 +663,11 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
     const size_t stage = (size_t)kTile * p.row_stride;
     int ns = (int)((kAtSmemBudget - ent - 2 * kMaxStages * 8 - 128) / stage);
     if (ns > kMaxStages) ns = kMaxStages;
+    // tile i uses stage i mod ns and the warps of wsel i mod (8 / hpc): with ns
+    // a multiple of that, every use of a stage has the same warps, which saw
+    // its previous phase complete before they wait on the next one
+    const int n_sel = kConsumers / p.hpc;
+    if (ns >= n_sel) ns = ns / n_sel * n_sel;
     p.n_stages = ns;
     p.bar_off = (int)ent;
     p.stage_off = (int)(ent + ((2 * kMaxStages * 8 + 127) / 128) * 128);

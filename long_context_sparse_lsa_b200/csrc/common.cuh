@@ -26,6 +26,10 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 // grid.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_enter() { pdl_wait(); }
+// Lets the next kernel on the stream be launched before this grid ends; the
+// next kernel still waits (pdl_wait) for this grid's completion and memory
+// flush, so this only moves its launch latency under this grid's tail.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
 __device__ __forceinline__ void flag(int32_t* status, int32_t bits) {

@@ -174,15 +174,20 @@ __global__ void __launch_bounds__(kScThreads, kFineCtasPerSm) fine_score_kernel(
 // Fine scores with HI on, d_I = 128, hi_block a multiple of 16: the kept
 // blocks are contiguous runs of key rows, so each one (or each 64-row part)
 // arrives as one TMA tensor copy (128-byte swizzle) instead of per-lane
-// gathers. A persistent CTA per SM takes a contiguous range of (row, kept
-// block, part) items. The producer warp looks up 32 items' kept-block ids
-// at once, then one lane issues their copies into a ring of 24 stages; item
-// k goes to stage k mod 24 and consumer warp k mod 8, which scores its
-// 16-row tiles from shared memory (the swizzle spreads the 8 rows a load
-// reads over all banks) and releases the stage.
-constexpr int kFtConsumers = 8;
+// gathers. Two persistent CTAs per SM each take a contiguous range of (row,
+// kept block, part) items. The producer warp looks up 32 items' kept-block
+// ids at once, then one lane issues their copies into a ring of kFtStages
+// stages; item k goes to stage k mod kFtStages and consumer warp k mod
+// kFtConsumers, which scores its 16-row tiles from shared memory (the swizzle
+// spreads the 8 rows a load reads over all banks) and releases the stage.
+constexpr int kFtConsumers = 6;
 constexpr int kFtThreads = (kFtConsumers + 1) * kWarp;
-constexpr int kFtStages = 24;
+constexpr int kFtCtasPerSm = 2;
+constexpr int kFtStages = 12;
+// Stage k mod S always goes to consumer k mod C, so every use of a stage has
+// the same consumer, which has seen the stage's previous phase complete
+// before it waits on the next one (a parity wait cannot tell them apart).
+static_assert(kFtStages % kFtConsumers == 0, "each stage needs a single consumer warp");
 constexpr int kFtRows = 64;                   // key rows per item (box rows)
 constexpr int kFtStageBytes = kFtRows * 128;  // 8 KB
 
@@ -212,7 +217,7 @@ struct FtShared {
 constexpr size_t kFtSmem = 1024 + (size_t)kFtStages * kFtStageBytes + sizeof(FtShared);
 
 template <int NT>
-__global__ void __launch_bounds__(kFtThreads, 1) fine_score_tma_kernel(const __grid_constant__ FineTmaArgs p) {
+__global__ void __launch_bounds__(kFtThreads, kFtCtasPerSm) fine_score_tma_kernel(const __grid_constant__ FineTmaArgs p) {
     pdl_enter();
     const IndexArgs& a = p.a;
     extern __shared__ __align__(16) uint8_t ft_raw[];
@@ -295,6 +300,7 @@ __global__ void __launch_bounds__(kFtThreads, 1) fine_score_tma_kernel(const __g
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             __syncwarp();
         }
+        pdl_trigger();  // every copy is issued
         // one end marker per consumer warp
         if (lane == 0) {
             for (int w = 0; w < kFtConsumers; ++w) {
@@ -375,7 +381,8 @@ cudaError_t launch_fine_tma(const IndexArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(fine_score_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kFtSmem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(fine_score_tma_kernel<NT>, dim3((unsigned)device_sm_count()), dim3(kFtThreads), kFtSmem, st, 0,
+    return launch_pdl(fine_score_tma_kernel<NT>, dim3((unsigned)(kFtCtasPerSm * device_sm_count())), dim3(kFtThreads),
+                      kFtSmem, st, 0,
                       p);
 }
 

@@ -682,6 +682,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     const uint32_t want = (uint32_t)(kTokens ? a.topk : a.hi_topblocks);
     uint32_t tb, above, in_bin;
     const uint32_t total = find_bin(sh, want, tb, above, in_bin);
+    pdl_trigger();  // what is left is the threshold and the compaction
     const uint32_t k = min(want, total);
     if (k > 0u) {
         K thr = K(1);
