@@ -600,7 +600,7 @@ __global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_consta
     const float* P = a.part_o + (row_q * a.n_splits * a.H_q + h) * kD;
     const float* PML = a.part_ml + (row_q * a.n_splits * a.H_q + h) * 2;
     const int64_t pstride = (int64_t)a.H_q;  // between consecutive splits, in rows
-    constexpr int kU = 8;
+    constexpr int kU = 16;  // up to 16 splits in one round of loads
     float M = -INFINITY, den = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int p0 = 0; p0 < a.n_splits; p0 += kU) {

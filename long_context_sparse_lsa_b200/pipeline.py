@@ -107,8 +107,38 @@ class LsaStep:
             else:
                 self.step()
         self.graphs["step"] = g
+        # the same step with timing events recorded around the index and
+        # attention calls inside the graph: their durations within a step,
+        # without the launch of a graph of their own
+        ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
+        self.call_events = {"index": (ev(), ev()), "attend": (ev(), ev())}
+        (ix0, ix1), (at0, at1) = self.call_events["index"], self.call_events["attend"]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            cur = torch.cuda.current_stream(self.device)
+            overlap = self.overlap_ok(1)
+            if overlap:
+                fork.wait_stream(cur)
+                with torch.cuda.stream(fork):
+                    self.update_block_sums(1)
+            else:
+                self.update_block_sums(1)
+            ix0.record(cur)
+            self.index()
+            ix1.record(cur)
+            if overlap:
+                cur.wait_stream(fork)
+            at0.record(cur)
+            self.attend()
+            at1.record(cur)
+        self.graphs["step_timed"] = g
         torch.cuda.synchronize(self.device)
         return self.graphs
+
+    def call_ms(self) -> dict:
+        """Index and attention durations (ms) inside the last replay of the
+        "step_timed" graph; call after it has completed."""
+        return {k: a.elapsed_time(b) for k, (a, b) in self.call_events.items()}
 
     def replay(self, name: str | None = None):
         """Replay one captured graph, or the whole step when name is None."""

@@ -250,4 +250,15 @@ def test_graph_replay_matches_eager():
     np.testing.assert_array_equal(parity.host(st.sets), sets0)
     for g in range(len(outs0)):
         np.testing.assert_array_equal(parity.host(st.out[g]), outs0[g])
+    # the step graph with timing events inside computes the same and times both calls
+    st.sets.fill_(-5)
+    for o in st.out:
+        o.fill_(float("nan"))
+    st.replay("step_timed")
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(parity.host(st.sets), sets0)
+    for g in range(len(outs0)):
+        np.testing.assert_array_equal(parity.host(st.out[g]), outs0[g])
+    ms = st.call_ms()
+    assert 0.0 < ms["index"] < 1000.0 and 0.0 < ms["attend"] < 1000.0
     parity.check_sets(sets0, parity.oracle_sets(wl, t), "graph")
