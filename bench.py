@@ -53,7 +53,6 @@ def step_bytes(wl) -> dict:
         e = min(L, wl.budget)
         attend += G * (2 * e * kv_row + wl.H_q * wl.d * 2 + wl.H_q * wl.d * 4 + wl.budget * 4)
     index = 0
-    bsum = 0
     for L in rows:
         s = min(wl.sink, L)
         ws = max(s, L - wl.window)
@@ -62,13 +61,29 @@ def step_bytes(wl) -> dict:
             nb = (ws + B - 1) // B - s // B if ws > s else 0
             kept = min(nb, wl.hi_topblocks)
             index += nb * 2 * wl.d_I + kept * B * wl.d_I  # block sums read + kept keys
-            bsum += B * wl.d_I + 2 * wl.d_I  # append update: re-read one block, write one row
         else:
             index += (ws - s) * wl.d_I
         index += wl.H_I * wl.d_I + wl.H_I * 4 + wl.budget * 4  # q, w, index-set write
     if wl.prefill_new:  # one cache shared by every row of the chunk: read it once
         index = wl.lens[0] * wl.d_I + n_q * (wl.H_I * wl.d_I + wl.H_I * 4 + wl.budget * 4)
-    return {"attend": attend, "index": index, "block_sums": bsum, "total": attend + index + bsum}
+    # decode append per sequence: the new tokens' key and K/V rows read and
+    # written once; with HI on, one block of keys re-read and its sum written
+    app = 0
+    if not wl.prefill_new:
+        for L in wl.lens:
+            app += 2 * wl.drafts * (wl.d_I + 2 * G * kv_row)
+            if wl.hi_block > 0:
+                app += wl.hi_block * wl.d_I + 2 * wl.d_I
+    return {"attend": attend, "index": index, "append": app, "total": attend + index + app}
+
+
+def cold_block_sum_bytes(wl) -> int:
+    """Bytes of a full block-sum build: every cached key read once, every
+    block's two byte planes written once."""
+    if wl.hi_block <= 0:
+        return 0
+    nb = sum((L + wl.hi_block - 1) // wl.hi_block for L in wl.lens)
+    return wl.total_tokens * wl.d_I + nb * 2 * wl.d_I
 
 
 def _rows(wl):
@@ -76,7 +91,7 @@ def _rows(wl):
     if wl.prefill_new:
         C = wl.lens[0] - wl.prefill_new
         return [C + i + 1 for i in range(wl.prefill_new)]
-    return list(wl.lens)
+    return [L - wl.drafts + 1 + j for L in wl.lens for j in range(wl.drafts)]
 
 
 def index_int8_ops(wl) -> int:
@@ -307,7 +322,7 @@ def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
     st.capture()
 
     def one_step(evs):
-        """The timed step: the captured step graph (block-sum update beside
+        """The timed step: the captured step graph (the append beside
         the index call when the two touch disjoint rows, then attention)."""
         flush.fill_(1)
         evs[0].record(stream)
@@ -318,7 +333,7 @@ def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
         """The three calls one after another, for the per-call breakdown."""
         flush.fill_(1)
         evs[0].record(stream)
-        st.replay("block_sums")
+        st.replay("append")
         evs[1].record(stream)
         st.replay("index")
         evs[2].record(stream)
@@ -366,12 +381,37 @@ def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
         st.replay("step_timed")
         torch.cuda.synchronize()
         in_step.append(st.call_ms())
+    # cold steps: the block sums rebuilt from the whole key cache inside each
+    # step (nothing resident between steps), then index and attention
+    cold = []
+    if "cold" in st.graphs:
+        cevs = [ev(2) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(1)
+            cevs[i][0].record(stream)
+            st.replay("cold")
+            cevs[i][1].record(stream)
+        torch.cuda.synchronize()
+        cold = [e[0].elapsed_time(e[1]) for e in cevs]
     if st.status_bits() != 0:
         raise RuntimeError(f"device status {st.status_bits():#x} after timing ({wl.name})")
-    return {"st": st, "t": t, "ms": ms, "clocks": clk, "n_kernels": st.kernels_per_step(),
+    return {"st": st, "t": t, "ms": ms, "clocks": clk, "n_kernels": st.kernels_per_step(), "cold": cold,
             "bs": [e[0].elapsed_time(e[1]) for e in sevs], "ix": [e[1].elapsed_time(e[2]) for e in sevs],
             "at": [e[2].elapsed_time(e[3]) for e in sevs],
             "ix_in_step": [c["index"] for c in in_step], "at_in_step": [c["attend"] for c in in_step]}
+
+
+def cold_line(wl, cold_ms, world, pg, dev):
+    """The cold-step numbers (block sums rebuilt inside every step), or None
+    when the workload has HI off."""
+    if not cold_ms:
+        return None
+    ms = max_over_ranks(sum(cold_ms) / len(cold_ms), pg, dev)
+    byts = step_bytes(wl)["total"] - step_bytes(wl)["append"] + cold_block_sum_bytes(wl)
+    return {"value": job_rate(wl.n_q, world, ms), "unit": UNIT, "ms_per_step": ms,
+            "algorithmic_bytes_per_step": byts, "step_gbs": byts / (ms / 1000.0) / 1e9,
+            "note": "block sums rebuilt from the whole key cache inside every step (full build, "
+                    "then index, then attention; one CUDA graph, L2 flushed before each step)"}
 
 
 def secondary(dev, flush, stream, steps, warmup, peak):
@@ -388,9 +428,10 @@ def secondary(dev, flush, stream, steps, warmup, peak):
         byts = step_bytes(wl)
         ix, at = mean(run["ix_in_step"]), mean(run["at_in_step"])
         rec = {"ms_per_step": ms, "steps": steps, "warmup": warmup,
-               "step_breakdown_ms": {"block_sums_update": mean(run["bs"]), "index": mean(run["ix"]),
+               "step_breakdown_ms": {"append": mean(run["bs"]), "index": mean(run["ix"]),
                                      "attend": mean(run["at"])},
                "call_ms_in_step": {"index": ix, "attend": at},
+               "cold": cold_line(wl, run["cold"], 1, None, dev),
                "algorithmic_bytes_per_step": byts,
                "step_gbs": byts["total"] / (ms / 1000.0) / 1e9,
                "step_frac_of_measured_hbm": byts["total"] / (ms / 1000.0) / 1e9 / peak,
@@ -471,8 +512,12 @@ def main(argv=None):
     pin = lambda x: x.cpu().pin_memory()
     h_q_idx, h_w = pin(t.q_idx), pin(t.w)
     h_q = [pin(x) for x in t.q]
+    # the appended tokens' rows come from the host too (the decode append)
+    d_new = ([st.k_idx_new] + st.k_new + st.v_new) if st.n_new else []
+    h_new = [pin(x) for x in d_new]
     h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.out]
-    h2d = h_q_idx.numel() + h_w.numel() * 4 + sum(x.numel() * 2 for x in h_q)
+    h2d = (h_q_idx.numel() + h_w.numel() * 4 + sum(x.numel() * 2 for x in h_q) +
+           sum(x.numel() * x.element_size() for x in h_new))
     d2h = sum(o.numel() * 4 for o in st.out)
     e2e_ms = []
     for i in range(args.warmup + args.steps):
@@ -483,6 +528,8 @@ def main(argv=None):
         t.w.copy_(h_w, non_blocking=True)
         for g in range(len(h_q)):
             t.q[g].copy_(h_q[g], non_blocking=True)
+        for dst, src in zip(d_new, h_new):
+            dst.copy_(src, non_blocking=True)
         st.replay()
         for g in range(len(h_out)):
             h_out[g].copy_(st.out[g], non_blocking=True)
@@ -521,10 +568,11 @@ def main(argv=None):
                                                             "hi_topblocks": wl.hi_topblocks},
                        "heads": {"H_I": wl.H_I, "d_I": wl.d_I, "H_q": wl.H_q, "H_kv": wl.H_kv, "d": wl.d},
                        "l2": "flushed before every timed step (2 x L2 write, outside the timed interval)",
-                       "launch": "each step replayed from one CUDA graph captured through the C ABI (block-sum update on a forked stream beside the index call); step_breakdown_ms from per-call graphs replayed in sequence (each with its own graph launch); call_ms_in_step from timing events inside the step graph",
+                       "launch": "each step replayed from one CUDA graph captured through the C ABI (the decode append -- new tokens' keys and K/V rows written, their block sums refreshed -- on a forked stream beside the index call); step_breakdown_ms from per-call graphs replayed in sequence (each with its own graph launch); call_ms_in_step from timing events inside the step graph",
                        "parallelism": f"replicas x{world} (independent batches, no collective)"},
-            "step_breakdown_ms": {"block_sums_update": bsu, "index": ix, "attend": at},
+            "step_breakdown_ms": {"append": bsu, "index": ix, "attend": at},
             "call_ms_in_step": {"index": ix_in, "attend": at_in},
+            "cold": cold_line(wl, run["cold"], world, pg, dev),
             "step_gbs": byts["total"] / (ms / 1000.0) / 1e9,
             "step_frac_of_measured_hbm": byts["total"] / (ms / 1000.0) / 1e9 / peak,
             "step_frac_of_8tbs": byts["total"] / (ms / 1000.0) / 1e9 / 8000.0,

@@ -146,6 +146,40 @@ lsa_status_t lsa_hi_block_sums(const int8_t *k_idx_cache, int32_t d_I,
                                void *stream);
 
 /* ----------------------------------------------------------------------- */
+/* Decode append                                                             */
+/* ----------------------------------------------------------------------- */
+/* Writes the n_new newest tokens of every sequence into the caches and, with
+ * HI on, refreshes the block sums of the blocks that hold them, in one
+ * launch: the step just before indexing in a decode loop, so that the block
+ * sums stay resident and exact as the cache grows (the HI block pass of the
+ * Flash-Lite-Sparse page, "기술적 특징", Hierarchical Indexing bullet, over
+ * a cache that gains a token per step).
+ *
+ * For sequence b the new tokens are positions seq_lens[b] - n_new ..
+ * seq_lens[b] - 1 (seq_lens already counts them; 1 <= n_new <= seq_lens[b],
+ * else LSA_DEV_BAD_LENGTH and the sequence is skipped).
+ * k_idx_new    device int8 [n_seq][n_new][d_I]: the new indexer keys.
+ * k_idx_cache  device int8 [total_tokens][d_I], written at the new positions.
+ * k_new, v_new host [layers] arrays of device bf16 [n_seq][n_new][H_kv][d].
+ * k_cache, v_cache host [layers] arrays of device bf16
+ *              [total_tokens][H_kv][d], written at the new positions.
+ *              layers may be 0 (indexer keys only); the arrays may then be NULL.
+ * block_sums   as for lsa_hi_block_sums, or NULL when hi_block == 0. The
+ *              refreshed blocks are summed from the new keys (read from
+ *              k_idx_new) and the older keys of the block (from the cache).
+ * All device pointers 16-byte aligned; the inputs must not overlap the
+ * cache rows being written. Supported: d_I in {32, 64, 128}; d == 128;
+ * 0 <= layers <= LSA_MAX_LAYERS; 0 <= hi_block <= LSA_MAX_HI_BLOCK.
+ */
+lsa_status_t lsa_append(const int8_t *k_idx_new, int8_t *k_idx_cache, int32_t d_I,
+                        const uint16_t *const *k_new, const uint16_t *const *v_new,
+                        uint16_t *const *k_cache, uint16_t *const *v_cache,
+                        int32_t H_kv, int32_t d, int32_t layers, int32_t hi_block,
+                        int8_t *block_sums, int64_t block_rows,
+                        const lsa_batch_t *batch, int32_t n_new,
+                        int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------------------------------- */
 /* Indexer: scores, HI, top-k, SI assembly                                   */
 /* ----------------------------------------------------------------------- */
 /* Workspace bytes lsa_index needs for this batch shape (reads only the host

@@ -25,7 +25,7 @@ LSA_DEV_TIMEOUT = 0x10
 STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "LSA_ERR_CUDA",
           4: "LSA_ERR_WORKSPACE"}
 
-EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums",
+EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums", "lsa_append",
            "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend",
            "lsa_attend_noalloc"]
 
@@ -116,6 +116,9 @@ def load_library():
     lib.lsa_status_string.argtypes = [i32]
     lib.lsa_hi_block_sums.restype = i32
     lib.lsa_hi_block_sums.argtypes = [vp, i32, i32, ctypes.POINTER(_Batch), i32, vp, i64, vp, vp]
+    lib.lsa_append.restype = i32
+    lib.lsa_append.argtypes = [vp, vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                               ctypes.POINTER(vp), i32, i32, i32, i32, vp, i64, ctypes.POINTER(_Batch), i32, vp, vp]
     lib.lsa_index_workspace_size.restype = sz
     lib.lsa_index_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
     lib.lsa_index_launches.restype = i32
@@ -209,6 +212,24 @@ def lsa_index(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, w_max: 
 def lsa_attend_workspace_size(batch: Batch, H_q: int, H_kv: int, d: int, budget: int, layers: int) -> int:
     cb = batch.c()
     return int(load_library().lsa_attend_workspace_size(ctypes.byref(cb), H_q, H_kv, d, budget, layers))
+
+
+def lsa_append(k_idx_new: torch.Tensor, k_idx: torch.Tensor, k_new: list, v_new: list, k: list, v: list,
+               hi_block: int, block_sums: torch.Tensor | None, batch: Batch, n_new: int,
+               dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """Write the n_new newest tokens of every sequence (keys k_idx_new [n_seq, n_new, d_I], per-layer K/V
+    rows k_new/v_new [n_seq, n_new, H_kv, d]) into the caches and refresh their blocks' sums (HI on)."""
+    lib = load_library()
+    G = len(k_new)
+    d_I = k_idx.shape[-1]
+    H_kv, d = (k[0].shape[1], k[0].shape[2]) if G else (0, 0)
+    arr = ctypes.c_void_p * max(G, 1)
+    kn, vn, kc, vc = (arr(*[t.data_ptr() for t in x]) for x in (k_new, v_new, k, v))
+    cb = batch.c()
+    rows = block_sums.shape[0] if block_sums is not None else 0
+    st = lib.lsa_append(_ptr(k_idx_new), _ptr(k_idx), d_I, kn, vn, kc, vc, H_kv, d, G, hi_block, _ptr(block_sums),
+                        rows, ctypes.byref(cb), n_new, _ptr(dev_status), _stream(stream))
+    _check("lsa_append", st)
 
 
 def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list,

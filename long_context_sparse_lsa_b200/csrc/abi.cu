@@ -115,6 +115,61 @@ lsa_status_t lsa_hi_block_sums(const int8_t* k_idx_cache, int32_t d_I, int32_t h
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 
+lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_I, const uint16_t* const* k_new,
+                        const uint16_t* const* v_new, uint16_t* const* k_cache, uint16_t* const* v_cache,
+                        int32_t H_kv, int32_t d, int32_t layers, int32_t hi_block, int8_t* block_sums,
+                        int64_t block_rows, const lsa_batch_t* batch, int32_t n_new, int32_t* dev_status,
+                        void* stream) {
+    if (!batch_ok(batch, false)) return LSA_ERR_INVALID_ARG;
+    if (n_new < 1 || d_I < 1 || layers < 0 || hi_block < 0 || block_rows < 0) return LSA_ERR_INVALID_ARG;
+    if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+    if (hi_block > LSA_MAX_HI_BLOCK || layers > LSA_MAX_LAYERS) return LSA_ERR_UNSUPPORTED;
+    if (k_idx_new == nullptr || k_idx_cache == nullptr || !aligned(k_idx_new, 16) || !aligned(k_idx_cache, 16))
+        return LSA_ERR_INVALID_ARG;
+    if (hi_block > 0 && (block_sums == nullptr || batch->blk_offset == nullptr || !aligned(block_sums, 16)))
+        return LSA_ERR_INVALID_ARG;
+    if (layers > 0) {
+        if (d != 128 || H_kv < 1) return d != 128 ? LSA_ERR_UNSUPPORTED : LSA_ERR_INVALID_ARG;
+        if (k_new == nullptr || v_new == nullptr || k_cache == nullptr || v_cache == nullptr)
+            return LSA_ERR_INVALID_ARG;
+        for (int g = 0; g < layers; ++g) {
+            if (k_new[g] == nullptr || v_new[g] == nullptr || k_cache[g] == nullptr || v_cache[g] == nullptr)
+                return LSA_ERR_INVALID_ARG;
+            if (!aligned(k_new[g], 16) || !aligned(v_new[g], 16) || !aligned(k_cache[g], 16) ||
+                !aligned(v_cache[g], 16))
+                return LSA_ERR_INVALID_ARG;
+        }
+    }
+    if (batch->n_seq > 65535) return LSA_ERR_UNSUPPORTED;
+    lsa::AppendArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.bs.k_idx = k_idx_cache;
+    a.bs.block_sums = block_sums;
+    a.bs.kv_offset = batch->kv_offset;
+    a.bs.seq_lens = batch->seq_lens;
+    a.bs.blk_offset = batch->blk_offset;
+    a.bs.dev_status = dev_status;
+    a.bs.total_tokens = batch->total_tokens;
+    a.bs.block_rows = block_rows;
+    a.bs.n_seq = batch->n_seq;
+    a.bs.max_len = batch->max_len;
+    a.bs.hi_block = hi_block;
+    a.bs.n_new = n_new;
+    a.k_idx_new = k_idx_new;
+    a.k_idx_cache = k_idx_cache;
+    for (int g = 0; g < layers; ++g) {
+        a.k_new[g] = k_new[g];
+        a.v_new[g] = v_new[g];
+        a.k_cache[g] = k_cache[g];
+        a.v_cache[g] = v_cache[g];
+    }
+    a.layers = layers;
+    a.kv_row_bytes = layers > 0 ? H_kv * d * 2 : 0;
+    a.sums = hi_block > 0 ? 1 : 0;
+    cudaError_t e = lsa::launch_append(a, d_I, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
 // ---------------------------------------------------------------------------
 size_t lsa_index_workspace_size(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, lsa_budget_t budget) {
     (void)H_I;

@@ -1,4 +1,5 @@
-// block_sums.cu — HI block-sum pre-pass.
+// block_sums.cu — HI block-sum pre-pass, and the decode append that writes
+// the newest tokens' keys and K/V rows and refreshes their blocks' sums.
 //
 // Hierarchical Indexing first scores whole blocks ("LongCat-Flash-Lite-Sparse
 // (aitrends.kr)", section "기술적 특징", HI bullet). The block score uses the
@@ -21,46 +22,22 @@ constexpr int kBsWarps = kBsThreads / kWarp;
 
 __device__ __forceinline__ int sbyte(uint32_t w, int i) { return static_cast<int>(static_cast<int8_t>(w >> (8 * i))); }
 
-// One CTA per block: thread t owns 16-byte chunk (t % CPR) of rows t / CPR,
-// t / CPR + RPP, ... so the whole block is read in B / RPP dependent rounds
-// of coalesced 16-byte loads (one round for hi_block <= 32 at d_I = 128).
-template <int D_I>
-__global__ void __launch_bounds__(kBsThreads) block_sums_kernel(const BlockSumArgs a) {
-    pdl_enter();
+// Thread t owns 16-byte chunk (t % CPR) of rows t / CPR, t / CPR + RPP, ...
+// of the block, so the block is read in B / RPP dependent rounds of coalesced
+// 16-byte loads (one round for hi_block <= 32 at d_I = 128). row_ptr(i) is
+// the address of the block's row i; the sum of rows [0, n) goes to out_row as
+// the two byte planes. Every thread of the CTA calls it (one CTA barrier).
+template <int D_I, typename RowPtr>
+__device__ __forceinline__ void sum_block(RowPtr row_ptr, int n, int8_t* out_row, int (&s_part)[kBsWarps][D_I]) {
     constexpr int kCPR = D_I / 16;           // 16-byte chunks per row
     constexpr int kRPP = kBsThreads / kCPR;  // rows per pass
-    __shared__ int s_part[kBsWarps][D_I];
-    const int seq = blockIdx.y;
     const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
-    const int64_t off = a.kv_offset[seq];
-    const int32_t len = a.seq_lens[seq];
-    if (len < 1 || len > a.max_len || off < 0 || off + len > a.total_tokens) {
-        if (tid == 0 && blockIdx.x == 0) flag(a.dev_status, LSA_DEV_BAD_LENGTH);
-        return;
-    }
-    const int B = a.hi_block;
-    const int nblk = (len + B - 1) / B;
-    const int64_t boff = a.blk_offset[seq];
-    if (boff < 0 || boff + nblk > a.block_rows) {
-        if (tid == 0 && blockIdx.x == 0) flag(a.dev_status, LSA_DEV_BAD_LENGTH);
-        return;
-    }
-    int first = 0;
-    if (a.n_new > 0) {
-        const int from = len - a.n_new;
-        first = from > 0 ? from / B : 0;
-    }
-    const int j = first + blockIdx.x;
-    if (j >= nblk) return;  // uniform over the CTA
-    const int t0 = j * B;
-    const int n = min(t0 + B, len) - t0;
     const int c = tid % kCPR;
     int acc[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) acc[i] = 0;
-    const int8_t* base = a.k_idx + (off + t0) * D_I + c * 16;
     for (int row = tid / kCPR; row < n; row += kRPP) {
-        const uint4 v = ldg16(base + (int64_t)row * D_I);
+        const uint4 v = ldg16(row_ptr(row) + c * 16);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -82,9 +59,114 @@ __global__ void __launch_bounds__(kBsThreads) block_sums_kernel(const BlockSumAr
 #pragma unroll
         for (int w2 = 0; w2 < kBsWarps; ++w2) S += s_part[w2][tid];
         // S = 256 * hi + lo with hi = S >> 8 (arithmetic), lo = S & 0xFF.
-        int8_t* row = a.block_sums + (boff + j) * (2 * D_I);
-        row[tid] = static_cast<int8_t>(S >> 8);
-        reinterpret_cast<uint8_t*>(row)[D_I + tid] = static_cast<uint8_t>(S & 0xFF);
+        out_row[tid] = static_cast<int8_t>(S >> 8);
+        reinterpret_cast<uint8_t*>(out_row)[D_I + tid] = static_cast<uint8_t>(S & 0xFF);
+    }
+}
+
+// The sequence's cache span and block rows, checked; false (and a status
+// bit) when they are out of range. The check is uniform over the CTA.
+__device__ __forceinline__ bool seq_ok(const BlockSumArgs& a, int seq, int64_t& off, int& len) {
+    off = a.kv_offset[seq];
+    len = a.seq_lens[seq];
+    bool ok = len >= 1 && len <= a.max_len && off >= 0 && off + len <= a.total_tokens;
+    if (ok && a.hi_block > 0) {
+        const int64_t boff = a.blk_offset[seq];
+        const int nblk = (len + a.hi_block - 1) / a.hi_block;
+        ok = boff >= 0 && boff + nblk <= a.block_rows;
+    }
+    if (!ok && threadIdx.x == 0 && blockIdx.x == 0) flag(a.dev_status, LSA_DEV_BAD_LENGTH);
+    return ok;
+}
+
+// One CTA per block (full build) or per block holding the n_new newest tokens
+// (append update).
+template <int D_I>
+__global__ void __launch_bounds__(kBsThreads) block_sums_kernel(const BlockSumArgs a) {
+    pdl_enter();
+    __shared__ int s_part[kBsWarps][D_I];
+    const int seq = blockIdx.y;
+    int64_t off;
+    int len;
+    if (!seq_ok(a, seq, off, len)) return;
+    const int B = a.hi_block;
+    const int nblk = (len + B - 1) / B;
+    int first = 0;
+    if (a.n_new > 0) {
+        const int from = len - a.n_new;
+        first = from > 0 ? from / B : 0;
+    }
+    const int j = first + blockIdx.x;
+    if (j >= nblk) return;  // uniform over the CTA
+    const int t0 = j * B;
+    const int n = min(t0 + B, len) - t0;
+    const int8_t* base = a.k_idx + (off + t0) * D_I;
+    sum_block<D_I>([&](int row) { return base + (int64_t)row * D_I; }, n,
+                   a.block_sums + (a.blk_offset[seq] + j) * (2 * D_I), s_part);
+}
+
+__device__ __forceinline__ void copy16(uint8_t* dst, const uint8_t* src, int64_t bytes) {
+    for (int64_t i = threadIdx.x; i < bytes / 16; i += kBsThreads)
+        reinterpret_cast<uint4*>(dst)[i] = ldg16(src + 16 * i);
+}
+
+constexpr int kAppendRowsPerCta = 64;  // HI off: new tokens per CTA
+
+// Decode append. CTA (x, b) owns the new tokens of sequence b that fall in
+// block first + x (HI on; the CTA also recomputes that block's sum) or the
+// x-th run of kAppendRowsPerCta new tokens (HI off). It copies their indexer
+// keys and every layer's K and V rows into the caches. The block sum reads
+// the new rows from the inputs and the older rows from the cache, so no CTA
+// reads what it (or another CTA) writes in this launch.
+template <int D_I>
+__global__ void __launch_bounds__(kBsThreads) append_kernel(const AppendArgs p) {
+    pdl_enter();
+    __shared__ int s_part[kBsWarps][D_I];
+    const BlockSumArgs& a = p.bs;
+    const int seq = blockIdx.y;
+    int64_t off;
+    int len;
+    if (!seq_ok(a, seq, off, len)) return;
+    const int n_new = a.n_new;
+    if (n_new > len) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) flag(a.dev_status, LSA_DEV_BAD_LENGTH);
+        return;
+    }
+    const int from = len - n_new;  // first new position
+    int lo, hi, t0 = 0, n = 0, j = 0;
+    if (p.sums) {
+        const int B = a.hi_block;
+        j = from / B + blockIdx.x;
+        if (j >= (len + B - 1) / B) return;  // uniform over the CTA
+        t0 = j * B;
+        n = min(t0 + B, len) - t0;
+        lo = max(t0, from);
+        hi = t0 + n;
+    } else {
+        lo = from + blockIdx.x * kAppendRowsPerCta;
+        hi = min(len, lo + kAppendRowsPerCta);
+        if (lo >= hi) return;
+    }
+    const int64_t src0 = (int64_t)seq * n_new + (lo - from);  // first input row
+    const int nr = hi - lo;
+    copy16(reinterpret_cast<uint8_t*>(p.k_idx_cache) + (off + lo) * D_I,
+           reinterpret_cast<const uint8_t*>(p.k_idx_new) + src0 * D_I, (int64_t)nr * D_I);
+    const int64_t kvb = p.kv_row_bytes;
+    for (int g = 0; g < p.layers; ++g) {
+        copy16(reinterpret_cast<uint8_t*>(p.k_cache[g]) + (off + lo) * kvb,
+               reinterpret_cast<const uint8_t*>(p.k_new[g]) + src0 * kvb, nr * kvb);
+        copy16(reinterpret_cast<uint8_t*>(p.v_cache[g]) + (off + lo) * kvb,
+               reinterpret_cast<const uint8_t*>(p.v_new[g]) + src0 * kvb, nr * kvb);
+    }
+    if (p.sums) {
+        const int8_t* cache = a.k_idx + (off + t0) * D_I;
+        const int8_t* fresh = p.k_idx_new + (int64_t)seq * n_new * D_I;
+        sum_block<D_I>(
+            [&](int row) {
+                const int pos = t0 + row;
+                return pos >= from ? fresh + (int64_t)(pos - from) * D_I : cache + (int64_t)row * D_I;
+            },
+            n, a.block_sums + (a.blk_offset[seq] + j) * (2 * D_I), s_part);
     }
 }
 
@@ -96,6 +178,25 @@ cudaError_t launch_block_sums(const BlockSumArgs& a, int d_I, cudaStream_t strea
         case 32: return launch_pdl(block_sums_kernel<32>, grid, dim3(kBsThreads), 0, stream, 0, a);
         case 64: return launch_pdl(block_sums_kernel<64>, grid, dim3(kBsThreads), 0, stream, 0, a);
         case 128: return launch_pdl(block_sums_kernel<128>, grid, dim3(kBsThreads), 0, stream, 0, a);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_append(const AppendArgs& a, int d_I, cudaStream_t stream) {
+    const int n_new = a.bs.n_new;
+    unsigned gx;
+    if (a.sums) {
+        int64_t full = ((int64_t)a.bs.max_len + a.bs.hi_block - 1) / a.bs.hi_block;
+        int64_t cover = ((int64_t)n_new + a.bs.hi_block - 1) / a.bs.hi_block + 1;
+        gx = (unsigned)(cover < full ? cover : full);
+    } else {
+        gx = (unsigned)((n_new + kAppendRowsPerCta - 1) / kAppendRowsPerCta);
+    }
+    dim3 grid(gx, (unsigned)a.bs.n_seq);
+    switch (d_I) {
+        case 32: return launch_pdl(append_kernel<32>, grid, dim3(kBsThreads), 0, stream, 0, a);
+        case 64: return launch_pdl(append_kernel<64>, grid, dim3(kBsThreads), 0, stream, 0, a);
+        case 128: return launch_pdl(append_kernel<128>, grid, dim3(kBsThreads), 0, stream, 0, a);
         default: return cudaErrorInvalidValue;
     }
 }

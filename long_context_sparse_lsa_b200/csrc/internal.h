@@ -31,6 +31,23 @@ struct BlockSumArgs {
 };
 cudaError_t launch_block_sums(const BlockSumArgs& a, int d_I, cudaStream_t stream);
 
+// Decode append: the n_new newest tokens of every sequence receive their
+// indexer key and per-layer K/V rows, and (HI on) the block sums of their
+// blocks are recomputed, in one launch.
+struct AppendArgs {
+    BlockSumArgs bs;               // k_idx: the cache being written; n_new > 0
+    const int8_t* k_idx_new;       // [n_seq][n_new][d_I]
+    int8_t* k_idx_cache;           // == bs.k_idx
+    const uint16_t* k_new[kMaxLayers];  // [n_seq][n_new][H_kv][d] per layer
+    const uint16_t* v_new[kMaxLayers];
+    uint16_t* k_cache[kMaxLayers];      // [total_tokens][H_kv][d] per layer
+    uint16_t* v_cache[kMaxLayers];
+    int32_t layers;
+    int32_t kv_row_bytes;          // H_kv * d * 2
+    int32_t sums;                  // 1: recompute the block sums (HI on)
+};
+cudaError_t launch_append(const AppendArgs& a, int d_I, cudaStream_t stream);
+
 // ---- indexer: scoring kernels + selection kernels -------------------------
 // Keys (score + 1) are histogrammed on a monotone logarithmic scale: the bit
 // length of the key and the 6 bits after its leading one (keys below 64 map

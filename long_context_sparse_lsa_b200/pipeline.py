@@ -1,8 +1,11 @@
 """A decode step of the LSA hot path over one workload, through the C ABI.
 
 Allocation and call sequencing only (device buffers via torch, calls via
-``binding``): the HI block-sum append update, one ``lsa_index`` per group of
-G layers (Cross-Layer Indexing) and one ``lsa_attend`` for the G layers.
+``binding``): the decode append (the newest tokens' keys and K/V rows written
+into the caches, their blocks' HI sums refreshed), one ``lsa_index`` per
+group of G layers (Cross-Layer Indexing) and one ``lsa_attend`` for the G
+layers. A prefill chunk (``wl.prefill_new``) has no append: its rows are
+already in the caches.
 """
 from __future__ import annotations
 
@@ -32,6 +35,18 @@ class LsaStep:
         ws_a = lsa.lsa_attend_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
         self.ws_attend = torch.zeros(max(256, ws_a), dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        # the tokens a decode step appends: each sequence's newest `drafts`
+        # tokens, whose rows the step writes (the synthetic draw already holds
+        # them, so the caches keep their contents)
+        self.n_new = 0 if wl.prefill_new else wl.drafts
+        if self.n_new:
+            offs, lens = t.kv_offset.tolist(), t.seq_lens.tolist()
+            pos = torch.tensor([o + L - self.n_new + j for o, L in zip(offs, lens) for j in range(self.n_new)],
+                               dtype=torch.int64, device=device)
+            n_seq = len(lens)
+            self.k_idx_new = t.k_idx.index_select(0, pos).view(n_seq, self.n_new, wl.d_I).clone()
+            self.k_new = [x.index_select(0, pos).view(n_seq, self.n_new, wl.H_kv, wl.d).clone() for x in t.k]
+            self.v_new = [x.index_select(0, pos).view(n_seq, self.n_new, wl.H_kv, wl.d).clone() for x in t.v]
 
     # -- the three calls --------------------------------------------------------
     def build_block_sums(self, stream=None):
@@ -43,6 +58,13 @@ class LsaStep:
             lsa.lsa_hi_block_sums(self.t.k_idx, self.wl.hi_block, self.batch, self.block_sums, n_new, self.status,
                                   stream)
 
+    def append(self, stream=None):
+        """The decode append: write the newest tokens' keys and K/V rows and
+        refresh the block sums of their blocks (one launch)."""
+        if self.n_new:
+            lsa.lsa_append(self.k_idx_new, self.t.k_idx, self.k_new, self.v_new, self.t.k, self.t.v,
+                           self.wl.hi_block, self.block_sums, self.batch, self.n_new, self.status, stream)
+
     def index(self, stream=None):
         lsa.lsa_index(self.t.q_idx, self.t.k_idx, self.t.w, self.wl.w_max, self.batch, self.budget, self.sets,
                       self.block_sums, self.ws_index, self.status, stream)
@@ -52,32 +74,41 @@ class LsaStep:
                        stream)
 
     def step(self, stream=None):
-        """One decode step: append update of the block sums, index, attend."""
-        self.update_block_sums(1, stream)
+        """One decode step: append, index, attend."""
+        self.append(stream)
         self.index(stream)
         self.attend(stream)
 
-    def overlap_ok(self, n_new: int = 1) -> bool:
-        """True when the block-sum append update may run beside the index call.
+    def overlap_ok(self) -> bool:
+        """True when the append may run beside the index call.
 
-        The update rewrites only the blocks holding the n_new newest tokens;
-        the coarse HI scores read only blocks that end before the window
-        start. With window >= hi_block + n_new - 1 those blocks lie inside the
-        window and the two calls touch disjoint rows."""
+        The append writes the n_new newest tokens' rows and, with HI on, the
+        sums of the blocks that hold them. The index call reads keys of the
+        middle only (positions below the window start) and, with HI on, the
+        sums of the blocks that meet the middle. With window >= n_new (HI
+        off) or window >= hi_block + n_new - 1 (HI on) none of those is
+        written, so the two calls touch disjoint memory; the attention, which
+        reads the new K/V rows, runs after both."""
         wl = self.wl
-        return self.block_sums is not None and wl.window >= wl.hi_block + n_new - 1
+        if not self.n_new:
+            return False
+        need = wl.hi_block + self.n_new - 1 if wl.hi_block > 0 else self.n_new
+        return wl.window >= need
 
     def status_bits(self) -> int:
         return int(self.status.item())
 
     # -- CUDA graphs ------------------------------------------------------------
     def capture(self):
-        """Capture the three calls as CUDA graphs (block-sum append update,
-        index, attend), and the whole step as one more graph ("step") in which
-        the block-sum update runs on a forked stream beside the index call when
-        overlap_ok(). A step then replays without host launch overhead. The
-        graphs keep this object's buffers; changing their contents between
-        replays is how new inputs enter."""
+        """Capture the three calls as CUDA graphs (append, index, attend), and
+        the whole step as one more graph ("step") in which the append runs on
+        a forked stream beside the index call when overlap_ok(). A step then
+        replays without host launch overhead. Two more graphs serve
+        measurement: "step_timed" (the step with timing events around the
+        index and attention calls) and, with HI on, "cold" (a full block-sum
+        build, then index and attention). The graphs keep this object's
+        buffers; changing their contents between replays is how new inputs
+        enter."""
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):  # one eager pass fills the launch-plan caches
@@ -85,9 +116,8 @@ class LsaStep:
         torch.cuda.current_stream(self.device).wait_stream(side)
         torch.cuda.synchronize(self.device)
         self.graphs = {}
-        for name, fn in (("block_sums", lambda: self.update_block_sums(1)), ("index", self.index),
-                         ("attend", self.attend)):
-            if name == "block_sums" and self.block_sums is None:
+        for name, fn in (("append", self.append), ("index", self.index), ("attend", self.attend)):
+            if name == "append" and not self.n_new:
                 continue
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
@@ -97,10 +127,10 @@ class LsaStep:
         fork = torch.cuda.Stream(self.device)
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             cur = torch.cuda.current_stream(self.device)
-            if self.overlap_ok(1):
+            if self.overlap_ok():
                 fork.wait_stream(cur)
                 with torch.cuda.stream(fork):
-                    self.update_block_sums(1)
+                    self.append()
                 self.index()
                 cur.wait_stream(fork)
                 self.attend()
@@ -116,13 +146,13 @@ class LsaStep:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             cur = torch.cuda.current_stream(self.device)
-            overlap = self.overlap_ok(1)
+            overlap = self.overlap_ok()
             if overlap:
                 fork.wait_stream(cur)
                 with torch.cuda.stream(fork):
-                    self.update_block_sums(1)
+                    self.append()
             else:
-                self.update_block_sums(1)
+                self.append()
             ix0.record(cur)
             self.index()
             ix1.record(cur)
@@ -132,6 +162,14 @@ class LsaStep:
             self.attend()
             at1.record(cur)
         self.graphs["step_timed"] = g
+        if self.block_sums is not None:
+            # a cold step: the block sums rebuilt from the whole key cache first
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                self.build_block_sums()
+                self.index()
+                self.attend()
+            self.graphs["cold"] = g
         torch.cuda.synchronize(self.device)
         return self.graphs
 
@@ -147,9 +185,9 @@ class LsaStep:
             self.graphs[name].replay()
 
     def kernels_per_step(self) -> int:
-        """Kernel launches of one step: the block-sum update (HI) and the
-        launches the index and attention calls report for this shape."""
+        """Kernel launches of one step: the append (decode) and the launches
+        the index and attention calls report for this shape."""
         wl = self.wl
         n_idx = lsa.lsa_index_launches(self.batch, wl.H_I, wl.d_I, self.budget)
         n_att = lsa.lsa_attend_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
-        return (1 if self.block_sums is not None else 0) + n_idx + n_att
+        return (1 if self.n_new else 0) + n_idx + n_att

@@ -35,6 +35,8 @@ class Workload:
     d: int
     G: int                         # layers sharing one index set
     prefill_new: int = 0           # > 0: a causal prefill chunk of this many tokens on sequence 0
+    drafts: int = 1                # decode rows per sequence (several draft tokens, MTP-style):
+                                   # row j of a sequence of L tokens sees L - drafts + 1 + j
     note: str = field(default="", compare=False)
 
     @property
@@ -51,7 +53,7 @@ class Workload:
 
     @property
     def n_q(self) -> int:
-        return self.prefill_new if self.prefill_new else self.n_seq
+        return self.prefill_new if self.prefill_new else self.n_seq * self.drafts
 
     @property
     def w_max(self) -> int:
@@ -137,8 +139,9 @@ def layout(wl: Workload, device, hi_block: int | None = None):
         q_seq = [0] * wl.prefill_new
         q_len = [C + i + 1 for i in range(wl.prefill_new)]
     else:
-        q_seq = list(range(len(lens)))
-        q_len = lens
+        D = wl.drafts
+        q_seq = [b for b in range(len(lens)) for _ in range(D)]
+        q_len = [L - D + 1 + j for L in lens for j in range(D)]
     t = lambda x, dt: torch.tensor(x, dtype=dt, device=device)
     return (t(offs, torch.int64), t(lens, torch.int32), t(boffs, torch.int64), t(q_seq, torch.int32),
             t(q_len, torch.int32), bacc)

@@ -172,6 +172,49 @@ def test_block_sums_exact_and_append_update():
         np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
 
 
+@pytest.mark.parametrize("n_new,hi_block", [(1, 64), (70, 64), (5, 0)])
+def test_append_writes_rows_and_refreshes_block_sums(n_new, hi_block):
+    """The decode append writes each sequence's newest n_new tokens (keys and
+    both layers' K/V rows) and, with HI on, re-sums their blocks: the caches
+    equal a host-side copy of the rows into place and the block sums equal
+    the oracle's sums of the updated cache; nothing else changes."""
+    wl = wls.small(BASE, name="append", lens=(1000, 71, 130, 5000), hi_block=hi_block,
+                   hi_topblocks=8 if hi_block else 0, G=2, seed=31)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    gen = torch.Generator().manual_seed(1000 + n_new)
+    n_seq = wl.n_seq
+    k_idx_new = torch.randint(-16, 16, (n_seq, n_new, wl.d_I), dtype=torch.int8, generator=gen)
+    k_new = [torch.randn((n_seq, n_new, wl.H_kv, wl.d), generator=gen).to(torch.bfloat16) for _ in range(wl.G)]
+    v_new = [torch.randn((n_seq, n_new, wl.H_kv, wl.d), generator=gen).to(torch.bfloat16) for _ in range(wl.G)]
+    want_k = parity.host(t.k_idx).copy()
+    want_K = [parity.u16(x).copy() for x in t.k]
+    want_V = [parity.u16(x).copy() for x in t.v]
+    offs = parity.host(t.kv_offset)
+    for b, L in enumerate(wl.lens):
+        lo = offs[b] + L - n_new
+        want_k[lo:lo + n_new] = k_idx_new[b].numpy()
+        for g in range(wl.G):
+            want_K[g][lo:lo + n_new] = k_new[g][b].view(torch.int16).numpy().view(np.uint16)
+            want_V[g][lo:lo + n_new] = v_new[g][b].view(torch.int16).numpy().view(np.uint16)
+    lsa.lsa_append(k_idx_new.to(DEV), t.k_idx, [x.to(DEV) for x in k_new], [x.to(DEV) for x in v_new], t.k, t.v,
+                   hi_block, st.block_sums, st.batch, n_new, st.status)
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    np.testing.assert_array_equal(parity.host(t.k_idx), want_k)
+    for g in range(wl.G):
+        np.testing.assert_array_equal(parity.u16(t.k[g]), want_K[g])
+        np.testing.assert_array_equal(parity.u16(t.v[g]), want_V[g])
+    if hi_block:
+        orc = oracle.get()
+        got = parity.decode_block_sums(st.block_sums, wl.d_I)
+        boffs = parity.host(t.blk_offset)
+        for b, L in enumerate(wl.lens):
+            want = orc.block_sums(want_k[offs[b]:offs[b] + L], hi_block)
+            np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
+
+
 def test_extreme_block_sums_hi_block_256():
     """|S| reaches 128 * 256 = 32768: the byte planes stay exact."""
     wl = wls.small(BASE, name="bs_extreme", lens=(512,), hi_block=256, hi_topblocks=1, seed=3)
@@ -228,6 +271,28 @@ def test_repeated_calls_are_deterministic():
         outs.append(parity.host(st.out[0]).copy())
     assert all(np.array_equal(sets[0], s) for s in sets)
     assert all(np.array_equal(outs[0], o) for o in outs)
+
+
+def test_draft_rows_per_sequence():
+    """Several draft tokens per sequence in one decode step (MTP-style): row j
+    of a sequence of L tokens sees L - 3 + j of them. Every row through the
+    decode kernels, HI on, two layers per index set."""
+    wl = wls.small(BASE, name="drafts", lens=(40000, 25000, 61000), drafts=4, hi_block=64, hi_topblocks=256,
+                   G=2, seed=23)
+    t = wls.make(wl, DEV)
+    assert wl.n_q == 12 and parity.host(t.q_len).tolist()[:4] == [39997, 39998, 39999, 40000]
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    st.index()
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    rows = np.arange(wl.n_q)
+    want = parity.oracle_sets(wl, t, rows=rows)
+    parity.check_sets(parity.host(st.sets), want, wl.name)
+    ref = parity.oracle_attend_rows(t, want, rows)
+    for g in range(wl.G):
+        parity.check_attention(parity.host(st.out[g]), ref[g], f"{wl.name} layer {g}")
 
 
 def test_graph_replay_matches_eager():
