@@ -23,8 +23,10 @@ constexpr int kBsWarps = kBsThreads / kWarp;
 __device__ __forceinline__ int sbyte(uint32_t w, int i) { return static_cast<int>(static_cast<int8_t>(w >> (8 * i))); }
 
 // Thread t owns 16-byte chunk (t % CPR) of rows t / CPR, t / CPR + RPP, ...
-// of the block, so the block is read in B / RPP dependent rounds of coalesced
-// 16-byte loads (one round for hi_block <= 32 at d_I = 128). row_ptr(i) is
+// of the block, so the block is read in B / RPP rounds of coalesced 16-byte
+// loads (one round for hi_block <= 32 at d_I = 128). Keeping four rows in
+// flight per thread was measured and dropped: 63 registers instead of 48
+// cost resident CTAs, and the full build got slower. row_ptr(i) is
 // the address of the block's row i; the sum of rows [0, n) goes to out_row as
 // the two byte planes. Every thread of the CTA calls it (one CTA barrier).
 template <int D_I, typename RowPtr>
