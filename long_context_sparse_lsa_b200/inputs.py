@@ -116,6 +116,23 @@ def normal_bf16(shape, seed: int, stream: int, device) -> torch.Tensor:
     return _fill(out, seed, stream, draw)
 
 
+def normal_e4m3(shape, seed: int, stream: int, device) -> torch.Tensor:
+    """FP8 E4M3 codes (uint8) of standard normal draws: the same Box-Muller
+    draws, rounded to E4M3 once by torch's float8_e4m3fn conversion."""
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    two_pi = 2.0 * math.pi
+
+    def draw(start, cnt):
+        h1 = hashes(seed, stream, start, cnt, device)
+        h2 = hashes(seed, stream + (1 << 16), start, cnt, device)
+        u1 = (_srl(h1, 11) + 1).to(torch.float64) * (2.0 ** -53)
+        u2 = _srl(h2, 11).to(torch.float64) * (2.0 ** -53)
+        z = torch.sqrt(-2.0 * torch.log(u1)) * torch.cos(two_pi * u2)
+        return z.to(torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+
+    return _fill(out, seed, stream, draw)
+
+
 def lognormal_lengths(n: int, median: float, sigma: float, lo: int, hi: int, cap: int,
                       seed: int, stream: int) -> list[int]:
     """Ragged sequence lengths: lognormal(ln median, sigma) drawn with the same
@@ -148,3 +165,5 @@ STREAM_LENS = 4
 STREAM_Q = 16   # + layer
 STREAM_K = 32   # + layer
 STREAM_V = 48   # + layer
+STREAM_K8 = 64  # + layer: FP8 E4M3 K cache
+STREAM_V8 = 80  # + layer: FP8 E4M3 V cache

@@ -27,6 +27,7 @@ _i8p = ctypes.POINTER(ctypes.c_int8)
 _i32p = ctypes.POINTER(ctypes.c_int32)
 _i64p = ctypes.POINTER(ctypes.c_int64)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 _f64p = ctypes.POINTER(ctypes.c_double)
 
 
@@ -78,6 +79,11 @@ class Oracle:
         lib.oracle_attend_query.restype = None
         lib.oracle_attend_query.argtypes = [_u16p, _u16p, _u16p, _i32p, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_int, _f64p]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_attend_query_fp8.restype = None
+        lib.oracle_attend_query_fp8.argtypes = [_u16p, _u8p, _u8p, ctypes.c_double, ctypes.c_double, _i32p,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f64p]
         lib.oracle_lsa_index.restype = ctypes.c_int
         lib.oracle_lsa_index.argtypes = [_i8p, _i8p, _i32p, _i64p, _i32p, _i32p, ctypes.c_int64,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -137,6 +143,24 @@ class Oracle:
         out = np.empty((H_q, d), np.float64)
         self.lib.oracle_attend_query(_p(q, _u16p), _p(kseq, _u16p), _p(vseq, _u16p), _p(s, _i32p),
                                      s.shape[0], H_q, H_kv, d, _p(out, _f64p))
+        return out
+
+    def e4m3_value(self, code: int) -> float:
+        """The value of one FP8 E4M3 code (NaN for S.1111.111)."""
+        return float(self.lib.oracle_e4m3_value(int(code) & 0xFF))
+
+    def attend_query_fp8(self, q, kseq, vseq, k_scale, v_scale, idx_set) -> np.ndarray:
+        """q: [H_q, d] bf16 bits (uint16); kseq/vseq: [L, H_kv, d] E4M3 codes (uint8);
+        k = k_scale * E4M3(code), v = v_scale * E4M3(code)."""
+        q = _c(q, np.uint16)
+        kseq = _c(kseq, np.uint8)
+        vseq = _c(vseq, np.uint8)
+        s = _c(idx_set, np.int32)
+        H_q, d = q.shape
+        H_kv = kseq.shape[1]
+        out = np.empty((H_q, d), np.float64)
+        self.lib.oracle_attend_query_fp8(_p(q, _u16p), _p(kseq, _u8p), _p(vseq, _u8p), float(k_scale),
+                                         float(v_scale), _p(s, _i32p), s.shape[0], H_q, H_kv, d, _p(out, _f64p))
         return out
 
     # -- batches ---------------------------------------------------------------

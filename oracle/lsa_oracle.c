@@ -266,6 +266,75 @@ void oracle_attend_query(const uint16_t *q, const uint16_t *kseq,
 }
 
 /* ----------------------------------------------------------------------- */
+/* Attention over an FP8 KV cache                                            */
+/* ----------------------------------------------------------------------- */
+/* The pages name FP8 variants of the models and a KV-cache data type, but
+ * not the FP8 format or its scaling. Reading used here: OCP FP8 E4M3 codes
+ * (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field
+ * 0 holds the subnormals m/8 * 2^-6; no infinities; S.1111.111 is NaN) with
+ * one scale per layer for K and one for V: value = scale * E4M3(code). */
+
+/* E4M3 code -> double, from the format's definition. */
+double oracle_e4m3_value(uint8_t code)
+{
+    int sign = code >> 7, E = (code >> 3) & 0xF, m = code & 7;
+    double v;
+    if (E == 15 && m == 7)
+        return NAN;
+    if (E == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, E - 7);
+    return sign ? -v : v;
+}
+
+/* oracle_attend_query with K and V given as E4M3 codes: k = k_scale *
+ * E4M3(k code), v = v_scale * E4M3(v code); everything else (GQA mapping,
+ * scale 1/sqrt(d), skipped -1 entries, empty set -> zeros) as there. */
+void oracle_attend_query_fp8(const uint16_t *q, const uint8_t *kseq,
+                             const uint8_t *vseq, double k_scale, double v_scale,
+                             const int32_t *set, int budget, int H_q, int H_kv,
+                             int d, double *out)
+{
+    double scale = 1.0 / sqrt((double)d);
+    double *z = (double *)malloc((size_t)(budget > 0 ? budget : 1) * sizeof(double));
+    for (int h = 0; h < H_q; ++h) {
+        int kvh = (int)(((int64_t)h * H_kv) / H_q);
+        double zmax = -INFINITY;
+        int any = 0;
+        for (int j = 0; j < budget; ++j) {
+            if (set[j] < 0)
+                continue;
+            const uint8_t *krow = kseq + ((int64_t)set[j] * H_kv + kvh) * d;
+            double dot = 0.0;
+            for (int e = 0; e < d; ++e)
+                dot += bf16_to_double(q[h * d + e]) * (k_scale * oracle_e4m3_value(krow[e]));
+            z[j] = dot * scale;
+            if (z[j] > zmax)
+                zmax = z[j];
+            any = 1;
+        }
+        for (int e = 0; e < d; ++e)
+            out[h * d + e] = 0.0;
+        if (!any)
+            continue;
+        double denom = 0.0;
+        for (int j = 0; j < budget; ++j) {
+            if (set[j] < 0)
+                continue;
+            double p = exp(z[j] - zmax);
+            denom += p;
+            const uint8_t *vrow = vseq + ((int64_t)set[j] * H_kv + kvh) * d;
+            for (int e = 0; e < d; ++e)
+                out[h * d + e] += p * (v_scale * oracle_e4m3_value(vrow[e]));
+        }
+        for (int e = 0; e < d; ++e)
+            out[h * d + e] /= denom;
+    }
+    free(z);
+}
+
+/* ----------------------------------------------------------------------- */
 /* Batch drivers (independent queries; optionally spread over threads)       */
 /* ----------------------------------------------------------------------- */
 
