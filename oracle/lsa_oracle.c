@@ -296,20 +296,20 @@ void oracle_attend_query_fp8(const uint16_t *q, const uint8_t *kseq,
                              const int32_t *set, int budget, int H_q, int H_kv,
                              int d, double *out)
 {
-    double scale = 1.0 / sqrt((double)d);
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
     double *z = (double *)malloc((size_t)(budget > 0 ? budget : 1) * sizeof(double));
     for (int h = 0; h < H_q; ++h) {
-        int kvh = (int)(((int64_t)h * H_kv) / H_q);
+        const int kv_head = (int)(((int64_t)h * H_kv) / H_q);
         double zmax = -INFINITY;
         int any = 0;
         for (int j = 0; j < budget; ++j) {
             if (set[j] < 0)
                 continue;
-            const uint8_t *krow = kseq + ((int64_t)set[j] * H_kv + kvh) * d;
+            const uint8_t *krow = kseq + ((int64_t)set[j] * H_kv + kv_head) * d;
             double dot = 0.0;
             for (int e = 0; e < d; ++e)
                 dot += bf16_to_double(q[h * d + e]) * (k_scale * oracle_e4m3_value(krow[e]));
-            z[j] = dot * scale;
+            z[j] = dot * inv_sqrt_d;
             if (z[j] > zmax)
                 zmax = z[j];
             any = 1;
@@ -324,12 +324,12 @@ void oracle_attend_query_fp8(const uint16_t *q, const uint8_t *kseq,
                 continue;
             double p = exp(z[j] - zmax);
             denom += p;
-            const uint8_t *vrow = vseq + ((int64_t)set[j] * H_kv + kvh) * d;
+            const uint8_t *vrow = vseq + ((int64_t)set[j] * H_kv + kv_head) * d;
             for (int e = 0; e < d; ++e)
                 out[h * d + e] += p * (v_scale * oracle_e4m3_value(vrow[e]));
         }
         for (int e = 0; e < d; ++e)
-            out[h * d + e] /= denom;
+            out[h * d + e] = out[h * d + e] / denom;
     }
     free(z);
 }

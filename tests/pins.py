@@ -470,4 +470,74 @@ def pin_batch_matches_single_queries(orc):
             assert np.array_equal(outs[g][r], want)
 
 
+# ---- FP8 KV cache --------------------------------------------------------
+def _e4m3_torch(codes: np.ndarray) -> np.ndarray:
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _e4m3_to_bf16_bits(codes: np.ndarray, scale: float) -> np.ndarray:
+    import torch
+    vals = torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float32) * scale
+    bits = vals.to(torch.bfloat16)
+    assert torch.equal(bits.to(torch.float32), vals)  # an E4M3 value times a power of two is a bf16
+    return bits.view(torch.int16).numpy().view(np.uint16)
+
+
+def _fp8_case(seed, L=40, H_q=8, H_kv=2, d=128):
+    import torch
+    rng = _rng(seed)
+    q = _bf16_bits(rng.standard_normal((H_q, d)))
+    k = torch.from_numpy(rng.standard_normal((L, H_kv, d)).astype(np.float32)).to(torch.float8_e4m3fn)
+    v = torch.from_numpy(rng.standard_normal((L, H_kv, d)).astype(np.float32)).to(torch.float8_e4m3fn)
+    s = np.array([0, 3, 4, -1, 17, 18, 19, 39, -1, -1], np.int32)
+    return q, k.view(torch.uint8).numpy(), v.view(torch.uint8).numpy(), s
+
+
+def pin_fp8_decode_matches_torch_on_every_code(orc):
+    """E4M3 decode of all 256 codes against torch's float8_e4m3fn type."""
+    codes = np.arange(256, dtype=np.uint8)
+    want = _e4m3_torch(codes)
+    got = np.array([orc.e4m3_value(c) for c in codes])
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2  # 0x7F and 0xFF
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+def pin_fp8_decode_closed_forms(orc):
+    """Values the format's definition fixes (bias 7, subnormals m/8 * 2^-6)."""
+    assert orc.e4m3_value(0x00) == 0.0
+    assert orc.e4m3_value(0x38) == 1.0
+    assert orc.e4m3_value(0xB8) == -1.0
+    assert orc.e4m3_value(0x7E) == 448.0
+    assert orc.e4m3_value(0x08) == 2.0 ** -6
+    assert orc.e4m3_value(0x01) == 2.0 ** -9
+    assert orc.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert np.isnan(orc.e4m3_value(0x7F))
+
+
+def pin_fp8_attention_is_bf16_attention_on_the_values(orc):
+    """FP8 attention = the bf16 attention on the decoded, scaled values."""
+    q, k8, v8, s = _fp8_case(1)
+    for ks, vs in ((1.0, 1.0), (0.5, 2.0), (0.125, 0.25)):
+        got = orc.attend_query_fp8(q, k8, v8, ks, vs, s)
+        want = orc.attend_query(q, _e4m3_to_bf16_bits(k8, ks), _e4m3_to_bf16_bits(v8, vs), s)
+        np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+def pin_fp8_attention_scales(orc):
+    """Linear in v_scale; k_scale = 0 gives the plain mean of the selected V rows;
+    an empty set gives zeros."""
+    q, k8, v8, s = _fp8_case(2)
+    base = orc.attend_query_fp8(q, k8, v8, 0.7, 1.0, s)
+    np.testing.assert_allclose(orc.attend_query_fp8(q, k8, v8, 0.7, 3.0, s), 3.0 * base, rtol=1e-13, atol=1e-13)
+    flat = orc.attend_query_fp8(q, k8, v8, 0.0, 1.0, s)
+    vals = _e4m3_torch(v8)
+    rows = s[s >= 0]
+    for h in range(q.shape[0]):
+        kvh = h * k8.shape[1] // q.shape[0]
+        np.testing.assert_allclose(flat[h], vals[rows, kvh].mean(axis=0), rtol=1e-13, atol=1e-13)
+    assert not orc.attend_query_fp8(q, k8, v8, 1.0, 1.0, np.full(6, -1, np.int32)).any()
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

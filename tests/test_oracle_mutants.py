@@ -37,6 +37,17 @@ MUTANTS = [
      "            const uint16_t *vrow = kseq + ((int64_t)set[j] * H_kv + kvh) * d;"),
     ("batch driver ignores the sequence offset", "        const int8_t *kseq = j->k_idx + j->kv_offset[j->q_seq[r]] * j->d_I;",
      "        const int8_t *kseq = j->k_idx;"),
+    ("E4M3 exponent bias 8", "        v = ldexp(1.0 + (double)m / 8.0, E - 7);", "        v = ldexp(1.0 + (double)m / 8.0, E - 8);"),
+    ("E4M3 subnormals read as normals", "        v = ldexp((double)m / 8.0, -6);", "        v = ldexp(1.0 + (double)m / 8.0, -6);"),
+    ("E4M3 sign dropped", "    return sign ? -v : v;", "    return v;"),
+    ("FP8 attention ignores the K scale",
+     "                dot += bf16_to_double(q[h * d + e]) * (k_scale * oracle_e4m3_value(krow[e]));",
+     "                dot += bf16_to_double(q[h * d + e]) * oracle_e4m3_value(krow[e]);"),
+    ("FP8 attention scales V by the K scale",
+     "                out[h * d + e] += p * (v_scale * oracle_e4m3_value(vrow[e]));",
+     "                out[h * d + e] += p * (k_scale * oracle_e4m3_value(vrow[e]));"),
+    ("FP8 attention softmax scale 1/d", "    const double inv_sqrt_d = 1.0 / sqrt((double)d);",
+     "    const double inv_sqrt_d = 1.0 / (double)d;"),
 ]
 
 
