@@ -44,9 +44,9 @@ PROFILES = os.path.join(ROOT, "profiles")
 # ---------------------------------------------------------------------------
 # algorithmic bytes (what the method must move; nothing avoided by HI counted)
 # ---------------------------------------------------------------------------
-def step_bytes(wl) -> dict:
+def step_bytes(wl, kv_fp8: bool = False) -> dict:
     n_q, G = wl.n_q, wl.G
-    kv_row = wl.H_kv * wl.d * 2  # bytes of one token's K (or V) in one layer
+    kv_row = wl.H_kv * wl.d * (1 if kv_fp8 else 2)  # bytes of one token's K (or V) in one layer
     rows = _rows(wl)
     attend = 0
     for L in rows:
@@ -309,14 +309,14 @@ def job_rate(units_per_rank: int, world: int, ms: float) -> float:
 
 
 # ---------------------------------------------------------------------------
-def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None):
+def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, kv_fp8=False):
     """Draws the workload, captures its step graphs and times `steps` steps
     (after `warmup`), each after an L2 flush: the whole step graph for the
     headline, then the three calls one by one for the breakdown."""
     from long_context_sparse_lsa_b200.pipeline import LsaStep
 
-    t = wls.make(wl, dev)
-    st = LsaStep(wl, t, dev)
+    t = wls.make(wl, dev, with_kv=not kv_fp8)
+    st = LsaStep(wl, t, dev, kv_fp8=kv_fp8)
     st.build_block_sums()
     torch.cuda.synchronize()
     st.capture()
@@ -421,11 +421,11 @@ def secondary(dev, flush, stream, steps, warmup, peak):
 
     out = {}
     mean = lambda xs: sum(xs) / len(xs)
-    for wl in (wls.CTX1M, wls.PREFILL):
-        run = time_workload(wl, dev, flush, stream, steps, warmup)
+    for wl, fp8 in ((wls.CTX1M, False), (wls.PREFILL, False), (wls.BATCH128K, True)):
+        run = time_workload(wl, dev, flush, stream, steps, warmup, kv_fp8=fp8)
         st = run["st"]
         ms = run["ms"]
-        byts = step_bytes(wl)
+        byts = step_bytes(wl, kv_fp8=fp8)
         ix, at = mean(run["ix_in_step"]), mean(run["at_in_step"])
         rec = {"ms_per_step": ms, "steps": steps, "warmup": warmup,
                "step_breakdown_ms": {"append": mean(run["bs"]), "index": mean(run["ix"]),
@@ -451,10 +451,15 @@ def secondary(dev, flush, stream, steps, warmup, peak):
                         "int8_peak_tops": p8, "int8_peak_kind": kind8,
                         "note": "index_tops: int8 ops of the fine-score contraction over the whole index call "
                                 "(scoring + selection), so a lower bound on the tensor kernel's rate"})
+        elif fp8:
+            rec.update({"metric": "LSA decode queries/s at 128K ctx, FP8 E4M3 KV cache", "unit": "queries/s",
+                        "value": wl.n_q / (ms / 1000.0), "kv_cache": "fp8 e4m3, one scale per layer for K and V",
+                        "note": "same workload as the headline with the K/V caches held as FP8 codes "
+                                "(lsa_attend_fp8); attention bytes per query halve"})
         else:
             rec.update({"metric": "LSA decode queries/s at 1M ctx", "unit": "queries/s",
                         "value": wl.n_q / (ms / 1000.0), "layers_per_index": wl.G})
-        out[wl.name] = rec
+        out[wl.name + ("_fp8kv" if fp8 else "")] = rec
         del run, st
         torch.cuda.synchronize()
         torch.cuda.empty_cache()

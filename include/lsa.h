@@ -160,21 +160,25 @@ lsa_status_t lsa_hi_block_sums(const int8_t *k_idx_cache, int32_t d_I,
  * else LSA_DEV_BAD_LENGTH and the sequence is skipped).
  * k_idx_new    device int8 [n_seq][n_new][d_I]: the new indexer keys.
  * k_idx_cache  device int8 [total_tokens][d_I], written at the new positions.
- * k_new, v_new host [layers] arrays of device bf16 [n_seq][n_new][H_kv][d].
- * k_cache, v_cache host [layers] arrays of device bf16
- *              [total_tokens][H_kv][d], written at the new positions.
- *              layers may be 0 (indexer keys only); the arrays may then be NULL.
+ * k_new, v_new host [layers] arrays of device [n_seq][n_new] rows of
+ *              kv_row_bytes bytes each (one token's K or V of one layer:
+ *              H_kv*d*2 for bf16 caches, H_kv*d for FP8 E4M3 caches).
+ * k_cache, v_cache host [layers] arrays of device [total_tokens] rows of
+ *              kv_row_bytes bytes, written at the new positions. The rows
+ *              are copied as bytes. layers may be 0 (indexer keys only);
+ *              the arrays may then be NULL.
  * block_sums   as for lsa_hi_block_sums, or NULL when hi_block == 0. The
  *              refreshed blocks are summed from the new keys (read from
  *              k_idx_new) and the older keys of the block (from the cache).
  * All device pointers 16-byte aligned; the inputs must not overlap the
- * cache rows being written. Supported: d_I in {32, 64, 128}; d == 128;
- * 0 <= layers <= LSA_MAX_LAYERS; 0 <= hi_block <= LSA_MAX_HI_BLOCK.
+ * cache rows being written. Supported: d_I in {32, 64, 128}; kv_row_bytes
+ * a positive multiple of 16 (when layers > 0); 0 <= layers <=
+ * LSA_MAX_LAYERS; 0 <= hi_block <= LSA_MAX_HI_BLOCK.
  */
 lsa_status_t lsa_append(const int8_t *k_idx_new, int8_t *k_idx_cache, int32_t d_I,
-                        const uint16_t *const *k_new, const uint16_t *const *v_new,
-                        uint16_t *const *k_cache, uint16_t *const *v_cache,
-                        int32_t H_kv, int32_t d, int32_t layers, int32_t hi_block,
+                        const void *const *k_new, const void *const *v_new,
+                        void *const *k_cache, void *const *v_cache,
+                        int32_t kv_row_bytes, int32_t layers, int32_t hi_block,
                         int8_t *block_sums, int64_t block_rows,
                         const lsa_batch_t *batch, int32_t n_new,
                         int32_t *dev_status, void *stream);
@@ -266,6 +270,28 @@ lsa_status_t lsa_attend(const uint16_t *const *q, const uint16_t *const *k_cache
                         const lsa_batch_t *batch, int32_t layers_per_index,
                         float *const *out, void *workspace, size_t workspace_bytes,
                         int32_t *dev_status, void *stream);
+
+/* lsa_attend over an FP8 KV cache. The pages name FP8 variants of the
+ * models and a KV-cache data type but fix neither the format nor its
+ * scaling; this call reads the cache as OCP FP8 E4M3 codes (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits, subnormals, no infinities)
+ * with one scale per layer for K and one for V: k = k_scale[g] * E4M3(code),
+ * v = v_scale[g] * E4M3(code). Everything else — the set, the softmax, the
+ * GQA mapping, the output, the workspace (lsa_attend_workspace_size) and the
+ * device-side errors — is lsa_attend's.
+ *
+ * k_cache, v_cache  host [G] arrays of device uint8 [total_tokens][H_kv][d]
+ *                   E4M3 codes (NaN codes give unspecified output).
+ * k_scale, v_scale  host [G] arrays of finite floats.
+ * Supported: as lsa_attend, with H_q / H_kv <= 8 (else LSA_ERR_UNSUPPORTED).
+ */
+lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_cache,
+                            const uint8_t *const *v_cache, const float *k_scale,
+                            const float *v_scale, int32_t H_q, int32_t H_kv, int32_t d,
+                            const int32_t *index_sets, int32_t budget,
+                            const lsa_batch_t *batch, int32_t layers_per_index,
+                            float *const *out, void *workspace, size_t workspace_bytes,
+                            int32_t *dev_status, void *stream);
 
 /* ----------------------------------------------------------------------- */
 /* Allocation-free attention (no counterpart in the pages)                   */

@@ -8,7 +8,7 @@ the library raises immediately: there is no fallback implementation.
 from __future__ import annotations
 
 _BINDING_NAMES = {
-    "lsa_hi_block_sums", "lsa_append", "lsa_index", "lsa_attend", "lsa_index_workspace_size",
+    "lsa_hi_block_sums", "lsa_append", "lsa_index", "lsa_attend", "lsa_attend_fp8", "lsa_index_workspace_size",
     "lsa_attend_workspace_size", "lsa_version", "Batch", "Budget", "LsaError", "library_path",
     "load_library",
 }

@@ -26,7 +26,7 @@ STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "L
           4: "LSA_ERR_WORKSPACE"}
 
 EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums", "lsa_append",
-           "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend",
+           "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend", "lsa_attend_fp8",
            "lsa_attend_noalloc"]
 
 
@@ -118,7 +118,7 @@ def load_library():
     lib.lsa_hi_block_sums.argtypes = [vp, i32, i32, ctypes.POINTER(_Batch), i32, vp, i64, vp, vp]
     lib.lsa_append.restype = i32
     lib.lsa_append.argtypes = [vp, vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
-                               ctypes.POINTER(vp), i32, i32, i32, i32, vp, i64, ctypes.POINTER(_Batch), i32, vp, vp]
+                               ctypes.POINTER(vp), i32, i32, i32, vp, i64, ctypes.POINTER(_Batch), i32, vp, vp]
     lib.lsa_index_workspace_size.restype = sz
     lib.lsa_index_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
     lib.lsa_index_launches.restype = i32
@@ -134,6 +134,10 @@ def load_library():
     lib.lsa_attend.restype = i32
     lib.lsa_attend.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp, i32,
                                ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, sz, vp, vp]
+    lib.lsa_attend_fp8.restype = i32
+    lib.lsa_attend_fp8.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                   ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float), i32, i32, i32, vp,
+                                   i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, sz, vp, vp]
     lib.lsa_attend_noalloc.restype = i32
     lib.lsa_attend_noalloc.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
                                        i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, vp]
@@ -218,16 +222,17 @@ def lsa_append(k_idx_new: torch.Tensor, k_idx: torch.Tensor, k_new: list, v_new:
                hi_block: int, block_sums: torch.Tensor | None, batch: Batch, n_new: int,
                dev_status: torch.Tensor | None = None, stream=None) -> None:
     """Write the n_new newest tokens of every sequence (keys k_idx_new [n_seq, n_new, d_I], per-layer K/V
-    rows k_new/v_new [n_seq, n_new, H_kv, d]) into the caches and refresh their blocks' sums (HI on)."""
+    rows k_new/v_new [n_seq, n_new, H_kv, d], bf16 or FP8 codes like the caches k/v) into the caches and
+    refresh their blocks' sums (HI on)."""
     lib = load_library()
     G = len(k_new)
     d_I = k_idx.shape[-1]
-    H_kv, d = (k[0].shape[1], k[0].shape[2]) if G else (0, 0)
+    row_bytes = k[0].shape[1] * k[0].shape[2] * k[0].element_size() if G else 0
     arr = ctypes.c_void_p * max(G, 1)
     kn, vn, kc, vc = (arr(*[t.data_ptr() for t in x]) for x in (k_new, v_new, k, v))
     cb = batch.c()
     rows = block_sums.shape[0] if block_sums is not None else 0
-    st = lib.lsa_append(_ptr(k_idx_new), _ptr(k_idx), d_I, kn, vn, kc, vc, H_kv, d, G, hi_block, _ptr(block_sums),
+    st = lib.lsa_append(_ptr(k_idx_new), _ptr(k_idx), d_I, kn, vn, kc, vc, row_bytes, G, hi_block, _ptr(block_sums),
                         rows, ctypes.byref(cb), n_new, _ptr(dev_status), _stream(stream))
     _check("lsa_append", st)
 
@@ -246,6 +251,25 @@ def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch
                         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
                         _stream(stream))
     _check("lsa_attend", st)
+
+
+def lsa_attend_fp8(q: list, k8: list, v8: list, k_scale: list, v_scale: list, index_sets: torch.Tensor,
+                   batch: Batch, out: list, workspace: torch.Tensor, dev_status: torch.Tensor | None = None,
+                   stream=None) -> None:
+    """lsa_attend over FP8 E4M3 K/V caches (uint8 tensors [T, H_kv, d]) with per-layer scales."""
+    lib = load_library()
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k8[0].shape[1]
+    arr = ctypes.c_void_p * G
+    qa, ka, va, oa = (arr(*[t.data_ptr() for t in x]) for x in (q, k8, v8, out))
+    fa = ctypes.c_float * G
+    ks, vs = fa(*[float(x) for x in k_scale]), fa(*[float(x) for x in v_scale])
+    cb = batch.c()
+    st = lib.lsa_attend_fp8(qa, ka, va, ks, vs, H_q, H_kv, d, _ptr(index_sets), index_sets.shape[1],
+                            ctypes.byref(cb), G, oa, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _ptr(dev_status), _stream(stream))
+    _check("lsa_attend_fp8", st)
 
 
 def lsa_attend_noalloc(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list,

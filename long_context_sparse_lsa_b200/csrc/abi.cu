@@ -115,9 +115,9 @@ lsa_status_t lsa_hi_block_sums(const int8_t* k_idx_cache, int32_t d_I, int32_t h
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 
-lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_I, const uint16_t* const* k_new,
-                        const uint16_t* const* v_new, uint16_t* const* k_cache, uint16_t* const* v_cache,
-                        int32_t H_kv, int32_t d, int32_t layers, int32_t hi_block, int8_t* block_sums,
+lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_I, const void* const* k_new,
+                        const void* const* v_new, void* const* k_cache, void* const* v_cache,
+                        int32_t kv_row_bytes, int32_t layers, int32_t hi_block, int8_t* block_sums,
                         int64_t block_rows, const lsa_batch_t* batch, int32_t n_new, int32_t* dev_status,
                         void* stream) {
     if (!batch_ok(batch, false)) return LSA_ERR_INVALID_ARG;
@@ -129,7 +129,7 @@ lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_
     if (hi_block > 0 && (block_sums == nullptr || batch->blk_offset == nullptr || !aligned(block_sums, 16)))
         return LSA_ERR_INVALID_ARG;
     if (layers > 0) {
-        if (d != 128 || H_kv < 1) return d != 128 ? LSA_ERR_UNSUPPORTED : LSA_ERR_INVALID_ARG;
+        if (kv_row_bytes < 16 || kv_row_bytes % 16 != 0) return LSA_ERR_INVALID_ARG;
         if (k_new == nullptr || v_new == nullptr || k_cache == nullptr || v_cache == nullptr)
             return LSA_ERR_INVALID_ARG;
         for (int g = 0; g < layers; ++g) {
@@ -164,7 +164,7 @@ lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_
         a.v_cache[g] = v_cache[g];
     }
     a.layers = layers;
-    a.kv_row_bytes = layers > 0 ? H_kv * d * 2 : 0;
+    a.kv_row_bytes = layers > 0 ? kv_row_bytes : 0;
     a.sums = hi_block > 0 ? 1 : 0;
     cudaError_t e = lsa::launch_append(a, d_I, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
@@ -320,15 +320,27 @@ int32_t lsa_attend_launches(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv,
     return p.n_splits > 1 ? 2 : 1;  // attention[, split merge]
 }
 
-lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache, const uint16_t* const* v_cache,
-                        int32_t H_q, int32_t H_kv, int32_t d, const int32_t* index_sets, int32_t budget,
-                        const lsa_batch_t* batch, int32_t layers_per_index, float* const* out, void* workspace,
-                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+}  // extern "C"
+
+// lsa_attend and lsa_attend_fp8: k_cache / v_cache point at bf16 elements, or
+// at E4M3 codes when kscale / vscale are given (FP8).
+static lsa_status_t attend_impl(const uint16_t* const* q, const void* const* k_cache, const void* const* v_cache,
+                                const float* kscale, const float* vscale, int32_t H_q, int32_t H_kv, int32_t d,
+                                const int32_t* index_sets, int32_t budget, const lsa_batch_t* batch,
+                                int32_t layers_per_index, float* const* out, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, void* stream) {
+    const bool fp8 = kscale != nullptr;
     if (!batch_ok(batch, true)) return LSA_ERR_INVALID_ARG;
     if (H_q < 1 || H_kv < 1 || d < 1 || budget < 0 || layers_per_index < 1) return LSA_ERR_INVALID_ARG;
     if (H_q % H_kv != 0) return LSA_ERR_INVALID_ARG;
     if (!attend_shape_ok(H_q, H_kv, d, budget, layers_per_index)) return LSA_ERR_UNSUPPORTED;
+    if (fp8 && H_q / H_kv > 8) return LSA_ERR_UNSUPPORTED;
     if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr) return LSA_ERR_INVALID_ARG;
+    if (fp8) {
+        if (vscale == nullptr) return LSA_ERR_INVALID_ARG;
+        for (int g = 0; g < layers_per_index; ++g)
+            if (!std::isfinite(kscale[g]) || !std::isfinite(vscale[g])) return LSA_ERR_INVALID_ARG;
+    }
     if (batch->n_q == 0) return LSA_OK;
     if (budget > 0 && (index_sets == nullptr || !aligned(index_sets, 4))) return LSA_ERR_INVALID_ARG;
     for (int g = 0; g < layers_per_index; ++g) {
@@ -345,10 +357,13 @@ lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache
     std::memset(&a, 0, sizeof a);
     for (int g = 0; g < layers_per_index; ++g) {
         a.q[g] = q[g];
-        a.k[g] = k_cache[g];
-        a.v[g] = v_cache[g];
+        a.k[g] = static_cast<const uint16_t*>(k_cache[g]);
+        a.v[g] = static_cast<const uint16_t*>(v_cache[g]);
         a.out[g] = out[g];
+        a.kscale[g] = fp8 ? kscale[g] : 1.f;
+        a.vscale[g] = fp8 ? vscale[g] : 1.f;
     }
+    a.kv_fp8 = fp8 ? 1 : 0;
     a.sets = index_sets;
     a.kv_offset = batch->kv_offset;
     a.seq_lens = batch->seq_lens;
@@ -381,6 +396,28 @@ lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     cudaError_t e = lsa::launch_attend(a, p.smem_bytes, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+extern "C" {
+
+lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache, const uint16_t* const* v_cache,
+                        int32_t H_q, int32_t H_kv, int32_t d, const int32_t* index_sets, int32_t budget,
+                        const lsa_batch_t* batch, int32_t layers_per_index, float* const* out, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    return attend_impl(q, reinterpret_cast<const void* const*>(k_cache), reinterpret_cast<const void* const*>(v_cache),
+                       nullptr, nullptr, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, workspace,
+                       workspace_bytes, dev_status, stream);
+}
+
+lsa_status_t lsa_attend_fp8(const uint16_t* const* q, const uint8_t* const* k_cache, const uint8_t* const* v_cache,
+                            const float* k_scale, const float* v_scale, int32_t H_q, int32_t H_kv, int32_t d,
+                            const int32_t* index_sets, int32_t budget, const lsa_batch_t* batch,
+                            int32_t layers_per_index, float* const* out, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+    if (k_scale == nullptr || v_scale == nullptr) return LSA_ERR_INVALID_ARG;
+    return attend_impl(q, reinterpret_cast<const void* const*>(k_cache), reinterpret_cast<const void* const*>(v_cache),
+                       k_scale, v_scale, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, workspace,
+                       workspace_bytes, dev_status, stream);
 }
 
 }  // extern "C"

@@ -35,6 +35,8 @@
 //  * Every mbarrier wait is bounded by a time limit; on expiry the kernel
 //    flags LSA_DEV_TIMEOUT, waits (bounded) for the copies it issued and
 //    returns.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -81,7 +83,7 @@ __device__ __forceinline__ uint32_t word(const uint4& x, int j) {
 // Online softmax of one 16-token tile's scores (sacc: S^T fragments, tokens g
 // and g+8 of this lane, masked where ok_g / ok_g8 is false) and O^T += V^T P^T
 // from the tile's V registers.
-template <int NT>
+template <int NT, bool F16 = false>
 __device__ __forceinline__ void softmax_pv(const float (&sacc)[NT][4], bool ok_g, bool ok_g8, float scale_log2,
                                            float (&m_run)[NT][2], float (&l_run)[NT][2], float (&o)[NT][kD / 16][4],
                                            const VTile& v) {
@@ -120,13 +122,23 @@ __device__ __forceinline__ void softmax_pv(const float (&sacc)[NT][4], bool ok_g
                 o[n][mt][3] *= al1;
             }
         }
-        const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
-        const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
-        const float2 fh01 = __bfloat1622float2(h01), fh23 = __bfloat1622float2(h23);
-        phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
-        phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-        plo[n][0] = movmatrix_trans(pack_bf16(p0 - fh01.x, p1 - fh01.y));
-        plo[n][1] = movmatrix_trans(pack_bf16(p2 - fh23.x, p3 - fh23.y));
+        if constexpr (F16) {
+            const __half2 h01 = __floats2half2_rn(p0, p1);
+            const __half2 h23 = __floats2half2_rn(p2, p3);
+            const float2 fh01 = __half22float2(h01), fh23 = __half22float2(h23);
+            phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+            phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+            plo[n][0] = movmatrix_trans(pack_f16(p0 - fh01.x, p1 - fh01.y));
+            plo[n][1] = movmatrix_trans(pack_f16(p2 - fh23.x, p3 - fh23.y));
+        } else {
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(p0, p1);
+            const __nv_bfloat162 h23 = __floats2bfloat162_rn(p2, p3);
+            const float2 fh01 = __bfloat1622float2(h01), fh23 = __bfloat1622float2(h23);
+            phi[n][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+            phi[n][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+            plo[n][0] = movmatrix_trans(pack_bf16(p0 - fh01.x, p1 - fh01.y));
+            plo[n][1] = movmatrix_trans(pack_bf16(p2 - fh23.x, p3 - fh23.y));
+        }
     }
     // O^T += V^T P^T from the registers of this tile's V
 #pragma unroll
@@ -138,8 +150,8 @@ __device__ __forceinline__ void softmax_pv(const float (&sacc)[NT][4], bool ok_g
                                  __byte_perm(w8, w9, 0x5410), __byte_perm(w8, w9, 0x7632)};
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            mma_bf16(o[n][mt], vfr, phi[n][0], phi[n][1]);
-            mma_bf16(o[n][mt], vfr, plo[n][0], plo[n][1]);
+            mma_16<F16>(o[n][mt], vfr, phi[n][0], phi[n][1]);
+            mma_16<F16>(o[n][mt], vfr, plo[n][0], plo[n][1]);
         }
     }
 }
@@ -153,7 +165,8 @@ __device__ __forceinline__ void softmax_pv(const float (&sacc)[NT][4], bool ok_g
 template <int NT>
 __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* merge_area, float (&o)[NT][kD / 16][4],
                                                 float (&m_run)[NT][2], float (&l_run)[NT][2], int warp, int lane,
-                                                int hpc, int hgrp, int r, int layer, int split, int ratio) {
+                                                int hpc, int hgrp, int r, int layer, int split, int ratio,
+                                                float vs = 1.f) {
     const int g = lane >> 2, t4 = lane & 3;
     // ---- merge the consumers of each kv head, in registers ----
     // All warps hold O^T in the same fragment layout, so warps with wsel > 0
@@ -216,7 +229,7 @@ __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* me
                 const float inv = l_run[n][c] > 0.f ? 1.f / l_run[n][c] : 0.f;
                 float* dst = direct ? a.out[layer] + ((int64_t)r * a.H_q + qh) * kD
                                     : a.part_o + ((row_q * a.n_splits + split) * a.H_q + qh) * kD;
-                const float sc = direct ? inv : 1.f;
+                const float sc = direct ? inv * vs : vs;  // vs: the FP8 V scale (1 for bf16)
 #pragma unroll
                 for (int mt = 0; mt < kD / 16; ++mt) {
                     const int d0 = 8 * ((mt >> 2) ? 8 + g : g) + 2 * (mt & 3);
@@ -456,11 +469,95 @@ __device__ __forceinline__ void load_ktile(KTile& k, const uint16_t* kbase, int6
     }
 }
 
+// ---- FP8 (E4M3) K/V ---------------------------------------------------------
+// With an FP8 cache each element is one byte: a lane loads the same dims as in
+// the bf16 tiles (8-byte chunks instead of 16-byte ones) and converts them to
+// fp16 at use. Every E4M3 value is an fp16 exactly, and so is every bf16 query
+// element in [2^-14, 65504] (the rest are fp16 subnormals or zero), so the
+// MMAs run in fp16; the per-layer scales multiply the scores (K) and the
+// output (V) in fp32.
+struct KTile8 {
+    uint2 r[2][4];
+};
+struct VTile8 {
+    uint2 r[4][2];
+};
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {  // bits 0..15: two codes, low first
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+__device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 c) {
+    return make_uint4(e4m3x2_to_f16x2(c.x), e4m3x2_to_f16x2(c.x >> 16), e4m3x2_to_f16x2(c.y),
+                      e4m3x2_to_f16x2(c.y >> 16));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
+    return pack_f16(f.x, f.y);
+}
+
+__device__ __forceinline__ void load_ktile8(KTile8& k, const uint8_t* kbase, int64_t tok_stride, const int32_t* ent,
+                                            int g, int t4) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int e = ent[g + 8 * rr];
+        if (e >= 0) {
+            const uint8_t* p = kbase + (int64_t)e * tok_stride + 8 * t4;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) k.r[rr][j] = ldg8(p + 32 * j);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) k.r[rr][j] = make_uint2(0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ void load_vtile8(VTile8& v, const uint8_t* vbase, int64_t tok_stride, const int32_t* ent,
+                                            int g, int t4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int row = 2 * t4 + (j & 1) + 8 * (j >> 1);
+        const int e = ent[row];
+        if (e >= 0) {
+            const uint8_t* p = vbase + (int64_t)e * tok_stride;
+            v.r[j][0] = ldg8(p + 8 * g);
+            v.r[j][1] = ldg8(p + 64 + 8 * g);
+        } else {
+            v.r[j][0] = make_uint2(0, 0);
+            v.r[j][1] = make_uint2(0, 0);
+        }
+    }
+}
+
+// The 16-bit fragments of a tile: bf16 tiles as they are, FP8 tiles converted.
+__device__ __forceinline__ const KTile& frag16(const KTile& k) { return k; }
+__device__ __forceinline__ const VTile& frag16(const VTile& v) { return v; }
+__device__ __forceinline__ KTile frag16(const KTile8& k) {
+    KTile x;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x.r[rr][j] = e4m3x8_to_f16(k.r[rr][j]);
+    return x;
+}
+__device__ __forceinline__ VTile frag16(const VTile8& v) {
+    VTile x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) x.r[j][c] = e4m3x8_to_f16(v.r[j][c]);
+    return x;
+}
+
 // The register-streaming variant (GQA groups of at most 8 query heads): every
 // warp gathers its own K and V rows with 16-byte loads straight into MMA
 // fragments, two tiles ahead of use, so no copy engine, shared-memory ring or
 // producer warp sits between HBM and the tensor cores. Eight warps per CTA;
 // warp w owns kv head w % hpc of the CTA and every (8/hpc)-th tile.
+// FP8: the K/V caches hold E4M3 codes (see the FP8 tiles above).
+template <bool FP8>
 __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const __grid_constant__ AttendArgs a) {
     constexpr int NT = 1;
     pdl_enter();
@@ -526,10 +623,21 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
     const int wsel = warp / hpc;
     const int n_sel = kConsumers / hpc;
     const int kvh = hgrp * hpc + h_local;
-    const int64_t tok_stride = (int64_t)a.H_kv * kD;
-    const uint16_t* kbase = a.k[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
-    const uint16_t* vbase = a.v[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
-    // query fragments in the permuted dim order of KTile
+    const int64_t tok_stride = (int64_t)a.H_kv * kD;  // elements (= bytes for FP8)
+    constexpr int kEB = FP8 ? 1 : 2;                    // bytes per element
+    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k[layer]) + (off * a.H_kv + (int64_t)kvh) * kD * kEB;
+    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v[layer]) + (off * a.H_kv + (int64_t)kvh) * kD * kEB;
+    using KT = std::conditional_t<FP8, KTile8, KTile>;
+    using VT = std::conditional_t<FP8, VTile8, VTile>;
+    auto load_k = [&](KT& k, const int32_t* ent) {
+        if constexpr (FP8) load_ktile8(k, kbase, tok_stride, ent, g, t4);
+        else load_ktile(k, reinterpret_cast<const uint16_t*>(kbase), tok_stride, ent, g, t4);
+    };
+    auto load_v = [&](VT& v, const int32_t* ent) {
+        if constexpr (FP8) load_vtile8(v, vbase, tok_stride, ent, g, t4);
+        else load_vtile(v, reinterpret_cast<const uint16_t*>(vbase), tok_stride, ent, g, t4);
+    };
+    // query fragments in the permuted dim order of KTile (fp16 for FP8 caches)
     uint32_t qb[kD / 16][2];
     {
         const uint16_t* qrow = a.q[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
@@ -539,36 +647,44 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
             const uint16_t* p = qrow + g * kD + 8 * (t4 + 4 * (ks >> 1)) + 4 * (ks & 1);
             qb[ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p)) : 0u;
             qb[ks][1] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p + 2)) : 0u;
+            if constexpr (FP8) {
+                qb[ks][0] = bf16x2_to_f16x2(qb[ks][0]);
+                qb[ks][1] = bf16x2_to_f16x2(qb[ks][1]);
+            }
         }
     }
-    KTile ka, kb2;
-    VTile va, vb2;
+    const float sl2 = FP8 ? a.scale_log2 * a.kscale[layer] : a.scale_log2;
+    KT ka, kb2;
+    VT va, vb2;
     if (wsel < n_tiles) {
-        load_ktile(ka, kbase, tok_stride, s_ent + wsel * kTile, g, t4);
-        load_vtile(va, vbase, tok_stride, s_ent + wsel * kTile, g, t4);
+        load_k(ka, s_ent + wsel * kTile);
+        load_v(va, s_ent + wsel * kTile);
     }
     if (wsel + n_sel < n_tiles) {
-        load_ktile(kb2, kbase, tok_stride, s_ent + (wsel + n_sel) * kTile, g, t4);
-        load_vtile(vb2, vbase, tok_stride, s_ent + (wsel + n_sel) * kTile, g, t4);
+        load_k(kb2, s_ent + (wsel + n_sel) * kTile);
+        load_v(vb2, s_ent + (wsel + n_sel) * kTile);
     }
-    auto tile = [&](int i, KTile& k, VTile& v) {
+    auto tile = [&](int i, KT& k, VT& v) {
         const int ent_lane = lane < kTile ? s_ent[i * kTile + lane] : 0;
         const uint32_t masked = __ballot_sync(0xffffffffu, lane < kTile && ent_lane < 0);
         const bool ok_g = !((masked >> g) & 1u);
         const bool ok_g8 = !((masked >> (g + 8)) & 1u);
         float sacc[NT][4] = {{0.f, 0.f, 0.f, 0.f}};
+        {
+            const auto& kf = frag16(k);
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            const int j = ks >> 1, w = 2 * (ks & 1);
-            const uint32_t afr[4] = {word(k.r[0][j], w), word(k.r[1][j], w), word(k.r[0][j], w + 1),
-                                     word(k.r[1][j], w + 1)};
-            mma_bf16(sacc[0], afr, qb[ks][0], qb[ks][1]);
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                const int j = ks >> 1, w = 2 * (ks & 1);
+                const uint32_t afr[4] = {word(kf.r[0][j], w), word(kf.r[1][j], w), word(kf.r[0][j], w + 1),
+                                         word(kf.r[1][j], w + 1)};
+                mma_16<FP8>(sacc[0], afr, qb[ks][0], qb[ks][1]);
+            }
         }
-        softmax_pv<NT>(sacc, ok_g, ok_g8, a.scale_log2, m_run, l_run, o, v);
+        softmax_pv<NT, FP8>(sacc, ok_g, ok_g8, sl2, m_run, l_run, o, frag16(v));
         // K and V two tiles ahead, in flight during the next tile's math
         if (i + 2 * n_sel < n_tiles) {
-            load_ktile(k, kbase, tok_stride, s_ent + (i + 2 * n_sel) * kTile, g, t4);
-            load_vtile(v, vbase, tok_stride, s_ent + (i + 2 * n_sel) * kTile, g, t4);
+            load_k(k, s_ent + (i + 2 * n_sel) * kTile);
+            load_v(v, s_ent + (i + 2 * n_sel) * kTile);
         }
     };
     for (int i = wsel; i < n_tiles; i += 2 * n_sel) {
@@ -581,7 +697,8 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
 #pragma unroll
         for (int msk = 4; msk < 32; msk <<= 1) l_run[0][j] += __shfl_xor_sync(0xffffffffu, l_run[0][j], msk);
     __syncthreads();  // the merge area reuses the entry list
-    merge_and_store<NT>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, hpc, hgrp, r, layer, split, ratio);
+    merge_and_store<NT>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, hpc, hgrp, r, layer, split, ratio,
+                        FP8 ? a.vscale[layer] : 1.f);
 }
 
 // Split merge: one warp per (query head, row, layer); lane l owns dims
@@ -693,12 +810,13 @@ cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t s
     const int ratio = a.H_q / a.H_kv;
     dim3 grid((unsigned)(a.n_splits * a.head_groups), (unsigned)a.n_q, (unsigned)a.G);
     if (ratio <= 8) {
-        cudaError_t e = cudaFuncSetAttribute(attend_rk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem_bytes);
+        auto kern = a.kv_fp8 ? attend_rk_kernel<true> : attend_rk_kernel<false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
         if (e != cudaSuccess) return e;
-        e = launch_pdl(attend_rk_kernel, grid, dim3(kConsumers * kWarp), smem_bytes, stream, 0, a);
+        e = launch_pdl(kern, grid, dim3(kConsumers * kWarp), smem_bytes, stream, 0, a);
         if (e != cudaSuccess) return e;
     } else {
+        if (a.kv_fp8) return cudaErrorInvalidValue;  // FP8 caches: groups of at most 8 query heads
         cudaError_t e = cudaFuncSetAttribute(attend_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem_bytes);
         if (e != cudaSuccess) return e;

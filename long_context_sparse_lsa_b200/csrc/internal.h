@@ -38,12 +38,12 @@ struct AppendArgs {
     BlockSumArgs bs;               // k_idx: the cache being written; n_new > 0
     const int8_t* k_idx_new;       // [n_seq][n_new][d_I]
     int8_t* k_idx_cache;           // == bs.k_idx
-    const uint16_t* k_new[kMaxLayers];  // [n_seq][n_new][H_kv][d] per layer
-    const uint16_t* v_new[kMaxLayers];
-    uint16_t* k_cache[kMaxLayers];      // [total_tokens][H_kv][d] per layer
-    uint16_t* v_cache[kMaxLayers];
+    const void* k_new[kMaxLayers];  // [n_seq][n_new] rows of kv_row_bytes, per layer
+    const void* v_new[kMaxLayers];
+    void* k_cache[kMaxLayers];      // [total_tokens] rows of kv_row_bytes, per layer
+    void* v_cache[kMaxLayers];
     int32_t layers;
-    int32_t kv_row_bytes;          // H_kv * d * 2
+    int32_t kv_row_bytes;          // one token's K (or V) row of one layer
     int32_t sums;                  // 1: recompute the block sums (HI on)
 };
 cudaError_t launch_append(const AppendArgs& a, int d_I, cudaStream_t stream);
@@ -142,6 +142,8 @@ struct AttendArgs {
     int32_t hpc;          // kv heads per CTA
     int32_t n_stages, row_stride, bar_off, stage_off;  // shared-memory plan
     float scale_log2;     // log2(e) / sqrt(d)
+    int32_t kv_fp8;       // K/V caches hold FP8 E4M3 codes (k, v point at bytes)
+    float kscale[kMaxLayers], vscale[kMaxLayers];  // FP8: value = scale * E4M3(code)
 };
 
 struct AttendPlan {

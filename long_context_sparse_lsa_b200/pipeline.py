@@ -12,15 +12,26 @@ from __future__ import annotations
 import torch
 
 from . import binding as lsa
+from . import inputs as gen
 from .workloads import Tensors, Workload
 
 
 class LsaStep:
-    def __init__(self, wl: Workload, t: Tensors, device="cuda"):
+    def __init__(self, wl: Workload, t: Tensors, device="cuda", kv_fp8: bool = False):
+        """kv_fp8: the K/V caches are FP8 E4M3 codes (drawn here, per layer,
+        with scales k_scale / v_scale) and the attention is lsa_attend_fp8;
+        the bf16 caches of `t` are then unused and may be empty."""
         self.wl = wl
         self.t = t
         self.device = device
         self.G = len(t.q)
+        self.kv_fp8 = kv_fp8
+        if kv_fp8:
+            shape = (wl.total_tokens, wl.H_kv, wl.d)
+            self.k8 = [gen.normal_e4m3(shape, wl.seed, gen.STREAM_K8 + g, device) for g in range(self.G)]
+            self.v8 = [gen.normal_e4m3(shape, wl.seed, gen.STREAM_V8 + g, device) for g in range(self.G)]
+            self.k_scale = [0.75 + 0.25 * g for g in range(self.G)]
+            self.v_scale = [1.5 - 0.25 * g for g in range(self.G)]
         self.batch = lsa.Batch(t.kv_offset, t.seq_lens, t.q_seq, t.q_len, max(wl.lens), wl.total_tokens,
                                t.blk_offset if wl.hi_block > 0 else None)
         self.budget = lsa.Budget(wl.sink, wl.window, wl.topk, wl.hi_block, wl.hi_topblocks)
@@ -45,8 +56,9 @@ class LsaStep:
                                dtype=torch.int64, device=device)
             n_seq = len(lens)
             self.k_idx_new = t.k_idx.index_select(0, pos).view(n_seq, self.n_new, wl.d_I).clone()
-            self.k_new = [x.index_select(0, pos).view(n_seq, self.n_new, wl.H_kv, wl.d).clone() for x in t.k]
-            self.v_new = [x.index_select(0, pos).view(n_seq, self.n_new, wl.H_kv, wl.d).clone() for x in t.v]
+            kc, vc = self.kv_caches()
+            self.k_new = [x.index_select(0, pos).view(n_seq, self.n_new, wl.H_kv, wl.d).clone() for x in kc]
+            self.v_new = [x.index_select(0, pos).view(n_seq, self.n_new, wl.H_kv, wl.d).clone() for x in vc]
 
     # -- the three calls --------------------------------------------------------
     def build_block_sums(self, stream=None):
@@ -58,11 +70,16 @@ class LsaStep:
             lsa.lsa_hi_block_sums(self.t.k_idx, self.wl.hi_block, self.batch, self.block_sums, n_new, self.status,
                                   stream)
 
+    def kv_caches(self):
+        """The K and V caches the attention reads (FP8 codes or bf16)."""
+        return (self.k8, self.v8) if self.kv_fp8 else (self.t.k, self.t.v)
+
     def append(self, stream=None):
         """The decode append: write the newest tokens' keys and K/V rows and
         refresh the block sums of their blocks (one launch)."""
         if self.n_new:
-            lsa.lsa_append(self.k_idx_new, self.t.k_idx, self.k_new, self.v_new, self.t.k, self.t.v,
+            kc, vc = self.kv_caches()
+            lsa.lsa_append(self.k_idx_new, self.t.k_idx, self.k_new, self.v_new, kc, vc,
                            self.wl.hi_block, self.block_sums, self.batch, self.n_new, self.status, stream)
 
     def index(self, stream=None):
@@ -70,8 +87,12 @@ class LsaStep:
                       self.block_sums, self.ws_index, self.status, stream)
 
     def attend(self, stream=None):
-        lsa.lsa_attend(self.t.q, self.t.k, self.t.v, self.sets, self.batch, self.out, self.ws_attend, self.status,
-                       stream)
+        if self.kv_fp8:
+            lsa.lsa_attend_fp8(self.t.q, self.k8, self.v8, self.k_scale, self.v_scale, self.sets, self.batch,
+                               self.out, self.ws_attend, self.status, stream)
+        else:
+            lsa.lsa_attend(self.t.q, self.t.k, self.t.v, self.sets, self.batch, self.out, self.ws_attend,
+                           self.status, stream)
 
     def step(self, stream=None):
         """One decode step: append, index, attend."""

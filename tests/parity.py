@@ -68,6 +68,30 @@ def oracle_attend_rows(t, sets, rows):
     return outs
 
 
+def oracle_attend_rows_fp8(st, sets, rows):
+    """oracle_attend_rows for a step whose K/V caches are FP8 codes
+    (st.k8 / st.v8 with per-layer scales st.k_scale / st.v_scale)."""
+    orc = oracle.get()
+    t = st.t
+    kv_off = host(t.kv_offset)
+    q_seq = host(t.q_seq)
+    outs = []
+    for g in range(len(t.q)):
+        per = []
+        for i, r in enumerate(rows):
+            s = sets[i]
+            valid = s[s >= 0]
+            base = int(kv_off[q_seq[r]])
+            idx = torch.as_tensor(valid.astype(np.int64) + base, device=st.k8[g].device)
+            kr = host(st.k8[g].index_select(0, idx))
+            vr = host(st.v8[g].index_select(0, idx))
+            local = np.full(s.shape[0], -1, np.int32)
+            local[: valid.shape[0]] = np.arange(valid.shape[0], dtype=np.int32)
+            per.append(orc.attend_query_fp8(u16(t.q[g][r]), kr, vr, st.k_scale[g], st.v_scale[g], local))
+        outs.append(np.stack(per))
+    return outs
+
+
 def check_attention(got: np.ndarray, want: np.ndarray, what=""):
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)

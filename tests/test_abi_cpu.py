@@ -98,17 +98,18 @@ def test_block_sums_rejects():
 
 def _append(lib, **kw):
     arr = (ctypes.c_void_p * 2)(P, P)
-    args = dict(kin=P, kc=P, d_I=128, kn=arr, vn=arr, kcache=arr, vcache=arr, H_kv=4, d=128, layers=2, hb=64,
+    args = dict(kin=P, kc=P, d_I=128, kn=arr, vn=arr, kcache=arr, vcache=arr, kvb=1024, layers=2, hb=64,
                 bs=P, rows=10, batch=_batch(), n_new=1)
     args.update(kw)
     return lib.lsa_append(args["kin"], args["kc"], args["d_I"], args["kn"], args["vn"], args["kcache"],
-                          args["vcache"], args["H_kv"], args["d"], args["layers"], args["hb"], args["bs"],
+                          args["vcache"], args["kvb"], args["layers"], args["hb"], args["bs"],
                           args["rows"], ctypes.byref(args["batch"]), args["n_new"], None, None)
 
 
 @pytest.mark.parametrize("kw,want", [
     (dict(n_new=0), 1), (dict(kin=None), 1), (dict(kc=None), 1), (dict(kc=P + 8), 1), (dict(d_I=48), 2),
-    (dict(layers=9), 2), (dict(layers=-1), 1), (dict(d=64), 2), (dict(kn=None), 1), (dict(hb=300), 2),
+    (dict(layers=9), 2), (dict(layers=-1), 1), (dict(kvb=1000), 1), (dict(kvb=0), 1), (dict(kn=None), 1),
+    (dict(hb=300), 2),
     (dict(bs=None), 1), (dict(batch=_batch(n_seq=0)), 1),
     (dict(kn=(ctypes.c_void_p * 2)(P, None)), 1),   # a null layer pointer
     (dict(vcache=(ctypes.c_void_p * 2)(P, P + 4)), 1),  # a misaligned layer pointer
@@ -116,6 +117,21 @@ def _append(lib, **kw):
 def test_append_rejects_before_launch(kw, want):
     lib = lsa.load_library()
     assert _append(lib, **kw) == want
+
+
+def test_attend_fp8_rejects_before_launch():
+    lib = lsa.load_library()
+    b = _batch(n_q=16, max_len=131072, total=16 * 131072)
+    arr = (ctypes.c_void_p * 1)(P)
+    one = (ctypes.c_float * 1)(1.0)
+    bad = (ctypes.c_float * 1)(float("inf"))
+    f = lib.lsa_attend_fp8
+    args = lambda H_q=32, ks=one, vs=one: (arr, arr, arr, ks, vs, H_q, 4, 128, P, 3136, ctypes.byref(b), 1, arr, P,
+                                           1 << 30, None, None)
+    assert f(*args(ks=None)) == 1
+    assert f(*args(vs=None)) == 1
+    assert f(*args(ks=bad)) == 1
+    assert f(*args(H_q=64)) == 2  # groups of 16 query heads: bf16 caches only
 
 
 def test_attend_rejects_and_sizes():

@@ -84,6 +84,29 @@ def test_ragged_batch_sample():
     _release(st, t)
 
 
+def test_fp8_kv_decode_128k_sample():
+    """The 16 x 131072 decode with FP8 E4M3 K/V caches, through the step graph
+    the bench times: index sets bit-exact on every row, the FP8 attention of a
+    sample of rows against the oracle's."""
+    wl = wls.BATCH128K
+    t = wls.make(wl, DEV, with_kv=False)
+    st = LsaStep(wl, t, DEV, kv_fp8=True)
+    st.build_block_sums()
+    torch.cuda.synchronize()
+    st.capture()
+    st.sets.fill_(-7)
+    st.replay()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    rows = np.arange(wl.n_q)
+    want = parity.oracle_sets(wl, t, rows=rows)
+    parity.check_sets(parity.host(st.sets), want, wl.name)
+    sample = np.array([0, 5, 11, 15])
+    ref = parity.oracle_attend_rows_fp8(st, want[sample], sample)
+    parity.check_attention(parity.host(st.out[0])[sample], ref[0], "fp8 128k")
+    _release(st, t)
+
+
 def test_prefill_chunk_sample():
     wl = wls.PREFILL
     st, t = _run_graph(wl)

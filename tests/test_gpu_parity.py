@@ -295,6 +295,30 @@ def test_draft_rows_per_sequence():
         parity.check_attention(parity.host(st.out[g]), ref[g], f"{wl.name} layer {g}")
 
 
+@pytest.mark.parametrize("lens,hi,G", [((6000,) * 16, False, 2), ((37, 1, 4096, 513, 2049), False, 1),
+                                       ((20000, 17000, 9000), True, 2)])
+def test_fp8_kv_attention(lens, hi, G):
+    """Attention over FP8 E4M3 K/V caches with per-layer scales against the
+    oracle's FP8 attention: 16 rows split 9 ways (two layers), ragged short
+    rows including a one-token sequence, and an HI-selected set."""
+    kw = dict(hi_block=64, hi_topblocks=64) if hi else dict(hi_block=0, hi_topblocks=0)
+    wl = wls.small(BASE, name="fp8", lens=lens, G=G, seed=41, **kw)
+    t = wls.make(wl, DEV, with_kv=False)
+    st = LsaStep(wl, t, DEV, kv_fp8=True)
+    st.build_block_sums()
+    st.index()
+    st.out[0].fill_(float("nan"))
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    rows = np.arange(wl.n_q)
+    want = parity.oracle_sets(wl, t, rows=rows)
+    parity.check_sets(parity.host(st.sets), want, wl.name)
+    ref = parity.oracle_attend_rows_fp8(st, want, rows)
+    for g in range(G):
+        parity.check_attention(parity.host(st.out[g]), ref[g], f"fp8 layer {g}")
+
+
 def test_graph_replay_matches_eager():
     wl = wls.small(BASE, name="graph", lens=(30000, 4000, 9000), hi_block=64, hi_topblocks=64, G=2, seed=13)
     t = wls.make(wl, DEV)
