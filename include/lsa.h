@@ -29,8 +29,10 @@
  * Conventions for every entry point:
  *  - Pointers marked "device" are CUDA device pointers (e.g. a torch tensor's
  *    data_ptr()); pointers marked "host" are ordinary host memory read during
- *    the call. The caller owns every buffer; the library allocates nothing,
- *    keeps no state between calls, and never frees caller memory.
+ *    the call. The caller owns every buffer; the library allocates nothing
+ *    and never frees caller memory. Between calls it keeps only read-only
+ *    facts (each device's SM count, the driver's tensor-map entry point) and
+ *    the static scratch of lsa_attend_noalloc.
  *  - `stream` is a cudaStream_t passed as void*. Every call is asynchronous
  *    on that stream and returns without synchronising.
  *  - Argument and shape errors are returned synchronously, before any launch,
@@ -40,10 +42,12 @@
  *    are OR-ed as LSA_DEV_* bits into *dev_status (device int32, may be
  *    NULL); the caller reads it after synchronising. The offending query's
  *    output is then unspecified but every access stays in bounds.
- *  - No kernel waits on another CTA, kernel or device. Waits inside a CTA
- *    (on its own asynchronous copies) are bounded by a time limit after which
- *    the kernel sets LSA_DEV_TIMEOUT and returns, so no call can hang; no
- *    kernel traps.
+ *  - No kernel spins on another CTA, kernel or device. The only cross-CTA
+ *    waits are hardware barriers: thread-block-cluster barriers (a cluster's
+ *    CTAs are scheduled together) and the programmatic-launch wait for the
+ *    preceding kernel on the stream. Waits on a CTA's own asynchronous copies
+ *    are bounded by a time limit after which the kernel sets LSA_DEV_TIMEOUT
+ *    and returns, so no call can hang; no kernel traps.
  *  - Calls are thread-safe when they use distinct workspaces.
  */
 #ifndef LSA_H_
