@@ -16,6 +16,22 @@ from . import inputs as gen
 from .workloads import Tensors, Workload
 
 
+def _pack(tensors, device):
+    """One contiguous uint8 device buffer holding copies of `tensors`, each
+    at a 256-byte aligned offset, and the views of it that replace them."""
+    offs, total = [], 0
+    for x in tensors:
+        offs.append(total)
+        total += (x.numel() * x.element_size() + 255) // 256 * 256
+    buf = torch.empty(max(total, 256), dtype=torch.uint8, device=device)
+    views = []
+    for x, o in zip(tensors, offs):
+        v = buf[o:o + x.numel() * x.element_size()].view(x.dtype).view(x.shape)
+        v.copy_(x)
+        views.append(v)
+    return buf, views
+
+
 class LsaStep:
     def __init__(self, wl: Workload, t: Tensors, device="cuda", kv_fp8: bool = False):
         """kv_fp8: the K/V caches are FP8 E4M3 codes (drawn here, per layer,
@@ -69,6 +85,25 @@ class LsaStep:
         if self.block_sums is not None:
             lsa.lsa_hi_block_sums(self.t.k_idx, self.wl.hi_block, self.batch, self.block_sums, n_new, self.status,
                                   stream)
+
+    def pack_io(self):
+        """Place the step's per-step inputs (indexer queries and weights, the
+        queries of every layer, the appended tokens' rows) in one contiguous
+        device buffer `in_buf` and its outputs in another, `out_buf`, so that a
+        serving loop moves them with one host-to-device and one device-to-host
+        copy per step. The tensors keep their values and become views of the
+        buffers. Call before capture(): the graphs keep these addresses."""
+        t, G = self.t, self.G
+        ins = [t.q_idx, t.w, *t.q]
+        if self.n_new:
+            ins += [self.k_idx_new, *self.k_new, *self.v_new]
+        self.in_buf, v = _pack(ins, self.device)
+        t.q_idx, t.w, t.q = v[0], v[1], list(v[2:2 + G])
+        if self.n_new:
+            self.k_idx_new = v[2 + G]
+            self.k_new = list(v[3 + G:3 + 2 * G])
+            self.v_new = list(v[3 + 2 * G:3 + 3 * G])
+        self.out_buf, self.out = _pack(self.out, self.device)
 
     def kv_caches(self):
         """The K and V caches the attention reads (FP8 codes or bf16)."""

@@ -328,6 +328,7 @@ def test_graph_replay_matches_eager():
     torch.cuda.synchronize()
     sets0 = parity.host(st.sets).copy()
     outs0 = [parity.host(o).copy() for o in st.out]
+    st.pack_io()  # the graphs then read and write the packed input and output buffers
     st.capture()
     st.sets.fill_(-5)
     for o in st.out:

@@ -91,3 +91,29 @@ def test_kernels_per_step(wl, n):
     # the plan depends on the shape's host fields only; use the real lengths for it
     st.batch.max_len = max(wl.lens)
     assert st.kernels_per_step() == n
+
+
+@pytest.mark.parametrize("kv_fp8", [False, True])
+def test_pack_io_keeps_values_in_one_aligned_buffer(kv_fp8):
+    """pack_io: the per-step inputs and the outputs become 256-byte aligned
+    views of one buffer each, with their values unchanged."""
+    wl = wls.small(wls.BATCH128K, lens=(300, 70), drafts=2, G=2, seed=7)
+    st = _step(wl, kv_fp8=kv_fp8)
+    t = st.t
+    before = [x.clone() for x in [t.q_idx, t.w, *t.q, st.k_idx_new, *st.k_new, *st.v_new]]
+    st.pack_io()
+    after = [t.q_idx, t.w, *t.q, st.k_idx_new, *st.k_new, *st.v_new]
+    lo = st.in_buf.data_ptr()
+    hi = lo + st.in_buf.numel()
+    for b, a in zip(before, after):
+        assert torch.equal(a, b) and a.dtype == b.dtype and a.is_contiguous()
+        assert (a.data_ptr() - lo) % 256 == 0 and lo <= a.data_ptr() and a.data_ptr() + a.numel() * a.element_size() <= hi
+    # the views do not overlap: writing one leaves the others unchanged
+    t.w.fill_(-1)
+    assert torch.equal(t.q_idx, before[0]) and torch.equal(t.q[0], before[2])
+    olo = st.out_buf.data_ptr()
+    assert len(st.out) == 2
+    for o in st.out:
+        assert o.dtype == torch.float32 and o.shape == (wl.n_q, wl.H_q, wl.d)
+        assert (o.data_ptr() - olo) % 256 == 0
+    assert st.out[1].data_ptr() - st.out[0].data_ptr() >= st.out[0].numel() * 4
