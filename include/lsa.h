@@ -227,7 +227,12 @@ int32_t lsa_index_launches(const lsa_batch_t *batch, int32_t H_I, int32_t d_I,
  *              when that size is 0). Not needed after the call returns on the
  *              stream.
  * Supported: d_I in {32, 64, 128}; 1 <= H_I <= LSA_MAX_HEADS_I;
- * budget <= LSA_MAX_BUDGET; hi_topblocks <= LSA_MAX_TOPBLOCKS.
+ * budget <= LSA_MAX_BUDGET; hi_topblocks <= LSA_MAX_TOPBLOCKS. With HI on,
+ * rows that see fewer tokens than their sequence holds (q_len < seq_lens:
+ * prefill chunks, draft rows) need window >= hi_block - 1, because a block's
+ * stored sum covers all of its cached tokens; a batch with more rows than
+ * sequences that breaks this returns LSA_ERR_UNSUPPORTED (other such rows
+ * give an unspecified set).
  */
 lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
                        const int32_t *w, int32_t w_max, int32_t H_I, int32_t d_I,

@@ -233,6 +233,12 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     if (st != LSA_OK) return st;
     if (batch->n_q == 0) return LSA_OK;
     if (budget.hi_block == 0) budget.hi_topblocks = 0;
+    // Block sums cover every cached token of a block. A row that sees fewer
+    // tokens than its sequence holds (a prefill chunk, draft rows) may score a
+    // block that reaches past its last visible token unless the window covers
+    // it (window >= hi_block - 1). More rows than sequences means such rows.
+    if (budget.hi_block > 0 && batch->n_q > batch->n_seq && budget.window < budget.hi_block - 1)
+        return LSA_ERR_UNSUPPORTED;
 
     const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget);
     if (plan.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < plan.ws_bytes || !aligned(workspace, 256)))

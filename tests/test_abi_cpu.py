@@ -73,6 +73,8 @@ def _index(lib, **kw):
     (dict(budget=_budget(hb=512, ht=8), bs=P, rows=10), 2),
     (dict(budget=_budget(hb=64, ht=5000), bs=P, rows=10), 2),
     (dict(batch=_batch(n_seq=0)), 1), (dict(batch=_batch(max_len=0)), 1), (dict(q=P + 4), 1),
+    # HI with causal rows (more rows than sequences) and a window shorter than a block
+    (dict(batch=_batch(n_q=4), budget=_budget(window=8, hb=64, ht=8), bs=P, rows=10), 2),
 ])
 def test_index_rejects_before_launch(kw, want):
     lib = lsa.load_library()
