@@ -586,7 +586,11 @@ def main(argv=None):
         del st, t, run
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
-        line["secondary"] = secondary(dev, flush, stream, min(args.steps, 10), args.warmup, peak)
+        try:
+            line["secondary"] = secondary(dev, flush, stream, min(args.steps, 10), args.warmup, peak)
+        except Exception as exc:  # the headline line still prints; the failure is reported in it
+            print(f"secondary workloads failed: {exc!r}", file=sys.stderr, flush=True)
+            line["secondary"] = {"error": repr(exc)}
     if pg:
         pg.barrier()
         pg.destroy_process_group()
