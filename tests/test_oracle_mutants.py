@@ -37,6 +37,10 @@ MUTANTS = [
      "            const uint16_t *vrow = kseq + ((int64_t)set[j] * H_kv + kvh) * d;"),
     ("batch driver ignores the sequence offset", "        const int8_t *kseq = j->k_idx + j->kv_offset[j->q_seq[r]] * j->d_I;",
      "        const int8_t *kseq = j->k_idx;"),
+    ("batch driver gives every row the first row's weights", "        int n = oracle_index_query(j->q_idx + r * j->H_I * j->d_I, j->w + r * j->H_I,",
+     "        int n = oracle_index_query(j->q_idx + r * j->H_I * j->d_I, j->w,"),
+    ("batch driver sees one token fewer", "                                   kseq, j->q_len[r], j->H_I, j->d_I, j->sink,",
+     "                                   kseq, j->q_len[r] - 1, j->H_I, j->d_I, j->sink,"),
     ("E4M3 exponent bias 8", "        v = ldexp(1.0 + (double)m / 8.0, E - 7);", "        v = ldexp(1.0 + (double)m / 8.0, E - 8);"),
     ("E4M3 subnormals read as normals", "        v = ldexp((double)m / 8.0, -6);", "        v = ldexp(1.0 + (double)m / 8.0, -6);"),
     ("E4M3 sign dropped", "    return sign ? -v : v;", "    return v;"),
