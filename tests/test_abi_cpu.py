@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from long_context_sparse_lsa_b200 import binding as lsa
 
@@ -179,3 +180,27 @@ def test_launch_counts_follow_the_shape():
     assert lsa.lsa_attend_launches(batch(16, 131072), 32, 4, 128, 3136, 1) == 2
     assert lsa.lsa_attend_launches(batch(1, 300000, n_q=8192), 32, 4, 128, 3136, 1) == 1
     assert lsa.lsa_attend_launches(batch(16, 131072), 32, 4, 96, 3136, 1) == 0  # d != 128: unsupported
+
+
+def test_binding_checks_batch_dtypes_before_any_call():
+    """The binding refuses tensors of the wrong dtype or layout rather than
+    passing a misread pointer across the ABI."""
+    n = 3
+    ok = dict(kv_offset=torch.zeros(n, dtype=torch.int64), seq_lens=torch.ones(n, dtype=torch.int32),
+              q_seq=torch.arange(n, dtype=torch.int32), q_len=torch.ones(n, dtype=torch.int32))
+    lsa.Batch(**ok, max_len=1, total_tokens=n).c()
+    for name, bad in (("kv_offset", torch.zeros(n, dtype=torch.int32)), ("seq_lens", torch.ones(n)),
+                      ("q_len", torch.ones(2 * n, dtype=torch.int32)[::2])):
+        with pytest.raises(TypeError):
+            lsa.Batch(**{**ok, name: bad}, max_len=1, total_tokens=n).c()
+    with pytest.raises(TypeError):
+        lsa.Batch(**ok, max_len=1, total_tokens=n, blk_offset=torch.zeros(n, dtype=torch.int32)).c()
+
+
+def test_noalloc_refuses_shapes_beyond_its_scratch_before_launch():
+    lib = lsa.load_library()
+    b = _batch(n_q=4096, max_len=131072, total=4096 * 131072)
+    arr = (ctypes.c_void_p * 1)(P)
+    need = lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 8192, 1)
+    assert need > 8 << 20
+    assert lib.lsa_attend_noalloc(arr, arr, arr, 32, 4, 128, P, 8192, ctypes.byref(b), 1, arr, None, None) == 2
