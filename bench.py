@@ -94,6 +94,22 @@ def _rows(wl):
     return [L - wl.drafts + 1 + j for L in wl.lens for j in range(wl.drafts)]
 
 
+def attend_flops(wl) -> int:
+    """Multiply-adds x 2 of the attention: q.k and p.v over every selected
+    entry, every query head and layer (4 * d flop per head and entry)."""
+    tot = 0
+    for L in _rows(wl):
+        tot += min(L, wl.budget)
+    return 4 * wl.d * wl.H_q * wl.G * tot
+
+
+def prefill_unique_kv_bytes(wl) -> int:
+    """Bytes of the distinct K and V rows a prefill chunk's sets can name: at
+    most the whole cache the chunk sees (every token once per layer)."""
+    kv_row = wl.H_kv * wl.d * 2
+    return 2 * wl.G * wl.lens[0] * kv_row
+
+
 def index_int8_ops(wl) -> int:
     """Multiply-adds x 2 of the fine scores (every middle token of every row)."""
     tot = 0
@@ -114,16 +130,41 @@ def _peaks():
     return 6650.0, "fallback"
 
 
-def _int8_peak():
-    """Dense int8 tensor peak in TOP/s: the measured bf16 GEMM rate x 2 (the
-    nominal int8/bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
+def _bf16_sustained():
+    """Dense bf16 tensor rate in TFLOP/s for kernels timed inside a long step:
+    the measured sustained cuBLAS rate, else the profiling fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        if "bf16_tflops" in d:
-            return 2.0 * float(d["bf16_tflops"]), "measured bf16 x 2 (nominal int8/bf16 ratio)"
-    return 2.0 * 1590.0, "fallback bf16 x 2 (nominal int8/bf16 ratio)"
+        if "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured (sustained cuBLAS bf16)"
+    return 1400.0, "fallback (sustained bf16)"
+
+
+def measure_int8_peak(dev, n: int = 8192, reps: int = 20) -> dict:
+    """Dense int8 tensor rate of this GPU, measured: a library int8 GEMM
+    (torch._int_mm, n x n x n, int32 accumulate) run back to back; best of
+    three bursts of `reps` (CUDA events). Only a denominator: the indexer
+    itself never calls it."""
+    a = torch.randint(-16, 16, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-16, 16, (n, n), dtype=torch.int8, device=dev)
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        best = ms if best is None else min(best, ms)
+    del a, b
+    return {"tops": 2.0 * n ** 3 / (best / 1000.0) / 1e12, "kind": f"measured: torch._int_mm {n}^3 int8 GEMM, best "
+            f"of 3 bursts of {reps}", "ms": best}
 
 
 def _kernel_hash() -> str:
@@ -258,27 +299,129 @@ def cpu_baseline(wl, t, max_seconds=20.0, max_queries=None, min_seconds=0.0):
                       f"oracle time"}
 
 
+def host_cpu() -> dict:
+    """The host's CPU model, its logical CPU count and the CPUs this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count() or 1
+    return {"cpu_model": model, "nproc": os.cpu_count(), "usable_cpus": usable}
+
+
+class OracleStep:
+    """One step of the workload evaluated by the oracle on host threads: the
+    index sets of every query row (oracle lsa_index), then the G-layer
+    attention of every row (oracle lsa_attend). The K/V rows each set names are
+    gathered once, outside the timed calls, into a packed per-row copy (the
+    oracle reads exactly those rows); only the two oracle calls are timed."""
+
+    def __init__(self, wl, t, n_threads: int):
+        import numpy as np
+
+        import oracle
+
+        self.np = np
+        self.orc = oracle.get()
+        self.wl = wl
+        self.n_threads = n_threads
+        h = lambda x: x.contiguous().cpu().numpy()
+        self.q_idx, self.k_idx, self.w = h(t.q_idx), h(t.k_idx), h(t.w)
+        self.kv_offset, self.q_seq, self.q_len = h(t.kv_offset), h(t.q_seq), h(t.q_len)
+        u16 = lambda x: x.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        self.q = [u16(x) for x in t.q]
+        sets = self.index()
+        n_q, budget = sets.shape
+        rows = np.zeros((n_q, budget), np.int64)
+        self.local = np.full((n_q, budget), -1, np.int32)
+        for r in range(n_q):
+            v = sets[r][sets[r] >= 0].astype(np.int64)
+            rows[r, : v.shape[0]] = v + self.kv_offset[self.q_seq[r]]
+            self.local[r, : v.shape[0]] = np.arange(v.shape[0], dtype=np.int32)
+        idx = torch.as_tensor(rows.reshape(-1), device=t.k[0].device)
+        self.k = [u16(x.index_select(0, idx)) for x in t.k]
+        self.v = [u16(x.index_select(0, idx)) for x in t.v]
+        self.offs = np.arange(n_q, dtype=np.int64) * budget
+        self.rows = np.arange(n_q, dtype=np.int32)
+
+    def index(self):
+        wl = self.wl
+        return self.orc.lsa_index(self.q_idx, self.k_idx, self.w, self.kv_offset, self.q_seq, self.q_len, wl.sink,
+                                  wl.window, wl.topk, wl.hi_block, wl.hi_topblocks, n_threads=self.n_threads)
+
+    def run(self) -> float:
+        """Seconds of one step (index + attention of every row)."""
+        c0 = time.perf_counter()
+        self.index()
+        self.orc.lsa_attend(self.q, self.k, self.v, self.local, self.offs, self.rows, n_threads=self.n_threads)
+        return time.perf_counter() - c0
+
+
+def cpu_baseline_all_cores(wl, t, max_seconds=10.0):
+    """The oracle on every usable host CPU (one thread per CPU, the queries of
+    a step spread over them), whole steps repeated until `max_seconds` of
+    oracle time."""
+    cpu = host_cpu()
+    n = max(1, cpu["usable_cpus"])
+    step = OracleStep(wl, t, n)
+    busy, steps = 0.0, 0
+    while busy < max_seconds or steps == 0:
+        busy += step.run()
+        steps += 1
+    return {"value": steps * wl.n_q / busy, "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": f"{steps} whole steps of {wl.name} ({wl.n_q} query rows each: index + {len(t.q)}-layer "
+                      f"attention), C oracle on {n} threads, {busy:.1f} s of oracle time",
+            **cpu}
+
+
+def reference_sample(wl):
+    """The reference arm's bounded sample: a step's worth of query rows on the
+    workload's first sequence (decode: n_q draft-layout rows seeing the last
+    n_q positions of that sequence; prefill: the chunk's first 16 rows), drawn
+    on the host."""
+    if wl.prefill_new:
+        n = min(wl.prefill_new, 16)
+        C = wl.lens[0] - wl.prefill_new
+        return wls.small(wl, lens=(C + n,), prefill_new=n)
+    return wls.small(wl, lens=wl.lens[:1], drafts=wl.n_q)
+
+
 def run_reference(args, wl):
-    """--impl reference: the CPU oracle as it stands, on a bounded sample
-    (the first sequence of the workload, drawn on the host)."""
+    """--impl reference: the CPU oracle as it stands, on the host cores. A step
+    evaluates the sample's query rows once (index + attention, every usable
+    CPU); ms_per_step is the measured time of one such step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sample = wls.small(wl, lens=wl.lens[:1], prefill_new=min(wl.prefill_new, 4) if wl.prefill_new else 0)
+    sample = reference_sample(wl)
     t = wls.make(sample, "cpu")
-    per_step = []
+    cpu = host_cpu()
+    n_threads = max(1, cpu["usable_cpus"])
+    step = OracleStep(sample, t, n_threads)
     for _ in range(args.warmup):
-        cpu_baseline(sample, t, max_seconds=args.ref_seconds)
-    for _ in range(args.steps):
-        per_step.append(cpu_baseline(sample, t, max_seconds=args.ref_seconds))
-    value = statistics.median(p["value"] for p in per_step)
+        step.run()
+    times = [step.run() for _ in range(args.steps)]
+    ms = 1000.0 * statistics.median(times)
+    value = sample.n_q / (ms / 1000.0)
+    desc = (f"{sample.n_q} query rows per step on the first sequence of {wl.name} "
+            f"(context {min(sample.lens[0], max(_rows(sample)))}), index + {sample.G}-layer attention, "
+            f"C oracle on {n_threads} threads; {args.steps} timed steps of {ms:.1f} ms (median)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.n_q / value,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
             "data": "synthetic (seeded SplitMix64 draws)",
-            "config": {"workload": wl.name, "n_queries": wl.n_q, "context": max(wl.lens), "layers_per_index": wl.G},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": per_step[-1]["sample"]},
+            "config": {"workload": wl.name, "n_queries": wl.n_q, "context": max(wl.lens), "layers_per_index": wl.G,
+                       "queries_per_step": sample.n_q},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_threads, "kind": "oracle", "sample": desc,
+                             **cpu},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -422,7 +565,11 @@ def secondary(dev, flush, stream, steps, warmup, peak):
 
     out = {}
     mean = lambda xs: sum(xs) / len(xs)
-    for wl, fp8 in ((wls.CTX1M, False), (wls.PREFILL, False), (wls.BATCH128K, True)):
+    try:
+        int8 = measure_int8_peak(dev)
+    except Exception as exc:  # reported, never silently replaced by an assumed figure
+        int8 = {"tops": None, "kind": f"int8 GEMM unavailable: {exc!r}"}
+    for wl, fp8 in ((wls.CTX1M, False), (wls.PREFILL, False), (wls.BATCH128K, True), (wls.ragged(), False)):
         run = time_workload(wl, dev, flush, stream, steps, warmup, kv_fp8=fp8)
         st = run["st"]
         ms = run["ms"]
@@ -434,32 +581,49 @@ def secondary(dev, flush, stream, steps, warmup, peak):
                "call_ms_in_step": {"index": ix, "attend": at},
                "cold": cold_line(wl, run["cold"], 1, None, dev),
                "algorithmic_bytes_per_step": byts,
-               "step_gbs": byts["total"] / (ms / 1000.0) / 1e9,
-               "step_frac_of_measured_hbm": byts["total"] / (ms / 1000.0) / 1e9 / peak,
-               "attend_gbs": byts["attend"] / (at / 1000.0) / 1e9,
-               "attend_frac_of_measured_hbm": byts["attend"] / (at / 1000.0) / 1e9 / peak,
                "gpu_launches_per_step": run["n_kernels"]}
+        if not wl.prefill_new:
+            # decode: every byte counted is read from HBM once (L2 flushed before each step)
+            rec.update({"step_gbs": byts["total"] / (ms / 1000.0) / 1e9,
+                        "step_frac_of_measured_hbm": byts["total"] / (ms / 1000.0) / 1e9 / peak,
+                        "index_gbs": byts["index"] / (ix / 1000.0) / 1e9,
+                        "index_frac_of_measured_hbm": byts["index"] / (ix / 1000.0) / 1e9 / peak,
+                        "attend_gbs": byts["attend"] / (at / 1000.0) / 1e9,
+                        "attend_frac_of_measured_hbm": byts["attend"] / (at / 1000.0) / 1e9 / peak})
         if wl.prefill_new:
             ops = index_int8_ops(wl)
-            p8, kind8 = _int8_peak()
+            fl = attend_flops(wl)
+            bf, bf_kind = _bf16_sustained()
             rec.update({"metric": "prefill tokens/s (index + attention of a causal chunk)", "unit": "tokens/s",
                         "value": wl.n_q / (ms / 1000.0),
                         "index_tensor_path": bool(lsa.lsa_index_uses_tensor_cores(st.batch, wl.H_I, wl.d_I,
                                                                                   st.budget)),
                         "index_int8_ops": ops,
                         "index_tops": ops / (ix / 1000.0) / 1e12,
-                        "index_tops_frac_of_int8_peak": ops / (ix / 1000.0) / 1e12 / p8,
-                        "int8_peak_tops": p8, "int8_peak_kind": kind8,
+                        "int8_peak_tops": int8["tops"], "int8_peak_kind": int8["kind"],
+                        "index_tops_frac_of_int8_peak": (ops / (ix / 1000.0) / 1e12 / int8["tops"]
+                                                         if int8["tops"] else None),
+                        "attend_flops": fl, "attend_tflops": fl / (at / 1000.0) / 1e12,
+                        "attend_frac_of_bf16": fl / (at / 1000.0) / 1e12 / bf, "bf16_peak_tflops": bf,
+                        "bf16_peak_kind": bf_kind,
+                        "attend_gather_gbs": byts["attend"] / (at / 1000.0) / 1e9,
+                        "attend_unique_kv_bytes": prefill_unique_kv_bytes(wl),
                         "note": "index_tops: int8 ops of the fine-score contraction over the whole index call "
-                                "(scoring + selection), so a lower bound on the tensor kernel's rate"})
+                                "(scoring + selection), so a lower bound on the tensor kernel's rate; "
+                                "attend_gather_gbs counts every row's gathered K/V rows (rows repeat across the "
+                                "chunk and come from L2), so it is a gather rate, not an HBM fraction"})
         elif fp8:
             rec.update({"metric": "LSA decode queries/s at 128K ctx, FP8 E4M3 KV cache", "unit": "queries/s",
                         "value": wl.n_q / (ms / 1000.0), "kv_cache": "fp8 e4m3, one scale per layer for K and V",
                         "note": "same workload as the headline with the K/V caches held as FP8 codes "
                                 "(lsa_attend_fp8); attention bytes per query halve"})
-        else:
+        elif wl.name == wls.CTX1M.name:
             rec.update({"metric": "LSA decode queries/s at 1M ctx", "unit": "queries/s",
                         "value": wl.n_q / (ms / 1000.0), "layers_per_index": wl.G})
+        else:
+            rec.update({"metric": "LSA decode queries/s, ragged batch", "unit": "queries/s",
+                        "value": wl.n_q / (ms / 1000.0), "layers_per_index": wl.G, "n_seq": wl.n_seq,
+                        "cached_tokens": wl.total_tokens, "min_len": min(wl.lens), "max_len": max(wl.lens)})
         out[wl.name + ("_fp8kv" if fp8 else "")] = rec
         del run, st
         torch.cuda.synchronize()
@@ -580,8 +744,12 @@ def main(argv=None):
             "gpu_launches": n_kernels * args.steps,
             "clocks": clk}
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, t, max_seconds=args.cpu_seconds,
-                                            min_seconds=min(10.0, args.cpu_seconds))
+        # the oracle on every usable host CPU (the baseline), and on one
+        # thread over a bounded sample of the same queries (for reference)
+        line["cpu_baseline"] = cpu_baseline_all_cores(wl, t, max_seconds=args.cpu_seconds)
+        one = cpu_baseline(wl, t, max_seconds=min(5.0, args.cpu_seconds), min_seconds=min(3.0, args.cpu_seconds))
+        line["cpu_baseline"]["single_thread"] = {"value": one["value"], "unit": UNIT, "cores": 1,
+                                                 "sample": one["sample"]}
     if world == 1 and not args.no_secondary:
         del st, t, run
         torch.cuda.synchronize()

@@ -51,9 +51,9 @@ def _check(wl, st, t, rows):
         parity.check_attention(parity.host(st.out[g])[rows], ref[g], f"{wl.name} layer {g}")
 
 
-def _release(*objs):
-    for o in objs:
-        del o
+def _free():
+    """Return the cached device memory once the caller has dropped its last
+    references to a workload's buffers (``del st, t`` first)."""
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
 
@@ -62,7 +62,8 @@ def test_batched_decode_128k_every_row():
     wl = wls.BATCH128K
     st, t = _run_graph(wl)
     _check(wl, st, t, np.arange(wl.n_q))
-    _release(st, t)
+    del st, t
+    _free()
 
 
 def test_1m_cross_layer_decode_every_layer():
@@ -70,7 +71,8 @@ def test_1m_cross_layer_decode_every_layer():
     st, t = _run_graph(wl)
     assert len(t.q) == 4
     _check(wl, st, t, np.arange(wl.n_q))
-    _release(st, t)
+    del st, t
+    _free()
 
 
 def test_ragged_batch_sample():
@@ -81,7 +83,8 @@ def test_ragged_batch_sample():
     rows |= {int(lens.argmax()), int(lens.argmin())}
     st, t = _run_graph(wl)
     _check(wl, st, t, sorted(rows))
-    _release(st, t)
+    del st, t
+    _free()
 
 
 def test_fp8_kv_decode_128k_sample():
@@ -104,7 +107,8 @@ def test_fp8_kv_decode_128k_sample():
     sample = np.array([0, 5, 11, 15])
     ref = parity.oracle_attend_rows_fp8(st, want[sample], sample)
     parity.check_attention(parity.host(st.out[0])[sample], ref[0], "fp8 128k")
-    _release(st, t)
+    del st, t
+    _free()
 
 
 def test_prefill_chunk_sample():
@@ -114,4 +118,5 @@ def test_prefill_chunk_sample():
     n = wl.n_q
     rows = [0, 1, 2047, 4096, 6000, n - 2, n - 1]
     _check(wl, st, t, rows)
-    _release(st, t)
+    del st, t
+    _free()
