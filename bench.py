@@ -729,7 +729,7 @@ def main(argv=None):
                                                             "hi_topblocks": wl.hi_topblocks},
                        "heads": {"H_I": wl.H_I, "d_I": wl.d_I, "H_q": wl.H_q, "H_kv": wl.H_kv, "d": wl.d},
                        "l2": "flushed before every timed step (2 x L2 write, outside the timed interval)",
-                       "launch": "each step replayed from one CUDA graph captured through the C ABI (the decode append -- new tokens' keys and K/V rows written, their block sums refreshed -- on a forked stream beside the index call); step_breakdown_ms from per-call graphs replayed in sequence (each with its own graph launch); call_ms_in_step from timing events inside the step graph",
+                       "launch": "each step replayed from one CUDA graph captured through the C ABI: the decode append (new tokens' keys and K/V rows written, their block sums refreshed), the index call and the attention call on one stream, every kernel launched with programmatic stream serialisation; step_breakdown_ms from per-call graphs replayed in sequence (each with its own graph launch); call_ms_in_step from timing events inside the step graph",
                        "parallelism": f"replicas x{world} (independent batches, no collective)"},
             "step_breakdown_ms": {"append": bsu, "index": ix, "attend": at},
             "call_ms_in_step": {"index": ix_in, "attend": at_in},

@@ -49,6 +49,13 @@
  *    are bounded by a time limit after which the kernel sets LSA_DEV_TIMEOUT
  *    and returns, so no call can hang; no kernel traps.
  *  - Calls are thread-safe when they use distinct workspaces.
+ *  - Kernels are launched with programmatic stream serialisation: a kernel
+ *    may start before the preceding kernel on the stream has finished when
+ *    that kernel allows it (griddepcontrol.launch_dependents), and it reads
+ *    the batch's row metadata (q_seq, q_len, kv_offset, seq_lens, blk_offset)
+ *    before waiting for it; everything else is read after the wait. A caller
+ *    whose own kernels trigger dependent launches must write those arrays
+ *    before triggering.
  */
 #ifndef LSA_H_
 #define LSA_H_
@@ -74,6 +81,9 @@ typedef enum {
 #define LSA_DEV_BAD_INDEX 0x4  /* an index-set entry < -1 or >= q_len (entry skipped) */
 #define LSA_DEV_BAD_WEIGHT 0x8 /* an indexer head weight outside [0, w_max] (treated as 0) */
 #define LSA_DEV_TIMEOUT 0x10   /* a bounded wait inside a kernel gave up (output unspecified) */
+#define LSA_DEV_BAD_QUERY 0x20 /* lsa_attend_fp8: a query element outside the fp16 range
+                                  (|q| >= 65536 as bf16, or not finite); the row's output is
+                                  unspecified */
 
 /* Selection budget. sink + window + topk is the index-set length ("budget").
  * hi_block == 0 switches HI off; otherwise blocks of hi_block tokens aligned
@@ -213,6 +223,22 @@ int32_t lsa_index_launches(const lsa_batch_t *batch, int32_t H_I, int32_t d_I,
 /* One index set per query row (CLI: call once per group of layers and pass
  * the result to lsa_attend with layers_per_index = G).
  *
+ * What the set is: LSA keeps DeepSeek Sparse Attention's indexer (every
+ * candidate cached token is scored, a top-k is kept) and adds three
+ * mechanisms ("LongCat-2.0 (molayo1419.me)", section "1M 토큰에서의 Sparse
+ * Attention 문제"). This call evaluates them as follows:
+ *  - SI ("LongCat-Flash-Lite-Sparse (aitrends.kr)", section "기술적 특징",
+ *    first bullet): the budget has a fixed sink run [0, s) and a local
+ *    window run [ws, L) that are always kept; the top-k competes only over
+ *    the middle [s, ws).
+ *  - HI (same section, third bullet): with hi_block > 0 the middle's blocks
+ *    are scored coarsely on their key sums, the hi_topblocks best are kept,
+ *    and the fine top-k runs only over the middle tokens inside them.
+ *  - CLI (same section, second bullet): one set serves G adjacent layers;
+ *    lsa_index runs once per group.
+ * The fine score, the coarse score and the tie rule are the ones fixed at
+ * the top of this file.
+ *
  * q_idx        device int8 [n_q][H_I][d_I] indexer queries.
  * k_idx_cache  device int8 [total_tokens][d_I] indexer keys (one per token,
  *              shared by all indexer heads).
@@ -227,12 +253,12 @@ int32_t lsa_index_launches(const lsa_batch_t *batch, int32_t H_I, int32_t d_I,
  *              when that size is 0). Not needed after the call returns on the
  *              stream.
  * Supported: d_I in {32, 64, 128}; 1 <= H_I <= LSA_MAX_HEADS_I;
- * budget <= LSA_MAX_BUDGET; hi_topblocks <= LSA_MAX_TOPBLOCKS. With HI on,
- * rows that see fewer tokens than their sequence holds (q_len < seq_lens:
- * prefill chunks, draft rows) need window >= hi_block - 1, because a block's
- * stored sum covers all of its cached tokens; a batch with more rows than
- * sequences that breaks this returns LSA_ERR_UNSUPPORTED (other such rows
- * give an unspecified set).
+ * budget <= LSA_MAX_BUDGET; hi_topblocks <= LSA_MAX_TOPBLOCKS. With HI on, a
+ * row's blocks are summed over the tokens the row sees: a row that sees
+ * fewer tokens than its sequence holds (q_len < seq_lens: prefill chunks,
+ * draft rows) has the block holding its last visible token, when that block
+ * is a candidate, re-summed from the keys instead of read from block_sums
+ * (whose row covers every cached token of the block).
  */
 lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
                        const int32_t *w, int32_t w_max, int32_t H_I, int32_t d_I,
@@ -262,6 +288,15 @@ int32_t lsa_attend_launches(const lsa_batch_t *batch, int32_t H_q,
  * index_sets[r] that are not -1, for every layer g < layers_per_index
  * (Cross-Layer Indexing: all G layers share one set).
  *
+ * This is the attention that follows LSA's token selection: softmax
+ * attention restricted to the selected KV rows ("LongCat-2.0 (molayo1419.me)",
+ * section "1M 토큰에서의 Sparse Attention 문제"). Its reads are the ones SI
+ * makes contiguous: the sink and window runs of every set are sequential KV
+ * reads ("LongCat-Flash-Lite-Sparse (aitrends.kr)", section "기술적 특징",
+ * first bullet), and CLI lets one set drive the G layers of a group (same
+ * section, second bullet). Scale 1/sqrt(d), GQA groups as fixed at the top
+ * of this file.
+ *
  * q            host [G] array of device bf16 [n_q][H_q][d] (bit patterns).
  * k_cache      host [G] array of device bf16 [total_tokens][H_kv][d].
  * v_cache      host [G] array of device bf16 [total_tokens][H_kv][d].
@@ -289,6 +324,11 @@ lsa_status_t lsa_attend(const uint16_t *const *q, const uint16_t *const *k_cache
  * GQA mapping, the output, the workspace (lsa_attend_workspace_size) and the
  * device-side errors — is lsa_attend's.
  *
+ * q                 as for lsa_attend. The products run on fp16 tensor cores:
+ *                   every E4M3 value is an fp16, and so is every bf16 query
+ *                   element of magnitude below 65536 (elements below 2^-14 keep
+ *                   fp16's subnormal precision). A query element of magnitude
+ *                   65536 or more, or not finite, sets LSA_DEV_BAD_QUERY.
  * k_cache, v_cache  host [G] arrays of device uint8 [total_tokens][H_kv][d]
  *                   E4M3 codes (NaN codes give unspecified output).
  * k_scale, v_scale  host [G] arrays of finite floats.
@@ -322,6 +362,10 @@ lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_ca
  *    LSA_NOALLOC_SCRATCH_BYTES returns LSA_ERR_UNSUPPORTED before any launch.
  *  - The first call on each device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
+ *    The address is kept per device ordinal for the life of the process: it
+ *    belongs to the device's primary context (the one the CUDA runtime uses),
+ *    so do not call this after cudaDeviceReset() or from a context of your
+ *    own made current with the driver API.
  *  - All calls on a device share the one array, which keeps the previous
  *    call's contents; nothing in it needs to start at zero, because every
  *    call writes the scratch it later reads. Calls that overlap on the GPU

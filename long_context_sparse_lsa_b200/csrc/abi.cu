@@ -171,13 +171,7 @@ lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_
 }
 
 // ---------------------------------------------------------------------------
-size_t lsa_index_workspace_size(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, lsa_budget_t budget) {
-    (void)H_I;
-    (void)d_I;
-    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1 || !budget_ok(budget)) return 0;
-    if (budget.hi_block == 0) budget.hi_topblocks = 0;
-    return lsa::plan_index(batch->n_q, batch->max_len, budget).ws_bytes;
-}
+}  // extern "C"
 
 // Rows from which a chunk of one sequence is scored as a dense contraction.
 constexpr int32_t kDenseMinRows = 64;
@@ -185,6 +179,14 @@ constexpr int32_t kDenseMinRows = 64;
 static bool index_dense(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, const lsa_budget_t& budget) {
     return budget.hi_block == 0 && batch->n_q >= kDenseMinRows &&
            lsa::prefill_tc_supported(H_I, d_I, batch->n_seq, batch->total_tokens);
+}
+
+extern "C" {
+
+size_t lsa_index_workspace_size(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, lsa_budget_t budget) {
+    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1 || !budget_ok(budget)) return 0;
+    if (budget.hi_block == 0) budget.hi_topblocks = 0;
+    return lsa::plan_index(batch->n_q, batch->max_len, budget, index_dense(batch, H_I, d_I, budget)).ws_bytes;
 }
 
 int32_t lsa_index_uses_tensor_cores(const lsa_batch_t* batch, int32_t H_I, int32_t d_I,
@@ -198,7 +200,8 @@ int32_t lsa_index_launches(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, l
     (void)d_I;
     if (budget.hi_block == 0) return 2;  // fine scores, token selection
     const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget);
-    const bool fused = lsa::coarse_in_select(budget.hi_block, plan.coarse_stage, H_I, batch->n_q);
+    const bool fused = plan.tk_kp_blocks == 0 && lsa::coarse_in_select(budget.hi_block, plan.coarse_stage, H_I,
+                                                                        batch->n_q);
     return (fused ? 1 : 2) + 2;  // [coarse scores,] block selection, fine scores, token selection
 }
 
@@ -233,14 +236,9 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     if (st != LSA_OK) return st;
     if (batch->n_q == 0) return LSA_OK;
     if (budget.hi_block == 0) budget.hi_topblocks = 0;
-    // Block sums cover every cached token of a block. A row that sees fewer
-    // tokens than its sequence holds (a prefill chunk, draft rows) may score a
-    // block that reaches past its last visible token unless the window covers
-    // it (window >= hi_block - 1). More rows than sequences means such rows.
-    if (budget.hi_block > 0 && batch->n_q > batch->n_seq && budget.window < budget.hi_block - 1)
-        return LSA_ERR_UNSUPPORTED;
 
-    const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget);
+    const bool dense = index_dense(batch, H_I, d_I, budget);
+    const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget, dense);
     if (plan.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < plan.ws_bytes || !aligned(workspace, 256)))
         return LSA_ERR_WORKSPACE;
     if (batch->n_q > 65535) return LSA_ERR_UNSUPPORTED;
@@ -276,6 +274,9 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     a.kept = reinterpret_cast<int32_t*>(ws + plan.off_kept);
     a.n_kept = reinterpret_cast<int32_t*>(ws + plan.off_nkept);
     a.fine_keys = reinterpret_cast<uint32_t*>(ws + plan.off_fine);
+    a.cand = dense ? reinterpret_cast<uint64_t*>(ws + plan.off_cand) : nullptr;
+    a.cand_seg = dense ? reinterpret_cast<int32_t*>(ws + plan.off_count) : nullptr;
+    a.tc_splits = dense ? lsa::prefill_tc_splits(batch->n_q) : 0;
     a.coarse_cap = plan.coarse_cap;
     a.fine_cap = plan.fine_cap;
     a.coarse_stage = plan.coarse_stage;
@@ -284,16 +285,25 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (budget.hi_block > 0) {
-        if (!lsa::coarse_in_select(a)) e = lsa::launch_index_scores(a, d_I, true, cs);
-        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, d_I, plan.cluster, plan.smem_blocks, cs);
+        if (plan.tk_kp_blocks > 0) {
+            // coarse scores of every candidate block, then one selection CTA per row
+            e = lsa::launch_index_scores(a, d_I, true, cs);
+            if (e == cudaSuccess) e = lsa::launch_topk(a, true, plan.tk_kp_blocks, plan.tk_cl_blocks, cs);
+        } else {
+            if (!lsa::coarse_in_select(a)) e = lsa::launch_index_scores(a, d_I, true, cs);
+            if (e == cudaSuccess) e = lsa::launch_index_select(a, true, d_I, plan.cluster, plan.smem_blocks, cs);
+        }
     }
     if (e == cudaSuccess) {
         // a prefill chunk (many rows of one sequence, HI off) is one dense
         // contraction: tensor-core path; otherwise per-row streaming scores
-        e = index_dense(batch, H_I, d_I, budget) ? lsa::launch_fine_scores_tc(a, cs)
-                                                  : lsa::launch_index_scores(a, d_I, false, cs);
+        e = dense ? lsa::launch_fine_scores_tc(a, cs) : lsa::launch_index_scores(a, d_I, false, cs);
     }
-    if (e == cudaSuccess) e = lsa::launch_index_select(a, false, d_I, plan.cluster, plan.smem_tokens, cs);
+    if (e == cudaSuccess) {
+        if (dense) e = lsa::launch_topk_pairs(a, cs);
+        else if (plan.tk_kp_tokens > 0) e = lsa::launch_topk(a, false, plan.tk_kp_tokens, plan.tk_cl_tokens, cs);
+        else e = lsa::launch_index_select(a, false, d_I, plan.cluster, plan.smem_tokens, cs);
+    }
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 
@@ -357,7 +367,7 @@ static lsa_status_t attend_impl(const uint16_t* const* q, const void* const* k_c
     }
     if ((int64_t)batch->n_q > 65535) return LSA_ERR_UNSUPPORTED;
     lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, budget, layers_per_index,
-                                         lsa::device_sm_count());
+                                         lsa::device_sm_count(), fp8);
     if (workspace == nullptr || workspace_bytes < p.ws_bytes || !aligned(workspace, 256)) return LSA_ERR_WORKSPACE;
     lsa::AttendArgs a;
     std::memset(&a, 0, sizeof a);

@@ -49,6 +49,7 @@ constexpr int kTile = 16;                              // tokens per stage
 constexpr int kD = 128;
 constexpr int kHeadBytes = kD * 2;                     // one (token, kv head) row
 constexpr int kMaxEntriesPerSplit = 4096;
+constexpr int kPrefetch = 4;  // attention: tiles prefetched into L2 beyond the two in registers
 constexpr int kMaxStages = 8;
 constexpr size_t kAtSmemBudget = 200 * 1024;
 
@@ -493,6 +494,12 @@ __device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 c) {
                       e4m3x2_to_f16x2(c.y >> 16));
 }
 
+// True when either bf16 of the pair has magnitude >= 65536 (0x4780: above
+// fp16's largest finite value 65504) or is not finite.
+__device__ __forceinline__ bool bf16x2_beyond_f16(uint32_t x) {
+    return (x & 0x7fffu) >= 0x4780u || ((x >> 16) & 0x7fffu) >= 0x4780u;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
     const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
     return pack_f16(f.x, f.y);
@@ -560,7 +567,6 @@ __device__ __forceinline__ VTile frag16(const VTile8& v) {
 template <bool FP8>
 __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const __grid_constant__ AttendArgs a) {
     constexpr int NT = 1;
-    pdl_enter();
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
     const int g = lane >> 2, t4 = lane & 3;
@@ -575,11 +581,14 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
     // The set entries and the row's sequence metadata are fetched together
     // (the entries are checked against q_len once it is known); nothing is
     // written before the row check.
+    // (the row's metadata is the caller's, never written by a kernel of this
+    // library: it is read before the wait for the preceding kernel)
     const int seq = a.q_seq[r];
     const int L = a.q_len[r];
     const int seq_c = min(max(seq, 0), a.n_seq - 1);
     const int64_t off = a.kv_offset[seq_c];
     const int slen = a.seq_lens[seq_c];
+    pdl_enter();
     const int e0 = split * a.entries_per_split;
     const int32_t* set = a.sets + (int64_t)r * a.budget + e0;
     const int n_cap = max(0, min(a.budget - e0, a.entries_per_split));  // entries this split may own
@@ -642,16 +651,19 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
     {
         const uint16_t* qrow = a.q[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
         const bool ok = g < ratio;
+        bool qbad = false;  // FP8: a query element fp16 cannot hold
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
             const uint16_t* p = qrow + g * kD + 8 * (t4 + 4 * (ks >> 1)) + 4 * (ks & 1);
             qb[ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p)) : 0u;
             qb[ks][1] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p + 2)) : 0u;
             if constexpr (FP8) {
+                qbad |= bf16x2_beyond_f16(qb[ks][0]) | bf16x2_beyond_f16(qb[ks][1]);
                 qb[ks][0] = bf16x2_to_f16x2(qb[ks][0]);
                 qb[ks][1] = bf16x2_to_f16x2(qb[ks][1]);
             }
         }
+        if (FP8 && __any_sync(0xffffffffu, qbad) && lane == 0) flag(a.dev_status, LSA_DEV_BAD_QUERY);
     }
     const float sl2 = FP8 ? a.scale_log2 * a.kscale[layer] : a.scale_log2;
     KT ka, kb2;
@@ -664,7 +676,25 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
         load_k(kb2, s_ent + (wsel + n_sel) * kTile);
         load_v(vb2, s_ent + (wsel + n_sel) * kTile);
     }
+    // L2 prefetch of the K and V rows of this warp's tile kPrefetch steps
+    // beyond the register loads: those loads then find their rows in L2, so
+    // the two tiles of registers in flight cover an L2 latency, not DRAM's.
+    // Lane l covers token l % 16: its K and V rows (one 128-byte line per
+    // FP8 row, two per bf16 row; lanes 16..31 take the second line).
+    auto prefetch = [&](int i) {
+        if (i >= n_tiles) return;
+        const int e = s_ent[i * kTile + (lane & 15)];
+        if (e < 0) return;
+        const int line = FP8 ? 0 : (lane >> 4);
+        if (FP8 && lane >= 16) return;
+        const uint8_t* pk = kbase + (int64_t)e * tok_stride * kEB + 128 * line;
+        const uint8_t* pv = vbase + (int64_t)e * tok_stride * kEB + 128 * line;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pk));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pv));
+    };
+    for (int p = 2; p < 2 + kPrefetch; ++p) prefetch(wsel + p * n_sel);
     auto tile = [&](int i, KT& k, VT& v) {
+        prefetch(i + (2 + kPrefetch) * n_sel);
         const int ent_lane = lane < kTile ? s_ent[i * kTile + lane] : 0;
         const uint32_t masked = __ballot_sync(0xffffffffu, lane < kTile && ent_lane < 0);
         const bool ok_g = !((masked >> g) & 1u);
@@ -701,11 +731,19 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
                         FP8 ? a.vscale[layer] : 1.f);
 }
 
-// Split merge: one warp per (query head, row, layer); lane l owns dims
-// 4l..4l+3. All partials are combined with the log-sum-exp rule.
-__global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_constant__ AttendArgs a) {
+// Split merge: one CTA per (query head, row, layer) with one warp per
+// kMergeSplitsPerWarp splits, so every partial is loaded in one round of
+// loads; lane l owns dims 4l..4l+3. Each warp folds its splits with the
+// log-sum-exp rule, and warp 0 folds the warps' results from shared memory.
+constexpr int kMergeSplitsPerWarp = 8;
+constexpr int kMergeMaxWarps = 16;
+
+__global__ void __launch_bounds__(kMergeMaxWarps * kWarp) attend_merge_kernel(const __grid_constant__ AttendArgs a) {
     pdl_enter();
-    const int h = blockIdx.x, r = blockIdx.y, layer = blockIdx.z, lane = threadIdx.x;
+    __shared__ float s_m[kMergeMaxWarps], s_den[kMergeMaxWarps];
+    __shared__ float4 s_acc[kMergeMaxWarps][kWarp];
+    const int h = blockIdx.x, r = blockIdx.y, layer = blockIdx.z, lane = lane_id(), w = warp_id();
+    const int nw = (int)(blockDim.x / kWarp);
     // the row check's loads overlap the partials' loads; the output is only
     // written for a valid row (an invalid row's output was zeroed already)
     const int seq = a.q_seq[r];
@@ -717,22 +755,23 @@ __global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_consta
     const float* P = a.part_o + (row_q * a.n_splits * a.H_q + h) * kD;
     const float* PML = a.part_ml + (row_q * a.n_splits * a.H_q + h) * 2;
     const int64_t pstride = (int64_t)a.H_q;  // between consecutive splits, in rows
-    constexpr int kU = 16;  // up to 16 splits in one round of loads
+    const int per = (a.n_splits + nw - 1) / nw;
+    const int p_lo = w * per, p_hi = min(a.n_splits, p_lo + per);
     float M = -INFINITY, den = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p0 = 0; p0 < a.n_splits; p0 += kU) {
-        float2 ml[kU];
-        float4 v[kU];
+    for (int p0 = p_lo; p0 < p_hi; p0 += kMergeSplitsPerWarp) {
+        float2 ml[kMergeSplitsPerWarp];
+        float4 v[kMergeSplitsPerWarp];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kMergeSplitsPerWarp; ++u) {
             const int p = p0 + u;
-            const bool ok = p < a.n_splits;
+            const bool ok = p < p_hi;
             ml[u] = ok ? __ldcg(reinterpret_cast<const float2*>(PML + p * pstride * 2)) : make_float2(-INFINITY, 0.f);
             v[u] = ok ? __ldcg(reinterpret_cast<const float4*>(P + p * pstride * kD) + lane)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kMergeSplitsPerWarp; ++u) {
             if (ml[u].x == -INFINITY) continue;
             const float nm = fmaxf(M, ml[u].x);
             const float so = exp2f(M - nm), sn = exp2f(ml[u].x - nm);
@@ -741,6 +780,31 @@ __global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_consta
             acc.y = acc.y * so + v[u].y * sn;
             acc.z = acc.z * so + v[u].z * sn;
             acc.w = acc.w * so + v[u].w * sn;
+            M = nm;
+        }
+    }
+    if (nw > 1) {
+        s_acc[w][lane] = acc;
+        if (lane == 0) {
+            s_m[w] = M;
+            s_den[w] = den;
+        }
+        __syncthreads();
+        if (w != 0) return;
+        M = -INFINITY;
+        den = 0.f;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < nw; ++j) {
+            const float mj = s_m[j];
+            if (mj == -INFINITY) continue;
+            const float nm = fmaxf(M, mj);
+            const float so = exp2f(M - nm), sn = exp2f(mj - nm);
+            const float4 aj = s_acc[j][lane];
+            den = den * so + s_den[j] * sn;
+            acc.x = acc.x * so + aj.x * sn;
+            acc.y = acc.y * so + aj.y * sn;
+            acc.z = acc.z * so + aj.z * sn;
+            acc.w = acc.w * so + aj.w * sn;
             M = nm;
         }
     }
@@ -753,7 +817,7 @@ __global__ void __launch_bounds__(kWarp) attend_merge_kernel(const __grid_consta
 
 }  // namespace
 
-AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms) {
+AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms, bool fp8) {
     AttendPlan p;
     (void)d;
     p.hpc = H_kv < 4 ? H_kv : 4;
@@ -775,10 +839,12 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
     if (splits < 1) splits = 1;
     p.n_splits = splits;
     p.entries_per_split = eps;
-    // shared memory: entries | barriers | K stages (the stages are reused for the merge)
+    // shared memory: entries | barriers | stages (the stages are reused for the merge)
     const size_t ent = ((size_t)eps * 4 + 127) / 128 * 128;
+    (void)fp8;
     const size_t stage = (size_t)kTile * p.row_stride;
-    int ns = (int)((kAtSmemBudget - ent - 2 * kMaxStages * 8 - 128) / stage);
+    const size_t bars = ((2 * (size_t)kMaxStages * 8 + 127) / 128) * 128;
+    int ns = (int)((kAtSmemBudget - ent - bars - 128) / stage);
     if (ns > kMaxStages) ns = kMaxStages;
     // tile i uses stage i mod ns and the warps of wsel i mod (8 / hpc): with ns
     // a multiple of that, every use of a stage has the same warps, which saw
@@ -787,7 +853,7 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
     if (ns >= n_sel) ns = ns / n_sel * n_sel;
     p.n_stages = ns;
     p.bar_off = (int)ent;
-    p.stage_off = (int)(ent + ((2 * kMaxStages * 8 + 127) / 128) * 128);
+    p.stage_off = (int)(ent + bars);
     const int NT = (H_q / H_kv + 7) / 8;
     size_t merge = (size_t)kConsumers * (NT * (kD / 16) * 4 + NT * 4) * kWarp * 4;
     size_t stages_bytes = (size_t)ns * stage;
@@ -825,8 +891,10 @@ cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t s
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.n_splits == 1) return e;
-    return launch_pdl(attend_merge_kernel, dim3((unsigned)a.H_q, (unsigned)a.n_q, (unsigned)a.G), dim3(kWarp), 0,
-                      stream, 0, a);
+    int nw = (a.n_splits + kMergeSplitsPerWarp - 1) / kMergeSplitsPerWarp;
+    if (nw > kMergeMaxWarps) nw = kMergeMaxWarps;
+    return launch_pdl(attend_merge_kernel, dim3((unsigned)a.H_q, (unsigned)a.n_q, (unsigned)a.G),
+                      dim3((unsigned)(nw * kWarp)), 0, stream, 0, a);
 }
 
 }  // namespace lsa

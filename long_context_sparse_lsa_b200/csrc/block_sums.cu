@@ -29,7 +29,9 @@ __device__ __forceinline__ int sbyte(uint32_t w, int i) { return static_cast<int
 // cost resident CTAs, and the full build got slower. row_ptr(i) is
 // the address of the block's row i; the sum of rows [0, n) goes to out_row as
 // the two byte planes. Every thread of the CTA calls it (one CTA barrier).
-template <int D_I, typename RowPtr>
+// ROWS: rows each thread loads at once (the decode append, one block per
+// CTA and latency-bound, issues a whole block's loads in one round).
+template <int D_I, int ROWS = 1, typename RowPtr>
 __device__ __forceinline__ void sum_block(RowPtr row_ptr, int n, int8_t* out_row, int (&s_part)[kBsWarps][D_I]) {
     constexpr int kCPR = D_I / 16;           // 16-byte chunks per row
     constexpr int kRPP = kBsThreads / kCPR;  // rows per pass
@@ -38,13 +40,21 @@ __device__ __forceinline__ void sum_block(RowPtr row_ptr, int n, int8_t* out_row
     int acc[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) acc[i] = 0;
-    for (int row = tid / kCPR; row < n; row += kRPP) {
-        const uint4 v = ldg16(row_ptr(row) + c * 16);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int row0 = tid / kCPR; row0 < n; row0 += kRPP * ROWS) {
+        uint4 v[ROWS];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int u = 0; u < ROWS; ++u) {
+            const int row = row0 + u * kRPP;
+            v[u] = row < n ? ldg16(row_ptr(row) + c * 16) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[4 * q + b] += sbyte(w[q], b);
+        for (int u = 0; u < ROWS; ++u) {
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[4 * q + b] += sbyte(w[q], b);
+        }
     }
     // lanes with the same chunk differ in the bits above log2(kCPR)
 #pragma unroll
@@ -114,15 +124,19 @@ __device__ __forceinline__ void copy16(uint8_t* dst, const uint8_t* src, int64_t
 
 constexpr int kAppendRowsPerCta = 64;  // HI off: new tokens per CTA
 
-// Decode append. CTA (x, b) owns the new tokens of sequence b that fall in
-// block first + x (HI on; the CTA also recomputes that block's sum) or the
-// x-th run of kAppendRowsPerCta new tokens (HI off). It copies their indexer
-// keys and every layer's K and V rows into the caches. The block sum reads
-// the new rows from the inputs and the older rows from the cache, so no CTA
-// reads what it (or another CTA) writes in this launch.
+// Decode append. CTA (x, b, 0) owns the new tokens of sequence b that fall in
+// block first + x (HI on) or the x-th run of kAppendRowsPerCta new tokens
+// (HI off) and copies their indexer keys and every layer's K and V rows into
+// the caches; with HI on, CTA (x, b, 1) recomputes that block's sum in the
+// same launch (one round of loads each). The block sum reads the new rows
+// from the inputs and the older rows from the cache, so no CTA reads what it
+// (or another CTA) writes in this launch.
 template <int D_I>
 __global__ void __launch_bounds__(kBsThreads) append_kernel(const AppendArgs p) {
     pdl_enter();
+    // a small grid: the next call's first kernel may be resident beside it
+    // (it still waits for this grid's completion before reading the caches)
+    pdl_trigger();
     __shared__ int s_part[kBsWarps][D_I];
     const BlockSumArgs& a = p.bs;
     const int seq = blockIdx.y;
@@ -149,21 +163,22 @@ __global__ void __launch_bounds__(kBsThreads) append_kernel(const AppendArgs p) 
         hi = min(len, lo + kAppendRowsPerCta);
         if (lo >= hi) return;
     }
-    const int64_t src0 = (int64_t)seq * n_new + (lo - from);  // first input row
-    const int nr = hi - lo;
-    copy16(reinterpret_cast<uint8_t*>(p.k_idx_cache) + (off + lo) * D_I,
-           reinterpret_cast<const uint8_t*>(p.k_idx_new) + src0 * D_I, (int64_t)nr * D_I);
-    const int64_t kvb = p.kv_row_bytes;
-    for (int g = 0; g < p.layers; ++g) {
-        copy16(reinterpret_cast<uint8_t*>(p.k_cache[g]) + (off + lo) * kvb,
-               reinterpret_cast<const uint8_t*>(p.k_new[g]) + src0 * kvb, nr * kvb);
-        copy16(reinterpret_cast<uint8_t*>(p.v_cache[g]) + (off + lo) * kvb,
-               reinterpret_cast<const uint8_t*>(p.v_new[g]) + src0 * kvb, nr * kvb);
-    }
-    if (p.sums) {
+    if (blockIdx.z == 0) {
+        const int64_t src0 = (int64_t)seq * n_new + (lo - from);  // first input row
+        const int nr = hi - lo;
+        copy16(reinterpret_cast<uint8_t*>(p.k_idx_cache) + (off + lo) * D_I,
+               reinterpret_cast<const uint8_t*>(p.k_idx_new) + src0 * D_I, (int64_t)nr * D_I);
+        const int64_t kvb = p.kv_row_bytes;
+        for (int g = 0; g < p.layers; ++g) {
+            copy16(reinterpret_cast<uint8_t*>(p.k_cache[g]) + (off + lo) * kvb,
+                   reinterpret_cast<const uint8_t*>(p.k_new[g]) + src0 * kvb, nr * kvb);
+            copy16(reinterpret_cast<uint8_t*>(p.v_cache[g]) + (off + lo) * kvb,
+                   reinterpret_cast<const uint8_t*>(p.v_new[g]) + src0 * kvb, nr * kvb);
+        }
+    } else if (p.sums) {
         const int8_t* cache = a.k_idx + (off + t0) * D_I;
         const int8_t* fresh = p.k_idx_new + (int64_t)seq * n_new * D_I;
-        sum_block<D_I>(
+        sum_block<D_I, 4>(
             [&](int row) {
                 const int pos = t0 + row;
                 return pos >= from ? fresh + (int64_t)(pos - from) * D_I : cache + (int64_t)row * D_I;
@@ -194,7 +209,7 @@ cudaError_t launch_append(const AppendArgs& a, int d_I, cudaStream_t stream) {
     } else {
         gx = (unsigned)((n_new + kAppendRowsPerCta - 1) / kAppendRowsPerCta);
     }
-    dim3 grid(gx, (unsigned)a.bs.n_seq);
+    dim3 grid(gx, (unsigned)a.bs.n_seq, a.sums ? 2u : 1u);
     switch (d_I) {
         case 32: return launch_pdl(append_kernel<32>, grid, dim3(kBsThreads), 0, stream, 0, a);
         case 64: return launch_pdl(append_kernel<64>, grid, dim3(kBsThreads), 0, stream, 0, a);

@@ -22,8 +22,10 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 // Programmatic dependent launch: every kernel of the path is launched with
 // programmatic stream serialisation and waits for the grids it depends on
-// (and their memory) before its first global access; the next kernel may be
-// launched as this grid's CTAs exit. (Triggering the next launch at kernel
+// (and their memory) before it reads anything a kernel of this library
+// writes; reads of the caller's row metadata (q_seq, q_len, kv_offset,
+// seq_lens, blk_offset), which no kernel here writes, may come first. The
+// next kernel may be launched as this grid's CTAs exit. (Triggering the next launch at kernel
 // entry measured slower: the early dependents took SM space from the running
 // grid.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -92,6 +94,12 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -136,10 +144,34 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Shared-memory histogram add of one value per lane (bin = 0xffffffff: none),
+// aggregated over the lanes that hold the same bin: one atomic per distinct
+// bin of the warp instead of one per lane (many keys fall into a few bins).
+// Every lane of the warp must call it.
+__device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t bin) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+    if (bin != 0xffffffffu && (threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1))
+        atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
+}
+
+// Warp-aggregated append to a shared-memory list: the lanes with `take`
+// reserve consecutive slots with one atomic on *count (by the first such
+// lane) and each gets its slot (in lane order), or 0xffffffff. Every lane of
+// the warp must call it.
+__device__ __forceinline__ uint32_t warp_append(uint32_t* count, bool take) {
+    const uint32_t m = __ballot_sync(0xffffffffu, take);
+    if (m == 0u) return 0xffffffffu;
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0;
+    if ((threadIdx.x & 31) == (uint32_t)leader) base = atomicAdd(count, (uint32_t)__popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    return take ? base + (uint32_t)__popc(m & lanemask_lt()) : 0xffffffffu;
 }
 
 // 16-byte read-only global load.
@@ -225,6 +257,21 @@ __device__ __forceinline__ uint32_t map_cta(uint32_t addr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
+}
+// Remote (distributed shared memory) add, fetch-add and stores.
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t addr, uint32_t v) {
+    uint32_t r;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(r) : "r"(addr), "r"(v) : "memory");
+    return r;
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, uint64_t v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"((unsigned long long)v) : "memory");
 }
 __device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
     float2 v;

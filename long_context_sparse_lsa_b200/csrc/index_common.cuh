@@ -139,5 +139,65 @@ __device__ __forceinline__ void coarse_tile(const QueryFrag<D_I, NT>& qf, const 
     y += __shfl_xor_sync(0xffffffffu, y, 2);
 }
 
+// HI blocks are summed over the tokens a row can see ([b*B, min((b+1)*B, L))).
+// The block-sum cache holds one sum per block over every cached token, so for
+// a row that sees fewer tokens than its sequence holds (L < seq_lens: a
+// prefill chunk, draft rows) the block holding its last visible token L-1 may
+// also count tokens the row cannot see. partial_block_fix() tells whether
+// that block is a candidate of the row and needs its sum recomputed;
+// partial_block_score() recomputes its coarse score from the keys.
+__device__ __forceinline__ bool partial_block_fix(int L, int slen, int B, int ws, int& b_p) {
+    b_p = (L - 1) / B;
+    return L < slen && L % B != 0 && b_p * B < ws;
+}
+
+// The coarse score of the block [t0, t0 + n) of `rows` (the sequence's keys)
+// for query row r, computed by every thread of the CTA (THREADS threads).
+// s_sum: D_I ints of shared scratch. Returns the score in every thread; holds
+// CTA barriers, so every thread must call it.
+template <int D_I, int THREADS>
+__device__ long long partial_block_score(const IndexArgs& a, int r, const int8_t* rows, int t0, int n,
+                                         int32_t* s_sum, long long* s_out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = THREADS / 32;
+    constexpr int kLanes = D_I / 4;  // lanes owning 4 dims each
+    for (int i = tid; i < D_I; i += THREADS) s_sum[i] = 0;
+    __syncthreads();
+    if (lane < kLanes) {
+        int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+        for (int i = warp; i < n; i += kWarps) {
+            const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(rows + (int64_t)(t0 + i) * D_I) + lane);
+            s0 += (int)(int8_t)(w & 0xffu);
+            s1 += (int)(int8_t)((w >> 8) & 0xffu);
+            s2 += (int)(int8_t)((w >> 16) & 0xffu);
+            s3 += (int)(int8_t)(w >> 24);
+        }
+        atomicAdd(&s_sum[4 * lane + 0], s0);
+        atomicAdd(&s_sum[4 * lane + 1], s1);
+        atomicAdd(&s_sum[4 * lane + 2], s2);
+        atomicAdd(&s_sum[4 * lane + 3], s3);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        long long score = 0;
+        for (int h = 0; h < a.H_I; ++h) {
+            int dot = 0;
+            if (lane < kLanes) {
+                const uint32_t qw =
+                    __ldg(reinterpret_cast<const uint32_t*>(a.q_idx + ((int64_t)r * a.H_I + h) * D_I) + lane);
+                dot = (int)(int8_t)(qw & 0xffu) * s_sum[4 * lane] + (int)(int8_t)((qw >> 8) & 0xffu) * s_sum[4 * lane + 1] +
+                      (int)(int8_t)((qw >> 16) & 0xffu) * s_sum[4 * lane + 2] + (int)(int8_t)(qw >> 24) * s_sum[4 * lane + 3];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            int32_t wh = __ldg(a.w + (int64_t)r * a.H_I + h);
+            if (wh < 0 || wh > a.w_max) wh = 0;  // flagged by the query loads of the scoring passes
+            score += (long long)wh * (long long)max(dot, 0);
+        }
+        if (lane == 0) *s_out = score;
+    }
+    __syncthreads();
+    return *s_out;
+}
 
 }  // namespace lsa

@@ -61,11 +61,33 @@ struct TcArgs {
     const int32_t* q_len;
     const int64_t* kv_offset;
     const int32_t* seq_lens;
-    uint32_t* fine_keys;
+    uint64_t* cand;        // [n_q][fine_cap] candidates: key << 32 | position
+    int32_t* cand_seg;     // [n_q][kTcMaxSplits][2] (first slot, count) of each token split's candidates
     int32_t* dev_status;
     int64_t total_tokens;
-    int32_t n_q, max_len, w_max, sink, window, fine_cap;
+    int32_t n_q, max_len, w_max, sink, window, fine_cap, topk;
 };
+
+// Candidate filter. A row's keys are counted in a histogram of kTcBins bins
+// on a logarithmic scale (bit length and the 3 bits after the leading one);
+// every kTcUpdate tiles the lower edge of the highest bin whose count from the
+// top reaches topk becomes the row's threshold. Keys this CTA has seen can
+// only add to the counts, so the threshold never exceeds the k-th largest
+// key of the CTA's tokens, itself at most the row's k-th largest key: every
+// key of the final top-k is at least the threshold in force when it is
+// scored, and is kept as a candidate.
+constexpr int kTcBins = 256;
+constexpr int kTcMaxSplits = LSA_TC_MAX_SPLITS;
+constexpr int kTcUpdate = 8;
+__device__ __forceinline__ uint32_t tc_bin(uint32_t key) {
+    if (key < 8u) return key;
+    const int nb = 32 - __clz((int)key);  // 4..32
+    return ((uint32_t)(nb - 3) << 3) | ((key >> (nb - 4)) & 7u);
+}
+__device__ __forceinline__ uint32_t tc_bin_floor(uint32_t b) {
+    if (b < 8u) return b;
+    return (8u | (b & 7u)) << ((b >> 3) - 1u);
+}
 
 struct TcShared {
     uint64_t full[kTcStages];
@@ -80,6 +102,10 @@ struct TcShared {
     int32_t row_ws[kTcCols];  // window start (= middle end),
     int32_t row_ok[kTcCols];  // and validity
     alignas(16) int32_t w[kTcCols];  // weight of each query-head row (read as 16-byte vectors)
+    uint32_t thr[kTcCols / 16];             // per query row of the CTA: candidate threshold
+    uint32_t count[kTcCols / 16];           // per query row: candidates written by this CTA
+    int32_t seg0[kTcCols / 16];             // per query row: first slot of this CTA's segment
+    uint32_t hist[kTcCols / 16][kTcBins];   // per query row: histogram of its keys here
 };
 static_assert(offsetof(TcShared, w) % 16 == 0, "weights are read with 16-byte shared loads");
 static_assert(sizeof(TcShared) % 16 == 0, "TcShared follows 1024-byte aligned tiles");
@@ -213,7 +239,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
         sh.row_ok[i] = ok;
         sh.row_s[i] = s;
         sh.row_ws[i] = ws;
+        sh.thr[i] = 1u;  // every key (score + 1 >= 1) until the histogram holds topk keys
+        sh.count[i] = 0u;
     }
+    for (int i = tid; i < R * kTcBins; i += kTcThreads) (&sh.hist[0][0])[i] = 0u;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -231,6 +260,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
     const int j_lo = (int)((int64_t)nt_all * blockIdx.x / gridDim.x);
     const int j_hi = (int)((int64_t)nt_all * (blockIdx.x + 1) / gridDim.x);
     const int nt = j_hi - j_lo;
+    // this CTA's candidates of row i go to the slots of its tokens: the
+    // segment starting at the row's first middle token it scores (token splits
+    // are disjoint, so the segments are, and none passes the row's fine_cap)
+    for (int i = tid; i < R; i += kTcThreads) sh.seg0[i] = max(0, t_lo + j_lo * kTcTokens - sh.row_s[i]);
+    __syncthreads();
 
     if (warp == 0) {
         // ---- TMA producer ---------------------------------------------------
@@ -290,8 +324,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             rs[i] = sh.row_ok[ri] ? sh.row_s[ri] : 0x7fffffff;  // invalid row: no token qualifies
             rws[i] = sh.row_ws[ri];
         }
-        uint32_t* keys0 = a.fine_keys + (int64_t)(row0 + half * kRows) * a.fine_cap;
-        // 32 columns (32 / H_I query rows) of accumulators -> keys
+        const int rl0 = half * kRows;  // first query row (of the CTA) of this warp's columns
+        uint64_t* cand0 = a.cand + (int64_t)(row0 + rl0) * a.fine_cap;
+        // 32 columns (32 / H_I query rows) of accumulators -> candidates
         auto rows_of = [&](const uint32_t (&v)[32], int c, int t) {
             int32_t w[32];
 #pragma unroll
@@ -309,7 +344,59 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
 #pragma unroll
                 for (int h = 0; h < H_I; ++h) acc4[h & 3] += max((int32_t)v[rr * H_I + h], 0) * w[rr * H_I + h];
                 const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                if (t >= rs[i] && t < rws[i]) keys0[(int64_t)i * a.fine_cap + (t - rs[i])] = (uint32_t)acc + 1u;
+                const bool in = t >= rs[i] && t < rws[i];
+                const uint32_t key = (uint32_t)acc + 1u;
+                warp_hist_add(sh.hist[rl0 + i], in ? tc_bin(key) : 0xffffffffu);
+                const bool emit = in && key >= *reinterpret_cast<volatile uint32_t*>(&sh.thr[rl0 + i]);
+                const uint32_t m = __ballot_sync(0xffffffffu, emit);
+                if (m != 0u) {
+                    // one reservation per warp and row in this CTA's segment, then
+                    // the warp's candidates in lane order
+                    const uint32_t p = warp_append(&sh.count[rl0 + i], emit);
+                    if (emit) {
+                        const uint32_t slot = (uint32_t)sh.seg0[rl0 + i] + p;
+                        if (slot < (uint32_t)a.fine_cap)  // a row holds at most fine_cap middle tokens
+                            cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
+                    }
+                }
+            }
+        };
+        // the thresholds of this warp's two query rows (rows 2w', 2w'+1 of the
+        // CTA, w' the epilogue warp index), from their histograms
+        auto update_thresholds = [&]() {
+            const int ew = warp - 2;
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int row = 2 * ew + q2;
+                uint32_t c8[8];
+                uint32_t own = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    c8[j] = *reinterpret_cast<volatile uint32_t*>(&sh.hist[row][8 * lane + j]);
+                    own += c8[j];
+                }
+                uint32_t x = own;  // keys in bins >= 8 * lane
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+                    if (lane + o < 32) x += y;
+                }
+                const uint32_t k = (uint32_t)a.topk;
+                uint32_t best = 0u;  // the highest bin whose suffix count reaches k, + 1 (0: none)
+                if (k > 0u && x >= k) {
+                    uint32_t run = x - own;
+#pragma unroll
+                    for (int j = 7; j >= 0; --j) {
+                        run += c8[j];
+                        if (run >= k && best == 0u) best = (uint32_t)(8 * lane + j) + 1u;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+                if (lane == 0 && best > 0u) {
+                    const uint32_t thr = tc_bin_floor(best - 1u);
+                    if (thr > sh.thr[row]) sh.thr[row] = thr;
+                }
             }
         };
         for (int j = 0; j < nt; ++j) {
@@ -335,12 +422,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
+            if (j % kTcUpdate == kTcUpdate - 1) update_thresholds();
         }
     }
 
     // ---- teardown: wait for every issued MMA, then free TMEM -----------------
     tc_fence_before();
     __syncthreads();
+    // this CTA's candidate segment of each of its rows
+    for (int i = tid; i < R; i += kTcThreads) {
+        const int r = row0 + i;
+        if (r < a.n_q) {
+            int2* seg = reinterpret_cast<int2*>(a.cand_seg) + ((int64_t)r * kTcMaxSplits + blockIdx.x);
+            *seg = make_int2(sh.seg0[i], (int)min(sh.count[i], (uint32_t)max(0, a.fine_cap - sh.seg0[i])));
+        }
+    }
     if (warp == 1 && lane == 0) {
         umma_commit(smem_u32(&sh.drain));  // arrives once all MMAs of this thread are complete
         mbar_wait_bounded(smem_u32(&sh.drain), 0, kWaitLimitNs);
@@ -353,6 +449,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
 }
 
 }  // namespace
+
+int prefill_tc_splits(int n_q) {
+    constexpr int R = kTcCols / 16;
+    const int row_tiles = (n_q + R - 1) / R;
+    // token splits per row tile: the fewest that fill the last wave of
+    // one-CTA-per-SM launches to >= 95% (or the best of 1..kTcMaxSplits)
+    const int sms = device_sm_count();
+    int splits = 1;
+    double best = 0.0;
+    for (int sp = 1; sp <= kTcMaxSplits; ++sp) {
+        const long ctas = (long)row_tiles * sp;
+        const long waves = (ctas + sms - 1) / sms;
+        const double eff = (double)ctas / (double)(waves * sms);
+        if (eff > best + 1e-9) {
+            best = eff;
+            splits = sp;
+        }
+        if (eff >= 0.95) break;
+    }
+    return splits;
+}
 
 bool prefill_tc_supported(int H_I, int d_I, int n_seq, int64_t total_tokens) {
     return d_I == kTcK && H_I == 16 && n_seq == 1 && total_tokens + kTcTokens < (int64_t)0x7fffffff &&
@@ -369,7 +486,9 @@ cudaError_t launch_fine_scores_tc(const IndexArgs& ia, cudaStream_t stream) {
     a.q_len = ia.q_len;
     a.kv_offset = ia.kv_offset;
     a.seq_lens = ia.seq_lens;
-    a.fine_keys = ia.fine_keys;
+    a.cand = ia.cand;
+    a.cand_seg = ia.cand_seg;
+    a.topk = ia.topk;
     a.dev_status = ia.dev_status;
     a.total_tokens = ia.total_tokens;
     a.n_q = ia.n_q;
@@ -380,21 +499,10 @@ cudaError_t launch_fine_scores_tc(const IndexArgs& ia, cudaStream_t stream) {
     a.fine_cap = ia.fine_cap;
     constexpr int R = kTcCols / 16;
     const int row_tiles = (ia.n_q + R - 1) / R;
-    // token splits per row tile: the fewest that fill the last wave of
-    // one-CTA-per-SM launches to >= 95% (or the best of 1..16)
-    const int sms = device_sm_count();
-    int splits = 1;
-    double best = 0.0;
-    for (int sp = 1; sp <= 16; ++sp) {
-        const long ctas = (long)row_tiles * sp;
-        const long waves = (ctas + sms - 1) / sms;
-        const double eff = (double)ctas / (double)(waves * sms);
-        if (eff > best + 1e-9) {
-            best = eff;
-            splits = sp;
-        }
-        if (eff >= 0.95) break;
-    }
+    const int splits = ia.tc_splits;
+    if (splits < 1 || splits > kTcMaxSplits) return cudaErrorInvalidValue;
+    // every split of a row writes its segment; the segments of splits that do
+    // not exist read as empty (the selection reads `splits` of them)
     cudaError_t e = cudaFuncSetAttribute(fine_score_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kTcSmem);
     if (e != cudaSuccess) return e;

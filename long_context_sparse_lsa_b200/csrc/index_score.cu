@@ -26,12 +26,12 @@ constexpr int kCoarseChunk = kScWarps * 16;     // 128 blocks per CTA
 
 // Validates query row r; on success sets the row's cache offset and visible
 // length. Uniform over a CTA; flags nothing (the selection kernel reports).
-__device__ __forceinline__ bool row_ok(const IndexArgs& a, int r, int64_t& off, int& L) {
+__device__ __forceinline__ bool row_ok(const IndexArgs& a, int r, int64_t& off, int& L, int& slen) {
     const int seq = a.q_seq[r];
     L = a.q_len[r];
     if (seq < 0 || seq >= a.n_seq) return false;
     off = a.kv_offset[seq];
-    const int slen = a.seq_lens[seq];
+    slen = a.seq_lens[seq];
     if (L < 1 || L > a.max_len || L > slen || off < 0 || off + slen > a.total_tokens) return false;
     if (a.hi_block > 0) {
         const int64_t bo = a.blk_offset[seq];
@@ -39,14 +39,22 @@ __device__ __forceinline__ bool row_ok(const IndexArgs& a, int r, int64_t& off, 
     }
     return true;
 }
+__device__ __forceinline__ bool row_ok(const IndexArgs& a, int r, int64_t& off, int& L) {
+    int slen;
+    return row_ok(a, r, off, L, slen);
+}
 
 template <int D_I, int NT>
 __global__ void __launch_bounds__(kScThreads) coarse_score_kernel(const __grid_constant__ IndexArgs a) {
-    pdl_enter();
     const int r = blockIdx.y;
     int64_t off;
-    int L;
-    if (!row_ok(a, r, off, L)) return;
+    int L, slen;
+    // the row's metadata is the caller's, never written by a kernel of this
+    // library: it is checked before the wait for the preceding kernel (which
+    // may write the block sums)
+    const bool ok = row_ok(a, r, off, L, slen);
+    pdl_enter();
+    if (!ok) return;
     const int s = min(a.sink, L);
     const int ws = max(s, L - a.window);
     if (ws <= s) return;
@@ -54,11 +62,20 @@ __global__ void __launch_bounds__(kScThreads) coarse_score_kernel(const __grid_c
     const int b_lo = s / B, b_hi = (ws + B - 1) / B;
     const int c0 = b_lo + blockIdx.x * kCoarseChunk;
     if (c0 >= b_hi) return;
+    // the block holding the row's last visible token, summed over what the
+    // row sees when the stored sum also counts later cached tokens (uniform)
+    __shared__ int32_t s_sum[D_I];
+    __shared__ long long s_fix;
+    int b_p;
+    const bool fix = partial_block_fix(L, slen, B, ws, b_p) && b_p >= c0 &&
+                     b_p < min(c0 + kCoarseChunk, b_hi);
+    long long fixed = 0;
+    if (fix) fixed = partial_block_score<D_I, kScThreads>(a, r, a.k_idx + off * D_I, b_p * B, L - b_p * B, s_sum, &s_fix);
     const int lane = lane_id(), warp = warp_id(), g = lane >> 2, t4 = lane & 3;
     const int j0 = c0 + warp * 16 + g, j1 = j0 + 8;  // block indices of rows g and g+8
     if (c0 + warp * 16 >= b_hi) return;                // warp-uniform
     const bool v0 = j0 < b_hi, v1 = j1 < b_hi;
-    const int8_t* rows = a.block_sums + a.blk_offset[a.q_seq[r]] * (2 * D_I);
+    const int8_t* rows = a.block_sums + a.blk_offset[a.q_seq[r]] * (2 * D_I);  // (cached by row_ok)
     RowFrag<D_I> hg, lg, hg8, lg8;
     hg.load(rows + (int64_t)j0 * (2 * D_I), t4, v0);
     lg.load(rows + (int64_t)j0 * (2 * D_I) + D_I, t4, v0);
@@ -68,6 +85,9 @@ __global__ void __launch_bounds__(kScThreads) coarse_score_kernel(const __grid_c
     load_query<D_I, NT>(qf, a, r);
     long long x, y;
     coarse_tile<D_I, NT>(qf, hg, lg, hg8, lg8, x, y);
+    pdl_trigger();  // only the stores are left
+    if (fix && j0 == b_p) x = fixed;
+    if (fix && j1 == b_p) y = fixed;
     uint64_t* keys = a.coarse_keys + (int64_t)r * a.coarse_cap;
     if (t4 == 0 && v0) keys[j0 - b_lo] = (unsigned long long)x + 1ull;
     if (t4 == 1 && v1) keys[j1 - b_lo] = (unsigned long long)y + 1ull;

@@ -90,23 +90,12 @@ __host__ __device__ __forceinline__ SelLayout sel_layout(int key_bytes, int stag
     return L;
 }
 
-__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
-    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t addr, uint32_t v) {
-    uint32_t r;
-    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(r) : "r"(addr), "r"(v) : "memory");
-    return r;
-}
-__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
 template <typename K>
 __device__ __forceinline__ void st_cluster_key(uint32_t addr, K v) {
     if constexpr (sizeof(K) == 4) {
         st_cluster(addr, (uint32_t)v);
     } else {
-        asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"((unsigned long long)v) : "memory");
+        st_cluster_u64(addr, (uint64_t)v);
     }
 }
 
@@ -667,6 +656,27 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     else if (Lq < 1 || Lq > a.max_len || Lq > slen_q || off_q < 0 || off_q + slen_q > a.total_tokens ||
              (a.hi_block > 0 && (boff_q < 0 || boff_q + (Lq + a.hi_block - 1) / a.hi_block > a.block_rows)))
         bits = LSA_DEV_BAD_LENGTH;
+    if constexpr (!kTokens && D_I > 0) {
+        // a valid row that sees fewer tokens than its sequence holds: the
+        // candidate block holding its last visible token is scored over the
+        // tokens the row sees, not from the stored sum (uniform over the CTA)
+        int b_p;
+        if (bits == 0 && partial_block_fix(L, slen_q, B, ws, b_p) && b_p - first - k_lo >= 0 &&
+            b_p - first - k_lo < m) {
+            const int j = b_p - first - k_lo;
+            const long long sc = partial_block_score<D_I, kSelThreads>(
+                a, r, a.k_idx + off_q * D_I, b_p * B, L - b_p * B, reinterpret_cast<int32_t*>(sh.gt_words),
+                reinterpret_cast<long long*>(sh.eq_words));
+            if (threadIdx.x == 0) {
+                uint64_t* st = reinterpret_cast<uint64_t*>(stage);
+                const uint64_t old = st[j], key = (unsigned long long)sc + 1ull;
+                st[j] = key;
+                atomicSub(&sh.local_hist[key_bin(old)], 1u);
+                atomicAdd(&sh.local_hist[key_bin(key)], 1u);
+            }
+            __syncthreads();
+        }
+    }
     cluster_wait();  // complete the barrier every CTA arrived at (an exiting CTA must too)
     if (bits != 0) {
         if (kTokens) {
@@ -739,7 +749,7 @@ static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // Staged slice keys plus kept-block ids stay within this much shared memory.
 constexpr size_t kStageSmem = 144 * 1024;
 
-IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
+IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b, bool dense) {
     IndexPlan p;
     const bool hi = b.hi_block > 0;
     if (hi) {
@@ -767,6 +777,8 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
         p.fine_stage = (size_t)sm * 4 + (size_t)p.kept_slots * 4 <= kStageSmem ? sm : 0;
         p.smem_tokens = sel_layout(4, p.fine_stage, p.kept_slots).bytes;
     }
+    if (hi && !topk_plan(p.coarse_cap, 8, p.tk_kp_blocks, p.tk_cl_blocks)) p.tk_kp_blocks = p.tk_cl_blocks = 0;
+    if (!topk_plan(p.fine_cap, 4, p.tk_kp_tokens, p.tk_cl_tokens)) p.tk_kp_tokens = p.tk_cl_tokens = 0;
     size_t off = 0;
     p.off_coarse = off;
     off = align256(off + (size_t)n_q * p.coarse_cap * 8);
@@ -775,7 +787,15 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b) {
     p.off_nkept = off;
     off = align256(off + (size_t)n_q * 4);
     p.off_fine = off;
-    off = align256(off + (size_t)n_q * p.fine_cap * 4);
+    if (dense) {
+        // candidate pairs (8 bytes) in place of the one-key-per-token array
+        p.off_cand = off;
+        off = align256(off + (size_t)n_q * p.fine_cap * 8);
+        p.off_count = off;
+        off = align256(off + (size_t)n_q * LSA_TC_MAX_SPLITS * 8);
+    } else {
+        off = align256(off + (size_t)n_q * p.fine_cap * 4);
+    }
     p.ws_bytes = off;
     return p;
 }

@@ -84,6 +84,9 @@ struct IndexArgs {
     int32_t* kept;          // [n_q][hi_topblocks] kept block ids, ascending
     int32_t* n_kept;        // [n_q]
     uint32_t* fine_keys;    // [n_q][fine_cap] token keys (score + 1, 0 = none)
+    uint64_t* cand;         // prefill chunks: [n_q][fine_cap] candidate pairs (key << 32 | position)
+    int32_t* cand_seg;      // prefill chunks: [n_q][LSA_TC_MAX_SPLITS][2] (first slot, count) per token split
+    int32_t tc_splits;      // prefill chunks: token splits of the tensor-core scoring
     int32_t coarse_cap, fine_cap;
     // selection: keys of one CTA's slice staged in shared memory (0 = read
     // from global memory) and kept-block slots per slice
@@ -92,13 +95,18 @@ struct IndexArgs {
 
 struct IndexPlan {
     int coarse_cap = 0, fine_cap = 0;
+    // register-held selection (index_topk.cu): keys per thread and CTAs per
+    // row, or 0 when a row's keys exceed it (the cluster kernels below)
+    int tk_kp_blocks = 0, tk_cl_blocks = 0, tk_kp_tokens = 0, tk_cl_tokens = 0;
     int cluster = 8;                          // CTAs per query row in the selection kernels
     int coarse_stage = 0, fine_stage = 0, kept_slots = 0;
     size_t smem_blocks = 0, smem_tokens = 0;  // dynamic smem of the selection kernels
-    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0;
+    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0, off_cand = 0, off_count = 0;
     size_t ws_bytes = 0;
 };
-IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b);
+// dense: the batch is a prefill chunk scored by the tensor-core contraction
+// (candidate pairs instead of one key per token)
+IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b, bool dense = false);
 cudaError_t launch_index_scores(const IndexArgs& a, int d_I, bool coarse, cudaStream_t stream);
 // Fine scores of a causal chunk of rows of one sequence (HI off) on the
 // tcgen05 tensor cores; same keys as launch_index_scores(coarse = false).
@@ -108,6 +116,9 @@ bool prefill_tc_supported(int H_I, int d_I, int n_seq, int64_t total_tokens);
 bool tensor_maps_available();
 bool tensor_map_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows);
 cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
+// Token splits of each 16-row tile in the tensor-core scoring (<= LSA_TC_MAX_SPLITS).
+#define LSA_TC_MAX_SPLITS 16
+int prefill_tc_splits(int n_q);
 // HI block selection computes the coarse scores itself when each cluster
 // CTA's slice of blocks fits in shared memory, the query has at most 16
 // indexer heads (more would not fit the selection kernel's 64 registers) and
@@ -118,6 +129,13 @@ inline bool coarse_in_select(int hi_block, int coarse_stage, int H_I, int n_q) {
     return hi_block > 0 && coarse_stage > 0 && H_I <= 16 && n_q >= 8;
 }
 inline bool coarse_in_select(const IndexArgs& a) { return coarse_in_select(a.hi_block, a.coarse_stage, a.H_I, a.n_q); }
+// Exact top-k with the keys of a row held by one CTA of 1024 threads (or a
+// cluster of up to 4): keys per thread and cluster size for rows of up to
+// `cap` keys of `key_bytes` bytes, false when more.
+bool topk_plan(int cap, int key_bytes, int& kp, int& cluster);
+cudaError_t launch_topk(const IndexArgs& a, bool blocks, int kp, int cluster, cudaStream_t stream);
+// Prefill chunks: exact top-k over each row's candidate pairs, SI assembly.
+cudaError_t launch_topk_pairs(const IndexArgs& a, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
                                 cudaStream_t stream);
 
@@ -152,7 +170,8 @@ struct AttendPlan {
     size_t smem_bytes = 0;
     size_t ws_bytes = 0;
 };
-AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms);
+AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms,
+                       bool fp8 = false);
 cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
 
 int device_sm_count();

@@ -155,16 +155,19 @@ class LsaStep:
         return int(self.status.item())
 
     # -- CUDA graphs ------------------------------------------------------------
-    def capture(self):
+    def capture(self, fork_append: bool = False):
         """Capture the three calls as CUDA graphs (append, index, attend), and
-        the whole step as one more graph ("step") in which the append runs on
-        a forked stream beside the index call when overlap_ok(). A step then
-        replays without host launch overhead. Two more graphs serve
-        measurement: "step_timed" (the step with timing events around the
-        index and attention calls) and, with HI on, "cold" (a full block-sum
-        build, then index and attention). The graphs keep this object's
-        buffers; changing their contents between replays is how new inputs
-        enter."""
+        the whole step as one more graph ("step"). In the step graph the three
+        calls follow each other on one stream, so every kernel boundary keeps
+        its programmatic (early) launch; with fork_append (and overlap_ok())
+        the append runs on a forked stream beside the index call instead,
+        which turns the attention's dependence on the index call into a full
+        graph edge. A step then replays without host launch overhead. Two
+        more graphs serve measurement: "step_timed" (the step with timing
+        events around the index and attention calls) and, with HI on, "cold"
+        (a full block-sum build, then index and attention). The graphs keep
+        this object's buffers; changing their contents between replays is how
+        new inputs enter."""
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):  # one eager pass fills the launch-plan caches
@@ -181,9 +184,10 @@ class LsaStep:
             self.graphs[name] = g
         g = torch.cuda.CUDAGraph()
         fork = torch.cuda.Stream(self.device)
+        fork_ok = fork_append and self.overlap_ok()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             cur = torch.cuda.current_stream(self.device)
-            if self.overlap_ok():
+            if fork_ok:
                 fork.wait_stream(cur)
                 with torch.cuda.stream(fork):
                     self.append()
@@ -202,7 +206,7 @@ class LsaStep:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             cur = torch.cuda.current_stream(self.device)
-            overlap = self.overlap_ok()
+            overlap = fork_ok
             if overlap:
                 fork.wait_stream(cur)
                 with torch.cuda.stream(fork):

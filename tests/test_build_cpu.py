@@ -4,7 +4,7 @@ Every kernel source is compiled for sm_100a with the library's flags and
 `-Xptxas -v`; no entry function may spill registers beyond the allowance
 below. The allowances are the spills measured today, all on paths that the
 timed workloads do not take, except the block selection with fused coarse
-scores at d_I = 128 (28 bytes), which is on the 16 x 128K decode path.
+scores at d_I = 128 (36 bytes), which is on the 16 x 128K decode path.
 """
 from __future__ import annotations
 
@@ -22,7 +22,7 @@ KNOWN_SPILLS = {
     "attend_kernelILi2E": 400,            # groups of 16 query heads (TMA bulk-copy K path)
     "fine_score_kernelILi128ELi8E": 400,  # 64 indexer heads, per-lane gathers
     "fine_score_tma_kernelILi8E": 128,    # 64 indexer heads
-    "select_kernelImLb0ELi128ELi2E": 32,  # block selection with coarse scores, d_I 128, <= 16 heads
+    "select_kernelImLb0ELi128ELi2E": 40,  # block selection with coarse scores, d_I 128, <= 16 heads
     "select_kernelImLb0ELi64ELi2E": 16,   # the same at d_I 64
     "select_kernelImLb0ELi64ELi1E": 8,    # d_I 64, <= 8 heads
 }

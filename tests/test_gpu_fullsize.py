@@ -5,10 +5,9 @@ index, attend) replayed once on seeded inputs.
   * batched decode, 16 sequences x 131072 tokens, HI 64 x 256: every row;
   * 1M-token decode with one index set for G = 4 layers, HI 128 x 512: the row
     and all four layers;
-  * 64 ragged sequences (lognormal lengths, G = 2): a seeded sample of rows
-    plus the longest and the shortest;
-  * a causal prefill chunk of 8192 rows on a 262144-token cache (HI off): a
-    sample spanning the chunk.
+  * 64 ragged sequences (lognormal lengths, G = 2): every row;
+  * a causal prefill chunk of 8192 rows on a 262144-token cache (HI off): 64
+    rows spanning the chunk.
 
 Index sets are compared bit-exact with the oracle; attention within
 max|err| 5e-3 and rel-L2 1e-3 of its fp64 evaluation on the K/V rows the
@@ -75,14 +74,10 @@ def test_1m_cross_layer_decode_every_layer():
     _free()
 
 
-def test_ragged_batch_sample():
+def test_ragged_batch_every_row():
     wl = wls.ragged()
-    lens = np.asarray(wl.lens)
-    rng = np.random.default_rng(4)
-    rows = set(rng.choice(wl.n_q, size=10, replace=False).tolist())
-    rows |= {int(lens.argmax()), int(lens.argmin())}
     st, t = _run_graph(wl)
-    _check(wl, st, t, sorted(rows))
+    _check(wl, st, t, np.arange(wl.n_q))
     del st, t
     _free()
 
@@ -116,7 +111,9 @@ def test_prefill_chunk_sample():
     st, t = _run_graph(wl)
     assert lsa.lsa_index_uses_tensor_cores(st.batch, wl.H_I, wl.d_I, st.budget)
     n = wl.n_q
-    rows = [0, 1, 2047, 4096, 6000, n - 2, n - 1]
+    # 64 rows spread over the chunk (both ends, every 1/62 of it between)
+    rows = sorted({0, 1, n - 2, n - 1} | {int(x) for x in np.linspace(2, n - 3, 60)})
+    assert len(rows) == 64
     _check(wl, st, t, rows)
     del st, t
     _free()

@@ -352,3 +352,68 @@ def test_graph_replay_matches_eager():
     ms = st.call_ms()
     assert 0.0 < ms["index"] < 1000.0 and 0.0 < ms["attend"] < 1000.0
     parity.check_sets(sets0, parity.oracle_sets(wl, t), "graph")
+
+
+# HI rows that see fewer tokens than their sequence holds, with a window
+# shorter than a block: the candidate block holding a row's last visible
+# token must be summed over the tokens the row sees (the oracle's block sums
+# over [b*B, min((b+1)*B, L))), not taken from the stored sum of the whole
+# cached block. Draft rows (more rows than sequences: coarse scores inside
+# the block selection), causal prefill rows, and rows whose q_len was moved
+# below seq_lens with as many rows as sequences (the separate coarse kernel).
+R5_CASES = {
+    "drafts_short_window": dict(lens=(5000, 3000, 7001), drafts=4, hi_block=64, hi_topblocks=16, sink=8,
+                                window=10, topk=300, G=2),
+    "drafts_one_seq_b128": dict(lens=(9000,), drafts=4, hi_block=128, hi_topblocks=12, sink=4, window=0,
+                                topk=500),
+    "prefill_rows_b32": dict(lens=(3000 + 40,), prefill_new=40, hi_block=32, hi_topblocks=20, sink=4, window=5,
+                             topk=200),
+}
+
+
+@pytest.mark.parametrize("name", sorted(R5_CASES))
+def test_hi_rows_shorter_than_their_sequence(name):
+    kw = dict(R5_CASES[name])
+    kw.setdefault("seed", 500 + sorted(R5_CASES).index(name))
+    wl = wls.small(BASE, name=name, **kw)
+    st, _ = run_case(wl)
+    assert st.status_bits() == 0
+
+
+def test_hi_q_len_below_seq_lens_one_row_per_sequence():
+    wl = wls.small(BASE, name="r5_qlen", lens=(4000, 6000, 2500), hi_block=64, hi_topblocks=10, sink=16, window=20,
+                   topk=250, seed=510)
+    t = wls.make(wl, DEV)
+    t.q_len.copy_(torch.tensor([3950, 5999, 2431], dtype=torch.int32, device=DEV))
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    st.index()
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    want = parity.oracle_sets(wl, t)
+    parity.check_sets(parity.host(st.sets), want, wl.name)
+    ref = parity.oracle_attend_full(t, want)
+    parity.check_attention(parity.host(st.out[0]), ref[0], wl.name)
+
+
+def test_fp8_query_outside_fp16_range_is_flagged():
+    """lsa_attend_fp8 multiplies on fp16 tensor cores: a bf16 query element
+    of magnitude 65536 or more has no fp16 value, so the call flags the row
+    (LSA_DEV_BAD_QUERY) instead of returning a silently wrong output; queries
+    inside the range leave the status clear."""
+    wl = wls.small(BASE, name="fp8_qrange", lens=(3000, 2000), hi_block=0, hi_topblocks=0, seed=43)
+    t = wls.make(wl, DEV, with_kv=False)
+    st = LsaStep(wl, t, DEV, kv_fp8=True)
+    st.index()
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    t.q[0][1, 3, 17] = 65280.0  # the largest bf16 below 65504: still an fp16
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    t.q[0][1, 3, 17] = -70000.0
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() & lsa.LSA_DEV_BAD_QUERY

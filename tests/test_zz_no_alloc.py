@@ -42,6 +42,10 @@ def test_noalloc_matches_workspace_version_twice(wl):
     t, st, want = _reference(wl)
     need = lsa.lsa_attend_workspace_size(st.batch, wl.H_q, wl.H_kv, wl.d, st.budget.length, len(t.q))
     assert 0 < need <= (8 << 20)
+    # the oracle's attention over the oracle's own sets (the GPU sets match them bit for bit)
+    sets = parity.oracle_sets(wl, t)
+    parity.check_sets(parity.host(st.sets), sets, wl.name)
+    ref = parity.oracle_attend_full(t, sets)
     for call in range(2):
         outs = [torch.full_like(o, float("nan")) for o in st.out]
         lsa.lsa_attend_noalloc(t.q, t.k, t.v, st.sets, st.batch, outs, st.status)
@@ -49,7 +53,8 @@ def test_noalloc_matches_workspace_version_twice(wl):
         assert st.status_bits() == 0
         for g in range(len(outs)):
             got = parity.host(outs[g])
-            parity.check_attention(got, want[g], f"{wl.name} call {call} layer {g}")
+            parity.check_attention(got, want[g], f"{wl.name} call {call} layer {g} vs lsa_attend")
+            parity.check_attention(got, ref[g], f"{wl.name} call {call} layer {g} vs oracle")
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
