@@ -200,8 +200,7 @@ int32_t lsa_index_launches(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, l
     (void)d_I;
     if (budget.hi_block == 0) return 2;  // fine scores, token selection
     const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, budget);
-    const bool fused = plan.tk_kp_blocks == 0 && lsa::coarse_in_select(budget.hi_block, plan.coarse_stage, H_I,
-                                                                        batch->n_q);
+    const bool fused = lsa::coarse_in_select(budget.hi_block, plan.coarse_stage, H_I, batch->n_q);
     return (fused ? 1 : 2) + 2;  // [coarse scores,] block selection, fine scores, token selection
 }
 
@@ -285,14 +284,8 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (budget.hi_block > 0) {
-        if (plan.tk_kp_blocks > 0) {
-            // coarse scores of every candidate block, then one selection CTA per row
-            e = lsa::launch_index_scores(a, d_I, true, cs);
-            if (e == cudaSuccess) e = lsa::launch_topk(a, true, plan.tk_kp_blocks, plan.tk_cl_blocks, cs);
-        } else {
-            if (!lsa::coarse_in_select(a)) e = lsa::launch_index_scores(a, d_I, true, cs);
-            if (e == cudaSuccess) e = lsa::launch_index_select(a, true, d_I, plan.cluster, plan.smem_blocks, cs);
-        }
+        if (!lsa::coarse_in_select(a)) e = lsa::launch_index_scores(a, d_I, true, cs);
+        if (e == cudaSuccess) e = lsa::launch_index_select(a, true, d_I, plan.cluster, plan.smem_blocks, cs);
     }
     if (e == cudaSuccess) {
         // a prefill chunk (many rows of one sequence, HI off) is one dense
@@ -300,9 +293,8 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
         e = dense ? lsa::launch_fine_scores_tc(a, cs) : lsa::launch_index_scores(a, d_I, false, cs);
     }
     if (e == cudaSuccess) {
-        if (dense) e = lsa::launch_topk_pairs(a, cs);
-        else if (plan.tk_kp_tokens > 0) e = lsa::launch_topk(a, false, plan.tk_kp_tokens, plan.tk_cl_tokens, cs);
-        else e = lsa::launch_index_select(a, false, d_I, plan.cluster, plan.smem_tokens, cs);
+        e = dense ? lsa::launch_topk_pairs(a, cs)
+                  : lsa::launch_index_select(a, false, d_I, plan.cluster, plan.smem_tokens, cs);
     }
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }

@@ -49,9 +49,9 @@ constexpr int kTile = 16;                              // tokens per stage
 constexpr int kD = 128;
 constexpr int kHeadBytes = kD * 2;                     // one (token, kv head) row
 constexpr int kMaxEntriesPerSplit = 4096;
-constexpr int kPrefetch = 4;  // attention: tiles prefetched into L2 beyond the two in registers
 constexpr int kMaxStages = 8;
 constexpr size_t kAtSmemBudget = 200 * 1024;
+constexpr size_t kSmemPerSm = 228 * 1024;  // the shared-memory carveout's 100%
 
 // V rows of one 16-token tile for one kv head, in the registers of lane
 // (g, t): tokens 2t, 2t+1, 2t+8, 2t+9 (index j = 0..3), 16-byte chunks g and
@@ -676,25 +676,7 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
         load_k(kb2, s_ent + (wsel + n_sel) * kTile);
         load_v(vb2, s_ent + (wsel + n_sel) * kTile);
     }
-    // L2 prefetch of the K and V rows of this warp's tile kPrefetch steps
-    // beyond the register loads: those loads then find their rows in L2, so
-    // the two tiles of registers in flight cover an L2 latency, not DRAM's.
-    // Lane l covers token l % 16: its K and V rows (one 128-byte line per
-    // FP8 row, two per bf16 row; lanes 16..31 take the second line).
-    auto prefetch = [&](int i) {
-        if (i >= n_tiles) return;
-        const int e = s_ent[i * kTile + (lane & 15)];
-        if (e < 0) return;
-        const int line = FP8 ? 0 : (lane >> 4);
-        if (FP8 && lane >= 16) return;
-        const uint8_t* pk = kbase + (int64_t)e * tok_stride * kEB + 128 * line;
-        const uint8_t* pv = vbase + (int64_t)e * tok_stride * kEB + 128 * line;
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(pk));
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(pv));
-    };
-    for (int p = 2; p < 2 + kPrefetch; ++p) prefetch(wsel + p * n_sel);
     auto tile = [&](int i, KT& k, VT& v) {
-        prefetch(i + (2 + kPrefetch) * n_sel);
         const int ent_lane = lane < kTile ? s_ent[i * kTile + lane] : 0;
         const uint32_t masked = __ballot_sync(0xffffffffu, lane < kTile && ent_lane < 0);
         const bool ok_g = !((masked >> g) & 1u);
@@ -878,6 +860,12 @@ cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t s
     if (ratio <= 8) {
         auto kern = a.kv_fp8 ? attend_rk_kernel<true> : attend_rk_kernel<false>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
+        if (e != cudaSuccess) return e;
+        // the register-streaming gather keeps its loads in flight in L1: ask
+        // for the smallest shared-memory carveout that holds the CTA, so the
+        // rest of the SM's 256 KB stays L1 whatever the previous kernel used
+        const int pct = (int)(((smem_bytes + 2048) * 100 + kSmemPerSm - 1) / kSmemPerSm);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct < 100 ? pct : 100);
         if (e != cudaSuccess) return e;
         e = launch_pdl(kern, grid, dim3(kConsumers * kWarp), smem_bytes, stream, 0, a);
         if (e != cudaSuccess) return e;

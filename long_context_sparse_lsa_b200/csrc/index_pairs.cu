@@ -1,0 +1,248 @@
+// index_pairs.cu — exact top-k of a prefill chunk's rows from the candidate
+// (key, position) pairs the tensor-core scoring kept, and the SI assembly of
+// their index sets.
+//
+// The method: the topk best middle tokens of each row, ties to the lower
+// position; the index set is the sink run, the selected tokens and the window
+// run in ascending order, padded with -1 ("LongCat-Flash-Lite-Sparse
+// (aitrends.kr)", section "기술적 특징", SI bullet; "LongCat-2.0
+// (molayo1419.me)", section "1M 토큰에서의 Sparse Attention 문제").
+#include "common.cuh"
+#include "index_common.cuh"
+#include "internal.h"
+
+namespace lsa {
+namespace {
+
+constexpr int kTkThreads = 1024;
+constexpr int kTkWarps = kTkThreads / kWarp;
+static_assert(kHistBins / kTkThreads == 4, "the scan gives each thread one 4-bin vector");
+constexpr int kTkCandCap = 2048;  // keys of the threshold bin held in the candidate list
+constexpr int kTkDigitBits = 12;
+
+__device__ __forceinline__ uint32_t tk_warp_sum(uint32_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Prefill rows: the tensor-core scoring kept, per row, the (key, position)
+// pairs that passed its running threshold, in no particular order. The row's
+// exact top-k by (key desc, position asc) is the top-k of the distinct
+// values key << 32 | (2^32 - 1 - position), found over the pairs in global
+// memory (histogram pass, then radix digits over the threshold bin's
+// candidates or, for a bin too full for the list, over all pairs); the kept
+// positions are sorted ascending in shared memory (bitonic) and written with
+// the SI sink and window runs. One CTA of 1024 threads per row.
+constexpr int kPairSortCap = LSA_MAX_BUDGET;  // topk <= budget
+
+struct PairShared {
+    uint32_t hist[kHistBins];
+    uint64_t cand[kTkCandCap];
+    uint32_t wsum[kTkWarps];
+    uint32_t wsum2[kTkWarps];
+    uint32_t bin, above, in_bin;
+    uint32_t n_cand, n_sel;
+};
+
+__device__ __forceinline__ uint64_t pair_value(uint64_t e) {
+    return (e & 0xffffffff00000000ull) | (uint64_t)(0xffffffffu - (uint32_t)e);
+}
+
+// Suffix scan of sh.hist (4 bins per thread). Returns the number of counted
+// keys; when 1 <= krem <= total sets sh.bin / sh.above / sh.in_bin to the bin
+// holding the krem-th largest value, the count above it and the count in it.
+__device__ uint32_t pair_find_bin(PairShared& sh, uint32_t krem) {
+    const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
+    const uint4 h = reinterpret_cast<const uint4*>(sh.hist)[tid];
+    const uint32_t c[4] = {h.x, h.y, h.z, h.w};
+    const uint32_t own = c[0] + c[1] + c[2] + c[3];
+    uint32_t x = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += v;
+    }
+    if (lane == 0) sh.wsum[wid] = x;
+    __syncthreads();
+    const uint32_t wt = sh.wsum[lane];
+    const uint32_t later = tk_warp_sum(lane > wid ? wt : 0u);
+    const uint32_t total = tk_warp_sum(wt);
+    const uint32_t S = x + later;
+    if (krem >= 1u && S >= krem && S - own < krem) {
+        uint32_t run = S - own;
+#pragma unroll
+        for (int j = 3; j >= 0; --j) {
+            if (run + c[j] >= krem) {
+                sh.bin = (uint32_t)(4 * tid + j);
+                sh.above = run;
+                sh.in_bin = c[j];
+                break;
+            }
+            run += c[j];
+        }
+    }
+    __syncthreads();
+    return total;
+}
+
+__global__ void __launch_bounds__(kTkThreads, 1) topk_pairs_kernel(const __grid_constant__ IndexArgs a) {
+    extern __shared__ __align__(16) uint8_t pr_dyn[];
+    PairShared& sh = *reinterpret_cast<PairShared*>(pr_dyn);
+    int32_t* sel = reinterpret_cast<int32_t*>(pr_dyn + (sizeof(PairShared) + 15) / 16 * 16);
+    const int r = blockIdx.x;
+    const int tid = threadIdx.x;
+    // the row's metadata (the caller's) before the wait for the scoring kernel
+    const int Lq = a.q_len[r];
+    const int seq_q = a.q_seq[r];
+    const int seq_c = min(max(seq_q, 0), a.n_seq - 1);
+    const int64_t off_q = a.kv_offset[seq_c];
+    const int slen_q = a.seq_lens[seq_c];
+    pdl_enter();
+    const int L = min(max(Lq, 0), a.max_len);
+    const int s = min(a.sink, L);
+    const int ws = max(s, L - a.window);
+    int32_t* out = a.index_sets + (int64_t)r * a.budget;
+    int32_t bits = 0;
+    if (seq_q < 0 || seq_q >= a.n_seq) bits = LSA_DEV_BAD_SEQ;
+    else if (Lq < 1 || Lq > a.max_len || Lq > slen_q || off_q < 0 || off_q + slen_q > a.total_tokens)
+        bits = LSA_DEV_BAD_LENGTH;
+    if (bits != 0) {
+        if (tid == 0) flag(a.dev_status, bits);
+        for (int e = tid; e < a.budget; e += kTkThreads) out[e] = -1;
+        return;
+    }
+    // the row's candidates: one segment per token split of the scoring
+    const uint64_t* pairs = a.cand + (int64_t)r * a.fine_cap;
+    __shared__ int32_t seg_lo[LSA_TC_MAX_SPLITS], seg_n[LSA_TC_MAX_SPLITS];
+    if (tid < a.tc_splits) {
+        const int2 sg = reinterpret_cast<const int2*>(a.cand_seg)[(int64_t)r * LSA_TC_MAX_SPLITS + tid];
+        const int lo = min(max(sg.x, 0), a.fine_cap);
+        seg_lo[tid] = lo;
+        seg_n[tid] = min(max(sg.y, 0), a.fine_cap - lo);
+    }
+    __syncthreads();
+    uint32_t n = 0;
+    for (int sp = 0; sp < a.tc_splits; ++sp) n += (uint32_t)seg_n[sp];
+    // every candidate pair once: f(pair)
+    // (every lane of a warp calls f the same number of times: f(pair, ok))
+    auto for_each_pair = [&](auto&& f) {
+        for (int sp = 0; sp < a.tc_splits; ++sp) {
+            const uint64_t* seg = pairs + seg_lo[sp];
+            const int cnt = seg_n[sp];
+            for (int i0 = tid - (tid & 31); i0 < cnt; i0 += kTkThreads) {
+                const int i = i0 + (tid & 31);
+                const bool ok = i < cnt;
+                f(ok ? __ldcg(seg + i) : 0ull, ok);
+            }
+        }
+    };
+    const uint32_t k = min((uint32_t)a.topk, (uint32_t)(ws - s));  // every middle token is a candidate
+    // the index set's sink and window runs and padding
+    {
+        const int win0 = s + (int)k;
+        const int n_win = L - ws;
+        for (int e = tid; e < a.budget; e += kTkThreads) {
+            if (e < s) out[e] = e;
+            else if (e >= win0 && e < win0 + n_win) out[e] = ws + (e - win0);
+            else if (e >= win0 + n_win) out[e] = -1;
+        }
+    }
+    if (k == 0u) return;
+    // the k largest values: value >= T
+    uint64_t T = 0ull;
+    if (n > k) {
+        for (int i = tid; i < kHistBins; i += kTkThreads) sh.hist[i] = 0u;
+        if (tid == 0) sh.n_cand = 0u;
+        __syncthreads();
+        for_each_pair([&](uint64_t e, bool ok) {
+            if (ok) atomicAdd(&sh.hist[key_bin(pair_value(e))], 1u);
+        });
+        __syncthreads();
+        pair_find_bin(sh, k);
+        const uint32_t tb = sh.bin, in_bin = sh.in_bin;
+        uint32_t kr = k - sh.above;
+        const int nb = (int)(tb >> 6) + 6;
+        int shift = tb < 64u ? 0 : nb - 7;
+        uint64_t prefix = tb < 64u ? (uint64_t)tb : (uint64_t)(64u | (tb & 63u));
+        const bool listed = in_bin <= (uint32_t)kTkCandCap;
+        if (listed) {
+            __syncthreads();
+            for_each_pair([&](uint64_t e, bool ok) {
+                const uint64_t v = pair_value(e);
+                const bool take = ok && key_bin(v) == tb;
+                const uint32_t p = warp_append(&sh.n_cand, take);
+                if (take && p < (uint32_t)kTkCandCap) sh.cand[p] = v;
+            });
+            __syncthreads();
+        }
+        const uint32_t nc = min(sh.n_cand, (uint32_t)kTkCandCap);
+        while (shift > 0) {
+            const int width = shift < kTkDigitBits ? shift : kTkDigitBits;
+            shift -= width;
+            const uint64_t mask = (1ull << width) - 1ull;
+            reinterpret_cast<uint4*>(sh.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+            __syncthreads();
+            if (listed) {
+                for (uint32_t i = tid; i < nc; i += kTkThreads) {
+                    const uint64_t v = sh.cand[i];
+                    if ((v >> (shift + width)) == prefix) atomicAdd(&sh.hist[(uint32_t)((v >> shift) & mask)], 1u);
+                }
+            } else {
+                for_each_pair([&](uint64_t e, bool ok) {
+                    const uint64_t v = pair_value(e);
+                    if (ok && (v >> (shift + width)) == prefix) atomicAdd(&sh.hist[(uint32_t)((v >> shift) & mask)], 1u);
+                });
+            }
+            __syncthreads();
+            pair_find_bin(sh, kr);
+            prefix = (prefix << width) | sh.bin;
+            kr -= sh.above;
+        }
+        T = prefix;  // values are distinct: exactly k are >= T
+    }
+    // the kept positions, then sorted ascending
+    if (tid == 0) sh.n_sel = 0u;
+    __syncthreads();
+    for_each_pair([&](uint64_t e, bool ok) {
+        const bool take = ok && pair_value(e) >= T;
+        const uint32_t p = warp_append(&sh.n_sel, take);
+        if (take && p < (uint32_t)kPairSortCap) sel[p] = (int32_t)(uint32_t)e;
+    });
+    __syncthreads();
+    const uint32_t m = min(sh.n_sel, k);
+    uint32_t P = 1;
+    while (P < m) P <<= 1;
+    for (uint32_t i = m + tid; i < P; i += kTkThreads) sel[i] = 0x7fffffff;
+    __syncthreads();
+    for (uint32_t size = 2; size <= P; size <<= 1) {
+        for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
+            for (uint32_t i = tid; i < P / 2; i += kTkThreads) {
+                const uint32_t lo = 2 * i - (i & (stride - 1));  // index with bit `stride` clear
+                const uint32_t hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const int32_t x = sel[lo], y = sel[hi];
+                if ((x > y) == up) {
+                    sel[lo] = y;
+                    sel[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    pdl_trigger();
+    for (uint32_t i = tid; i < m; i += kTkThreads) out[s + i] = sel[i];
+}
+
+}  // namespace
+
+size_t topk_pairs_smem() { return (sizeof(PairShared) + 15) / 16 * 16 + (size_t)kPairSortCap * 4; }
+
+cudaError_t launch_topk_pairs(const IndexArgs& a, cudaStream_t stream) {
+    const size_t smem = topk_pairs_smem();
+    cudaError_t e = cudaFuncSetAttribute(topk_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_pairs_kernel, dim3((unsigned)a.n_q), dim3(kTkThreads), smem, stream, 0, a);
+}
+
+}  // namespace lsa

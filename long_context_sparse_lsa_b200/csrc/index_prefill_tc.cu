@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
                 const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 const bool in = t >= rs[i] && t < rws[i];
                 const uint32_t key = (uint32_t)acc + 1u;
-                warp_hist_add(sh.hist[rl0 + i], in ? tc_bin(key) : 0xffffffffu);
+                if (in) atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
                 const bool emit = in && key >= *reinterpret_cast<volatile uint32_t*>(&sh.thr[rl0 + i]);
                 const uint32_t m = __ballot_sync(0xffffffffu, emit);
                 if (m != 0u) {

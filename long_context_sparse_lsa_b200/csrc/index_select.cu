@@ -204,12 +204,14 @@ __device__ __forceinline__ void zero_hists(SelShared& sh) {
     h[threadIdx.x + kSelThreads] = z;
 }
 
-// One pass over the slice's m keys in 16-byte vectors: copies them to `stage`
-// when given and adds the nonzero ones to sh.local_hist.
+// One pass over the slice's keys in 16-byte vectors: copies them to `stage`
+// when given and adds the nonzero ones of the first m to sh.local_hist.
 template <typename K>
-__device__ void stage_pass(SelShared& sh, const Keys<K>& src, int m, K* stage) {
+// m_load >= m keys are loaded (and staged), the first m are counted: the
+// loads can be issued before m is known.
+__device__ void stage_pass(SelShared& sh, const Keys<K>& src, int m, int m_load, K* stage) {
     constexpr int kPer = 16 / (int)sizeof(K);
-    const int nv = (m + kPer - 1) / kPer;
+    const int nv = (m_load + kPer - 1) / kPer;
     for (int i0 = threadIdx.x; i0 < nv; i0 += kSelThreads * kUnroll) {
         uint4 v[kUnroll];
 #pragma unroll
@@ -275,7 +277,8 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uin
     if (in_bin <= (uint32_t)kCandCap) {
         // gather this slice's keys of the bin, then append them to every
         // CTA's candidate list
-        for (int i0 = threadIdx.x; i0 < m; i0 += kSelThreads * kUnroll) {
+        // (warp-uniform trip count: every lane of a warp takes part in warp_append)
+        for (int i0 = threadIdx.x; i0 - lane_id() < m; i0 += kSelThreads * kUnroll) {
             K kv[kUnroll];
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
@@ -284,10 +287,9 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uin
             }
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
-                if (i0 + u * kSelThreads < m && kv[u] != K(0) && (K)(kv[u] >> shift) == prefix) {
-                    const uint32_t p = atomicAdd(&sh.local_count, 1u);
-                    if (p < (uint32_t)kCandCap) mine[p] = kv[u];
-                }
+                const bool take = i0 + u * kSelThreads < m && kv[u] != K(0) && (K)(kv[u] >> shift) == prefix;
+                const uint32_t p = warp_append(&sh.local_count, take);  // one atomic per warp
+                if (take && p < (uint32_t)kCandCap) mine[p] = kv[u];
             }
         }
         // this slice's keys above the bin
@@ -340,12 +342,20 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uin
         }
         __syncthreads();
         const K T = prefix;
-        for (int i = threadIdx.x; i < mm; i += kSelThreads) {
-            const uint64_t e = cand[i];
+        // per CTA of origin, with warp ballots (the list's entries share few counters)
+        for (int i0 = threadIdx.x - lane_id(); i0 < mm; i0 += kSelThreads) {
+            const int i = i0 + lane_id();
+            const uint64_t e = i < mm ? cand[i] : 0ull;
             const K key = (K)(e & kKeyMask);
             const uint32_t o = (uint32_t)(e >> kOriginShift);
-            if (key > T) atomicAdd(&sh.og_gt[o], 1u);
-            else if (key == T) atomicAdd(&sh.og_eq[o], 1u);
+            for (uint32_t t = 0; t < C; ++t) {
+                const uint32_t g = __ballot_sync(0xffffffffu, i < mm && o == t && key > T);
+                const uint32_t q = __ballot_sync(0xffffffffu, i < mm && o == t && key == T);
+                if (lane_id() == 0) {
+                    if (g) atomicAdd(&sh.og_gt[t], (uint32_t)__popc(g));
+                    if (q) atomicAdd(&sh.og_eq[t], (uint32_t)__popc(q));
+                }
+            }
         }
         __syncthreads();
         carry_g = 0;
@@ -587,7 +597,6 @@ __device__ void coarse_pass(SelShared& sh, const IndexArgs& a, int r, int64_t bo
 // (coarse_pass) instead of read from the coarse scoring kernel's workspace.
 template <typename K, bool kTokens, int D_I = 0, int NT = 0>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_constant__ IndexArgs a) {
-    pdl_enter();
     extern __shared__ __align__(16) uint8_t dyn[];
     SelShared& sh = *reinterpret_cast<SelShared*>(dyn);
     const int r = blockIdx.y;
@@ -601,14 +610,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     int32_t* out = a.index_sets + (int64_t)r * a.budget;
     // Row geometry from q_len alone (clamped so every read below stays in
     // bounds), so that the slice's keys stream in while the row's sequence
-    // metadata is fetched and checked; nothing is written before the check.
-    const int n_kept_row = (kTokens && a.hi_block > 0) ? min(max(a.n_kept[r], 0), a.hi_topblocks) : 0;
+    // metadata is checked; nothing is written before the check. The metadata
+    // is the caller's, never written by a kernel of this library: it is read
+    // before the wait for the preceding kernel.
     const int Lq = a.q_len[r];
     const int seq_q = a.q_seq[r];
     const int seq_c = min(max(seq_q, 0), a.n_seq - 1);
     const int64_t off_q = a.kv_offset[seq_c];
     const int slen_q = a.seq_lens[seq_c];
     const int64_t boff_q = a.hi_block > 0 ? a.blk_offset[seq_c] : 0;
+    pdl_enter();
+    const int n_kept_row = (kTokens && a.hi_block > 0) ? min(max(a.n_kept[r], 0), a.hi_topblocks) : 0;
     const int L = min(max(Lq, 0), a.max_len);
     const int s = min(a.sink, L);
     const int ws = max(s, L - a.window);
@@ -621,8 +633,16 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
         first = s / B;
         n = ws > s ? (ws + B - 1) / B - first : 0;
     }
-    int k_lo, m;
-    slice_of(n, C, c, k_lo, m);
+    int k_lo, m, m_load;
+    if (kTokens && B > 0) {
+        // slices of the row's capacity: the keys load before the kept-block
+        // count (written by the block selection) is known
+        slice_of(a.fine_cap, C, c, k_lo, m_load);
+        m = max(0, min(n - k_lo, m_load));
+    } else {
+        slice_of(n, C, c, k_lo, m);
+        m_load = m;
+    }
     const K* row_keys = kTokens ? reinterpret_cast<const K*>(a.fine_keys + (int64_t)r * a.fine_cap)
                                 : reinterpret_cast<const K*>(a.coarse_keys + (int64_t)r * a.coarse_cap);
     Keys<K> keys{row_keys + k_lo, 0u};
@@ -645,7 +665,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     if constexpr (!kTokens && D_I > 0) {
         coarse_pass<D_I, NT>(sh, a, r, boff_q, first + k_lo, m, reinterpret_cast<uint64_t*>(stage));
     } else {
-        stage_pass<K>(sh, keys, m, stage);
+        stage_pass<K>(sh, keys, m, m_load, stage);
     }
     __syncthreads();
     if (stage != nullptr) keys.s = smem_u32(stage);
@@ -777,8 +797,6 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b, bool dense) {
         p.fine_stage = (size_t)sm * 4 + (size_t)p.kept_slots * 4 <= kStageSmem ? sm : 0;
         p.smem_tokens = sel_layout(4, p.fine_stage, p.kept_slots).bytes;
     }
-    if (hi && !topk_plan(p.coarse_cap, 8, p.tk_kp_blocks, p.tk_cl_blocks)) p.tk_kp_blocks = p.tk_cl_blocks = 0;
-    if (!topk_plan(p.fine_cap, 4, p.tk_kp_tokens, p.tk_cl_tokens)) p.tk_kp_tokens = p.tk_cl_tokens = 0;
     size_t off = 0;
     p.off_coarse = off;
     off = align256(off + (size_t)n_q * p.coarse_cap * 8);

@@ -95,9 +95,6 @@ struct IndexArgs {
 
 struct IndexPlan {
     int coarse_cap = 0, fine_cap = 0;
-    // register-held selection (index_topk.cu): keys per thread and CTAs per
-    // row, or 0 when a row's keys exceed it (the cluster kernels below)
-    int tk_kp_blocks = 0, tk_cl_blocks = 0, tk_kp_tokens = 0, tk_cl_tokens = 0;
     int cluster = 8;                          // CTAs per query row in the selection kernels
     int coarse_stage = 0, fine_stage = 0, kept_slots = 0;
     size_t smem_blocks = 0, smem_tokens = 0;  // dynamic smem of the selection kernels
@@ -129,11 +126,6 @@ inline bool coarse_in_select(int hi_block, int coarse_stage, int H_I, int n_q) {
     return hi_block > 0 && coarse_stage > 0 && H_I <= 16 && n_q >= 8;
 }
 inline bool coarse_in_select(const IndexArgs& a) { return coarse_in_select(a.hi_block, a.coarse_stage, a.H_I, a.n_q); }
-// Exact top-k with the keys of a row held by one CTA of 1024 threads (or a
-// cluster of up to 4): keys per thread and cluster size for rows of up to
-// `cap` keys of `key_bytes` bytes, false when more.
-bool topk_plan(int cap, int key_bytes, int& kp, int& cluster);
-cudaError_t launch_topk(const IndexArgs& a, bool blocks, int kp, int cluster, cudaStream_t stream);
 // Prefill chunks: exact top-k over each row's candidate pairs, SI assembly.
 cudaError_t launch_topk_pairs(const IndexArgs& a, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,

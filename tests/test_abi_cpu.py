@@ -166,13 +166,10 @@ def test_launch_counts_follow_the_shape():
 
     hi = lsa.Budget(64, 1024, 2048, 64, 256)
     flat = lsa.Budget(64, 1024, 2048, 0, 0)
-    # rows whose blocks fit one selection CTA: coarse scores, block selection,
-    # fine scores, token selection (4 launches)
-    assert lsa.lsa_index_launches(batch(16, 131072), 16, 128, hi) == 4
+    # 16 rows, 16 heads: coarse scores inside the block selection (3 launches)
+    assert lsa.lsa_index_launches(batch(16, 131072), 16, 128, hi) == 3
+    # one row: the coarse scoring kernel runs on its own (4 launches)
     assert lsa.lsa_index_launches(batch(1, 131072), 16, 128, hi) == 4
-    # blocks beyond one selection CTA's registers with 16 rows: the coarse
-    # scores run inside the cluster block selection (3 launches)
-    assert lsa.lsa_index_launches(batch(16, 1 << 20), 16, 128, lsa.Budget(64, 1024, 2048, 16, 256)) == 3
     # more than 16 indexer heads: separate coarse kernel
     assert lsa.lsa_index_launches(batch(16, 131072), 20, 128, hi) == 4
     # HI off: fine scores + token selection

@@ -82,10 +82,10 @@ def test_new_rows_are_the_newest_cached_tokens():
     assert torch.equal(st8.v_new[1][1], st8.v8[1][o + L - 2:o + L])
 
 
-@pytest.mark.parametrize("wl,n", [(wls.BATCH128K, 7), (wls.CTX1M, 7)])
+@pytest.mark.parametrize("wl,n", [(wls.BATCH128K, 6), (wls.CTX1M, 7)])
 def test_kernels_per_step(wl, n):
-    """Append, coarse scores, block selection, fine scores, token selection,
-    attention, merge."""
+    """16 rows: append, block selection with the coarse scores inside, fine scores, token
+    selection, attention, merge; one 1M row adds the separate coarse-score kernel."""
     small = wls.small(wl, lens=tuple(min(L, 4096) for L in wl.lens))
     st = _step(small)
     # the plan depends on the shape's host fields only; use the real lengths for it
