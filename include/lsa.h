@@ -343,6 +343,66 @@ lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_ca
                             int32_t *dev_status, void *stream);
 
 /* ----------------------------------------------------------------------- */
+/* Context-parallel merge                                                    */
+/* ----------------------------------------------------------------------- */
+/* When one sequence's cache is split by token range over several GPUs, each
+ * GPU keeps its own best candidates (HI blocks, then middle tokens) and the
+ * exact global choice is the best of their union: a block or token among
+ * the global top-k is among the top-k of its own shard under the same order.
+ * This call is that merge step, after the candidates of every shard have
+ * been gathered (e.g. with one all-gather). It keeps the order of the
+ * selection rules fixed at the top of this file (score descending, ties to
+ * the lower id), the HI bullet and the top-k of "LongCat-Flash-Lite-Sparse
+ * (aitrends.kr)", section "기술적 특징", and "LongCat-2.0 (molayo1419.me)",
+ * section "1M 토큰에서의 Sparse Attention 문제".
+ *
+ * pairs   device uint64 [n_rows][cap]. Entry = (key << LSA_MERGE_ID_BITS) |
+ *         (2^LSA_MERGE_ID_BITS - 1 - id) with 0 <= id < 2^LSA_MERGE_ID_BITS and
+ *         1 <= key < 2^(64 - LSA_MERGE_ID_BITS) (e.g. the score + 1); a value of 0
+ *         is an empty slot and is skipped. The entries of a row must be
+ *         distinct (distinct ids). Larger values rank first: key descending,
+ *         ties to the lower id.
+ * counts  device int32 [n_rows]: slots used in each row (outside [0, cap]: the
+ *         row is clamped and LSA_DEV_BAD_LENGTH is set).
+ * out     device int32 [n_rows][k]: the ids of the k best entries of each row,
+ *         ascending, then -1 for rows with fewer than k entries.
+ * out_values  device uint64 [n_rows][k] or NULL: the kept entries themselves,
+ *         in the order of out (0 after), e.g. for a second round of merging.
+ * Supported: 0 <= k <= LSA_MAX_BUDGET, cap >= 0, n_rows <= 65535.
+ */
+#define LSA_MERGE_ID_BITS 24
+
+/* The keys (score + 1) of given candidates, for callers that choose them
+ * (the ranks of a context-parallel index, each scoring its own token range):
+ * lsa_score_tokens gives the fine score of token positions, lsa_score_blocks
+ * the HI coarse score of blocks from their stored sums (the block sums must
+ * cover the tokens the row sees; see lsa_index for rows that see fewer).
+ *
+ * q_idx, w, w_max, H_I, d_I   as for lsa_index, n_q query rows.
+ * row_offset    device int64 [n_q]: cache row of position 0 of each query row's
+ *               sequence (lsa_score_tokens); total_tokens bounds the cache.
+ * blk_row_offset device int64 [n_q]: block-sum row of block 0 of each query
+ *               row's sequence (lsa_score_blocks); block_rows bounds block_sums.
+ * positions, blocks device int32 [n_q][n]: the candidates (-1: empty slot,
+ *               key 0). A candidate outside the cache sets LSA_DEV_BAD_INDEX
+ *               and reads as empty.
+ * keys          device uint32 [n_q][n] (tokens) or uint64 [n_q][n] (blocks).
+ */
+lsa_status_t lsa_score_tokens(const int8_t *q_idx, const int8_t *k_idx_cache, const int32_t *w,
+                              int32_t w_max, int32_t H_I, int32_t d_I, int32_t n_q,
+                              const int64_t *row_offset, int64_t total_tokens,
+                              const int32_t *positions, int32_t n, uint32_t *keys,
+                              int32_t *dev_status, void *stream);
+lsa_status_t lsa_score_blocks(const int8_t *q_idx, const int32_t *w, int32_t w_max, int32_t H_I,
+                              int32_t d_I, int32_t n_q, const int8_t *block_sums,
+                              int64_t block_rows, const int64_t *blk_row_offset,
+                              const int32_t *blocks, int32_t n, uint64_t *keys,
+                              int32_t *dev_status, void *stream);
+lsa_status_t lsa_merge_pairs(const uint64_t *pairs, const int32_t *counts, int32_t n_rows,
+                             int32_t cap, int32_t k, int32_t *out, uint64_t *out_values,
+                             int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------------------------------- */
 /* Allocation-free attention (no counterpart in the pages)                   */
 /* ----------------------------------------------------------------------- */
 /* Largest scratch lsa_attend_noalloc can use. Every GPU on which the library

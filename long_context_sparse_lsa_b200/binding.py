@@ -28,7 +28,9 @@ STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "L
 
 EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums", "lsa_append",
            "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend", "lsa_attend_fp8",
-           "lsa_attend_noalloc"]
+           "lsa_merge_pairs", "lsa_score_tokens", "lsa_score_blocks", "lsa_attend_noalloc"]
+
+MERGE_ID_BITS = 24  # LSA_MERGE_ID_BITS
 
 
 class LsaError(RuntimeError):
@@ -139,6 +141,12 @@ def load_library():
     lib.lsa_attend_fp8.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                    ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float), i32, i32, i32, vp,
                                    i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, sz, vp, vp]
+    lib.lsa_score_tokens.restype = i32
+    lib.lsa_score_tokens.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i64, vp, i32, vp, vp, vp]
+    lib.lsa_score_blocks.restype = i32
+    lib.lsa_score_blocks.argtypes = [vp, vp, i32, i32, i32, i32, vp, i64, vp, vp, i32, vp, vp, vp]
+    lib.lsa_merge_pairs.restype = i32
+    lib.lsa_merge_pairs.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp]
     lib.lsa_attend_noalloc.restype = i32
     lib.lsa_attend_noalloc.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
                                        i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, vp]
@@ -288,3 +296,58 @@ def lsa_attend_noalloc(q: list, k: list, v: list, index_sets: torch.Tensor, batc
     st = lib.lsa_attend_noalloc(qa, ka, va, H_q, H_kv, d, _ptr(index_sets), index_sets.shape[1], ctypes.byref(cb),
                                 G, oa, _ptr(dev_status), _stream(stream))
     _check("lsa_attend_noalloc", st)
+
+
+def lsa_merge_pairs(pairs: torch.Tensor, counts: torch.Tensor, k: int, out: torch.Tensor,
+                    out_values: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                    stream=None) -> None:
+    """Exact top-k of each row's packed (key, id) values (include/lsa.h):
+    pairs int64 [n_rows, cap] holding the uint64 bit patterns (0 = empty),
+    counts int32 [n_rows], out int32 [n_rows, k] (ids ascending, -1 padded),
+    out_values int64 [n_rows, k] or None (the kept entries, 0 padded)."""
+    lib = load_library()
+    if pairs.dtype != torch.int64 or counts.dtype != torch.int32 or out.dtype != torch.int32:
+        raise TypeError("pairs must be int64, counts and out int32")
+    if not (pairs.is_contiguous() and counts.is_contiguous() and out.is_contiguous()):
+        raise TypeError("pairs, counts and out must be contiguous")
+    n_rows, cap = pairs.shape
+    if counts.shape != (n_rows,) or out.shape != (n_rows, k):
+        raise ValueError("counts must be [n_rows] and out [n_rows, k]")
+    if out_values is not None and (out_values.dtype != torch.int64 or out_values.shape != (n_rows, k)
+                                   or not out_values.is_contiguous()):
+        raise TypeError("out_values must be a contiguous int64 [n_rows, k] tensor")
+    st = lib.lsa_merge_pairs(_ptr(pairs), _ptr(counts), n_rows, cap, k, _ptr(out), _ptr(out_values),
+                             _ptr(dev_status), _stream(stream))
+    _check("lsa_merge_pairs", st)
+
+
+def lsa_score_tokens(q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, w_max: int,
+                     row_offset: torch.Tensor, positions: torch.Tensor, keys: torch.Tensor,
+                     dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """Fine indexer keys (score + 1) of given positions: q_idx int8 [n_q, H_I,
+    d_I], k_idx int8 [T, d_I], w int32 [n_q, H_I], row_offset int64 [n_q],
+    positions int32 [n_q, n] (-1 empty), keys int32 [n_q, n] (uint32 bits)."""
+    lib = load_library()
+    n_q, H_I, d_I = q_idx.shape
+    n = positions.shape[1]
+    if keys.shape != (n_q, n) or keys.dtype != torch.int32 or positions.dtype != torch.int32:
+        raise TypeError("positions and keys must be int32 [n_q, n]")
+    st = lib.lsa_score_tokens(_ptr(q_idx), _ptr(k_idx), _ptr(w), w_max, H_I, d_I, n_q, _ptr(row_offset),
+                              k_idx.shape[0], _ptr(positions), n, _ptr(keys), _ptr(dev_status), _stream(stream))
+    _check("lsa_score_tokens", st)
+
+
+def lsa_score_blocks(q_idx: torch.Tensor, w: torch.Tensor, w_max: int, block_sums: torch.Tensor,
+                     blk_row_offset: torch.Tensor, blocks: torch.Tensor, keys: torch.Tensor,
+                     dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """HI coarse keys (score + 1) of given blocks: block_sums int8 [rows,
+    2*d_I] (byte planes), blk_row_offset int64 [n_q], blocks int32 [n_q, n]
+    (-1 empty), keys int64 [n_q, n] (uint64 bits)."""
+    lib = load_library()
+    n_q, H_I, d_I = q_idx.shape
+    n = blocks.shape[1]
+    if keys.shape != (n_q, n) or keys.dtype != torch.int64 or blocks.dtype != torch.int32:
+        raise TypeError("blocks must be int32 and keys int64 [n_q, n]")
+    st = lib.lsa_score_blocks(_ptr(q_idx), _ptr(w), w_max, H_I, d_I, n_q, _ptr(block_sums), block_sums.shape[0],
+                              _ptr(blk_row_offset), _ptr(blocks), n, _ptr(keys), _ptr(dev_status), _stream(stream))
+    _check("lsa_score_blocks", st)

@@ -417,6 +417,77 @@ lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache
                        workspace_bytes, dev_status, stream);
 }
 
+static lsa_status_t point_common(const int8_t* q_idx, const int32_t* w, int32_t w_max, int32_t H_I, int32_t d_I,
+                                 int32_t n_q, const int64_t* row_base, const int32_t* ids, int32_t n,
+                                 lsa::PointArgs& p) {
+    if (n_q < 0 || n < 0 || H_I < 1 || d_I < 1 || w_max < 0) return LSA_ERR_INVALID_ARG;
+    if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
+    if (H_I > LSA_MAX_HEADS_I || n_q > 65535) return LSA_ERR_UNSUPPORTED;
+    if ((double)H_I * (double)w_max * (double)d_I * 16384.0 >= 2147483648.0) return LSA_ERR_UNSUPPORTED;
+    if (n_q == 0 || n == 0) return LSA_OK;
+    if (q_idx == nullptr || w == nullptr || row_base == nullptr || ids == nullptr) return LSA_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(row_base, 8) || !aligned(ids, 4))
+        return LSA_ERR_INVALID_ARG;
+    std::memset(&p, 0, sizeof p);
+    p.a.q_idx = q_idx;
+    p.a.w = w;
+    p.a.w_max = w_max;
+    p.a.H_I = H_I;
+    p.a.n_q = n_q;
+    p.ids = ids;
+    p.row_base = row_base;
+    p.n = n;
+    return LSA_OK;
+}
+
+lsa_status_t lsa_score_tokens(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max,
+                              int32_t H_I, int32_t d_I, int32_t n_q, const int64_t* row_offset, int64_t total_tokens,
+                              const int32_t* positions, int32_t n, uint32_t* keys, int32_t* dev_status,
+                              void* stream) {
+    lsa::PointArgs p;
+    lsa_status_t st = point_common(q_idx, w, w_max, H_I, d_I, n_q, row_offset, positions, n, p);
+    if (st != LSA_OK || n_q == 0 || n == 0) return st;
+    if (k_idx_cache == nullptr || keys == nullptr || total_tokens < 0) return LSA_ERR_INVALID_ARG;
+    if (!aligned(k_idx_cache, 16) || !aligned(keys, 4)) return LSA_ERR_INVALID_ARG;
+    p.a.k_idx = k_idx_cache;
+    p.a.dev_status = dev_status;
+    p.rows = total_tokens;
+    p.out_tokens = keys;
+    p.blocks = 0;
+    cudaError_t e = lsa::launch_point_scores(p, d_I, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+lsa_status_t lsa_score_blocks(const int8_t* q_idx, const int32_t* w, int32_t w_max, int32_t H_I, int32_t d_I,
+                              int32_t n_q, const int8_t* block_sums, int64_t block_rows, const int64_t* blk_row_offset,
+                              const int32_t* blocks, int32_t n, uint64_t* keys, int32_t* dev_status, void* stream) {
+    lsa::PointArgs p;
+    lsa_status_t st = point_common(q_idx, w, w_max, H_I, d_I, n_q, blk_row_offset, blocks, n, p);
+    if (st != LSA_OK || n_q == 0 || n == 0) return st;
+    if (block_sums == nullptr || keys == nullptr || block_rows < 0) return LSA_ERR_INVALID_ARG;
+    if (!aligned(block_sums, 16) || !aligned(keys, 8)) return LSA_ERR_INVALID_ARG;
+    p.a.block_sums = block_sums;
+    p.a.dev_status = dev_status;
+    p.rows = block_rows;
+    p.out_blocks = keys;
+    p.blocks = 1;
+    cudaError_t e = lsa::launch_point_scores(p, d_I, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+lsa_status_t lsa_merge_pairs(const uint64_t* pairs, const int32_t* counts, int32_t n_rows, int32_t cap, int32_t k,
+                             int32_t* out, uint64_t* out_values, int32_t* dev_status, void* stream) {
+    if (n_rows < 0 || cap < 0 || k < 0) return LSA_ERR_INVALID_ARG;
+    if (k > LSA_MAX_BUDGET || n_rows > 65535) return LSA_ERR_UNSUPPORTED;
+    if (n_rows == 0 || k == 0) return LSA_OK;
+    if (pairs == nullptr || counts == nullptr || out == nullptr) return LSA_ERR_INVALID_ARG;
+    if (!aligned(pairs, 16) || !aligned(counts, 4) || !aligned(out, 4)) return LSA_ERR_INVALID_ARG;
+    if (out_values != nullptr && !aligned(out_values, 8)) return LSA_ERR_INVALID_ARG;
+    cudaError_t e = lsa::launch_merge_pairs(pairs, counts, n_rows, cap, k, out, out_values, dev_status,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
 lsa_status_t lsa_attend_fp8(const uint16_t* const* q, const uint8_t* const* k_cache, const uint8_t* const* v_cache,
                             const float* k_scale, const float* v_scale, int32_t H_q, int32_t H_kv, int32_t d,
                             const int32_t* index_sets, int32_t budget, const lsa_batch_t* batch,

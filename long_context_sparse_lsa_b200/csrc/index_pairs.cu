@@ -19,6 +19,8 @@ constexpr int kTkWarps = kTkThreads / kWarp;
 static_assert(kHistBins / kTkThreads == 4, "the scan gives each thread one 4-bin vector");
 constexpr int kTkCandCap = 2048;  // keys of the threshold bin held in the candidate list
 constexpr int kTkDigitBits = 12;
+constexpr int kMergeIdBits = LSA_MERGE_ID_BITS;  // id field of a merge value
+constexpr uint32_t kMergeIdMask = (1u << kMergeIdBits) - 1u;
 
 __device__ __forceinline__ uint32_t tk_warp_sum(uint32_t v) {
 #pragma unroll
@@ -86,6 +88,102 @@ __device__ uint32_t pair_find_bin(PairShared& sh, uint32_t krem) {
     return total;
 }
 
+// The k largest of the distinct values value(e) over the pairs that
+// for_each_pair presents (n of them), their ids id(e) left sorted ascending in
+// sel[0, m); returns m (= k when n >= k, else n). A histogram pass on the
+// logarithmic scale of key_bin, then radix digits over the threshold bin's
+// candidates (or, for a bin too full for the list, over all pairs), then a
+// pass collecting the kept ids and a bitonic sort in shared memory. Every
+// thread of the CTA calls it.
+template <typename ForEach, typename Value, typename Id>
+__device__ uint32_t select_sorted(PairShared& sh, int32_t* sel, uint32_t n, uint32_t k, ForEach for_each_pair,
+                                  Value value, Id id) {
+    const int tid = threadIdx.x;
+    if (k == 0u) return 0u;
+    // the k largest values: value >= T
+    uint64_t T = 0ull;
+    if (n > k) {
+        for (int i = tid; i < kHistBins; i += kTkThreads) sh.hist[i] = 0u;
+        if (tid == 0) sh.n_cand = 0u;
+        __syncthreads();
+        for_each_pair([&](uint64_t e, bool ok) {
+            if (ok) atomicAdd(&sh.hist[key_bin(value(e))], 1u);
+        });
+        __syncthreads();
+        pair_find_bin(sh, k);
+        const uint32_t tb = sh.bin, in_bin = sh.in_bin;
+        uint32_t kr = k - sh.above;
+        const int nb = (int)(tb >> 6) + 6;
+        int shift = tb < 64u ? 0 : nb - 7;
+        uint64_t prefix = tb < 64u ? (uint64_t)tb : (uint64_t)(64u | (tb & 63u));
+        const bool listed = in_bin <= (uint32_t)kTkCandCap;
+        if (listed) {
+            __syncthreads();
+            for_each_pair([&](uint64_t e, bool ok) {
+                const uint64_t v = value(e);
+                const bool take = ok && key_bin(v) == tb;
+                const uint32_t p = warp_append(&sh.n_cand, take);
+                if (take && p < (uint32_t)kTkCandCap) sh.cand[p] = v;
+            });
+            __syncthreads();
+        }
+        const uint32_t nc = min(sh.n_cand, (uint32_t)kTkCandCap);
+        while (shift > 0) {
+            const int width = shift < kTkDigitBits ? shift : kTkDigitBits;
+            shift -= width;
+            const uint64_t mask = (1ull << width) - 1ull;
+            reinterpret_cast<uint4*>(sh.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+            __syncthreads();
+            if (listed) {
+                for (uint32_t i = tid; i < nc; i += kTkThreads) {
+                    const uint64_t v = sh.cand[i];
+                    if ((v >> (shift + width)) == prefix) atomicAdd(&sh.hist[(uint32_t)((v >> shift) & mask)], 1u);
+                }
+            } else {
+                for_each_pair([&](uint64_t e, bool ok) {
+                    const uint64_t v = value(e);
+                    if (ok && (v >> (shift + width)) == prefix) atomicAdd(&sh.hist[(uint32_t)((v >> shift) & mask)], 1u);
+                });
+            }
+            __syncthreads();
+            pair_find_bin(sh, kr);
+            prefix = (prefix << width) | sh.bin;
+            kr -= sh.above;
+        }
+        T = prefix;  // values are distinct: exactly k are >= T
+    }
+    // the kept positions, then sorted ascending
+    if (tid == 0) sh.n_sel = 0u;
+    __syncthreads();
+    for_each_pair([&](uint64_t e, bool ok) {
+        const bool take = ok && value(e) >= T;
+        const uint32_t p = warp_append(&sh.n_sel, take);
+        if (take && p < (uint32_t)kPairSortCap) sel[p] = id(e);
+    });
+    __syncthreads();
+    const uint32_t m = min(sh.n_sel, k);
+    uint32_t P = 1;
+    while (P < m) P <<= 1;
+    for (uint32_t i = m + tid; i < P; i += kTkThreads) sel[i] = 0x7fffffff;
+    __syncthreads();
+    for (uint32_t size = 2; size <= P; size <<= 1) {
+        for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
+            for (uint32_t i = tid; i < P / 2; i += kTkThreads) {
+                const uint32_t lo = 2 * i - (i & (stride - 1));  // index with bit `stride` clear
+                const uint32_t hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const int32_t x = sel[lo], y = sel[hi];
+                if ((x > y) == up) {
+                    sel[lo] = y;
+                    sel[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    return m;
+}
+
 __global__ void __launch_bounds__(kTkThreads, 1) topk_pairs_kernel(const __grid_constant__ IndexArgs a) {
     extern __shared__ __align__(16) uint8_t pr_dyn[];
     PairShared& sh = *reinterpret_cast<PairShared*>(pr_dyn);
@@ -149,94 +247,94 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_pairs_kernel(const __grid_
         }
     }
     if (k == 0u) return;
-    // the k largest values: value >= T
-    uint64_t T = 0ull;
-    if (n > k) {
-        for (int i = tid; i < kHistBins; i += kTkThreads) sh.hist[i] = 0u;
-        if (tid == 0) sh.n_cand = 0u;
-        __syncthreads();
-        for_each_pair([&](uint64_t e, bool ok) {
-            if (ok) atomicAdd(&sh.hist[key_bin(pair_value(e))], 1u);
-        });
-        __syncthreads();
-        pair_find_bin(sh, k);
-        const uint32_t tb = sh.bin, in_bin = sh.in_bin;
-        uint32_t kr = k - sh.above;
-        const int nb = (int)(tb >> 6) + 6;
-        int shift = tb < 64u ? 0 : nb - 7;
-        uint64_t prefix = tb < 64u ? (uint64_t)tb : (uint64_t)(64u | (tb & 63u));
-        const bool listed = in_bin <= (uint32_t)kTkCandCap;
-        if (listed) {
-            __syncthreads();
-            for_each_pair([&](uint64_t e, bool ok) {
-                const uint64_t v = pair_value(e);
-                const bool take = ok && key_bin(v) == tb;
-                const uint32_t p = warp_append(&sh.n_cand, take);
-                if (take && p < (uint32_t)kTkCandCap) sh.cand[p] = v;
-            });
-            __syncthreads();
-        }
-        const uint32_t nc = min(sh.n_cand, (uint32_t)kTkCandCap);
-        while (shift > 0) {
-            const int width = shift < kTkDigitBits ? shift : kTkDigitBits;
-            shift -= width;
-            const uint64_t mask = (1ull << width) - 1ull;
-            reinterpret_cast<uint4*>(sh.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
-            __syncthreads();
-            if (listed) {
-                for (uint32_t i = tid; i < nc; i += kTkThreads) {
-                    const uint64_t v = sh.cand[i];
-                    if ((v >> (shift + width)) == prefix) atomicAdd(&sh.hist[(uint32_t)((v >> shift) & mask)], 1u);
-                }
-            } else {
-                for_each_pair([&](uint64_t e, bool ok) {
-                    const uint64_t v = pair_value(e);
-                    if (ok && (v >> (shift + width)) == prefix) atomicAdd(&sh.hist[(uint32_t)((v >> shift) & mask)], 1u);
-                });
-            }
-            __syncthreads();
-            pair_find_bin(sh, kr);
-            prefix = (prefix << width) | sh.bin;
-            kr -= sh.above;
-        }
-        T = prefix;  // values are distinct: exactly k are >= T
-    }
-    // the kept positions, then sorted ascending
-    if (tid == 0) sh.n_sel = 0u;
-    __syncthreads();
-    for_each_pair([&](uint64_t e, bool ok) {
-        const bool take = ok && pair_value(e) >= T;
-        const uint32_t p = warp_append(&sh.n_sel, take);
-        if (take && p < (uint32_t)kPairSortCap) sel[p] = (int32_t)(uint32_t)e;
-    });
-    __syncthreads();
-    const uint32_t m = min(sh.n_sel, k);
-    uint32_t P = 1;
-    while (P < m) P <<= 1;
-    for (uint32_t i = m + tid; i < P; i += kTkThreads) sel[i] = 0x7fffffff;
-    __syncthreads();
-    for (uint32_t size = 2; size <= P; size <<= 1) {
-        for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
-            for (uint32_t i = tid; i < P / 2; i += kTkThreads) {
-                const uint32_t lo = 2 * i - (i & (stride - 1));  // index with bit `stride` clear
-                const uint32_t hi = lo + stride;
-                const bool up = (lo & size) == 0;
-                const int32_t x = sel[lo], y = sel[hi];
-                if ((x > y) == up) {
-                    sel[lo] = y;
-                    sel[hi] = x;
-                }
-            }
-            __syncthreads();
-        }
-    }
+    const uint32_t m = select_sorted(sh, sel, n, k, for_each_pair, [](uint64_t e) { return pair_value(e); },
+                                     [](uint64_t e) { return (int32_t)(uint32_t)e; });
     pdl_trigger();
     for (uint32_t i = tid; i < m; i += kTkThreads) out[s + i] = sel[i];
+}
+
+
+// Context-parallel merge: row r's pairs [r][0, counts[r]) hold values
+// score << kMergeIdBits | (2^kMergeIdBits - 1 - id), distinct per row, or 0
+// for an empty slot; the ids of the k largest values (score desc, id asc) are
+// written ascending to out[r][0, m), -1 after, and (out_values) their values
+// in the same order, 0 after.
+__global__ void __launch_bounds__(kTkThreads, 1) merge_pairs_kernel(const uint64_t* __restrict__ pairs,
+                                                                    const int32_t* __restrict__ counts, int32_t cap,
+                                                                    int32_t k, int32_t* __restrict__ out,
+                                                                    uint64_t* __restrict__ out_values,
+                                                                    int32_t* dev_status) {
+    extern __shared__ __align__(16) uint8_t pr_dyn[];
+    PairShared& sh = *reinterpret_cast<PairShared*>(pr_dyn);
+    int32_t* sel = reinterpret_cast<int32_t*>(pr_dyn + (sizeof(PairShared) + 15) / 16 * 16);
+    const int r = blockIdx.x, tid = threadIdx.x;
+    pdl_enter();
+    const int cnt_raw = counts[r];
+    if (cnt_raw < 0 || cnt_raw > cap) {
+        if (tid == 0) flag(dev_status, LSA_DEV_BAD_LENGTH);
+    }
+    const int cnt = min(max(cnt_raw, 0), cap);
+    const uint64_t* row = pairs + (int64_t)r * cap;
+    auto for_each_pair = [&](auto&& f) {
+        for (int i0 = tid - (tid & 31); i0 < cnt; i0 += kTkThreads) {
+            const int i = i0 + (tid & 31);
+            const uint64_t e = i < cnt ? __ldcg(row + i) : 0ull;
+            f(e, e != 0ull);
+        }
+    };
+    // the row's entries (nonzero values)
+    if (tid == 0) sh.n_cand = 0u;
+    __syncthreads();
+    for_each_pair([&](uint64_t e, bool ok) {
+        const uint32_t c = (uint32_t)__popc(__ballot_sync(0xffffffffu, ok));
+        if ((tid & 31) == 0 && c) atomicAdd(&sh.n_cand, c);
+    });
+    __syncthreads();
+    const uint32_t n = sh.n_cand;
+    __syncthreads();
+    const uint32_t m = select_sorted(sh, sel, n, (uint32_t)k, for_each_pair, [](uint64_t e) { return e; },
+                                     [](uint64_t e) {
+                                         return (int32_t)((kMergeIdMask - (uint32_t)(e & kMergeIdMask)));
+                                     });
+    pdl_trigger();
+    int32_t* o = out + (int64_t)r * k;
+    for (int i = tid; i < k; i += kTkThreads) o[i] = i < (int)m ? sel[i] : -1;
+    if (out_values != nullptr) {
+        // each kept id's value, found again among the row's entries
+        uint64_t* ov = out_values + (int64_t)r * k;
+        for (int i = tid; i < k; i += kTkThreads)
+            if (i >= (int)m) ov[i] = 0ull;
+        for_each_pair([&](uint64_t e, bool ok) {
+            if (!ok) return;
+            const int32_t id = (int32_t)(kMergeIdMask - (uint32_t)(e & kMergeIdMask));
+            // binary search of id in the sorted ids
+            int lo = 0, hi = (int)m - 1;
+            while (lo <= hi) {
+                const int mid = (lo + hi) >> 1;
+                const int32_t x = sel[mid];
+                if (x == id) {
+                    ov[mid] = e;
+                    break;
+                }
+                if (x < id) lo = mid + 1;
+                else hi = mid - 1;
+            }
+        });
+    }
 }
 
 }  // namespace
 
 size_t topk_pairs_smem() { return (sizeof(PairShared) + 15) / 16 * 16 + (size_t)kPairSortCap * 4; }
+
+cudaError_t launch_merge_pairs(const uint64_t* pairs, const int32_t* counts, int n_rows, int cap, int k, int32_t* out,
+                               uint64_t* out_values, int32_t* dev_status, cudaStream_t stream) {
+    const size_t smem = topk_pairs_smem();
+    cudaError_t e = cudaFuncSetAttribute(merge_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(merge_pairs_kernel, dim3((unsigned)n_rows), dim3(kTkThreads), smem, stream, 0, pairs, counts,
+                      cap, k, out, out_values, dev_status);
+}
 
 cudaError_t launch_topk_pairs(const IndexArgs& a, cudaStream_t stream) {
     const size_t smem = topk_pairs_smem();

@@ -128,8 +128,26 @@ inline bool coarse_in_select(int hi_block, int coarse_stage, int H_I, int n_q) {
 inline bool coarse_in_select(const IndexArgs& a) { return coarse_in_select(a.hi_block, a.coarse_stage, a.H_I, a.n_q); }
 // Prefill chunks: exact top-k over each row's candidate pairs, SI assembly.
 cudaError_t launch_topk_pairs(const IndexArgs& a, cudaStream_t stream);
+// Context-parallel merge of (score, id) values (lsa_merge_pairs).
+cudaError_t launch_merge_pairs(const uint64_t* pairs, const int32_t* counts, int n_rows, int cap, int k, int32_t* out,
+                               uint64_t* out_values, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
                                 cudaStream_t stream);
+
+// Indexer scores of given token positions or HI blocks (lsa_score_tokens,
+// lsa_score_blocks): q_idx, k_idx, w, w_max, H_I, n_q, block_sums and
+// dev_status of `a` are used.
+struct PointArgs {
+    IndexArgs a;
+    const int32_t* ids;       // [n_q][n] positions or block indices (-1: empty slot)
+    const int64_t* row_base;  // [n_q] first cache row / block-sum row of each query row's sequence
+    int64_t rows;             // rows of the key cache / block-sum cache
+    uint32_t* out_tokens;     // [n_q][n]
+    uint64_t* out_blocks;     // [n_q][n]
+    int32_t n;
+    int32_t blocks;
+};
+cudaError_t launch_point_scores(const PointArgs& p, int d_I, cudaStream_t stream);
 
 // ---- sparse attention -----------------------------------------------------
 struct AttendArgs {
