@@ -452,14 +452,14 @@ def job_rate(units_per_rank: int, world: int, ms: float) -> float:
 
 
 # ---------------------------------------------------------------------------
-def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, kv_fp8=False):
+def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, kv_fp8=False, grouped=False):
     """Draws the workload, captures its step graphs and times `steps` steps
     (after `warmup`), each after an L2 flush: the whole step graph for the
     headline, then the three calls one by one for the breakdown."""
     from long_context_sparse_lsa_b200.pipeline import LsaStep
 
     t = wls.make(wl, dev, with_kv=not kv_fp8)
-    st = LsaStep(wl, t, dev, kv_fp8=kv_fp8)
+    st = LsaStep(wl, t, dev, kv_fp8=kv_fp8, grouped=grouped)
     st.pack_io()  # one input and one output buffer per step (the e2e leg copies each once)
     st.build_block_sums()
     torch.cuda.synchronize()
@@ -545,6 +545,15 @@ def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, k
             "ix_in_step": [c["index"] for c in in_step], "at_in_step": [c["attend"] for c in in_step]}
 
 
+def draft_union_entries(sets: torch.Tensor, drafts: int) -> int:
+    """Distinct positions over each sequence's draft rows, summed (the K/V rows
+    the grouped attention gathers per kv head and layer)."""
+    total = 0
+    for grp in sets.view(-1, drafts * sets.shape[1]):
+        total += int(torch.unique(grp[grp >= 0]).numel())
+    return total
+
+
 def cold_line(wl, cold_ms, world, pg, dev):
     """The cold-step numbers (block sums rebuilt inside every step), or None
     when the workload has HI off."""
@@ -569,11 +578,20 @@ def secondary(dev, flush, stream, steps, warmup, peak):
         int8 = measure_int8_peak(dev)
     except Exception as exc:  # reported, never silently replaced by an assumed figure
         int8 = {"tops": None, "kind": f"int8 GEMM unavailable: {exc!r}"}
-    for wl, fp8 in ((wls.CTX1M, False), (wls.PREFILL, False), (wls.BATCH128K, True), (wls.ragged(), False)):
-        run = time_workload(wl, dev, flush, stream, steps, warmup, kv_fp8=fp8)
+    for wl, fp8 in ((wls.CTX1M, False), (wls.PREFILL, False), (wls.BATCH128K, True), (wls.ragged(), False),
+                    (wls.DRAFTS128K, False)):
+        grouped = wl.drafts > 1
+        run = time_workload(wl, dev, flush, stream, steps, warmup, kv_fp8=fp8, grouped=grouped)
         st = run["st"]
         ms = run["ms"]
         byts = step_bytes(wl, kv_fp8=fp8)
+        if grouped:
+            # the grouped attention reads each sequence's union of K/V rows once
+            union = draft_union_entries(st.sets, wl.drafts)
+            kv_row = wl.H_kv * wl.d * 2
+            byts = dict(byts)
+            byts["attend"] = wl.G * (2 * union * kv_row + wl.n_q * (wl.H_q * wl.d * 6 + wl.budget * 4))
+            byts["total"] = byts["attend"] + byts["index"] + byts["append"]
         ix, at = mean(run["ix_in_step"]), mean(run["at_in_step"])
         rec = {"ms_per_step": ms, "steps": steps, "warmup": warmup,
                "step_breakdown_ms": {"append": mean(run["bs"]), "index": mean(run["ix"]),
@@ -617,6 +635,22 @@ def secondary(dev, flush, stream, steps, warmup, peak):
                         "value": wl.n_q / (ms / 1000.0), "kv_cache": "fp8 e4m3, one scale per layer for K and V",
                         "note": "same workload as the headline with the K/V caches held as FP8 codes "
                                 "(lsa_attend_fp8); attention bytes per query halve"})
+        elif grouped:
+            # the same step with every row gathering its own set, for comparison
+            plain = time_workload(wl, dev, flush, stream, steps, warmup)
+            per_entry = wl.H_kv * 2 * wl.d * 2 * wl.G  # K and V of every kv head, every layer
+            rec.update({"metric": "LSA decode queries/s, draft rows sharing one gather", "unit": "queries/s",
+                        "value": wl.n_q / (ms / 1000.0), "drafts_per_seq": wl.drafts,
+                        "draft_query_share_pct": wl.draft_share,
+                        "set_entries": int((st.sets >= 0).sum().item()), "union_entries": union,
+                        "kv_bytes_gathered_grouped": union * per_entry,
+                        "kv_bytes_gathered_per_row": int((st.sets >= 0).sum().item()) * per_entry,
+                        "per_row_gather": {"ms_per_step": plain["ms"], "value": wl.n_q / (plain["ms"] / 1000.0),
+                                           "attend_ms_in_step": mean(plain["at_in_step"]),
+                                           "gpu_launches_per_step": plain["n_kernels"]},
+                        "note": "lsa_attend_grouped: each sequence's draft rows gather the union of their sets once; "
+                                "per_row_gather is the same step with lsa_attend (every row its own set)"})
+            del plain
         elif wl.name == wls.CTX1M.name:
             rec.update({"metric": "LSA decode queries/s at 1M ctx", "unit": "queries/s",
                         "value": wl.n_q / (ms / 1000.0), "layers_per_index": wl.G})

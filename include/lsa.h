@@ -343,6 +343,50 @@ lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_ca
                             int32_t *dev_status, void *stream);
 
 /* ----------------------------------------------------------------------- */
+/* Draft rows sharing one gather                                             */
+/* ----------------------------------------------------------------------- */
+/* A decode step that verifies several draft tokens of a sequence at once
+ * (multi-token prediction for speculative decoding, "LongCat-2.0
+ * (molayo1419.me)", section "1M 토큰에서의 Sparse Attention 문제") has one
+ * decode row per draft token. Their index sets share the sink run, nearly all
+ * of the window run and, where the drafts' indexer queries agree, much of
+ * the selection.
+ *
+ * lsa_attend_grouped computes exactly what lsa_attend computes for the same
+ * arguments, for batches whose rows come in groups of group_rows consecutive
+ * rows of one sequence (row g * group_rows + j is draft j of group g, as the
+ * decode rows of lsa_batch_t with several rows per sequence are laid out):
+ * the sets of each group are merged into one ascending union with a mask of
+ * the rows holding each position, each K/V row of the union is gathered once
+ * per group and kv head, and every row attends over its own entries. Each
+ * row's set is taken as a set: an entry repeated within one row counts once
+ * (lsa_index never repeats one).
+ *
+ * Arguments, output and device-side errors as lsa_attend, plus
+ * group_rows  1, 2, 4 or 8; n_q must be a multiple of it. A group whose rows
+ *             name different sequences sets LSA_DEV_BAD_SEQ and its output is
+ *             zero.
+ * workspace   lsa_attend_grouped_workspace_size() bytes (split partials and
+ *             the unions; no initialisation needed).
+ * Supported: the shapes lsa_attend supports with H_q / H_kv <= 8, bf16
+ * caches, and group_rows * (8192 + 4 * budget) <= 227 KiB (the union's
+ * shared memory); n_q / group_rows <= 65535. Three launches (union,
+ * attention, split merge) or two with one split.
+ */
+size_t lsa_attend_grouped_workspace_size(const lsa_batch_t *batch, int32_t H_q, int32_t H_kv,
+                                         int32_t d, int32_t budget, int32_t layers_per_index,
+                                         int32_t group_rows);
+int32_t lsa_attend_grouped_launches(const lsa_batch_t *batch, int32_t H_q, int32_t H_kv,
+                                    int32_t d, int32_t budget, int32_t layers_per_index,
+                                    int32_t group_rows);
+lsa_status_t lsa_attend_grouped(const uint16_t *const *q, const uint16_t *const *k_cache,
+                                const uint16_t *const *v_cache, int32_t H_q, int32_t H_kv,
+                                int32_t d, const int32_t *index_sets, int32_t budget,
+                                const lsa_batch_t *batch, int32_t layers_per_index,
+                                int32_t group_rows, float *const *out, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------------------------------- */
 /* Context-parallel merge                                                    */
 /* ----------------------------------------------------------------------- */
 /* When one sequence's cache is split by token range over several GPUs, each
@@ -401,6 +445,57 @@ lsa_status_t lsa_score_blocks(const int8_t *q_idx, const int32_t *w, int32_t w_m
 lsa_status_t lsa_merge_pairs(const uint64_t *pairs, const int32_t *counts, int32_t n_rows,
                              int32_t cap, int32_t k, int32_t *out, uint64_t *out_values,
                              int32_t *dev_status, void *stream);
+
+/* Context-parallel attention: each GPU attends over the entries of the set
+ * that fall in its token range and returns its partial as the normalised
+ * output plus the log of the softmax denominator; the exact attention over
+ * the whole set is the log-sum-exp combination of the partials. This is the
+ * softmax attention over the selected rows of "LongCat-2.0 (molayo1419.me)",
+ * section "1M 토큰에서의 Sparse Attention 문제", split by rows of the cache
+ * instead of by entries of the set; the arithmetic is lsa_attend's.
+ *
+ * lsa_attend_lse is lsa_attend that also writes, for every layer g, row r
+ * and query head h,
+ *   lse[g][r][h] = ln( sum_j exp(q . k_j / sqrt(d)) )
+ * over the row's entries (-INFINITY for a row with no entry, or an invalid
+ * row, whose output is zero as for lsa_attend).
+ * lse   host [G] array of device fp32 [n_q][H_q].
+ * Every other argument, the workspace and the device-side errors are
+ * lsa_attend's.
+ */
+lsa_status_t lsa_attend_lse(const uint16_t *const *q, const uint16_t *const *k_cache,
+                            const uint16_t *const *v_cache, int32_t H_q, int32_t H_kv, int32_t d,
+                            const int32_t *index_sets, int32_t budget,
+                            const lsa_batch_t *batch, int32_t layers_per_index,
+                            float *const *out, float *const *lse, void *workspace,
+                            size_t workspace_bytes, int32_t *dev_status, void *stream);
+
+/* The part of each row's index set that one GPU holds: the entries e with
+ * lo <= e < hi, as e - lo, in the set's order, then -1 up to the budget.
+ *
+ * index_sets  device int32 [n_q][budget] (positions relative to the sequence
+ *             start, -1 padded, e.g. from lsa_index).
+ * local_sets  device int32 [n_q][budget] output (may not alias index_sets).
+ * lo, hi      host: the GPU's token range of the sequence, 0 <= lo <= hi.
+ * An entry below -1 sets LSA_DEV_BAD_INDEX in dev_status and is dropped.
+ * Supported: budget <= LSA_MAX_BUDGET, n_q <= 65535.
+ */
+lsa_status_t lsa_shard_sets(const int32_t *index_sets, int32_t n_q, int32_t budget, int32_t lo,
+                            int32_t hi, int32_t *local_sets, int32_t *dev_status, void *stream);
+
+/* The exact combination of n_parts attention partials of the same rows:
+ *   M      = max_p lse[p][i]
+ *   out[i] = sum_p exp(lse[p][i] - M) * o[p][i] / sum_p exp(lse[p][i] - M)
+ *   lse_out[i] = M + ln(sum_p exp(lse[p][i] - M))
+ * (zeros and -INFINITY when every part of row i is empty).
+ *
+ * o_parts    device fp32 [n_parts][rows][d]: each part's normalised output.
+ * lse_parts  device fp32 [n_parts][rows]: each part's lse (-INFINITY: empty).
+ * out        device fp32 [rows][d]; lse_out device fp32 [rows] or NULL.
+ * Supported: d % 4 == 0, 1 <= n_parts <= 65535.
+ */
+lsa_status_t lsa_combine(const float *o_parts, const float *lse_parts, int32_t n_parts, int64_t rows,
+                         int32_t d, float *out, float *lse_out, void *stream);
 
 /* ----------------------------------------------------------------------- */
 /* Allocation-free attention (no counterpart in the pages)                   */

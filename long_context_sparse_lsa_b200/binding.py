@@ -28,7 +28,9 @@ STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "L
 
 EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_block_sums", "lsa_append",
            "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend", "lsa_attend_fp8",
-           "lsa_merge_pairs", "lsa_score_tokens", "lsa_score_blocks", "lsa_attend_noalloc"]
+           "lsa_merge_pairs", "lsa_score_tokens", "lsa_score_blocks", "lsa_attend_lse", "lsa_shard_sets",
+           "lsa_combine", "lsa_attend_grouped_workspace_size", "lsa_attend_grouped_launches", "lsa_attend_grouped",
+           "lsa_attend_noalloc"]
 
 MERGE_ID_BITS = 24  # LSA_MERGE_ID_BITS
 
@@ -147,6 +149,20 @@ def load_library():
     lib.lsa_score_blocks.argtypes = [vp, vp, i32, i32, i32, i32, vp, i64, vp, vp, i32, vp, vp, vp]
     lib.lsa_merge_pairs.restype = i32
     lib.lsa_merge_pairs.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp]
+    lib.lsa_attend_lse.restype = i32
+    lib.lsa_attend_lse.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp, i32,
+                                   ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, sz, vp, vp]
+    lib.lsa_shard_sets.restype = i32
+    lib.lsa_shard_sets.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+    lib.lsa_combine.restype = i32
+    lib.lsa_combine.argtypes = [vp, vp, i32, i64, i32, vp, vp, vp]
+    lib.lsa_attend_grouped_workspace_size.restype = sz
+    lib.lsa_attend_grouped_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, i32, i32, i32, i32]
+    lib.lsa_attend_grouped_launches.restype = i32
+    lib.lsa_attend_grouped_launches.argtypes = [ctypes.POINTER(_Batch), i32, i32, i32, i32, i32, i32]
+    lib.lsa_attend_grouped.restype = i32
+    lib.lsa_attend_grouped.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
+                                       i32, ctypes.POINTER(_Batch), i32, i32, ctypes.POINTER(vp), vp, sz, vp, vp]
     lib.lsa_attend_noalloc.restype = i32
     lib.lsa_attend_noalloc.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
                                        i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, vp]
@@ -260,6 +276,90 @@ def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch
                         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
                         _stream(stream))
     _check("lsa_attend", st)
+
+
+def lsa_attend_grouped_workspace_size(batch: Batch, H_q: int, H_kv: int, d: int, budget: int, layers: int,
+                                      group_rows: int) -> int:
+    return load_library().lsa_attend_grouped_workspace_size(ctypes.byref(batch.c()), H_q, H_kv, d, budget, layers,
+                                                            group_rows)
+
+
+def lsa_attend_grouped_launches(batch: Batch, H_q: int, H_kv: int, d: int, budget: int, layers: int,
+                                group_rows: int) -> int:
+    return load_library().lsa_attend_grouped_launches(ctypes.byref(batch.c()), H_q, H_kv, d, budget, layers,
+                                                      group_rows)
+
+
+def lsa_attend_grouped(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, group_rows: int,
+                       out: list, workspace: torch.Tensor, dev_status: torch.Tensor | None = None,
+                       stream=None) -> None:
+    """lsa_attend for rows in groups of group_rows draft rows of one sequence:
+    each group's sets are gathered once as their union."""
+    lib = load_library()
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k[0].shape[1]
+    arr = ctypes.c_void_p * G
+    qa, ka, va, oa = (arr(*[t.data_ptr() for t in x]) for x in (q, k, v, out))
+    cb = batch.c()
+    st = lib.lsa_attend_grouped(qa, ka, va, H_q, H_kv, d, _ptr(index_sets), index_sets.shape[1], ctypes.byref(cb),
+                                G, group_rows, oa, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(dev_status), _stream(stream))
+    _check("lsa_attend_grouped", st)
+
+
+def lsa_attend_lse(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list, lse: list,
+                   workspace: torch.Tensor, dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """lsa_attend that also writes lse[g] (fp32 [n_q, H_q]): the log of each
+    row and head's softmax denominator (-inf for an empty set)."""
+    lib = load_library()
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k[0].shape[1]
+    for t in lse:
+        if t.dtype != torch.float32 or t.shape != (n_q, H_q) or not t.is_contiguous():
+            raise TypeError("lse must hold contiguous float32 [n_q, H_q] tensors")
+    arr = ctypes.c_void_p * G
+    qa, ka, va, oa, la = (arr(*[t.data_ptr() for t in x]) for x in (q, k, v, out, lse))
+    cb = batch.c()
+    st = lib.lsa_attend_lse(qa, ka, va, H_q, H_kv, d, _ptr(index_sets), index_sets.shape[1], ctypes.byref(cb), G, oa,
+                            la, _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                            _stream(stream))
+    _check("lsa_attend_lse", st)
+
+
+def lsa_shard_sets(index_sets: torch.Tensor, lo: int, hi: int, local_sets: torch.Tensor,
+                   dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """The entries of each row's set inside [lo, hi), as e - lo in set order,
+    -1 after (int32 [n_q, budget] in and out)."""
+    lib = load_library()
+    if index_sets.dtype != torch.int32 or local_sets.dtype != torch.int32:
+        raise TypeError("index sets must be int32")
+    if local_sets.shape != index_sets.shape or not (index_sets.is_contiguous() and local_sets.is_contiguous()):
+        raise TypeError("local_sets must be a contiguous tensor shaped like index_sets")
+    n_q, budget = index_sets.shape
+    st = lib.lsa_shard_sets(_ptr(index_sets), n_q, budget, int(lo), int(hi), _ptr(local_sets), _ptr(dev_status),
+                            _stream(stream))
+    _check("lsa_shard_sets", st)
+
+
+def lsa_combine(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor,
+                lse_out: torch.Tensor | None = None, stream=None) -> None:
+    """Exact log-sum-exp combination of attention partials: o_parts fp32
+    [n_parts, rows..., d], lse_parts fp32 [n_parts, rows...], out fp32
+    [rows..., d], lse_out fp32 [rows...] or None."""
+    lib = load_library()
+    for t in (o_parts, lse_parts, out) + ((lse_out,) if lse_out is not None else ()):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError("lsa_combine takes contiguous float32 tensors")
+    n_parts, d = o_parts.shape[0], o_parts.shape[-1]
+    rows = o_parts[0].numel() // max(d, 1)
+    if lse_parts.numel() != n_parts * rows or out.numel() != rows * d:
+        raise ValueError("lse_parts must hold n_parts x rows values and out rows x d")
+    if lse_out is not None and lse_out.numel() != rows:
+        raise ValueError("lse_out must hold one value per row")
+    st = lib.lsa_combine(_ptr(o_parts), _ptr(lse_parts), n_parts, rows, d, _ptr(out), _ptr(lse_out), _stream(stream))
+    _check("lsa_combine", st)
 
 
 def lsa_attend_fp8(q: list, k8: list, v8: list, k_scale: list, v_scale: list, index_sets: torch.Tensor,

@@ -18,6 +18,13 @@ So each rank
      best topk of the union are the selected tokens;
   3. assembles the index set [0, s) + selected + [ws, L), -1 padded.
 
+The attention over that set splits the same way (ContextParallelAttention):
+each rank takes the entries in its range (lsa_shard_sets), attends over them
+with its own K/V rows (lsa_attend_lse: normalised output and the log of the
+softmax denominator), all-gathers the partials in one collective, and the
+log-sum-exp combination of the partials (lsa_combine) is the attention over
+the whole set.
+
 Candidates travel as packed 64-bit values, key << ID_BITS | (2^ID_BITS - 1 -
 id) (key = score + 1), so that larger values rank first and ties go to the
 lower id; a zero is an empty slot. Only the caller's device buffers, the
@@ -202,3 +209,78 @@ class ContextParallelIndex:
         local = self.local_best(self.token_candidates(q_idx, w, k_idx, L, kept), self.b.topk)
         selected = self.global_best(self.exchange(local), self.b.topk)
         return self.assemble(L, selected)
+
+
+class ContextParallelAttention:
+    """Attention of decode rows of one sequence whose K/V caches are split
+    over ranks by token range.
+
+    The rank holds positions [lo, hi) of every layer's K and V (bf16 [hi - lo,
+    H_kv, d]). Every rank passes the same index sets (int32 [n_q, budget],
+    positions relative to the sequence start, e.g. from
+    ContextParallelIndex); every rank returns the same output. shard,
+    partial, combine and exchange default to the library's kernels and an
+    all-gather over `group`; they are parameters so that the exchange logic
+    can be exercised without GPUs."""
+
+    def __init__(self, bounds: list[tuple[int, int]], rank: int, group=None, shard=None, partial=None,
+                 combine=None, exchange=None):
+        self.bounds = bounds
+        self.rank = rank
+        self.group = group
+        self.shard = shard or self._gpu_shard
+        self.partial = partial or self._gpu_partial
+        self.combine = combine or self._gpu_combine
+        self.exchange = exchange or (lambda x: dist_exchange(x, group))
+        lo, hi = bounds[rank]
+        if hi <= lo:
+            raise ValueError("every rank needs a non-empty token range")
+
+    # -- the library's kernels -------------------------------------------------
+    @staticmethod
+    def _gpu_shard(sets: torch.Tensor, lo: int, hi: int) -> torch.Tensor:
+        local = torch.empty_like(sets)
+        lsa.lsa_shard_sets(sets.contiguous(), lo, hi, local)
+        return local
+
+    @staticmethod
+    def _gpu_partial(q: list, k: list, v: list, local_sets: torch.Tensor, n_tokens: int):
+        dev = q[0].device
+        n_q, H_q, d = q[0].shape
+        H_kv = k[0].shape[1]
+        batch = lsa.Batch(kv_offset=torch.zeros(1, dtype=torch.int64, device=dev),
+                          seq_lens=torch.full((1,), n_tokens, dtype=torch.int32, device=dev),
+                          q_seq=torch.zeros(n_q, dtype=torch.int32, device=dev),
+                          q_len=torch.full((n_q,), n_tokens, dtype=torch.int32, device=dev),
+                          max_len=n_tokens, total_tokens=n_tokens)
+        G = len(q)
+        ws = torch.empty(max(1, lsa.lsa_attend_workspace_size(batch, H_q, H_kv, d, local_sets.shape[1], G)),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty((G, n_q, H_q, d), dtype=torch.float32, device=dev)
+        lse = torch.empty((G, n_q, H_q), dtype=torch.float32, device=dev)
+        lsa.lsa_attend_lse(q, k, v, local_sets, batch, list(out.unbind(0)), list(lse.unbind(0)), ws)
+        return out, lse
+
+    @staticmethod
+    def _gpu_combine(o_parts: torch.Tensor, lse_parts: torch.Tensor) -> torch.Tensor:
+        out = torch.empty(o_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+        lsa.lsa_combine(o_parts.contiguous(), lse_parts.contiguous(), out)
+        return out
+
+    # -- the steps -------------------------------------------------------------
+    def attend(self, q: list, k: list, v: list, sets: torch.Tensor) -> torch.Tensor:
+        """Every layer's output (fp32 [G, n_q, H_q, d]) over the whole set.
+
+        q: G tensors bf16 [n_q, H_q, d] (the same on every rank); k, v: this
+        rank's G tensors bf16 [hi - lo, H_kv, d]."""
+        lo, hi = self.bounds[self.rank]
+        local = self.shard(sets, lo, hi)
+        o, lse = self.partial(q, k, v, local, hi - lo)
+        n_o = o.numel()
+        # one collective: every rank's outputs and lse values in one vector
+        gathered = self.exchange(torch.cat([o.reshape(-1), lse.reshape(-1)]))
+        world = gathered.numel() // (n_o + lse.numel())
+        parts = gathered.reshape(world, -1)
+        o_parts = parts[:, :n_o].reshape((world,) + tuple(o.shape))
+        lse_parts = parts[:, n_o:].reshape((world,) + tuple(lse.shape))
+        return self.combine(o_parts, lse_parts)

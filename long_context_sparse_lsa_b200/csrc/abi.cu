@@ -275,6 +275,7 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     a.fine_keys = reinterpret_cast<uint32_t*>(ws + plan.off_fine);
     a.cand = dense ? reinterpret_cast<uint64_t*>(ws + plan.off_cand) : nullptr;
     a.cand_seg = dense ? reinterpret_cast<int32_t*>(ws + plan.off_count) : nullptr;
+    a.ghist = dense ? reinterpret_cast<uint32_t*>(ws + plan.off_ghist) : nullptr;
     a.tc_splits = dense ? lsa::prefill_tc_splits(batch->n_q) : 0;
     a.coarse_cap = plan.coarse_cap;
     a.fine_cap = plan.fine_cap;
@@ -335,8 +336,8 @@ int32_t lsa_attend_launches(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv,
 static lsa_status_t attend_impl(const uint16_t* const* q, const void* const* k_cache, const void* const* v_cache,
                                 const float* kscale, const float* vscale, int32_t H_q, int32_t H_kv, int32_t d,
                                 const int32_t* index_sets, int32_t budget, const lsa_batch_t* batch,
-                                int32_t layers_per_index, float* const* out, void* workspace, size_t workspace_bytes,
-                                int32_t* dev_status, void* stream) {
+                                int32_t layers_per_index, float* const* out, float* const* lse, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, void* stream) {
     const bool fp8 = kscale != nullptr;
     if (!batch_ok(batch, true)) return LSA_ERR_INVALID_ARG;
     if (H_q < 1 || H_kv < 1 || d < 1 || budget < 0 || layers_per_index < 1) return LSA_ERR_INVALID_ARG;
@@ -356,6 +357,7 @@ static lsa_status_t attend_impl(const uint16_t* const* q, const void* const* k_c
             return LSA_ERR_INVALID_ARG;
         if (!aligned(q[g], 16) || !aligned(k_cache[g], 16) || !aligned(v_cache[g], 16) || !aligned(out[g], 16))
             return LSA_ERR_INVALID_ARG;
+        if (lse != nullptr && (lse[g] == nullptr || !aligned(lse[g], 4))) return LSA_ERR_INVALID_ARG;
     }
     if ((int64_t)batch->n_q > 65535) return LSA_ERR_UNSUPPORTED;
     lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, budget, layers_per_index,
@@ -368,6 +370,7 @@ static lsa_status_t attend_impl(const uint16_t* const* q, const void* const* k_c
         a.k[g] = static_cast<const uint16_t*>(k_cache[g]);
         a.v[g] = static_cast<const uint16_t*>(v_cache[g]);
         a.out[g] = out[g];
+        a.lse[g] = lse != nullptr ? lse[g] : nullptr;
         a.kscale[g] = fp8 ? kscale[g] : 1.f;
         a.vscale[g] = fp8 ? vscale[g] : 1.f;
     }
@@ -413,8 +416,180 @@ lsa_status_t lsa_attend(const uint16_t* const* q, const uint16_t* const* k_cache
                         const lsa_batch_t* batch, int32_t layers_per_index, float* const* out, void* workspace,
                         size_t workspace_bytes, int32_t* dev_status, void* stream) {
     return attend_impl(q, reinterpret_cast<const void* const*>(k_cache), reinterpret_cast<const void* const*>(v_cache),
-                       nullptr, nullptr, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, workspace,
-                       workspace_bytes, dev_status, stream);
+                       nullptr, nullptr, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, nullptr,
+                       workspace, workspace_bytes, dev_status, stream);
+}
+
+lsa_status_t lsa_attend_lse(const uint16_t* const* q, const uint16_t* const* k_cache, const uint16_t* const* v_cache,
+                            int32_t H_q, int32_t H_kv, int32_t d, const int32_t* index_sets, int32_t budget,
+                            const lsa_batch_t* batch, int32_t layers_per_index, float* const* out,
+                            float* const* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+    if (lse == nullptr) return LSA_ERR_INVALID_ARG;
+    return attend_impl(q, reinterpret_cast<const void* const*>(k_cache), reinterpret_cast<const void* const*>(v_cache),
+                       nullptr, nullptr, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, lse,
+                       workspace, workspace_bytes, dev_status, stream);
+}
+
+// ---- draft-row groups --------------------------------------------------------
+static bool grouped_shape_ok(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, int32_t budget,
+                             int32_t G, int32_t group_rows) {
+    if (!attend_shape_ok(H_q, H_kv, d, budget, G) || H_q / H_kv > 8) return false;
+    if (group_rows != 1 && group_rows != 2 && group_rows != 4 && group_rows != 8) return false;
+    if (batch->n_q % group_rows != 0 || batch->n_q / group_rows > 65535) return false;
+    if (lsa::union_smem_bytes(group_rows, budget) > 227 * 1024) return false;
+    return true;
+}
+
+struct GroupedLayout {
+    lsa::AttendPlan p;
+    size_t off_pos, off_msk, off_len, bytes;
+    int cap;
+};
+
+static GroupedLayout grouped_layout(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t budget, int32_t G,
+                                    int32_t group_rows) {
+    GroupedLayout l;
+    l.p = lsa::plan_attend_grouped(batch->n_q, group_rows, H_q, H_kv, budget, G, lsa::device_sm_count());
+    l.cap = group_rows * budget;
+    const size_t groups = (size_t)(batch->n_q / group_rows);
+    size_t off = (l.p.ws_bytes + 255) / 256 * 256;
+    l.off_pos = off;
+    off = (off + groups * l.cap * 4 + 255) / 256 * 256;
+    l.off_msk = off;
+    off = (off + groups * l.cap + 255) / 256 * 256;
+    l.off_len = off;
+    off = (off + groups * 4 + 255) / 256 * 256;
+    l.bytes = off;
+    return l;
+}
+
+size_t lsa_attend_grouped_workspace_size(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d,
+                                         int32_t budget, int32_t layers_per_index, int32_t group_rows) {
+    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1) return 0;
+    if (!grouped_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index, group_rows)) return 0;
+    return grouped_layout(batch, H_q, H_kv, budget, layers_per_index, group_rows).bytes;
+}
+
+int32_t lsa_attend_grouped_launches(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, int32_t budget,
+                                    int32_t layers_per_index, int32_t group_rows) {
+    if (batch == nullptr || batch->n_q <= 0) return 0;
+    if (!grouped_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index, group_rows)) return 0;
+    const GroupedLayout l = grouped_layout(batch, H_q, H_kv, budget, layers_per_index, group_rows);
+    return l.p.n_splits > 1 ? 3 : 2;  // union, attention[, split merge]
+}
+
+lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const* k_cache,
+                                const uint16_t* const* v_cache, int32_t H_q, int32_t H_kv, int32_t d,
+                                const int32_t* index_sets, int32_t budget, const lsa_batch_t* batch,
+                                int32_t layers_per_index, int32_t group_rows, float* const* out, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    if (!batch_ok(batch, true)) return LSA_ERR_INVALID_ARG;
+    if (H_q < 1 || H_kv < 1 || d < 1 || budget < 0 || layers_per_index < 1 || group_rows < 1)
+        return LSA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0 || batch->n_q % group_rows != 0) return LSA_ERR_INVALID_ARG;
+    if (!grouped_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index, group_rows)) return LSA_ERR_UNSUPPORTED;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr) return LSA_ERR_INVALID_ARG;
+    if (batch->n_q == 0) return LSA_OK;
+    if (budget > 0 && (index_sets == nullptr || !aligned(index_sets, 4))) return LSA_ERR_INVALID_ARG;
+    for (int g = 0; g < layers_per_index; ++g) {
+        if (q[g] == nullptr || k_cache[g] == nullptr || v_cache[g] == nullptr || out[g] == nullptr)
+            return LSA_ERR_INVALID_ARG;
+        if (!aligned(q[g], 16) || !aligned(k_cache[g], 16) || !aligned(v_cache[g], 16) || !aligned(out[g], 16))
+            return LSA_ERR_INVALID_ARG;
+    }
+    const GroupedLayout l = grouped_layout(batch, H_q, H_kv, budget, layers_per_index, group_rows);
+    if (workspace == nullptr || workspace_bytes < l.bytes || !aligned(workspace, 256)) return LSA_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    lsa::UnionArgs u;
+    std::memset(&u, 0, sizeof u);
+    u.sets = index_sets;
+    u.q_seq = batch->q_seq;
+    u.q_len = batch->q_len;
+    u.kv_offset = batch->kv_offset;
+    u.seq_lens = batch->seq_lens;
+    u.union_pos = reinterpret_cast<int32_t*>(ws + l.off_pos);
+    u.union_msk = ws + l.off_msk;
+    u.union_len = reinterpret_cast<int32_t*>(ws + l.off_len);
+    u.dev_status = dev_status;
+    u.total_tokens = batch->total_tokens;
+    u.n_groups = batch->n_q / group_rows;
+    u.group_rows = group_rows;
+    u.budget = budget;
+    u.union_cap = l.cap;
+    u.n_seq = batch->n_seq;
+    u.max_len = batch->max_len;
+    cudaError_t e = lsa::launch_union_sets(u, cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    lsa::AttendArgs a;
+    std::memset(&a, 0, sizeof a);
+    for (int g = 0; g < layers_per_index; ++g) {
+        a.q[g] = q[g];
+        a.k[g] = k_cache[g];
+        a.v[g] = v_cache[g];
+        a.out[g] = out[g];
+        a.kscale[g] = 1.f;
+        a.vscale[g] = 1.f;
+    }
+    a.sets = index_sets;
+    a.kv_offset = batch->kv_offset;
+    a.seq_lens = batch->seq_lens;
+    a.q_seq = batch->q_seq;
+    a.q_len = batch->q_len;
+    a.dev_status = dev_status;
+    const size_t rows_q = (size_t)layers_per_index * batch->n_q;
+    if (l.p.n_splits > 1) {
+        a.part_o = reinterpret_cast<float*>(ws);
+        const size_t off = (rows_q * l.p.n_splits * H_q * 128 * 4 + 255) / 256 * 256;
+        a.part_ml = reinterpret_cast<float*>(ws + off);
+    }
+    a.total_tokens = batch->total_tokens;
+    a.n_seq = batch->n_seq;
+    a.n_q = batch->n_q;
+    a.max_len = batch->max_len;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.budget = budget;
+    a.G = layers_per_index;
+    a.n_splits = l.p.n_splits;
+    a.entries_per_split = l.p.entries_per_split;
+    a.head_groups = H_kv;
+    a.hpc = 1;
+    a.stage_off = l.p.stage_off;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    a.union_pos = u.union_pos;
+    a.union_msk = u.union_msk;
+    a.union_len = u.union_len;
+    a.group_rows = group_rows;
+    a.union_cap = l.cap;
+    e = lsa::launch_attend_grouped(a, l.p.smem_bytes, cs);
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+lsa_status_t lsa_shard_sets(const int32_t* index_sets, int32_t n_q, int32_t budget, int32_t lo, int32_t hi,
+                            int32_t* local_sets, int32_t* dev_status, void* stream) {
+    if (n_q < 0 || budget < 0 || lo < 0 || hi < lo) return LSA_ERR_INVALID_ARG;
+    if (budget > LSA_MAX_BUDGET || n_q > 65535) return LSA_ERR_UNSUPPORTED;
+    if (n_q == 0 || budget == 0) return LSA_OK;
+    if (index_sets == nullptr || local_sets == nullptr || index_sets == local_sets) return LSA_ERR_INVALID_ARG;
+    if (!aligned(index_sets, 4) || !aligned(local_sets, 4)) return LSA_ERR_INVALID_ARG;
+    cudaError_t e = lsa::launch_shard_sets(index_sets, n_q, budget, lo, hi, local_sets, dev_status,
+                                           reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+lsa_status_t lsa_combine(const float* o_parts, const float* lse_parts, int32_t n_parts, int64_t rows, int32_t d,
+                         float* out, float* lse_out, void* stream) {
+    if (n_parts < 1 || rows < 0 || d < 0 || d % 4 != 0) return LSA_ERR_INVALID_ARG;
+    if (n_parts > 65535 || (rows + 7) / 8 > 0x7fffffff) return LSA_ERR_UNSUPPORTED;
+    if (rows == 0 || d == 0) return LSA_OK;
+    if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return LSA_ERR_INVALID_ARG;
+    if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16)) return LSA_ERR_INVALID_ARG;
+    if (lse_out != nullptr && !aligned(lse_out, 4)) return LSA_ERR_INVALID_ARG;
+    cudaError_t e = lsa::launch_combine(o_parts, lse_parts, n_parts, rows, d, out, lse_out,
+                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 
 static lsa_status_t point_common(const int8_t* q_idx, const int32_t* w, int32_t w_max, int32_t H_I, int32_t d_I,
@@ -495,8 +670,8 @@ lsa_status_t lsa_attend_fp8(const uint16_t* const* q, const uint8_t* const* k_ca
                             int32_t* dev_status, void* stream) {
     if (k_scale == nullptr || v_scale == nullptr) return LSA_ERR_INVALID_ARG;
     return attend_impl(q, reinterpret_cast<const void* const*>(k_cache), reinterpret_cast<const void* const*>(v_cache),
-                       k_scale, v_scale, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, workspace,
-                       workspace_bytes, dev_status, stream);
+                       k_scale, v_scale, H_q, H_kv, d, index_sets, budget, batch, layers_per_index, out, nullptr,
+                       workspace, workspace_bytes, dev_status, stream);
 }
 
 }  // extern "C"

@@ -157,13 +157,31 @@ __device__ __forceinline__ void softmax_pv(const float (&sacc)[NT][4], bool ok_g
     }
 }
 
+// ln(sum_j exp(s_j)) from the running max m (log2 units of the scaled
+// scores) and the denominator l = sum_j exp2(m_j - m): (m + log2 l) ln 2.
+__device__ __forceinline__ float lse_of(float m, float l) {
+    return l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+}
+
+// Zeroes the output of an invalid row's query heads [h0, h0 + nh) and marks
+// their lse empty (split 0 of the row does it).
+__device__ __forceinline__ void clear_row(const AttendArgs& a, int layer, int r, int h0, int nh, int tid,
+                                          int nthreads) {
+    float* orow = a.out[layer] + ((int64_t)r * a.H_q + h0) * kD;
+    for (int i = tid; i < nh * kD; i += nthreads) orow[i] = 0.f;
+    if (a.lse[layer] != nullptr)
+        for (int i = tid; i < nh; i += nthreads) a.lse[layer][(int64_t)r * a.H_q + h0 + i] = -INFINITY;
+}
+
 // Merges the consumer warps of each kv head (in registers: warps with
 // wsel > 0 park their fragments in `merge_area`, lane-major, and the wsel == 0
 // warp folds them in with the log-sum-exp rule), then writes the head's query
 // heads: the final output when there is one split, else one partial. Every
 // thread of the CTA calls it (it holds a CTA barrier); warps >= kConsumers
 // only take part in the barrier.
-template <int NT>
+// GROUPED (draft-row groups): the warps w % hpc == j work for row r + j of the
+// group (hpc = the group's rows) and all of them for kv head hgrp.
+template <int NT, bool GROUPED = false>
 __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* merge_area, float (&o)[NT][kD / 16][4],
                                                 float (&m_run)[NT][2], float (&l_run)[NT][2], int warp, int lane,
                                                 int hpc, int hgrp, int r, int layer, int split, int ratio,
@@ -192,9 +210,10 @@ __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* me
     }
     __syncthreads();
     const bool direct = a.n_splits == 1;
-    const int64_t row_q = (int64_t)layer * a.n_q + r;
     if (warp < kConsumers && wsel_me == 0) {
         const int h_local = warp % hpc;
+        if (GROUPED) r += h_local;
+        const int64_t row_q = (int64_t)layer * a.n_q + r;
         const int n_sel = kConsumers / hpc;
         for (int j = 1; j < n_sel; ++j) {
             const int w = h_local + hpc * j;
@@ -219,7 +238,7 @@ __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* me
             }
         }
         // write this kv head's query heads: the final output, or one split partial
-        const int kvh = hgrp * hpc + h_local;
+        const int kvh = GROUPED ? hgrp : hgrp * hpc + h_local;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
 #pragma unroll
@@ -239,6 +258,8 @@ __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* me
                 if (!direct && g == 0)
                     *reinterpret_cast<float2*>(a.part_ml + ((row_q * a.n_splits + split) * a.H_q + qh) * 2) =
                         make_float2(m_run[n][c], l_run[n][c]);
+                if (direct && g == 0 && a.lse[layer] != nullptr)
+                    a.lse[layer][(int64_t)r * a.H_q + qh] = lse_of(m_run[n][c], l_run[n][c]);
             }
         }
     }
@@ -276,10 +297,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) attend_kernel(const __grid_cons
     if (bad) {
         if (tid == 0 && blockIdx.x == 0 && layer == 0)
             flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
-        if (split == 0) {
-            float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)hgrp * q_heads_cta) * kD;
-            for (int i = tid; i < q_heads_cta * kD; i += kAtThreads) orow[i] = 0.f;
-        }
+        if (split == 0) clear_row(a, layer, r, hgrp * q_heads_cta, q_heads_cta, tid, kAtThreads);
         return;
     }
 
@@ -599,10 +617,7 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
     if (bad) {
         if (tid == 0 && blockIdx.x == 0 && layer == 0)
             flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
-        if (split == 0) {
-            float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)hgrp * q_heads_cta) * kD;
-            for (int i = tid; i < q_heads_cta * kD; i += kConsumers * kWarp) orow[i] = 0.f;
-        }
+        if (split == 0) clear_row(a, layer, r, hgrp * q_heads_cta, q_heads_cta, tid, kConsumers * kWarp);
         return;
     }
     const int n_entries = min(L, a.budget);
@@ -713,6 +728,137 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
                         FP8 ? a.vscale[layer] : 1.f);
 }
 
+// Draft-row groups: rows come in groups of D consecutive rows of one
+// sequence, and the union of each group's index sets (positions ascending,
+// each with a mask of the rows holding it; union_sets_kernel) is split over
+// the CTAs of the group and kv head. Warp w attends for row w % D over the
+// union tiles w / D, w / D + 8 / D, ...: the D warps of a phase gather the
+// same tiles at the same time, each its own row's members (the others read as
+// masked), so a K/V row held by several rows of the group is fetched from L2
+// once per CTA and from L1 by the others. The tile loop, the fragments and the
+// softmax are attend_rk_kernel's (bf16 caches, GQA groups of at most 8 query
+// heads); the partials merge as lsa_attend's.
+__global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(const __grid_constant__ AttendArgs a) {
+    constexpr int NT = 1;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+    const int g = lane >> 2, t4 = lane & 3;
+    const int D = a.group_rows;
+    const int split = blockIdx.x / a.H_kv;
+    const int kvh = blockIdx.x % a.H_kv;
+    const int grp = blockIdx.y;
+    const int layer = blockIdx.z;
+    const int ratio = a.H_q / a.H_kv;
+    const int jr = warp % D;             // this warp's row of the group
+    const int ph = warp / D, n_ph = kConsumers / D;
+    const int r = grp * D + jr;
+    // the row's metadata (the caller's) before the wait
+    const int seq = a.q_seq[r];
+    const int L = a.q_len[r];
+    const int seq_c = min(max(seq, 0), a.n_seq - 1);
+    const int64_t off = a.kv_offset[seq_c];
+    const int slen = a.seq_lens[seq_c];
+    pdl_enter();
+    const bool bad = seq < 0 || seq >= a.n_seq || L < 1 || L > a.max_len || L > slen || off < 0 ||
+                     off + slen > a.total_tokens;
+    if (bad && split == 0 && kvh == 0 && layer == 0 && lane == 0 && ph == 0)
+        flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
+    if (bad && split == 0 && ph == 0) {  // an invalid row's output is zero
+        float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
+        for (int i = lane; i < ratio * kD; i += kWarp) orow[i] = 0.f;
+    }
+    // this CTA's part of the union, as one entry list per row (other rows'
+    // members read as -1)
+    const int U = min(max(a.union_len[grp], 0), a.union_cap);
+    const int e0 = (int)((int64_t)U * split / a.n_splits);
+    const int n_local = min((int)((int64_t)U * (split + 1) / a.n_splits) - e0, a.entries_per_split);
+    const int n_tiles = (n_local + kTile - 1) / kTile;
+    const int stride = a.entries_per_split;  // per-row list length in shared memory
+    int32_t* s_rows = reinterpret_cast<int32_t*>(smem);
+    const int32_t* up = a.union_pos + (int64_t)grp * a.union_cap + e0;
+    const uint8_t* um = a.union_msk + (int64_t)grp * a.union_cap + e0;
+    for (int i = tid; i < n_tiles * kTile; i += kConsumers * kWarp) {
+        const int p = i < n_local ? up[i] : -1;
+        const uint32_t m = i < n_local ? um[i] : 0u;
+        for (int j = 0; j < D; ++j) s_rows[j * stride + i] = ((m >> j) & 1u) && p >= 0 ? p : -1;
+    }
+    __syncthreads();
+    int32_t* s_ent = s_rows + jr * stride;
+    if (bad) {  // nothing of an invalid row is read (its entries were checked against nothing)
+        for (int i = lane; i < n_tiles * kTile; i += kWarp) s_ent[i] = -1;
+    } else {
+        for (int i = lane; i < n_tiles * kTile; i += kWarp)
+            if (s_ent[i] >= L) s_ent[i] = -1;  // the union holds only members; a row never reads past q_len
+    }
+    __syncthreads();
+
+    float o[NT][kD / 16][4];
+    float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+    for (int mt = 0; mt < kD / 16; ++mt) o[0][mt][0] = o[0][mt][1] = o[0][mt][2] = o[0][mt][3] = 0.f;
+    m_run[0][0] = m_run[0][1] = -INFINITY;
+    l_run[0][0] = l_run[0][1] = 0.f;
+    const int64_t tok_stride = (int64_t)a.H_kv * kD;
+    const uint16_t* kbase = a.k[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
+    const uint16_t* vbase = a.v[layer] + (off * a.H_kv + (int64_t)kvh) * kD;
+    uint32_t qb[kD / 16][2];
+    {
+        const uint16_t* qrow = a.q[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
+        const bool ok = g < ratio;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint16_t* p = qrow + g * kD + 8 * (t4 + 4 * (ks >> 1)) + 4 * (ks & 1);
+            qb[ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p)) : 0u;
+            qb[ks][1] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p + 2)) : 0u;
+        }
+    }
+    KTile ka, kb2;
+    VTile va, vb2;
+    if (ph < n_tiles) {
+        load_ktile(ka, kbase, tok_stride, s_ent + ph * kTile, g, t4);
+        load_vtile(va, vbase, tok_stride, s_ent + ph * kTile, g, t4);
+    }
+    if (ph + n_ph < n_tiles) {
+        load_ktile(kb2, kbase, tok_stride, s_ent + (ph + n_ph) * kTile, g, t4);
+        load_vtile(vb2, vbase, tok_stride, s_ent + (ph + n_ph) * kTile, g, t4);
+    }
+    auto tile = [&](int i, KTile& k, VTile& v) {
+        const int ent_lane = lane < kTile ? s_ent[i * kTile + lane] : 0;
+        const uint32_t masked = __ballot_sync(0xffffffffu, lane < kTile && ent_lane < 0);
+        const bool ok_g = !((masked >> g) & 1u);
+        const bool ok_g8 = !((masked >> (g + 8)) & 1u);
+        float sacc[NT][4] = {{0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const int j = ks >> 1, w = 2 * (ks & 1);
+            const uint32_t afr[4] = {word(k.r[0][j], w), word(k.r[1][j], w), word(k.r[0][j], w + 1),
+                                     word(k.r[1][j], w + 1)};
+            mma_16<false>(sacc[0], afr, qb[ks][0], qb[ks][1]);
+        }
+        softmax_pv<NT, false>(sacc, ok_g, ok_g8, a.scale_log2, m_run, l_run, o, v);
+        if (i + 2 * n_ph < n_tiles) {
+            load_ktile(k, kbase, tok_stride, s_ent + (i + 2 * n_ph) * kTile, g, t4);
+            load_vtile(v, vbase, tok_stride, s_ent + (i + 2 * n_ph) * kTile, g, t4);
+        }
+    };
+    for (int i = ph; i < n_tiles; i += 2 * n_ph) {
+        tile(i, ka, va);
+        if (i + n_ph < n_tiles) tile(i + n_ph, kb2, vb2);
+    }
+    pdl_trigger();
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int msk = 4; msk < 32; msk <<= 1) l_run[0][j] += __shfl_xor_sync(0xffffffffu, l_run[0][j], msk);
+    __syncthreads();  // the merge area reuses the entry lists
+    if (bad) {        // keep the zeros written above (a partial of nothing merges to zero too)
+#pragma unroll
+        for (int mt = 0; mt < kD / 16; ++mt) o[0][mt][0] = o[0][mt][1] = o[0][mt][2] = o[0][mt][3] = 0.f;
+    }
+    merge_and_store<NT, true>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, D, kvh, grp * D, layer, split,
+                              ratio);
+}
+
 // Split merge: one CTA per (query head, row, layer) with one warp per
 // kMergeSplitsPerWarp splits, so every partial is loaded in one round of
 // loads; lane l owns dims 4l..4l+3. Each warp folds its splits with the
@@ -795,6 +941,7 @@ __global__ void __launch_bounds__(kMergeMaxWarps * kWarp) attend_merge_kernel(co
     const float inv = den > 0.f ? 1.f / den : 0.f;
     reinterpret_cast<float4*>(a.out[layer] + ((int64_t)r * a.H_q + h) * kD)[lane] =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (lane == 0 && a.lse[layer] != nullptr) a.lse[layer][(int64_t)r * a.H_q + h] = lse_of(M, den);
 }
 
 }  // namespace
@@ -852,6 +999,55 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
     }
     p.ws_bytes = ws;
     return p;
+}
+
+AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int budget, int G, int num_sms) {
+    AttendPlan p;
+    p.hpc = 1;
+    p.head_groups = H_kv;
+    const int cap = group_rows * budget;  // the union holds at most this many entries
+    const long units = (long)(n_q / group_rows) * H_kv * G;
+    int splits = units > 0 ? (int)((num_sms + units / 2) / units) : 1;
+    const int min_splits = (cap + kMaxEntriesPerSplit - 1) / kMaxEntriesPerSplit;
+    const int max_splits = (cap + 63) / 64;
+    if (splits > max_splits) splits = max_splits;
+    if (splits < min_splits) splits = min_splits;
+    if (splits < 1) splits = 1;
+    p.n_splits = splits;
+    int eps = (cap + splits - 1) / splits;  // a CTA's share of the longest union
+    eps = (eps + kTile - 1) / kTile * kTile;
+    if (eps < kTile) eps = kTile;
+    p.entries_per_split = eps;
+    const size_t ent = ((size_t)group_rows * eps * 4 + 127) / 128 * 128;
+    p.stage_off = (int)ent;
+    const size_t merge = (size_t)kConsumers * ((kD / 16) * 4 + 4) * kWarp * 4;
+    p.smem_bytes = ent + merge;
+    const size_t rows_q = (size_t)G * n_q;
+    size_t ws = 0;
+    if (splits > 1) {
+        ws = rows_q * splits * H_q * kD * 4;
+        ws = (ws + 255) / 256 * 256;
+        ws += rows_q * splits * H_q * 2 * 4;
+        ws = (ws + 255) / 256 * 256;
+    }
+    p.ws_bytes = ws;  // the caller adds the union arrays
+    return p;
+}
+
+cudaError_t launch_attend_grouped(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(attend_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_bytes);
+    if (e != cudaSuccess) return e;
+    const int pct = (int)(((smem_bytes + 2048) * 100 + kSmemPerSm - 1) / kSmemPerSm);
+    e = cudaFuncSetAttribute(attend_group_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, pct < 100 ? pct : 100);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)(a.n_splits * a.H_kv), (unsigned)(a.n_q / a.group_rows), (unsigned)a.G);
+    e = launch_pdl(attend_group_kernel, grid, dim3(kConsumers * kWarp), smem_bytes, stream, 0, a);
+    if (e != cudaSuccess || a.n_splits == 1) return e;
+    int nw = (a.n_splits + kMergeSplitsPerWarp - 1) / kMergeSplitsPerWarp;
+    if (nw > kMergeMaxWarps) nw = kMergeMaxWarps;
+    return launch_pdl(attend_merge_kernel, dim3((unsigned)a.H_q, (unsigned)a.n_q, (unsigned)a.G),
+                      dim3((unsigned)(nw * kWarp)), 0, stream, 0, a);
 }
 
 cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream) {

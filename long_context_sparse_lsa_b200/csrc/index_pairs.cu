@@ -19,6 +19,7 @@ constexpr int kTkWarps = kTkThreads / kWarp;
 static_assert(kHistBins / kTkThreads == 4, "the scan gives each thread one 4-bin vector");
 constexpr int kTkCandCap = 2048;  // keys of the threshold bin held in the candidate list
 constexpr int kTkDigitBits = 12;
+constexpr int kPassUnroll = 8;  // pair loads in flight per thread in a pass
 constexpr int kMergeIdBits = LSA_MERGE_ID_BITS;  // id field of a merge value
 constexpr uint32_t kMergeIdMask = (1u << kMergeIdBits) - 1u;
 
@@ -166,6 +167,9 @@ __device__ uint32_t select_sorted(PairShared& sh, int32_t* sel, uint32_t n, uint
     while (P < m) P <<= 1;
     for (uint32_t i = m + tid; i < P; i += kTkThreads) sel[i] = 0x7fffffff;
     __syncthreads();
+    // (with one pair per thread, a stride of at most 32 keeps each warp inside
+    // its own 64 elements: a warp barrier suffices between two such steps)
+    const bool one_pair = P <= 2u * kTkThreads;
     for (uint32_t size = 2; size <= P; size <<= 1) {
         for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
             for (uint32_t i = tid; i < P / 2; i += kTkThreads) {
@@ -178,7 +182,11 @@ __device__ uint32_t select_sorted(PairShared& sh, int32_t* sel, uint32_t n, uint
                     sel[hi] = x;
                 }
             }
-            __syncthreads();
+            // the next step stays inside the warp's 64 elements too: a stride
+            // halved, or (after stride 1) the next size's first stride <= 32
+            const bool next_local = stride > 1u || (size < P && size <= 32u);
+            if (one_pair && stride <= 32u && next_local) __syncwarp();
+            else __syncthreads();
         }
     }
     return m;
@@ -210,28 +218,36 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_pairs_kernel(const __grid_
         for (int e = tid; e < a.budget; e += kTkThreads) out[e] = -1;
         return;
     }
-    // the row's candidates: one segment per token split of the scoring
+    // the row's candidates: one segment per token split and lane quarter of the scoring
     const uint64_t* pairs = a.cand + (int64_t)r * a.fine_cap;
-    __shared__ int32_t seg_lo[LSA_TC_MAX_SPLITS], seg_n[LSA_TC_MAX_SPLITS];
-    if (tid < a.tc_splits) {
-        const int2 sg = reinterpret_cast<const int2*>(a.cand_seg)[(int64_t)r * LSA_TC_MAX_SPLITS + tid];
+    constexpr int kMaxSegs = LSA_TC_MAX_SPLITS * LSA_TC_SEGS;
+    __shared__ int32_t seg_lo[kMaxSegs], seg_n[kMaxSegs];
+    const int n_segs = a.tc_splits * LSA_TC_SEGS;
+    if (tid < n_segs) {
+        const int2 sg = reinterpret_cast<const int2*>(a.cand_seg)[(int64_t)r * kMaxSegs + tid];
         const int lo = min(max(sg.x, 0), a.fine_cap);
         seg_lo[tid] = lo;
         seg_n[tid] = min(max(sg.y, 0), a.fine_cap - lo);
     }
     __syncthreads();
     uint32_t n = 0;
-    for (int sp = 0; sp < a.tc_splits; ++sp) n += (uint32_t)seg_n[sp];
+    for (int sp = 0; sp < n_segs; ++sp) n += (uint32_t)seg_n[sp];
     // every candidate pair once: f(pair)
     // (every lane of a warp calls f the same number of times: f(pair, ok))
+    // (8 loads in flight per thread per round: a pass is a few L2 round trips)
     auto for_each_pair = [&](auto&& f) {
-        for (int sp = 0; sp < a.tc_splits; ++sp) {
+        for (int sp = 0; sp < n_segs; ++sp) {
             const uint64_t* seg = pairs + seg_lo[sp];
             const int cnt = seg_n[sp];
-            for (int i0 = tid - (tid & 31); i0 < cnt; i0 += kTkThreads) {
-                const int i = i0 + (tid & 31);
-                const bool ok = i < cnt;
-                f(ok ? __ldcg(seg + i) : 0ull, ok);
+            for (int i0 = tid - (tid & 31); i0 < cnt; i0 += kTkThreads * kPassUnroll) {
+                uint64_t e[kPassUnroll];
+#pragma unroll
+                for (int u = 0; u < kPassUnroll; ++u) {
+                    const int i = i0 + u * kTkThreads + (tid & 31);
+                    e[u] = i < cnt ? __ldcg(seg + i) : 0ull;
+                }
+#pragma unroll
+                for (int u = 0; u < kPassUnroll; ++u) f(e[u], i0 + u * kTkThreads + (tid & 31) < cnt);
             }
         }
     };
@@ -276,10 +292,15 @@ __global__ void __launch_bounds__(kTkThreads, 1) merge_pairs_kernel(const uint64
     const int cnt = min(max(cnt_raw, 0), cap);
     const uint64_t* row = pairs + (int64_t)r * cap;
     auto for_each_pair = [&](auto&& f) {
-        for (int i0 = tid - (tid & 31); i0 < cnt; i0 += kTkThreads) {
-            const int i = i0 + (tid & 31);
-            const uint64_t e = i < cnt ? __ldcg(row + i) : 0ull;
-            f(e, e != 0ull);
+        for (int i0 = tid - (tid & 31); i0 < cnt; i0 += kTkThreads * kPassUnroll) {
+            uint64_t e[kPassUnroll];
+#pragma unroll
+            for (int u = 0; u < kPassUnroll; ++u) {
+                const int i = i0 + u * kTkThreads + (tid & 31);
+                e[u] = i < cnt ? __ldcg(row + i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < kPassUnroll; ++u) f(e[u], e[u] != 0ull);
         }
     };
     // the row's entries (nonzero values)

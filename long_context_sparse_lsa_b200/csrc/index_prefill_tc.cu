@@ -38,7 +38,7 @@
 namespace lsa {
 namespace {
 
-constexpr int kTcTokens = 128;                       // M: cached tokens per tile
+constexpr int kTcTokens = LSA_TC_TOKENS;             // M: cached tokens per tile
 constexpr int kTcCols = 256;                         // N: query-head rows per CTA
 constexpr int kTcK = 128;                            // d_I bytes per key row
 constexpr int kTcStages = 6;                         // A-tile ring
@@ -62,22 +62,26 @@ struct TcArgs {
     const int64_t* kv_offset;
     const int32_t* seq_lens;
     uint64_t* cand;        // [n_q][fine_cap] candidates: key << 32 | position
-    int32_t* cand_seg;     // [n_q][kTcMaxSplits][2] (first slot, count) of each token split's candidates
+    int32_t* cand_seg;     // [n_q][kTcMaxSplits][4][2] (first slot, count) per token split and lane quarter
+    uint32_t* ghist;       // [n_q][kTcBins] the row's counts over every split (zeroed before the launch)
     int32_t* dev_status;
     int64_t total_tokens;
     int32_t n_q, max_len, w_max, sink, window, fine_cap, topk;
 };
 
-// Candidate filter. A row's keys are counted in a histogram of kTcBins bins
-// on a logarithmic scale (bit length and the 3 bits after the leading one);
-// every kTcUpdate tiles the lower edge of the highest bin whose count from the
-// top reaches topk becomes the row's threshold. Keys this CTA has seen can
-// only add to the counts, so the threshold never exceeds the k-th largest
-// key of the CTA's tokens, itself at most the row's k-th largest key: every
-// key of the final top-k is at least the threshold in force when it is
-// scored, and is kept as a candidate.
-constexpr int kTcBins = 256;
+// Candidate filter. A row's kept keys (those at or above its threshold) are
+// counted in a histogram of kTcBins bins on a logarithmic scale (bit length
+// and the 3 bits after the leading one). Every kTcUpdate tiles each CTA adds
+// its counts into the row's histogram in global memory, shared by the CTAs
+// of every token split, and reads it back; the lower edge of the highest bin
+// whose count from the top reaches topk becomes the row's threshold. Every
+// counted key is a distinct token of the row, so at least topk of the row's
+// keys lie at or above the threshold: it never exceeds the row's k-th largest
+// key, and every key of the final top-k, being at least the threshold in
+// force when it is scored, is kept as a candidate.
+constexpr int kTcBins = LSA_TC_BINS;
 constexpr int kTcMaxSplits = LSA_TC_MAX_SPLITS;
+static_assert(LSA_TC_SEGS == 4, "one candidate segment per TMEM lane quarter");
 constexpr int kTcUpdate = 8;
 __device__ __forceinline__ uint32_t tc_bin(uint32_t key) {
     if (key < 8u) return key;
@@ -103,9 +107,7 @@ struct TcShared {
     int32_t row_ok[kTcCols];  // and validity
     alignas(16) int32_t w[kTcCols];  // weight of each query-head row (read as 16-byte vectors)
     uint32_t thr[kTcCols / 16];             // per query row of the CTA: candidate threshold
-    uint32_t count[kTcCols / 16];           // per query row: candidates written by this CTA
-    int32_t seg0[kTcCols / 16];             // per query row: first slot of this CTA's segment
-    uint32_t hist[kTcCols / 16][kTcBins];   // per query row: histogram of its keys here
+    uint32_t hist[kTcCols / 16][kTcBins];   // per query row: kept keys here not yet added to ghist
 };
 static_assert(offsetof(TcShared, w) % 16 == 0, "weights are read with 16-byte shared loads");
 static_assert(sizeof(TcShared) % 16 == 0, "TcShared follows 1024-byte aligned tiles");
@@ -240,7 +242,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
         sh.row_s[i] = s;
         sh.row_ws[i] = ws;
         sh.thr[i] = 1u;  // every key (score + 1 >= 1) until the histogram holds topk keys
-        sh.count[i] = 0u;
     }
     for (int i = tid; i < R * kTcBins; i += kTcThreads) (&sh.hist[0][0])[i] = 0u;
     tc_fence_before();
@@ -260,11 +261,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
     const int j_lo = (int)((int64_t)nt_all * blockIdx.x / gridDim.x);
     const int j_hi = (int)((int64_t)nt_all * (blockIdx.x + 1) / gridDim.x);
     const int nt = j_hi - j_lo;
-    // this CTA's candidates of row i go to the slots of its tokens: the
-    // segment starting at the row's first middle token it scores (token splits
-    // are disjoint, so the segments are, and none passes the row's fine_cap)
-    for (int i = tid; i < R; i += kTcThreads) sh.seg0[i] = max(0, t_lo + j_lo * kTcTokens - sh.row_s[i]);
-    __syncthreads();
 
     if (warp == 0) {
         // ---- TMA producer ---------------------------------------------------
@@ -325,7 +321,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             rws[i] = sh.row_ws[ri];
         }
         const int rl0 = half * kRows;  // first query row (of the CTA) of this warp's columns
-        uint64_t* cand0 = a.cand + (int64_t)(row0 + rl0) * a.fine_cap;
+        // This warp's candidates of each of its rows go to its own slots: the
+        // slots of the CTA's tokens (from the union's first middle token; splits
+        // are disjoint and the union spans at most fine_cap slots), quarter q of
+        // them for lane quarter q: one slot per token the warp scores, so the
+        // count lives in a register and no slot is reserved atomically.
+        const int64_t seg_q = (int64_t)j_lo * kTcTokens + (int64_t)quarter * nt * kWarp;
+        const int64_t room = (int64_t)a.fine_cap - seg_q;
+        uint64_t* cand0 = a.cand + (int64_t)(row0 + rl0) * a.fine_cap + seg_q;
+        const uint32_t lt_mask = (1u << lane) - 1u;
+        uint32_t cnt[kRows], thr[kRows];
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+            cnt[i] = 0u;
+            thr[i] = 1u;
+        }
         // 32 columns (32 / H_I query rows) of accumulators -> candidates
         auto rows_of = [&](const uint32_t (&v)[32], int c, int t) {
             int32_t w[32];
@@ -346,35 +356,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
                 const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 const bool in = t >= rs[i] && t < rws[i];
                 const uint32_t key = (uint32_t)acc + 1u;
-                if (in) atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
-                const bool emit = in && key >= *reinterpret_cast<volatile uint32_t*>(&sh.thr[rl0 + i]);
+                const bool emit = in && key >= thr[i];
+                if (emit) atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
                 const uint32_t m = __ballot_sync(0xffffffffu, emit);
-                if (m != 0u) {
-                    // one reservation per warp and row in this CTA's segment, then
-                    // the warp's candidates in lane order
-                    const uint32_t p = warp_append(&sh.count[rl0 + i], emit);
-                    if (emit) {
-                        const uint32_t slot = (uint32_t)sh.seg0[rl0 + i] + p;
-                        if (slot < (uint32_t)a.fine_cap)  // a row holds at most fine_cap middle tokens
-                            cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
-                    }
+                if (emit) {
+                    const uint32_t slot = cnt[i] + __popc(m & lt_mask);
+                    if ((int64_t)slot < room) cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
                 }
+                cnt[i] += __popc(m);
             }
         };
-        // the thresholds of this warp's two query rows (rows 2w', 2w'+1 of the
-        // CTA, w' the epilogue warp index), from their histograms
-        auto update_thresholds = [&]() {
-            const int ew = warp - 2;
+        // Threshold updates of this warp's two query rows (rows 2w', 2w'+1 of
+        // the CTA, w' the epilogue warp index), spread over two tiles so that
+        // the global round trip overlaps a tile's work: flush() moves the CTA's
+        // new counts into the row's global histogram and keeps the returned
+        // totals (lane l: bins 8l .. 8l+7); settle() turns them into the
+        // threshold; the warps of the rows read it back one tile later.
+        const int ew = warp - 2;
+        uint32_t gc[2][8];
+        auto flush = [&]() {
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int row = 2 * ew + q2;
-                uint32_t c8[8];
-                uint32_t own = 0;
+                const bool live = row0 + row < a.n_q;
+                uint32_t* g = a.ghist + (int64_t)(live ? row0 + row : 0) * kTcBins + 8 * lane;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    c8[j] = *reinterpret_cast<volatile uint32_t*>(&sh.hist[row][8 * lane + j]);
-                    own += c8[j];
+                    const uint32_t d = atomicExch(&sh.hist[row][8 * lane + j], 0u);
+                    gc[q2][j] = !live ? 0u : d != 0u ? atomicAdd(g + j, d) + d : __ldcg(g + j);
                 }
+            }
+        };
+        auto settle = [&]() {
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int row = 2 * ew + q2;
+                uint32_t own = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) own += gc[q2][j];
                 uint32_t x = own;  // keys in bins >= 8 * lane
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -387,17 +406,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
                     uint32_t run = x - own;
 #pragma unroll
                     for (int j = 7; j >= 0; --j) {
-                        run += c8[j];
+                        run += gc[q2][j];
                         if (run >= k && best == 0u) best = (uint32_t)(8 * lane + j) + 1u;
                     }
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
                 if (lane == 0 && best > 0u) {
-                    const uint32_t thr = tc_bin_floor(best - 1u);
-                    if (thr > sh.thr[row]) sh.thr[row] = thr;
+                    const uint32_t th = tc_bin_floor(best - 1u);
+                    volatile uint32_t* st = &sh.thr[row];
+                    if (th > *st) *st = th;
                 }
             }
+        };
+        auto refresh = [&]() {
+#pragma unroll
+            for (int i = 0; i < kRows; ++i) thr[i] = max(thr[i], *reinterpret_cast<volatile uint32_t*>(&sh.thr[rl0 + i]));
         };
         for (int j = 0; j < nt; ++j) {
             const int buf = j & 1, use = j >> 1;
@@ -422,21 +446,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
-            if (j % kTcUpdate == kTcUpdate - 1) update_thresholds();
+            const int ph = j % kTcUpdate;
+            if (ph == kTcUpdate - 1) flush();
+            else if (ph == 0 && j > 0) settle();
+            else if (ph == 1 && j > 1) refresh();
+        }
+        // this warp's segment of each of its rows
+        if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < kRows; ++i) {
+                const int r = row0 + rl0 + i;
+                if (r < a.n_q)
+                    reinterpret_cast<int2*>(a.cand_seg)[((int64_t)r * kTcMaxSplits + blockIdx.x) * 4 + quarter] =
+                        make_int2((int)seg_q, (int)min((int64_t)cnt[i], max(room, (int64_t)0)));
+            }
         }
     }
 
     // ---- teardown: wait for every issued MMA, then free TMEM -----------------
     tc_fence_before();
     __syncthreads();
-    // this CTA's candidate segment of each of its rows
-    for (int i = tid; i < R; i += kTcThreads) {
-        const int r = row0 + i;
-        if (r < a.n_q) {
-            int2* seg = reinterpret_cast<int2*>(a.cand_seg) + ((int64_t)r * kTcMaxSplits + blockIdx.x);
-            *seg = make_int2(sh.seg0[i], (int)min(sh.count[i], (uint32_t)max(0, a.fine_cap - sh.seg0[i])));
-        }
-    }
     if (warp == 1 && lane == 0) {
         umma_commit(smem_u32(&sh.drain));  // arrives once all MMAs of this thread are complete
         mbar_wait_bounded(smem_u32(&sh.drain), 0, kWaitLimitNs);
@@ -488,6 +517,7 @@ cudaError_t launch_fine_scores_tc(const IndexArgs& ia, cudaStream_t stream) {
     a.seq_lens = ia.seq_lens;
     a.cand = ia.cand;
     a.cand_seg = ia.cand_seg;
+    a.ghist = ia.ghist;
     a.topk = ia.topk;
     a.dev_status = ia.dev_status;
     a.total_tokens = ia.total_tokens;
@@ -505,6 +535,8 @@ cudaError_t launch_fine_scores_tc(const IndexArgs& ia, cudaStream_t stream) {
     // not exist read as empty (the selection reads `splits` of them)
     cudaError_t e = cudaFuncSetAttribute(fine_score_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kTcSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(a.ghist, 0, (size_t)ia.n_q * kTcBins * sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     return launch_pdl(fine_score_tc_kernel<16>, dim3((unsigned)splits, (unsigned)row_tiles), dim3(kTcThreads),
                       kTcSmem, stream, 0, a);

@@ -776,6 +776,10 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b, bool dense) {
         p.coarse_cap = (max_len + b.hi_block - 1) / b.hi_block + 1;
         p.coarse_cap = (p.coarse_cap + 1) / 2 * 2;
         p.fine_cap = b.hi_topblocks * b.hi_block;
+    } else if (dense) {
+        // the tensor-core scoring's slots span the union of its rows' middles
+        // in whole tiles
+        p.fine_cap = (max_len + LSA_TC_TOKENS - 1) / LSA_TC_TOKENS * LSA_TC_TOKENS;
     } else {
         p.fine_cap = max_len;
     }
@@ -810,7 +814,9 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b, bool dense) {
         p.off_cand = off;
         off = align256(off + (size_t)n_q * p.fine_cap * 8);
         p.off_count = off;
-        off = align256(off + (size_t)n_q * LSA_TC_MAX_SPLITS * 8);
+        off = align256(off + (size_t)n_q * LSA_TC_MAX_SPLITS * LSA_TC_SEGS * 8);
+        p.off_ghist = off;
+        off = align256(off + (size_t)n_q * LSA_TC_BINS * 4);
     } else {
         off = align256(off + (size_t)n_q * p.fine_cap * 4);
     }

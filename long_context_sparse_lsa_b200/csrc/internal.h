@@ -85,7 +85,9 @@ struct IndexArgs {
     int32_t* n_kept;        // [n_q]
     uint32_t* fine_keys;    // [n_q][fine_cap] token keys (score + 1, 0 = none)
     uint64_t* cand;         // prefill chunks: [n_q][fine_cap] candidate pairs (key << 32 | position)
-    int32_t* cand_seg;      // prefill chunks: [n_q][LSA_TC_MAX_SPLITS][2] (first slot, count) per token split
+    int32_t* cand_seg;      // prefill chunks: [n_q][LSA_TC_MAX_SPLITS][4][2] (first slot, count) per token split
+                            // and lane quarter of the scoring
+    uint32_t* ghist;        // prefill chunks: [n_q][LSA_TC_BINS] candidate-filter counts over all splits
     int32_t tc_splits;      // prefill chunks: token splits of the tensor-core scoring
     int32_t coarse_cap, fine_cap;
     // selection: keys of one CTA's slice staged in shared memory (0 = read
@@ -98,7 +100,7 @@ struct IndexPlan {
     int cluster = 8;                          // CTAs per query row in the selection kernels
     int coarse_stage = 0, fine_stage = 0, kept_slots = 0;
     size_t smem_blocks = 0, smem_tokens = 0;  // dynamic smem of the selection kernels
-    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0, off_cand = 0, off_count = 0;
+    size_t off_coarse = 0, off_kept = 0, off_nkept = 0, off_fine = 0, off_cand = 0, off_count = 0, off_ghist = 0;
     size_t ws_bytes = 0;
 };
 // dense: the batch is a prefill chunk scored by the tensor-core contraction
@@ -115,6 +117,9 @@ bool tensor_map_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_
 cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
 // Token splits of each 16-row tile in the tensor-core scoring (<= LSA_TC_MAX_SPLITS).
 #define LSA_TC_MAX_SPLITS 16
+#define LSA_TC_SEGS 4     // candidate segments per token split (one per TMEM lane quarter)
+#define LSA_TC_BINS 256   // candidate-filter histogram bins per row
+#define LSA_TC_TOKENS 128 // cached tokens per tensor-core tile
 int prefill_tc_splits(int n_q);
 // HI block selection computes the coarse scores itself when each cluster
 // CTA's slice of blocks fits in shared memory, the query has at most 16
@@ -149,12 +154,37 @@ struct PointArgs {
 };
 cudaError_t launch_point_scores(const PointArgs& p, int d_I, cudaStream_t stream);
 
+// Draft-row groups (draft_union.cu): the union of each group's index sets.
+constexpr int kMaxGroupRows = 8;
+struct UnionArgs {
+    const int32_t* sets;     // [n_groups * group_rows][budget]
+    const int32_t* q_seq;
+    const int32_t* q_len;
+    const int64_t* kv_offset;
+    const int32_t* seq_lens;
+    int32_t* union_pos;      // [n_groups][union_cap] positions, ascending
+    uint8_t* union_msk;      // [n_groups][union_cap] rows of the group holding each position (bit j: row j)
+    int32_t* union_len;      // [n_groups]
+    int32_t* dev_status;
+    int64_t total_tokens;
+    int32_t n_groups, group_rows, budget, union_cap, n_seq, max_len;
+};
+size_t union_smem_bytes(int group_rows, int budget);
+cudaError_t launch_union_sets(const UnionArgs& u, cudaStream_t stream);
+
+// Context-parallel attention (context_parallel.cu).
+cudaError_t launch_shard_sets(const int32_t* sets, int n_q, int budget, int lo, int hi, int32_t* local,
+                              int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows, int d, float* out,
+                           float* lse_out, cudaStream_t stream);
+
 // ---- sparse attention -----------------------------------------------------
 struct AttendArgs {
     const uint16_t* q[kMaxLayers];
     const uint16_t* k[kMaxLayers];
     const uint16_t* v[kMaxLayers];
     float* out[kMaxLayers];
+    float* lse[kMaxLayers];  // optional: ln of the softmax denominator per (row, query head)
     const int32_t* sets;
     const int64_t* kv_offset;
     const int32_t* seq_lens;
@@ -172,6 +202,11 @@ struct AttendArgs {
     float scale_log2;     // log2(e) / sqrt(d)
     int32_t kv_fp8;       // K/V caches hold FP8 E4M3 codes (k, v point at bytes)
     float kscale[kMaxLayers], vscale[kMaxLayers];  // FP8: value = scale * E4M3(code)
+    // draft-row groups (attend_group_kernel): the union of each group's sets
+    const int32_t* union_pos;
+    const uint8_t* union_msk;
+    const int32_t* union_len;
+    int32_t group_rows, union_cap;
 };
 
 struct AttendPlan {
@@ -183,6 +218,9 @@ struct AttendPlan {
 AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms,
                        bool fp8 = false);
 cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
+// Draft-row groups: the union's splits, shared memory and workspace.
+AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int budget, int G, int num_sms);
+cudaError_t launch_attend_grouped(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
 
 int device_sm_count();
 

@@ -162,6 +162,7 @@ STREAM_Q_IDX = 1
 STREAM_K_IDX = 2
 STREAM_W = 3
 STREAM_LENS = 4
+STREAM_DRAFT = 5  # which indexer-query elements a later draft row copies from the first
 STREAM_Q = 16   # + layer
 STREAM_K = 32   # + layer
 STREAM_V = 48   # + layer

@@ -1,4 +1,4 @@
-"""The five synthetic workloads of the LSA hot path and their seeded tensors.
+"""The synthetic workloads of the LSA hot path and their seeded tensors.
 
 Shapes follow the pages' serving picture (a 69B / 3B-active MoE with native
 1,024K context served on one node: "LongCat-Flash-Lite-Sparse (aitrends.kr)",
@@ -37,6 +37,8 @@ class Workload:
     prefill_new: int = 0           # > 0: a causal prefill chunk of this many tokens on sequence 0
     drafts: int = 1                # decode rows per sequence (several draft tokens, MTP-style):
                                    # row j of a sequence of L tokens sees L - drafts + 1 + j
+    draft_share: int = 0           # percent of each later draft row's indexer-query elements (and all of
+                                   # its head weights, when > 0) taken from the sequence's first draft row
     note: str = field(default="", compare=False)
 
     @property
@@ -70,6 +72,12 @@ BATCH128K = Workload("decode_b16_128k_hi64x256", 1, (131072,) * 16, 16, 128, -16
                      64, 256, 32, 4, 128, 1, note="batched decode, 16 seqs x 131072, HI 64x256")
 CTX1M = Workload("decode_b1_1m_cli4_hi128x512", 2, (1048576,), 16, 128, -16, 15, 8, 64, 2048, 2048,
                  128, 512, 32, 4, 128, 4, note="1M decode, G=4 layers per index set, HI 128x512")
+# Draft rows: 4 sequences x 4 draft tokens on the 128K shape (16 decode rows,
+# as the batched case); later drafts share 75% of the first draft's indexer
+# query elements.
+DRAFTS128K = Workload("decode_b4x4_128k_drafts_hi64x256", 5, (131072,) * 4, 16, 128, -16, 15, 8, 64, 1024, 2048,
+                      64, 256, 32, 4, 128, 1, drafts=4, draft_share=75,
+                      note="4 seqs x 4 draft rows, 131072 tokens, HI 64x256, drafts share 75% of the indexer query")
 PREFILL = Workload("prefill_8192_on_262144", 3, (262144 + 8192,), 16, 128, -16, 15, 8, 64, 1024, 2048,
                    0, 0, 32, 4, 128, 1, prefill_new=8192,
                    note="causal prefill chunk of 8192 tokens on a 262144-token cache, HI off")
@@ -95,7 +103,7 @@ def ragged() -> Workload:
 
 
 def all_workloads() -> list[Workload]:
-    return [TINY, BATCH128K, CTX1M, PREFILL, ragged(), PROFILE32K, PREFILL_PROFILE]
+    return [TINY, BATCH128K, CTX1M, PREFILL, ragged(), PROFILE32K, PREFILL_PROFILE, DRAFTS128K]
 
 
 def by_name(name: str) -> Workload:
@@ -156,6 +164,14 @@ def make(wl: Workload, device, layers: int | None = None, with_kv: bool = True) 
     q_idx = gen.uniform_int8((n_q, wl.H_I, wl.d_I), wl.qk_lo, wl.qk_hi, s, gen.STREAM_Q_IDX, device)
     k_idx = gen.uniform_int8((T, wl.d_I), wl.qk_lo, wl.qk_hi, s, gen.STREAM_K_IDX, device)
     w = gen.uniform_weights((n_q, wl.H_I), wl.w_hi, s, gen.STREAM_W, device)
+    if wl.drafts > 1 and wl.draft_share > 0 and not wl.prefill_new:
+        # draft tokens of one sequence ask for similar context: later drafts
+        # copy a share of the first draft's indexer query and its weights
+        D = wl.drafts
+        pick = gen.uniform_int8((n_q, wl.H_I, wl.d_I), 0, 99, s, gen.STREAM_DRAFT, device) < wl.draft_share
+        first = torch.arange(n_q, device=device) // D * D
+        q_idx = torch.where(pick, q_idx[first], q_idx)
+        w = w[first].clone()
     q, k, v = [], [], []
     for g in range(G):
         q.append(gen.normal_bf16((n_q, wl.H_q, wl.d), s, gen.STREAM_Q + g, device))

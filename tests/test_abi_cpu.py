@@ -202,3 +202,39 @@ def test_noalloc_refuses_shapes_beyond_its_scratch_before_launch():
     need = lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 8192, 1)
     assert need > 8 << 20
     assert lib.lsa_attend_noalloc(arr, arr, arr, 32, 4, 128, P, 8192, ctypes.byref(b), 1, arr, None, None) == 2
+
+
+def test_grouped_attention_rejects_and_counts_before_launch():
+    """lsa_attend_grouped: group sizes, divisibility, GQA width and the
+    union's shared memory are checked before any launch."""
+    lib = lsa.load_library()
+    b = _batch(n_q=16, max_len=131072, total=4 * 131072)
+    arr = (ctypes.c_void_p * 1)(P)
+    f = lib.lsa_attend_grouped
+    args = lambda H_q=32, H_kv=4, budget=3136, D=4, ws=1 << 40: (arr, arr, arr, H_q, H_kv, 128, P, budget,
+                                                                 ctypes.byref(b), 1, D, arr, P, ws, None, None)
+    assert f(*args(D=3)) == 1                       # 16 rows are not groups of 3
+    assert f(*args(D=16)) == 2                      # at most 8 rows per group
+    assert f(*args(H_q=64)) == 2                    # GQA groups of at most 8 query heads
+    assert f(*args(D=8, budget=16384)) == 2         # the union's staging would not fit in shared memory
+    assert f(*args(ws=16)) == 4                     # workspace too small
+    need = lib.lsa_attend_grouped_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 1, 4)
+    # the unions (positions, masks, lengths of 4 groups) come on top of the split partials
+    assert need >= lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 1) // 4 + 4 * 4 * 3136 * 5
+    assert lib.lsa_attend_grouped_launches(ctypes.byref(b), 32, 4, 128, 3136, 1, 4) == 3
+    assert lib.lsa_attend_grouped_launches(ctypes.byref(b), 32, 4, 128, 3136, 1, 3) == 0
+
+
+def test_context_parallel_calls_reject_before_launch():
+    lib = lsa.load_library()
+    assert lib.lsa_shard_sets(P, 4, 100, 10, 5, P + 4096, None, None) == 1      # hi < lo
+    assert lib.lsa_shard_sets(P, 4, 100, 0, 5, P, None, None) == 1              # in place
+    assert lib.lsa_shard_sets(P, 4, 1 << 20, 0, 5, P + 4096, None, None) == 2   # budget too large
+    assert lib.lsa_shard_sets(P, 0, 100, 0, 5, P + 4096, None, None) == 0       # nothing to do
+    assert lib.lsa_combine(P, P, 0, 10, 128, P, None, None) == 1                # no parts
+    assert lib.lsa_combine(P, P, 2, 10, 126, P, None, None) == 1                # d % 4
+    assert lib.lsa_combine(P, P, 2, 0, 128, P, None, None) == 0                 # no rows
+    b = _batch(n_q=16, max_len=131072, total=16 * 131072)
+    arr = (ctypes.c_void_p * 1)(P)
+    assert lib.lsa_attend_lse(arr, arr, arr, 32, 4, 128, P, 3136, ctypes.byref(b), 1, arr, None, P, 1 << 30,
+                              None, None) == 1                                  # lse is required

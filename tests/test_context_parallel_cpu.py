@@ -2,7 +2,10 @@
 ranks, each holding one token range of the caches, through the exchange and
 stage logic of long_context_sparse_lsa_b200.context_parallel, must equal the
 single-device oracle's set bit for bit, including when many scores tie
-across the two ranges (the lower position must win across ranks too).
+across the two ranges (the lower position must win across ranks too); and
+the attention over such a set, each rank attending over its own entries and
+the partials combined by their log-sum-exp after one all-gather, must equal
+the oracle's attention over the whole set.
 
 The library's kernels need a GPU; here each rank's scores come from the
 oracle (its fine and coarse score functions on the rank's own keys) and the
@@ -98,6 +101,121 @@ def _rank_main(rank: int, world: int, port: int, name: str, out):
         dist.barrier()
     finally:
         dist.destroy_process_group()
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def numpy_shard(sets: torch.Tensor, lo: int, hi: int) -> torch.Tensor:
+    s = sets.numpy()
+    out = np.full_like(s, -1)
+    for r in range(s.shape[0]):
+        keep = s[r][(s[r] >= lo) & (s[r] < hi)] - lo
+        out[r, : keep.size] = keep
+    return torch.from_numpy(out)
+
+
+def numpy_partial(q, k, v, local_sets, n_tokens):
+    """Softmax attention over each row's local entries in fp64 (scale
+    1/sqrt(d), q head h -> kv head h // (H_q / H_kv)): the normalised output
+    and ln of the denominator (-inf and zeros for no entry)."""
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k[0].shape[1]
+    ratio = H_q // H_kv
+    out = np.zeros((G, n_q, H_q, d))
+    lse = np.full((G, n_q, H_q), -np.inf)
+    s = local_sets.numpy()
+    for g in range(G):
+        qg, kg, vg = (bf16_to_f64(x[g].view(torch.int16).numpy().view(np.uint16)) for x in (q, k, v))
+        for r in range(n_q):
+            e = s[r][s[r] >= 0]
+            if e.size == 0:
+                continue
+            for h in range(H_q):
+                sc = kg[e, h // ratio] @ qg[r, h] / np.sqrt(d)
+                m = sc.max()
+                p = np.exp(sc - m)
+                out[g, r, h] = p @ vg[e, h // ratio] / p.sum()
+                lse[g, r, h] = m + np.log(p.sum())
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def numpy_combine(o_parts: torch.Tensor, lse_parts: torch.Tensor) -> torch.Tensor:
+    o, l = o_parts.numpy(), lse_parts.numpy()
+    M = l.max(axis=0)
+    wgt = np.where(np.isfinite(l), np.exp(l - np.where(np.isfinite(M), M, 0.0)), 0.0)
+    den = wgt.sum(axis=0)
+    out = (wgt[..., None] * o).sum(axis=0) / np.where(den > 0, den, 1.0)[..., None]
+    return torch.from_numpy(out)
+
+
+def _attend_rank_main(rank: int, world: int, port: int, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # one sequence of 3000 tokens, G = 2, three decode rows whose sets
+        # (from the oracle's index) spread over both token ranges; a fourth
+        # row's set holds only sink tokens (rank 1 has none of them)
+        base = wls.small(wls.BATCH128K, name="cpa", lens=(3000,), G=2)
+        wl = wls.small(base, lens=(3000,), drafts=3, hi_block=64, hi_topblocks=10, sink=16, window=64, topk=200,
+                       seed=75)
+        t = wls.make(wl, "cpu")
+        orc = oracle.get()
+        L = wl.lens[0]
+        sets = []
+        for r in range(wl.n_q):
+            Lr = int(t.q_len[r])
+            sets.append(orc.index_query(t.q_idx[r].numpy(), t.w[r].numpy(), t.k_idx.numpy(), Lr, wl.sink,
+                                        wl.window, wl.topk, wl.hi_block, wl.hi_topblocks))
+        sink_only = np.full_like(sets[0], -1)
+        sink_only[:5] = np.arange(5)
+        sets = np.stack(sets + [sink_only]).astype(np.int32)
+        q = [torch.cat([x, x[:1]]) for x in t.q]  # the fourth row reuses row 0's query
+        bounds = cp.shard_bounds(L, world, 64)
+        lo, hi = bounds[rank]
+        att = cp.ContextParallelAttention(bounds, rank, shard=numpy_shard, partial=numpy_partial,
+                                          combine=numpy_combine)
+        got = att.attend(q, [x[lo:hi] for x in t.k], [x[lo:hi] for x in t.v], torch.from_numpy(sets)).numpy()
+        want = []
+        for g in range(wl.G):
+            kk, vv = (x[g].view(torch.int16).numpy().view(np.uint16) for x in (t.k, t.v))
+            qq = q[g].view(torch.int16).numpy().view(np.uint16)
+            want.append(np.stack([orc.attend_query(qq[r], kk, vv, sets[r]) for r in range(sets.shape[0])]))
+        out.put((rank, float(np.abs(got - np.stack(want)).max())))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_attention_equals_the_whole_set():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_attend_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # the combination is exact: the fp64 partials combine to the oracle's
+    # fp64 attention up to rounding
+    assert all(err < 1e-9 for _, err in res), res
+
+
+def test_combine_of_one_part_is_that_part_and_empty_parts_drop_out():
+    rng = np.random.default_rng(3)
+    o = torch.from_numpy(rng.normal(size=(3, 5, 8)))
+    lse = torch.from_numpy(rng.normal(size=(3, 5)))
+    lse[1] = -np.inf
+    lse[2] = -np.inf
+    np.testing.assert_allclose(numpy_combine(o, lse).numpy(), o[0].numpy())
+    # two parts with equal lse: the mean of their outputs
+    lse2 = torch.zeros((2, 5), dtype=torch.float64)
+    np.testing.assert_allclose(numpy_combine(o[:2], lse2).numpy(), o[:2].mean(0).numpy())
 
 
 @pytest.mark.parametrize("name", sorted(_cases()))
