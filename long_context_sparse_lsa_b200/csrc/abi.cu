@@ -443,7 +443,7 @@ static bool grouped_shape_ok(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv
 
 struct GroupedLayout {
     lsa::AttendPlan p;
-    size_t off_pos, off_msk, off_len, bytes;
+    size_t off_pos, off_msk, off_len, off_split, bytes;
     int cap;
 };
 
@@ -460,6 +460,8 @@ static GroupedLayout grouped_layout(const lsa_batch_t* batch, int32_t H_q, int32
     off = (off + groups * l.cap + 255) / 256 * 256;
     l.off_len = off;
     off = (off + groups * 4 + 255) / 256 * 256;
+    l.off_split = off;
+    off = (off + groups * (l.p.n_splits + 1) * 4 + 255) / 256 * 256;
     l.bytes = off;
     return l;
 }
@@ -512,6 +514,8 @@ lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const*
     u.union_pos = reinterpret_cast<int32_t*>(ws + l.off_pos);
     u.union_msk = ws + l.off_msk;
     u.union_len = reinterpret_cast<int32_t*>(ws + l.off_len);
+    u.union_split = reinterpret_cast<int32_t*>(ws + l.off_split);
+    u.n_splits = l.p.n_splits;
     u.dev_status = dev_status;
     u.total_tokens = batch->total_tokens;
     u.n_groups = batch->n_q / group_rows;
@@ -561,6 +565,7 @@ lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const*
     a.union_pos = u.union_pos;
     a.union_msk = u.union_msk;
     a.union_len = u.union_len;
+    a.union_split = u.union_split;
     a.group_rows = group_rows;
     a.union_cap = l.cap;
     e = lsa::launch_attend_grouped(a, l.p.smem_bytes, cs);

@@ -730,14 +730,16 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
 
 // Draft-row groups: rows come in groups of D consecutive rows of one
 // sequence, and the union of each group's index sets (positions ascending,
-// each with a mask of the rows holding it; union_sets_kernel) is split over
-// the CTAs of the group and kv head. Warp w attends for row w % D over the
-// union tiles w / D, w / D + 8 / D, ...: the D warps of a phase gather the
-// same tiles at the same time, each its own row's members (the others read as
-// masked), so a K/V row held by several rows of the group is fetched from L2
-// once per CTA and from L1 by the others. The tile loop, the fragments and the
-// softmax are attend_rk_kernel's (bf16 caches, GQA groups of at most 8 query
-// heads); the partials merge as lsa_attend's.
+// each with a mask of the rows holding it; union_sets_kernel) is split into
+// stretches of equal work (members summed over the rows) over the CTAs of the
+// group and kv head. A CTA lists each
+// row's members of its stretch (in position order); warp w attends for row
+// w % D over the 16-entry tiles w / D, w / D + 8 / D, ... of that list. The D
+// warps of a phase so walk the same stretch of positions together, and a K/V
+// row held by several rows of the group is fetched from L2 once per CTA and
+// from L1 by the others. The tile loop, the fragments and the softmax are
+// attend_rk_kernel's (bf16 caches, GQA groups of at most 8 query heads); the
+// partials merge as lsa_attend's.
 __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(const __grid_constant__ AttendArgs a) {
     constexpr int NT = 1;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -767,27 +769,56 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(con
         float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
         for (int i = lane; i < ratio * kD; i += kWarp) orow[i] = 0.f;
     }
-    // this CTA's part of the union, as one entry list per row (other rows'
-    // members read as -1)
+    // this CTA's part of the union, split into one list per row: the row's
+    // members in union (= position) order, so the D warps of a phase walk the
+    // same stretch of positions together
     const int U = min(max(a.union_len[grp], 0), a.union_cap);
-    const int e0 = (int)((int64_t)U * split / a.n_splits);
-    const int n_local = min((int)((int64_t)U * (split + 1) / a.n_splits) - e0, a.entries_per_split);
-    const int n_tiles = (n_local + kTile - 1) / kTile;
-    const int stride = a.entries_per_split;  // per-row list length in shared memory
+    const int32_t* cut = a.union_split + (int64_t)grp * (a.n_splits + 1) + split;
+    const int e0 = min(max(cut[0], 0), U);
+    const int n_local = min(min(max(cut[1], e0), U) - e0, a.entries_per_split);
+    const int stride = a.entries_per_split;  // per-row list capacity in shared memory
     int32_t* s_rows = reinterpret_cast<int32_t*>(smem);
+    __shared__ uint32_t s_cnt[kConsumers][kMaxGroupRows];  // members per (warp, row) of a chunk
+    __shared__ uint32_t s_tot[kMaxGroupRows];              // members per row so far
+    if (tid < kMaxGroupRows) s_tot[tid] = 0u;
     const int32_t* up = a.union_pos + (int64_t)grp * a.union_cap + e0;
     const uint8_t* um = a.union_msk + (int64_t)grp * a.union_cap + e0;
-    for (int i = tid; i < n_tiles * kTile; i += kConsumers * kWarp) {
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int c0 = 0; c0 < n_local; c0 += kConsumers * kWarp) {
+        const int i = c0 + tid;
         const int p = i < n_local ? up[i] : -1;
-        const uint32_t m = i < n_local ? um[i] : 0u;
-        for (int j = 0; j < D; ++j) s_rows[j * stride + i] = ((m >> j) & 1u) && p >= 0 ? p : -1;
+        const uint32_t m = i < n_local && p >= 0 ? um[i] : 0u;
+        uint32_t bal[kMaxGroupRows];
+#pragma unroll
+        for (int j = 0; j < kMaxGroupRows; ++j) {
+            bal[j] = __ballot_sync(0xffffffffu, j < D && ((m >> j) & 1u));
+            if (lane == 0) s_cnt[warp][j] = __popc(bal[j]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kMaxGroupRows; ++j) {
+            if (j < D && ((m >> j) & 1u)) {
+                uint32_t before = s_tot[j];
+                for (int w = 0; w < warp; ++w) before += s_cnt[w][j];
+                s_rows[j * stride + before + __popc(bal[j] & lt_mask)] = p;
+            }
+        }
+        __syncthreads();
+        if (tid < D) {
+            uint32_t add = 0;
+            for (int w = 0; w < kConsumers; ++w) add += s_cnt[w][tid];
+            s_tot[tid] += add;
+        }
+        __syncthreads();
     }
-    __syncthreads();
+    const int n_mine = (int)s_tot[jr];  // this warp's row: members in this CTA's stretch
+    const int n_tiles = (n_mine + kTile - 1) / kTile;
     int32_t* s_ent = s_rows + jr * stride;
-    if (bad) {  // nothing of an invalid row is read (its entries were checked against nothing)
+    for (int i = n_mine + lane; i < n_tiles * kTile; i += kWarp) s_ent[i] = -1;  // pad the last tile
+    if (bad) {  // nothing of an invalid row is read
         for (int i = lane; i < n_tiles * kTile; i += kWarp) s_ent[i] = -1;
     } else {
-        for (int i = lane; i < n_tiles * kTile; i += kWarp)
+        for (int i = lane; i < n_mine; i += kWarp)
             if (s_ent[i] >= L) s_ent[i] = -1;  // the union holds only members; a row never reads past q_len
     }
     __syncthreads();
@@ -1014,7 +1045,9 @@ AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int b
     if (splits < min_splits) splits = min_splits;
     if (splits < 1) splits = 1;
     p.n_splits = splits;
-    int eps = (cap + splits - 1) / splits;  // a CTA's share of the longest union
+    // a stretch of equal work holds at most ceil(work / splits) + D entries
+    // (every entry has a member; the last may carry D): its list capacity
+    int eps = (cap + splits - 1) / splits + group_rows;
     eps = (eps + kTile - 1) / kTile * kTile;
     if (eps < kTile) eps = kTile;
     p.entries_per_split = eps;

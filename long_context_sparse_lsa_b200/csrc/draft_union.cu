@@ -16,7 +16,9 @@
 // row's entries in the chunk set bits of a per-row bitmap, then each thread
 // takes two 32-position words, ORs the rows' words, and a CTA prefix sum of
 // the bit counts places its positions (ascending) and their row masks in the
-// output. Duplicate entries of one row count once.
+// output. Duplicate entries of one row count once. Last, a prefix sum of the
+// masks' member counts cuts the union into the attention's splits of equal
+// work.
 #include "common.cuh"
 #include "internal.h"
 
@@ -61,6 +63,7 @@ __global__ void __launch_bounds__(kUnThreads, 1) union_sets_kernel(const __grid_
             flag(u.dev_status, LSA_DEV_BAD_SEQ);
             u.union_len[grp] = 0;
         }
+        for (int sp = tid; sp <= u.n_splits; sp += kUnThreads) u.union_split[(int64_t)grp * (u.n_splits + 1) + sp] = 0;
         return;
     }
     int l_max = 0;
@@ -135,8 +138,49 @@ __global__ void __launch_bounds__(kUnThreads, 1) union_sets_kernel(const __grid_
         base += total;
         __syncthreads();  // the bitmaps and s_warp are rewritten by the next chunk
     }
+    // The attention splits the union into n_splits stretches of equal work
+    // (members summed over the rows, not entries: the window run is held by
+    // every row, the selected tokens by few). The members before each entry
+    // go to shared memory (over the staged lists, no longer needed), then
+    // thread s finds the first entry of stretch s by binary search.
+    const int U = (int)min(base, (uint32_t)u.union_cap);
+    int32_t* cum = lists;  // U <= D x budget entries
+    __syncthreads();       // the masks written above are visible to the whole CTA
+    uint32_t run = 0;
+    for (int c0 = 0; c0 < U; c0 += kUnThreads) {
+        const int k = c0 + tid;
+        const uint32_t w = k < U ? (uint32_t)__popc(out_msk[k]) : 0u;
+        uint32_t incl = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_warp[warp] = incl;
+        __syncthreads();
+        uint32_t before = 0, total = 0;
+        for (int w2 = 0; w2 < kUnWarps; ++w2) {
+            const uint32_t c = s_warp[w2];
+            before += w2 < warp ? c : 0u;
+            total += c;
+        }
+        if (k < U) cum[k] = (int32_t)(run + before + incl - w);
+        run += total;
+        __syncthreads();
+    }
     pdl_trigger();
-    if (tid == 0) u.union_len[grp] = (int32_t)min(base, (uint32_t)u.union_cap);
+    int32_t* split = u.union_split + (int64_t)grp * (u.n_splits + 1);
+    for (int sp = tid; sp <= u.n_splits; sp += kUnThreads) {
+        const int64_t target = (int64_t)run * sp / u.n_splits;
+        int lo = 0, hi = U;  // first entry whose members-before reach the target (U if none)
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)cum[mid] >= target) hi = mid;
+            else lo = mid + 1;
+        }
+        split[sp] = sp == u.n_splits ? U : lo;
+    }
+    if (tid == 0) u.union_len[grp] = U;
 }
 
 }  // namespace

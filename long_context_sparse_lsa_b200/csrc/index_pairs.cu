@@ -14,9 +14,12 @@
 namespace lsa {
 namespace {
 
-constexpr int kTkThreads = 1024;
+// 512 threads and at most 64 registers: two rows' CTAs per SM, so one row's
+// barriers and L2 round trips overlap the other's
+constexpr int kTkThreads = 512;
 constexpr int kTkWarps = kTkThreads / kWarp;
-static_assert(kHistBins / kTkThreads == 4, "the scan gives each thread one 4-bin vector");
+constexpr int kTkBinsPer = kHistBins / kTkThreads;  // histogram bins per thread in a scan
+static_assert(kTkBinsPer % 4 == 0, "the scan reads each thread's bins as 4-bin vectors");
 constexpr int kTkCandCap = 2048;  // keys of the threshold bin held in the candidate list
 constexpr int kTkDigitBits = 12;
 constexpr int kPassUnroll = 8;  // pair loads in flight per thread in a pass
@@ -36,14 +39,13 @@ __device__ __forceinline__ uint32_t tk_warp_sum(uint32_t v) {
 // memory (histogram pass, then radix digits over the threshold bin's
 // candidates or, for a bin too full for the list, over all pairs); the kept
 // positions are sorted ascending in shared memory (bitonic) and written with
-// the SI sink and window runs. One CTA of 1024 threads per row.
+// the SI sink and window runs. One CTA of 512 threads per row.
 constexpr int kPairSortCap = LSA_MAX_BUDGET;  // topk <= budget
 
 struct PairShared {
     uint32_t hist[kHistBins];
     uint64_t cand[kTkCandCap];
     uint32_t wsum[kTkWarps];
-    uint32_t wsum2[kTkWarps];
     uint32_t bin, above, in_bin;
     uint32_t n_cand, n_sel;
 };
@@ -52,14 +54,24 @@ __device__ __forceinline__ uint64_t pair_value(uint64_t e) {
     return (e & 0xffffffff00000000ull) | (uint64_t)(0xffffffffu - (uint32_t)e);
 }
 
-// Suffix scan of sh.hist (4 bins per thread). Returns the number of counted
-// keys; when 1 <= krem <= total sets sh.bin / sh.above / sh.in_bin to the bin
-// holding the krem-th largest value, the count above it and the count in it.
+// Suffix scan of sh.hist (kTkBinsPer bins per thread). Returns the number of
+// counted keys; when 1 <= krem <= total sets sh.bin / sh.above / sh.in_bin to
+// the bin holding the krem-th largest value, the count above it and the count
+// in it.
 __device__ uint32_t pair_find_bin(PairShared& sh, uint32_t krem) {
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
-    const uint4 h = reinterpret_cast<const uint4*>(sh.hist)[tid];
-    const uint32_t c[4] = {h.x, h.y, h.z, h.w};
-    const uint32_t own = c[0] + c[1] + c[2] + c[3];
+    uint32_t c[kTkBinsPer];
+#pragma unroll
+    for (int q = 0; q < kTkBinsPer / 4; ++q) {
+        const uint4 h = reinterpret_cast<const uint4*>(sh.hist)[tid * (kTkBinsPer / 4) + q];
+        c[4 * q] = h.x;
+        c[4 * q + 1] = h.y;
+        c[4 * q + 2] = h.z;
+        c[4 * q + 3] = h.w;
+    }
+    uint32_t own = 0;
+#pragma unroll
+    for (int j = 0; j < kTkBinsPer; ++j) own += c[j];
     uint32_t x = own;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -68,16 +80,16 @@ __device__ uint32_t pair_find_bin(PairShared& sh, uint32_t krem) {
     }
     if (lane == 0) sh.wsum[wid] = x;
     __syncthreads();
-    const uint32_t wt = sh.wsum[lane];
+    const uint32_t wt = lane < kTkWarps ? sh.wsum[lane] : 0u;
     const uint32_t later = tk_warp_sum(lane > wid ? wt : 0u);
     const uint32_t total = tk_warp_sum(wt);
     const uint32_t S = x + later;
     if (krem >= 1u && S >= krem && S - own < krem) {
         uint32_t run = S - own;
 #pragma unroll
-        for (int j = 3; j >= 0; --j) {
+        for (int j = kTkBinsPer - 1; j >= 0; --j) {
             if (run + c[j] >= krem) {
-                sh.bin = (uint32_t)(4 * tid + j);
+                sh.bin = (uint32_t)(kTkBinsPer * tid + j);
                 sh.above = run;
                 sh.in_bin = c[j];
                 break;
@@ -133,7 +145,9 @@ __device__ uint32_t select_sorted(PairShared& sh, int32_t* sel, uint32_t n, uint
             const int width = shift < kTkDigitBits ? shift : kTkDigitBits;
             shift -= width;
             const uint64_t mask = (1ull << width) - 1ull;
-            reinterpret_cast<uint4*>(sh.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int q = 0; q < kTkBinsPer / 4; ++q)
+                reinterpret_cast<uint4*>(sh.hist)[tid * (kTkBinsPer / 4) + q] = make_uint4(0u, 0u, 0u, 0u);
             __syncthreads();
             if (listed) {
                 for (uint32_t i = tid; i < nc; i += kTkThreads) {
@@ -167,9 +181,8 @@ __device__ uint32_t select_sorted(PairShared& sh, int32_t* sel, uint32_t n, uint
     while (P < m) P <<= 1;
     for (uint32_t i = m + tid; i < P; i += kTkThreads) sel[i] = 0x7fffffff;
     __syncthreads();
-    // (with one pair per thread, a stride of at most 32 keeps each warp inside
-    // its own 64 elements: a warp barrier suffices between two such steps)
-    const bool one_pair = P <= 2u * kTkThreads;
+    // (a stride of at most 32 keeps each warp inside its own 64-element blocks
+    // 64 (w + m kTkWarps): a warp barrier suffices between two such steps)
     for (uint32_t size = 2; size <= P; size <<= 1) {
         for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
             for (uint32_t i = tid; i < P / 2; i += kTkThreads) {
@@ -185,14 +198,14 @@ __device__ uint32_t select_sorted(PairShared& sh, int32_t* sel, uint32_t n, uint
             // the next step stays inside the warp's 64 elements too: a stride
             // halved, or (after stride 1) the next size's first stride <= 32
             const bool next_local = stride > 1u || (size < P && size <= 32u);
-            if (one_pair && stride <= 32u && next_local) __syncwarp();
+            if (stride <= 32u && next_local) __syncwarp();
             else __syncthreads();
         }
     }
     return m;
 }
 
-__global__ void __launch_bounds__(kTkThreads, 1) topk_pairs_kernel(const __grid_constant__ IndexArgs a) {
+__global__ void __launch_bounds__(kTkThreads, 2) topk_pairs_kernel(const __grid_constant__ IndexArgs a) {
     extern __shared__ __align__(16) uint8_t pr_dyn[];
     PairShared& sh = *reinterpret_cast<PairShared*>(pr_dyn);
     int32_t* sel = reinterpret_cast<int32_t*>(pr_dyn + (sizeof(PairShared) + 15) / 16 * 16);
@@ -275,7 +288,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_pairs_kernel(const __grid_
 // for an empty slot; the ids of the k largest values (score desc, id asc) are
 // written ascending to out[r][0, m), -1 after, and (out_values) their values
 // in the same order, 0 after.
-__global__ void __launch_bounds__(kTkThreads, 1) merge_pairs_kernel(const uint64_t* __restrict__ pairs,
+__global__ void __launch_bounds__(kTkThreads, 2) merge_pairs_kernel(const uint64_t* __restrict__ pairs,
                                                                     const int32_t* __restrict__ counts, int32_t cap,
                                                                     int32_t k, int32_t* __restrict__ out,
                                                                     uint64_t* __restrict__ out_values,

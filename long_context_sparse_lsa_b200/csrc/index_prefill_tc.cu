@@ -354,16 +354,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
 #pragma unroll
                 for (int h = 0; h < H_I; ++h) acc4[h & 3] += max((int32_t)v[rr * H_I + h], 0) * w[rr * H_I + h];
                 const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                const bool in = t >= rs[i] && t < rws[i];
                 const uint32_t key = (uint32_t)acc + 1u;
-                const bool emit = in && key >= thr[i];
-                if (emit) atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
+                const bool emit = key >= thr[i] && t >= rs[i] && t < rws[i];
                 const uint32_t m = __ballot_sync(0xffffffffu, emit);
-                if (emit) {
-                    const uint32_t slot = cnt[i] + __popc(m & lt_mask);
-                    if ((int64_t)slot < room) cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
+                if (m != 0u) {  // warp-uniform: most chunks of a row emit nothing once its threshold has risen
+                    if (emit) {
+                        atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
+                        const uint32_t slot = cnt[i] + __popc(m & lt_mask);
+                        if ((int64_t)slot < room)
+                            cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
+                    }
+                    cnt[i] += __popc(m);
                 }
-                cnt[i] += __popc(m);
             }
         };
         // Threshold updates of this warp's two query rows (rows 2w', 2w'+1 of

@@ -165,9 +165,10 @@ struct UnionArgs {
     int32_t* union_pos;      // [n_groups][union_cap] positions, ascending
     uint8_t* union_msk;      // [n_groups][union_cap] rows of the group holding each position (bit j: row j)
     int32_t* union_len;      // [n_groups]
+    int32_t* union_split;    // [n_groups][n_splits + 1] first union entry of each attention split
     int32_t* dev_status;
     int64_t total_tokens;
-    int32_t n_groups, group_rows, budget, union_cap, n_seq, max_len;
+    int32_t n_groups, group_rows, budget, union_cap, n_seq, max_len, n_splits;
 };
 size_t union_smem_bytes(int group_rows, int budget);
 cudaError_t launch_union_sets(const UnionArgs& u, cudaStream_t stream);
@@ -206,6 +207,7 @@ struct AttendArgs {
     const int32_t* union_pos;
     const uint8_t* union_msk;
     const int32_t* union_len;
+    const int32_t* union_split;  // [groups][n_splits + 1]: equal shares of the rows' members
     int32_t group_rows, union_cap;
 };
 
