@@ -437,48 +437,27 @@ static bool grouped_shape_ok(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv
     if (!attend_shape_ok(H_q, H_kv, d, budget, G) || H_q / H_kv > 8) return false;
     if (group_rows != 1 && group_rows != 2 && group_rows != 4 && group_rows != 8) return false;
     if (batch->n_q % group_rows != 0 || batch->n_q / group_rows > 65535) return false;
-    if (lsa::union_smem_bytes(group_rows, budget) > 227 * 1024) return false;
-    return true;
-}
-
-struct GroupedLayout {
-    lsa::AttendPlan p;
-    size_t off_pos, off_msk, off_len, off_split, bytes;
-    int cap;
-};
-
-static GroupedLayout grouped_layout(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t budget, int32_t G,
-                                    int32_t group_rows) {
-    GroupedLayout l;
-    l.p = lsa::plan_attend_grouped(batch->n_q, group_rows, H_q, H_kv, budget, G, lsa::device_sm_count());
-    l.cap = group_rows * budget;
-    const size_t groups = (size_t)(batch->n_q / group_rows);
-    size_t off = (l.p.ws_bytes + 255) / 256 * 256;
-    l.off_pos = off;
-    off = (off + groups * l.cap * 4 + 255) / 256 * 256;
-    l.off_msk = off;
-    off = (off + groups * l.cap + 255) / 256 * 256;
-    l.off_len = off;
-    off = (off + groups * 4 + 255) / 256 * 256;
-    l.off_split = off;
-    off = (off + groups * (l.p.n_splits + 1) * 4 + 255) / 256 * 256;
-    l.bytes = off;
-    return l;
+    const lsa::AttendPlan p =
+        lsa::plan_attend_grouped(batch->n_q, group_rows, H_q, H_kv, budget, G, lsa::device_sm_count());
+    return p.smem_bytes <= 220 * 1024;  // the rows' sets are staged in shared memory
 }
 
 size_t lsa_attend_grouped_workspace_size(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d,
                                          int32_t budget, int32_t layers_per_index, int32_t group_rows) {
     if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1) return 0;
     if (!grouped_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index, group_rows)) return 0;
-    return grouped_layout(batch, H_q, H_kv, budget, layers_per_index, group_rows).bytes;
+    return lsa::plan_attend_grouped(batch->n_q, group_rows, H_q, H_kv, budget, layers_per_index,
+                                    lsa::device_sm_count())
+        .ws_bytes;
 }
 
 int32_t lsa_attend_grouped_launches(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, int32_t budget,
                                     int32_t layers_per_index, int32_t group_rows) {
     if (batch == nullptr || batch->n_q <= 0) return 0;
     if (!grouped_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index, group_rows)) return 0;
-    const GroupedLayout l = grouped_layout(batch, H_q, H_kv, budget, layers_per_index, group_rows);
-    return l.p.n_splits > 1 ? 3 : 2;  // union, attention[, split merge]
+    const lsa::AttendPlan p = lsa::plan_attend_grouped(batch->n_q, group_rows, H_q, H_kv, budget, layers_per_index,
+                                                       lsa::device_sm_count());
+    return p.n_splits > 1 ? 2 : 1;  // attention[, split merge]
 }
 
 lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const* k_cache,
@@ -500,32 +479,10 @@ lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const*
         if (!aligned(q[g], 16) || !aligned(k_cache[g], 16) || !aligned(v_cache[g], 16) || !aligned(out[g], 16))
             return LSA_ERR_INVALID_ARG;
     }
-    const GroupedLayout l = grouped_layout(batch, H_q, H_kv, budget, layers_per_index, group_rows);
-    if (workspace == nullptr || workspace_bytes < l.bytes || !aligned(workspace, 256)) return LSA_ERR_WORKSPACE;
+    const lsa::AttendPlan p = lsa::plan_attend_grouped(batch->n_q, group_rows, H_q, H_kv, budget, layers_per_index,
+                                                       lsa::device_sm_count());
+    if (workspace == nullptr || workspace_bytes < p.ws_bytes || !aligned(workspace, 256)) return LSA_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    lsa::UnionArgs u;
-    std::memset(&u, 0, sizeof u);
-    u.sets = index_sets;
-    u.q_seq = batch->q_seq;
-    u.q_len = batch->q_len;
-    u.kv_offset = batch->kv_offset;
-    u.seq_lens = batch->seq_lens;
-    u.union_pos = reinterpret_cast<int32_t*>(ws + l.off_pos);
-    u.union_msk = ws + l.off_msk;
-    u.union_len = reinterpret_cast<int32_t*>(ws + l.off_len);
-    u.union_split = reinterpret_cast<int32_t*>(ws + l.off_split);
-    u.n_splits = l.p.n_splits;
-    u.dev_status = dev_status;
-    u.total_tokens = batch->total_tokens;
-    u.n_groups = batch->n_q / group_rows;
-    u.group_rows = group_rows;
-    u.budget = budget;
-    u.union_cap = l.cap;
-    u.n_seq = batch->n_seq;
-    u.max_len = batch->max_len;
-    cudaError_t e = lsa::launch_union_sets(u, cs);
-    if (e != cudaSuccess) return cuda_fail(e);
     lsa::AttendArgs a;
     std::memset(&a, 0, sizeof a);
     for (int g = 0; g < layers_per_index; ++g) {
@@ -543,9 +500,9 @@ lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const*
     a.q_len = batch->q_len;
     a.dev_status = dev_status;
     const size_t rows_q = (size_t)layers_per_index * batch->n_q;
-    if (l.p.n_splits > 1) {
+    if (p.n_splits > 1) {
         a.part_o = reinterpret_cast<float*>(ws);
-        const size_t off = (rows_q * l.p.n_splits * H_q * 128 * 4 + 255) / 256 * 256;
+        const size_t off = (rows_q * p.n_splits * H_q * 128 * 4 + 255) / 256 * 256;
         a.part_ml = reinterpret_cast<float*>(ws + off);
     }
     a.total_tokens = batch->total_tokens;
@@ -556,19 +513,15 @@ lsa_status_t lsa_attend_grouped(const uint16_t* const* q, const uint16_t* const*
     a.H_kv = H_kv;
     a.budget = budget;
     a.G = layers_per_index;
-    a.n_splits = l.p.n_splits;
-    a.entries_per_split = l.p.entries_per_split;
-    a.head_groups = H_kv;
-    a.hpc = 1;
-    a.stage_off = l.p.stage_off;
+    a.n_splits = p.n_splits;
+    a.entries_per_split = p.entries_per_split;
+    a.head_groups = p.head_groups;
+    a.hpc = p.hpc;
+    a.rows_per_cta = p.rows_per_cta;
+    a.stage_off = p.stage_off;
     a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
-    a.union_pos = u.union_pos;
-    a.union_msk = u.union_msk;
-    a.union_len = u.union_len;
-    a.union_split = u.union_split;
     a.group_rows = group_rows;
-    a.union_cap = l.cap;
-    e = lsa::launch_attend_grouped(a, l.p.smem_bytes, cs);
+    cudaError_t e = lsa::launch_attend_grouped(a, p.smem_bytes, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 

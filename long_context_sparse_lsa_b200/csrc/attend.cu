@@ -179,13 +179,14 @@ __device__ __forceinline__ void clear_row(const AttendArgs& a, int layer, int r,
 // heads: the final output when there is one split, else one partial. Every
 // thread of the CTA calls it (it holds a CTA barrier); warps >= kConsumers
 // only take part in the barrier.
-// GROUPED (draft-row groups): the warps w % hpc == j work for row r + j of the
-// group (hpc = the group's rows) and all of them for kv head hgrp.
+// GROUPED (draft-row groups): hpc is the CTA's (kv head, row) pairs; the
+// warps w % hpc == key work for kv head hgrp * kvpc + key % kvpc of row
+// r + key / kvpc.
 template <int NT, bool GROUPED = false>
 __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* merge_area, float (&o)[NT][kD / 16][4],
                                                 float (&m_run)[NT][2], float (&l_run)[NT][2], int warp, int lane,
                                                 int hpc, int hgrp, int r, int layer, int split, int ratio,
-                                                float vs = 1.f) {
+                                                float vs = 1.f, int kvpc = 1) {
     const int g = lane >> 2, t4 = lane & 3;
     // ---- merge the consumers of each kv head, in registers ----
     // All warps hold O^T in the same fragment layout, so warps with wsel > 0
@@ -212,7 +213,7 @@ __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* me
     const bool direct = a.n_splits == 1;
     if (warp < kConsumers && wsel_me == 0) {
         const int h_local = warp % hpc;
-        if (GROUPED) r += h_local;
+        if (GROUPED) r += h_local / kvpc;
         const int64_t row_q = (int64_t)layer * a.n_q + r;
         const int n_sel = kConsumers / hpc;
         for (int j = 1; j < n_sel; ++j) {
@@ -238,7 +239,7 @@ __device__ __forceinline__ void merge_and_store(const AttendArgs& a, uint8_t* me
             }
         }
         // write this kv head's query heads: the final output, or one split partial
-        const int kvh = GROUPED ? hgrp : hgrp * hpc + h_local;
+        const int kvh = GROUPED ? hgrp * kvpc + h_local % kvpc : hgrp * hpc + h_local;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
 #pragma unroll
@@ -729,15 +730,18 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
 }
 
 // Draft-row groups: rows come in groups of D consecutive rows of one
-// sequence, and the union of each group's index sets (positions ascending,
-// each with a mask of the rows holding it; union_sets_kernel) is split into
-// stretches of equal work (members summed over the rows) over the CTAs of the
-// group and kv head. A CTA lists each
-// row's members of its stretch (in position order); warp w attends for row
-// w % D over the 16-entry tiles w / D, w / D + 8 / D, ... of that list. The D
-// warps of a phase so walk the same stretch of positions together, and a K/V
-// row held by several rows of the group is fetched from L2 once per CTA and
-// from L1 by the others. The tile loop, the fragments and the softmax are
+// sequence (the draft tokens of a decode step), whose index sets share the
+// sink run, nearly all of the window run and, where the drafts' indexer
+// queries agree, much of the selection. A CTA covers hpc kv heads (whole
+// tokens, as attend_rk_kernel) for rpc rows of a group; it stages those rows'
+// whole sets and cuts every one of them at the same positions: the positions
+// of its first row's entries at n_splits equal steps. Split s of every row is
+// then the stretch of positions between two cuts, so the CTA's rows walk the
+// same positions together and a K/V row that several of them hold is fetched
+// from L2 once and served from L1 to the others. The cuts are taken as
+// indices into each row's set (made non-decreasing), so every entry of a row
+// belongs to exactly one split whatever the set holds: the output is
+// lsa_attend's. The tile loop, the fragments and the softmax are
 // attend_rk_kernel's (bf16 caches, GQA groups of at most 8 query heads); the
 // partials merge as lsa_attend's.
 __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(const __grid_constant__ AttendArgs a) {
@@ -746,13 +750,22 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(con
     const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
     const int g = lane >> 2, t4 = lane & 3;
     const int D = a.group_rows;
-    const int split = blockIdx.x / a.H_kv;
-    const int kvh = blockIdx.x % a.H_kv;
+    // CTA (split, kv-head group, row block): hpc kv heads x rpc rows of the
+    // group, n_ph warps on each (kv head, row); warp w: key w % (hpc rpc)
+    const int hpc = a.hpc, rpc = a.rows_per_cta;
+    const int keys = hpc * rpc;
+    const int row_blocks = D / rpc;
+    const int rb = blockIdx.x % row_blocks;
+    const int hgrp = (blockIdx.x / row_blocks) % a.head_groups;
+    const int split = blockIdx.x / (row_blocks * a.head_groups);
     const int grp = blockIdx.y;
     const int layer = blockIdx.z;
     const int ratio = a.H_q / a.H_kv;
-    const int jr = warp % D;             // this warp's row of the group
-    const int ph = warp / D, n_ph = kConsumers / D;
+    const int key = warp % keys;
+    const int kvh = hgrp * hpc + key % hpc;
+    const int jl = key / hpc;            // this warp's row of the CTA
+    const int jr = rb * rpc + jl;        // ... of the group
+    const int ph = warp / keys, n_ph = kConsumers / keys;
     const int r = grp * D + jr;
     // the row's metadata (the caller's) before the wait
     const int seq = a.q_seq[r];
@@ -763,65 +776,110 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(con
     pdl_enter();
     const bool bad = seq < 0 || seq >= a.n_seq || L < 1 || L > a.max_len || L > slen || off < 0 ||
                      off + slen > a.total_tokens;
-    if (bad && split == 0 && kvh == 0 && layer == 0 && lane == 0 && ph == 0)
+    if (bad && split == 0 && hgrp == 0 && key % hpc == 0 && layer == 0 && lane == 0 && ph == 0)
         flag(a.dev_status, seq < 0 || seq >= a.n_seq ? LSA_DEV_BAD_SEQ : LSA_DEV_BAD_LENGTH);
     if (bad && split == 0 && ph == 0) {  // an invalid row's output is zero
         float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
         for (int i = lane; i < ratio * kD; i += kWarp) orow[i] = 0.f;
     }
-    // this CTA's part of the union, split into one list per row: the row's
-    // members in union (= position) order, so the D warps of a phase walk the
-    // same stretch of positions together
-    const int U = min(max(a.union_len[grp], 0), a.union_cap);
-    const int32_t* cut = a.union_split + (int64_t)grp * (a.n_splits + 1) + split;
-    const int e0 = min(max(cut[0], 0), U);
-    const int n_local = min(min(max(cut[1], e0), U) - e0, a.entries_per_split);
-    const int stride = a.entries_per_split;  // per-row list capacity in shared memory
-    int32_t* s_rows = reinterpret_cast<int32_t*>(smem);
-    __shared__ uint32_t s_cnt[kConsumers][kMaxGroupRows];  // members per (warp, row) of a chunk
-    __shared__ uint32_t s_tot[kMaxGroupRows];              // members per row so far
-    if (tid < kMaxGroupRows) s_tot[tid] = 0u;
-    const int32_t* up = a.union_pos + (int64_t)grp * a.union_cap + e0;
-    const uint8_t* um = a.union_msk + (int64_t)grp * a.union_cap + e0;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    for (int c0 = 0; c0 < n_local; c0 += kConsumers * kWarp) {
-        const int i = c0 + tid;
-        const int p = i < n_local ? up[i] : -1;
-        const uint32_t m = i < n_local && p >= 0 ? um[i] : 0u;
-        uint32_t bal[kMaxGroupRows];
-#pragma unroll
-        for (int j = 0; j < kMaxGroupRows; ++j) {
-            bal[j] = __ballot_sync(0xffffffffu, j < D && ((m >> j) & 1u));
-            if (lane == 0) s_cnt[warp][j] = __popc(bal[j]);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < kMaxGroupRows; ++j) {
-            if (j < D && ((m >> j) & 1u)) {
-                uint32_t before = s_tot[j];
-                for (int w = 0; w < warp; ++w) before += s_cnt[w][j];
-                s_rows[j * stride + before + __popc(bal[j] & lt_mask)] = p;
-            }
-        }
-        __syncthreads();
-        if (tid < D) {
-            uint32_t add = 0;
-            for (int w = 0; w < kConsumers; ++w) add += s_cnt[w][tid];
-            s_tot[tid] += add;
-        }
-        __syncthreads();
-    }
-    const int n_mine = (int)s_tot[jr];  // this warp's row: members in this CTA's stretch
-    const int n_tiles = (n_mine + kTile - 1) / kTile;
-    int32_t* s_ent = s_rows + jr * stride;
-    for (int i = n_mine + lane; i < n_tiles * kTile; i += kWarp) s_ent[i] = -1;  // pad the last tile
-    if (bad) {  // nothing of an invalid row is read
-        for (int i = lane; i < n_tiles * kTile; i += kWarp) s_ent[i] = -1;
-    } else {
-        for (int i = lane; i < n_mine; i += kWarp)
-            if (s_ent[i] >= L) s_ent[i] = -1;  // the union holds only members; a row never reads past q_len
+    // the CTA's rows' whole sets, checked as lsa_attend checks them (entries
+    // below -1 or at or past q_len flagged and skipped; an invalid row's
+    // entries all skipped)
+    const int B = a.budget;
+    const int stride = a.entries_per_split;   // per-row working list: B rounded up to whole tiles
+    int32_t* s_set = reinterpret_cast<int32_t*>(smem);         // [rpc][B]
+    int32_t* s_work = s_set + rpc * B;                         // [rpc][stride]
+    int32_t* s_cut = s_work + rpc * stride;                    // [rpc][n_splits + 1]
+    __shared__ int32_t s_len[kMaxGroupRows];
+    if (tid < rpc) {
+        const int rr = grp * D + rb * rpc + tid;
+        const int sq = a.q_seq[rr], Lr = a.q_len[rr];
+        const int sc = min(max(sq, 0), a.n_seq - 1);
+        const int64_t o2 = a.kv_offset[sc];
+        const int sl = a.seq_lens[sc];
+        const bool ok = sq >= 0 && sq < a.n_seq && Lr >= 1 && Lr <= a.max_len && Lr <= sl && o2 >= 0 &&
+                        o2 + sl <= a.total_tokens;
+        s_len[tid] = ok ? Lr : 0;
     }
     __syncthreads();
+    // (the CTA's rows are consecutive: their sets are one contiguous run,
+    // read with 16-byte loads, all of a thread's in flight together)
+    const int32_t* run = a.sets + (int64_t)(grp * D + rb * rpc) * B;
+    const int n_run = rpc * B;
+    if ((B & 3) == 0 && (reinterpret_cast<uintptr_t>(run) & 15u) == 0) {
+        constexpr int kU = 8;
+        for (int v0 = tid; v0 < n_run / 4; v0 += kConsumers * kWarp * kU) {
+            int4 x[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int v = v0 + u * kConsumers * kWarp;
+                x[u] = v < n_run / 4 ? __ldg(reinterpret_cast<const int4*>(run) + v) : make_int4(-1, -1, -1, -1);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int v = v0 + u * kConsumers * kWarp;
+                if (v < n_run / 4) reinterpret_cast<int4*>(s_set)[v] = x[u];
+            }
+        }
+    } else {
+        for (int i = tid; i < n_run; i += kConsumers * kWarp) s_set[i] = __ldg(run + i);
+    }
+    __syncthreads();
+    bool bad_entry = false;
+    for (int i = tid; i < n_run; i += kConsumers * kWarp) {
+        const int Lj = s_len[i / B];
+        const int32_t e = s_set[i];
+        if (e < -1 || e >= Lj) {
+            bad_entry |= Lj > 0;
+            s_set[i] = -1;
+        }
+    }
+    if (bad_entry) flag(a.dev_status, LSA_DEV_BAD_INDEX);
+    __syncthreads();
+    // the cuts: cut t of row j = the first entry of row j not below position
+    // P_t = the CTA's first row's entry B t / n (a -1 there: no bound); made
+    // non-decreasing in t, so the splits of a row cover its set exactly once
+    const int n_sp = a.n_splits;
+    for (int q = tid; q < rpc * (n_sp + 1); q += kConsumers * kWarp) {
+        const int j = q / (n_sp + 1), t = q - j * (n_sp + 1);
+        int c;
+        if (t == 0) {
+            c = 0;
+        } else if (t == n_sp) {
+            c = B;
+        } else {
+            const int32_t pr = s_set[(int)((int64_t)B * t / n_sp)];
+            const int32_t P = pr >= 0 ? pr : 0x7fffffff;
+            const int32_t* row = s_set + j * B;
+            int lo = 0, hi = B;  // entries in [0, P) form a prefix of an ascending set
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (row[mid] >= 0 && row[mid] < P) lo = mid + 1;
+                else hi = mid;
+            }
+            c = lo;
+        }
+        s_cut[q] = c;
+    }
+    __syncthreads();
+    if (tid < rpc) {
+        int m = 0;
+        for (int t = 0; t <= n_sp; ++t) {
+            m = max(m, s_cut[tid * (n_sp + 1) + t]);
+            s_cut[tid * (n_sp + 1) + t] = m;
+        }
+    }
+    __syncthreads();
+    // this split of each row, padded with -1 to whole tiles
+    for (int q = tid; q < rpc * stride; q += kConsumers * kWarp) {
+        const int j = q / stride, i = q - j * stride;
+        const int lo = s_cut[j * (n_sp + 1) + split], hi = s_cut[j * (n_sp + 1) + split + 1];
+        s_work[q] = lo + i < hi ? s_set[j * B + lo + i] : -1;
+    }
+    __syncthreads();
+    const int n_mine = s_cut[jl * (n_sp + 1) + split + 1] - s_cut[jl * (n_sp + 1) + split];
+    const int n_tiles = (n_mine + kTile - 1) / kTile;
+    int32_t* s_ent = s_work + jl * stride;
 
     float o[NT][kD / 16][4];
     float m_run[NT][2], l_run[NT][2];
@@ -886,8 +944,8 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(con
 #pragma unroll
         for (int mt = 0; mt < kD / 16; ++mt) o[0][mt][0] = o[0][mt][1] = o[0][mt][2] = o[0][mt][3] = 0.f;
     }
-    merge_and_store<NT, true>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, D, kvh, grp * D, layer, split,
-                              ratio);
+    merge_and_store<NT, true>(a, smem + a.stage_off, o, m_run, l_run, warp, lane, keys, hgrp,
+                              grp * D + rb * rpc, layer, split, ratio, 1.f, hpc);
 }
 
 // Split merge: one CTA per (query head, row, layer) with one warp per
@@ -1034,36 +1092,36 @@ AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budge
 
 AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int budget, int G, int num_sms) {
     AttendPlan p;
-    p.hpc = 1;
-    p.head_groups = H_kv;
-    const int cap = group_rows * budget;  // the union holds at most this many entries
-    const long units = (long)(n_q / group_rows) * H_kv * G;
-    int splits = units > 0 ? (int)((num_sms + units / 2) / units) : 1;
-    const int min_splits = (cap + kMaxEntriesPerSplit - 1) / kMaxEntriesPerSplit;
-    const int max_splits = (cap + 63) / 64;
+    // a CTA reads whole tokens (all its kv heads, as attend_rk_kernel) for as
+    // many rows of the group as its 8 warps hold
+    p.hpc = H_kv < 4 ? H_kv : 4;
+    p.head_groups = H_kv / p.hpc;
+    p.rows_per_cta = group_rows < kConsumers / p.hpc ? group_rows : kConsumers / p.hpc;
+    const int row_blocks = group_rows / p.rows_per_cta;
+    const long units = (long)(n_q / group_rows) * p.head_groups * row_blocks * G;
+    // one CTA per SM: the grid must not pass one wave (a few CTAs of a second
+    // wave would double the call)
+    int splits = units > 0 ? (int)(num_sms / units) : 1;
+    const int max_splits = (budget + 63) / 64;  // at least 4 tiles per split on average
     if (splits > max_splits) splits = max_splits;
-    if (splits < min_splits) splits = min_splits;
     if (splits < 1) splits = 1;
     p.n_splits = splits;
-    // a stretch of equal work holds at most ceil(work / splits) + D entries
-    // (every entry has a member; the last may carry D): its list capacity
-    int eps = (cap + splits - 1) / splits + group_rows;
-    eps = (eps + kTile - 1) / kTile * kTile;
-    if (eps < kTile) eps = kTile;
-    p.entries_per_split = eps;
-    const size_t ent = ((size_t)group_rows * eps * 4 + 127) / 128 * 128;
-    p.stage_off = (int)ent;
+    // a split of a row may hold its whole set (cuts follow the first row)
+    p.entries_per_split = (budget + kTile - 1) / kTile * kTile;
+    if (p.entries_per_split < kTile) p.entries_per_split = kTile;
+    const size_t lists = (size_t)p.rows_per_cta * ((size_t)budget + p.entries_per_split + splits + 1) * 4;
     const size_t merge = (size_t)kConsumers * ((kD / 16) * 4 + 4) * kWarp * 4;
-    p.smem_bytes = ent + merge;
+    p.stage_off = 0;  // the merge area reuses the lists once the tiles are done
+    p.smem_bytes = (lists + 127) / 128 * 128 > merge ? (lists + 127) / 128 * 128 : merge;
     const size_t rows_q = (size_t)G * n_q;
-    size_t ws = 0;
+    size_t ws = 256;
     if (splits > 1) {
         ws = rows_q * splits * H_q * kD * 4;
         ws = (ws + 255) / 256 * 256;
         ws += rows_q * splits * H_q * 2 * 4;
         ws = (ws + 255) / 256 * 256;
     }
-    p.ws_bytes = ws;  // the caller adds the union arrays
+    p.ws_bytes = ws;
     return p;
 }
 
@@ -1074,7 +1132,8 @@ cudaError_t launch_attend_grouped(const AttendArgs& a, size_t smem_bytes, cudaSt
     const int pct = (int)(((smem_bytes + 2048) * 100 + kSmemPerSm - 1) / kSmemPerSm);
     e = cudaFuncSetAttribute(attend_group_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, pct < 100 ? pct : 100);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)(a.n_splits * a.H_kv), (unsigned)(a.n_q / a.group_rows), (unsigned)a.G);
+    const dim3 grid((unsigned)(a.n_splits * a.head_groups * (a.group_rows / a.rows_per_cta)),
+                    (unsigned)(a.n_q / a.group_rows), (unsigned)a.G);
     e = launch_pdl(attend_group_kernel, grid, dim3(kConsumers * kWarp), smem_bytes, stream, 0, a);
     if (e != cudaSuccess || a.n_splits == 1) return e;
     int nw = (a.n_splits + kMergeSplitsPerWarp - 1) / kMergeSplitsPerWarp;

@@ -31,6 +31,7 @@
 
 #include <cstddef>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -71,7 +72,7 @@ struct TcArgs {
 
 // Candidate filter. A row's kept keys (those at or above its threshold) are
 // counted in a histogram of kTcBins bins on a logarithmic scale (bit length
-// and the 3 bits after the leading one). Every kTcUpdate tiles each CTA adds
+// and the 4 bits after the leading one). Every kTcUpdate tiles each CTA adds
 // its counts into the row's histogram in global memory, shared by the CTAs
 // of every token split, and reads it back; the lower edge of the highest bin
 // whose count from the top reaches topk becomes the row's threshold. Every
@@ -83,14 +84,16 @@ constexpr int kTcBins = LSA_TC_BINS;
 constexpr int kTcMaxSplits = LSA_TC_MAX_SPLITS;
 static_assert(LSA_TC_SEGS == 4, "one candidate segment per TMEM lane quarter");
 constexpr int kTcUpdate = 8;
+constexpr int kTcBinsPerLane = kTcBins / 32;  // a warp scans a row's histogram, lane l bins l*this..
+static_assert(kTcBins == 512, "bit length (5 bits) x 16 sub-bins");
 __device__ __forceinline__ uint32_t tc_bin(uint32_t key) {
-    if (key < 8u) return key;
-    const int nb = 32 - __clz((int)key);  // 4..32
-    return ((uint32_t)(nb - 3) << 3) | ((key >> (nb - 4)) & 7u);
+    if (key < 16u) return key;
+    const int nb = 32 - __clz((int)key);  // 5..32
+    return ((uint32_t)(nb - 4) << 4) | ((key >> (nb - 5)) & 15u);
 }
 __device__ __forceinline__ uint32_t tc_bin_floor(uint32_t b) {
-    if (b < 8u) return b;
-    return (8u | (b & 7u)) << ((b >> 3) - 1u);
+    if (b < 16u) return b;
+    return (16u | (b & 15u)) << ((b >> 4) - 1u);
 }
 
 struct TcShared {
@@ -262,6 +265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
     const int j_hi = (int)((int64_t)nt_all * (blockIdx.x + 1) / gridDim.x);
     const int nt = j_hi - j_lo;
 
+
     if (warp == 0) {
         // ---- TMA producer ---------------------------------------------------
         if (lane == 0 && nt > 0) {
@@ -321,6 +325,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             rws[i] = sh.row_ws[ri];
         }
         const int rl0 = half * kRows;  // first query row (of the CTA) of this warp's columns
+        int rs_max = 0, rws_min = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+            rs_max = max(rs_max, rs[i]);
+            rws_min = min(rws_min, rws[i]);
+        }
         // This warp's candidates of each of its rows go to its own slots: the
         // slots of the CTA's tokens (from the union's first middle token; splits
         // are disjoint and the union spans at most fine_cap slots), quarter q of
@@ -337,7 +347,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             thr[i] = 1u;
         }
         // 32 columns (32 / H_I query rows) of accumulators -> candidates
-        auto rows_of = [&](const uint32_t (&v)[32], int c, int t) {
+        auto rows_of = [&](const uint32_t (&v)[32], int c, int t, auto all_in) {
             int32_t w[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -355,7 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
                 for (int h = 0; h < H_I; ++h) acc4[h & 3] += max((int32_t)v[rr * H_I + h], 0) * w[rr * H_I + h];
                 const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 const uint32_t key = (uint32_t)acc + 1u;
-                const bool emit = key >= thr[i] && t >= rs[i] && t < rws[i];
+                const bool emit = key >= thr[i] && (decltype(all_in)::value || (t >= rs[i] && t < rws[i]));
                 const uint32_t m = __ballot_sync(0xffffffffu, emit);
                 if (m != 0u) {  // warp-uniform: most chunks of a row emit nothing once its threshold has risen
                     if (emit) {
@@ -369,23 +379,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             }
         };
         // Threshold updates of this warp's two query rows (rows 2w', 2w'+1 of
-        // the CTA, w' the epilogue warp index), spread over two tiles so that
-        // the global round trip overlaps a tile's work: flush() moves the CTA's
-        // new counts into the row's global histogram and keeps the returned
-        // totals (lane l: bins 8l .. 8l+7); settle() turns them into the
-        // threshold; the warps of the rows read it back one tile later.
+        // the CTA, w' the epilogue warp index), spread over three tiles so that
+        // the global round trip overlaps the tiles' work: flush() adds the CTA's
+        // new counts into the row's global histogram (reductions, no value
+        // returned) and loads its totals (lane l: its kTcBinsPerLane bins, the
+        // loads in flight while the next tiles are scored); settle() turns them
+        // into the threshold two tiles later; the warps of the rows read it
+        // back a tile after that. A load may miss other CTAs' latest counts:
+        // fewer counted keys only lower the threshold.
         const int ew = warp - 2;
-        uint32_t gc[2][8];
+        uint32_t gc[2][kTcBinsPerLane];
+        // Only the bins at or above the row's threshold bin are touched: no
+        // key below the threshold is counted, and the threshold only rises.
         auto flush = [&]() {
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int row = 2 * ew + q2;
                 const bool live = row0 + row < a.n_q;
-                uint32_t* g = a.ghist + (int64_t)(live ? row0 + row : 0) * kTcBins + 8 * lane;
+                const uint32_t tb = tc_bin(*reinterpret_cast<volatile uint32_t*>(&sh.thr[row]));
+                uint32_t* g = a.ghist + (int64_t)(live ? row0 + row : 0) * kTcBins + kTcBinsPerLane * lane;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t d = atomicExch(&sh.hist[row][8 * lane + j], 0u);
-                    gc[q2][j] = !live ? 0u : d != 0u ? atomicAdd(g + j, d) + d : __ldcg(g + j);
+                for (int j = 0; j < kTcBinsPerLane; ++j) {
+                    const uint32_t b = (uint32_t)(kTcBinsPerLane * lane + j);
+                    uint32_t c = 0u;
+                    if (live && b >= tb) {
+                        const uint32_t d = atomicExch(&sh.hist[row][b], 0u);
+                        if (d != 0u) atomicAdd(g + j, d);  // result unused: a reduction
+                        c = __ldcg(g + j);
+                    }
+                    gc[q2][j] = c;
                 }
             }
         };
@@ -395,8 +417,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
                 const int row = 2 * ew + q2;
                 uint32_t own = 0;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) own += gc[q2][j];
-                uint32_t x = own;  // keys in bins >= 8 * lane
+                for (int j = 0; j < kTcBinsPerLane; ++j) own += gc[q2][j];
+                uint32_t x = own;  // keys in bins >= kTcBinsPerLane * lane
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
@@ -407,9 +429,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
                 if (k > 0u && x >= k) {
                     uint32_t run = x - own;
 #pragma unroll
-                    for (int j = 7; j >= 0; --j) {
+                    for (int j = kTcBinsPerLane - 1; j >= 0; --j) {
                         run += gc[q2][j];
-                        if (run >= k && best == 0u) best = (uint32_t)(8 * lane + j) + 1u;
+                        if (run >= k && best == 0u) best = (uint32_t)(kTcBinsPerLane * lane + j) + 1u;
                     }
                 }
 #pragma unroll
@@ -429,29 +451,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             const int buf = j & 1, use = j >> 1;
             if (!tc_wait(sh, smem_u32(&sh.tfull[buf]), use & 1, a.dev_status)) break;
             tc_fence_after();
-            const int t = t_lo + (j_lo + j) * kTcTokens + lane_tok;
+            const int tt0 = t_lo + (j_lo + j) * kTcTokens;  // the tile's first token
+            const int t = tt0 + lane_tok;
             const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(buf * kTcCols + 128 * half);
             // two register buffers: the load of chunk c+1 is in flight while chunk c is reduced
-            uint32_t va[32], vb[32];
-            tmem_ld32(tbase, va);
-            tmem_wait(va);
-            tmem_ld32(tbase + 32u, vb);
-            rows_of(va, 0, t);
-            tmem_wait(vb);
-            tmem_ld32(tbase + 64u, va);
-            rows_of(vb, 1, t);
-            tmem_wait(va);
-            tmem_ld32(tbase + 96u, vb);
-            rows_of(va, 2, t);
-            tmem_wait(vb);
-            rows_of(vb, 3, t);
+            auto drain = [&](auto all_in) {
+                uint32_t va[32], vb[32];
+                tmem_ld32(tbase, va);
+                tmem_wait(va);
+                tmem_ld32(tbase + 32u, vb);
+                rows_of(va, 0, t, all_in);
+                tmem_wait(vb);
+                tmem_ld32(tbase + 64u, va);
+                rows_of(vb, 1, t, all_in);
+                tmem_wait(va);
+                tmem_ld32(tbase + 96u, vb);
+                rows_of(va, 2, t, all_in);
+                tmem_wait(vb);
+                rows_of(vb, 3, t, all_in);
+            };
+            // a tile inside the middle of every row of the warp needs no
+            // per-token range test (most tiles of a chunk)
+            if (tt0 >= rs_max && tt0 + kTcTokens <= rws_min) drain(std::true_type{});
+            else drain(std::false_type{});
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sh.tempty[buf]));
             const int ph = j % kTcUpdate;
-            if (ph == kTcUpdate - 1) flush();
-            else if (ph == 0 && j > 0) settle();
-            else if (ph == 1 && j > 1) refresh();
+            if (ph == kTcUpdate - 3) flush();
+            else if (ph == kTcUpdate - 1) settle();
+            else if (ph == 0 && j > 0) refresh();
         }
         // this warp's segment of each of its rows
         if (lane == 0) {

@@ -118,7 +118,7 @@ cudaError_t launch_fine_scores_tc(const IndexArgs& a, cudaStream_t stream);
 // Token splits of each 16-row tile in the tensor-core scoring (<= LSA_TC_MAX_SPLITS).
 #define LSA_TC_MAX_SPLITS 16
 #define LSA_TC_SEGS 4     // candidate segments per token split (one per TMEM lane quarter)
-#define LSA_TC_BINS 256   // candidate-filter histogram bins per row
+#define LSA_TC_BINS 512   // candidate-filter histogram bins per row
 #define LSA_TC_TOKENS 128 // cached tokens per tensor-core tile
 int prefill_tc_splits(int n_q);
 // HI block selection computes the coarse scores itself when each cluster
@@ -154,24 +154,8 @@ struct PointArgs {
 };
 cudaError_t launch_point_scores(const PointArgs& p, int d_I, cudaStream_t stream);
 
-// Draft-row groups (draft_union.cu): the union of each group's index sets.
+// Draft-row groups (attend_group_kernel): at most this many rows per group.
 constexpr int kMaxGroupRows = 8;
-struct UnionArgs {
-    const int32_t* sets;     // [n_groups * group_rows][budget]
-    const int32_t* q_seq;
-    const int32_t* q_len;
-    const int64_t* kv_offset;
-    const int32_t* seq_lens;
-    int32_t* union_pos;      // [n_groups][union_cap] positions, ascending
-    uint8_t* union_msk;      // [n_groups][union_cap] rows of the group holding each position (bit j: row j)
-    int32_t* union_len;      // [n_groups]
-    int32_t* union_split;    // [n_groups][n_splits + 1] first union entry of each attention split
-    int32_t* dev_status;
-    int64_t total_tokens;
-    int32_t n_groups, group_rows, budget, union_cap, n_seq, max_len, n_splits;
-};
-size_t union_smem_bytes(int group_rows, int budget);
-cudaError_t launch_union_sets(const UnionArgs& u, cudaStream_t stream);
 
 // Context-parallel attention (context_parallel.cu).
 cudaError_t launch_shard_sets(const int32_t* sets, int n_q, int budget, int lo, int hi, int32_t* local,
@@ -203,16 +187,12 @@ struct AttendArgs {
     float scale_log2;     // log2(e) / sqrt(d)
     int32_t kv_fp8;       // K/V caches hold FP8 E4M3 codes (k, v point at bytes)
     float kscale[kMaxLayers], vscale[kMaxLayers];  // FP8: value = scale * E4M3(code)
-    // draft-row groups (attend_group_kernel): the union of each group's sets
-    const int32_t* union_pos;
-    const uint8_t* union_msk;
-    const int32_t* union_len;
-    const int32_t* union_split;  // [groups][n_splits + 1]: equal shares of the rows' members
-    int32_t group_rows, union_cap;
+    // draft-row groups (attend_group_kernel): rows per group and per CTA
+    int32_t group_rows, rows_per_cta;
 };
 
 struct AttendPlan {
-    int n_splits = 1, entries_per_split = 16, head_groups = 1, hpc = 1;
+    int n_splits = 1, entries_per_split = 16, head_groups = 1, hpc = 1, rows_per_cta = 1;
     int n_stages = 2, row_stride = 272, bar_off = 0, stage_off = 0;
     size_t smem_bytes = 0;
     size_t ws_bytes = 0;
@@ -220,7 +200,7 @@ struct AttendPlan {
 AttendPlan plan_attend(int n_q, int max_len, int H_q, int H_kv, int d, int budget, int G, int num_sms,
                        bool fp8 = false);
 cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
-// Draft-row groups: the union's splits, shared memory and workspace.
+// Draft-row groups: splits, shared memory and workspace of attend_group_kernel.
 AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int budget, int G, int num_sms);
 cudaError_t launch_attend_grouped(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
 

@@ -206,7 +206,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch_before_launch():
 
 def test_grouped_attention_rejects_and_counts_before_launch():
     """lsa_attend_grouped: group sizes, divisibility, GQA width and the
-    union's shared memory are checked before any launch."""
+    staged sets' shared memory are checked before any launch."""
     lib = lsa.load_library()
     b = _batch(n_q=16, max_len=131072, total=4 * 131072)
     arr = (ctypes.c_void_p * 1)(P)
@@ -216,12 +216,11 @@ def test_grouped_attention_rejects_and_counts_before_launch():
     assert f(*args(D=3)) == 1                       # 16 rows are not groups of 3
     assert f(*args(D=16)) == 2                      # at most 8 rows per group
     assert f(*args(H_q=64)) == 2                    # GQA groups of at most 8 query heads
-    assert f(*args(D=8, budget=16384)) == 2         # the union's staging would not fit in shared memory
+    assert f(*args(D=8, budget=16384)) == 2         # the rows' sets would not fit in shared memory
     assert f(*args(ws=16)) == 4                     # workspace too small
     need = lib.lsa_attend_grouped_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 1, 4)
-    # the unions (positions, masks, lengths of 4 groups) come on top of the split partials
-    assert need >= lib.lsa_attend_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 1) // 4 + 4 * 4 * 3136 * 5
-    assert lib.lsa_attend_grouped_launches(ctypes.byref(b), 32, 4, 128, 3136, 1, 4) == 3
+    assert need >= 16 * 32 * 128 * 4                # split partials of every (row, head)
+    assert lib.lsa_attend_grouped_launches(ctypes.byref(b), 32, 4, 128, 3136, 1, 4) == 2
     assert lib.lsa_attend_grouped_launches(ctypes.byref(b), 32, 4, 128, 3136, 1, 3) == 0
 
 

@@ -112,6 +112,9 @@ PREFILL_CASES = {
     "tc_wide_window": dict(lens=(1500 + 130,), prefill_new=130, sink=64, window=1400, topk=50),
     "tc_full_range": dict(lens=(3000 + 96,), prefill_new=96, qk_lo=-128, qk_hi=127, w_hi=4, topk=500),
     "tc_ties": dict(lens=(4000 + 64,), prefill_new=64, qk_lo=-1, qk_hi=1, w_hi=1, topk=700),
+    # wider query/key ranges and weights than the default draw
+    "tc_qk32_w4": dict(lens=(3000 + 80,), prefill_new=80, qk_lo=-32, qk_hi=31, w_hi=4, topk=400),
+    "tc_qk64_w3": dict(lens=(3000 + 80,), prefill_new=80, qk_lo=-64, qk_hi=63, w_hi=3, topk=400),
 }
 
 
