@@ -357,21 +357,20 @@ lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_ca
  * skipped alike), for batches whose rows come in groups of group_rows
  * consecutive rows of one sequence (row g * group_rows + j is draft j of group
  * g, as the decode rows of lsa_batch_t with several rows per sequence are laid
- * out). The rows of a group are attended together: their sets are cut at the
- * same positions, so the rows walk the same stretch of the cache at the same
- * time and a K/V row several of them hold is read from HBM once and served to
- * the others on chip. Sets as lsa_index writes them (ascending) get the
- * sharing; any other set is still attended exactly.
+ * out). The rows of a group are attended together: each stretch of their
+ * sets (the same entry range of every row) runs in one CTA, so for sets as
+ * lsa_index writes them (ascending, sink run first, window run last) the rows
+ * walk the same positions at the same time and a K/V row several of them hold
+ * is read from HBM once and served to the others on chip. Any other set is
+ * still attended exactly.
  *
  * Arguments, output and device-side errors as lsa_attend, plus
  * group_rows  1, 2, 4 or 8; n_q must be a multiple of it.
  * workspace   lsa_attend_grouped_workspace_size() bytes (split partials; no
  *             initialisation needed).
  * Supported: the shapes lsa_attend supports with H_q / H_kv <= 8 and bf16
- * caches, n_q / group_rows <= 65535, and a budget whose sets fit the
- * kernel's shared memory (rows per CTA x budget x 8 bytes, rows per CTA =
- * min(group_rows, 8 / min(H_kv, 4)), within 220 KiB; the shape queries
- * return 0 otherwise). One launch, plus a split merge with several splits.
+ * caches, n_q / group_rows <= 65535. One launch, plus a split merge with
+ * several splits.
  */
 size_t lsa_attend_grouped_workspace_size(const lsa_batch_t *batch, int32_t H_q, int32_t H_kv,
                                          int32_t d, int32_t budget, int32_t layers_per_index,

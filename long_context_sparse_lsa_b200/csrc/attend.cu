@@ -733,15 +733,14 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
 // sequence (the draft tokens of a decode step), whose index sets share the
 // sink run, nearly all of the window run and, where the drafts' indexer
 // queries agree, much of the selection. A CTA covers hpc kv heads (whole
-// tokens, as attend_rk_kernel) for rpc rows of a group; it stages those rows'
-// whole sets and cuts every one of them at the same positions: the positions
-// of its first row's entries at n_splits equal steps. Split s of every row is
-// then the stretch of positions between two cuts, so the CTA's rows walk the
-// same positions together and a K/V row that several of them hold is fetched
-// from L2 once and served from L1 to the others. The cuts are taken as
-// indices into each row's set (made non-decreasing), so every entry of a row
-// belongs to exactly one split whatever the set holds: the output is
-// lsa_attend's. The tile loop, the fragments and the softmax are
+// tokens, as attend_rk_kernel) for rpc rows of a group, one warp per (kv
+// head, row), all over the same stretch of their sets: entries [B s / n,
+// B (s + 1) / n) of every row for split s. Sets as lsa_index writes them
+// are ascending with the sink run first and the window run last, so the
+// rows' stretches cover the same positions (exactly, for the sink and window
+// runs), and a K/V row that several rows hold is fetched from L2 once and
+// served from L1 to the others; the work per warp is the same as in
+// attend_rk_kernel. The tile loop, the fragments and the softmax are
 // attend_rk_kernel's (bf16 caches, GQA groups of at most 8 query heads); the
 // partials merge as lsa_attend's.
 __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(const __grid_constant__ AttendArgs a) {
@@ -782,14 +781,13 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(con
         float* orow = a.out[layer] + ((int64_t)r * a.H_q + (int64_t)kvh * ratio) * kD;
         for (int i = lane; i < ratio * kD; i += kWarp) orow[i] = 0.f;
     }
-    // the CTA's rows' whole sets, checked as lsa_attend checks them (entries
-    // below -1 or at or past q_len flagged and skipped; an invalid row's
-    // entries all skipped)
+    // split s of each of the CTA's rows: entries [B s / n, B (s + 1) / n) of
+    // its set, checked as lsa_attend checks them (entries below -1 or at or
+    // past q_len flagged and skipped; an invalid row's entries all skipped)
+    // and padded with -1 to whole tiles
     const int B = a.budget;
-    const int stride = a.entries_per_split;   // per-row working list: B rounded up to whole tiles
-    int32_t* s_set = reinterpret_cast<int32_t*>(smem);         // [rpc][B]
-    int32_t* s_work = s_set + rpc * B;                         // [rpc][stride]
-    int32_t* s_cut = s_work + rpc * stride;                    // [rpc][n_splits + 1]
+    const int stride = a.entries_per_split;  // per-row list capacity
+    int32_t* s_work = reinterpret_cast<int32_t*>(smem);  // [rpc][stride]
     __shared__ int32_t s_len[kMaxGroupRows];
     if (tid < rpc) {
         const int rr = grp * D + rb * rpc + tid;
@@ -802,83 +800,25 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_group_kernel(con
         s_len[tid] = ok ? Lr : 0;
     }
     __syncthreads();
-    // (the CTA's rows are consecutive: their sets are one contiguous run,
-    // read with 16-byte loads, all of a thread's in flight together)
-    const int32_t* run = a.sets + (int64_t)(grp * D + rb * rpc) * B;
-    const int n_run = rpc * B;
-    if ((B & 3) == 0 && (reinterpret_cast<uintptr_t>(run) & 15u) == 0) {
-        constexpr int kU = 8;
-        for (int v0 = tid; v0 < n_run / 4; v0 += kConsumers * kWarp * kU) {
-            int4 x[kU];
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int v = v0 + u * kConsumers * kWarp;
-                x[u] = v < n_run / 4 ? __ldg(reinterpret_cast<const int4*>(run) + v) : make_int4(-1, -1, -1, -1);
-            }
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int v = v0 + u * kConsumers * kWarp;
-                if (v < n_run / 4) reinterpret_cast<int4*>(s_set)[v] = x[u];
-            }
-        }
-    } else {
-        for (int i = tid; i < n_run; i += kConsumers * kWarp) s_set[i] = __ldg(run + i);
-    }
-    __syncthreads();
+    const int e_lo = (int)((int64_t)B * split / a.n_splits);
+    const int n_mine = (int)((int64_t)B * (split + 1) / a.n_splits) - e_lo;  // the same for every row
+    const int n_tiles = (n_mine + kTile - 1) / kTile;
     bool bad_entry = false;
-    for (int i = tid; i < n_run; i += kConsumers * kWarp) {
-        const int Lj = s_len[i / B];
-        const int32_t e = s_set[i];
-        if (e < -1 || e >= Lj) {
-            bad_entry |= Lj > 0;
-            s_set[i] = -1;
+    for (int q = tid; q < rpc * n_tiles * kTile; q += kConsumers * kWarp) {
+        const int j = q / (n_tiles * kTile), i = q - j * (n_tiles * kTile);
+        int32_t e = -1;
+        if (i < n_mine) {
+            e = a.sets[(int64_t)(grp * D + rb * rpc + j) * B + e_lo + i];
+            const int Lj = s_len[j];
+            if (e < -1 || e >= Lj) {
+                bad_entry |= Lj > 0;
+                e = -1;
+            }
         }
+        s_work[j * stride + i] = e;
     }
     if (bad_entry) flag(a.dev_status, LSA_DEV_BAD_INDEX);
     __syncthreads();
-    // the cuts: cut t of row j = the first entry of row j not below position
-    // P_t = the CTA's first row's entry B t / n (a -1 there: no bound); made
-    // non-decreasing in t, so the splits of a row cover its set exactly once
-    const int n_sp = a.n_splits;
-    for (int q = tid; q < rpc * (n_sp + 1); q += kConsumers * kWarp) {
-        const int j = q / (n_sp + 1), t = q - j * (n_sp + 1);
-        int c;
-        if (t == 0) {
-            c = 0;
-        } else if (t == n_sp) {
-            c = B;
-        } else {
-            const int32_t pr = s_set[(int)((int64_t)B * t / n_sp)];
-            const int32_t P = pr >= 0 ? pr : 0x7fffffff;
-            const int32_t* row = s_set + j * B;
-            int lo = 0, hi = B;  // entries in [0, P) form a prefix of an ascending set
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (row[mid] >= 0 && row[mid] < P) lo = mid + 1;
-                else hi = mid;
-            }
-            c = lo;
-        }
-        s_cut[q] = c;
-    }
-    __syncthreads();
-    if (tid < rpc) {
-        int m = 0;
-        for (int t = 0; t <= n_sp; ++t) {
-            m = max(m, s_cut[tid * (n_sp + 1) + t]);
-            s_cut[tid * (n_sp + 1) + t] = m;
-        }
-    }
-    __syncthreads();
-    // this split of each row, padded with -1 to whole tiles
-    for (int q = tid; q < rpc * stride; q += kConsumers * kWarp) {
-        const int j = q / stride, i = q - j * stride;
-        const int lo = s_cut[j * (n_sp + 1) + split], hi = s_cut[j * (n_sp + 1) + split + 1];
-        s_work[q] = lo + i < hi ? s_set[j * B + lo + i] : -1;
-    }
-    __syncthreads();
-    const int n_mine = s_cut[jl * (n_sp + 1) + split + 1] - s_cut[jl * (n_sp + 1) + split];
-    const int n_tiles = (n_mine + kTile - 1) / kTile;
     int32_t* s_ent = s_work + jl * stride;
 
     float o[NT][kD / 16][4];
@@ -1102,14 +1042,16 @@ AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int b
     // one CTA per SM: the grid must not pass one wave (a few CTAs of a second
     // wave would double the call)
     int splits = units > 0 ? (int)(num_sms / units) : 1;
-    const int max_splits = (budget + 63) / 64;  // at least 4 tiles per split on average
+    const int min_splits = (budget + kMaxEntriesPerSplit - 1) / kMaxEntriesPerSplit;
+    const int max_splits = (budget + 63) / 64;  // at least 4 tiles per split
     if (splits > max_splits) splits = max_splits;
+    if (splits < min_splits) splits = min_splits;
     if (splits < 1) splits = 1;
     p.n_splits = splits;
-    // a split of a row may hold its whole set (cuts follow the first row)
-    p.entries_per_split = (budget + kTile - 1) / kTile * kTile;
-    if (p.entries_per_split < kTile) p.entries_per_split = kTile;
-    const size_t lists = (size_t)p.rows_per_cta * ((size_t)budget + p.entries_per_split + splits + 1) * 4;
+    int eps = (budget + splits - 1) / splits;  // each row's entries in a split
+    eps = (eps + kTile - 1) / kTile * kTile;
+    p.entries_per_split = eps < kTile ? kTile : eps;
+    const size_t lists = (size_t)p.rows_per_cta * p.entries_per_split * 4;
     const size_t merge = (size_t)kConsumers * ((kD / 16) * 4 + 4) * kWarp * 4;
     p.stage_off = 0;  // the merge area reuses the lists once the tiles are done
     p.smem_bytes = (lists + 127) / 128 * 128 > merge ? (lists + 127) / 128 * 128 : merge;

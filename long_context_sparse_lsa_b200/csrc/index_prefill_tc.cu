@@ -17,13 +17,15 @@
 //  * Tokens are the MMA's M dimension so that the head reduction is a
 //    per-thread loop in the epilogue: a thread owns one TMEM lane (one token),
 //    reads its row of accumulators, applies ReLU and the query row's weights,
-//    sums each row's heads and stores the key (score + 1) of that (row,
-//    token); a warp stores 32 consecutive tokens of one row at a time, in the
-//    layout the selection kernels read.
+//    sums each row's heads into the key (score + 1) of that (row, token), and
+//    keeps the key as a candidate only if it passes the row's running
+//    threshold (the filter below), so the selection reads a few percent of
+//    the keys instead of all of them.
 //  * Warp roles: warp 0 issues the TMA loads, one thread of warp 1 issues the
-//    MMAs, warps 2..9 drain the accumulators (two warps per TMEM lane quarter,
-//    each taking half of the columns). TMEM holds two 256-column accumulators
-//    so the MMAs of tile j+1 overlap the epilogue of tile j.
+//    MMAs, warps 2..17 drain the accumulators (four warps per TMEM lane
+//    quarter, each taking a quarter of the columns: four query rows, read 16
+//    columns at a time). TMEM holds two 256-column accumulators so the MMAs of
+//    tile j+1 overlap the epilogue of tile j.
 //  * Every mbarrier wait is bounded; on expiry the kernel flags
 //    LSA_DEV_TIMEOUT, stops issuing work, waits (bounded) for what it issued,
 //    frees its TMEM and returns.
@@ -43,7 +45,7 @@ constexpr int kTcTokens = LSA_TC_TOKENS;             // M: cached tokens per til
 constexpr int kTcCols = 256;                         // N: query-head rows per CTA
 constexpr int kTcK = 128;                            // d_I bytes per key row
 constexpr int kTcStages = 6;                         // A-tile ring
-constexpr int kTcEpiWarps = 8;
+constexpr int kTcEpiWarps = 16;  // four per TMEM lane quarter, each a quarter of the columns
 constexpr int kTcThreads = (2 + kTcEpiWarps) * kWarp;
 constexpr uint32_t kATileBytes = kTcTokens * kTcK;   // 16 KB
 constexpr uint32_t kBTileBytes = kTcCols * kTcK;     // 32 KB
@@ -164,6 +166,24 @@ __device__ __forceinline__ void tmem_wait(uint32_t (&v)[32]) {
                    "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
                    "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
                    "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
+}
+
+// 16 consecutive accumulator columns of this warp's 32 TMEM lanes (as tmem_ld32).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];\n"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait(uint32_t (&v)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                   "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                   "+r"(v[15])
                  :
                  : "memory");
 }
@@ -309,22 +329,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
         }
     } else {
         // ---- epilogue: TMEM -> keys ---------------------------------------------
-        constexpr int kRows = 128 / H_I;         // query rows of this warp's 128 columns
-        const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
-        const int half = (warp - 2) >> 2;        // accumulator columns 128*half .. +127
+        static_assert(H_I == 16, "one 16-column TMEM load per query row");
+        constexpr int kParts = kTcEpiWarps / 4;        // warps per TMEM lane quarter
+        constexpr int kCols = kTcCols / kParts;        // accumulator columns of a warp
+        constexpr int kRows = kCols / H_I;             // its query rows
+        const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
+        const int part = (warp - 2) >> 2;              // accumulator columns kCols*part ..
         const int lane_tok = 32 * quarter + lane;
-        // the warp's row bounds stay in registers for every tile; its 128
-        // weights are re-read per 32-column chunk with warp-wide broadcast
-        // 16-byte loads (volatile, so they are not hoisted out of the tile loop)
-        const uint32_t wsh = smem_u32(&sh.w[128 * half]);
+        // the warp's row bounds stay in registers for every tile; its weights
+        // are re-read per row with warp-wide broadcast 16-byte loads (volatile,
+        // so they are not hoisted out of the tile loop)
+        const uint32_t wsh = smem_u32(&sh.w[kCols * part]);
+        const int rl0 = kRows * part;  // first query row (of the CTA) of this warp's columns
         int32_t rs[kRows], rws[kRows];
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
-            const int ri = half * kRows + i;
-            rs[i] = sh.row_ok[ri] ? sh.row_s[ri] : 0x7fffffff;  // invalid row: no token qualifies
-            rws[i] = sh.row_ws[ri];
+            rs[i] = sh.row_ok[rl0 + i] ? sh.row_s[rl0 + i] : 0x7fffffff;  // invalid row: no token qualifies
+            rws[i] = sh.row_ws[rl0 + i];
         }
-        const int rl0 = half * kRows;  // first query row (of the CTA) of this warp's columns
         int rs_max = 0, rws_min = 0x7fffffff;
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
@@ -346,101 +368,88 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             cnt[i] = 0u;
             thr[i] = 1u;
         }
-        // 32 columns (32 / H_I query rows) of accumulators -> candidates
-        auto rows_of = [&](const uint32_t (&v)[32], int c, int t, auto all_in) {
-            int32_t w[32];
+        // one query row's 16 accumulator columns -> its key, kept if it passes
+        auto row_of = [&](const uint32_t (&v)[16], int i, int t, auto all_in) {
+            int32_t w[16];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
+            for (int q = 0; q < 4; ++q)
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(w[4 * q]), "=r"(w[4 * q + 1]), "=r"(w[4 * q + 2]), "=r"(w[4 * q + 3])
-                             : "r"(wsh + 4u * (uint32_t)(32 * c + 4 * q)));
+                             : "r"(wsh + 4u * (uint32_t)(H_I * i + 4 * q)));
+            // four independent partial sums: a 16-long chain of dependent
+            // multiply-adds would stall on its own latency
+            int32_t acc4[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int rr = 0; rr < 32 / H_I; ++rr) {
-                const int col = 32 * c + rr * H_I;  // first of this query row's columns
-                const int i = col / H_I;
-                // four independent partial sums: a 16-long chain of dependent
-                // multiply-adds would stall on its own latency
-                int32_t acc4[4] = {0, 0, 0, 0};
-#pragma unroll
-                for (int h = 0; h < H_I; ++h) acc4[h & 3] += max((int32_t)v[rr * H_I + h], 0) * w[rr * H_I + h];
-                const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                const uint32_t key = (uint32_t)acc + 1u;
-                const bool emit = key >= thr[i] && (decltype(all_in)::value || (t >= rs[i] && t < rws[i]));
-                const uint32_t m = __ballot_sync(0xffffffffu, emit);
-                if (m != 0u) {  // warp-uniform: most chunks of a row emit nothing once its threshold has risen
-                    if (emit) {
-                        atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
-                        const uint32_t slot = cnt[i] + __popc(m & lt_mask);
-                        if ((int64_t)slot < room)
-                            cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
-                    }
-                    cnt[i] += __popc(m);
+            for (int h = 0; h < H_I; ++h) acc4[h & 3] += max((int32_t)v[h], 0) * w[h];
+            const int32_t acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+            const uint32_t key = (uint32_t)acc + 1u;
+            const bool emit = key >= thr[i] && (decltype(all_in)::value || (t >= rs[i] && t < rws[i]));
+            const uint32_t m = __ballot_sync(0xffffffffu, emit);
+            if (m != 0u) {  // warp-uniform: most rows of a tile keep nothing once their threshold has risen
+                if (emit) {
+                    atomicAdd(&sh.hist[rl0 + i][tc_bin(key)], 1u);
+                    const uint32_t slot = cnt[i] + __popc(m & lt_mask);
+                    if ((int64_t)slot < room)
+                        cand0[(int64_t)i * a.fine_cap + slot] = ((uint64_t)key << 32) | (uint32_t)t;
                 }
+                cnt[i] += __popc(m);
             }
         };
-        // Threshold updates of this warp's two query rows (rows 2w', 2w'+1 of
-        // the CTA, w' the epilogue warp index), spread over three tiles so that
-        // the global round trip overlaps the tiles' work: flush() adds the CTA's
-        // new counts into the row's global histogram (reductions, no value
+        // Threshold updates of this warp's query row (row w' of the CTA, w'
+        // the epilogue warp index), spread over three tiles so that the global
+        // round trip overlaps the tiles' work: flush() adds the CTA's new
+        // counts into the row's global histogram (reductions, no value
         // returned) and loads its totals (lane l: its kTcBinsPerLane bins, the
         // loads in flight while the next tiles are scored); settle() turns them
-        // into the threshold two tiles later; the warps of the rows read it
-        // back a tile after that. A load may miss other CTAs' latest counts:
-        // fewer counted keys only lower the threshold.
-        const int ew = warp - 2;
-        uint32_t gc[2][kTcBinsPerLane];
+        // into the threshold two tiles later; the warps of the row read it back
+        // a tile after that. A load may miss other CTAs' latest counts: fewer
+        // counted keys only lower the threshold.
+        const int urow = warp - 2;
+        const bool ulive = row0 + urow < a.n_q;
+        uint32_t gc[kTcBinsPerLane];
         // Only the bins at or above the row's threshold bin are touched: no
         // key below the threshold is counted, and the threshold only rises.
         auto flush = [&]() {
+            const uint32_t tb = tc_bin(*reinterpret_cast<volatile uint32_t*>(&sh.thr[urow]));
+            uint32_t* g = a.ghist + (int64_t)(ulive ? row0 + urow : 0) * kTcBins + kTcBinsPerLane * lane;
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                const int row = 2 * ew + q2;
-                const bool live = row0 + row < a.n_q;
-                const uint32_t tb = tc_bin(*reinterpret_cast<volatile uint32_t*>(&sh.thr[row]));
-                uint32_t* g = a.ghist + (int64_t)(live ? row0 + row : 0) * kTcBins + kTcBinsPerLane * lane;
-#pragma unroll
-                for (int j = 0; j < kTcBinsPerLane; ++j) {
-                    const uint32_t b = (uint32_t)(kTcBinsPerLane * lane + j);
-                    uint32_t c = 0u;
-                    if (live && b >= tb) {
-                        const uint32_t d = atomicExch(&sh.hist[row][b], 0u);
-                        if (d != 0u) atomicAdd(g + j, d);  // result unused: a reduction
-                        c = __ldcg(g + j);
-                    }
-                    gc[q2][j] = c;
+            for (int j = 0; j < kTcBinsPerLane; ++j) {
+                const uint32_t b = (uint32_t)(kTcBinsPerLane * lane + j);
+                uint32_t c = 0u;
+                if (ulive && b >= tb) {
+                    const uint32_t d = atomicExch(&sh.hist[urow][b], 0u);
+                    if (d != 0u) atomicAdd(g + j, d);  // result unused: a reduction
+                    c = __ldcg(g + j);
                 }
+                gc[j] = c;
             }
         };
         auto settle = [&]() {
+            uint32_t own = 0;
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                const int row = 2 * ew + q2;
-                uint32_t own = 0;
+            for (int j = 0; j < kTcBinsPerLane; ++j) own += gc[j];
+            uint32_t x = own;  // keys in bins >= kTcBinsPerLane * lane
 #pragma unroll
-                for (int j = 0; j < kTcBinsPerLane; ++j) own += gc[q2][j];
-                uint32_t x = own;  // keys in bins >= kTcBinsPerLane * lane
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+                if (lane + o < 32) x += y;
+            }
+            const uint32_t k = (uint32_t)a.topk;
+            uint32_t best = 0u;  // the highest bin whose suffix count reaches k, + 1 (0: none)
+            if (k > 0u && x >= k) {
+                uint32_t run = x - own;
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
-                    if (lane + o < 32) x += y;
+                for (int j = kTcBinsPerLane - 1; j >= 0; --j) {
+                    run += gc[j];
+                    if (run >= k && best == 0u) best = (uint32_t)(kTcBinsPerLane * lane + j) + 1u;
                 }
-                const uint32_t k = (uint32_t)a.topk;
-                uint32_t best = 0u;  // the highest bin whose suffix count reaches k, + 1 (0: none)
-                if (k > 0u && x >= k) {
-                    uint32_t run = x - own;
+            }
 #pragma unroll
-                    for (int j = kTcBinsPerLane - 1; j >= 0; --j) {
-                        run += gc[q2][j];
-                        if (run >= k && best == 0u) best = (uint32_t)(kTcBinsPerLane * lane + j) + 1u;
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-                if (lane == 0 && best > 0u) {
-                    const uint32_t th = tc_bin_floor(best - 1u);
-                    volatile uint32_t* st = &sh.thr[row];
-                    if (th > *st) *st = th;
-                }
+            for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+            if (lane == 0 && best > 0u) {
+                const uint32_t th = tc_bin_floor(best - 1u);
+                volatile uint32_t* st = &sh.thr[urow];
+                if (th > *st) *st = th;
             }
         };
         auto refresh = [&]() {
@@ -453,22 +462,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) fine_score_tc_kernel(const __gr
             tc_fence_after();
             const int tt0 = t_lo + (j_lo + j) * kTcTokens;  // the tile's first token
             const int t = tt0 + lane_tok;
-            const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(buf * kTcCols + 128 * half);
-            // two register buffers: the load of chunk c+1 is in flight while chunk c is reduced
+            const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(buf * kTcCols + kCols * part);
+            // two register buffers: the load of row i+1 is in flight while row i is reduced
             auto drain = [&](auto all_in) {
-                uint32_t va[32], vb[32];
-                tmem_ld32(tbase, va);
+                static_assert(kRows == 4, "the drain below walks four rows");
+                uint32_t va[16], vb[16];
+                tmem_ld16(tbase, va);
                 tmem_wait(va);
-                tmem_ld32(tbase + 32u, vb);
-                rows_of(va, 0, t, all_in);
+                tmem_ld16(tbase + 16u, vb);
+                row_of(va, 0, t, all_in);
                 tmem_wait(vb);
-                tmem_ld32(tbase + 64u, va);
-                rows_of(vb, 1, t, all_in);
+                tmem_ld16(tbase + 32u, va);
+                row_of(vb, 1, t, all_in);
                 tmem_wait(va);
-                tmem_ld32(tbase + 96u, vb);
-                rows_of(va, 2, t, all_in);
+                tmem_ld16(tbase + 48u, vb);
+                row_of(va, 2, t, all_in);
                 tmem_wait(vb);
-                rows_of(vb, 3, t, all_in);
+                row_of(vb, 3, t, all_in);
             };
             // a tile inside the middle of every row of the warp needs no
             // per-token range test (most tiles of a chunk)
