@@ -757,6 +757,16 @@ def main(argv=None):
             "bytes_per_launch": byts["attend"], "ms_per_launch": at_in,
             "timing": "CUDA events recorded inside the step graph around the lsa_attend call, mean over "
                       "one replay per timed step (L2 flushed before each)"}
+    # the index call against the same roofline: its algorithmic bytes (block
+    # sums of the candidate blocks, the kept blocks' keys, queries, weights,
+    # the written sets) over its duration inside the step
+    roof_index = {"bound": "hbm", "kernel": "lsa_index call (block selection with the HI coarse scores, fine "
+                                            "scores, token selection with the SI assembly)",
+                  "achieved": byts["index"] / (ix_in / 1000.0) / 1e9, "peak": peak, "unit": "GB/s",
+                  "frac": byts["index"] / (ix_in / 1000.0) / 1e9 / peak, "peak_kind": peak_kind,
+                  "traffic": None, "bytes_per_launch": byts["index"], "ms_per_launch": ix_in,
+                  "timing": "CUDA events recorded inside the step graph around the lsa_index call, mean over "
+                            "one replay per timed step (L2 flushed before each)"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8->int32 (indexer), bf16->f32 (attention)",
@@ -777,6 +787,7 @@ def main(argv=None):
             "step_frac_of_8tbs": byts["total"] / (ms / 1000.0) / 1e9 / 8000.0,
             "algorithmic_bytes_per_step": byts,
             "roofline": roof,
+            "roofline_index": roof_index,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e},
             "gpu_launches": n_kernels * args.steps,
