@@ -682,6 +682,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the 1M decode and prefill chunk measurements")
+    ap.add_argument("--grouped", action="store_true",
+                    help="draft-row workloads: attend through lsa_attend_grouped")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     wl = wls.by_name(args.workload)
@@ -709,7 +711,8 @@ def main(argv=None):
     # each rank draws its own independent batch (weak scaling)
     wl_r = rank_workload(wl, rank)
     clocks = ClockSampler(local)
-    run = time_workload(wl_r, dev, flush, stream, args.steps, args.warmup, pg, clocks)
+    run = time_workload(wl_r, dev, flush, stream, args.steps, args.warmup, pg, clocks,
+                        grouped=args.grouped and wl.drafts > 1)
     st, t = run["st"], run["t"]
     ms = max_over_ranks(run["ms"], pg, dev)
     clk = run["clocks"]
