@@ -343,6 +343,39 @@ lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_ca
                             int32_t *dev_status, void *stream);
 
 /* ----------------------------------------------------------------------- */
+/* Prefill attention: sink and window runs as dense tiles                    */
+/* ----------------------------------------------------------------------- */
+/* lsa_attend_si is the attention of lsa_attend over sets with the SI
+ * structure lsa_index writes: the sink run [0, s), the selected tokens, the
+ * window run [ws, L) ("LongCat-Flash-Lite-Sparse (aitrends.kr)", section
+ * "기술적 특징", SI bullet; s = min(sink, L), ws = max(s, L - window)). It
+ * attends each row over
+ *    [0, s)  +  entries [s, s + m) of its set  +  [ws, L),   m = min(topk, ws - s),
+ * taking the two runs from the positions, not from the set: for a set
+ * lsa_index wrote with this budget it equals lsa_attend. Meant for the rows of
+ * a causal prefill chunk, whose neighbouring rows share their sink and (all
+ * but one position of) their window runs: those runs are attended as dense
+ * tiles of 16 rows over K/V tiles in shared memory, the selected entries by
+ * the per-row gather, and the two partials combined by their log-sum-exp.
+ *
+ * Arguments and device-side errors as lsa_attend, with the budget (sink,
+ * window, topk; hi_block and hi_topblocks unused) instead of the set length
+ * (sets are [n_q][sink + window + topk]); workspace of
+ * lsa_attend_si_workspace_size() bytes.
+ * Supported: one sequence (n_seq == 1), d == 128, H_q / H_kv <= 8, bf16 caches.
+ */
+size_t lsa_attend_si_workspace_size(const lsa_batch_t *batch, int32_t H_q, int32_t H_kv, int32_t d,
+                                    lsa_budget_t budget, int32_t layers_per_index);
+int32_t lsa_attend_si_launches(const lsa_batch_t *batch, int32_t H_q, int32_t H_kv, int32_t d,
+                               lsa_budget_t budget, int32_t layers_per_index);
+lsa_status_t lsa_attend_si(const uint16_t *const *q, const uint16_t *const *k_cache,
+                           const uint16_t *const *v_cache, int32_t H_q, int32_t H_kv, int32_t d,
+                           const int32_t *index_sets, lsa_budget_t budget,
+                           const lsa_batch_t *batch, int32_t layers_per_index,
+                           float *const *out, void *workspace, size_t workspace_bytes,
+                           int32_t *dev_status, void *stream);
+
+/* ----------------------------------------------------------------------- */
 /* Draft rows sharing one gather                                             */
 /* ----------------------------------------------------------------------- */
 /* A decode step that verifies several draft tokens of a sequence at once

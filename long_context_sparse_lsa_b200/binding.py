@@ -30,6 +30,7 @@ EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_bl
            "lsa_index_workspace_size", "lsa_index", "lsa_attend_workspace_size", "lsa_attend", "lsa_attend_fp8",
            "lsa_merge_pairs", "lsa_score_tokens", "lsa_score_blocks", "lsa_attend_lse", "lsa_shard_sets",
            "lsa_combine", "lsa_attend_grouped_workspace_size", "lsa_attend_grouped_launches", "lsa_attend_grouped",
+           "lsa_attend_si_workspace_size", "lsa_attend_si_launches", "lsa_attend_si",
            "lsa_attend_noalloc"]
 
 MERGE_ID_BITS = 24  # LSA_MERGE_ID_BITS
@@ -163,6 +164,13 @@ def load_library():
     lib.lsa_attend_grouped.restype = i32
     lib.lsa_attend_grouped.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
                                        i32, ctypes.POINTER(_Batch), i32, i32, ctypes.POINTER(vp), vp, sz, vp, vp]
+    lib.lsa_attend_si_workspace_size.restype = sz
+    lib.lsa_attend_si_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, i32, _Budget, i32]
+    lib.lsa_attend_si_launches.restype = i32
+    lib.lsa_attend_si_launches.argtypes = [ctypes.POINTER(_Batch), i32, i32, i32, _Budget, i32]
+    lib.lsa_attend_si.restype = i32
+    lib.lsa_attend_si.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
+                                  _Budget, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, sz, vp, vp]
     lib.lsa_attend_noalloc.restype = i32
     lib.lsa_attend_noalloc.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32, i32, vp,
                                        i32, ctypes.POINTER(_Batch), i32, ctypes.POINTER(vp), vp, vp]
@@ -306,6 +314,33 @@ def lsa_attend_grouped(q: list, k: list, v: list, index_sets: torch.Tensor, batc
                                 G, group_rows, oa, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _ptr(dev_status), _stream(stream))
     _check("lsa_attend_grouped", st)
+
+
+def lsa_attend_si_workspace_size(batch: Batch, H_q: int, H_kv: int, d: int, budget: Budget, layers: int) -> int:
+    return load_library().lsa_attend_si_workspace_size(ctypes.byref(batch.c()), H_q, H_kv, d, budget.c(), layers)
+
+
+def lsa_attend_si_launches(batch: Batch, H_q: int, H_kv: int, d: int, budget: Budget, layers: int) -> int:
+    return load_library().lsa_attend_si_launches(ctypes.byref(batch.c()), H_q, H_kv, d, budget.c(), layers)
+
+
+def lsa_attend_si(q: list, k: list, v: list, index_sets: torch.Tensor, budget: Budget, batch: Batch, out: list,
+                  workspace: torch.Tensor, dev_status: torch.Tensor | None = None, stream=None) -> None:
+    """lsa_attend over SI-structured sets (as lsa_index writes them): the sink
+    and window runs as dense tiles, the selected entries gathered per row."""
+    lib = load_library()
+    G = len(q)
+    n_q, H_q, d = q[0].shape
+    H_kv = k[0].shape[1]
+    if index_sets.shape[1] != budget.length:
+        raise ValueError("index_sets must be [n_q, sink + window + topk]")
+    arr = ctypes.c_void_p * G
+    qa, ka, va, oa = (arr(*[t.data_ptr() for t in x]) for x in (q, k, v, out))
+    cb = batch.c()
+    st = lib.lsa_attend_si(qa, ka, va, H_q, H_kv, d, _ptr(index_sets), budget.c(), ctypes.byref(cb), G, oa,
+                           _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                           _stream(stream))
+    _check("lsa_attend_si", st)
 
 
 def lsa_attend_lse(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list, lse: list,

@@ -431,6 +431,114 @@ lsa_status_t lsa_attend_lse(const uint16_t* const* q, const uint16_t* const* k_c
                        workspace, workspace_bytes, dev_status, stream);
 }
 
+// ---- SI split attention (prefill chunks) ---------------------------------------
+static bool si_shape_ok(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, const lsa_budget_t& b,
+                        int32_t G) {
+    const int32_t budget = b.sink + b.window + b.topk;
+    if (b.sink < 0 || b.window < 0 || b.topk < 0) return false;
+    if (!attend_shape_ok(H_q, H_kv, d, budget, G) || H_q / H_kv > 8) return false;
+    return batch->n_seq == 1 && (batch->n_q + 15) / 16 <= 0x7fffffff;
+}
+
+static lsa::AttendPlan si_plan(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d,
+                               const lsa_budget_t& b, int32_t G, size_t* lse_off) {
+    // the gather kernel's splits cover the selected entries only
+    lsa::AttendPlan p = lsa::plan_attend(batch->n_q, batch->max_len, H_q, H_kv, d, b.topk > 0 ? b.topk : 1, G,
+                                         lsa::device_sm_count());
+    *lse_off = (p.ws_bytes + 255) / 256 * 256;
+    p.ws_bytes = *lse_off + ((size_t)G * batch->n_q * H_q * 4 + 255) / 256 * 256;
+    return p;
+}
+
+size_t lsa_attend_si_workspace_size(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d,
+                                    lsa_budget_t budget, int32_t layers_per_index) {
+    if (batch == nullptr || batch->n_q <= 0 || batch->max_len < 1) return 0;
+    if (!si_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index)) return 0;
+    size_t lo;
+    return si_plan(batch, H_q, H_kv, d, budget, layers_per_index, &lo).ws_bytes;
+}
+
+int32_t lsa_attend_si_launches(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, lsa_budget_t budget,
+                               int32_t layers_per_index) {
+    if (batch == nullptr || batch->n_q <= 0) return 0;
+    if (!si_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index)) return 0;
+    size_t lo;
+    const lsa::AttendPlan p = si_plan(batch, H_q, H_kv, d, budget, layers_per_index, &lo);
+    return p.n_splits > 1 ? 3 : 2;  // gather[, split merge], sink and window tiles
+}
+
+lsa_status_t lsa_attend_si(const uint16_t* const* q, const uint16_t* const* k_cache, const uint16_t* const* v_cache,
+                           int32_t H_q, int32_t H_kv, int32_t d, const int32_t* index_sets, lsa_budget_t budget,
+                           const lsa_batch_t* batch, int32_t layers_per_index, float* const* out, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    if (!batch_ok(batch, true)) return LSA_ERR_INVALID_ARG;
+    if (H_q < 1 || H_kv < 1 || d < 1 || layers_per_index < 1) return LSA_ERR_INVALID_ARG;
+    if (budget.sink < 0 || budget.window < 0 || budget.topk < 0 || H_q % H_kv != 0) return LSA_ERR_INVALID_ARG;
+    if (!si_shape_ok(batch, H_q, H_kv, d, budget, layers_per_index)) return LSA_ERR_UNSUPPORTED;
+    if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr) return LSA_ERR_INVALID_ARG;
+    if (batch->n_q == 0) return LSA_OK;
+    const int32_t nb = budget.sink + budget.window + budget.topk;
+    if (nb > 0 && (index_sets == nullptr || !aligned(index_sets, 4))) return LSA_ERR_INVALID_ARG;
+    for (int g = 0; g < layers_per_index; ++g) {
+        if (q[g] == nullptr || k_cache[g] == nullptr || v_cache[g] == nullptr || out[g] == nullptr)
+            return LSA_ERR_INVALID_ARG;
+        if (!aligned(q[g], 16) || !aligned(k_cache[g], 16) || !aligned(v_cache[g], 16) || !aligned(out[g], 16))
+            return LSA_ERR_INVALID_ARG;
+    }
+    size_t lse_off = 0;
+    const lsa::AttendPlan p = si_plan(batch, H_q, H_kv, d, budget, layers_per_index, &lse_off);
+    if (workspace == nullptr || workspace_bytes < p.ws_bytes || !aligned(workspace, 256)) return LSA_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    lsa::AttendArgs a;
+    std::memset(&a, 0, sizeof a);
+    for (int g = 0; g < layers_per_index; ++g) {
+        a.q[g] = q[g];
+        a.k[g] = k_cache[g];
+        a.v[g] = v_cache[g];
+        a.out[g] = out[g];
+        a.lse[g] = reinterpret_cast<float*>(ws + lse_off) + (size_t)g * batch->n_q * H_q;
+        a.kscale[g] = 1.f;
+        a.vscale[g] = 1.f;
+    }
+    a.sets = index_sets;
+    a.kv_offset = batch->kv_offset;
+    a.seq_lens = batch->seq_lens;
+    a.q_seq = batch->q_seq;
+    a.q_len = batch->q_len;
+    a.dev_status = dev_status;
+    const size_t rows_q = (size_t)layers_per_index * batch->n_q;
+    if (p.n_splits > 1) {
+        a.part_o = reinterpret_cast<float*>(ws);
+        const size_t off = (rows_q * p.n_splits * H_q * 128 * 4 + 255) / 256 * 256;
+        a.part_ml = reinterpret_cast<float*>(ws + off);
+    }
+    a.total_tokens = batch->total_tokens;
+    a.n_seq = batch->n_seq;
+    a.n_q = batch->n_q;
+    a.max_len = batch->max_len;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.budget = nb;
+    a.G = layers_per_index;
+    a.n_splits = p.n_splits;
+    a.entries_per_split = p.entries_per_split;
+    a.head_groups = p.head_groups;
+    a.hpc = p.hpc;
+    a.n_stages = p.n_stages;
+    a.row_stride = p.row_stride;
+    a.bar_off = p.bar_off;
+    a.stage_off = p.stage_off;
+    a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    a.si_split = 1;
+    a.si_sink = budget.sink;
+    a.si_window = budget.window;
+    a.si_topk = budget.topk;
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = lsa::launch_attend(a, p.smem_bytes, cs);
+    if (e == cudaSuccess) e = lsa::launch_attend_window(a, cs);
+    return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
 // ---- draft-row groups --------------------------------------------------------
 static bool grouped_shape_ok(const lsa_batch_t* batch, int32_t H_q, int32_t H_kv, int32_t d, int32_t budget,
                              int32_t G, int32_t group_rows) {

@@ -607,10 +607,20 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
     const int seq_c = min(max(seq, 0), a.n_seq - 1);
     const int64_t off = a.kv_offset[seq_c];
     const int slen = a.seq_lens[seq_c];
+    // the row's entries: the whole set, or (lsa_attend_si) its selected
+    // entries [s, s + m) only, m = min(topk, ws - s)
+    int e_begin = 0, e_end = a.budget;
+    if (a.si_split) {
+        const int Lc = min(max(L, 0), a.max_len);
+        const int s = min(a.si_sink, Lc);
+        const int ws = max(s, Lc - a.si_window);
+        e_begin = min(s, a.budget);
+        e_end = min(e_begin + min(a.si_topk, ws - s), a.budget);
+    }
     pdl_enter();
     const int e0 = split * a.entries_per_split;
-    const int32_t* set = a.sets + (int64_t)r * a.budget + e0;
-    const int n_cap = max(0, min(a.budget - e0, a.entries_per_split));  // entries this split may own
+    const int32_t* set = a.sets + (int64_t)r * a.budget + e_begin + e0;
+    const int n_cap = max(0, min(e_end - e_begin - e0, a.entries_per_split));  // entries this split may own
     int32_t* s_ent = reinterpret_cast<int32_t*>(smem);
     for (int i = tid; i < n_cap; i += kConsumers * kWarp) s_ent[i] = set[i];
     const bool bad = seq < 0 || seq >= a.n_seq || L < 1 || L > a.max_len || L > slen || off < 0 ||
@@ -621,7 +631,7 @@ __global__ void __launch_bounds__(kConsumers * kWarp, 1) attend_rk_kernel(const 
         if (split == 0) clear_row(a, layer, r, hgrp * q_heads_cta, q_heads_cta, tid, kConsumers * kWarp);
         return;
     }
-    const int n_entries = min(L, a.budget);
+    const int n_entries = a.si_split ? e_end - e_begin : min(L, a.budget);
     const int n_local = max(0, min(n_entries - e0, a.entries_per_split));
     const int n_tiles = (n_local + kTile - 1) / kTile;
     for (int i = tid; i < n_tiles * kTile; i += kConsumers * kWarp) {

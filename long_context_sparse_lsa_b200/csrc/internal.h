@@ -189,6 +189,9 @@ struct AttendArgs {
     float kscale[kMaxLayers], vscale[kMaxLayers];  // FP8: value = scale * E4M3(code)
     // draft-row groups (attend_group_kernel): rows per group and per CTA
     int32_t group_rows, rows_per_cta;
+    // lsa_attend_si: the gather kernel attends only the selected entries
+    // [s, s + m) of each set; the sink and window runs are attend_window_kernel's
+    int32_t si_split, si_sink, si_window, si_topk;
 };
 
 struct AttendPlan {
@@ -203,6 +206,8 @@ cudaError_t launch_attend(const AttendArgs& a, size_t smem_bytes, cudaStream_t s
 // Draft-row groups: splits, shared memory and workspace of attend_group_kernel.
 AttendPlan plan_attend_grouped(int n_q, int group_rows, int H_q, int H_kv, int budget, int G, int num_sms);
 cudaError_t launch_attend_grouped(const AttendArgs& a, size_t smem_bytes, cudaStream_t stream);
+// lsa_attend_si's sink and window part (attend_window.cu), after the gather.
+cudaError_t launch_attend_window(const AttendArgs& a, cudaStream_t stream);
 
 int device_sm_count();
 

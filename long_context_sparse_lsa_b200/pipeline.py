@@ -33,12 +33,15 @@ def _pack(tensors, device):
 
 
 class LsaStep:
-    def __init__(self, wl: Workload, t: Tensors, device="cuda", kv_fp8: bool = False, grouped: bool = False):
+    def __init__(self, wl: Workload, t: Tensors, device="cuda", kv_fp8: bool = False, grouped: bool = False,
+                 si_attend: bool | None = None):
         """kv_fp8: the K/V caches are FP8 E4M3 codes (drawn here, per layer,
         with scales k_scale / v_scale) and the attention is lsa_attend_fp8;
         the bf16 caches of `t` are then unused and may be empty.
         grouped: the decode rows of each sequence (wl.drafts of them) attend
-        through lsa_attend_grouped, one gather of their sets' union."""
+        through lsa_attend_grouped (the rows of a group in one CTA).
+        si_attend: attend through lsa_attend_si (sink and window runs as dense
+        tiles); by default for a prefill chunk with bf16 caches."""
         self.wl = wl
         self.t = t
         self.device = device
@@ -47,6 +50,9 @@ class LsaStep:
         self.grouped = grouped
         if grouped and (kv_fp8 or wl.prefill_new):
             raise ValueError("grouped attention serves bf16 decode rows")
+        if si_attend is None:
+            si_attend = bool(wl.prefill_new) and not kv_fp8 and not grouped and wl.n_seq == 1
+        self.si_attend = si_attend
         if kv_fp8:
             shape = (wl.total_tokens, wl.H_kv, wl.d)
             self.k8 = [gen.normal_e4m3(shape, wl.seed, gen.STREAM_K8 + g, device) for g in range(self.G)]
@@ -64,9 +70,13 @@ class LsaStep:
             self.block_sums = torch.zeros((max(1, t.n_blk_rows), 2 * wl.d_I), dtype=torch.int8, device=device)
         ws_i = lsa.lsa_index_workspace_size(self.batch, wl.H_I, wl.d_I, self.budget)
         self.ws_index = torch.empty(max(1, ws_i), dtype=torch.uint8, device=device) if ws_i else None
-        ws_a = (lsa.lsa_attend_grouped_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G,
-                                                      wl.drafts) if grouped else
-                lsa.lsa_attend_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G))
+        if grouped:
+            ws_a = lsa.lsa_attend_grouped_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length,
+                                                         self.G, wl.drafts)
+        elif si_attend:
+            ws_a = lsa.lsa_attend_si_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget, self.G)
+        else:
+            ws_a = lsa.lsa_attend_workspace_size(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
         self.ws_attend = torch.zeros(max(256, ws_a), dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         # the tokens a decode step appends: each sequence's newest `drafts`
@@ -135,6 +145,9 @@ class LsaStep:
         elif self.grouped:
             lsa.lsa_attend_grouped(self.t.q, self.t.k, self.t.v, self.sets, self.batch, self.wl.drafts, self.out,
                                    self.ws_attend, self.status, stream)
+        elif self.si_attend:
+            lsa.lsa_attend_si(self.t.q, self.t.k, self.t.v, self.sets, self.budget, self.batch, self.out,
+                              self.ws_attend, self.status, stream)
         else:
             lsa.lsa_attend(self.t.q, self.t.k, self.t.v, self.sets, self.batch, self.out, self.ws_attend,
                            self.status, stream)
@@ -259,7 +272,11 @@ class LsaStep:
         the index and attention calls report for this shape."""
         wl = self.wl
         n_idx = lsa.lsa_index_launches(self.batch, wl.H_I, wl.d_I, self.budget)
-        n_att = (lsa.lsa_attend_grouped_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G,
-                                                 wl.drafts) if self.grouped else
-                 lsa.lsa_attend_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G))
+        if self.grouped:
+            n_att = lsa.lsa_attend_grouped_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G,
+                                                    wl.drafts)
+        elif self.si_attend:
+            n_att = lsa.lsa_attend_si_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget, self.G)
+        else:
+            n_att = lsa.lsa_attend_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
         return (1 if self.n_new else 0) + n_idx + n_att

@@ -206,7 +206,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch_before_launch():
 
 def test_grouped_attention_rejects_and_counts_before_launch():
     """lsa_attend_grouped: group sizes, divisibility, GQA width and the
-    staged sets' shared memory are checked before any launch."""
+    budget are checked before any launch."""
     lib = lsa.load_library()
     b = _batch(n_q=16, max_len=131072, total=4 * 131072)
     arr = (ctypes.c_void_p * 1)(P)
@@ -216,7 +216,7 @@ def test_grouped_attention_rejects_and_counts_before_launch():
     assert f(*args(D=3)) == 1                       # 16 rows are not groups of 3
     assert f(*args(D=16)) == 2                      # at most 8 rows per group
     assert f(*args(H_q=64)) == 2                    # GQA groups of at most 8 query heads
-    assert f(*args(D=8, budget=16384)) == 2         # the rows' sets would not fit in shared memory
+    assert f(*args(budget=16385)) == 2              # past LSA_MAX_BUDGET
     assert f(*args(ws=16)) == 4                     # workspace too small
     need = lib.lsa_attend_grouped_workspace_size(ctypes.byref(b), 32, 4, 128, 3136, 1, 4)
     assert need >= 16 * 32 * 128 * 4                # split partials of every (row, head)
@@ -237,3 +237,23 @@ def test_context_parallel_calls_reject_before_launch():
     arr = (ctypes.c_void_p * 1)(P)
     assert lib.lsa_attend_lse(arr, arr, arr, 32, 4, 128, P, 3136, ctypes.byref(b), 1, arr, None, P, 1 << 30,
                               None, None) == 1                                  # lse is required
+
+
+def test_si_attention_rejects_and_counts_before_launch():
+    """lsa_attend_si: one sequence, GQA groups of at most 8 heads, d = 128."""
+    lib = lsa.load_library()
+    arr = (ctypes.c_void_p * 1)(P)
+    bud = _budget(64, 1024, 2048)
+    one = _batch(n_seq=1, n_q=8192, max_len=270336, total=270336)
+    two = _batch(n_seq=2, n_q=8192, max_len=270336, total=2 * 270336)
+    f = lib.lsa_attend_si
+    assert f(arr, arr, arr, 32, 4, 128, P, bud, ctypes.byref(two), 1, arr, P, 1 << 40, None, None) == 2
+    assert f(arr, arr, arr, 64, 4, 128, P, bud, ctypes.byref(one), 1, arr, P, 1 << 40, None, None) == 2
+    assert f(arr, arr, arr, 32, 4, 64, P, bud, ctypes.byref(one), 1, arr, P, 1 << 40, None, None) == 2
+    assert f(arr, arr, arr, 32, 4, 128, P, _budget(-1, 8, 8), ctypes.byref(one), 1, arr, P, 1 << 40, None,
+             None) == 1
+    assert f(arr, arr, arr, 32, 4, 128, P, bud, ctypes.byref(one), 1, arr, P, 16, None, None) == 4
+    need = lib.lsa_attend_si_workspace_size(ctypes.byref(one), 32, 4, 128, bud, 1)
+    assert need >= 8192 * 32 * 4  # the gather's log-sum-exp per (row, head)
+    assert lib.lsa_attend_si_launches(ctypes.byref(one), 32, 4, 128, bud, 1) == 2  # gather, dense runs
+    assert lib.lsa_attend_si_launches(ctypes.byref(two), 32, 4, 128, bud, 1) == 0

@@ -420,3 +420,43 @@ def test_fp8_query_outside_fp16_range_is_flagged():
     st.attend()
     torch.cuda.synchronize()
     assert st.status_bits() & lsa.LSA_DEV_BAD_QUERY
+
+
+# lsa_attend_si on prefill chunks: the sink and window runs as dense tiles,
+# the selected entries gathered per row, against the oracle's attention over
+# the whole set and against lsa_attend on the same sets. Budgets with empty
+# runs, rows shorter than the budget, row counts off the 16-row tiles, G = 2.
+SI_CASES = {
+    "si_default": dict(lens=(5000 + 77,), prefill_new=77),
+    "si_short_rows": dict(lens=(40 + 300,), prefill_new=300, sink=16, window=64, topk=100),
+    "si_no_sink": dict(lens=(3000 + 50,), prefill_new=50, sink=0, window=128, topk=200),
+    "si_no_window": dict(lens=(3000 + 33,), prefill_new=33, sink=32, window=0, topk=200),
+    "si_no_topk": dict(lens=(2000 + 40,), prefill_new=40, sink=16, window=300, topk=0),
+    "si_wide_window": dict(lens=(1500 + 130,), prefill_new=130, sink=64, window=1400, topk=50),
+    "si_two_layers": dict(lens=(4000 + 48,), prefill_new=48, G=2),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SI_CASES))
+def test_si_attention_on_prefill_chunks(name):
+    wl = wls.small(wls.PREFILL, name=name, seed=61, **SI_CASES[name])
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    assert st.si_attend
+    st.index()
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    sets = parity.host(st.sets)
+    parity.check_sets(sets, parity.oracle_sets(wl, t), name)
+    ref = parity.oracle_attend_full(t, sets)
+    got = [parity.host(o).copy() for o in st.out]
+    for g in range(len(t.q)):
+        parity.check_attention(got[g], ref[g], f"{name} layer {g}")
+    # the same sets through lsa_attend
+    plain = LsaStep(wl, t, DEV, si_attend=False)
+    plain.sets.copy_(st.sets)
+    plain.attend()
+    torch.cuda.synchronize()
+    for g in range(len(t.q)):
+        parity.check_attention(got[g], parity.host(plain.out[g]).astype(np.float64), f"{name} vs lsa_attend")
