@@ -84,6 +84,9 @@ typedef enum {
 #define LSA_DEV_BAD_QUERY 0x20 /* lsa_attend_fp8: a query element outside the fp16 range
                                   (|q| >= 65536 as bf16, or not finite); the row's output is
                                   unspecified */
+#define LSA_DEV_BAD_VALUE 0x40 /* lsa_attend_si: a V element of magnitude >= 65520 (or not
+                                  finite) in a sink or window run, which that call multiplies
+                                  in fp16; the outputs of the rows that read it are unspecified */
 
 /* Selection budget. sink + window + topk is the index-set length ("budget").
  * hi_block == 0 switches HI off; otherwise blocks of hi_block tokens aligned
@@ -362,6 +365,9 @@ lsa_status_t lsa_attend_fp8(const uint16_t *const *q, const uint8_t *const *k_ca
  * window, topk; hi_block and hi_topblocks unused) instead of the set length
  * (sets are [n_q][sink + window + topk]); workspace of
  * lsa_attend_si_workspace_size() bytes.
+ * The dense tiles multiply P V in fp16 (every bf16 below 65520 in magnitude
+ * is an fp16; P keeps 11 significant bits): a V element of the sink or window
+ * runs of magnitude 65520 or more sets LSA_DEV_BAD_VALUE.
  * Supported: one sequence (n_seq == 1), d == 128, H_q / H_kv <= 8, bf16 caches.
  */
 size_t lsa_attend_si_workspace_size(const lsa_batch_t *batch, int32_t H_q, int32_t H_kv, int32_t d,

@@ -22,6 +22,7 @@ LSA_DEV_BAD_INDEX = 0x4
 LSA_DEV_BAD_WEIGHT = 0x8
 LSA_DEV_TIMEOUT = 0x10
 LSA_DEV_BAD_QUERY = 0x20
+LSA_DEV_BAD_VALUE = 0x40
 
 STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED", 3: "LSA_ERR_CUDA",
           4: "LSA_ERR_WORKSPACE"}

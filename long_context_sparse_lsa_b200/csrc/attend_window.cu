@@ -12,15 +12,19 @@
 // only and leaves its normalised output and log-sum-exp; this kernel attends
 // the rows over their sink and window runs and combines the two partials.
 //
-// Design: one CTA of 8 warps per (16 consecutive rows, kv head, layer). K and V
-// tiles of 16 positions (the kv head's 256-byte rows, padded to 272 bytes so
-// fragment loads are conflict free) stream through a 4-stage shared-memory
-// ring filled by 16-byte cp.async copies from all threads (positions outside
-// the runs are zero-filled). Warp w takes rows 2w and 2w + 1 of the CTA with
-// the group's query heads as the 16 rows of an m16n8k16 MMA: S = Q K^T from
-// the tile's K rows, a mask per (row, position), online softmax in fp32, P
-// split into a bf16 high part and a bf16 remainder (two MMAs, as in the
-// gather kernel) for O += P V from the tile's V rows (ldmatrix.trans).
+// Design: one CTA of 8 warps per (16 consecutive rows, kv head, layer), two
+// CTAs per SM (128 registers). K and V tiles of 16 positions (the kv head's
+// 256-byte rows, padded to 272 bytes so fragment loads are conflict free)
+// stream through a 4-stage shared-memory ring filled by 16-byte cp.async
+// copies from all threads (positions outside the runs are zero-filled). Warp
+// w takes rows 2w and 2w + 1 of the CTA with the group's query heads as the
+// 16 rows of an m16n8k16 MMA (its Q rows staged in shared memory, read as
+// ldmatrix fragments): S = Q K^T from the tile's K rows (ldmatrix; even and
+// odd k-steps in separate accumulators), a mask per (row, position), online
+// softmax in fp32, and O += P V in fp16: each V tile is converted from bf16
+// to fp16 once in shared memory (exact for magnitudes below 65520, else
+// LSA_DEV_BAD_VALUE), and P in fp16 keeps 11 significant bits, so one MMA
+// does what the gather kernel's bf16 high part and remainder do in two.
 #include "common.cuh"
 #include "internal.h"
 
@@ -36,8 +40,32 @@ constexpr int kWinRow = 128 * 2 + 16;        // bytes of one staged (position, k
 constexpr int kWinStageBytes = 2 * kWinTile * kWinRow;  // K rows then V rows
 constexpr int kD = 128;
 
-__global__ void __launch_bounds__(kWinThreads, 1) attend_window_kernel(const __grid_constant__ AttendArgs a) {
-    __shared__ __align__(128) uint8_t ring[kWinStages * kWinStageBytes];
+// Tile t's V rows from bf16 to fp16 in place, one 16-byte chunk per thread:
+// every bf16 of magnitude below 65520 is an fp16 (subnormal below 2^-14), so
+// P V can run with P in fp16 (11 significant bits: one MMA instead of a bf16
+// pair); returns false if an element does not fit.
+__device__ __forceinline__ bool v_to_f16(uint8_t* vtile, int tid) {
+    bool fits = true;
+    for (int c = tid; c < kWinTile * 16; c += kWinThreads) {
+        uint4* p = reinterpret_cast<uint4*>(vtile + (c / 16) * kWinRow + 16 * (c % 16));
+        uint4 x = *p;
+        uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+            const uint32_t h = pack_f16(f.x, f.y);
+            fits &= (h & 0x7c00u) != 0x7c00u && ((h >> 16) & 0x7c00u) != 0x7c00u;
+            w[i] = h;
+        }
+        *p = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return fits;
+}
+
+__global__ void __launch_bounds__(kWinThreads, 2) attend_window_kernel(const __grid_constant__ AttendArgs a) {
+    extern __shared__ __align__(128) uint8_t win_dyn[];
+    uint8_t* ring = win_dyn;                                        // kWinStages x (K tile, V tile)
+    uint8_t* s_qall = win_dyn + kWinStages * kWinStageBytes;        // each warp's 16 MMA rows of Q
     __shared__ int32_t s_L[kWinRows], s_s[kWinRows], s_ws[kWinRows];
     __shared__ int32_t s_span[3];  // sink run end, window runs start, end (over the CTA's rows)
     const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
@@ -112,49 +140,68 @@ __global__ void __launch_bounds__(kWinThreads, 1) attend_window_kernel(const __g
     const int ra = 2 * warp, rb = ra + 1;
     const int La = s_L[ra], sa = s_s[ra], wsa = s_ws[ra];
     const int Lb = s_L[rb], sb_ = s_s[rb], wsb = s_ws[rb];
-    uint32_t qa[kD / 16][4];
+    // the warp's Q rows into shared memory (MMA row m: row 2w + m / 8, head m % 8),
+    // read back per k-step as ldmatrix A fragments
     {
-        const bool ok = g < ratio;
-        const uint16_t* q0 = a.q[layer] + ((int64_t)(r0 + ra) * a.H_q + (int64_t)kvh * ratio + g) * kD;
-        const uint16_t* q1 = q0 + (int64_t)a.H_q * kD;
-        const bool okA = ok && La > 0, okB = ok && Lb > 0;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            const int d0 = 16 * ks + 2 * t4;
-            qa[ks][0] = okA ? __ldg(reinterpret_cast<const uint32_t*>(q0 + d0)) : 0u;
-            qa[ks][1] = okB ? __ldg(reinterpret_cast<const uint32_t*>(q1 + d0)) : 0u;
-            qa[ks][2] = okA ? __ldg(reinterpret_cast<const uint32_t*>(q0 + d0 + 8)) : 0u;
-            qa[ks][3] = okB ? __ldg(reinterpret_cast<const uint32_t*>(q1 + d0 + 8)) : 0u;
+        uint8_t* qs = s_qall + warp * 16 * kWinRow;
+        for (int c = lane; c < 16 * 16; c += kWarp) {  // 16 rows x 16 chunks of 16 bytes
+            const int m = c / 16, ch = c % 16;
+            const int rl = ra + (m >> 3), h = m & 7;
+            const bool ok = h < ratio && s_L[rl] > 0;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (ok)
+                v = __ldg(reinterpret_cast<const uint4*>(
+                    a.q[layer] + ((int64_t)(r0 + rl) * a.H_q + (int64_t)kvh * ratio + h) * kD) + ch);
+            *reinterpret_cast<uint4*>(qs + m * kWinRow + 16 * ch) = v;
         }
+        __syncwarp();
     }
+    // lane l addresses row (l & 7) + 8 ((l >> 3) & 1), 16-byte column (l >> 4)
+    // of each k-step's 16 x 16 block: the four 8 x 8 matrices of the A fragment
+    const uint32_t qrow = smem_u32(s_qall + warp * 16 * kWinRow) + (uint32_t)(((lane & 7) + 8 * ((lane >> 3) & 1)) * kWinRow + 16 * (lane >> 4));
+    // and for K: matrices (positions 0-7 | 8-15) x (dims lo | hi) of a k-step
+    const uint32_t krow_off = (uint32_t)(((lane & 7) + 8 * (lane >> 4)) * kWinRow + 16 * ((lane >> 3) & 1));
     float o[kD / 8][4];
 #pragma unroll
     for (int j = 0; j < kD / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
     const float sl2 = a.scale_log2;
 
-    for (int t = 0; t < n_t; ++t) {
+    bool v_fits = true;
+    if (n_t > 0) {
         cp_async_wait<kWinStages - 2>();
-        __syncthreads();                 // tile t landed for every thread; tile t - 1 is no longer read
+        __syncthreads();
+        v_fits &= v_to_f16(ring + kWinTile * kWinRow, tid);  // tile 0's V rows
+    }
+    for (int t = 0; t < n_t; ++t) {
+        // tiles t and t + 1 have landed for every thread, tile t's V rows are
+        // fp16 (converted an iteration ago), tile t - 1 is no longer read
+        cp_async_wait<kWinStages - 3>();
+        __syncthreads();
+        if (t + 1 < n_t) v_fits &= v_to_f16(ring + ((t + 1) % kWinStages) * kWinStageBytes + kWinTile * kWinRow, tid);
         stage(t + kWinStages - 1);       // into the stage tile t - 1 used
         const uint8_t* st = ring + (t % kWinStages) * kWinStageBytes;
         const uint32_t kbase = smem_u32(st), vbase = smem_u32(st + kWinTile * kWinRow);
         const int pb = tile_base(t), pe = tile_end(t);
-        // S = Q K^T: two n-tiles of 8 positions
-        float sacc[2][4];
+        // S = Q K^T: two n-tiles of 8 positions, even and odd k-steps in
+        // separate accumulators (four independent MMA chains)
+        float sacc[2][4], sodd[2][4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sacc[n][c] = sodd[n][c] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                const uint32_t rowa = kbase + (uint32_t)((8 * n + g) * kWinRow + 2 * (16 * ks + 2 * t4));
-                uint32_t b0, b1;
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b0) : "r"(rowa));
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b1) : "r"(rowa + 16u));
-                mma_16<false>(sacc[n], qa[ks], b0, b1);
-            }
+            uint32_t qa[4], kb[4];
+            ldmatrix_x4(qa, qrow + (uint32_t)(32 * ks));
+            ldmatrix_x4(kb, kbase + krow_off + (uint32_t)(32 * ks));
+            mma_16<false>((ks & 1) ? sodd[0] : sacc[0], qa, kb[0], kb[1]);
+            mma_16<false>((ks & 1) ? sodd[1] : sacc[1], qa, kb[2], kb[3]);
         }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sacc[n][c] += sodd[n][c];
         // mask: row A holds positions [0, sa) and [wsa, La), row B likewise
         float z[2][4];
 #pragma unroll
@@ -201,36 +248,22 @@ __global__ void __launch_bounds__(kWinThreads, 1) attend_window_kernel(const __g
         mA = nA;
         mB = nB;
         // P as the A operand (the two n-tiles' accumulators are the k16
-        // fragment), split into a bf16 high part and its remainder
-        uint32_t ph[4], pl[4];
-        {
-            const float2 h0 = __bfloat1622float2(__floats2bfloat162_rn(p[0][0], p[0][1]));
-            const float2 h1 = __bfloat1622float2(__floats2bfloat162_rn(p[0][2], p[0][3]));
-            const float2 h2 = __bfloat1622float2(__floats2bfloat162_rn(p[1][0], p[1][1]));
-            const float2 h3 = __bfloat1622float2(__floats2bfloat162_rn(p[1][2], p[1][3]));
-            ph[0] = pack_bf16(h0.x, h0.y);
-            ph[1] = pack_bf16(h1.x, h1.y);
-            ph[2] = pack_bf16(h2.x, h2.y);
-            ph[3] = pack_bf16(h3.x, h3.y);
-            pl[0] = pack_bf16(p[0][0] - h0.x, p[0][1] - h0.y);
-            pl[1] = pack_bf16(p[0][2] - h1.x, p[0][3] - h1.y);
-            pl[2] = pack_bf16(p[1][0] - h2.x, p[1][1] - h2.y);
-            pl[3] = pack_bf16(p[1][2] - h3.x, p[1][3] - h3.y);
-        }
-        // O += P V: V rows (positions) x dims through ldmatrix.trans, two
-        // n-tiles of 8 dims per load
+        // fragment), in fp16: p in [0, 1] keeps 11 significant bits
+        const uint32_t ph[4] = {pack_f16(p[0][0], p[0][1]), pack_f16(p[0][2], p[0][3]), pack_f16(p[1][0], p[1][1]),
+                                pack_f16(p[1][2], p[1][3])};
+        // O += P V: the tile's fp16 V rows (positions) x dims through
+        // ldmatrix.trans, two n-tiles of 8 dims per load
         const uint32_t vrow = vbase + (uint32_t)(((lane & 7) + 8 * ((lane >> 3) & 1)) * kWinRow + 16 * (lane >> 4));
 #pragma unroll
         for (int j = 0; j < kD / 8; j += 2) {
             uint32_t vb[4];
             ldmatrix_x4_trans(vb, vrow + (uint32_t)(16 * j));
-            mma_16<false>(o[j], ph, vb[0], vb[1]);
-            mma_16<false>(o[j], pl, vb[0], vb[1]);
-            mma_16<false>(o[j + 1], ph, vb[2], vb[3]);
-            mma_16<false>(o[j + 1], pl, vb[2], vb[3]);
+            mma_16<true>(o[j], ph, vb[0], vb[1]);
+            mma_16<true>(o[j + 1], ph, vb[2], vb[3]);
         }
     }
     cp_async_wait<0>();
+    if (!v_fits) flag(a.dev_status, LSA_DEV_BAD_VALUE);
 
     // the rows' denominators over their quad, then the window part's lse and
     // its combination with the selected part (attend_rk_kernel's output and
@@ -272,8 +305,11 @@ __global__ void __launch_bounds__(kWinThreads, 1) attend_window_kernel(const __g
 }  // namespace
 
 cudaError_t launch_attend_window(const AttendArgs& a, cudaStream_t stream) {
+    constexpr size_t smem = (size_t)kWinStages * kWinStageBytes + (size_t)kWinWarps * 16 * kWinRow;
+    cudaError_t e = cudaFuncSetAttribute(attend_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.n_q + kWinRows - 1) / kWinRows), (unsigned)a.H_kv, (unsigned)a.G);
-    return launch_pdl(attend_window_kernel, grid, dim3(kWinThreads), 0, stream, 0, a);
+    return launch_pdl(attend_window_kernel, grid, dim3(kWinThreads), smem, stream, 0, a);
 }
 
 }  // namespace lsa

@@ -460,3 +460,16 @@ def test_si_attention_on_prefill_chunks(name):
     torch.cuda.synchronize()
     for g in range(len(t.q)):
         parity.check_attention(got[g], parity.host(plain.out[g]).astype(np.float64), f"{name} vs lsa_attend")
+
+
+def test_si_attention_flags_values_beyond_fp16():
+    """A V element of magnitude >= 65520 inside a window run cannot enter the
+    fp16 P V of the dense tiles: LSA_DEV_BAD_VALUE."""
+    wl = wls.small(wls.PREFILL, name="si_big_v", lens=(2000 + 32,), prefill_new=32, seed=62)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.index()
+    t.v[0][wl.lens[0] - wl.prefill_new - 5, 0, 3] = 1.0e6  # inside every row's window run
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() & lsa.LSA_DEV_BAD_VALUE
