@@ -473,3 +473,22 @@ def test_si_attention_flags_values_beyond_fp16():
     st.attend()
     torch.cuda.synchronize()
     assert st.status_bits() & lsa.LSA_DEV_BAD_VALUE
+
+
+def test_si_attention_on_a_2048_row_chunk():
+    """lsa_attend_si on 2048 rows of a 65,536-token cache (128 dense tiles of
+    16 rows per kv head): 64 rows spread over the chunk (first and last
+    included) against the oracle."""
+    wl = wls.PREFILL_PROFILE
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    assert st.si_attend
+    st.index()
+    st.attend()
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    rows = sorted(set(np.linspace(0, wl.n_q - 1, 64).astype(int).tolist()))
+    sets = parity.host(st.sets)[rows]
+    want = parity.oracle_attend_rows(t, sets, rows)
+    for g in range(len(t.q)):
+        parity.check_attention(parity.host(st.out[g])[rows], want[g], f"2048-row chunk layer {g}")
