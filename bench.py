@@ -452,14 +452,15 @@ def job_rate(units_per_rank: int, world: int, ms: float) -> float:
 
 
 # ---------------------------------------------------------------------------
-def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, kv_fp8=False, grouped=False):
+def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, kv_fp8=False, grouped=False,
+                  fuse_append=True):
     """Draws the workload, captures its step graphs and times `steps` steps
     (after `warmup`), each after an L2 flush: the whole step graph for the
     headline, then the three calls one by one for the breakdown."""
     from long_context_sparse_lsa_b200.pipeline import LsaStep
 
     t = wls.make(wl, dev, with_kv=not kv_fp8)
-    st = LsaStep(wl, t, dev, kv_fp8=kv_fp8, grouped=grouped)
+    st = LsaStep(wl, t, dev, kv_fp8=kv_fp8, grouped=grouped, fuse_append=fuse_append)
     st.pack_io()  # one input and one output buffer per step (the e2e leg copies each once)
     st.build_block_sums()
     torch.cuda.synchronize()
@@ -542,7 +543,8 @@ def time_workload(wl, dev, flush, stream, steps, warmup, pg=None, clocks=None, k
     return {"st": st, "t": t, "ms": ms, "clocks": clk, "n_kernels": st.kernels_per_step(), "cold": cold,
             "bs": [e[0].elapsed_time(e[1]) for e in sevs], "ix": [e[1].elapsed_time(e[2]) for e in sevs],
             "at": [e[2].elapsed_time(e[3]) for e in sevs],
-            "ix_in_step": [c["index"] for c in in_step], "at_in_step": [c["attend"] for c in in_step]}
+            "ix_in_step": [c["index"] for c in in_step], "at_in_step": [c["attend"] for c in in_step],
+            "fused_append": bool(st.n_new) and st.fuse_append}
 
 
 def draft_union_entries(sets: torch.Tensor, drafts: int) -> int:
@@ -567,7 +569,7 @@ def cold_line(wl, cold_ms, world, pg, dev):
                     "then index, then attention; one CUDA graph, L2 flushed before each step)"}
 
 
-def secondary(dev, flush, stream, steps, warmup, peak):
+def secondary(dev, flush, stream, steps, warmup, peak, fuse_append=True):
     """The 1M-token decode (G = 4) and the 8192-token prefill chunk, each
     measured like the headline (step graph, L2 flush, CUDA events)."""
     from long_context_sparse_lsa_b200 import binding as lsa
@@ -581,7 +583,7 @@ def secondary(dev, flush, stream, steps, warmup, peak):
     for wl, fp8 in ((wls.CTX1M, False), (wls.PREFILL, False), (wls.BATCH128K, True), (wls.ragged(), False),
                     (wls.DRAFTS128K, False)):
         drafts = wl.drafts > 1
-        run = time_workload(wl, dev, flush, stream, steps, warmup, kv_fp8=fp8)
+        run = time_workload(wl, dev, flush, stream, steps, warmup, kv_fp8=fp8, fuse_append=fuse_append)
         st = run["st"]
         ms = run["ms"]
         byts = step_bytes(wl, kv_fp8=fp8)
@@ -684,6 +686,8 @@ def main(argv=None):
                     help="skip the 1M decode and prefill chunk measurements")
     ap.add_argument("--grouped", action="store_true",
                     help="draft-row workloads: attend through lsa_attend_grouped")
+    ap.add_argument("--no-fuse-append", action="store_true",
+                    help="decode steps: lsa_append then lsa_index instead of lsa_append_index")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     wl = wls.by_name(args.workload)
@@ -712,7 +716,7 @@ def main(argv=None):
     wl_r = rank_workload(wl, rank)
     clocks = ClockSampler(local)
     run = time_workload(wl_r, dev, flush, stream, args.steps, args.warmup, pg, clocks,
-                        grouped=args.grouped and wl.drafts > 1)
+                        grouped=args.grouped and wl.drafts > 1, fuse_append=not args.no_fuse_append)
     st, t = run["st"], run["t"]
     ms = max_over_ranks(run["ms"], pg, dev)
     clk = run["clocks"]
@@ -762,13 +766,18 @@ def main(argv=None):
                       "one replay per timed step (L2 flushed before each)"}
     # the index call against the same roofline: its algorithmic bytes (block
     # sums of the candidate blocks, the kept blocks' keys, queries, weights,
-    # the written sets) over its duration inside the step
-    roof_index = {"bound": "hbm", "kernel": "lsa_index call (block selection with the HI coarse scores, fine "
-                                            "scores, token selection with the SI assembly)",
-                  "achieved": byts["index"] / (ix_in / 1000.0) / 1e9, "peak": peak, "unit": "GB/s",
-                  "frac": byts["index"] / (ix_in / 1000.0) / 1e9 / peak, "peak_kind": peak_kind,
-                  "traffic": None, "bytes_per_launch": byts["index"], "ms_per_launch": ix_in,
-                  "timing": "CUDA events recorded inside the step graph around the lsa_index call, mean over "
+    # the written sets; plus the append's when the call is lsa_append_index)
+    # over its duration inside the step
+    fused = run["fused_append"]
+    ix_bytes = byts["index"] + (byts["append"] if fused else 0)
+    ix_call = "lsa_append_index" if fused else "lsa_index"
+    roof_index = {"bound": "hbm", "kernel": f"{ix_call} call (block selection with the HI coarse scores"
+                                            f"{' and the decode append' if fused else ''}, fine scores, token "
+                                            "selection with the SI assembly)",
+                  "achieved": ix_bytes / (ix_in / 1000.0) / 1e9, "peak": peak, "unit": "GB/s",
+                  "frac": ix_bytes / (ix_in / 1000.0) / 1e9 / peak, "peak_kind": peak_kind,
+                  "traffic": None, "bytes_per_launch": ix_bytes, "ms_per_launch": ix_in,
+                  "timing": f"CUDA events recorded inside the step graph around the {ix_call} call, mean over "
                             "one replay per timed step (L2 flushed before each)"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -780,7 +789,17 @@ def main(argv=None):
                                                             "hi_topblocks": wl.hi_topblocks},
                        "heads": {"H_I": wl.H_I, "d_I": wl.d_I, "H_q": wl.H_q, "H_kv": wl.H_kv, "d": wl.d},
                        "l2": "flushed before every timed step (2 x L2 write, outside the timed interval)",
-                       "launch": "each step replayed from one CUDA graph captured through the C ABI: the decode append (new tokens' keys and K/V rows written, their block sums refreshed), the index call and the attention call on one stream, every kernel launched with programmatic stream serialisation; step_breakdown_ms from per-call graphs replayed in sequence (each with its own graph launch); call_ms_in_step from timing events inside the step graph",
+                       "launch": ("each step replayed from one CUDA graph captured through the C ABI: "
+                                  + ("lsa_append_index (the decode append, new tokens' keys and K/V rows written "
+                                     "and their block sums refreshed, run by extra CTAs of the block selection; "
+                                     "then the index call's kernels)" if fused else
+                                     "the decode append (new tokens' keys and K/V rows written, their block sums "
+                                     "refreshed), the index call")
+                                  + " and the attention call on one stream, every kernel launched with "
+                                  "programmatic stream serialisation; step_breakdown_ms from per-call graphs "
+                                  "replayed in sequence (each with its own graph launch: lsa_append, lsa_index, "
+                                  "lsa_attend); call_ms_in_step from timing events inside the step graph"
+                                  + (" (its index figure includes the fused append)" if fused else "")),
                        "parallelism": f"replicas x{world} (independent batches, no collective)"},
             "step_breakdown_ms": {"append": bsu, "index": ix, "attend": at},
             "call_ms_in_step": {"index": ix_in, "attend": at_in},
@@ -807,7 +826,8 @@ def main(argv=None):
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
         try:
-            line["secondary"] = secondary(dev, flush, stream, min(args.steps, 10), args.warmup, peak)
+            line["secondary"] = secondary(dev, flush, stream, min(args.steps, 10), args.warmup, peak,
+                                          fuse_append=not args.no_fuse_append)
         except Exception as exc:  # the headline line still prints; the failure is reported in it
             print(f"secondary workloads failed: {exc!r}", file=sys.stderr, flush=True)
             line["secondary"] = {"error": repr(exc)}

@@ -272,6 +272,49 @@ lsa_status_t lsa_index(const int8_t *q_idx, const int8_t *k_idx_cache,
                        int32_t *dev_status, void *stream);
 
 /* ----------------------------------------------------------------------- */
+/* Decode append and index in one call                                       */
+/* ----------------------------------------------------------------------- */
+/* lsa_append followed by lsa_index on the same batch, with the results of
+ * those two calls in that order (a decode step's first two calls: the new
+ * tokens enter the cache whose keys and block sums the HI block pass of the
+ * Flash-Lite-Sparse page, "기술적 특징", Hierarchical Indexing bullet,
+ * scores).
+ *
+ * When HI is on and budget.window >= hi_block + n_new - 1, the n_new newest
+ * tokens of every sequence lie in every row's window: the index call reads
+ * no key, block sum or K/V row that the append writes, and the append runs in
+ * extra CTAs of the block selection's grid instead of a launch of its own
+ * (one kernel boundary fewer in the step). Otherwise the two calls' kernels
+ * are launched one after the other.
+ *
+ * Arguments: those of lsa_append (k_idx_new, k_new, v_new, k_cache, v_cache,
+ * kv_row_bytes, layers, n_new; hi_block is budget.hi_block) and of lsa_index
+ * (q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums,
+ * block_rows, index_sets, workspace, workspace_bytes), with the same meaning,
+ * layout, ownership and support limits; workspace is lsa_index's. Every check
+ * of both calls runs before the first launch: a refused call launches
+ * nothing. Device errors set the same dev_status bits as the two calls.
+ */
+lsa_status_t lsa_append_index(const int8_t *k_idx_new, const void *const *k_new,
+                              const void *const *v_new, void *const *k_cache,
+                              void *const *v_cache, int32_t kv_row_bytes,
+                              int32_t layers, int32_t n_new,
+                              const int8_t *q_idx, int8_t *k_idx_cache,
+                              const int32_t *w, int32_t w_max, int32_t H_I,
+                              int32_t d_I, const lsa_batch_t *batch,
+                              lsa_budget_t budget, int8_t *block_sums,
+                              int64_t block_rows, int32_t *index_sets,
+                              void *workspace, size_t workspace_bytes,
+                              int32_t *dev_status, void *stream);
+
+/* Kernel launches lsa_append_index makes for this shape (reads only host
+ * fields): lsa_index_launches, plus one when the append is not fused. 0 for
+ * invalid arguments. */
+int32_t lsa_append_index_launches(const lsa_batch_t *batch, int32_t H_I,
+                                  int32_t d_I, lsa_budget_t budget,
+                                  int32_t n_new);
+
+/* ----------------------------------------------------------------------- */
 /* Sparse attention over the index sets (all G layers of a CLI group)        */
 /* ----------------------------------------------------------------------- */
 /* Workspace bytes lsa_attend needs (split partials; contents need no

@@ -32,7 +32,7 @@ EXPORTS = ["lsa_version", "lsa_last_cuda_error", "lsa_status_string", "lsa_hi_bl
            "lsa_merge_pairs", "lsa_score_tokens", "lsa_score_blocks", "lsa_attend_lse", "lsa_shard_sets",
            "lsa_combine", "lsa_attend_grouped_workspace_size", "lsa_attend_grouped_launches", "lsa_attend_grouped",
            "lsa_attend_si_workspace_size", "lsa_attend_si_launches", "lsa_attend_si",
-           "lsa_attend_noalloc"]
+           "lsa_attend_noalloc", "lsa_append_index", "lsa_append_index_launches"]
 
 MERGE_ID_BITS = 24  # LSA_MERGE_ID_BITS
 
@@ -126,6 +126,12 @@ def load_library():
     lib.lsa_append.restype = i32
     lib.lsa_append.argtypes = [vp, vp, i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                ctypes.POINTER(vp), i32, i32, i32, vp, i64, ctypes.POINTER(_Batch), i32, vp, vp]
+    lib.lsa_append_index.restype = i32
+    lib.lsa_append_index.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                     i32, i32, i32, vp, vp, vp, i32, i32, i32, ctypes.POINTER(_Batch), _Budget, vp, i64,
+                                     vp, vp, sz, vp, vp]
+    lib.lsa_append_index_launches.restype = i32
+    lib.lsa_append_index_launches.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget, i32]
     lib.lsa_index_workspace_size.restype = sz
     lib.lsa_index_workspace_size.argtypes = [ctypes.POINTER(_Batch), i32, i32, _Budget]
     lib.lsa_index_launches.restype = i32
@@ -269,6 +275,34 @@ def lsa_append(k_idx_new: torch.Tensor, k_idx: torch.Tensor, k_new: list, v_new:
     st = lib.lsa_append(_ptr(k_idx_new), _ptr(k_idx), d_I, kn, vn, kc, vc, row_bytes, G, hi_block, _ptr(block_sums),
                         rows, ctypes.byref(cb), n_new, _ptr(dev_status), _stream(stream))
     _check("lsa_append", st)
+
+
+def lsa_append_index(k_idx_new: torch.Tensor, k_new: list, v_new: list, k: list, v: list, n_new: int,
+                     q_idx: torch.Tensor, k_idx: torch.Tensor, w: torch.Tensor, w_max: int, batch: Batch,
+                     budget: Budget, index_sets: torch.Tensor, block_sums: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                     stream=None) -> None:
+    """lsa_append (the n_new newest tokens' keys and K/V rows, their blocks' sums) followed by lsa_index, in one
+    call; with HI on and the new tokens inside every window the append runs inside the block selection."""
+    lib = load_library()
+    G = len(k_new)
+    n_q, H_I, d_I = q_idx.shape
+    row_bytes = k[0].shape[1] * k[0].shape[2] * k[0].element_size() if G else 0
+    arr = ctypes.c_void_p * max(G, 1)
+    kn, vn, kc, vc = (arr(*[t.data_ptr() for t in x]) for x in (k_new, v_new, k, v))
+    cb = batch.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rows = block_sums.shape[0] if block_sums is not None else 0
+    st = lib.lsa_append_index(_ptr(k_idx_new), kn, vn, kc, vc, row_bytes, G, n_new, _ptr(q_idx), _ptr(k_idx), _ptr(w),
+                              w_max, H_I, d_I, ctypes.byref(cb), budget.c(), _ptr(block_sums), rows,
+                              _ptr(index_sets), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    _check("lsa_append_index", st)
+
+
+def lsa_append_index_launches(batch: Batch, H_I: int, d_I: int, budget: Budget, n_new: int) -> int:
+    """Kernel launches lsa_append_index issues for this shape."""
+    cb = batch.c()
+    return int(load_library().lsa_append_index_launches(ctypes.byref(cb), H_I, d_I, budget.c(), n_new))
 
 
 def lsa_attend(q: list, k: list, v: list, index_sets: torch.Tensor, batch: Batch, out: list,

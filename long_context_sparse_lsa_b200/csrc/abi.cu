@@ -115,11 +115,14 @@ lsa_status_t lsa_hi_block_sums(const int8_t* k_idx_cache, int32_t d_I, int32_t h
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
 
-lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_I, const void* const* k_new,
-                        const void* const* v_new, void* const* k_cache, void* const* v_cache,
-                        int32_t kv_row_bytes, int32_t layers, int32_t hi_block, int8_t* block_sums,
-                        int64_t block_rows, const lsa_batch_t* batch, int32_t n_new, int32_t* dev_status,
-                        void* stream) {
+}  // extern "C"
+
+// Checks lsa_append's arguments and fills the kernel arguments.
+static lsa_status_t append_args(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_I, const void* const* k_new,
+                                const void* const* v_new, void* const* k_cache, void* const* v_cache,
+                                int32_t kv_row_bytes, int32_t layers, int32_t hi_block, int8_t* block_sums,
+                                int64_t block_rows, const lsa_batch_t* batch, int32_t n_new, int32_t* dev_status,
+                                lsa::AppendArgs& a) {
     if (!batch_ok(batch, false)) return LSA_ERR_INVALID_ARG;
     if (n_new < 1 || d_I < 1 || layers < 0 || hi_block < 0 || block_rows < 0) return LSA_ERR_INVALID_ARG;
     if (d_I != 32 && d_I != 64 && d_I != 128) return LSA_ERR_UNSUPPORTED;
@@ -141,7 +144,6 @@ lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_
         }
     }
     if (batch->n_seq > 65535) return LSA_ERR_UNSUPPORTED;
-    lsa::AppendArgs a;
     std::memset(&a, 0, sizeof a);
     a.bs.k_idx = k_idx_cache;
     a.bs.block_sums = block_sums;
@@ -166,6 +168,20 @@ lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_
     a.layers = layers;
     a.kv_row_bytes = layers > 0 ? kv_row_bytes : 0;
     a.sums = hi_block > 0 ? 1 : 0;
+    return LSA_OK;
+}
+
+extern "C" {
+
+lsa_status_t lsa_append(const int8_t* k_idx_new, int8_t* k_idx_cache, int32_t d_I, const void* const* k_new,
+                        const void* const* v_new, void* const* k_cache, void* const* v_cache,
+                        int32_t kv_row_bytes, int32_t layers, int32_t hi_block, int8_t* block_sums,
+                        int64_t block_rows, const lsa_batch_t* batch, int32_t n_new, int32_t* dev_status,
+                        void* stream) {
+    lsa::AppendArgs a;
+    const lsa_status_t st = append_args(k_idx_new, k_idx_cache, d_I, k_new, v_new, k_cache, v_cache, kv_row_bytes,
+                                        layers, hi_block, block_sums, block_rows, batch, n_new, dev_status, a);
+    if (st != LSA_OK) return st;
     cudaError_t e = lsa::launch_append(a, d_I, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
 }
@@ -226,14 +242,24 @@ static lsa_status_t index_validate(const int8_t* q_idx, const int8_t* k_idx_cach
     return LSA_OK;
 }
 
-lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max, int32_t H_I,
-                       int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget, const int8_t* block_sums,
-                       int64_t block_rows, int32_t* index_sets, void* workspace, size_t workspace_bytes,
-                       int32_t* dev_status, void* stream) {
-    lsa_status_t st = index_validate(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums, block_rows,
-                                     index_sets);
-    if (st != LSA_OK) return st;
-    if (batch->n_q == 0) return LSA_OK;
+}  // extern "C"
+
+// The append may run inside the block selection when the two touch disjoint
+// memory: HI on, and the n_new newest tokens' blocks inside every row's
+// window (window >= hi_block + n_new - 1), so that no candidate block sum
+// and no candidate key is written by the append; the fine scores and the
+// token selection wait for the whole block-selection grid.
+static bool append_fusable(const lsa_budget_t& b, int32_t n_new) {
+    return b.hi_block > 0 && n_new >= 1 && (int64_t)b.window >= (int64_t)b.hi_block + n_new - 1;
+}
+
+// lsa_index after validation; app (nullable) is a decode append to run in
+// extra CTAs of the block selection (append_fusable holds).
+static lsa_status_t index_impl(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max,
+                               int32_t H_I, int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget,
+                               const int8_t* block_sums, int64_t block_rows, int32_t* index_sets, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream,
+                               const lsa::AppendArgs* app) {
     if (budget.hi_block == 0) budget.hi_topblocks = 0;
 
     const bool dense = index_dense(batch, H_I, d_I, budget);
@@ -282,11 +308,19 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
     a.coarse_stage = plan.coarse_stage;
     a.fine_stage = plan.fine_stage;
     a.kept_slots = plan.kept_slots;
+    if (app != nullptr) {
+        a.app = *app;
+        a.app_per_seq = lsa::append_ctas_per_seq(app->bs.n_new, app->bs.hi_block, app->bs.max_len);
+        a.app_tasks = a.app_per_seq * app->bs.n_seq * 2;  // copy and block-sum roles
+        a.app_dI = d_I;
+        if ((int64_t)batch->n_q + lsa::index_select_append_rows(a, plan.cluster) > 65535) return LSA_ERR_UNSUPPORTED;
+    }
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (budget.hi_block > 0) {
         if (!lsa::coarse_in_select(a)) e = lsa::launch_index_scores(a, d_I, true, cs);
         if (e == cudaSuccess) e = lsa::launch_index_select(a, true, d_I, plan.cluster, plan.smem_blocks, cs);
+        a.app_tasks = 0;  // the later kernels carry no append
     }
     if (e == cudaSuccess) {
         // a prefill chunk (many rows of one sequence, HI off) is one dense
@@ -298,6 +332,61 @@ lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int
                   : lsa::launch_index_select(a, false, d_I, plan.cluster, plan.smem_tokens, cs);
     }
     return e == cudaSuccess ? LSA_OK : cuda_fail(e);
+}
+
+extern "C" {
+
+lsa_status_t lsa_index(const int8_t* q_idx, const int8_t* k_idx_cache, const int32_t* w, int32_t w_max, int32_t H_I,
+                       int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget, const int8_t* block_sums,
+                       int64_t block_rows, int32_t* index_sets, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, void* stream) {
+    const lsa_status_t st = index_validate(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums,
+                                           block_rows, index_sets);
+    if (st != LSA_OK) return st;
+    if (batch->n_q == 0) return LSA_OK;
+    return index_impl(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums, block_rows, index_sets,
+                      workspace, workspace_bytes, dev_status, stream, nullptr);
+}
+
+int32_t lsa_append_index_launches(const lsa_batch_t* batch, int32_t H_I, int32_t d_I, lsa_budget_t budget,
+                                  int32_t n_new) {
+    if (batch == nullptr || n_new < 1) return 0;
+    const int32_t n_idx = batch->n_q > 0 ? lsa_index_launches(batch, H_I, d_I, budget) : 0;
+    if (n_idx == 0 && batch->n_q > 0) return 0;
+    return n_idx + (batch->n_q > 0 && append_fusable(budget, n_new) ? 0 : 1);
+}
+
+lsa_status_t lsa_append_index(const int8_t* k_idx_new, const void* const* k_new, const void* const* v_new,
+                              void* const* k_cache, void* const* v_cache, int32_t kv_row_bytes, int32_t layers,
+                              int32_t n_new, const int8_t* q_idx, int8_t* k_idx_cache, const int32_t* w,
+                              int32_t w_max, int32_t H_I, int32_t d_I, const lsa_batch_t* batch, lsa_budget_t budget,
+                              int8_t* block_sums, int64_t block_rows, int32_t* index_sets, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    if (!budget_ok(budget)) return LSA_ERR_INVALID_ARG;
+    lsa::AppendArgs app;
+    lsa_status_t st = append_args(k_idx_new, k_idx_cache, d_I, k_new, v_new, k_cache, v_cache, kv_row_bytes, layers,
+                                  budget.hi_block, block_sums, block_rows, batch, n_new, dev_status, app);
+    if (st != LSA_OK) return st;
+    st = index_validate(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums, block_rows, index_sets);
+    if (st != LSA_OK) return st;
+    if (batch->n_q > 0 && append_fusable(budget, n_new))  // (index_impl checks everything before its first launch)
+        return index_impl(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums, block_rows, index_sets,
+                          workspace, workspace_bytes, dev_status, stream, &app);
+    if (batch->n_q > 0) {
+        // the checks index_impl makes before its first launch, ahead of the
+        // append's launch, so that a refused call launches nothing
+        lsa_budget_t b = budget;
+        if (b.hi_block == 0) b.hi_topblocks = 0;
+        const lsa::IndexPlan plan = lsa::plan_index(batch->n_q, batch->max_len, b, index_dense(batch, H_I, d_I, b));
+        if (plan.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < plan.ws_bytes || !aligned(workspace, 256)))
+            return LSA_ERR_WORKSPACE;
+        if (batch->n_q > 65535) return LSA_ERR_UNSUPPORTED;
+    }
+    cudaError_t e = lsa::launch_append(app, d_I, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (batch->n_q == 0) return LSA_OK;
+    return index_impl(q_idx, k_idx_cache, w, w_max, H_I, d_I, batch, budget, block_sums, block_rows, index_sets,
+                      workspace, workspace_bytes, dev_status, stream, nullptr);
 }
 
 // ---------------------------------------------------------------------------

@@ -27,6 +27,7 @@
 //      with one CTA prefix give every kept key its rank in position order.
 #include <algorithm>
 
+#include "append.cuh"
 #include "common.cuh"
 #include "index_common.cuh"
 #include "internal.h"
@@ -595,9 +596,34 @@ __device__ void coarse_pass(SelShared& sh, const IndexArgs& a, int r, int64_t bo
 // assembly of the index set; otherwise the HI block top-k.
 // D_I > 0 (HI blocks only): the coarse scores are computed in place
 // (coarse_pass) instead of read from the coarse scoring kernel's workspace.
+//
+// Block selection only: rows n_q onwards of the grid are a decode step's
+// append (append_task), one task per CTA, when the caller fuses it here. The
+// block selection and the append then touch disjoint memory (the new tokens'
+// blocks lie in the window, never among the candidate blocks), and every
+// later kernel of the step waits for this grid, so the append costs no
+// kernel boundary of its own.
 template <typename K, bool kTokens, int D_I = 0, int NT = 0>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_constant__ IndexArgs a) {
     extern __shared__ __align__(16) uint8_t dyn[];
+    if constexpr (!kTokens) {
+        if (blockIdx.y >= (unsigned)a.n_q) {  // uniform over the cluster: no cluster barrier is used
+            pdl_enter();                      // the caches may still be read by the preceding kernels
+            const int t = (int)((blockIdx.y - (unsigned)a.n_q) * gridDim.x + blockIdx.x);
+            if (t < a.app_tasks) {
+                const int per_role = a.app_per_seq * a.app.bs.n_seq;
+                const int role = t / per_role, rem = t - role * per_role;
+                const int seq = rem / a.app_per_seq, x = rem - seq * a.app_per_seq;
+                int* s_part = reinterpret_cast<int*>(dyn);
+                switch (a.app_dI) {
+                    case 32: append_task<32, kSelThreads>(a.app, x, seq, role, s_part); break;
+                    case 64: append_task<64, kSelThreads>(a.app, x, seq, role, s_part); break;
+                    default: append_task<128, kSelThreads>(a.app, x, seq, role, s_part); break;
+                }
+            }
+            return;
+        }
+    }
     SelShared& sh = *reinterpret_cast<SelShared*>(dyn);
     const int r = blockIdx.y;
     const uint32_t C = cluster_size(), c = cluster_rank();
@@ -824,32 +850,45 @@ IndexPlan plan_index(int n_q, int max_len, const lsa_budget_t& b, bool dense) {
     return p;
 }
 
+// extra_rows: grid rows past n_q (the fused append's CTAs, block selection only)
 template <typename Kern>
-static cudaError_t launch_cluster(Kern kern, const IndexArgs& a, int cluster, size_t smem, cudaStream_t stream) {
+static cudaError_t launch_cluster(Kern kern, const IndexArgs& a, int cluster, size_t smem, cudaStream_t stream,
+                                  int extra_rows = 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (cluster > 8) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(kern, dim3((unsigned)cluster, (unsigned)a.n_q, 1), dim3(kSelThreads), smem, stream, cluster, a);
+    return launch_pdl(kern, dim3((unsigned)cluster, (unsigned)(a.n_q + extra_rows), 1), dim3(kSelThreads), smem,
+                      stream, cluster, a);
 }
 
 template <int D_I>
-static cudaError_t launch_blocks_fused(const IndexArgs& a, int cluster, size_t smem, cudaStream_t stream) {
-    if (a.H_I <= 8) return launch_cluster(select_kernel<uint64_t, false, D_I, 1>, a, cluster, smem, stream);
-    return launch_cluster(select_kernel<uint64_t, false, D_I, 2>, a, cluster, smem, stream);  // H_I <= 16
+static cudaError_t launch_blocks_fused(const IndexArgs& a, int cluster, size_t smem, cudaStream_t stream, int extra) {
+    if (a.H_I <= 8) return launch_cluster(select_kernel<uint64_t, false, D_I, 1>, a, cluster, smem, stream, extra);
+    return launch_cluster(select_kernel<uint64_t, false, D_I, 2>, a, cluster, smem, stream, extra);  // H_I <= 16
+}
+
+int index_select_append_rows(const IndexArgs& a, int cluster) {
+    return a.app_tasks > 0 ? (a.app_tasks + cluster - 1) / cluster : 0;
 }
 
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
                                 cudaStream_t stream) {
     if (cluster < 1 || cluster > kMaxCluster) return cudaErrorInvalidValue;
-    if (!blocks) return launch_cluster(select_kernel<uint32_t, true>, a, cluster, smem, stream);
-    if (!coarse_in_select(a)) return launch_cluster(select_kernel<uint64_t, false>, a, cluster, smem, stream);
+    if (!blocks) {
+        if (a.app_tasks > 0) return cudaErrorInvalidValue;  // the append rides on the block selection only
+        return launch_cluster(select_kernel<uint32_t, true>, a, cluster, smem, stream);
+    }
+    if (a.app_tasks > 0 && (a.app_dI != 32 && a.app_dI != 64 && a.app_dI != 128)) return cudaErrorInvalidValue;
+    const int extra = index_select_append_rows(a, cluster);
+    if (!coarse_in_select(a))
+        return launch_cluster(select_kernel<uint64_t, false>, a, cluster, smem, stream, extra);
     switch (d_I) {
-        case 32: return launch_blocks_fused<32>(a, cluster, smem, stream);
-        case 64: return launch_blocks_fused<64>(a, cluster, smem, stream);
-        case 128: return launch_blocks_fused<128>(a, cluster, smem, stream);
+        case 32: return launch_blocks_fused<32>(a, cluster, smem, stream, extra);
+        case 64: return launch_blocks_fused<64>(a, cluster, smem, stream, extra);
+        case 128: return launch_blocks_fused<128>(a, cluster, smem, stream, extra);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -47,6 +47,17 @@ struct AppendArgs {
     int32_t sums;                  // 1: recompute the block sums (HI on)
 };
 cudaError_t launch_append(const AppendArgs& a, int d_I, cudaStream_t stream);
+constexpr int kAppendRowsPerCta = 64;  // HI off: new tokens per append CTA
+// CTAs per sequence and role of the decode append: with HI on, the blocks that
+// the n_new newest tokens can fall in; otherwise runs of kAppendRowsPerCta.
+__host__ __device__ __forceinline__ int append_ctas_per_seq(int n_new, int hi_block, int max_len) {
+    if (hi_block > 0) {
+        const int64_t full = ((int64_t)max_len + hi_block - 1) / hi_block;
+        const int64_t cover = ((int64_t)n_new + hi_block - 1) / hi_block + 1;
+        return (int)(cover < full ? cover : full);
+    }
+    return (n_new + kAppendRowsPerCta - 1) / kAppendRowsPerCta;
+}
 
 // ---- indexer: scoring kernels + selection kernels -------------------------
 // Keys (score + 1) are histogrammed on a monotone logarithmic scale: the bit
@@ -93,6 +104,11 @@ struct IndexArgs {
     // selection: keys of one CTA's slice staged in shared memory (0 = read
     // from global memory) and kept-block slots per slice
     int32_t coarse_stage, fine_stage, kept_slots;
+    // a decode append run by extra CTAs of the block selection's grid (rows
+    // n_q onwards): app_tasks tasks of app_per_seq CTAs per sequence and role
+    // (0 = no append in this call)
+    AppendArgs app;
+    int32_t app_tasks, app_per_seq, app_dI;
 };
 
 struct IndexPlan {
@@ -138,6 +154,8 @@ cudaError_t launch_merge_pairs(const uint64_t* pairs, const int32_t* counts, int
                                uint64_t* out_values, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexArgs& a, bool blocks, int d_I, int cluster, size_t smem,
                                 cudaStream_t stream);
+// Grid rows the block selection adds for a fused append (a.app_tasks tasks).
+int index_select_append_rows(const IndexArgs& a, int cluster);
 
 // Indexer scores of given token positions or HI blocks (lsa_score_tokens,
 // lsa_score_blocks): q_idx, k_idx, w, w_max, H_I, n_q, block_sums and

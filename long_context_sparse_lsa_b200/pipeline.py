@@ -34,14 +34,17 @@ def _pack(tensors, device):
 
 class LsaStep:
     def __init__(self, wl: Workload, t: Tensors, device="cuda", kv_fp8: bool = False, grouped: bool = False,
-                 si_attend: bool | None = None):
+                 si_attend: bool | None = None, fuse_append: bool = True):
         """kv_fp8: the K/V caches are FP8 E4M3 codes (drawn here, per layer,
         with scales k_scale / v_scale) and the attention is lsa_attend_fp8;
         the bf16 caches of `t` are then unused and may be empty.
         grouped: the decode rows of each sequence (wl.drafts of them) attend
         through lsa_attend_grouped (the rows of a group in one CTA).
         si_attend: attend through lsa_attend_si (sink and window runs as dense
-        tiles); by default for a prefill chunk with bf16 caches."""
+        tiles); by default for a prefill chunk with bf16 caches.
+        fuse_append: a decode step's append and index calls go through
+        lsa_append_index (the append inside the block selection when the new
+        tokens lie in every window); otherwise lsa_append, then lsa_index."""
         self.wl = wl
         self.t = t
         self.device = device
@@ -53,6 +56,7 @@ class LsaStep:
         if si_attend is None:
             si_attend = bool(wl.prefill_new) and not kv_fp8 and not grouped and wl.n_seq == 1
         self.si_attend = si_attend
+        self.fuse_append = fuse_append
         if kv_fp8:
             shape = (wl.total_tokens, wl.H_kv, wl.d)
             self.k8 = [gen.normal_e4m3(shape, wl.seed, gen.STREAM_K8 + g, device) for g in range(self.G)]
@@ -134,6 +138,13 @@ class LsaStep:
             lsa.lsa_append(self.k_idx_new, self.t.k_idx, self.k_new, self.v_new, kc, vc,
                            self.wl.hi_block, self.block_sums, self.batch, self.n_new, self.status, stream)
 
+    def append_index(self, stream=None):
+        """The append and the index call in one: lsa_append_index."""
+        kc, vc = self.kv_caches()
+        lsa.lsa_append_index(self.k_idx_new, self.k_new, self.v_new, kc, vc, self.n_new, self.t.q_idx, self.t.k_idx,
+                             self.t.w, self.wl.w_max, self.batch, self.budget, self.sets, self.block_sums,
+                             self.ws_index, self.status, stream)
+
     def index(self, stream=None):
         lsa.lsa_index(self.t.q_idx, self.t.k_idx, self.t.w, self.wl.w_max, self.batch, self.budget, self.sets,
                       self.block_sums, self.ws_index, self.status, stream)
@@ -154,8 +165,11 @@ class LsaStep:
 
     def step(self, stream=None):
         """One decode step: append, index, attend."""
-        self.append(stream)
-        self.index(stream)
+        if self.n_new and self.fuse_append:
+            self.append_index(stream)
+        else:
+            self.append(stream)
+            self.index(stream)
         self.attend(stream)
 
     def overlap_ok(self) -> bool:
@@ -207,7 +221,7 @@ class LsaStep:
             self.graphs[name] = g
         g = torch.cuda.CUDAGraph()
         fork = torch.cuda.Stream(self.device)
-        fork_ok = fork_append and self.overlap_ok()
+        fork_ok = fork_append and self.overlap_ok() and not self.fuse_append
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             cur = torch.cuda.current_stream(self.device)
             if fork_ok:
@@ -230,14 +244,18 @@ class LsaStep:
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
             cur = torch.cuda.current_stream(self.device)
             overlap = fork_ok
+            fused = bool(self.n_new) and self.fuse_append
             if overlap:
                 fork.wait_stream(cur)
                 with torch.cuda.stream(fork):
                     self.append()
-            else:
+            elif not fused:
                 self.append()
             ix0.record(cur)
-            self.index()
+            if fused:
+                self.append_index()  # the index call's time then includes the append
+            else:
+                self.index()
             ix1.record(cur)
             if overlap:
                 cur.wait_stream(fork)
@@ -271,7 +289,10 @@ class LsaStep:
         """Kernel launches of one step: the append (decode) and the launches
         the index and attention calls report for this shape."""
         wl = self.wl
-        n_idx = lsa.lsa_index_launches(self.batch, wl.H_I, wl.d_I, self.budget)
+        if self.n_new and self.fuse_append:
+            n_idx = lsa.lsa_append_index_launches(self.batch, wl.H_I, wl.d_I, self.budget, self.n_new)
+        else:
+            n_idx = (1 if self.n_new else 0) + lsa.lsa_index_launches(self.batch, wl.H_I, wl.d_I, self.budget)
         if self.grouped:
             n_att = lsa.lsa_attend_grouped_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G,
                                                     wl.drafts)
@@ -279,4 +300,4 @@ class LsaStep:
             n_att = lsa.lsa_attend_si_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget, self.G)
         else:
             n_att = lsa.lsa_attend_launches(self.batch, wl.H_q, wl.H_kv, wl.d, self.budget.length, self.G)
-        return (1 if self.n_new else 0) + n_idx + n_att
+        return n_idx + n_att

@@ -120,6 +120,47 @@ def test_append_rejects_before_launch(kw, want):
     assert _append(lib, **kw) == want
 
 
+def _append_index(lib, **kw):
+    arr = (ctypes.c_void_p * 2)(P, P)
+    args = dict(kin=P, kn=arr, vn=arr, kcache=arr, vcache=arr, kvb=1024, layers=2, n_new=1, q=P, kc=P, w=P,
+                w_max=8, H_I=16, d_I=128, batch=_batch(), budget=_budget(window=100, hb=64, ht=8), bs=P, rows=10,
+                sets=P, ws=None, ws_bytes=0)
+    args.update(kw)
+    return lib.lsa_append_index(args["kin"], args["kn"], args["vn"], args["kcache"], args["vcache"], args["kvb"],
+                                args["layers"], args["n_new"], args["q"], args["kc"], args["w"], args["w_max"],
+                                args["H_I"], args["d_I"], ctypes.byref(args["batch"]), args["budget"], args["bs"],
+                                args["rows"], args["sets"], args["ws"], args["ws_bytes"], None, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(n_new=0), 1), (dict(kin=None), 1), (dict(kvb=1000), 1), (dict(layers=9), 2),
+    (dict(q=None), 1), (dict(sets=None), 1), (dict(d_I=96), 2), (dict(w_max=1 << 20), 2),
+    (dict(bs=None), 1),                                   # HI on without block sums
+    (dict(budget=_budget(sink=-1)), 1),
+    (dict(ws=None, ws_bytes=0), 4),                       # fused path: the index workspace is checked first
+    (dict(budget=_budget(window=10, hb=64, ht=8)), 4),    # sequential path: checked before the append's launch
+    (dict(budget=_budget(hb=0, ht=0), bs=None), 4),       # HI off
+])
+def test_append_index_rejects_before_launch(kw, want):
+    lib = lsa.load_library()
+    assert _append_index(lib, **kw) == want
+
+
+def test_append_index_launch_counts():
+    lib = lsa.load_library()
+    b = _batch(n_seq=16, n_q=16, max_len=131072, total=16 * 131072)
+    fused = _budget(sink=64, window=1024, topk=2048, hb=64, ht=256)
+    n_idx = lib.lsa_index_launches(ctypes.byref(b), 16, 128, fused)
+    assert n_idx >= 3
+    assert lib.lsa_append_index_launches(ctypes.byref(b), 16, 128, fused, 1) == n_idx
+    assert lib.lsa_append_index_launches(ctypes.byref(b), 16, 128, fused, 961) == n_idx  # window == 64 + 961 - 1
+    assert lib.lsa_append_index_launches(ctypes.byref(b), 16, 128, fused, 962) == n_idx + 1
+    flat = _budget(sink=64, window=1024, topk=2048)
+    assert lib.lsa_append_index_launches(ctypes.byref(b), 16, 128, flat, 1) == \
+        lib.lsa_index_launches(ctypes.byref(b), 16, 128, flat) + 1
+    assert lib.lsa_append_index_launches(ctypes.byref(b), 16, 128, fused, 0) == 0
+
+
 def test_attend_fp8_rejects_before_launch():
     lib = lsa.load_library()
     b = _batch(n_q=16, max_len=131072, total=16 * 131072)

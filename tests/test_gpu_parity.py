@@ -218,6 +218,96 @@ def test_append_writes_rows_and_refreshes_block_sums(n_new, hi_block):
             np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
 
 
+APPEND_INDEX_CASES = {
+    # HI on, the new tokens inside every window: the append runs in the block selection (8-CTA clusters)
+    "fused_b64": dict(lens=(3000, 71, 130, 5000, 2600, 4100, 900, 3500, 1200), hi_block=64, hi_topblocks=8,
+                      window=100, sink=16, topk=300, n_new=1),
+    "fused_b64_nnew4": dict(lens=(3000, 5000, 2600, 4100, 900, 3500, 1200, 6000), hi_block=64, hi_topblocks=6,
+                            window=67, sink=8, topk=200, n_new=4),
+    # few rows: separate coarse scores, 16-CTA clusters, two blocks of new tokens
+    "fused_one_row_b128": dict(lens=(40000,), hi_block=128, hi_topblocks=40, window=260, sink=64, topk=1024,
+                               n_new=130),
+    # draft rows (q_len < seq_lens), n_new = drafts
+    "fused_drafts": dict(lens=(4000, 6000), hi_block=64, hi_topblocks=10, window=80, sink=16, topk=300, n_new=4,
+                         drafts=4),
+    # not fusable: a new token's block meets the middle (window < hi_block + n_new - 1), HI off
+    "sequential_window": dict(lens=(3000, 5000), hi_block=64, hi_topblocks=8, window=40, sink=16, topk=300,
+                              n_new=1),
+    "sequential_flat": dict(lens=(3000, 5000), hi_block=0, hi_topblocks=0, window=64, sink=16, topk=300, n_new=3),
+}
+
+
+@pytest.mark.parametrize("case", list(APPEND_INDEX_CASES))
+def test_append_index_equals_append_then_index(case):
+    """lsa_append_index: the caches hold the new rows, the block sums are the
+    oracle's sums of the updated cache and the index sets are the oracle's
+    sets over it, bit for bit, whether the append runs inside the block
+    selection or as its own launch."""
+    kw = dict(APPEND_INDEX_CASES[case])
+    n_new = kw.pop("n_new")
+    wl = wls.small(BASE, name=case, G=2, seed=41, **kw)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    fused = wl.hi_block > 0 and wl.window >= wl.hi_block + n_new - 1
+    n_idx = lsa.lsa_index_launches(st.batch, wl.H_I, wl.d_I, st.budget)
+    assert lsa.lsa_append_index_launches(st.batch, wl.H_I, wl.d_I, st.budget, n_new) == n_idx + (0 if fused else 1)
+    gen = torch.Generator().manual_seed(2000 + n_new)
+    n_seq = wl.n_seq
+    k_idx_new = torch.randint(-16, 16, (n_seq, n_new, wl.d_I), dtype=torch.int8, generator=gen)
+    k_new = [torch.randn((n_seq, n_new, wl.H_kv, wl.d), generator=gen).to(torch.bfloat16) for _ in range(wl.G)]
+    v_new = [torch.randn((n_seq, n_new, wl.H_kv, wl.d), generator=gen).to(torch.bfloat16) for _ in range(wl.G)]
+    want_k = parity.host(t.k_idx).copy()
+    want_K = [parity.u16(x).copy() for x in t.k]
+    want_V = [parity.u16(x).copy() for x in t.v]
+    offs = parity.host(t.kv_offset)
+    for b, L in enumerate(wl.lens):
+        lo = offs[b] + L - n_new
+        want_k[lo:lo + n_new] = k_idx_new[b].numpy()
+        for g in range(wl.G):
+            want_K[g][lo:lo + n_new] = k_new[g][b].view(torch.int16).numpy().view(np.uint16)
+            want_V[g][lo:lo + n_new] = v_new[g][b].view(torch.int16).numpy().view(np.uint16)
+    st.sets.fill_(-7)
+    lsa.lsa_append_index(k_idx_new.to(DEV), [x.to(DEV) for x in k_new], [x.to(DEV) for x in v_new], t.k, t.v, n_new,
+                         t.q_idx, t.k_idx, t.w, wl.w_max, st.batch, st.budget, st.sets, st.block_sums, st.ws_index,
+                         st.status)
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    np.testing.assert_array_equal(parity.host(t.k_idx), want_k)
+    for g in range(wl.G):
+        np.testing.assert_array_equal(parity.u16(t.k[g]), want_K[g])
+        np.testing.assert_array_equal(parity.u16(t.v[g]), want_V[g])
+    if wl.hi_block:
+        orc = oracle.get()
+        got = parity.decode_block_sums(st.block_sums, wl.d_I)
+        boffs = parity.host(t.blk_offset)
+        for b, L in enumerate(wl.lens):
+            want = orc.block_sums(want_k[offs[b]:offs[b] + L], wl.hi_block)
+            np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
+    parity.check_sets(parity.host(st.sets), parity.oracle_sets(wl, t), wl.name)
+
+
+def test_append_index_flags_a_bad_sequence():
+    """A sequence whose new tokens outnumber its tokens is skipped and flagged
+    by the fused append (LSA_DEV_BAD_LENGTH); the other sequences' rows are
+    still written."""
+    wl = wls.small(BASE, name="ai_bad", lens=(3000, 5000), hi_block=64, hi_topblocks=8, window=100, sink=16,
+                   topk=300, G=1, seed=43)
+    t = wls.make(wl, DEV)
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    n_new = 1
+    k_idx_new = torch.full((wl.n_seq, n_new, wl.d_I), 5, dtype=torch.int8, device=DEV)
+    kn = [torch.zeros((wl.n_seq, n_new, wl.H_kv, wl.d), dtype=torch.bfloat16, device=DEV)]
+    t.seq_lens[0] = 0  # sequence 0 now holds no token
+    lsa.lsa_append_index(k_idx_new, kn, kn, t.k, t.v, n_new, t.q_idx, t.k_idx, t.w, wl.w_max, st.batch, st.budget,
+                         st.sets, st.block_sums, st.ws_index, st.status)
+    torch.cuda.synchronize()
+    assert st.status_bits() & lsa.LSA_DEV_BAD_LENGTH
+    offs = parity.host(t.kv_offset)
+    assert np.all(parity.host(t.k_idx)[offs[1] + 5000 - 1] == 5)
+
+
 def test_extreme_block_sums_hi_block_256():
     """|S| reaches 128 * 256 = 32768: the byte planes stay exact."""
     wl = wls.small(BASE, name="bs_extreme", lens=(512,), hi_block=256, hi_topblocks=1, seed=3)

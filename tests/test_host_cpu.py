@@ -82,12 +82,14 @@ def test_new_rows_are_the_newest_cached_tokens():
     assert torch.equal(st8.v_new[1][1], st8.v8[1][o + L - 2:o + L])
 
 
-@pytest.mark.parametrize("wl,n", [(wls.BATCH128K, 6), (wls.CTX1M, 7)])
-def test_kernels_per_step(wl, n):
-    """16 rows: append, block selection with the coarse scores inside, fine scores, token
-    selection, attention, merge; one 1M row adds the separate coarse-score kernel."""
+@pytest.mark.parametrize("wl,n,fuse", [(wls.BATCH128K, 5, True), (wls.CTX1M, 6, True), (wls.BATCH128K, 6, False),
+                                       (wls.CTX1M, 7, False)])
+def test_kernels_per_step(wl, n, fuse):
+    """16 rows: block selection with the coarse scores and the append inside, fine scores,
+    token selection, attention, merge; one 1M row adds the separate coarse-score kernel;
+    without the fused call the append is a launch of its own."""
     small = wls.small(wl, lens=tuple(min(L, 4096) for L in wl.lens))
-    st = _step(small)
+    st = _step(small, fuse_append=fuse)
     # the plan depends on the shape's host fields only; use the real lengths for it
     st.batch.max_len = max(wl.lens)
     assert st.kernels_per_step() == n
