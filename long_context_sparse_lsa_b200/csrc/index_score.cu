@@ -238,7 +238,8 @@ constexpr size_t kFtSmem = 1024 + (size_t)kFtStages * kFtStageBytes + sizeof(FtS
 
 template <int NT>
 __global__ void __launch_bounds__(kFtThreads, kFtCtasPerSm) fine_score_tma_kernel(const __grid_constant__ FineTmaArgs p) {
-    pdl_enter();
+    // Before the wait for the block selection: only the caller's inputs (row
+    // metadata, queries, weights), which no kernel of this library writes.
     const IndexArgs& a = p.a;
     extern __shared__ __align__(16) uint8_t ft_raw[];
     const uint32_t raw = smem_u32(ft_raw);
@@ -263,6 +264,17 @@ __global__ void __launch_bounds__(kFtThreads, kFtCtasPerSm) fine_score_tma_kerne
 
     if (warp == kFtConsumers) {
         // ------------------------------ producer ------------------------------
+        // the CTA's first and last rows (a range spans at most two rows when
+        // there are fewer rows than CTAs) are checked before the wait
+        const int r_first = i_lo < i_hi ? (int)(i_lo / per_row) : 0;
+        const int r_last = i_lo < i_hi ? (int)((i_hi - 1) / per_row) : 0;
+        int64_t c_off = 0;
+        int c_L = 0;
+        const bool c_ok = lane < 2 && row_ok(a, lane == 0 ? r_first : r_last, c_off, c_L);
+        const bool ok_first = __shfl_sync(0xffffffffu, c_ok, 0), ok_last = __shfl_sync(0xffffffffu, c_ok, 1);
+        const int64_t off_first = __shfl_sync(0xffffffffu, c_off, 0), off_last = __shfl_sync(0xffffffffu, c_off, 1);
+        const int L_first = __shfl_sync(0xffffffffu, c_L, 0), L_last = __shfl_sync(0xffffffffu, c_L, 1);
+        pdl_enter();
         int k = 0;  // items issued
         auto next_stage = [&](int kk) -> bool {  // lane 0: wait until stage kk % S is free
             const int st = kk % kFtStages;
@@ -286,9 +298,11 @@ __global__ void __launch_bounds__(kFtThreads, kFtCtasPerSm) fine_score_tma_kerne
                 // the kept count and id are fetched together with the row check
                 const int nk = a.n_kept[r];
                 const int kid = a.kept[(int64_t)r * a.hi_topblocks + q];
-                int64_t off;
-                int L;
-                if (row_ok(a, r, off, L) && q < min(max(nk, 0), a.hi_topblocks)) {
+                int64_t off = r == r_first ? off_first : off_last;
+                int L = r == r_first ? L_first : L_last;
+                bool ok = r == r_first ? ok_first : ok_last;
+                if (r != r_first && r != r_last) ok = row_ok(a, r, off, L);
+                if (ok && q < min(max(nk, 0), a.hi_topblocks)) {
                     it.row = r;
                     it.slot0 = q * B + part * SB;
                     it.tok0 = kid * B + part * SB;
@@ -340,6 +354,7 @@ __global__ void __launch_bounds__(kFtThreads, kFtCtasPerSm) fine_score_tma_kerne
         int qrow = i_lo < i_hi ? (int)(i_lo / per_row) : -1;
         QueryFrag<128, NT> qf;
         if (qrow >= 0) load_query<128, NT>(qf, a, qrow);
+        pdl_enter();
         uint32_t* keys = qrow >= 0 ? a.fine_keys + (int64_t)qrow * a.fine_cap : nullptr;
         for (int k = warp;; k += kFtConsumers) {
             const int st = k % kFtStages;

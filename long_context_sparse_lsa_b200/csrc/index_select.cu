@@ -672,12 +672,27 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     const K* row_keys = kTokens ? reinterpret_cast<const K*>(a.fine_keys + (int64_t)r * a.fine_cap)
                                 : reinterpret_cast<const K*>(a.coarse_keys + (int64_t)r * a.coarse_cap);
     Keys<K> keys{row_keys + k_lo, 0u};
+    // kept blocks that this slice's slots fall in (used by the compaction).
+    // With at most one per thread, every id the slice's capacity may hold is
+    // loaded into a register here, beside the kept count and the keys, and
+    // stored after the staging pass: the three loads share one round trip.
     int kb_lo = 0;
-    if (kTokens && B > 0 && m > 0) {  // kept blocks that this slice's slots fall in
+    int32_t kid = 0;
+    bool has_kid = false;
+    if (kTokens && B > 0) {
         kb_lo = k_lo / B;
-        const int kb_hi = (k_lo + m - 1) / B;
         const int32_t* kept = a.kept + (int64_t)r * a.hi_topblocks;
-        for (int i = threadIdx.x; i <= kb_hi - kb_lo && i < a.kept_slots; i += kSelThreads) s_kept[i] = kept[kb_lo + i];
+        if (a.kept_slots <= kSelThreads) {
+            const int i = threadIdx.x;
+            if (m_load > 0 && i <= (k_lo + m_load - 1) / B - kb_lo && i < a.kept_slots && kb_lo + i < a.hi_topblocks) {
+                kid = kept[kb_lo + i];
+                has_kid = true;
+            }
+        } else if (m > 0) {
+            const int kb_hi = (k_lo + m - 1) / B;
+            for (int i = threadIdx.x; i <= kb_hi - kb_lo && i < a.kept_slots; i += kSelThreads)
+                s_kept[i] = kept[kb_lo + i];
+        }
     }
     zero_hists(sh);
     if (threadIdx.x == 0) {
@@ -693,6 +708,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     } else {
         stage_pass<K>(sh, keys, m, m_load, stage);
     }
+    if (has_kid) s_kept[threadIdx.x] = kid;
     __syncthreads();
     if (stage != nullptr) keys.s = smem_u32(stage);
     // the row check (as in the scoring kernels): uniform over the cluster, and
