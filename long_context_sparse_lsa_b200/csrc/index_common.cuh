@@ -156,7 +156,7 @@ __device__ __forceinline__ bool partial_block_fix(int L, int slen, int B, int ws
 // s_sum: D_I ints of shared scratch. Returns the score in every thread; holds
 // CTA barriers, so every thread must call it.
 template <int D_I, int THREADS>
-__device__ long long partial_block_score(const IndexArgs& a, int r, const int8_t* rows, int t0, int n,
+__device__ __noinline__ long long partial_block_score(const IndexArgs& a, int r, const int8_t* rows, int t0, int n,
                                          int32_t* s_sum, long long* s_out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int kWarps = THREADS / 32;

@@ -61,6 +61,9 @@ struct SelShared {
     uint32_t bin, above, in_bin;
     uint32_t count;        // length of the row's candidate list (remote adds)
     uint32_t local_count;  // candidates of this slice
+    unsigned long long few[kWarp];  // the last <= 32 candidates of the threshold (few_rank)
+    unsigned long long few_T;
+    uint32_t few_quota;
 };
 
 // Candidate list entries: the key in the low 60 bits (scores stay below 2^40
@@ -186,7 +189,7 @@ __device__ uint32_t find_bin(SelShared& sh, uint32_t krem, uint32_t& bin, uint32
 // histogram; the caller brackets it with cluster barriers.
 __device__ void push_hist(SelShared& sh, uint32_t C) {
     const uint32_t base = smem_u32(sh.hist);
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < kBinsPerThread; ++j) {
         const int b = threadIdx.x + j * kSelThreads;
         const uint32_t v = sh.local_hist[b];
@@ -251,6 +254,69 @@ __device__ void digit_hist(uint32_t* hist, Get get, int m, int shift, int width,
         for (int u = 0; u < kUnroll; ++u)
             if (i0 + u * kSelThreads < m && (K)(kv[u] >> (shift + width)) == prefix)
                 atomicAdd(&hist[(uint32_t)(kv[u] >> shift) & mask], 1u);
+    }
+}
+
+// The krem-th largest of the n <= 32 keys of list[0, mm) whose bits above
+// `shift` equal `prefix`, and how many keys equal to it that rank takes
+// (quota): one warp gathers them by ballot and ranks them by shuffles, in
+// place of further radix levels (each a 4096-bin histogram and four CTA
+// barriers). Every thread of the CTA calls it; the result is in every thread.
+template <typename K, typename Get>
+__device__ void few_rank(SelShared& sh, Get get, int mm, int shift, K prefix, uint32_t n, uint32_t krem, K& T,
+                         uint32_t& quota) {
+    if (warp_id() == 0) {
+        const int lane = lane_id();
+        uint32_t got = 0;
+        for (int i0 = 0; i0 < mm; i0 += kWarp) {  // warp-uniform trip count
+            const int i = i0 + lane;
+            const K key = i < mm ? get(i) : K(0);
+            const bool match = i < mm && (K)(key >> shift) == prefix;
+            const uint32_t bal = __ballot_sync(0xffffffffu, match);
+            const uint32_t pos = got + (uint32_t)__popc(bal & ((1u << lane) - 1u));
+            if (match && pos < (uint32_t)kWarp) sh.few[pos] = (unsigned long long)key;
+            got += (uint32_t)__popc(bal);
+        }
+        __syncwarp();
+        const uint32_t cnt = min(got, min(n, (uint32_t)kWarp));
+        const K x = lane < (int)cnt ? (K)sh.few[lane] : K(0);
+        uint32_t g = 0, e = 0;
+        for (uint32_t j = 0; j < cnt; ++j) {
+            const K y = (K)__shfl_sync(0xffffffffu, (unsigned long long)x, (int)j);
+            g += y > x ? 1u : 0u;
+            e += y == x ? 1u : 0u;
+        }
+        // the lanes holding the rank's key (equal keys write equal values)
+        if (lane < (int)cnt && g < krem && krem <= g + e) {
+            sh.few_T = (unsigned long long)x;
+            sh.few_quota = krem - g;
+        }
+    }
+    __syncthreads();
+    T = (K)sh.few_T;
+    quota = sh.few_quota;
+}
+
+// A threshold bin too full for the candidate list: the remaining digits are
+// resolved by cluster histograms over the slices (one per 12-bit digit). Out
+// of line: a rare path, kept away from the common one's instructions.
+template <typename K>
+__device__ __noinline__ void refine_over_slices(SelShared& sh, const Keys<K>& keys, int m, uint32_t C, int shift,
+                                                K& prefix, uint32_t& krem) {
+    while (shift > 0) {
+        const int width = shift < kDigitBits ? shift : kDigitBits;
+        shift -= width;
+        zero_hists(sh);
+        __syncthreads();
+        digit_hist<K>(sh.local_hist, [&](int i) { return keys[i]; }, m, shift, width, prefix);
+        __syncthreads();
+        cluster_sync();  // every CTA's row histogram is clear and its slice counted
+        push_hist(sh, C);
+        cluster_sync();
+        uint32_t d, ab, ib;
+        find_bin(sh, krem, d, ab, ib);
+        prefix = (K)((prefix << width) | (K)d);
+        krem -= ab;
     }
 }
 
@@ -322,7 +388,17 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uin
         }
         cluster_sync();  // after this no CTA touches another CTA's shared memory
         const int mm = (int)min(sh.count, (uint32_t)kCandCap);
+        uint32_t n_match = in_bin;  // candidates whose bits above shift equal prefix
         while (shift > 0) {  // identical in every CTA
+            if (n_match <= (uint32_t)kWarp) {
+                K T;
+                uint32_t q;
+                few_rank<K>(sh, [&](int i) { return (K)(cand[i] & kKeyMask); }, mm, shift, prefix, n_match, krem, T,
+                            q);
+                prefix = T;
+                krem = q;
+                break;
+            }
             const int width = shift < kDigitBits ? shift : kDigitBits;
             shift -= width;
             reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
@@ -334,6 +410,7 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uin
             find_bin(sh, krem, d, ab, ib);
             prefix = (K)((prefix << width) | (K)d);
             krem -= ab;
+            n_match = ib;
         }
         // kept counts per originating slice: keys above the bin plus its
         // candidates > T, and its candidates == T
@@ -367,22 +444,7 @@ __device__ void resolve_threshold(SelShared& sh, const Keys<K>& keys, int m, uin
         }
         carried = true;
     } else {
-        // refine over the slices: one cluster histogram per digit
-        while (shift > 0) {
-            const int width = shift < kDigitBits ? shift : kDigitBits;
-            shift -= width;
-            zero_hists(sh);
-            __syncthreads();
-            digit_hist<K>(sh.local_hist, [&](int i) { return keys[i]; }, m, shift, width, prefix);
-            __syncthreads();
-            cluster_sync();  // every CTA's row histogram is clear and its slice counted
-            push_hist(sh, C);
-            cluster_sync();
-            uint32_t d, ab, ib;
-            find_bin(sh, krem, d, ab, ib);
-            prefix = (K)((prefix << width) | (K)d);
-            krem -= ab;
-        }
+        refine_over_slices<K>(sh, keys, m, C, shift, prefix, krem);
     }
     thresh = prefix;
     quota = krem;
@@ -592,7 +654,29 @@ __device__ void coarse_pass(SelShared& sh, const IndexArgs& a, int r, int64_t bo
     }
 }
 
-// Selection of one row by one cluster. kTokens: fine top-k and the SI
+// The fused decode append's CTAs (grid rows n_q onwards of the block
+// selection): one append task per CTA. Out of line, away from the
+// selection's instructions.
+template <int D_I>
+__device__ __noinline__ void fused_append(const IndexArgs& a, int* s_part) {
+    pdl_enter();  // the caches may still be read by the preceding kernels
+    const int t = (int)((blockIdx.y - (unsigned)a.n_q) * gridDim.x + blockIdx.x);
+    if (t >= a.app_tasks) return;
+    const int per_role = a.app_per_seq * a.app.bs.n_seq;
+    const int role = t / per_role, rem = t - role * per_role;
+    const int seq = rem / a.app_per_seq, x = rem - seq * a.app_per_seq;
+    if constexpr (D_I > 0) {  // the indexer key width is the kernel's (one copy of the append code)
+        append_task<D_I, kSelThreads>(a.app, x, seq, role, s_part);
+    } else {
+        switch (a.app_dI) {
+            case 32: append_task<32, kSelThreads>(a.app, x, seq, role, s_part); break;
+            case 64: append_task<64, kSelThreads>(a.app, x, seq, role, s_part); break;
+            default: append_task<128, kSelThreads>(a.app, x, seq, role, s_part); break;
+        }
+    }
+}
+
+// Selection of one row by one cluster. kTokens: fine top-k and the SI// Selection of one row by one cluster. kTokens: fine top-k and the SI
 // assembly of the index set; otherwise the HI block top-k.
 // D_I > 0 (HI blocks only): the coarse scores are computed in place
 // (coarse_pass) instead of read from the coarse scoring kernel's workspace.
@@ -608,19 +692,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_con
     extern __shared__ __align__(16) uint8_t dyn[];
     if constexpr (!kTokens) {
         if (blockIdx.y >= (unsigned)a.n_q) {  // uniform over the cluster: no cluster barrier is used
-            pdl_enter();                      // the caches may still be read by the preceding kernels
-            const int t = (int)((blockIdx.y - (unsigned)a.n_q) * gridDim.x + blockIdx.x);
-            if (t < a.app_tasks) {
-                const int per_role = a.app_per_seq * a.app.bs.n_seq;
-                const int role = t / per_role, rem = t - role * per_role;
-                const int seq = rem / a.app_per_seq, x = rem - seq * a.app_per_seq;
-                int* s_part = reinterpret_cast<int*>(dyn);
-                switch (a.app_dI) {
-                    case 32: append_task<32, kSelThreads>(a.app, x, seq, role, s_part); break;
-                    case 64: append_task<64, kSelThreads>(a.app, x, seq, role, s_part); break;
-                    default: append_task<128, kSelThreads>(a.app, x, seq, role, s_part); break;
-                }
-            }
+            fused_append<D_I>(a, reinterpret_cast<int*>(dyn));
             return;
         }
     }
