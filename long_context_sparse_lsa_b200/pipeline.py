@@ -115,15 +115,21 @@ class LsaStep:
         copy per step. The tensors keep their values and become views of the
         buffers. Call before capture(): the graphs keep these addresses."""
         t, G = self.t, self.G
-        ins = [t.q_idx, t.w, *t.q]
+        # the index call's inputs first, the attention's queries last: the
+        # e2e graph copies the two parts on two streams (capture_e2e)
+        ins = [t.q_idx, t.w]
         if self.n_new:
             ins += [self.k_idx_new, *self.k_new, *self.v_new]
+        n_head = len(ins)
+        ins += list(t.q)
         self.in_buf, v = _pack(ins, self.device)
-        t.q_idx, t.w, t.q = v[0], v[1], list(v[2:2 + G])
+        t.q_idx, t.w = v[0], v[1]
         if self.n_new:
-            self.k_idx_new = v[2 + G]
-            self.k_new = list(v[3 + G:3 + 2 * G])
-            self.v_new = list(v[3 + 2 * G:3 + 3 * G])
+            self.k_idx_new = v[2]
+            self.k_new = list(v[3:3 + G])
+            self.v_new = list(v[3 + G:3 + 2 * G])
+        t.q = list(v[n_head:])
+        self.in_split = t.q[0].data_ptr() - self.in_buf.data_ptr()  # first byte of the queries
         self.out_buf, self.out = _pack(self.out, self.device)
 
     def kv_caches(self):
@@ -273,6 +279,35 @@ class LsaStep:
             self.graphs["cold"] = g
         torch.cuda.synchronize(self.device)
         return self.graphs
+
+    def capture_e2e(self, h_in: torch.Tensor, h_out: torch.Tensor):
+        """Capture graph "e2e": one step with its host copies, for a serving
+        loop whose inputs and outputs live in pinned host memory (h_in, h_out:
+        uint8, the sizes of in_buf and out_buf; call pack_io() first). The
+        index call's inputs are copied first; the queries (read only by the
+        attention) are copied on a second stream while the index call runs,
+        and the attention waits for them; the outputs are copied back last."""
+        cut = self.in_split
+        side = torch.cuda.Stream(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            cur = torch.cuda.current_stream(self.device)
+            side.wait_stream(cur)
+            with torch.cuda.stream(side):
+                self.in_buf[cut:].copy_(h_in[cut:], non_blocking=True)
+            self.in_buf[:cut].copy_(h_in[:cut], non_blocking=True)
+            if self.n_new and self.fuse_append:
+                self.append_index()
+            else:
+                if self.n_new:
+                    self.append()
+                self.index()
+            cur.wait_stream(side)
+            self.attend()
+            h_out.copy_(self.out_buf, non_blocking=True)
+        self.graphs["e2e"] = g
+        torch.cuda.synchronize(self.device)
+        return g
 
     def call_ms(self) -> dict:
         """Index and attention durations (ms) inside the last replay of the

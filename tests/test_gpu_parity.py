@@ -445,6 +445,23 @@ def test_graph_replay_matches_eager():
     ms = st.call_ms()
     assert 0.0 < ms["index"] < 1000.0 and 0.0 < ms["attend"] < 1000.0
     parity.check_sets(sets0, parity.oracle_sets(wl, t), "graph")
+    # the e2e graph: inputs from pinned host memory (the queries on a second
+    # stream), outputs back to it; the device buffers start cleared
+    h_in = st.in_buf.cpu().pin_memory()
+    h_out = torch.zeros(st.out_buf.shape, dtype=torch.uint8, pin_memory=True)
+    st.capture_e2e(h_in, h_out)
+    st.in_buf.zero_()
+    st.out_buf.zero_()
+    st.sets.fill_(-5)
+    st.replay("e2e")
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    np.testing.assert_array_equal(parity.host(st.sets), sets0)
+    assert torch.equal(st.in_buf.cpu(), h_in)
+    for g in range(len(outs0)):
+        lo = st.out[g].data_ptr() - st.out_buf.data_ptr()
+        got = h_out[lo:lo + st.out[g].numel() * 4].view(torch.float32).view(st.out[g].shape).numpy()
+        np.testing.assert_array_equal(got, outs0[g])
 
 
 # HI rows that see fewer tokens than their sequence holds, with a window
