@@ -287,6 +287,48 @@ def test_append_index_equals_append_then_index(case):
     parity.check_sets(parity.host(st.sets), parity.oracle_sets(wl, t), wl.name)
 
 
+def test_append_index_appends_to_sequences_without_rows():
+    """The fused append covers every sequence of the batch, also one that no
+    query row reads (rows of sequences 0 and 2 only): its new rows and block
+    sum are written, and the rows' sets equal the oracle's on the updated
+    cache."""
+    wl = wls.small(BASE, name="ai_norows", lens=(3000, 5000, 2600), hi_block=64, hi_topblocks=8, window=100,
+                   sink=16, topk=300, G=1, seed=47)
+    t = wls.make(wl, DEV)
+    t.q_seq.copy_(torch.tensor([0, 0, 2], dtype=torch.int32))
+    t.q_len.copy_(torch.tensor([3000, 2990, 2600], dtype=torch.int32))
+    st = LsaStep(wl, t, DEV)
+    st.build_block_sums()
+    n_new = 2
+    gen = torch.Generator().manual_seed(49)
+    k_idx_new = torch.randint(-16, 16, (wl.n_seq, n_new, wl.d_I), dtype=torch.int8, generator=gen)
+    kn = [torch.randn((wl.n_seq, n_new, wl.H_kv, wl.d), generator=gen).to(torch.bfloat16)]
+    vn = [torch.randn((wl.n_seq, n_new, wl.H_kv, wl.d), generator=gen).to(torch.bfloat16)]
+    want_k = parity.host(t.k_idx).copy()
+    want_V = parity.u16(t.v[0]).copy()
+    offs = parity.host(t.kv_offset)
+    for b, L in enumerate(wl.lens):
+        lo = offs[b] + L - n_new
+        want_k[lo:lo + n_new] = k_idx_new[b].numpy()
+        want_V[lo:lo + n_new] = vn[0][b].view(torch.int16).numpy().view(np.uint16)
+    assert lsa.lsa_append_index_launches(st.batch, wl.H_I, wl.d_I, st.budget, n_new) == \
+        lsa.lsa_index_launches(st.batch, wl.H_I, wl.d_I, st.budget)
+    lsa.lsa_append_index(k_idx_new.to(DEV), [x.to(DEV) for x in kn], [x.to(DEV) for x in vn], t.k, t.v, n_new,
+                         t.q_idx, t.k_idx, t.w, wl.w_max, st.batch, st.budget, st.sets, st.block_sums, st.ws_index,
+                         st.status)
+    torch.cuda.synchronize()
+    assert st.status_bits() == 0
+    np.testing.assert_array_equal(parity.host(t.k_idx), want_k)
+    np.testing.assert_array_equal(parity.u16(t.v[0]), want_V)
+    orc = oracle.get()
+    got = parity.decode_block_sums(st.block_sums, wl.d_I)
+    boffs = parity.host(t.blk_offset)
+    for b, L in enumerate(wl.lens):
+        want = orc.block_sums(want_k[offs[b]:offs[b] + L], wl.hi_block)
+        np.testing.assert_array_equal(got[boffs[b]:boffs[b] + want.shape[0]], want)
+    parity.check_sets(parity.host(st.sets), parity.oracle_sets(wl, t), wl.name)
+
+
 def test_append_index_flags_a_bad_sequence():
     """A sequence whose new tokens outnumber its tokens is skipped and flagged
     by the fused append (LSA_DEV_BAD_LENGTH); the other sequences' rows are
