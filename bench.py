@@ -167,18 +167,23 @@ def measure_int8_peak(dev, n: int = 8192, reps: int = 20) -> dict:
             f"of 3 bursts of {reps}", "ms": best}
 
 
-def _kernel_hash() -> str:
+ATTEND_SOURCES = ("attend.cu", "common.cuh")
+INDEX_SOURCES = ("index_select.cu", "index_score.cu", "index_common.cuh", "append.cuh", "common.cuh", "internal.h")
+
+
+def _kernel_hash(files=ATTEND_SOURCES) -> str:
     h = hashlib.sha256()
-    for f in ("attend.cu", "common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "long_context_sparse_lsa_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def _ncu_traffic(kernel_hash: str, workload: str):
-    """DRAM bytes per launch of the attention kernel from the committed ncu
-    summary, if it was taken on this exact kernel source and workload."""
-    p = os.path.join(PROFILES, f"attend_{workload}.txt")
+def _ncu_traffic(kernel_hash: str, workload: str, kind: str = "attend"):
+    """DRAM bytes per launch of the call's kernels (kind "attend": the attention
+    kernel; "index": the index call's kernels) from the committed ncu summary,
+    if it was taken on this exact kernel source and workload."""
+    p = os.path.join(PROFILES, f"{kind}_{workload}.txt")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -777,7 +782,8 @@ def main(argv=None):
                                             "selection with the SI assembly)",
                   "achieved": ix_bytes / (ix_in / 1000.0) / 1e9, "peak": peak, "unit": "GB/s",
                   "frac": ix_bytes / (ix_in / 1000.0) / 1e9 / peak, "peak_kind": peak_kind,
-                  "traffic": None, "bytes_per_launch": ix_bytes, "ms_per_launch": ix_in,
+                  "traffic": _ncu_traffic(_kernel_hash(INDEX_SOURCES), wl.name, "index") if fused else None,
+                  "bytes_per_launch": ix_bytes, "ms_per_launch": ix_in,
                   "timing": f"CUDA events recorded inside the step graph around the {ix_call} call, mean over "
                             "one replay per timed step (L2 flushed before each)"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
