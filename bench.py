@@ -733,7 +733,8 @@ def main(argv=None):
     # tokens' keys and K/V rows) sit in one pinned host buffer and the outputs
     # come back into another; one graph per step (LsaStep.capture_e2e): the
     # index call's inputs copied in, the queries copied on a second stream
-    # while the index call runs, the attention, the outputs copied out
+    # while the index call runs, the attention writing the outputs into the
+    # host buffer (or a copy back when the device cannot address it)
     h_in = st.in_buf.cpu().pin_memory()
     h_out = torch.empty(st.out_buf.shape, dtype=torch.uint8, pin_memory=True)
     h2d = h_in.numel()
@@ -819,8 +820,11 @@ def main(argv=None):
             "roofline_index": roof_index,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "how": "one CUDA graph per step: the index call's inputs copied from pinned host memory, the "
-                           "queries copied on a second stream while the index call runs, the attention, the "
-                           "outputs copied back to pinned host memory; L2 flushed before each step",
+                           "queries copied on a second stream while the index call runs, the attention, "
+                           + ("which writes the outputs straight into pinned host memory (device-addressable "
+                              "under unified addressing)" if getattr(st, "e2e_direct_out", False) else
+                              "the outputs copied back to pinned host memory")
+                           + "; L2 flushed before each step",
                     "ms_per_step": e2e},
             "gpu_launches": n_kernels * args.steps,
             "clocks": clk}

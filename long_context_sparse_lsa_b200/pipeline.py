@@ -16,6 +16,19 @@ from . import inputs as gen
 from .workloads import Tensors, Workload
 
 
+def _device_addressable(t: torch.Tensor) -> bool:
+    """True when the pinned host tensor t can be written by a kernel at its
+    own address (unified addressing maps page-locked host memory into the
+    device's address space); checked with cudaPointerGetAttributes."""
+    try:
+        from cuda.bindings import runtime as rt
+    except ImportError:
+        return False
+    err, attr = rt.cudaPointerGetAttributes(t.data_ptr())
+    return (err == rt.cudaError_t.cudaSuccess and attr.type == rt.cudaMemoryType.cudaMemoryTypeHost
+            and int(attr.devicePointer) == t.data_ptr())
+
+
 def _pack(tensors, device):
     """One contiguous uint8 device buffer holding copies of `tensors`, each
     at a 256-byte aligned offset, and the views of it that replace them."""
@@ -286,8 +299,17 @@ class LsaStep:
         uint8, the sizes of in_buf and out_buf; call pack_io() first). The
         index call's inputs are copied first; the queries (read only by the
         attention) are copied on a second stream while the index call runs,
-        and the attention waits for them; the outputs are copied back last."""
+        and the attention waits for them. The bf16 attention writes its
+        outputs straight into h_out when the device can address it (the
+        result crosses to the host as the kernel stores it); otherwise they
+        are copied back last."""
         cut = self.in_split
+        direct = not (self.kv_fp8 or self.grouped or self.si_attend) and _device_addressable(h_out)
+        host_out = []
+        if direct:
+            for o in self.out:
+                lo = o.data_ptr() - self.out_buf.data_ptr()
+                host_out.append(h_out[lo:lo + o.numel() * o.element_size()].view(o.dtype).view(o.shape))
         side = torch.cuda.Stream(self.device)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, capture_error_mode="thread_local"):
@@ -303,8 +325,13 @@ class LsaStep:
                     self.append()
                 self.index()
             cur.wait_stream(side)
-            self.attend()
-            h_out.copy_(self.out_buf, non_blocking=True)
+            if direct:
+                lsa.lsa_attend(self.t.q, self.t.k, self.t.v, self.sets, self.batch, host_out, self.ws_attend,
+                               self.status)
+            else:
+                self.attend()
+                h_out.copy_(self.out_buf, non_blocking=True)
+        self.e2e_direct_out = direct
         self.graphs["e2e"] = g
         torch.cuda.synchronize(self.device)
         return g
