@@ -119,3 +119,10 @@ def test_pack_io_keeps_values_in_one_aligned_buffer(kv_fp8):
         assert o.dtype == torch.float32 and o.shape == (wl.n_q, wl.H_q, wl.d)
         assert (o.data_ptr() - olo) % 256 == 0
     assert st.out[1].data_ptr() - st.out[0].data_ptr() >= st.out[0].numel() * 4
+
+
+def test_pageable_host_memory_is_not_written_by_kernels():
+    """The e2e graph lets the attention write into a host buffer only when the
+    device can address it at its own address; pageable memory never can."""
+    from long_context_sparse_lsa_b200.pipeline import _device_addressable
+    assert not _device_addressable(torch.empty(4096, dtype=torch.uint8))
